@@ -1,0 +1,373 @@
+"""Plain fp64 CPU oracle for Hessian-aware layer-wise weight quantization (GPTQ / Babai).
+
+TEST INFRASTRUCTURE ONLY.  This module is the checker the CUDA path is compared against; it is
+called by ``tests/``, by ``__graft_entry__.smoke()`` and by the CPU-baseline leg of ``bench.py``
+and by nothing else.  It shares no code with the CUDA library and imports nothing from the
+package; it is slow on purpose (unblocked, column by column, numpy fp64).
+
+Sources, by page title and section:
+
+* [GEOM] "The Geometry of LLM Quantization: GPTQ as Babai's Nearest Plane Algorithm"
+  - section 2.1: the layer objective is a closest-vector problem; the basis comes from the
+    calibration inputs and the per-column scales, the target from the float weights; Theorem 1:
+    any factor of the Hessian X^T X gives an equivalent instance, so a square Cholesky factor
+    may replace the tall input matrix.
+  - section 2.2: GPTQ's error propagation is Babai's nearest-plane step; Theorem 4: GPTQ run
+    back to front is exactly Babai; one more propagation after the projection changes nothing.
+  - section 2.3: Theorem 5: without clipping, the error is at most one quarter of
+    (T^-1 s)^T D (T^-1 s), D the diagonal of the LDL factorisation of the order-permuted
+    Hessian, T the quantization order.
+* [WSIC] "WaterSIC: information-theoretically (near) optimal linear layer quantization",
+  section 2: Cholesky Sigma = L L^T, columns decided from the last to the first with the
+  already-decided ones cancelled (successive interference cancellation); "dead feature
+  erasure" of zero-variance inputs.
+* [INIT] "Initialisation Determines the Basin", OA-EM section: the per-layer Hessian is the
+  input Gram matrix plus a lambda-multiple of the identity.
+* [RDQ] "RDQ: Residual Distribution Quantization", setup: group-128 asymmetric integer format.
+
+The pages do not print GPTQ's update, its min-max quantizer or its Cholesky trick; where they
+are silent the plainest reading is taken and flagged ``reading:`` below.
+
+Pins (tests/test_oracle_pins.py, tests/test_oracle_golden.py): every public function here is
+pinned against a closed form, a hand-derived example, an independent textbook construction
+(Gram-Schmidt Babai, brute-force CVP) or an invariant.  No function is "parity unpinned".
+"""
+from __future__ import annotations
+
+import numpy as np
+
+__all__ = [
+    "hessian",
+    "fix_dead_features",
+    "dampen",
+    "hinv_upper_factor",
+    "minmax_grid",
+    "clipfree_grid",
+    "gptq_columns",
+    "babai_sic_reverse",
+    "pack_codes",
+    "proxy_loss",
+    "quadratic_loss",
+    "babai_bound",
+    "quantize_layer",
+]
+
+
+def _f64(a) -> np.ndarray:
+    if hasattr(a, "detach"):  # a torch tensor: bf16/fp32 -> fp64 is exact
+        a = a.detach().to("cpu").double().numpy()
+    return np.asarray(a, dtype=np.float64)
+
+
+# ---------------------------------------------------------------------------------------------
+# Hessian, dead features, damping, the factor
+# ---------------------------------------------------------------------------------------------
+
+def hessian(X) -> np.ndarray:
+    """H = 2 X^T X for X stored tokens x features ([GEOM] 2.1, Hessian X^T X; [INIT] OA-EM).
+
+    reading: the factor 2 is the second derivative of the squared output error; H is not
+    divided by the token count (codes do not depend on a positive scale of H).
+    """
+    x = _f64(X)
+    return 2.0 * (x.T @ x)
+
+
+def fix_dead_features(H, W):
+    """Zero-variance inputs: H_ii == 0 -> H_ii = 1 and W[:, i] = 0 ([WSIC] dead feature erasure).
+
+    Returns (H', W', dead mask).
+    """
+    h = _f64(H).copy()
+    w = _f64(W).copy()
+    dead = np.diag(h) == 0.0
+    idx = np.nonzero(dead)[0]
+    h[idx, idx] = 1.0
+    w[:, idx] = 0.0
+    return h, w, dead
+
+
+def dampen(H, damp: float):
+    """H_d = H + damp * mean(diag H) * I, applied after the dead-feature fix ([INIT] +lambda I).
+
+    reading: lambda is relative to the mean diagonal, damp = 0.01.  Returns (H_d, delta).
+    """
+    h = _f64(H)
+    delta = damp * float(np.mean(np.diag(h)))
+    return h + delta * np.eye(h.shape[0]), delta
+
+
+def hinv_upper_factor(Hd) -> np.ndarray:
+    """U upper triangular, positive diagonal, with U^T U = H_d^-1.
+
+    Literal three-step route: Cholesky H_d = L L^T; inverse H_d^-1 = L^-T L^-1; then the
+    upper Cholesky factor of that inverse (the transpose of its lower factor).  A non-positive
+    pivot raises numpy's LinAlgError.
+    """
+    h = _f64(Hd)
+    L = np.linalg.cholesky(h)
+    Linv = np.linalg.inv(L)
+    hinv = Linv.T @ Linv
+    hinv = 0.5 * (hinv + hinv.T)
+    return np.linalg.cholesky(hinv).T
+
+
+# ---------------------------------------------------------------------------------------------
+# The quantization grid
+# ---------------------------------------------------------------------------------------------
+
+def minmax_grid(w, bits: int):
+    """Asymmetric min-max grid per row of ``w`` (rows x k) ([RDQ] group-128 asymmetric format).
+
+    reading: the range always contains 0 (lo = min(min w, 0), hi = max(max w, 0)); an all-zero
+    range becomes [-1, 1]; scale s = (hi - lo) / (2^b - 1); zero point z = rint(-lo / s), so
+    z lies in [0, 2^b - 1].  rint is round-half-to-even.  Returns (s, z) as fp64 vectors.
+    """
+    w = _f64(w)
+    maxq = float(2 ** bits - 1)
+    lo = np.minimum(w.min(axis=1), 0.0)
+    hi = np.maximum(w.max(axis=1), 0.0)
+    flat = (lo == 0.0) & (hi == 0.0)
+    lo = np.where(flat, -1.0, lo)
+    hi = np.where(flat, 1.0, hi)
+    s = (hi - lo) / maxq
+    z = np.rint(-lo / s)
+    return s, z
+
+
+def clipfree_grid(w, bits: int, alpha):
+    """Per-row uniform grid for the clip-free variant ([GEOM] 2.3, no-clipping setting).
+
+    reading: the step is alpha * (hi - lo) / (2^b - 1) with [lo, hi] as in ``minmax_grid`` and
+    alpha >= 1 a per-row widening factor; the zero point centres the row's range on the code
+    range, z = rint((2^b - 1)/2 - (hi + lo) / (2 s)) (equal to rint(-lo/s) when alpha = 1).
+    """
+    w = _f64(w)
+    maxq = float(2 ** bits - 1)
+    lo = np.minimum(w.min(axis=1), 0.0)
+    hi = np.maximum(w.max(axis=1), 0.0)
+    flat = (lo == 0.0) & (hi == 0.0)
+    lo = np.where(flat, -1.0, lo)
+    hi = np.where(flat, 1.0, hi)
+    s = np.asarray(alpha, dtype=np.float64) * (hi - lo) / maxq
+    z = np.rint(maxq / 2.0 - (hi + lo) / (2.0 * s))
+    return s, z
+
+
+# ---------------------------------------------------------------------------------------------
+# Column loops
+# ---------------------------------------------------------------------------------------------
+
+def gptq_columns(W, U, bits: int, group: int = 0, clip: bool = True, alpha=None, grid=None):
+    """GPTQ error-feedback loop, columns 0..n-1 in order ([GEOM] 2.2).
+
+    For each column j: quantize the current column on the row's grid, error
+    e = (w_j - q_j) / U_jj, and feed it forward, w_k -= e U_jk for k > j.  U is the upper
+    factor of the inverse damped Hessian in this processing order.
+
+    Grid (reading): per row (group == 0) from the row as given; per group of ``group`` columns,
+    recomputed at the group's first column from the current, error-fed weights of the group.
+    clip=False: codes are unconstrained integers (no clamp) on the ``clipfree_grid`` with the
+    per-row factor ``alpha`` (group must be 0).  ``grid`` = (s, z) fixes the per-row grid
+    instead (a fixed lattice).
+
+    Returns dict(codes, scales, zeros, Q, e) in processing order; e is the m x n matrix of
+    scaled errors, whose squares sum to tr(D H_d D^T).
+    """
+    w = _f64(W).copy()
+    u = _f64(U)
+    m, n = w.shape
+    maxq = 2 ** bits - 1
+    if not clip and group:
+        raise ValueError("the clip-free variant uses a per-row grid")
+    ngroups = 1 if group == 0 else -(-n // group)
+    scales = np.zeros((m, ngroups))
+    zeros = np.zeros((m, ngroups))
+    codes = np.zeros((m, n), dtype=np.int64)
+    Q = np.zeros((m, n))
+    E = np.zeros((m, n))
+    if group == 0:
+        if grid is not None:
+            s, z = (np.asarray(g, dtype=np.float64).copy() for g in grid)
+        elif clip:
+            s, z = minmax_grid(w, bits)
+        else:
+            s, z = clipfree_grid(w, bits, np.ones(m) if alpha is None else alpha)
+        scales[:, 0], zeros[:, 0] = s, z
+    for j in range(n):
+        if group and j % group == 0:
+            s, z = minmax_grid(w[:, j:j + group], bits)
+            scales[:, j // group], zeros[:, j // group] = s, z
+        c = np.rint(w[:, j] / s) + z
+        if clip:
+            c = np.clip(c, 0, maxq)
+        q = s * (c - z)
+        e = (w[:, j] - q) / u[j, j]
+        w[:, j + 1:] -= np.outer(e, u[j, j + 1:])
+        codes[:, j] = c.astype(np.int64)
+        Q[:, j] = q
+        E[:, j] = e
+    return dict(codes=codes, scales=scales, zeros=zeros, Q=Q, e=E)
+
+
+def babai_sic_reverse(W, L, bits: int, clip: bool = False, alpha=None):
+    """Last-to-first successive interference cancellation ([WSIC] 2; [GEOM] 2.2 Theorem 4).
+
+    With H_d = L L^T (L lower), column j (from n-1 down to 0) is rounded on the row grid at the
+    target w_j + sum_{k>j} (L_kj / L_jj) (w_k - q_k), i.e. the decided columns' residuals are
+    cancelled through the Cholesky factor.  Per-row grid (``clipfree_grid`` with ``alpha`` when
+    clip=False, ``minmax_grid`` when clip=True).  Returns dict(codes, scales, zeros, Q, D).
+    """
+    w = _f64(W)
+    l = _f64(L)
+    m, n = w.shape
+    maxq = 2 ** bits - 1
+    if clip:
+        s, z = minmax_grid(w, bits)
+    else:
+        s, z = clipfree_grid(w, bits, np.ones(m) if alpha is None else alpha)
+    D = np.zeros((m, n))
+    codes = np.zeros((m, n), dtype=np.int64)
+    Q = np.zeros((m, n))
+    for j in range(n - 1, -1, -1):
+        target = w[:, j] + D[:, j + 1:] @ (l[j + 1:, j] / l[j, j])
+        c = np.rint(target / s) + z
+        if clip:
+            c = np.clip(c, 0, maxq)
+        q = s * (c - z)
+        D[:, j] = w[:, j] - q
+        codes[:, j] = c.astype(np.int64)
+        Q[:, j] = q
+    return dict(codes=codes, scales=s[:, None].copy(), zeros=z[:, None].copy(), Q=Q, D=D)
+
+
+# ---------------------------------------------------------------------------------------------
+# Packing, losses, bound
+# ---------------------------------------------------------------------------------------------
+
+def pack_codes(codes, bits: int) -> np.ndarray:
+    """Per row, an LSB-first bitstream of b-bit codes in uint32 words.
+
+    reading: code of column c occupies bits [b c, b c + b) of the row's stream; the row stride is
+    ceil(n b / 32) words; unused high bits of the last word are 0.
+    """
+    codes = np.asarray(codes, dtype=np.uint64)
+    m, n = codes.shape
+    nwords = -(-n * bits // 32)
+    out = np.zeros((m, nwords), dtype=np.uint64)
+    for col in range(n):
+        pos = col * bits
+        wi, off = divmod(pos, 32)
+        out[:, wi] |= (codes[:, col] << np.uint64(off)) & np.uint64(0xFFFFFFFF)
+        if off + bits > 32:
+            out[:, wi + 1] |= codes[:, col] >> np.uint64(32 - off)
+    return out.astype(np.uint32)
+
+
+def proxy_loss(W0, Q, X) -> float:
+    """||(W0 - Q) X^T||_F^2: squared output error over the calibration tokens ([GEOM] 2.1)."""
+    d = _f64(W0) - _f64(Q)
+    y = d @ _f64(X).T
+    return float(np.sum(y * y))
+
+
+def quadratic_loss(W0, Q, H) -> float:
+    """tr(D H D^T) with D = W0 - Q ([GEOM] 2.1 objective in Hessian form)."""
+    d = _f64(W0) - _f64(Q)
+    return float(np.sum((d @ _f64(H)) * d))
+
+
+def babai_bound(scales_per_col, pivots) -> float:
+    """Theorem 5 ([GEOM] 2.3): sum over rows of (1/4) sum_p s_{r,p}^2 D_pp.
+
+    ``scales_per_col`` is rows x n (the step of each entry, in processing order); ``pivots`` is
+    the diagonal D of the LDL factorisation of the processing-order Hessian, i.e. the squared
+    Cholesky pivots.
+    """
+    s = _f64(scales_per_col)
+    return float(0.25 * np.sum((s * s) @ _f64(pivots)))
+
+
+# ---------------------------------------------------------------------------------------------
+# The whole layer
+# ---------------------------------------------------------------------------------------------
+
+def quantize_layer(W, X, bits: int, group: int = 0, reverse: bool = False, clip: bool = True,
+                   damp: float = 0.01, ladder: float = 1.25, ladder_max: int = 8,
+                   rows=None, H=None):
+    """Quantize one linear layer: H, dead fix, damping, factor, column loop, losses.
+
+    ``W`` is m x n (output rows x input features), ``X`` is T x n.  ``rows`` restricts the
+    column loop to a subset of rows (rows are independent once the factor is known).  ``H``
+    may be passed precomputed (2 X^T X) to share it across layers.
+
+    Forward order uses the GPTQ form with U (``gptq_columns``).  Reverse order uses the SIC
+    form with the lower Cholesky factor of H_d (``babai_sic_reverse``); per-row grids only.
+
+    clip=False (reading of "per-row step set so that no entry needs clipping"): run unclamped;
+    a row whose codes leave [0, 2^b - 1] is rerun with alpha multiplied by ``ladder``, at most
+    ``ladder_max`` times; rows still outside raise ValueError.
+
+    Returns a dict; codes / scales / zeros / Q are in the original column order.
+    """
+    w_in = _f64(W)
+    m, n = w_in.shape
+    if H is None:
+        H = hessian(X)
+    h_fix, w0, dead = fix_dead_features(H, w_in)
+    hd, delta = dampen(h_fix, damp)
+    sel = np.arange(m) if rows is None else np.asarray(rows)
+    w_sel = w0[sel]
+    maxq = 2 ** bits - 1
+    if reverse and group:
+        raise ValueError("the last-to-first variant uses a per-row grid")
+
+    if reverse:
+        L = np.linalg.cholesky(hd)
+        pivots = np.diag(L) ** 2
+
+        def run(rows_w, alpha):
+            return babai_sic_reverse(rows_w, L, bits, clip=clip, alpha=alpha)
+    else:
+        U = hinv_upper_factor(hd)
+        pivots = 1.0 / np.diag(U) ** 2
+
+        def run(rows_w, alpha):
+            return gptq_columns(rows_w, U, bits, group=group, clip=clip, alpha=alpha)
+
+    alpha = np.ones(len(sel))
+    res = run(w_sel, alpha)
+    retries = 0
+    if not clip:
+        for _ in range(ladder_max):
+            bad = np.nonzero((res["codes"] < 0).any(axis=1) | (res["codes"] > maxq).any(axis=1))[0]
+            if bad.size == 0:
+                break
+            retries += 1
+            alpha[bad] *= ladder
+            sub = run(w_sel[bad], alpha[bad])
+            for key in ("codes", "scales", "zeros", "Q"):
+                res[key][bad] = sub[key]
+        bad = (res["codes"] < 0).any(axis=1) | (res["codes"] > maxq).any(axis=1)
+        if bad.any():
+            raise ValueError(f"{int(bad.sum())} rows still overflow after the scale ladder")
+
+    Q = res["Q"]
+    g = group if group else n
+    s_cols = np.repeat(res["scales"], g, axis=1)[:, :n]
+    out = dict(H=H, dead=dead, delta=delta, Hd=hd, codes=res["codes"], scales=res["scales"],
+               zeros=res["zeros"], Q=Q, alpha=alpha, ladder_rounds=retries)
+    if reverse:
+        out["L"] = L
+    else:
+        out["U"] = U
+        out["sum_e2"] = float(np.sum(res["e"] ** 2))
+    w0_sel = w0[sel]
+    out["loss_damped"] = quadratic_loss(w0_sel, Q, hd)
+    if X is not None:
+        out["loss_proxy"] = proxy_loss(w0_sel, Q, X)
+    out["loss_proxy_h"] = 0.5 * quadratic_loss(w0_sel, Q, h_fix)
+    # pivots are indexed by original column in both orders: 1/U_jj^2 (forward), L_jj^2 (reverse)
+    out["bound"] = babai_bound(s_cols, pivots)
+    out["packed"] = pack_codes(np.clip(res["codes"], 0, maxq), bits)
+    return out

@@ -1,0 +1,387 @@
+"""Pins of the fp64 oracle against what the pages and the mathematics fix (CPU only).
+
+Each test names the passage it pins.  None of them re-derives a result with the oracle's own
+formula: they use hand-derived values, closed forms, an independent textbook Babai
+(Gram-Schmidt on a tall basis), brute-force enumeration, or invariants, chosen so that a dropped
+term, a wrong sign or index, or a transposed operand in the oracle fails one of them.
+"""
+import itertools
+import json
+import os
+
+import numpy as np
+import pytest
+
+from oracle import gptq_oracle as O
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _rand_problem(T, n, m, seed, decay=0.8):
+    rng = np.random.default_rng(seed)
+    x = rng.standard_normal((T, n)) * (np.arange(1, n + 1) ** -decay)
+    x = x @ np.linalg.qr(rng.standard_normal((n, n)))[0].T
+    w = 0.02 * rng.standard_normal((m, n))
+    return w, x
+
+
+# --------------------------------------------------------------------------------------------
+# hand-derived two-column example (tests/golden/gptq_two_column_hand.json)
+# --------------------------------------------------------------------------------------------
+
+def test_golden_two_column_forward_reverse_bound():
+    g = json.load(open(os.path.join(GOLDEN, "gptq_two_column_hand.json")))
+    hd = np.array(g["Hd"])
+    w = np.array([g["w"]])
+    s, z = O.minmax_grid(w, g["bits"])
+    assert s[0] == pytest.approx(g["grid"]["scale"], rel=1e-15)
+    assert z[0] == g["grid"]["zero"]
+    U = O.hinv_upper_factor(hd)
+    np.testing.assert_allclose(U, np.array(g["U"]), rtol=1e-13, atol=1e-15)
+    f = O.gptq_columns(w, U, g["bits"])
+    assert f["codes"][0].tolist() == g["forward_codes"]
+    np.testing.assert_allclose(f["Q"][0], g["forward_Q"], rtol=1e-13)
+    assert O.quadratic_loss(w, f["Q"], hd) == pytest.approx(g["forward_loss_damped"], rel=1e-12)
+    assert float(np.sum(f["e"] ** 2)) == pytest.approx(g["forward_loss_damped"], rel=1e-12)
+    L = np.linalg.cholesky(hd)
+    np.testing.assert_allclose(L, np.array(g["L"]), rtol=1e-13, atol=1e-15)
+    r = O.babai_sic_reverse(w, L, g["bits"], clip=False)
+    assert r["codes"][0].tolist() == g["reverse_codes"]
+    assert O.quadratic_loss(w, r["Q"], hd) == pytest.approx(g["reverse_loss_damped"], rel=1e-12)
+    bound = O.babai_bound(np.full((1, 2), g["grid"]["scale"]), np.diag(L) ** 2)
+    assert bound == pytest.approx(g["reverse_bound"], rel=1e-12)
+
+
+def test_golden_brute_force_minimum():
+    g = json.load(open(os.path.join(GOLDEN, "gptq_two_column_hand.json")))
+    hd = np.array(g["Hd"])
+    w = np.array([g["w"]])
+    best = min(O.quadratic_loss(w, np.array([[0.15 * a, 0.15 * b]]), hd)
+               for a in range(4) for b in range(4))
+    assert best == pytest.approx(g["brute_force_min_loss"], rel=1e-12)
+
+
+# --------------------------------------------------------------------------------------------
+# Hessian, dead features, damping, factor
+# --------------------------------------------------------------------------------------------
+
+def test_loss_identity_pins_hessian_convention():
+    """||(W-Q) X^T||^2 = tr(D (X^T X) D^T) = tr(D H D^T)/2 (GEOM 2.1; H = 2 X^T X).
+
+    X is T x n with T != n, so a transposed X, a missing factor 2 or a D^T H D slip fails."""
+    w, x = _rand_problem(T=37, n=9, m=5, seed=1)
+    q = w + 0.01 * np.random.default_rng(2).standard_normal(w.shape)
+    direct = sum(float(np.dot(w[r] - q[r], x[t]) ** 2) for r in range(5) for t in range(37))
+    assert O.proxy_loss(w, q, x) == pytest.approx(direct, rel=1e-12)
+    H = O.hessian(x)
+    assert H.shape == (9, 9)
+    assert 0.5 * O.quadratic_loss(w, q, H) == pytest.approx(direct, rel=1e-12)
+
+
+def test_dead_features_then_damping_hand_values():
+    """Dead feature erasure (WaterSIC, additional techniques) before relative damping."""
+    H = np.array([[0.0, 0.0, 0.0], [0.0, 2.0, 0.5], [0.0, 0.5, 4.0]])
+    W = np.array([[1.0, 2.0, 3.0], [-1.0, -2.0, -3.0]])
+    h, w, dead = O.fix_dead_features(H, W)
+    assert dead.tolist() == [True, False, False]
+    assert h[0, 0] == 1.0 and h[1, 2] == 0.5
+    assert w[:, 0].tolist() == [0.0, 0.0] and w[:, 1:].tolist() == [[2.0, 3.0], [-2.0, -3.0]]
+    hd, delta = O.dampen(h, 0.01)
+    assert delta == pytest.approx(0.01 * 7.0 / 3.0, rel=1e-15)
+    np.testing.assert_allclose(np.diag(hd), [1.0 + 0.07 / 3, 2.0 + 0.07 / 3, 4.0 + 0.07 / 3])
+    assert hd[1, 2] == 0.5 and hd[2, 1] == 0.5
+
+
+def test_hinv_factor_closed_form():
+    """U upper, positive diagonal, U^T U H_d = I (the defining property of GPTQ's factor)."""
+    _, x = _rand_problem(T=40, n=24, m=1, seed=3)
+    hd, _ = O.dampen(O.hessian(x), 0.01)
+    U = O.hinv_upper_factor(hd)
+    assert np.all(np.tril(U, -1) == 0.0)
+    assert np.all(np.diag(U) > 0)
+    np.testing.assert_allclose(U.T @ U @ hd, np.eye(24), atol=1e-9)
+
+
+def test_hinv_factor_rejects_indefinite():
+    with pytest.raises(np.linalg.LinAlgError):
+        O.hinv_upper_factor(np.array([[1.0, 2.0], [2.0, 1.0]]))
+
+
+# --------------------------------------------------------------------------------------------
+# grid
+# --------------------------------------------------------------------------------------------
+
+def test_minmax_grid_hand_values():
+    w = np.array([[-0.3, 0.6], [0.2, 0.5], [0.0, 0.0], [-0.4, -0.1]])
+    s, z = O.minmax_grid(w, 2)
+    np.testing.assert_allclose(s, [0.3, 0.5 / 3, 2.0 / 3, 0.4 / 3], rtol=1e-15)
+    # -lo/s: 1; 0; 1.5 -> 2 (half to even); 3
+    assert z.tolist() == [1.0, 0.0, 2.0, 3.0]
+
+
+def test_clipfree_grid_reduces_to_minmax_at_alpha_one_and_widens():
+    rng = np.random.default_rng(4)
+    w = rng.standard_normal((50, 16)) * 0.02
+    s1, z1 = O.minmax_grid(w, 3)
+    s2, z2 = O.clipfree_grid(w, 3, np.ones(50))
+    np.testing.assert_allclose(s2, s1, rtol=1e-14)
+    assert np.array_equal(z1, z2)
+    s3, z3 = O.clipfree_grid(w, 3, np.full(50, 2.0))
+    np.testing.assert_allclose(s3, 2 * s1, rtol=1e-14)
+    # the widened range still maps [lo, hi] inside the code range
+    lo = np.minimum(w.min(1), 0)
+    hi = np.maximum(w.max(1), 0)
+    assert np.all(np.rint(lo / s3) + z3 >= 0) and np.all(np.rint(hi / s3) + z3 <= 7)
+
+
+# --------------------------------------------------------------------------------------------
+# column loop: special cases, independent Babai, brute force, invariants
+# --------------------------------------------------------------------------------------------
+
+def _rtn(w, s, z, maxq):
+    return np.clip(np.rint(w / s[:, None]) + z[:, None], 0, maxq)
+
+
+@pytest.mark.parametrize("group", [0, 4])
+def test_diagonal_hessian_gptq_equals_rtn(group):
+    """No cross-column coupling => no feedback => GPTQ = round-to-nearest (GEOM 4 baseline)."""
+    rng = np.random.default_rng(5)
+    w = 0.02 * rng.standard_normal((30, 16))
+    hd = np.diag(rng.uniform(0.5, 3.0, 16))
+    U = O.hinv_upper_factor(hd)
+    res = O.gptq_columns(w, U, 3, group=group)
+    if group == 0:
+        s, z = O.minmax_grid(w, 3)
+        expect = _rtn(w, s, z, 7)
+    else:
+        expect = np.concatenate([_rtn(w[:, k:k + 4], *O.minmax_grid(w[:, k:k + 4], 3), 7)
+                                 for k in range(0, 16, 4)], axis=1)
+    assert np.array_equal(res["codes"], expect.astype(np.int64))
+
+
+def _babai_gram_schmidt(Bm, t):
+    """Textbook nearest plane: Gram-Schmidt of the basis columns, last basis vector first."""
+    d = Bm.shape[1]
+    gs = np.zeros_like(Bm)
+    for i in range(d):
+        v = Bm[:, i].copy()
+        for k in range(i):
+            v -= (v @ gs[:, k]) / (gs[:, k] @ gs[:, k]) * gs[:, k]
+        gs[:, i] = v
+    r = t.copy()
+    u = np.zeros(d)
+    for i in range(d - 1, -1, -1):
+        c = np.rint((r @ gs[:, i]) / (gs[:, i] @ gs[:, i]))
+        u[i] = c
+        r = r - c * Bm[:, i]
+    return u
+
+
+@pytest.mark.parametrize("seed", range(4))
+def test_gptq_is_babai_on_tall_factor(seed):
+    """GEOM 2.2 Theorem 4 with 2.1 Theorem 1: the oracle's GPTQ (forward, unclamped) equals
+    textbook Babai on the basis [sqrt2 X; sqrt(delta) I] diag(s) with basis order reversed; the
+    last-to-first SIC form equals Babai in the natural order."""
+    n, T, m = 12, 40, 60
+    w, x = _rand_problem(T, n, m, seed=10 + seed)
+    hd, delta = O.dampen(O.hessian(x), 0.01)
+    F = np.vstack([np.sqrt(2.0) * x, np.sqrt(delta) * np.eye(n)])
+    U = O.hinv_upper_factor(hd)
+    L = np.linalg.cholesky(hd)
+    fwd = O.gptq_columns(w, U, 3, clip=False)
+    rev = O.babai_sic_reverse(w, L, 3, clip=False)
+    s = fwd["scales"][:, 0]
+    for r in range(m):
+        tgt = F @ w[r]
+        u_f = _babai_gram_schmidt((F * s[r])[:, ::-1], tgt)[::-1]
+        u_r = _babai_gram_schmidt(F * s[r], tgt)
+        assert np.array_equal(fwd["codes"][r] - fwd["zeros"][r, 0], u_f.astype(np.int64))
+        assert np.array_equal(rev["codes"][r] - rev["zeros"][r, 0], u_r.astype(np.int64))
+
+
+def test_extra_propagation_after_projection_changes_nothing():
+    """GEOM 2.2: a further GPTQ pass over the Babai result, on the same lattice (grid), leaves
+    it unchanged: the result is a lattice point, every error is zero and nothing propagates."""
+    w, x = _rand_problem(64, 16, 40, seed=20)
+    hd, _ = O.dampen(O.hessian(x), 0.01)
+    U = O.hinv_upper_factor(hd)
+    first = O.gptq_columns(w, U, 4)
+    s, z = first["scales"][:, 0], first["zeros"][:, 0]
+    again = O.gptq_columns(first["Q"], U, 4, grid=(s, z))
+    assert np.array_equal(again["codes"], first["codes"])
+    np.testing.assert_allclose(again["e"], 0.0, atol=1e-15)
+    assert np.array_equal(again["zeros"][:, 0], z) and np.allclose(again["scales"][:, 0], s)
+
+
+@pytest.mark.parametrize("bits,d", [(2, 6), (3, 5), (4, 4)])
+def test_brute_force_cvp_lower_bounds_gptq(bits, d):
+    """The exact CVP over the clamped code box is <= GPTQ's loss (NP-hard problem, greedy
+    heuristic), and GPTQ is never worse than round-to-nearest on these instances' average."""
+    w, x = _rand_problem(3 * d, d, 25, seed=30 + bits)
+    hd, _ = O.dampen(O.hessian(x), 0.01)
+    U = O.hinv_upper_factor(hd)
+    res = O.gptq_columns(w, U, bits)
+    s, z = res["scales"][:, 0], res["zeros"][:, 0]
+    maxq = 2 ** bits - 1
+    grid = np.array(list(itertools.product(range(maxq + 1), repeat=d)), dtype=np.float64)
+    tot_g = tot_r = 0.0
+    for r in range(w.shape[0]):
+        qs = s[r] * (grid - z[r])
+        dd = w[r][None, :] - qs
+        best = np.min(np.einsum("ki,ij,kj->k", dd, hd, dd))
+        dg = w[r] - res["Q"][r]
+        lg = dg @ hd @ dg
+        assert best <= lg * (1 + 1e-12)
+        qr = s[r] * (_rtn(w[r:r + 1], s[r:r + 1], z[r:r + 1], maxq)[0] - z[r])
+        tot_g += lg
+        tot_r += (w[r] - qr) @ hd @ (w[r] - qr)
+    assert tot_g <= tot_r
+
+
+def _gptq_blocked(w, U, bits, group, B):
+    w = w.copy()
+    m, n = w.shape
+    maxq = 2 ** bits - 1
+    codes = np.zeros((m, n), dtype=np.int64)
+    if group == 0:
+        s, z = O.minmax_grid(w, bits)
+    for b0 in range(0, n, B):
+        b1 = min(b0 + B, n)
+        blk = w[:, b0:b1].copy()
+        E = np.zeros((m, b1 - b0))
+        for jj in range(b1 - b0):
+            j = b0 + jj
+            if group and j % group == 0:
+                s, z = O.minmax_grid(blk[:, jj:jj + group], bits)
+            c = np.clip(np.rint(blk[:, jj] / s) + z, 0, maxq)
+            e = (blk[:, jj] - s * (c - z)) / U[j, j]
+            blk[:, jj + 1:] -= np.outer(e, U[j, j + 1:b1])
+            E[:, jj] = e
+            codes[:, j] = c
+        w[:, b1:] -= E @ U[b0:b1, b1:]
+    return codes
+
+
+@pytest.mark.parametrize("group,B", [(0, 8), (8, 16), (4, 8)])
+def test_lazy_block_update_is_exact_reassociation(group, B):
+    """Deferring the trailing update to block ends changes no code (exact re-association)."""
+    w, x = _rand_problem(96, 40, 50, seed=40 + B)
+    hd, _ = O.dampen(O.hessian(x), 0.01)
+    U = O.hinv_upper_factor(hd)
+    ref = O.gptq_columns(w, U, 3, group=group)["codes"]
+    assert np.array_equal(_gptq_blocked(w, U, 3, group, B), ref)
+
+
+def test_sum_of_scaled_errors_equals_damped_loss():
+    """sum_j e_j^2 = tr(D H_d D^T), since D = U^T E."""
+    w, x = _rand_problem(80, 32, 30, seed=50)
+    hd, _ = O.dampen(O.hessian(x), 0.01)
+    U = O.hinv_upper_factor(hd)
+    res = O.gptq_columns(w, U, 3, group=8)
+    assert float(np.sum(res["e"] ** 2)) == pytest.approx(O.quadratic_loss(w, res["Q"], hd),
+                                                         rel=1e-10)
+
+
+def test_scale_invariance_and_order_reversal():
+    """Codes do not change under H -> cH (c > 0, damping is relative); the last-to-first SIC
+    form equals the forward GPTQ form run on column-reversed W and J H J."""
+    w, x = _rand_problem(70, 24, 40, seed=60)
+    h = O.hessian(x)
+    hd, _ = O.dampen(h, 0.01)
+    hd7, _ = O.dampen(7.0 * h, 0.01)
+    a = O.gptq_columns(w, O.hinv_upper_factor(hd), 4, group=8)["codes"]
+    b = O.gptq_columns(w, O.hinv_upper_factor(hd7), 4, group=8)["codes"]
+    assert np.array_equal(a, b)
+    for clip in (True, False):
+        sic = O.babai_sic_reverse(w, np.linalg.cholesky(hd), 3, clip=clip)
+        fw = O.gptq_columns(w[:, ::-1], O.hinv_upper_factor(hd[::-1, ::-1]), 3, clip=clip)
+        assert np.array_equal(sic["codes"], fw["codes"][:, ::-1])
+        np.testing.assert_allclose(sic["Q"], fw["Q"][:, ::-1], rtol=0, atol=1e-15)
+
+
+@pytest.mark.parametrize("reverse", [False, True])
+def test_clipfree_loss_within_babai_bound(reverse):
+    """GEOM 2.3 Theorem 5: without clipping the damped loss of every row is at most
+    (1/4) sum_p s^2 D_pp, D the LDL pivots in the processing order."""
+    w, x = _rand_problem(200, 48, 64, seed=70)
+    h = O.hessian(x)
+    hd, _ = O.dampen(h, 0.01)
+    if reverse:
+        L = np.linalg.cholesky(hd)
+        res = O.babai_sic_reverse(w, L, 3, clip=False)
+        piv = np.diag(L) ** 2
+    else:
+        U = O.hinv_upper_factor(hd)
+        res = O.gptq_columns(w, U, 3, clip=False)
+        piv = 1.0 / np.diag(U) ** 2
+    # pivots must be those of the processing order: LDL of the permuted Hessian
+    P = np.arange(48)[::-1] if reverse else np.arange(48)
+    hp = hd[np.ix_(P, P)]
+    # UDU^T of the permuted matrix (last pivot first): Cholesky of J hp J, read backwards
+    Lr = np.linalg.cholesky(hp[::-1, ::-1])
+    piv_ldl = (np.diag(Lr) ** 2)[::-1][np.argsort(P)]
+    np.testing.assert_allclose(piv, piv_ldl, rtol=1e-10)
+    s = res["scales"][:, 0]
+    for r in range(64):
+        d = w[r] - res["Q"][r]
+        assert d @ hd @ d <= 0.25 * s[r] ** 2 * piv.sum() * (1 + 1e-12)
+
+
+# --------------------------------------------------------------------------------------------
+# packing
+# --------------------------------------------------------------------------------------------
+
+def test_pack_codes_hand_values_and_roundtrip():
+    codes = np.array([[1, 2, 3, 15, 0, 7, 8, 9, 10]])
+    p = O.pack_codes(codes, 4)
+    assert p.shape == (1, 2)
+    assert int(p[0, 0]) == (1 | 2 << 4 | 3 << 8 | 15 << 12 | 0 << 16 | 7 << 20 | 8 << 24 | 9 << 28)
+    assert int(p[0, 1]) == 10
+    # 3-bit codes straddle word boundaries: code 10 sits at bits [30, 33)
+    rng = np.random.default_rng(80)
+    c3 = rng.integers(0, 8, size=(5, 77))
+    p3 = O.pack_codes(c3, 3)
+    assert p3.shape == (5, -(-77 * 3 // 32))
+    bits = np.unpackbits(p3.view(np.uint8).reshape(5, -1), axis=1, bitorder="little")
+    back = np.stack([bits[:, 3 * k] + 2 * bits[:, 3 * k + 1] + 4 * bits[:, 3 * k + 2]
+                     for k in range(77)], axis=1)
+    assert np.array_equal(back, c3)
+    assert bits[:, 3 * 77:].sum() == 0
+
+
+# --------------------------------------------------------------------------------------------
+# the whole layer
+# --------------------------------------------------------------------------------------------
+
+def test_quantize_layer_clipfree_ladder_fits_every_row():
+    w, x = _rand_problem(300, 32, 80, seed=90)
+    out = O.quantize_layer(w, x, bits=2, reverse=True, clip=False)
+    assert out["codes"].min() >= 0 and out["codes"].max() <= 3
+    assert out["ladder_rounds"] >= 1          # 2-bit unclamped rounding overflows at alpha = 1
+    assert np.all(out["alpha"] >= 1.0)
+    assert out["loss_damped"] <= out["bound"]
+
+
+def test_quantize_layer_dead_feature_and_loss_bookkeeping():
+    w, x = _rand_problem(120, 20, 16, seed=91)
+    x[:, 5] = 0.0
+    out = O.quantize_layer(w, x, bits=4, group=8)
+    assert out["dead"][5] and out["dead"].sum() == 1
+    # the dead column quantizes a zeroed weight: q = 0 exactly
+    assert np.all(out["Q"][:, 5] == 0.0)
+    assert out["loss_proxy"] == pytest.approx(out["loss_proxy_h"], rel=1e-10)
+    assert out["sum_e2"] == pytest.approx(out["loss_damped"], rel=1e-10)
+    # damped = undamped + delta ||D||^2 (what the GPU reports without X)
+    d = (w - out["Q"])
+    d[:, 5] = 0.0
+    assert out["loss_damped"] == pytest.approx(2 * out["loss_proxy"] + out["delta"] * np.sum(d * d),
+                                               rel=1e-10)
+
+
+def test_quantize_layer_sampled_rows_match_full():
+    w, x = _rand_problem(90, 24, 40, seed=92)
+    full = O.quantize_layer(w, x, bits=3, group=8)
+    rows = [3, 17, 39]
+    part = O.quantize_layer(w, x, bits=3, group=8, rows=rows)
+    assert np.array_equal(part["codes"], full["codes"][rows])
+    np.testing.assert_allclose(part["scales"], full["scales"][rows])
