@@ -1,0 +1,166 @@
+/*
+ * gq.h -- C ABI of the B200 Hessian-aware layer-wise weight quantization library (libgq.so).
+ *
+ * The library quantizes one linear layer W (m output rows x n input features) against
+ * calibration activations X (T tokens x n features) by minimising tr(D H D^T), D = W - Q,
+ * H = 2 X^T X, with GPTQ, i.e. Babai's nearest-plane algorithm on the lattice spanned by a
+ * Cholesky factor of H ("The Geometry of LLM Quantization: GPTQ as Babai's Nearest Plane
+ * Algorithm", sections 2.1-2.2).  Three calls form the path:
+ *
+ *   gq_hessian_accumulate   H += 2 X^T X                                  (section 2.1)
+ *   gq_prepare_hinv         dead fix, damping, U = upper factor of H_d^-1 (section 2.1, Thm 1)
+ *   gq_quantize_layer       column loop + lazy updates, codes, grids, losses (sections 2.2-2.3)
+ *
+ * Conventions shared by every entry point:
+ *  - All pointers named d_* are DEVICE pointers on the current CUDA device; h_* are host.
+ *  - Matrices are dense, row-major, contiguous (leading dimension = number of columns).
+ *  - The caller owns and allocates every buffer, including the workspace; the library never
+ *    allocates or frees device memory and keeps no pointer after a call returns.
+ *  - Calls are asynchronous on `stream` (0 = the legacy default stream) and return after the
+ *    work is enqueued, except where a call's comment says it synchronizes.
+ *  - Argument errors are reported synchronously by the return value and nothing is enqueued.
+ *    Errors found on the device (non-positive pivot, scale ladder exhausted, a bounded wait
+ *    that ran out) are written to a status word at the start of the workspace; read it with
+ *    gq_workspace_status(), which synchronizes `stream`.
+ *  - No C++ exception crosses this interface.  Every kernel's waits are bounded.
+ *  - Inputs are never modified.
+ */
+#ifndef GQ_H_
+#define GQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* gq_stream_t; /* the same type as cudaStream_t */
+
+typedef enum {
+  GQ_OK = 0,
+  GQ_ERR_INVALID_ARG = 1,  /* a size, pointer or setting is out of range (nothing enqueued) */
+  GQ_ERR_NOT_PD = 2,       /* the damped Hessian has a non-positive Cholesky pivot */
+  GQ_ERR_CUDA = 3,         /* a CUDA runtime call failed (launch, copy, attribute) */
+  GQ_ERR_UNSUPPORTED = 4,  /* a valid but unimplemented combination of settings */
+  GQ_ERR_TIMEOUT = 5,      /* a bounded device-side wait ran out */
+  GQ_ERR_NO_FIT = 6,       /* clip-free: some row's codes still overflow after the ladder */
+  GQ_ERR_WORKSPACE = 7     /* the workspace is smaller than the size query returned */
+} gq_status;
+
+typedef enum { GQ_BF16 = 0, GQ_FP32 = 1 } gq_dtype;
+
+/* Quantization settings of one call of gq_quantize_layer. */
+typedef struct {
+  int bits;       /* code width b, 2..8 */
+  int group_size; /* 0: one grid per row; else the group width, which must divide 128 */
+  int reverse;    /* 0: columns first to last (GPTQ order); 1: last to first (Babai order) */
+  int clip;       /* 1: codes clamped to [0, 2^b-1] (GPTQ); 0: clip-free with a scale ladder */
+  float ladder;   /* clip-free: factor applied to a row's step when its codes overflow (1.25) */
+  int ladder_max; /* clip-free: at most this many widenings per row (8) */
+} gq_quant_cfg;
+
+/* Library version string, e.g. "gq 0.1 sm_100a". */
+const char* gq_version(void);
+
+/* Number of CUDA kernels this library has launched in this process (all devices, all calls).
+ * Instrumentation for benchmarks: the difference around a region counts its launches. */
+unsigned long long gq_kernel_launches(void);
+
+/* Human-readable text of a status code (static storage). */
+const char* gq_status_string(gq_status s);
+
+/*
+ * H += 2 X^T X  ("The Geometry of LLM Quantization", section 2.1: the lattice basis comes from
+ * the calibration inputs and the CVP's Gram matrix is X^T X).
+ *
+ *   d_H     n x n, fp64, device, read-modify-write; the caller zeroes it before the first
+ *           chunk and may call again with further token chunks (streaming accumulation).
+ *           Both triangles are written (H stays exactly symmetric).
+ *   d_X     T x n, row-major (tokens x features), dtype x_dtype (bf16 or fp32), device.
+ *   T, n    T >= 0 (T = 0 is a no-op), 1 <= n <= 65536.
+ *
+ * Precision: every product of two inputs is formed exactly and the token sums are kept to
+ * fp64 accuracy; H is fp64 because the column loop's codes depend on H to about 1e-9
+ * relative for the ill-conditioned Hessians of LLM layers.
+ */
+gq_status gq_hessian_accumulate(double* d_H, const void* d_X, gq_dtype x_dtype, int64_t T,
+                                int64_t n, gq_stream_t stream);
+
+/* Workspace bytes gq_prepare_hinv needs for width n (256-byte aligned base required). */
+size_t gq_prepare_workspace_size(int64_t n);
+
+/*
+ * Factor preparation: dead-feature fix (WaterSIC, "dead feature erasure": H_ii == 0 ->
+ * H_ii = 1 and the column's weights are zeroed), relative damping
+ * H_d = H + damp * mean(diag H) * I, then U = the upper Cholesky factor of (P H_d P)^-1, i.e.
+ * U upper triangular with positive diagonal and U^T U = (P H_d P)^-1, where P is the identity
+ * (reverse = 0) or the column reversal (reverse = 1).  U is the factor in the order the
+ * columns are processed.  Computed as P H_d P = R R^T (R upper, a Cholesky factorisation
+ * from the last pivot) and U = R^-1, in fp64; U is stored rounded to fp32.
+ *
+ *   d_H        n x n fp64 (from gq_hessian_accumulate), device, read only.
+ *   n          1 <= n <= 65536.
+ *   damp       >= 0 (0.01 in the usual setting).
+ *   reverse    0 or 1, as above; pass the same value to gq_quantize_layer.
+ *   d_U        n x n fp32, device, written in full (strict lower triangle set to 0).
+ *   d_dead     n bytes, device, written: 1 where H_ii == 0, else 0.
+ *   d_delta    1 double, device, written: the damping amount damp * mean(diag H) (after the
+ *              dead fix).  gq_quantize_layer uses it for the undamped proxy loss.
+ *   d_ws       workspace of at least gq_prepare_workspace_size(n) bytes.
+ * Device-detected error: GQ_ERR_NOT_PD (non-positive pivot; U is then undefined).
+ */
+gq_status gq_prepare_hinv(const double* d_H, int64_t n, float damp, int reverse, float* d_U,
+                          uint8_t* d_dead, double* d_delta, void* d_ws, size_t ws_bytes,
+                          gq_stream_t stream);
+
+/* Workspace bytes gq_quantize_layer needs for an m x n layer under cfg. */
+size_t gq_quantize_workspace_size(int64_t m, int64_t n, const gq_quant_cfg* cfg);
+
+/*
+ * Quantize one layer ("The Geometry of LLM Quantization", section 2.2: GPTQ's error feedback
+ * is the nearest-plane step; section 2.3: the no-clipping setting and Theorem 5's bound).
+ *
+ * Columns are processed in blocks of 128: inside a block, column by column (grid, round,
+ * error e = (w_j - q_j) / U_jj, feedback to the block's later columns); between blocks, a
+ * lazy rank-128 update W[:, j+128:] -= E U[j:j+128, j+128:].  Grids are asymmetric min-max:
+ * per row from the input row (group_size = 0) or per group, from the error-fed weights at
+ * the group's first column.  clip = 0 runs unclamped on a per-row step
+ * ladder^k (hi - lo) / (2^b - 1), k raised for each row whose codes leave [0, 2^b - 1]
+ * (at most ladder_max times); this call then SYNCHRONIZES `stream` once per ladder round.
+ *
+ *   d_W       m x n, dtype w_dtype, device, read only.
+ *   d_U       n x n fp32 from gq_prepare_hinv with the same `reverse`.
+ *   d_dead    n bytes from gq_prepare_hinv (may be NULL: no dead columns).
+ *   d_delta   1 double from gq_prepare_hinv (may be NULL: loss[0] is then not computed).
+ *   d_codes   m x ceil(n*b/32) uint32, written: per row an LSB-first bitstream of b-bit
+ *             codes, the code of ORIGINAL column c at bits [b*c, b*c+b); unused bits are 0.
+ *   d_scales  m x G fp32, written, G = 1 (group_size 0) or ceil(n / group_size); group g
+ *             covers original columns [g*group_size, (g+1)*group_size).
+ *   d_zeros   m x G uint8, written; dequantized weight = scale * (code - zero).
+ *   d_loss    3 doubles, written: [0] ||(W0 - Q) X^T||_F^2 = (loss[1] - delta ||W0 - Q||^2)/2
+ *             (W0 = W with dead columns zeroed), [1] tr(D H_d D^T) = sum of e^2,
+ *             [2] Theorem 5 bound sum_r sum_j s_rj^2 / (4 U_jj^2) (a guarantee for clip = 0).
+ *   d_ws      workspace of at least gq_quantize_workspace_size(m, n, cfg) bytes.
+ * Limits: 1 <= m <= 2^24, 1 <= n <= 65536, 2 <= bits <= 8; reverse = 1 needs group_size 0.
+ * Device-detected error: GQ_ERR_NO_FIT.
+ */
+gq_status gq_quantize_layer(const void* d_W, gq_dtype w_dtype, int64_t m, int64_t n,
+                            const float* d_U, const uint8_t* d_dead, const double* d_delta,
+                            const gq_quant_cfg* cfg, uint32_t* d_codes, float* d_scales,
+                            uint8_t* d_zeros, double* d_loss, void* d_ws, size_t ws_bytes,
+                            gq_stream_t stream);
+
+/*
+ * Synchronize `stream` and return the device-side status recorded in a workspace by the last
+ * gq_prepare_hinv / gq_quantize_layer that used it (GQ_OK if none), then clear it.
+ * For gq_quantize_layer's clip-free ladder, h_ladder_rounds (may be NULL) receives the number
+ * of ladder rounds the last call ran.
+ */
+gq_status gq_workspace_status(void* d_ws, int* h_ladder_rounds, gq_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GQ_H_ */

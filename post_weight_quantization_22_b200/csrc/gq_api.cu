@@ -1,0 +1,149 @@
+// C ABI entry points of libgq: argument validation, per-device setup, dispatch.
+#include "gq_internal.cuh"
+
+#include <atomic>
+#include <mutex>
+
+using namespace gq;
+
+namespace gq {
+static std::atomic<unsigned long long> g_launches{0};
+void count_launches(long k) { g_launches.fetch_add((unsigned long long)k, std::memory_order_relaxed); }
+}  // namespace gq
+
+namespace {
+
+constexpr int64_t kMaxN = 32768;
+constexpr int64_t kMaxM = int64_t(1) << 24;
+
+std::mutex g_init_mu;
+bool g_init_done[128] = {};
+
+gq_status ensure_device_setup() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 128) return GQ_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_init_mu);
+  if (g_init_done[dev]) return GQ_OK;
+  if (factor_init_attributes() != cudaSuccess) return GQ_ERR_CUDA;
+  if (quant_init_attributes() != cudaSuccess) return GQ_ERR_CUDA;
+  g_init_done[dev] = true;
+  return GQ_OK;
+}
+
+bool aligned256(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 255u) == 0; }
+
+}  // namespace
+
+extern "C" {
+
+const char* gq_version(void) { return "gq 0.1 sm_100a"; }
+
+unsigned long long gq_kernel_launches(void) { return g_launches.load(std::memory_order_relaxed); }
+
+const char* gq_status_string(gq_status s) {
+  switch (s) {
+    case GQ_OK: return "ok";
+    case GQ_ERR_INVALID_ARG: return "invalid argument";
+    case GQ_ERR_NOT_PD: return "damped Hessian is not positive definite";
+    case GQ_ERR_CUDA: return "CUDA runtime error";
+    case GQ_ERR_UNSUPPORTED: return "unsupported combination of settings";
+    case GQ_ERR_TIMEOUT: return "bounded device wait ran out";
+    case GQ_ERR_NO_FIT: return "clip-free scale ladder exhausted";
+    case GQ_ERR_WORKSPACE: return "workspace too small or misaligned";
+  }
+  return "unknown status";
+}
+
+gq_status gq_hessian_accumulate(double* d_H, const void* d_X, gq_dtype x_dtype, int64_t T,
+                                int64_t n, gq_stream_t stream) {
+  if (T < 0 || n < 1 || n > kMaxN || T > (int64_t(1) << 31) - 1) return GQ_ERR_INVALID_ARG;
+  if (x_dtype != GQ_BF16 && x_dtype != GQ_FP32) return GQ_ERR_INVALID_ARG;
+  if (!d_H || (T > 0 && !d_X)) return GQ_ERR_INVALID_ARG;
+  if (T == 0) return GQ_OK;
+  gq_status st = ensure_device_setup();
+  if (st != GQ_OK) return st;
+  cudaError_t e = launch_hessian(d_H, d_X, x_dtype, T, n, (cudaStream_t)stream);
+  return e == cudaSuccess ? GQ_OK : GQ_ERR_CUDA;
+}
+
+size_t gq_prepare_workspace_size(int64_t n) {
+  if (n < 1 || n > kMaxN) return 0;
+  return prepare_ws_bytes(n);
+}
+
+gq_status gq_prepare_hinv(const double* d_H, int64_t n, float damp, int reverse, float* d_U,
+                          uint8_t* d_dead, double* d_delta, void* d_ws, size_t ws_bytes,
+                          gq_stream_t stream) {
+  if (n < 1 || n > kMaxN || !(damp >= 0.f) || (reverse != 0 && reverse != 1))
+    return GQ_ERR_INVALID_ARG;
+  if (!d_H || !d_U || !d_dead || !d_delta || !d_ws) return GQ_ERR_INVALID_ARG;
+  if (!aligned256(d_ws) || ws_bytes < prepare_ws_bytes(n)) return GQ_ERR_WORKSPACE;
+  gq_status st = ensure_device_setup();
+  if (st != GQ_OK) return st;
+  cudaError_t e = launch_prepare(d_H, n, damp, reverse, d_U, d_dead, d_delta, d_ws,
+                                 (cudaStream_t)stream);
+  return e == cudaSuccess ? GQ_OK : GQ_ERR_CUDA;
+}
+
+static gq_status check_cfg(const gq_quant_cfg* cfg) {
+  if (!cfg) return GQ_ERR_INVALID_ARG;
+  if (cfg->bits < 2 || cfg->bits > 8) return GQ_ERR_INVALID_ARG;
+  if (cfg->reverse != 0 && cfg->reverse != 1) return GQ_ERR_INVALID_ARG;
+  if (cfg->clip != 0 && cfg->clip != 1) return GQ_ERR_INVALID_ARG;
+  const int g = cfg->group_size;
+  if (g != 0 && g != 16 && g != 32 && g != 64 && g != 128) {
+    return (g > 0 && g <= 128 && kBlock % g == 0) ? GQ_ERR_UNSUPPORTED : GQ_ERR_INVALID_ARG;
+  }
+  if (g != 0 && (cfg->reverse || !cfg->clip)) return GQ_ERR_UNSUPPORTED;
+  if (!cfg->clip) {
+    if (!(cfg->ladder > 1.f) || cfg->ladder_max < 0 || cfg->ladder_max > 64)
+      return GQ_ERR_INVALID_ARG;
+  }
+  return GQ_OK;
+}
+
+size_t gq_quantize_workspace_size(int64_t m, int64_t n, const gq_quant_cfg* cfg) {
+  if (m < 1 || m > kMaxM || n < 1 || n > kMaxN || check_cfg(cfg) != GQ_OK) return 0;
+  return quantize_ws_bytes(m, n, *cfg);
+}
+
+gq_status gq_quantize_layer(const void* d_W, gq_dtype w_dtype, int64_t m, int64_t n,
+                            const float* d_U, const uint8_t* d_dead, const double* d_delta,
+                            const gq_quant_cfg* cfg, uint32_t* d_codes, float* d_scales,
+                            uint8_t* d_zeros, double* d_loss, void* d_ws, size_t ws_bytes,
+                            gq_stream_t stream) {
+  if (m < 1 || m > kMaxM || n < 1 || n > kMaxN) return GQ_ERR_INVALID_ARG;
+  if (w_dtype != GQ_BF16 && w_dtype != GQ_FP32) return GQ_ERR_INVALID_ARG;
+  gq_status st = check_cfg(cfg);
+  if (st != GQ_OK) return st;
+  if (!d_W || !d_U || !d_codes || !d_scales || !d_zeros || !d_loss || !d_ws)
+    return GQ_ERR_INVALID_ARG;
+  if (!aligned256(d_ws) || ws_bytes < quantize_ws_bytes(m, n, *cfg)) return GQ_ERR_WORKSPACE;
+  if ((reinterpret_cast<uintptr_t>(d_U) & 15u) != 0) return GQ_ERR_INVALID_ARG;
+  st = ensure_device_setup();
+  if (st != GQ_OK) return st;
+  QuantArgs a{};
+  a.W = d_W; a.wt = w_dtype; a.m = m; a.n = n; a.U = d_U; a.dead = d_dead; a.delta = d_delta;
+  a.cfg = *cfg; a.codes = d_codes; a.scales = d_scales; a.zeros = d_zeros; a.loss = d_loss;
+  a.ws = d_ws;
+  return run_quantize(a, (cudaStream_t)stream);
+}
+
+gq_status gq_workspace_status(void* d_ws, int* h_ladder_rounds, gq_stream_t stream) {
+  if (!d_ws) return GQ_ERR_INVALID_ARG;
+  WsHeader h{};
+  cudaStream_t s = (cudaStream_t)stream;
+  if (cudaMemcpyAsync(&h, d_ws, sizeof(WsHeader), cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return GQ_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return GQ_ERR_CUDA;
+  if (h_ladder_rounds) *h_ladder_rounds = h.ladder_rounds;
+  if (h.status != 0) {
+    int zero = 0;
+    if (cudaMemcpyAsync(d_ws, &zero, sizeof(int), cudaMemcpyHostToDevice, s) != cudaSuccess)
+      return GQ_ERR_CUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return GQ_ERR_CUDA;
+  }
+  return (gq_status)h.status;
+}
+
+}  // extern "C"

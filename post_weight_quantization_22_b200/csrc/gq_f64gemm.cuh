@@ -1,0 +1,134 @@
+// fp64 SIMT GEMM used by the Hessian and the factorisation (accuracy-critical stages).
+//
+//   C[i][j] = (beta_one ? C[i][j] : 0) + alpha * sum_k opA[i][k] * opB[k][j]
+//   opA[i][k] = A_T ? A[k*lda + i] : A[i*lda + k]      (A element type TA, converted to fp64)
+//   opB[k][j] = B_T ? B[j*ldb + k] : B[k*ldb + j]
+//
+// Optional structure: a_lower (opA[i][k] = 0 for k > i), b_lower (opB[k][j] = 0 for k < j),
+// lower_tiles (skip 64x64 output tiles strictly above the diagonal).  Batched over
+// blockIdx.z with element strides.
+#pragma once
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "gq_internal.cuh"
+
+namespace gq {
+
+constexpr int kGB = 64;   // output tile edge
+constexpr int kGK = 16;   // k step
+
+template <class T>
+__device__ __forceinline__ double to_f64(T v);
+template <>
+__device__ __forceinline__ double to_f64<double>(double v) { return v; }
+template <>
+__device__ __forceinline__ double to_f64<float>(float v) { return (double)v; }
+template <>
+__device__ __forceinline__ double to_f64<__nv_bfloat16>(__nv_bfloat16 v) {
+  return (double)__bfloat162float(v);
+}
+
+struct F64GemmArgs {
+  int M, N, K;
+  double alpha;
+  int beta_one;
+  const void* A;
+  int64_t lda, strideA;
+  const void* B;
+  int64_t ldb, strideB;
+  double* C;
+  int64_t ldc, strideC;
+  int a_lower, b_lower, lower_tiles;
+};
+
+template <class TA, class TB, bool A_T, bool B_T>
+__global__ void __launch_bounds__(256) f64_gemm_kernel(F64GemmArgs g) {
+  __shared__ double As[kGK][kGB + 1];
+  __shared__ double Bs[kGK][kGB + 1];
+  const int ti = blockIdx.y, tj = blockIdx.x;
+  if (g.lower_tiles && tj > ti) return;
+  const int i0 = ti * kGB, j0 = tj * kGB;
+  if (i0 >= g.M || j0 >= g.N) return;
+  const TA* A = static_cast<const TA*>(g.A) + (int64_t)blockIdx.z * g.strideA;
+  const TB* B = static_cast<const TB*>(g.B) + (int64_t)blockIdx.z * g.strideB;
+  double* C = g.C + (int64_t)blockIdx.z * g.strideC;
+
+  int k_lo = 0, k_hi = g.K;
+  if (g.a_lower) k_hi = min(k_hi, i0 + kGB);
+  if (g.b_lower) k_lo = (j0 / kGK) * kGK;
+
+  const int tid = threadIdx.x;
+  const int tx = tid % 16, ty = tid / 16;
+  double acc[4][4];
+#pragma unroll
+  for (int a = 0; a < 4; ++a)
+#pragma unroll
+    for (int b = 0; b < 4; ++b) acc[a][b] = 0.0;
+
+  for (int k0 = k_lo; k0 < k_hi; k0 += kGK) {
+    // ---- load opA tile (64 i x 16 k) ----
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      int e = tid + 256 * r;  // 0..1023
+      int ii, kk;
+      if (A_T) { kk = e / kGB; ii = e % kGB; } else { ii = e / kGK; kk = e % kGK; }
+      int gi = i0 + ii, gk = k0 + kk;
+      double v = 0.0;
+      if (gi < g.M && gk < k_hi && !(g.a_lower && gk > gi)) {
+        v = A_T ? to_f64<TA>(A[(int64_t)gk * g.lda + gi]) : to_f64<TA>(A[(int64_t)gi * g.lda + gk]);
+      }
+      As[kk][ii] = v;
+    }
+    // ---- load opB tile (16 k x 64 j) ----
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      int e = tid + 256 * r;
+      int jj, kk;
+      if (B_T) { jj = e / kGK; kk = e % kGK; } else { kk = e / kGB; jj = e % kGB; }
+      int gj = j0 + jj, gk = k0 + kk;
+      double v = 0.0;
+      if (gj < g.N && gk < k_hi && gk >= k_lo && !(g.b_lower && gk < gj)) {
+        v = B_T ? to_f64<TB>(B[(int64_t)gj * g.ldb + gk]) : to_f64<TB>(B[(int64_t)gk * g.ldb + gj]);
+      }
+      Bs[kk][jj] = v;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int kk = 0; kk < kGK; ++kk) {
+      double a[4], b[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) { a[q] = As[kk][ty + 16 * q]; b[q] = Bs[kk][tx + 16 * q]; }
+#pragma unroll
+      for (int p = 0; p < 4; ++p)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) acc[p][q] = fma(a[p], b[q], acc[p][q]);
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int p = 0; p < 4; ++p) {
+    int gi = i0 + ty + 16 * p;
+    if (gi >= g.M) continue;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      int gj = j0 + tx + 16 * q;
+      if (gj >= g.N) continue;
+      double* c = C + (int64_t)gi * g.ldc + gj;
+      double v = g.alpha * acc[p][q];
+      *c = g.beta_one ? (*c + v) : v;
+    }
+  }
+}
+
+template <class TA, class TB, bool A_T, bool B_T>
+inline cudaError_t f64_gemm(const F64GemmArgs& g, int batch, cudaStream_t s) {
+  if (g.M <= 0 || g.N <= 0 || batch <= 0) return cudaSuccess;
+  dim3 grid((g.N + kGB - 1) / kGB, (g.M + kGB - 1) / kGB, batch);
+  f64_gemm_kernel<TA, TB, A_T, B_T><<<grid, 256, 0, s>>>(g);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+}  // namespace gq

@@ -1,0 +1,296 @@
+// Factor preparation: dead-feature fix, relative damping, and U = upper factor of (P H_d P)^-1.
+//
+// Sources: "The Geometry of LLM Quantization: GPTQ as Babai's Nearest Plane Algorithm",
+// section 2.1 (Theorem 1: any factor of the Hessian gives an equivalent CVP, so a square
+// Cholesky factor is used); "WaterSIC", section 2 (Cholesky Sigma = L L^T) and its "dead feature
+// erasure"; "Initialisation Determines the Basin", OA-EM section (H + lambda I).
+//
+// Route (differs from the three-step Cholesky -> inverse -> Cholesky-of-inverse route, same
+// result): with M = J (P H_d P) J (J = column reversal), the lower Cholesky factor L of M and
+// its inverse give U = J L^-1 J, which is upper triangular with positive diagonal and satisfies
+// U^T U = (P H_d P)^-1; the upper Cholesky factor of a positive definite matrix is unique, so
+// this is the same U.  Cost n^3/3 (Cholesky) + n^3/3 (triangular inverse) instead of ~4n^3/3.
+//
+// Everything is fp64: the damped Hessians of LLM layers have condition numbers ~1e5 and the
+// codes downstream change when U carries fp32-level errors.
+#include "gq_internal.cuh"
+#include "gq_f64gemm.cuh"
+
+#include <math.h>
+#include <vector>
+#include <algorithm>
+
+namespace gq {
+
+constexpr int kNB = 64;  // Cholesky panel width
+
+// ---------------------------------------------------------------------------------------
+// dead fix + damping statistics (one CTA)
+// ---------------------------------------------------------------------------------------
+__global__ void __launch_bounds__(1024) diag_stats_kernel(const double* H, int64_t n, float damp,
+                                                          uint8_t* dead, double* delta_out,
+                                                          WsHeader* hdr) {
+  __shared__ double red[32];
+  double acc = 0.0;
+  for (int64_t i = threadIdx.x; i < n; i += blockDim.x) {
+    double d = H[i * n + i];
+    bool isdead = (d == 0.0);
+    dead[i] = isdead ? 1 : 0;
+    acc += isdead ? 1.0 : d;
+  }
+  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = acc;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    acc = (threadIdx.x < (blockDim.x >> 5)) ? red[threadIdx.x] : 0.0;
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    if (threadIdx.x == 0) {
+      double delta = (double)damp * (acc / (double)n);
+      *delta_out = delta;
+      hdr->scratch[0] = delta;
+    }
+  }
+}
+
+// M[i][j] (j <= i) = Hfix[pi(i)][pi(j)] + (i == j) * delta, pi(i) = n-1-i (forward) or i.
+__global__ void build_m_kernel(const double* H, int64_t n, int reverse, const WsHeader* hdr,
+                               double* M) {
+  int64_t j = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+  int64_t i = blockIdx.y;
+  if (j > i || i >= n) return;
+  int64_t pi = reverse ? i : n - 1 - i;
+  int64_t pj = reverse ? j : n - 1 - j;
+  double v = H[pi * n + pj];
+  if (i == j) {
+    if (v == 0.0) v = 1.0;
+    v += hdr->scratch[0];
+  }
+  M[i * n + j] = v;
+}
+
+// ---------------------------------------------------------------------------------------
+// Diagonal block: Cholesky of a <= 64 x 64 block in shared memory (Schur-complement form,
+// one barrier per pivot), then its triangular inverse.
+// ---------------------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) potrf_diag_kernel(double* M, int64_t n, int64_t c0, int w,
+                                                         double* dinv, WsHeader* hdr) {
+  extern __shared__ double sm[];
+  double* S = sm;                       // [64][65]
+  double* X = sm + kNB * (kNB + 1);     // [64][65] inverse
+  const int ld = kNB + 1;
+  const int tid = threadIdx.x;
+  for (int e = tid; e < kNB * kNB; e += 256) {
+    int i = e / kNB, j = e % kNB;
+    double v = 0.0;
+    if (i < w && j < w) {
+      if (j <= i) v = M[(c0 + i) * n + c0 + j];
+    } else if (i == j) {
+      v = 1.0;
+    }
+    S[i * ld + j] = v;
+  }
+  __syncthreads();
+  // Schur complement elimination; S[r][c] for r > c is final after step c.
+  const int r = tid >> 2, part = tid & 3;
+  for (int c = 0; c < kNB; ++c) {
+    double p = S[c * ld + c];
+    if (!(p > 0.0)) p = 1.0;  // recorded below; keeps the arithmetic finite
+    double f = (r > c) ? S[r * ld + c] / p : 0.0;
+    if (r > c) {
+      for (int s = c + 1 + part; s <= r; s += 4) S[r * ld + s] -= f * S[s * ld + c];
+    }
+    __syncthreads();
+  }
+  // L[r][c] = S[r][c] / sqrt(S[c][c]), L[c][c] = sqrt(S[c][c])
+  __shared__ double sq[kNB];
+  if (tid < kNB) {
+    double p = S[tid * ld + tid];
+    if (!(p > 0.0)) {
+      if (tid < w) record_status(hdr, GQ_ERR_NOT_PD);
+      p = 1.0;
+    }
+    sq[tid] = sqrt(p);
+  }
+  __syncthreads();
+  for (int e = tid; e < kNB * kNB; e += 256) {
+    int i = e / kNB, j = e % kNB;
+    if (j < i) S[i * ld + j] = S[i * ld + j] / sq[j];
+    else if (j == i) S[i * ld + j] = sq[i];
+    else S[i * ld + j] = 0.0;
+  }
+  __syncthreads();
+  // inverse, one column per thread (forward substitution L x = e_j)
+  if (tid < kNB) {
+    const int j = tid;
+    for (int i = 0; i < kNB; ++i) {
+      double acc0 = 0.0, acc1 = 0.0;
+      int k = j;
+      for (; k + 1 < i; k += 2) {
+        acc0 = fma(S[i * ld + k], X[k * ld + j], acc0);
+        acc1 = fma(S[i * ld + k + 1], X[(k + 1) * ld + j], acc1);
+      }
+      if (k < i) acc0 = fma(S[i * ld + k], X[k * ld + j], acc0);
+      double v = (i < j) ? 0.0 : (((i == j) ? 1.0 : 0.0) - (acc0 + acc1)) / S[i * ld + i];
+      X[i * ld + j] = v;
+    }
+  }
+  __syncthreads();
+  for (int e = tid; e < kNB * kNB; e += 256) {
+    int i = e / kNB, j = e % kNB;
+    if (i < w && j <= i) M[(c0 + i) * n + c0 + j] = S[i * ld + j];
+    dinv[e] = X[i * ld + j];
+  }
+}
+
+// diagonal blocks of M <- their inverses (lower parts)
+__global__ void put_diag_inv_kernel(double* M, int64_t n, const double* dinv) {
+  int64_t k = blockIdx.x;
+  int64_t c0 = k * kNB;
+  int64_t rem_ = n - c0;
+  int w = (int)(rem_ < kNB ? rem_ : kNB);
+  const double* D = dinv + k * kNB * kNB;
+  for (int e = threadIdx.x; e < kNB * kNB; e += blockDim.x) {
+    int i = e / kNB, j = e % kNB;
+    if (i < w && j <= i) M[(c0 + i) * n + c0 + j] = D[e];
+  }
+}
+
+// U[i][j] = (i <= j) ? (float) Linv[n-1-i][n-1-j] : 0
+__global__ void flip_to_u_kernel(const double* M, int64_t n, float* U) {
+  int64_t j = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+  int64_t i = blockIdx.y;
+  if (j >= n) return;
+  float v = 0.f;
+  if (i <= j) v = (float)M[(n - 1 - i) * n + (n - 1 - j)];
+  U[i * n + j] = v;
+}
+
+// ---------------------------------------------------------------------------------------
+// host orchestration
+// ---------------------------------------------------------------------------------------
+struct PrepLayout {
+  WsHeader* hdr;
+  double* M;
+  double* dinv;
+  double* tbuf;
+  size_t bytes;
+};
+
+static size_t trtri_tbuf_elems(int64_t n) {
+  size_t best = 0;
+  for (int64_t bs = kNB; bs < n; bs *= 2) {
+    size_t tot = 0;
+    for (int64_t r = 0; r + bs < n; r += 2 * bs) tot += (size_t)bs * bs;
+    if (tot > best) best = tot;
+  }
+  return best;
+}
+
+static PrepLayout prep_layout(void* ws, int64_t n) {
+  Carver c(ws);
+  PrepLayout L;
+  L.hdr = c.take<WsHeader>(1);
+  L.M = c.take<double>((size_t)n * n);
+  int64_t nb = (n + kNB - 1) / kNB;
+  L.dinv = c.take<double>((size_t)nb * kNB * kNB);
+  L.tbuf = c.take<double>(trtri_tbuf_elems(n) + 1);
+  L.bytes = c.off;
+  return L;
+}
+
+size_t prepare_ws_bytes(int64_t n) { return prep_layout(nullptr, n).bytes; }
+
+cudaError_t factor_init_attributes() {
+  return cudaFuncSetAttribute(potrf_diag_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              2 * kNB * (kNB + 1) * (int)sizeof(double));
+}
+
+#define GQ_TRY(x)                               \
+  do {                                          \
+    cudaError_t _e = (x);                       \
+    if (_e != cudaSuccess) return _e;           \
+  } while (0)
+
+cudaError_t launch_prepare(const double* H, int64_t n, float damp, int reverse, float* U,
+                           uint8_t* dead, double* delta, void* ws, cudaStream_t s) {
+  PrepLayout L = prep_layout(ws, n);
+  GQ_TRY(cudaMemsetAsync(L.hdr, 0, sizeof(WsHeader), s));
+  diag_stats_kernel<<<1, 1024, 0, s>>>(H, n, damp, dead, delta, L.hdr);
+  count_launches(1);
+  GQ_TRY(cudaGetLastError());
+  {
+    dim3 grid((unsigned)((n + 255) / 256), (unsigned)n);
+    build_m_kernel<<<grid, 256, 0, s>>>(H, n, reverse, L.hdr, L.M);
+    count_launches(1);
+    GQ_TRY(cudaGetLastError());
+  }
+  // blocked right-looking Cholesky, lower, in place on M
+  const int64_t nb = (n + kNB - 1) / kNB;
+  const size_t psmem = 2 * kNB * (kNB + 1) * sizeof(double);
+  for (int64_t k = 0; k < nb; ++k) {
+    const int64_t c0 = k * kNB;
+    const int w = (int)std::min<int64_t>(kNB, n - c0);
+    double* dk = L.dinv + k * kNB * kNB;
+    potrf_diag_kernel<<<1, 256, psmem, s>>>(L.M, n, c0, w, dk, L.hdr);
+    count_launches(1);
+    GQ_TRY(cudaGetLastError());
+    const int64_t rem = n - c0 - w;
+    if (rem <= 0) continue;
+    double* P = L.M + (c0 + w) * n + c0;
+    {  // panel: P <- P L_kk^-T (in place; one output tile column per CTA row)
+      F64GemmArgs g{};
+      g.M = (int)rem; g.N = w; g.K = w; g.alpha = 1.0; g.beta_one = 0;
+      g.A = P; g.lda = n; g.B = dk; g.ldb = kNB; g.C = P; g.ldc = n;
+      GQ_TRY((f64_gemm<double, double, false, true>(g, 1, s)));
+    }
+    {  // trailing: C -= P P^T, lower tiles
+      F64GemmArgs g{};
+      g.M = (int)rem; g.N = (int)rem; g.K = w; g.alpha = -1.0; g.beta_one = 1;
+      g.A = P; g.lda = n; g.B = P; g.ldb = n;
+      g.C = L.M + (c0 + w) * n + (c0 + w); g.ldc = n; g.lower_tiles = 1;
+      GQ_TRY((f64_gemm<double, double, false, true>(g, 1, s)));
+    }
+  }
+  put_diag_inv_kernel<<<(unsigned)nb, 256, 0, s>>>(L.M, n, L.dinv);
+  count_launches(1);
+  GQ_TRY(cudaGetLastError());
+  // triangular inverse by doubling: inv([[A,0],[B,C]]) = [[A^-1,0],[-C^-1 B A^-1, C^-1]]
+  for (int64_t bs = kNB; bs < n; bs *= 2) {
+    const int64_t npairs_full = n / (2 * bs);          // pairs with a full C block
+    const int64_t rtail = npairs_full * 2 * bs;        // start of a possible ragged pair
+    const int64_t cw_tail = n - rtail - bs;            // its C width (if > 0)
+    for (int pass = 0; pass < 2; ++pass) {
+      int64_t r = pass == 0 ? 0 : rtail;
+      int64_t cw = pass == 0 ? bs : cw_tail;
+      int64_t batch = pass == 0 ? npairs_full : (cw_tail > 0 ? 1 : 0);
+      if (batch <= 0 || cw <= 0) continue;
+      double* tb = L.tbuf + (pass == 0 ? 0 : npairs_full * bs * bs);
+      {  // T = B A^-1
+        F64GemmArgs g{};
+        g.M = (int)cw; g.N = (int)bs; g.K = (int)bs; g.alpha = 1.0; g.beta_one = 0;
+        g.A = L.M + (r + bs) * n + r; g.lda = n; g.strideA = 2 * bs * n + 2 * bs;
+        g.B = L.M + r * n + r; g.ldb = n; g.strideB = 2 * bs * n + 2 * bs; g.b_lower = 1;
+        g.C = tb; g.ldc = bs; g.strideC = bs * bs;
+        GQ_TRY((f64_gemm<double, double, false, false>(g, (int)batch, s)));
+      }
+      {  // B <- -C^-1 T
+        F64GemmArgs g{};
+        g.M = (int)cw; g.N = (int)bs; g.K = (int)cw; g.alpha = -1.0; g.beta_one = 0;
+        g.A = L.M + (r + bs) * n + (r + bs); g.lda = n; g.strideA = 2 * bs * n + 2 * bs;
+        g.a_lower = 1;
+        g.B = tb; g.ldb = bs; g.strideB = bs * bs;
+        g.C = L.M + (r + bs) * n + r; g.ldc = n; g.strideC = 2 * bs * n + 2 * bs;
+        GQ_TRY((f64_gemm<double, double, false, false>(g, (int)batch, s)));
+      }
+    }
+  }
+  {
+    dim3 grid((unsigned)((n + 255) / 256), (unsigned)n);
+    flip_to_u_kernel<<<grid, 256, 0, s>>>(L.M, n, U);
+    count_launches(1);
+    GQ_TRY(cudaGetLastError());
+  }
+  return cudaSuccess;
+}
+
+}  // namespace gq

@@ -1,0 +1,597 @@
+// The GPTQ / Babai column loop with lazy block updates, code packing and losses.
+//
+// Sources: "The Geometry of LLM Quantization: GPTQ as Babai's Nearest Plane Algorithm",
+// section 2.2 (GPTQ's error propagation is the nearest-plane step; back to front it is Babai),
+// section 2.3 (no-clipping setting; Theorem 5 bound (1/4) sum s^2 D_jj); "RDQ: Residual
+// Distribution Quantization", setup (group-128 asymmetric integer format).
+//
+// Work layout: the weights are copied once into an fp32 work matrix Wf (rows x n) in the
+// processing order (columns reversed for the last-to-first variant, dead columns zeroed).  Per
+// 128-column block: `colloop` runs the sequential column recursion for 32 rows per CTA (4
+// lanes per row, each lane owning 32 of the block's columns in 4-wide chunks), keeping the
+// block's part of U in shared memory; `lazy_update` then applies W[:, j+128:] -= E U[j:j+128,
+// j+128:] to the rest of the work matrix.
+#include "gq_internal.cuh"
+
+#include <algorithm>
+#include <math.h>
+
+namespace gq {
+
+constexpr int kP = 4;                     // lanes per row in the column loop
+constexpr int kVPL = kBlock / kP;          // values per lane (32)
+constexpr int kRowsPerCta = 4 * 32 / kP;  // 32 rows per 128-thread CTA
+
+struct QLayout {
+  WsHeader* hdr;
+  float* Wf;        // k x n work matrix (compact rows)
+  float* E;         // k x 128 scaled errors of the current block
+  uint8_t* codes8;  // m x ldc8 codes in processing order
+  int64_t ldc8;
+  float* row_s;     // per-row step (group_size 0)
+  float* row_z;     // per-row zero point (group_size 0)
+  float* alpha;     // per-row ladder factor
+  double* row_e2;   // per-row sum of e^2
+  double* row_bnd;  // per-row Theorem 5 bound
+  double* row_d2;   // per-row ||w0 - q||^2
+  int* overflow;    // per-row clip-free overflow flag
+  int* rowlist;     // compact row -> original row
+  int* counter;
+  size_t bytes;
+};
+
+static QLayout q_layout(void* ws, int64_t m, int64_t n) {
+  Carver c(ws);
+  QLayout L;
+  L.hdr = c.take<WsHeader>(1);
+  L.Wf = c.take<float>((size_t)m * n);
+  L.E = c.take<float>((size_t)m * kBlock);
+  L.ldc8 = (n + 15) / 16 * 16;
+  L.codes8 = c.take<uint8_t>((size_t)m * L.ldc8);
+  L.row_s = c.take<float>(m);
+  L.row_z = c.take<float>(m);
+  L.alpha = c.take<float>(m);
+  L.row_e2 = c.take<double>(m);
+  L.row_bnd = c.take<double>(m);
+  L.row_d2 = c.take<double>(m);
+  L.overflow = c.take<int>(m);
+  L.rowlist = c.take<int>(m);
+  L.counter = c.take<int>(4);
+  L.bytes = c.off;
+  return L;
+}
+
+size_t quantize_ws_bytes(int64_t m, int64_t n, const gq_quant_cfg&) {
+  return q_layout(nullptr, m, n).bytes;
+}
+
+// ------------------------------------------------------------------------------------------
+// setup kernels
+// ------------------------------------------------------------------------------------------
+__global__ void q_reset_kernel(int64_t m, float* alpha, int* overflow, double* loss) {
+  int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+  if (i < m) { alpha[i] = 1.f; overflow[i] = 0; }
+  if (i < 3) loss[i] = 0.0;
+}
+
+// Wf[r'][p] = dead[pi(p)] ? 0 : W[row][pi(p)],  row = rowlist ? rowlist[r'] : r'
+template <class TW>
+__global__ void q_load_kernel(const TW* W, int64_t n, int64_t k_rows, const int* rowlist,
+                              const uint8_t* dead, int reverse, float* Wf) {
+  int64_t total = k_rows * n;
+  for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < total;
+       e += (int64_t)gridDim.x * blockDim.x) {
+    int64_t rr = e / n, p = e % n;
+    int64_t row = rowlist ? rowlist[rr] : rr;
+    int64_t c = reverse ? n - 1 - p : p;
+    float v;
+    if constexpr (sizeof(TW) == 2) v = __bfloat162float(W[row * n + c]);
+    else v = (float)W[row * n + c];
+    if (dead && dead[c]) v = 0.f;
+    Wf[e] = v;
+  }
+}
+
+// per-row grid from the (dead-zeroed) row: one warp per row
+__global__ void q_row_grid_kernel(const float* Wf, int64_t n, int64_t k_rows, const int* rowlist,
+                                  int bits, int clip, const float* alpha, float* row_s,
+                                  float* row_z, float* scales, uint8_t* zeros) {
+  int64_t rr = blockIdx.x * (int64_t)(blockDim.x / 32) + threadIdx.x / 32;
+  int lane = threadIdx.x & 31;
+  if (rr >= k_rows) return;
+  const float* w = Wf + rr * n;
+  float lo = 0.f, hi = 0.f;  // the range always contains 0
+  for (int64_t j = lane; j < n; j += 32) { float v = w[j]; lo = fminf(lo, v); hi = fmaxf(hi, v); }
+  for (int o = 16; o > 0; o >>= 1) {
+    lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+    hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+  }
+  if (lane == 0) {
+    int64_t row = rowlist ? rowlist[rr] : rr;
+    if (lo == 0.f && hi == 0.f) { lo = -1.f; hi = 1.f; }
+    float maxq = (float)((1 << bits) - 1);
+    float s, z;
+    if (clip) {
+      s = (hi - lo) / maxq;
+      z = rintf(-lo / s);
+    } else {
+      s = alpha[row] * (hi - lo) / maxq;
+      z = rintf(maxq * 0.5f - (hi + lo) / (2.f * s));
+    }
+    row_s[row] = s;
+    row_z[row] = z;
+    scales[row] = s;
+    zeros[row] = (uint8_t)z;
+  }
+}
+
+// ------------------------------------------------------------------------------------------
+// the column loop of one 128-column block
+// ------------------------------------------------------------------------------------------
+struct ColArgs {
+  const float* Wf;
+  int64_t n;
+  int64_t k_rows;
+  const int* rowlist;
+  int64_t j0;
+  int bw;
+  const float* U;
+  int bits;
+  int clip;
+  float* E;
+  uint8_t* codes8;
+  int64_t ldc8;
+  float* scales;
+  uint8_t* zeros;
+  int64_t ngroups;
+  const float* row_s;
+  const float* row_z;
+  double* row_e2;
+  double* row_bnd;
+  int* overflow;
+};
+
+// Lane ownership: lane t of a row owns columns k = 4*P*(i/4) + 4*t + (i%4), i in [0, 32):
+// 4-wide chunks interleaved across the P lanes (balanced work, 16-byte shared-memory loads).
+template <int G>
+__global__ void __launch_bounds__(128) colloop_kernel(ColArgs a) {
+  extern __shared__ __align__(16) float q_smem[];
+  float* Us = q_smem;                       // [128][128]
+  float* invd = q_smem + kBlock * kBlock;   // [128]  1/U_jj
+  float* invd2 = invd + kBlock;             // [128]  1/U_jj^2
+  const int tid = threadIdx.x;
+  const int bw = a.bw;
+  const int64_t n = a.n, j0 = a.j0;
+  for (int e = tid * 4; e < kBlock * kBlock; e += 128 * 4) {
+    int jj = e / kBlock, kk = e % kBlock;
+    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (jj < bw) {
+      const float* src = a.U + (j0 + jj) * n + j0 + kk;
+      float* dv = &v.x;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) dv[u] = (kk + u >= jj && kk + u < bw) ? src[u] : 0.f;
+    }
+    *reinterpret_cast<float4*>(&Us[e]) = v;
+  }
+  if (tid < kBlock) {
+    float d = (tid < bw) ? a.U[(j0 + tid) * n + j0 + tid] : 1.f;
+    invd[tid] = 1.f / d;
+    invd2[tid] = (float)(1.0 / ((double)d * (double)d));
+  }
+  __syncthreads();
+
+  const int lane = tid & 31, warp = tid >> 5;
+  const int t = lane % kP;
+  const int64_t rr = (int64_t)blockIdx.x * kRowsPerCta + warp * (32 / kP) + lane / kP;
+  const bool active = rr < a.k_rows;
+  const int64_t row = active ? (a.rowlist ? a.rowlist[rr] : rr) : 0;
+  const float maxq = (float)((1 << a.bits) - 1);
+
+  float v[kVPL];
+#pragma unroll
+  for (int ci = 0; ci < kVPL / 4; ++ci) {
+    int k = 4 * kP * ci + 4 * t;
+    float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (active) {
+      const float* src = a.Wf + rr * n + j0 + k;
+      if (k + 3 < bw && ((j0 + k + rr * n) & 3) == 0) {
+        x = *reinterpret_cast<const float4*>(src);
+      } else {
+        float* dx = &x.x;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) dx[u] = (k + u < bw) ? src[u] : 0.f;
+      }
+    }
+    v[4 * ci + 0] = x.x; v[4 * ci + 1] = x.y; v[4 * ci + 2] = x.z; v[4 * ci + 3] = x.w;
+  }
+  float s = 1.f, inv_s = 1.f, z = 0.f;
+  if (G == 0 && active) { s = a.row_s[row]; z = a.row_z[row]; inv_s = 1.f / s; }
+  float eo[kVPL];
+  uint32_t cw[kVPL / 4];
+#pragma unroll
+  for (int i = 0; i < kVPL; ++i) eo[i] = 0.f;
+#pragma unroll
+  for (int i = 0; i < kVPL / 4; ++i) cw[i] = 0u;
+  double e2 = 0.0, bnd = 0.0;
+  int ovf = 0;
+  const unsigned full = 0xffffffffu;
+  const int gbase = lane & ~(kP - 1);
+
+#pragma unroll
+  for (int jj = 0; jj < kBlock; ++jj) {
+    if (jj < bw) {
+    if constexpr (G > 0) {
+      if (jj % G == 0) {
+        float lo = 0.f, hi = 0.f;
+#pragma unroll
+        for (int i = 0; i < kVPL; ++i) {
+          // owned column of slot i
+          const int k = 4 * kP * (i / 4) + 4 * t + (i % 4);
+          if (k >= jj && k < jj + G && k < bw) { lo = fminf(lo, v[i]); hi = fmaxf(hi, v[i]); }
+        }
+#pragma unroll
+        for (int o = kP / 2; o > 0; o >>= 1) {
+          lo = fminf(lo, __shfl_xor_sync(full, lo, o));
+          hi = fmaxf(hi, __shfl_xor_sync(full, hi, o));
+        }
+        if (lo == 0.f && hi == 0.f) { lo = -1.f; hi = 1.f; }
+        s = (hi - lo) / maxq;
+        z = rintf(-lo / s);
+        inv_s = 1.f / s;
+        if (active && t == 0) {
+          int64_t g = (j0 + jj) / G;
+          a.scales[row * a.ngroups + g] = s;
+          a.zeros[row * a.ngroups + g] = (uint8_t)z;
+        }
+      }
+    }
+    const int owner = (jj / 4) % kP;
+    const int idx = (jj / (4 * kP)) * 4 + (jj % 4);
+    const float x = __shfl_sync(full, v[idx], gbase + owner);
+    float c = rintf(x * inv_s) + z;
+    if (a.clip) {
+      c = fminf(fmaxf(c, 0.f), maxq);
+    } else if (c < 0.f || c > maxq) {
+      ovf = 1;
+    }
+    const float q = s * (c - z);
+    const float e = (x - q) * invd[jj];
+    if (t == owner) {
+      eo[idx] = e;
+      uint32_t cb = (uint32_t)(int)fminf(fmaxf(c, 0.f), maxq);
+      cw[idx / 4] |= cb << (8 * (idx % 4));
+    }
+    e2 += (double)e * (double)e;
+    bnd += (double)(s * s) * (double)invd2[jj];
+    // feedback to this lane's later columns of the block
+    const float* urow = Us + jj * kBlock;
+#pragma unroll
+    for (int ci = jj / (4 * kP); ci < kVPL / 4; ++ci) {
+      const float4 u4 = *reinterpret_cast<const float4*>(urow + 4 * kP * ci + 4 * t);
+      if (ci > jj / (4 * kP)) {
+        v[4 * ci + 0] = fmaf(-e, u4.x, v[4 * ci + 0]);
+        v[4 * ci + 1] = fmaf(-e, u4.y, v[4 * ci + 1]);
+        v[4 * ci + 2] = fmaf(-e, u4.z, v[4 * ci + 2]);
+        v[4 * ci + 3] = fmaf(-e, u4.w, v[4 * ci + 3]);
+      } else {
+        // the chunk that holds column jj: U's upper structure zeroes k <= jj, so the update
+        // is harmless for those slots (U[jj][k] = 0 for k < jj; k == jj is never read again)
+        if (t >= owner) {
+          if (t > owner || 0 > (jj % 4)) v[4 * ci + 0] = fmaf(-e, u4.x, v[4 * ci + 0]);
+          if (t > owner || 1 > (jj % 4)) v[4 * ci + 1] = fmaf(-e, u4.y, v[4 * ci + 1]);
+          if (t > owner || 2 > (jj % 4)) v[4 * ci + 2] = fmaf(-e, u4.z, v[4 * ci + 2]);
+          if (t > owner || 3 > (jj % 4)) v[4 * ci + 3] = fmaf(-e, u4.w, v[4 * ci + 3]);
+        }
+      }
+    }
+    }
+  }
+  // per-row overflow flag (all lanes of the warp take part in the shuffle)
+  int ovf_row = ovf;
+#pragma unroll
+  for (int o = kP / 2; o > 0; o >>= 1) ovf_row |= __shfl_xor_sync(0xffffffffu, ovf_row, o);
+  if (!active) return;
+  // write back this lane's errors and codes
+  float* Erow = a.E + rr * kBlock;
+  uint8_t* crow = a.codes8 + row * a.ldc8 + j0;
+#pragma unroll
+  for (int ci = 0; ci < kVPL / 4; ++ci) {
+    int k = 4 * kP * ci + 4 * t;
+    *reinterpret_cast<float4*>(Erow + k) =
+        make_float4(eo[4 * ci + 0], eo[4 * ci + 1], eo[4 * ci + 2], eo[4 * ci + 3]);
+    if (k + 3 < bw) {
+      *reinterpret_cast<uint32_t*>(crow + k) = cw[ci];
+    } else {
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        if (k + u < bw) crow[k + u] = (uint8_t)(cw[ci] >> (8 * u));
+    }
+  }
+  // per-row totals (all lanes of a row hold the same e2 / bnd)
+  if (t == 0) {
+    if (j0 == 0) { a.row_e2[row] = e2; a.row_bnd[row] = bnd; a.overflow[row] = ovf_row; }
+    else { a.row_e2[row] += e2; a.row_bnd[row] += bnd; a.overflow[row] |= ovf_row; }
+  }
+}
+
+// ------------------------------------------------------------------------------------------
+// lazy rank-<=128 update: Wf[:, j1:] -= E[:, :bw] U[j0:j0+bw, j1:]   (fp32 SIMT, v1)
+// ------------------------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) lazy_update_kernel(float* Wf, int64_t n, int64_t k_rows,
+                                                          int64_t j0, int bw, int64_t j1,
+                                                          const float* E, const float* U) {
+  __shared__ float As[16][64 + 4];
+  __shared__ float Bs[16][64 + 4];
+  const int64_t r0 = (int64_t)blockIdx.y * 64, c0 = j1 + (int64_t)blockIdx.x * 64;
+  const int tid = threadIdx.x, tx = tid % 16, ty = tid / 16;
+  float acc[4][4] = {};
+  for (int k0 = 0; k0 < bw; k0 += 16) {
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      int e = tid + 256 * r;
+      int ii = e / 16, kk = e % 16;
+      int64_t gr = r0 + ii;
+      As[kk][ii] = (gr < k_rows && k0 + kk < bw) ? E[gr * kBlock + k0 + kk] : 0.f;
+      int kb = e / 64, jj = e % 64;
+      int64_t gc = c0 + jj;
+      Bs[kb][jj] = (gc < n && k0 + kb < bw) ? U[(j0 + k0 + kb) * n + gc] : 0.f;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int kk = 0; kk < 16; ++kk) {
+      float av[4], bv[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) { av[q] = As[kk][ty + 16 * q]; bv[q] = Bs[kk][tx + 16 * q]; }
+#pragma unroll
+      for (int p = 0; p < 4; ++p)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) acc[p][q] = fmaf(av[p], bv[q], acc[p][q]);
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int p = 0; p < 4; ++p) {
+    int64_t gr = r0 + ty + 16 * p;
+    if (gr >= k_rows) continue;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      int64_t gc = c0 + tx + 16 * q;
+      if (gc < n) Wf[gr * n + gc] -= acc[p][q];
+    }
+  }
+}
+
+// ------------------------------------------------------------------------------------------
+// packing + ||w0 - q||^2 per row (one CTA per original row)
+// ------------------------------------------------------------------------------------------
+template <class TW>
+__global__ void __launch_bounds__(128) pack_kernel(const TW* W, const uint8_t* dead, int64_t n,
+                                                   const uint8_t* codes8, int64_t ldc8,
+                                                   int reverse, int bits, int group,
+                                                   int64_t ngroups, const float* scales,
+                                                   const uint8_t* zeros, uint32_t* codes,
+                                                   double* row_d2) {
+  const int64_t r = blockIdx.x;
+  const uint8_t* crow = codes8 + r * ldc8;
+  const int64_t nwords = (n * bits + 31) / 32;
+  for (int64_t w = threadIdx.x; w < nwords; w += blockDim.x) {
+    uint32_t word = 0u;
+    int64_t cf = (32 * w) / bits, cl = (32 * w + 31) / bits;
+    if (cl > n - 1) cl = n - 1;
+    for (int64_t c = cf; c <= cl; ++c) {
+      uint32_t code = crow[reverse ? n - 1 - c : c];
+      int64_t pos = (int64_t)bits * c - 32 * w;
+      if (pos >= 0) word |= code << pos;
+      else word |= code >> (-pos);
+    }
+    codes[r * nwords + w] = word;
+  }
+  double acc = 0.0;
+  for (int64_t c = threadIdx.x; c < n; c += blockDim.x) {
+    float w0;
+    if constexpr (sizeof(TW) == 2) w0 = __bfloat162float(W[r * n + c]);
+    else w0 = (float)W[r * n + c];
+    if (dead && dead[c]) w0 = 0.f;
+    int64_t g = group ? c / group : 0;
+    float s = scales[r * ngroups + g], z = (float)zeros[r * ngroups + g];
+    float code = (float)crow[reverse ? n - 1 - c : c];
+    double d = (double)w0 - (double)s * (double)(code - z);
+    acc += d * d;
+  }
+  __shared__ double red[4];
+  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = acc;
+  __syncthreads();
+  if (threadIdx.x == 0) row_d2[r] = red[0] + red[1] + red[2] + red[3];
+}
+
+__global__ void __launch_bounds__(1024) q_reduce_kernel(int64_t m, const double* row_e2,
+                                                        const double* row_bnd,
+                                                        const double* row_d2,
+                                                        const double* delta, double* loss) {
+  __shared__ double red[3][32];
+  double a0 = 0, a1 = 0, a2 = 0;
+  for (int64_t i = threadIdx.x; i < m; i += blockDim.x) {
+    a0 += row_e2[i]; a1 += row_bnd[i]; a2 += row_d2[i];
+  }
+  for (int o = 16; o > 0; o >>= 1) {
+    a0 += __shfl_xor_sync(0xffffffffu, a0, o);
+    a1 += __shfl_xor_sync(0xffffffffu, a1, o);
+    a2 += __shfl_xor_sync(0xffffffffu, a2, o);
+  }
+  if ((threadIdx.x & 31) == 0) {
+    red[0][threadIdx.x >> 5] = a0; red[1][threadIdx.x >> 5] = a1; red[2][threadIdx.x >> 5] = a2;
+  }
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    int nw = blockDim.x >> 5;
+    a0 = threadIdx.x < nw ? red[0][threadIdx.x] : 0;
+    a1 = threadIdx.x < nw ? red[1][threadIdx.x] : 0;
+    a2 = threadIdx.x < nw ? red[2][threadIdx.x] : 0;
+    for (int o = 16; o > 0; o >>= 1) {
+      a0 += __shfl_xor_sync(0xffffffffu, a0, o);
+      a1 += __shfl_xor_sync(0xffffffffu, a1, o);
+      a2 += __shfl_xor_sync(0xffffffffu, a2, o);
+    }
+    if (threadIdx.x == 0) {
+      loss[1] = a0;
+      loss[2] = a1 * 0.25;
+      loss[0] = delta ? 0.5 * (a0 - (*delta) * a2) : 0.0;
+    }
+  }
+}
+
+// clip-free ladder: rows that overflowed -> rowlist, alpha *= ladder
+__global__ void q_ladder_kernel(int64_t m, int* overflow, float* alpha, float ladder, int* rowlist,
+                                int* counter) {
+  int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+  if (i >= m) return;
+  if (overflow[i]) {
+    int k = atomicAdd(counter, 1);
+    rowlist[k] = (int)i;
+    alpha[i] *= ladder;
+  }
+}
+
+// ------------------------------------------------------------------------------------------
+// orchestration
+// ------------------------------------------------------------------------------------------
+#define Q_TRY(x)                                    \
+  do {                                              \
+    cudaError_t _e = (x);                           \
+    if (_e != cudaSuccess) return GQ_ERR_CUDA;      \
+  } while (0)
+
+constexpr size_t kColSmem = (size_t)(kBlock * kBlock + 2 * kBlock) * sizeof(float);
+
+cudaError_t quant_init_attributes() {
+  const int smem = (int)kColSmem;
+  cudaError_t e;
+  if ((e = cudaFuncSetAttribute(colloop_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem))) return e;
+  if ((e = cudaFuncSetAttribute(colloop_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem))) return e;
+  if ((e = cudaFuncSetAttribute(colloop_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem))) return e;
+  if ((e = cudaFuncSetAttribute(colloop_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem))) return e;
+  return cudaFuncSetAttribute(colloop_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+}
+
+template <int G>
+static cudaError_t launch_colloop(const ColArgs& ca, cudaStream_t s) {
+  const size_t smem = kColSmem;
+  unsigned grid = (unsigned)((ca.k_rows + kRowsPerCta - 1) / kRowsPerCta);
+  colloop_kernel<G><<<grid, 128, smem, s>>>(ca);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+static cudaError_t colloop_dispatch(int group, const ColArgs& ca, cudaStream_t s) {
+  switch (group) {
+    case 0: return launch_colloop<0>(ca, s);
+    case 16: return launch_colloop<16>(ca, s);
+    case 32: return launch_colloop<32>(ca, s);
+    case 64: return launch_colloop<64>(ca, s);
+    case 128: return launch_colloop<128>(ca, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+gq_status run_quantize(const QuantArgs& a, cudaStream_t s) {
+  const int64_t m = a.m, n = a.n;
+  QLayout L = q_layout(a.ws, m, n);
+  const gq_quant_cfg& cfg = a.cfg;
+  const int G = cfg.group_size;
+  const int64_t ngroups = G ? (n + G - 1) / G : 1;
+  Q_TRY(cudaMemsetAsync(L.hdr, 0, sizeof(WsHeader), s));
+  q_reset_kernel<<<(unsigned)((m + 255) / 256), 256, 0, s>>>(m, L.alpha, L.overflow, a.loss);
+  count_launches(1);
+  Q_TRY(cudaGetLastError());
+  int64_t k_rows = m;
+  const int* rowlist = nullptr;
+  const int nblocks = (int)((n + kBlock - 1) / kBlock);
+  const int max_rounds = cfg.clip ? 1 : cfg.ladder_max + 1;
+  int rounds_run = 0;
+  for (int round = 0; round < max_rounds; ++round) {
+    rounds_run = round;
+    {
+      int64_t total = k_rows * n;
+      unsigned grid = (unsigned)std::min<int64_t>((total + 255) / 256, 148 * 64);
+      if (a.wt == GQ_BF16)
+        q_load_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(
+            static_cast<const __nv_bfloat16*>(a.W), n, k_rows, rowlist, a.dead, cfg.reverse, L.Wf);
+      else
+        q_load_kernel<float><<<grid, 256, 0, s>>>(static_cast<const float*>(a.W), n, k_rows,
+                                                  rowlist, a.dead, cfg.reverse, L.Wf);
+      count_launches(1);
+      Q_TRY(cudaGetLastError());
+    }
+    if (G == 0) {
+      unsigned grid = (unsigned)((k_rows + 7) / 8);
+      q_row_grid_kernel<<<grid, 256, 0, s>>>(L.Wf, n, k_rows, rowlist, cfg.bits, cfg.clip,
+                                             L.alpha, L.row_s, L.row_z, a.scales, a.zeros);
+      count_launches(1);
+      Q_TRY(cudaGetLastError());
+    }
+    for (int b = 0; b < nblocks; ++b) {
+      const int64_t j0 = (int64_t)b * kBlock;
+      const int bw = (int)std::min<int64_t>(kBlock, n - j0);
+      ColArgs ca{};
+      ca.Wf = L.Wf; ca.n = n; ca.k_rows = k_rows; ca.rowlist = rowlist; ca.j0 = j0; ca.bw = bw;
+      ca.U = a.U; ca.bits = cfg.bits; ca.clip = cfg.clip; ca.E = L.E; ca.codes8 = L.codes8;
+      ca.ldc8 = L.ldc8; ca.scales = a.scales; ca.zeros = a.zeros; ca.ngroups = ngroups;
+      ca.row_s = L.row_s; ca.row_z = L.row_z; ca.row_e2 = L.row_e2; ca.row_bnd = L.row_bnd;
+      ca.overflow = L.overflow;
+      Q_TRY(colloop_dispatch(G, ca, s));
+      const int64_t j1 = j0 + bw;
+      if (j1 < n) {
+        dim3 grid((unsigned)((n - j1 + 63) / 64), (unsigned)((k_rows + 63) / 64));
+        lazy_update_kernel<<<grid, 256, 0, s>>>(L.Wf, n, k_rows, j0, bw, j1, L.E, a.U);
+        count_launches(1);
+        Q_TRY(cudaGetLastError());
+      }
+    }
+    if (cfg.clip) break;
+    // clip-free: collect rows whose codes left [0, 2^b - 1] and rerun them on a wider step
+    Q_TRY(cudaMemsetAsync(L.counter, 0, sizeof(int), s));
+    q_ladder_kernel<<<(unsigned)((m + 255) / 256), 256, 0, s>>>(m, L.overflow, L.alpha,
+                                                                 cfg.ladder, L.rowlist, L.counter);
+    count_launches(1);
+    Q_TRY(cudaGetLastError());
+    int cnt = 0;
+    Q_TRY(cudaMemcpyAsync(&cnt, L.counter, sizeof(int), cudaMemcpyDeviceToHost, s));
+    Q_TRY(cudaStreamSynchronize(s));
+    if (cnt == 0) break;
+    if (round == max_rounds - 1) {
+      int code = GQ_ERR_NO_FIT;
+      // first error wins: write only if the status word is still clear
+      int cur = 0;
+      Q_TRY(cudaMemcpyAsync(&cur, &L.hdr->status, sizeof(int), cudaMemcpyDeviceToHost, s));
+      Q_TRY(cudaStreamSynchronize(s));
+      if (cur == 0) Q_TRY(cudaMemcpyAsync(&L.hdr->status, &code, sizeof(int),
+                                          cudaMemcpyHostToDevice, s));
+      Q_TRY(cudaStreamSynchronize(s));
+      break;
+    }
+    k_rows = cnt;
+    rowlist = L.rowlist;
+  }
+  if (!cfg.clip) {
+    int rr = rounds_run;
+    Q_TRY(cudaMemcpyAsync(&L.hdr->ladder_rounds, &rr, sizeof(int), cudaMemcpyHostToDevice, s));
+    Q_TRY(cudaStreamSynchronize(s));
+  }
+  if (a.wt == GQ_BF16)
+    pack_kernel<__nv_bfloat16><<<(unsigned)m, 128, 0, s>>>(
+        static_cast<const __nv_bfloat16*>(a.W), a.dead, n, L.codes8, L.ldc8, cfg.reverse,
+        cfg.bits, G, ngroups, a.scales, a.zeros, a.codes, L.row_d2);
+  else
+    pack_kernel<float><<<(unsigned)m, 128, 0, s>>>(static_cast<const float*>(a.W), a.dead, n,
+                                                   L.codes8, L.ldc8, cfg.reverse, cfg.bits, G,
+                                                   ngroups, a.scales, a.zeros, a.codes, L.row_d2);
+  count_launches(1);
+  Q_TRY(cudaGetLastError());
+  q_reduce_kernel<<<1, 1024, 0, s>>>(m, L.row_e2, L.row_bnd, L.row_d2, a.delta, a.loss);
+  count_launches(1);
+  Q_TRY(cudaGetLastError());
+  return GQ_OK;
+}
+
+}  // namespace gq

@@ -1,0 +1,189 @@
+"""Thin ctypes binding of libgq (include/gq.h): argument marshalling only.
+
+Every function here has the name of the C entry point it calls and does nothing but convert
+torch tensors to pointers, check dtypes/shapes/devices, and raise on a non-OK status.  All
+computation happens in the CUDA library; torch provides device memory and the stream.  The
+library must be built (``python -m post_weight_quantization_22_b200.build``); importing this
+module without it raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libgq.so")
+
+GQ_BF16, GQ_FP32 = 0, 1
+STATUS = {0: "ok", 1: "invalid argument", 2: "not positive definite", 3: "CUDA error",
+          4: "unsupported", 5: "timeout", 6: "no fit", 7: "workspace"}
+
+
+class GQError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        super().__init__(f"{what}: gq status {code} ({STATUS.get(code, '?')})")
+        self.code = code
+
+
+class _Cfg(ctypes.Structure):
+    _fields_ = [("bits", ctypes.c_int), ("group_size", ctypes.c_int), ("reverse", ctypes.c_int),
+                ("clip", ctypes.c_int), ("ladder", ctypes.c_float), ("ladder_max", ctypes.c_int)]
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"libgq.so is not built ({LIB_PATH}); run "
+                          "`python -m post_weight_quantization_22_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    P, I64, SZ, I, F = ctypes.c_void_p, ctypes.c_int64, ctypes.c_size_t, ctypes.c_int, ctypes.c_float
+    lib.gq_version.restype = ctypes.c_char_p
+    lib.gq_status_string.restype = ctypes.c_char_p
+    lib.gq_status_string.argtypes = [I]
+    lib.gq_hessian_accumulate.restype = I
+    lib.gq_hessian_accumulate.argtypes = [P, P, I, I64, I64, P]
+    lib.gq_prepare_workspace_size.restype = SZ
+    lib.gq_prepare_workspace_size.argtypes = [I64]
+    lib.gq_prepare_hinv.restype = I
+    lib.gq_prepare_hinv.argtypes = [P, I64, F, I, P, P, P, P, SZ, P]
+    lib.gq_quantize_workspace_size.restype = SZ
+    lib.gq_quantize_workspace_size.argtypes = [I64, I64, ctypes.POINTER(_Cfg)]
+    lib.gq_quantize_layer.restype = I
+    lib.gq_quantize_layer.argtypes = [P, I, I64, I64, P, P, P, ctypes.POINTER(_Cfg), P, P, P, P,
+                                      P, SZ, P]
+    lib.gq_workspace_status.restype = I
+    lib.gq_workspace_status.argtypes = [P, ctypes.POINTER(ctypes.c_int), P]
+    return lib
+
+
+LIB = _load()
+EXPORTED = ("gq_version", "gq_status_string", "gq_hessian_accumulate", "gq_prepare_workspace_size",
+            "gq_prepare_hinv", "gq_quantize_workspace_size", "gq_quantize_layer",
+            "gq_workspace_status")
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return GQ_BF16
+    if t.dtype == torch.float32:
+        return GQ_FP32
+    raise TypeError(f"unsupported dtype {t.dtype} (bf16 or fp32)")
+
+
+def _check(code: int, what: str):
+    if code != 0:
+        raise GQError(code, what)
+
+
+def _need(t: torch.Tensor, dtype, shape, name):
+    if not t.is_cuda or t.dtype != dtype or tuple(t.shape) != tuple(shape) or not t.is_contiguous():
+        raise ValueError(f"{name}: expected contiguous cuda {dtype} {tuple(shape)}, got "
+                         f"{t.device} {t.dtype} {tuple(t.shape)}")
+
+
+def workspace(nbytes: int, device) -> torch.Tensor:
+    """A 256-byte aligned device byte buffer of at least nbytes (torch allocations are)."""
+    return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+
+
+def gq_version() -> str:
+    return LIB.gq_version().decode()
+
+
+def gq_hessian_accumulate(H: torch.Tensor, X: torch.Tensor, stream=None) -> torch.Tensor:
+    """H += 2 X^T X on the GPU (H fp64 n x n, X bf16/fp32 T x n, both on the same device)."""
+    T, n = X.shape
+    _need(H, torch.float64, (n, n), "H")
+    if not X.is_cuda or not X.is_contiguous():
+        raise ValueError("X must be a contiguous cuda tensor")
+    _check(LIB.gq_hessian_accumulate(_ptr(H), _ptr(X), _dtype_code(X), T, n, _stream(stream)),
+           "gq_hessian_accumulate")
+    return H
+
+
+def gq_prepare_workspace_size(n: int) -> int:
+    return int(LIB.gq_prepare_workspace_size(n))
+
+
+def gq_prepare_hinv(H: torch.Tensor, damp: float = 0.01, reverse: bool = False, U=None,
+                    dead=None, delta=None, ws=None, stream=None):
+    """U (fp32 n x n upper), dead mask (uint8 n), delta (fp64 [1]) from fp64 H."""
+    n = H.shape[0]
+    _need(H, torch.float64, (n, n), "H")
+    dev = H.device
+    U = torch.empty((n, n), dtype=torch.float32, device=dev) if U is None else U
+    dead = torch.empty(n, dtype=torch.uint8, device=dev) if dead is None else dead
+    delta = torch.empty(1, dtype=torch.float64, device=dev) if delta is None else delta
+    need = gq_prepare_workspace_size(n)
+    ws = workspace(need, dev) if ws is None else ws
+    _need(U, torch.float32, (n, n), "U")
+    _check(LIB.gq_prepare_hinv(_ptr(H), n, float(damp), int(bool(reverse)), _ptr(U), _ptr(dead),
+                               _ptr(delta), _ptr(ws), ws.numel(), _stream(stream)),
+           "gq_prepare_hinv")
+    return U, dead, delta, ws
+
+
+@dataclass
+class QuantCfg:
+    bits: int = 4
+    group_size: int = 0
+    reverse: bool = False
+    clip: bool = True
+    ladder: float = 1.25
+    ladder_max: int = 8
+
+    def c(self) -> _Cfg:
+        return _Cfg(int(self.bits), int(self.group_size), int(bool(self.reverse)),
+                    int(bool(self.clip)), float(self.ladder), int(self.ladder_max))
+
+
+def gq_quantize_workspace_size(m: int, n: int, cfg: QuantCfg) -> int:
+    c = cfg.c()
+    return int(LIB.gq_quantize_workspace_size(m, n, ctypes.byref(c)))
+
+
+def n_words(n: int, bits: int) -> int:
+    return (n * bits + 31) // 32
+
+
+def gq_quantize_layer(W: torch.Tensor, U: torch.Tensor, dead, delta, cfg: QuantCfg,
+                      codes=None, scales=None, zeros=None, loss=None, ws=None, stream=None):
+    """Run the column loop; returns (codes uint32 [m, words] as int32 view, scales, zeros, loss, ws)."""
+    m, n = W.shape
+    if not W.is_cuda or not W.is_contiguous():
+        raise ValueError("W must be a contiguous cuda tensor")
+    dev = W.device
+    _need(U, torch.float32, (n, n), "U")
+    G = 1 if cfg.group_size == 0 else -(-n // cfg.group_size)
+    codes = torch.empty((m, n_words(n, cfg.bits)), dtype=torch.int32, device=dev) if codes is None else codes
+    scales = torch.empty((m, G), dtype=torch.float32, device=dev) if scales is None else scales
+    zeros = torch.empty((m, G), dtype=torch.uint8, device=dev) if zeros is None else zeros
+    loss = torch.empty(3, dtype=torch.float64, device=dev) if loss is None else loss
+    need = gq_quantize_workspace_size(m, n, cfg)
+    if need == 0:
+        raise GQError(1, "gq_quantize_workspace_size")
+    ws = workspace(need, dev) if ws is None else ws
+    c = cfg.c()
+    _check(LIB.gq_quantize_layer(_ptr(W), _dtype_code(W), m, n, _ptr(U), _ptr(dead), _ptr(delta),
+                                 ctypes.byref(c), _ptr(codes), _ptr(scales), _ptr(zeros),
+                                 _ptr(loss), _ptr(ws), ws.numel(), _stream(stream)),
+           "gq_quantize_layer")
+    return codes, scales, zeros, loss, ws
+
+
+def gq_workspace_status(ws: torch.Tensor, stream=None):
+    """(status code, ladder rounds) recorded in a workspace by its last call; synchronizes."""
+    r = ctypes.c_int(0)
+    code = LIB.gq_workspace_status(_ptr(ws), ctypes.byref(r), _stream(stream))
+    return int(code), int(r.value)

@@ -1,0 +1,54 @@
+"""The C-ABI library loads on a machine without a GPU and exports every declared entry point.
+
+No compute call is made here (no GPU); only the size queries and string functions, which touch
+no device, are exercised.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    text = open(os.path.join(ROOT, "include", "gq.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(gq_[a-z_]+)\s*\(", text)))
+
+
+def test_library_exports_every_declared_symbol():
+    from post_weight_quantization_22_b200 import gq as G
+    names = _declared()
+    assert "gq_hessian_accumulate" in names and "gq_quantize_layer" in names
+    missing = [n for n in names if not hasattr(G.LIB, n)]
+    assert not missing, missing
+    assert set(G.EXPORTED) <= set(names)
+
+
+def test_size_queries_and_strings_without_gpu():
+    from post_weight_quantization_22_b200 import gq as G
+    assert G.gq_version().startswith("gq ")
+    assert G.LIB.gq_status_string(2) == b"damped Hessian is not positive definite"
+    n = 4096
+    ps = G.gq_prepare_workspace_size(n)
+    assert ps >= 8 * n * n
+    cfg = G.QuantCfg(bits=4, group_size=128)
+    qs = G.gq_quantize_workspace_size(4096, 4096, cfg)
+    assert qs >= 4 * 4096 * 4096
+    assert G.gq_prepare_workspace_size(0) == 0
+    assert G.gq_quantize_workspace_size(4096, 4096, G.QuantCfg(bits=9)) == 0
+    assert G.gq_quantize_workspace_size(16, 16, G.QuantCfg(bits=3, group_size=64, reverse=True)) == 0
+    assert G.LIB.gq_kernel_launches() == 0
+
+
+def test_package_has_no_cpu_fallback():
+    """The product path never imports the oracle."""
+    pkg = os.path.join(ROOT, "post_weight_quantization_22_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith(".py"):
+                src = open(os.path.join(dirpath, f)).read()
+                assert not re.search(r"^\s*(from|import)\s+oracle", src, flags=re.M), f
+                assert "gptq_oracle" not in src, f
