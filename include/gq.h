@@ -110,7 +110,7 @@ size_t gq_prepare_workspace_size(int64_t n);
  *   d_ws       workspace of at least gq_prepare_workspace_size(n) bytes.
  * Device-detected error: GQ_ERR_NOT_PD (non-positive pivot; U is then undefined).
  */
-gq_status gq_prepare_hinv(const double* d_H, int64_t n, float damp, int reverse, float* d_U,
+gq_status gq_prepare_hinv(const double* d_H, int64_t n, double damp, int reverse, float* d_U,
                           uint8_t* d_dead, double* d_delta, void* d_ws, size_t ws_bytes,
                           gq_stream_t stream);
 

@@ -71,10 +71,10 @@ size_t gq_prepare_workspace_size(int64_t n) {
   return prepare_ws_bytes(n);
 }
 
-gq_status gq_prepare_hinv(const double* d_H, int64_t n, float damp, int reverse, float* d_U,
+gq_status gq_prepare_hinv(const double* d_H, int64_t n, double damp, int reverse, float* d_U,
                           uint8_t* d_dead, double* d_delta, void* d_ws, size_t ws_bytes,
                           gq_stream_t stream) {
-  if (n < 1 || n > kMaxN || !(damp >= 0.f) || (reverse != 0 && reverse != 1))
+  if (n < 1 || n > kMaxN || !(damp >= 0.0) || (reverse != 0 && reverse != 1))
     return GQ_ERR_INVALID_ARG;
   if (!d_H || !d_U || !d_dead || !d_delta || !d_ws) return GQ_ERR_INVALID_ARG;
   if (!aligned256(d_ws) || ws_bytes < prepare_ws_bytes(n)) return GQ_ERR_WORKSPACE;

@@ -27,7 +27,7 @@ constexpr int kNB = 64;  // Cholesky panel width
 // ---------------------------------------------------------------------------------------
 // dead fix + damping statistics (one CTA)
 // ---------------------------------------------------------------------------------------
-__global__ void __launch_bounds__(1024) diag_stats_kernel(const double* H, int64_t n, float damp,
+__global__ void __launch_bounds__(1024) diag_stats_kernel(const double* H, int64_t n, double damp,
                                                           uint8_t* dead, double* delta_out,
                                                           WsHeader* hdr) {
   __shared__ double red[32];
@@ -45,7 +45,7 @@ __global__ void __launch_bounds__(1024) diag_stats_kernel(const double* H, int64
     acc = (threadIdx.x < (blockDim.x >> 5)) ? red[threadIdx.x] : 0.0;
     for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
     if (threadIdx.x == 0) {
-      double delta = (double)damp * (acc / (double)n);
+      double delta = damp * (acc / (double)n);
       *delta_out = delta;
       hdr->scratch[0] = delta;
     }
@@ -211,7 +211,7 @@ cudaError_t factor_init_attributes() {
     if (_e != cudaSuccess) return _e;           \
   } while (0)
 
-cudaError_t launch_prepare(const double* H, int64_t n, float damp, int reverse, float* U,
+cudaError_t launch_prepare(const double* H, int64_t n, double damp, int reverse, float* U,
                            uint8_t* dead, double* delta, void* ws, cudaStream_t s) {
   PrepLayout L = prep_layout(ws, n);
   GQ_TRY(cudaMemsetAsync(L.hdr, 0, sizeof(WsHeader), s));

@@ -46,7 +46,7 @@ cudaError_t launch_hessian(double* H, const void* X, gq_dtype xt, int64_t T, int
 
 // ---- factor preparation ----
 size_t prepare_ws_bytes(int64_t n);
-cudaError_t launch_prepare(const double* H, int64_t n, float damp, int reverse, float* U,
+cudaError_t launch_prepare(const double* H, int64_t n, double damp, int reverse, float* U,
                            uint8_t* dead, double* delta, void* ws, cudaStream_t s);
 
 // ---- quantization ----

@@ -28,8 +28,8 @@ struct QLayout {
   float* E;         // k x 128 scaled errors of the current block
   uint8_t* codes8;  // m x ldc8 codes in processing order
   int64_t ldc8;
-  float* row_s;     // per-row step (group_size 0)
-  float* row_z;     // per-row zero point (group_size 0)
+  double* row_s;    // per-row step (group_size 0)
+  double* row_z;    // per-row zero point (group_size 0)
   float* alpha;     // per-row ladder factor
   double* row_e2;   // per-row sum of e^2
   double* row_bnd;  // per-row Theorem 5 bound
@@ -48,8 +48,8 @@ static QLayout q_layout(void* ws, int64_t m, int64_t n) {
   L.E = c.take<float>((size_t)m * kBlock);
   L.ldc8 = (n + 15) / 16 * 16;
   L.codes8 = c.take<uint8_t>((size_t)m * L.ldc8);
-  L.row_s = c.take<float>(m);
-  L.row_z = c.take<float>(m);
+  L.row_s = c.take<double>(m);
+  L.row_z = c.take<double>(m);
   L.alpha = c.take<float>(m);
   L.row_e2 = c.take<double>(m);
   L.row_bnd = c.take<double>(m);
@@ -94,8 +94,8 @@ __global__ void q_load_kernel(const TW* W, int64_t n, int64_t k_rows, const int*
 
 // per-row grid from the (dead-zeroed) row: one warp per row
 __global__ void q_row_grid_kernel(const float* Wf, int64_t n, int64_t k_rows, const int* rowlist,
-                                  int bits, int clip, const float* alpha, float* row_s,
-                                  float* row_z, float* scales, uint8_t* zeros) {
+                                  int bits, int clip, const float* alpha, double* row_s,
+                                  double* row_z, float* scales, uint8_t* zeros) {
   int64_t rr = blockIdx.x * (int64_t)(blockDim.x / 32) + threadIdx.x / 32;
   int lane = threadIdx.x & 31;
   if (rr >= k_rows) return;
@@ -108,19 +108,20 @@ __global__ void q_row_grid_kernel(const float* Wf, int64_t n, int64_t k_rows, co
   }
   if (lane == 0) {
     int64_t row = rowlist ? rowlist[rr] : rr;
-    if (lo == 0.f && hi == 0.f) { lo = -1.f; hi = 1.f; }
-    float maxq = (float)((1 << bits) - 1);
-    float s, z;
+    double dlo = lo, dhi = hi;
+    if (dlo == 0.0 && dhi == 0.0) { dlo = -1.0; dhi = 1.0; }
+    double maxq = (double)((1 << bits) - 1);
+    double s, z;
     if (clip) {
-      s = (hi - lo) / maxq;
-      z = rintf(-lo / s);
+      s = (dhi - dlo) / maxq;
+      z = rint(-dlo / s);
     } else {
-      s = alpha[row] * (hi - lo) / maxq;
-      z = rintf(maxq * 0.5f - (hi + lo) / (2.f * s));
+      s = (double)alpha[row] * (dhi - dlo) / maxq;
+      z = rint(maxq * 0.5 - (dhi + dlo) / (2.0 * s));
     }
     row_s[row] = s;
     row_z[row] = z;
-    scales[row] = s;
+    scales[row] = (float)s;
     zeros[row] = (uint8_t)z;
   }
 }
@@ -144,8 +145,8 @@ struct ColArgs {
   float* scales;
   uint8_t* zeros;
   int64_t ngroups;
-  const float* row_s;
-  const float* row_z;
+  const double* row_s;
+  const double* row_z;
   double* row_e2;
   double* row_bnd;
   int* overflow;
@@ -153,30 +154,34 @@ struct ColArgs {
 
 // Lane ownership: lane t of a row owns columns k = 4*P*(i/4) + 4*t + (i%4), i in [0, 32):
 // 4-wide chunks interleaved across the P lanes (balanced work, 16-byte shared-memory loads).
+//
+// The recursion runs in fp64: the in-block feedback sums cancel strongly when the per-row
+// grid is coarse, and an fp32 recursion flips ~1-3 % of the codes on ill-conditioned layers
+// (measured against the fp64 oracle), while fp64 here with fp32 storage of W, E and U between
+// blocks reproduces the oracle's codes.
 template <int G>
 __global__ void __launch_bounds__(128) colloop_kernel(ColArgs a) {
-  extern __shared__ __align__(16) float q_smem[];
-  float* Us = q_smem;                       // [128][128]
-  float* invd = q_smem + kBlock * kBlock;   // [128]  1/U_jj
-  float* invd2 = invd + kBlock;             // [128]  1/U_jj^2
+  extern __shared__ __align__(16) double q_smem[];
+  double* Us = q_smem;                       // [128][128]
+  double* invd = q_smem + kBlock * kBlock;   // [128]  1/U_jj
+  double* invd2 = invd + kBlock;             // [128]  1/U_jj^2
   const int tid = threadIdx.x;
   const int bw = a.bw;
   const int64_t n = a.n, j0 = a.j0;
-  for (int e = tid * 4; e < kBlock * kBlock; e += 128 * 4) {
+  for (int e = tid * 2; e < kBlock * kBlock; e += 128 * 2) {
     int jj = e / kBlock, kk = e % kBlock;
-    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+    double2 v = make_double2(0.0, 0.0);
     if (jj < bw) {
       const float* src = a.U + (j0 + jj) * n + j0 + kk;
-      float* dv = &v.x;
-#pragma unroll
-      for (int u = 0; u < 4; ++u) dv[u] = (kk + u >= jj && kk + u < bw) ? src[u] : 0.f;
+      if (kk >= jj && kk < bw) v.x = (double)src[0];
+      if (kk + 1 >= jj && kk + 1 < bw) v.y = (double)src[1];
     }
-    *reinterpret_cast<float4*>(&Us[e]) = v;
+    *reinterpret_cast<double2*>(&Us[e]) = v;
   }
   if (tid < kBlock) {
-    float d = (tid < bw) ? a.U[(j0 + tid) * n + j0 + tid] : 1.f;
-    invd[tid] = 1.f / d;
-    invd2[tid] = (float)(1.0 / ((double)d * (double)d));
+    double d = (tid < bw) ? (double)a.U[(j0 + tid) * n + j0 + tid] : 1.0;
+    invd[tid] = 1.0 / d;
+    invd2[tid] = 1.0 / (d * d);
   }
   __syncthreads();
 
@@ -185,9 +190,9 @@ __global__ void __launch_bounds__(128) colloop_kernel(ColArgs a) {
   const int64_t rr = (int64_t)blockIdx.x * kRowsPerCta + warp * (32 / kP) + lane / kP;
   const bool active = rr < a.k_rows;
   const int64_t row = active ? (a.rowlist ? a.rowlist[rr] : rr) : 0;
-  const float maxq = (float)((1 << a.bits) - 1);
+  const double maxq = (double)((1 << a.bits) - 1);
 
-  float v[kVPL];
+  double v[kVPL];
 #pragma unroll
   for (int ci = 0; ci < kVPL / 4; ++ci) {
     int k = 4 * kP * ci + 4 * t;
@@ -204,8 +209,8 @@ __global__ void __launch_bounds__(128) colloop_kernel(ColArgs a) {
     }
     v[4 * ci + 0] = x.x; v[4 * ci + 1] = x.y; v[4 * ci + 2] = x.z; v[4 * ci + 3] = x.w;
   }
-  float s = 1.f, inv_s = 1.f, z = 0.f;
-  if (G == 0 && active) { s = a.row_s[row]; z = a.row_z[row]; inv_s = 1.f / s; }
+  double s = 1.0, inv_s = 1.0, z = 0.0;
+  if (G == 0 && active) { s = a.row_s[row]; z = a.row_z[row]; inv_s = 1.0 / s; }
   float eo[kVPL];
   uint32_t cw[kVPL / 4];
 #pragma unroll
@@ -222,66 +227,64 @@ __global__ void __launch_bounds__(128) colloop_kernel(ColArgs a) {
     if (jj < bw) {
     if constexpr (G > 0) {
       if (jj % G == 0) {
-        float lo = 0.f, hi = 0.f;
+        double lo = 0.0, hi = 0.0;
 #pragma unroll
         for (int i = 0; i < kVPL; ++i) {
           // owned column of slot i
           const int k = 4 * kP * (i / 4) + 4 * t + (i % 4);
-          if (k >= jj && k < jj + G && k < bw) { lo = fminf(lo, v[i]); hi = fmaxf(hi, v[i]); }
+          if (k >= jj && k < jj + G && k < bw) { lo = fmin(lo, v[i]); hi = fmax(hi, v[i]); }
         }
 #pragma unroll
         for (int o = kP / 2; o > 0; o >>= 1) {
-          lo = fminf(lo, __shfl_xor_sync(full, lo, o));
-          hi = fmaxf(hi, __shfl_xor_sync(full, hi, o));
+          lo = fmin(lo, __shfl_xor_sync(full, lo, o));
+          hi = fmax(hi, __shfl_xor_sync(full, hi, o));
         }
-        if (lo == 0.f && hi == 0.f) { lo = -1.f; hi = 1.f; }
+        if (lo == 0.0 && hi == 0.0) { lo = -1.0; hi = 1.0; }
         s = (hi - lo) / maxq;
-        z = rintf(-lo / s);
-        inv_s = 1.f / s;
+        z = rint(-lo / s);
+        inv_s = 1.0 / s;
         if (active && t == 0) {
           int64_t g = (j0 + jj) / G;
-          a.scales[row * a.ngroups + g] = s;
+          a.scales[row * a.ngroups + g] = (float)s;
           a.zeros[row * a.ngroups + g] = (uint8_t)z;
         }
       }
     }
     const int owner = (jj / 4) % kP;
     const int idx = (jj / (4 * kP)) * 4 + (jj % 4);
-    const float x = __shfl_sync(full, v[idx], gbase + owner);
-    float c = rintf(x * inv_s) + z;
+    const double x = __shfl_sync(full, v[idx], gbase + owner);
+    double c = rint(x * inv_s) + z;
     if (a.clip) {
-      c = fminf(fmaxf(c, 0.f), maxq);
-    } else if (c < 0.f || c > maxq) {
+      c = fmin(fmax(c, 0.0), maxq);
+    } else if (c < 0.0 || c > maxq) {
       ovf = 1;
     }
-    const float q = s * (c - z);
-    const float e = (x - q) * invd[jj];
+    const double q = s * (c - z);
+    const double e = (x - q) * invd[jj];
     if (t == owner) {
-      eo[idx] = e;
-      uint32_t cb = (uint32_t)(int)fminf(fmaxf(c, 0.f), maxq);
+      eo[idx] = (float)e;
+      uint32_t cb = (uint32_t)(int)fmin(fmax(c, 0.0), maxq);
       cw[idx / 4] |= cb << (8 * (idx % 4));
     }
-    e2 += (double)e * (double)e;
-    bnd += (double)(s * s) * (double)invd2[jj];
+    e2 = fma(e, e, e2);
+    bnd = fma(s * s, invd2[jj], bnd);
     // feedback to this lane's later columns of the block
-    const float* urow = Us + jj * kBlock;
+    const double* urow = Us + jj * kBlock;
 #pragma unroll
     for (int ci = jj / (4 * kP); ci < kVPL / 4; ++ci) {
-      const float4 u4 = *reinterpret_cast<const float4*>(urow + 4 * kP * ci + 4 * t);
+      const double2 u01 = *reinterpret_cast<const double2*>(urow + 4 * kP * ci + 4 * t);
+      const double2 u23 = *reinterpret_cast<const double2*>(urow + 4 * kP * ci + 4 * t + 2);
       if (ci > jj / (4 * kP)) {
-        v[4 * ci + 0] = fmaf(-e, u4.x, v[4 * ci + 0]);
-        v[4 * ci + 1] = fmaf(-e, u4.y, v[4 * ci + 1]);
-        v[4 * ci + 2] = fmaf(-e, u4.z, v[4 * ci + 2]);
-        v[4 * ci + 3] = fmaf(-e, u4.w, v[4 * ci + 3]);
-      } else {
-        // the chunk that holds column jj: U's upper structure zeroes k <= jj, so the update
-        // is harmless for those slots (U[jj][k] = 0 for k < jj; k == jj is never read again)
-        if (t >= owner) {
-          if (t > owner || 0 > (jj % 4)) v[4 * ci + 0] = fmaf(-e, u4.x, v[4 * ci + 0]);
-          if (t > owner || 1 > (jj % 4)) v[4 * ci + 1] = fmaf(-e, u4.y, v[4 * ci + 1]);
-          if (t > owner || 2 > (jj % 4)) v[4 * ci + 2] = fmaf(-e, u4.z, v[4 * ci + 2]);
-          if (t > owner || 3 > (jj % 4)) v[4 * ci + 3] = fmaf(-e, u4.w, v[4 * ci + 3]);
-        }
+        v[4 * ci + 0] = fma(-e, u01.x, v[4 * ci + 0]);
+        v[4 * ci + 1] = fma(-e, u01.y, v[4 * ci + 1]);
+        v[4 * ci + 2] = fma(-e, u23.x, v[4 * ci + 2]);
+        v[4 * ci + 3] = fma(-e, u23.y, v[4 * ci + 3]);
+      } else if (t >= owner) {
+        // the chunk that holds column jj: only its later columns
+        if (t > owner || 0 > (jj % 4)) v[4 * ci + 0] = fma(-e, u01.x, v[4 * ci + 0]);
+        if (t > owner || 1 > (jj % 4)) v[4 * ci + 1] = fma(-e, u01.y, v[4 * ci + 1]);
+        if (t > owner || 2 > (jj % 4)) v[4 * ci + 2] = fma(-e, u23.x, v[4 * ci + 2]);
+        if (t > owner || 3 > (jj % 4)) v[4 * ci + 3] = fma(-e, u23.y, v[4 * ci + 3]);
       }
     }
     }
@@ -462,7 +465,7 @@ __global__ void q_ladder_kernel(int64_t m, int* overflow, float* alpha, float la
     if (_e != cudaSuccess) return GQ_ERR_CUDA;      \
   } while (0)
 
-constexpr size_t kColSmem = (size_t)(kBlock * kBlock + 2 * kBlock) * sizeof(float);
+constexpr size_t kColSmem = (size_t)(kBlock * kBlock + 2 * kBlock) * sizeof(double);
 
 cudaError_t quant_init_attributes() {
   const int smem = (int)kColSmem;

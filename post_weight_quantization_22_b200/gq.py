@@ -47,7 +47,7 @@ def _load():
     lib.gq_prepare_workspace_size.restype = SZ
     lib.gq_prepare_workspace_size.argtypes = [I64]
     lib.gq_prepare_hinv.restype = I
-    lib.gq_prepare_hinv.argtypes = [P, I64, F, I, P, P, P, P, SZ, P]
+    lib.gq_prepare_hinv.argtypes = [P, I64, ctypes.c_double, I, P, P, P, P, SZ, P]
     lib.gq_quantize_workspace_size.restype = SZ
     lib.gq_quantize_workspace_size.argtypes = [I64, I64, ctypes.POINTER(_Cfg)]
     lib.gq_quantize_layer.restype = I
@@ -170,10 +170,8 @@ def gq_quantize_layer(W: torch.Tensor, U: torch.Tensor, dead, delta, cfg: QuantC
     scales = torch.empty((m, G), dtype=torch.float32, device=dev) if scales is None else scales
     zeros = torch.empty((m, G), dtype=torch.uint8, device=dev) if zeros is None else zeros
     loss = torch.empty(3, dtype=torch.float64, device=dev) if loss is None else loss
-    need = gq_quantize_workspace_size(m, n, cfg)
-    if need == 0:
-        raise GQError(1, "gq_quantize_workspace_size")
-    ws = workspace(need, dev) if ws is None else ws
+    # a rejected configuration sizes to 0; the call itself then reports the precise status
+    ws = workspace(gq_quantize_workspace_size(m, n, cfg), dev) if ws is None else ws
     c = cfg.c()
     _check(LIB.gq_quantize_layer(_ptr(W), _dtype_code(W), m, n, _ptr(U), _ptr(dead), _ptr(delta),
                                  ctypes.byref(c), _ptr(codes), _ptr(scales), _ptr(zeros),
