@@ -2,7 +2,10 @@
 #include "gq_internal.cuh"
 
 #include <atomic>
+#include <cstring>
+#include <list>
 #include <mutex>
+#include <vector>
 
 using namespace gq;
 
@@ -31,6 +34,79 @@ gq_status ensure_device_setup() {
 }
 
 bool aligned256(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 255u) == 0; }
+
+// ---- launch-sequence graphs -------------------------------------------------------------
+// A call's kernel sequence (hundreds of small dependent launches for the factorisation) is
+// captured once per distinct argument list on a private stream, instantiated, and replayed on
+// the caller's stream; replay costs one graph launch instead of one launch per kernel.  A
+// caller that is itself capturing gets the plain launches recorded into its own graph.
+struct GraphEntry {
+  int device;
+  std::vector<uint64_t> key;
+  cudaGraphExec_t exec;
+  unsigned long long kernels;  // kernel nodes, counted in gq_kernel_launches per replay
+};
+std::mutex g_graph_mu;
+std::list<GraphEntry> g_graphs;  // most recently used first
+constexpr size_t kMaxGraphs = 32;
+cudaStream_t g_capture_stream[128] = {};
+
+template <class Enqueue>
+gq_status run_graphed(std::vector<uint64_t> key, cudaStream_t user, Enqueue enqueue) {
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(user, &cs) != cudaSuccess) return GQ_ERR_CUDA;
+  if (cs != cudaStreamCaptureStatusNone) return enqueue(user);
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return GQ_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_graph_mu);
+  for (auto it = g_graphs.begin(); it != g_graphs.end(); ++it) {
+    if (it->device == dev && it->key == key) {
+      g_graphs.splice(g_graphs.begin(), g_graphs, it);
+      if (cudaGraphLaunch(it->exec, user) != cudaSuccess) return GQ_ERR_CUDA;
+      count_launches((long)it->kernels);
+      return GQ_OK;
+    }
+  }
+  if (!g_capture_stream[dev] &&
+      cudaStreamCreateWithFlags(&g_capture_stream[dev], cudaStreamNonBlocking) != cudaSuccess)
+    return GQ_ERR_CUDA;
+  cudaStream_t cap = g_capture_stream[dev];
+  if (cudaStreamBeginCapture(cap, cudaStreamCaptureModeThreadLocal) != cudaSuccess)
+    return GQ_ERR_CUDA;
+  const unsigned long long before = g_launches.load();
+  gq_status st = enqueue(cap);
+  const unsigned long long kernels = g_launches.load() - before;
+  g_launches.fetch_sub(kernels);  // captured, not yet run
+  cudaGraph_t graph = nullptr;
+  cudaError_t ec = cudaStreamEndCapture(cap, &graph);
+  if (st != GQ_OK || ec != cudaSuccess || !graph) {
+    if (graph) cudaGraphDestroy(graph);
+    (void)cudaGetLastError();
+    return st != GQ_OK ? st : GQ_ERR_CUDA;
+  }
+  cudaGraphExec_t exec = nullptr;
+  ec = cudaGraphInstantiate(&exec, graph, 0);
+  cudaGraphDestroy(graph);
+  if (ec != cudaSuccess) {
+    (void)cudaGetLastError();
+    return enqueue(user);  // not instantiable: plain launches on the caller's stream
+  }
+  if (g_graphs.size() >= kMaxGraphs) {
+    cudaGraphExecDestroy(g_graphs.back().exec);
+    g_graphs.pop_back();
+  }
+  g_graphs.push_front(GraphEntry{dev, std::move(key), exec, kernels});
+  if (cudaGraphLaunch(exec, user) != cudaSuccess) return GQ_ERR_CUDA;
+  count_launches((long)kernels);
+  return GQ_OK;
+}
+
+uint64_t bits_of(double d) {
+  uint64_t u;
+  std::memcpy(&u, &d, sizeof u);
+  return u;
+}
+uint64_t P(const void* p) { return (uint64_t)(uintptr_t)p; }
 
 }  // namespace
 
@@ -80,9 +156,13 @@ gq_status gq_prepare_hinv(const double* d_H, int64_t n, double damp, int reverse
   if (!aligned256(d_ws) || ws_bytes < prepare_ws_bytes(n)) return GQ_ERR_WORKSPACE;
   gq_status st = ensure_device_setup();
   if (st != GQ_OK) return st;
-  cudaError_t e = launch_prepare(d_H, n, damp, reverse, d_U, d_dead, d_delta, d_ws,
-                                 (cudaStream_t)stream);
-  return e == cudaSuccess ? GQ_OK : GQ_ERR_CUDA;
+  auto enqueue = [&](cudaStream_t s) {
+    return launch_prepare(d_H, n, damp, reverse, d_U, d_dead, d_delta, d_ws, s) == cudaSuccess
+               ? GQ_OK : GQ_ERR_CUDA;
+  };
+  return run_graphed({1, P(d_H), (uint64_t)n, bits_of(damp), (uint64_t)reverse, P(d_U),
+                      P(d_dead), P(d_delta), P(d_ws)},
+                     (cudaStream_t)stream, enqueue);
 }
 
 static gq_status check_cfg(const gq_quant_cfg* cfg) {
@@ -126,7 +206,13 @@ gq_status gq_quantize_layer(const void* d_W, gq_dtype w_dtype, int64_t m, int64_
   a.W = d_W; a.wt = w_dtype; a.m = m; a.n = n; a.U = d_U; a.dead = d_dead; a.delta = d_delta;
   a.cfg = *cfg; a.codes = d_codes; a.scales = d_scales; a.zeros = d_zeros; a.loss = d_loss;
   a.ws = d_ws;
-  return run_quantize(a, (cudaStream_t)stream);
+  if (!cfg->clip) return run_quantize(a, (cudaStream_t)stream);  // the ladder reads back counts
+  auto enqueue = [&](cudaStream_t s) { return run_quantize(a, s); };
+  return run_graphed({2, P(d_W), (uint64_t)w_dtype, (uint64_t)m, (uint64_t)n, P(d_U), P(d_dead),
+                      P(d_delta), (uint64_t)cfg->bits, (uint64_t)cfg->group_size,
+                      (uint64_t)cfg->reverse, (uint64_t)cfg->clip, P(d_codes), P(d_scales),
+                      P(d_zeros), P(d_loss), P(d_ws)},
+                     (cudaStream_t)stream, enqueue);
 }
 
 gq_status gq_workspace_status(void* d_ws, int* h_ladder_rounds, gq_stream_t stream) {

@@ -4,9 +4,14 @@
 //   opA[i][k] = A_T ? A[k*lda + i] : A[i*lda + k]      (A element type TA, converted to fp64)
 //   opB[k][j] = B_T ? B[j*ldb + k] : B[k*ldb + j]
 //
-// Optional structure: a_lower (opA[i][k] = 0 for k > i), b_lower (opB[k][j] = 0 for k < j),
-// lower_tiles (skip 64x64 output tiles strictly above the diagonal).  Batched over
-// blockIdx.z with element strides.
+// Optional structure (skipped work and masked loads, never reads of the masked entries):
+//   a_lower:  opA[i][k] = 0 for k > i        b_lower: opB[k][j] = 0 for k < j
+//   b_upper:  opB[k][j] = 0 for k > j        lower_tiles: skip output tiles above the diagonal
+// Batched over blockIdx.z with element strides.
+//
+// Tile BT x BT x 8 (BT = 64 or 128, chosen by the launcher from the grid size), 256 threads,
+// (BT/16)^2 outputs per thread (rows ty + 16 i, columns tx + 16 j: conflict-free
+// shared-memory reads), register-staged double buffering.
 #pragma once
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
@@ -16,8 +21,7 @@
 
 namespace gq {
 
-constexpr int kGB = 64;   // output tile edge
-constexpr int kGK = 16;   // k step
+constexpr int kGK = 8;    // k step
 
 template <class T>
 __device__ __forceinline__ double to_f64(T v);
@@ -40,13 +44,15 @@ struct F64GemmArgs {
   int64_t ldb, strideB;
   double* C;
   int64_t ldc, strideC;
-  int a_lower, b_lower, lower_tiles;
+  int a_lower, b_lower, b_upper, lower_tiles;
 };
 
-template <class TA, class TB, bool A_T, bool B_T>
+template <class TA, class TB, bool A_T, bool B_T, int kGB>
 __global__ void __launch_bounds__(256) f64_gemm_kernel(F64GemmArgs g) {
-  __shared__ double As[kGK][kGB + 1];
-  __shared__ double Bs[kGK][kGB + 1];
+  constexpr int TM = kGB / 16;   // outputs per thread per dimension
+  constexpr int LPT = kGB / 32;  // tile elements loaded per thread per operand and k step
+  __shared__ double As[2][kGK][kGB];
+  __shared__ double Bs[2][kGK][kGB];
   const int ti = blockIdx.y, tj = blockIdx.x;
   if (g.lower_tiles && tj > ti) return;
   const int i0 = ti * kGB, j0 = tj * kGB;
@@ -57,62 +63,84 @@ __global__ void __launch_bounds__(256) f64_gemm_kernel(F64GemmArgs g) {
 
   int k_lo = 0, k_hi = g.K;
   if (g.a_lower) k_hi = min(k_hi, i0 + kGB);
+  if (g.b_upper) k_hi = min(k_hi, j0 + kGB);
   if (g.b_lower) k_lo = (j0 / kGK) * kGK;
 
   const int tid = threadIdx.x;
   const int tx = tid % 16, ty = tid / 16;
-  double acc[4][4];
+  double acc[TM][TM];
 #pragma unroll
-  for (int a = 0; a < 4; ++a)
+  for (int a = 0; a < TM; ++a)
 #pragma unroll
-    for (int b = 0; b < 4; ++b) acc[a][b] = 0.0;
+    for (int b = 0; b < TM; ++b) acc[a][b] = 0.0;
 
-  for (int k0 = k_lo; k0 < k_hi; k0 += kGK) {
-    // ---- load opA tile (64 i x 16 k) ----
+  double ra[LPT], rb[LPT];
+  auto load_tiles = [&](int k0) {
 #pragma unroll
-    for (int r = 0; r < 4; ++r) {
-      int e = tid + 256 * r;  // 0..1023
+    for (int r = 0; r < LPT; ++r) {
+      int e = tid + 256 * r;
       int ii, kk;
       if (A_T) { kk = e / kGB; ii = e % kGB; } else { ii = e / kGK; kk = e % kGK; }
       int gi = i0 + ii, gk = k0 + kk;
       double v = 0.0;
-      if (gi < g.M && gk < k_hi && !(g.a_lower && gk > gi)) {
+      if (gi < g.M && gk < k_hi && !(g.a_lower && gk > gi))
         v = A_T ? to_f64<TA>(A[(int64_t)gk * g.lda + gi]) : to_f64<TA>(A[(int64_t)gi * g.lda + gk]);
-      }
-      As[kk][ii] = v;
-    }
-    // ---- load opB tile (16 k x 64 j) ----
-#pragma unroll
-    for (int r = 0; r < 4; ++r) {
-      int e = tid + 256 * r;
-      int jj, kk;
+      ra[r] = v;
+      int jj;
       if (B_T) { jj = e / kGK; kk = e % kGK; } else { kk = e / kGB; jj = e % kGB; }
-      int gj = j0 + jj, gk = k0 + kk;
-      double v = 0.0;
-      if (gj < g.N && gk < k_hi && gk >= k_lo && !(g.b_lower && gk < gj)) {
+      int gj = j0 + jj;
+      gk = k0 + kk;
+      v = 0.0;
+      if (gj < g.N && gk < k_hi && gk >= k_lo && !(g.b_lower && gk < gj) &&
+          !(g.b_upper && gk > gj))
         v = B_T ? to_f64<TB>(B[(int64_t)gj * g.ldb + gk]) : to_f64<TB>(B[(int64_t)gk * g.ldb + gj]);
+      rb[r] = v;
+    }
+  };
+  auto store_tiles = [&](int buf) {
+#pragma unroll
+    for (int r = 0; r < LPT; ++r) {
+      int e = tid + 256 * r;
+      int ii, kk;
+      if (A_T) { kk = e / kGB; ii = e % kGB; } else { ii = e / kGK; kk = e % kGK; }
+      As[buf][kk][ii] = ra[r];
+      int jj;
+      if (B_T) { jj = e / kGK; kk = e % kGK; } else { kk = e / kGB; jj = e % kGB; }
+      Bs[buf][kk][jj] = rb[r];
+    }
+  };
+
+  if (k_lo < k_hi) {
+    load_tiles(k_lo);
+    store_tiles(0);
+    __syncthreads();
+    int buf = 0;
+    for (int k0 = k_lo; k0 < k_hi; k0 += kGK) {
+      const bool more = k0 + kGK < k_hi;
+      if (more) load_tiles(k0 + kGK);
+#pragma unroll
+      for (int kk = 0; kk < kGK; ++kk) {
+        double a[TM], b[TM];
+#pragma unroll
+        for (int q = 0; q < TM; ++q) { a[q] = As[buf][kk][ty + 16 * q]; b[q] = Bs[buf][kk][tx + 16 * q]; }
+#pragma unroll
+        for (int p = 0; p < TM; ++p)
+#pragma unroll
+          for (int q = 0; q < TM; ++q) acc[p][q] = fma(a[p], b[q], acc[p][q]);
       }
-      Bs[kk][jj] = v;
+      if (more) {
+        store_tiles(buf ^ 1);
+        __syncthreads();
+        buf ^= 1;
+      }
     }
-    __syncthreads();
-#pragma unroll
-    for (int kk = 0; kk < kGK; ++kk) {
-      double a[4], b[4];
-#pragma unroll
-      for (int q = 0; q < 4; ++q) { a[q] = As[kk][ty + 16 * q]; b[q] = Bs[kk][tx + 16 * q]; }
-#pragma unroll
-      for (int p = 0; p < 4; ++p)
-#pragma unroll
-        for (int q = 0; q < 4; ++q) acc[p][q] = fma(a[p], b[q], acc[p][q]);
-    }
-    __syncthreads();
   }
 #pragma unroll
-  for (int p = 0; p < 4; ++p) {
+  for (int p = 0; p < TM; ++p) {
     int gi = i0 + ty + 16 * p;
     if (gi >= g.M) continue;
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
+    for (int q = 0; q < TM; ++q) {
       int gj = j0 + tx + 16 * q;
       if (gj >= g.N) continue;
       double* c = C + (int64_t)gi * g.ldc + gj;
@@ -125,8 +153,16 @@ __global__ void __launch_bounds__(256) f64_gemm_kernel(F64GemmArgs g) {
 template <class TA, class TB, bool A_T, bool B_T>
 inline cudaError_t f64_gemm(const F64GemmArgs& g, int batch, cudaStream_t s) {
   if (g.M <= 0 || g.N <= 0 || batch <= 0) return cudaSuccess;
-  dim3 grid((g.N + kGB - 1) / kGB, (g.M + kGB - 1) / kGB, batch);
-  f64_gemm_kernel<TA, TB, A_T, B_T><<<grid, 256, 0, s>>>(g);
+  // 128-wide tiles only when they still give every SM two tiles
+  const int64_t t128 = (int64_t)((g.M + 127) / 128) * ((g.N + 127) / 128) * batch;
+  const int64_t busy = g.lower_tiles ? t128 / 2 : t128;
+  if (busy >= 2 * 148) {
+    dim3 grid((g.N + 127) / 128, (g.M + 127) / 128, batch);
+    f64_gemm_kernel<TA, TB, A_T, B_T, 128><<<grid, 256, 0, s>>>(g);
+  } else {
+    dim3 grid((g.N + 63) / 64, (g.M + 63) / 64, batch);
+    f64_gemm_kernel<TA, TB, A_T, B_T, 64><<<grid, 256, 0, s>>>(g);
+  }
   count_launches(1);
   return cudaGetLastError();
 }

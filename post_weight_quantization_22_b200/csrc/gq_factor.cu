@@ -69,15 +69,18 @@ __global__ void build_m_kernel(const double* H, int64_t n, int reverse, const Ws
 }
 
 // ---------------------------------------------------------------------------------------
-// Diagonal block: Cholesky of a <= 64 x 64 block in shared memory (Schur-complement form,
-// one barrier per pivot), then its triangular inverse.
+// Diagonal block (w <= 64): inverse of its Cholesky factor, in place, in one elimination pass.
+// Unnormalised elimination of [S | I] (S the block, symmetric, lower part used): at pivot c,
+// rows r > c take S[r][s] -= f_r S[s][c] (s in (c, r]) and A[r][j] -= f_r A[c][j] (j <= c),
+// f_r = S[r][c] / S[c][c].  Then A = L_unit^-1, the pivots are D of S = L_unit D L_unit^T, and
+// L^-1 = D^-1/2 A.  One barrier per pivot; 4 threads per row.
 // ---------------------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) potrf_diag_kernel(double* M, int64_t n, int64_t c0, int w,
-                                                         double* dinv, WsHeader* hdr) {
+                                                         WsHeader* hdr) {
   extern __shared__ double sm[];
-  double* S = sm;                       // [64][65]
-  double* X = sm + kNB * (kNB + 1);     // [64][65] inverse
   const int ld = kNB + 1;
+  double* S = sm;                 // [64][65] Schur complement (lower)
+  double* A = sm + kNB * ld;      // [64][65] eliminated identity (lower)
   const int tid = threadIdx.x;
   for (int e = tid; e < kNB * kNB; e += 256) {
     int i = e / kNB, j = e % kNB;
@@ -88,70 +91,40 @@ __global__ void __launch_bounds__(256) potrf_diag_kernel(double* M, int64_t n, i
       v = 1.0;
     }
     S[i * ld + j] = v;
+    A[i * ld + j] = (i == j) ? 1.0 : 0.0;
   }
   __syncthreads();
-  // Schur complement elimination; S[r][c] for r > c is final after step c.
   const int r = tid >> 2, part = tid & 3;
-  for (int c = 0; c < kNB; ++c) {
-    double p = S[c * ld + c];
-    if (!(p > 0.0)) p = 1.0;  // recorded below; keeps the arithmetic finite
-    double f = (r > c) ? S[r * ld + c] / p : 0.0;
+  for (int c = 0; c < kNB - 1; ++c) {
     if (r > c) {
-      for (int s = c + 1 + part; s <= r; s += 4) S[r * ld + s] -= f * S[s * ld + c];
+      double p = S[c * ld + c];
+      if (!(p > 0.0)) p = 1.0;  // recorded below; keeps the arithmetic finite
+      const double f = S[r * ld + c] / p;
+      // fixed trip counts with predicates: all loads of a pivot step issue back to back
+#pragma unroll
+      for (int i = 0; i < kNB / 4; ++i) {
+        const int q = c + 1 + part + 4 * i;
+        if (q <= r) S[r * ld + q] = fma(-f, S[q * ld + c], S[r * ld + q]);
+      }
+#pragma unroll
+      for (int i = 0; i < kNB / 4; ++i) {
+        const int j = part + 4 * i;
+        if (j <= c) A[r * ld + j] = fma(-f, A[c * ld + j], A[r * ld + j]);
+      }
     }
     __syncthreads();
   }
-  // L[r][c] = S[r][c] / sqrt(S[c][c]), L[c][c] = sqrt(S[c][c])
-  __shared__ double sq[kNB];
-  if (tid < kNB) {
-    double p = S[tid * ld + tid];
-    if (!(p > 0.0)) {
-      if (tid < w) record_status(hdr, GQ_ERR_NOT_PD);
-      p = 1.0;
-    }
-    sq[tid] = sqrt(p);
-  }
-  __syncthreads();
+  // L^-1[r][j] = A[r][j] / sqrt(D_r)
   for (int e = tid; e < kNB * kNB; e += 256) {
     int i = e / kNB, j = e % kNB;
-    if (j < i) S[i * ld + j] = S[i * ld + j] / sq[j];
-    else if (j == i) S[i * ld + j] = sq[i];
-    else S[i * ld + j] = 0.0;
-  }
-  __syncthreads();
-  // inverse, one column per thread (forward substitution L x = e_j)
-  if (tid < kNB) {
-    const int j = tid;
-    for (int i = 0; i < kNB; ++i) {
-      double acc0 = 0.0, acc1 = 0.0;
-      int k = j;
-      for (; k + 1 < i; k += 2) {
-        acc0 = fma(S[i * ld + k], X[k * ld + j], acc0);
-        acc1 = fma(S[i * ld + k + 1], X[(k + 1) * ld + j], acc1);
+    if (i < w && j <= i) {
+      double p = S[i * ld + i];
+      if (!(p > 0.0)) {
+        if (j == 0) record_status(hdr, GQ_ERR_NOT_PD);
+        p = 1.0;
       }
-      if (k < i) acc0 = fma(S[i * ld + k], X[k * ld + j], acc0);
-      double v = (i < j) ? 0.0 : (((i == j) ? 1.0 : 0.0) - (acc0 + acc1)) / S[i * ld + i];
-      X[i * ld + j] = v;
+      M[(c0 + i) * n + c0 + j] = A[i * ld + j] / sqrt(p);
     }
-  }
-  __syncthreads();
-  for (int e = tid; e < kNB * kNB; e += 256) {
-    int i = e / kNB, j = e % kNB;
-    if (i < w && j <= i) M[(c0 + i) * n + c0 + j] = S[i * ld + j];
-    dinv[e] = X[i * ld + j];
-  }
-}
-
-// diagonal blocks of M <- their inverses (lower parts)
-__global__ void put_diag_inv_kernel(double* M, int64_t n, const double* dinv) {
-  int64_t k = blockIdx.x;
-  int64_t c0 = k * kNB;
-  int64_t rem_ = n - c0;
-  int w = (int)(rem_ < kNB ? rem_ : kNB);
-  const double* D = dinv + k * kNB * kNB;
-  for (int e = threadIdx.x; e < kNB * kNB; e += blockDim.x) {
-    int i = e / kNB, j = e % kNB;
-    if (i < w && j <= i) M[(c0 + i) * n + c0 + j] = D[e];
   }
 }
 
@@ -170,9 +143,8 @@ __global__ void flip_to_u_kernel(const double* M, int64_t n, float* U) {
 // ---------------------------------------------------------------------------------------
 struct PrepLayout {
   WsHeader* hdr;
-  double* M;
-  double* dinv;
-  double* tbuf;
+  double* M;     // n x n: lower triangle = J P H_d P J, then the inverse of its Cholesky factor
+  double* tbuf;  // doubling scratch of the triangular inverse
   size_t bytes;
 };
 
@@ -181,7 +153,7 @@ static size_t trtri_tbuf_elems(int64_t n) {
   for (int64_t bs = kNB; bs < n; bs *= 2) {
     size_t tot = 0;
     for (int64_t r = 0; r + bs < n; r += 2 * bs) tot += (size_t)bs * bs;
-    if (tot > best) best = tot;
+    best = std::max(best, tot);
   }
   return best;
 }
@@ -191,8 +163,6 @@ static PrepLayout prep_layout(void* ws, int64_t n) {
   PrepLayout L;
   L.hdr = c.take<WsHeader>(1);
   L.M = c.take<double>((size_t)n * n);
-  int64_t nb = (n + kNB - 1) / kNB;
-  L.dinv = c.take<double>((size_t)nb * kNB * kNB);
   L.tbuf = c.take<double>(trtri_tbuf_elems(n) + 1);
   L.bytes = c.off;
   return L;
@@ -224,23 +194,25 @@ cudaError_t launch_prepare(const double* H, int64_t n, double damp, int reverse,
     count_launches(1);
     GQ_TRY(cudaGetLastError());
   }
-  // blocked right-looking Cholesky, lower, in place on M
+  // Blocked right-looking Cholesky of M (lower, in place, 64-wide panels).  Each diagonal block
+  // is replaced by the inverse of its factor; the panel below becomes L21 = A21 L11^-T; the
+  // trailing matrix takes A22 -= L21 L21^T.
   const int64_t nb = (n + kNB - 1) / kNB;
   const size_t psmem = 2 * kNB * (kNB + 1) * sizeof(double);
   for (int64_t k = 0; k < nb; ++k) {
     const int64_t c0 = k * kNB;
     const int w = (int)std::min<int64_t>(kNB, n - c0);
-    double* dk = L.dinv + k * kNB * kNB;
-    potrf_diag_kernel<<<1, 256, psmem, s>>>(L.M, n, c0, w, dk, L.hdr);
+    potrf_diag_kernel<<<1, 256, psmem, s>>>(L.M, n, c0, w, L.hdr);
     count_launches(1);
     GQ_TRY(cudaGetLastError());
     const int64_t rem = n - c0 - w;
     if (rem <= 0) continue;
     double* P = L.M + (c0 + w) * n + c0;
-    {  // panel: P <- P L_kk^-T (in place; one output tile column per CTA row)
+    {  // P <- P (L11^-1)^T  (in place: one output tile column, each CTA owns its rows)
       F64GemmArgs g{};
       g.M = (int)rem; g.N = w; g.K = w; g.alpha = 1.0; g.beta_one = 0;
-      g.A = P; g.lda = n; g.B = dk; g.ldb = kNB; g.C = P; g.ldc = n;
+      g.A = P; g.lda = n; g.B = L.M + c0 * n + c0; g.ldb = n; g.b_upper = 1;
+      g.C = P; g.ldc = n;
       GQ_TRY((f64_gemm<double, double, false, true>(g, 1, s)));
     }
     {  // trailing: C -= P P^T, lower tiles
@@ -251,14 +223,12 @@ cudaError_t launch_prepare(const double* H, int64_t n, double damp, int reverse,
       GQ_TRY((f64_gemm<double, double, false, true>(g, 1, s)));
     }
   }
-  put_diag_inv_kernel<<<(unsigned)nb, 256, 0, s>>>(L.M, n, L.dinv);
-  count_launches(1);
-  GQ_TRY(cudaGetLastError());
-  // triangular inverse by doubling: inv([[A,0],[B,C]]) = [[A^-1,0],[-C^-1 B A^-1, C^-1]]
+  // Triangular inverse by doubling over the diagonal blocks (already inverted):
+  //   inv([[A, 0], [B, C]]) = [[A^-1, 0], [-C^-1 B A^-1, C^-1]], all pairs of a level batched.
   for (int64_t bs = kNB; bs < n; bs *= 2) {
-    const int64_t npairs_full = n / (2 * bs);          // pairs with a full C block
-    const int64_t rtail = npairs_full * 2 * bs;        // start of a possible ragged pair
-    const int64_t cw_tail = n - rtail - bs;            // its C width (if > 0)
+    const int64_t npairs_full = n / (2 * bs);
+    const int64_t rtail = npairs_full * 2 * bs;
+    const int64_t cw_tail = n - rtail - bs;
     for (int pass = 0; pass < 2; ++pass) {
       int64_t r = pass == 0 ? 0 : rtail;
       int64_t cw = pass == 0 ? bs : cw_tail;

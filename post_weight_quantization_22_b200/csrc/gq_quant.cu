@@ -152,15 +152,18 @@ struct ColArgs {
   int* overflow;
 };
 
-// Lane ownership: lane t of a row owns columns k = 4*P*(i/4) + 4*t + (i%4), i in [0, 32):
-// 4-wide chunks interleaved across the P lanes (balanced work, 16-byte shared-memory loads).
+// Lane ownership: the block's 128 columns form 8 segments of 16; in each segment lane t of a
+// row owns the 4-column chunk [16 seg + 4t, 16 seg + 4t + 4).  Each lane keeps its 8 chunks in
+// registers, v[4c + u] = chunk (seg + c); after a segment the array is rotated by one chunk,
+// so the unrolled 16-step body refers to fixed registers and the segment loop stays a small
+// runtime loop (a fully unrolled 128-step body does not fit the instruction cache).
 //
-// The recursion runs in fp64: the in-block feedback sums cancel strongly when the per-row
-// grid is coarse, and an fp32 recursion flips ~1-3 % of the codes on ill-conditioned layers
-// (measured against the fp64 oracle), while fp64 here with fp32 storage of W, E and U between
-// blocks reproduces the oracle's codes.
+// The recursion runs in fp64: the in-block feedback sums cancel strongly when the grid is
+// coarse, and an fp32 recursion flips ~1-3 % of the codes on ill-conditioned layers (measured
+// against the fp64 oracle), while fp64 here with fp32 storage of W, E and U between blocks
+// reproduces the oracle's codes.
 template <int G>
-__global__ void __launch_bounds__(128) colloop_kernel(ColArgs a) {
+__global__ void __launch_bounds__(128, 1) colloop_kernel(ColArgs a) {
   extern __shared__ __align__(16) double q_smem[];
   double* Us = q_smem;                       // [128][128]
   double* invd = q_smem + kBlock * kBlock;   // [128]  1/U_jj
@@ -194,8 +197,8 @@ __global__ void __launch_bounds__(128) colloop_kernel(ColArgs a) {
 
   double v[kVPL];
 #pragma unroll
-  for (int ci = 0; ci < kVPL / 4; ++ci) {
-    int k = 4 * kP * ci + 4 * t;
+  for (int c = 0; c < kVPL / 4; ++c) {
+    int k = 16 * c + 4 * t;
     float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
     if (active) {
       const float* src = a.Wf + rr * n + j0 + k;
@@ -207,33 +210,27 @@ __global__ void __launch_bounds__(128) colloop_kernel(ColArgs a) {
         for (int u = 0; u < 4; ++u) dx[u] = (k + u < bw) ? src[u] : 0.f;
       }
     }
-    v[4 * ci + 0] = x.x; v[4 * ci + 1] = x.y; v[4 * ci + 2] = x.z; v[4 * ci + 3] = x.w;
+    v[4 * c + 0] = x.x; v[4 * c + 1] = x.y; v[4 * c + 2] = x.z; v[4 * c + 3] = x.w;
   }
   double s = 1.0, inv_s = 1.0, z = 0.0;
   if (G == 0 && active) { s = a.row_s[row]; z = a.row_z[row]; inv_s = 1.0 / s; }
-  float eo[kVPL];
-  uint32_t cw[kVPL / 4];
-#pragma unroll
-  for (int i = 0; i < kVPL; ++i) eo[i] = 0.f;
-#pragma unroll
-  for (int i = 0; i < kVPL / 4; ++i) cw[i] = 0u;
   double e2 = 0.0, bnd = 0.0;
   int ovf = 0;
   const unsigned full = 0xffffffffu;
   const int gbase = lane & ~(kP - 1);
+  float* Erow = a.E + rr * kBlock;
+  uint8_t* crow = a.codes8 + row * a.ldc8 + j0;
 
-#pragma unroll
-  for (int jj = 0; jj < kBlock; ++jj) {
-    if (jj < bw) {
+  for (int seg = 0; seg < kBlock / 16; ++seg) {
+    if (16 * seg >= bw) break;
     if constexpr (G > 0) {
-      if (jj % G == 0) {
+      if ((16 * seg) % G == 0) {
         double lo = 0.0, hi = 0.0;
 #pragma unroll
-        for (int i = 0; i < kVPL; ++i) {
-          // owned column of slot i
-          const int k = 4 * kP * (i / 4) + 4 * t + (i % 4);
-          if (k >= jj && k < jj + G && k < bw) { lo = fmin(lo, v[i]); hi = fmax(hi, v[i]); }
-        }
+        for (int c = 0; c < (G / 16 < 8 ? G / 16 : 8); ++c)
+#pragma unroll
+          for (int u = 0; u < 4; ++u)
+            if (16 * (seg + c) + 4 * t + u < bw) { lo = fmin(lo, v[4 * c + u]); hi = fmax(hi, v[4 * c + u]); }
 #pragma unroll
         for (int o = kP / 2; o > 0; o >>= 1) {
           lo = fmin(lo, __shfl_xor_sync(full, lo, o));
@@ -244,72 +241,80 @@ __global__ void __launch_bounds__(128) colloop_kernel(ColArgs a) {
         z = rint(-lo / s);
         inv_s = 1.0 / s;
         if (active && t == 0) {
-          int64_t g = (j0 + jj) / G;
+          int64_t g = (j0 + 16 * seg) / G;
           a.scales[row * a.ngroups + g] = (float)s;
           a.zeros[row * a.ngroups + g] = (uint8_t)z;
         }
       }
     }
-    const int owner = (jj / 4) % kP;
-    const int idx = (jj / (4 * kP)) * 4 + (jj % 4);
-    const double x = __shfl_sync(full, v[idx], gbase + owner);
-    double c = rint(x * inv_s) + z;
-    if (a.clip) {
-      c = fmin(fmax(c, 0.0), maxq);
-    } else if (c < 0.0 || c > maxq) {
-      ovf = 1;
-    }
-    const double q = s * (c - z);
-    const double e = (x - q) * invd[jj];
-    if (t == owner) {
-      eo[idx] = (float)e;
-      uint32_t cb = (uint32_t)(int)fmin(fmax(c, 0.0), maxq);
-      cw[idx / 4] |= cb << (8 * (idx % 4));
-    }
-    e2 = fma(e, e, e2);
-    bnd = fma(s * s, invd2[jj], bnd);
-    // feedback to this lane's later columns of the block
-    const double* urow = Us + jj * kBlock;
+    const double cmin = -z, cmax = maxq - z;  // code range in the shifted domain c - z
+    float eo[4] = {0.f, 0.f, 0.f, 0.f};
+    uint32_t cw = 0u;
 #pragma unroll
-    for (int ci = jj / (4 * kP); ci < kVPL / 4; ++ci) {
-      const double2 u01 = *reinterpret_cast<const double2*>(urow + 4 * kP * ci + 4 * t);
-      const double2 u23 = *reinterpret_cast<const double2*>(urow + 4 * kP * ci + 4 * t + 2);
-      if (ci > jj / (4 * kP)) {
-        v[4 * ci + 0] = fma(-e, u01.x, v[4 * ci + 0]);
-        v[4 * ci + 1] = fma(-e, u01.y, v[4 * ci + 1]);
-        v[4 * ci + 2] = fma(-e, u23.x, v[4 * ci + 2]);
-        v[4 * ci + 3] = fma(-e, u23.y, v[4 * ci + 3]);
-      } else if (t >= owner) {
-        // the chunk that holds column jj: only its later columns
-        if (t > owner || 0 > (jj % 4)) v[4 * ci + 0] = fma(-e, u01.x, v[4 * ci + 0]);
-        if (t > owner || 1 > (jj % 4)) v[4 * ci + 1] = fma(-e, u01.y, v[4 * ci + 1]);
-        if (t > owner || 2 > (jj % 4)) v[4 * ci + 2] = fma(-e, u23.x, v[4 * ci + 2]);
-        if (t > owner || 3 > (jj % 4)) v[4 * ci + 3] = fma(-e, u23.y, v[4 * ci + 3]);
+    for (int jl = 0; jl < 16; ++jl) {
+      const int jj = 16 * seg + jl;
+      if (jj < bw) {
+        const int owner = jl / 4, slot = jl % 4;
+        const double id = invd[jj];
+        const double sd = s * id;
+        const double x = __shfl_sync(full, v[slot], gbase + owner);
+        const double xi = x * id;
+        double c = rint(x * inv_s);
+        if (a.clip) {
+          c = fmin(fmax(c, cmin), cmax);
+        } else if (c < cmin || c > cmax) {
+          ovf = 1;
+        }
+        const double e = fma(-c, sd, xi);  // (x - s c) / U_jj
+        if (t == owner) {
+          eo[slot] = (float)e;
+          cw |= (uint32_t)(int)fmin(fmax(c + z, 0.0), maxq) << (8 * slot);
+        }
+        e2 = fma(e, e, e2);
+        bnd = fma(s * s, invd2[jj], bnd);
+        const double* urow = Us + jj * kBlock + 16 * seg + 4 * t;
+        if (t >= owner) {  // the chunk that holds column jj: only its later columns
+          const double2 u01 = *reinterpret_cast<const double2*>(urow);
+          const double2 u23 = *reinterpret_cast<const double2*>(urow + 2);
+          if (t > owner || 0 > slot) v[0] = fma(-e, u01.x, v[0]);
+          if (t > owner || 1 > slot) v[1] = fma(-e, u01.y, v[1]);
+          if (t > owner || 2 > slot) v[2] = fma(-e, u23.x, v[2]);
+          if (t > owner || 3 > slot) v[3] = fma(-e, u23.y, v[3]);
+        }
+#pragma unroll
+        for (int c2 = 1; c2 < kVPL / 4; ++c2) {
+          if (c2 < kBlock / 16 - seg) {
+            const double2 u01 = *reinterpret_cast<const double2*>(urow + 16 * c2);
+            const double2 u23 = *reinterpret_cast<const double2*>(urow + 16 * c2 + 2);
+            v[4 * c2 + 0] = fma(-e, u01.x, v[4 * c2 + 0]);
+            v[4 * c2 + 1] = fma(-e, u01.y, v[4 * c2 + 1]);
+            v[4 * c2 + 2] = fma(-e, u23.x, v[4 * c2 + 2]);
+            v[4 * c2 + 3] = fma(-e, u23.y, v[4 * c2 + 3]);
+          }
+        }
       }
     }
+    // this segment's errors and codes
+    if (active) {
+      const int k = 16 * seg + 4 * t;
+      *reinterpret_cast<float4*>(Erow + k) = make_float4(eo[0], eo[1], eo[2], eo[3]);
+      if (k + 3 < bw) {
+        *reinterpret_cast<uint32_t*>(crow + k) = cw;
+      } else {
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+          if (k + u < bw) crow[k + u] = (uint8_t)(cw >> (8 * u));
+      }
     }
+    // rotate: chunk seg + 1 moves to registers 0..3
+#pragma unroll
+    for (int i = 0; i < kVPL - 4; ++i) v[i] = v[i + 4];
   }
   // per-row overflow flag (all lanes of the warp take part in the shuffle)
   int ovf_row = ovf;
 #pragma unroll
   for (int o = kP / 2; o > 0; o >>= 1) ovf_row |= __shfl_xor_sync(0xffffffffu, ovf_row, o);
   if (!active) return;
-  // write back this lane's errors and codes
-  float* Erow = a.E + rr * kBlock;
-  uint8_t* crow = a.codes8 + row * a.ldc8 + j0;
-#pragma unroll
-  for (int ci = 0; ci < kVPL / 4; ++ci) {
-    int k = 4 * kP * ci + 4 * t;
-    *reinterpret_cast<float4*>(Erow + k) =
-        make_float4(eo[4 * ci + 0], eo[4 * ci + 1], eo[4 * ci + 2], eo[4 * ci + 3]);
-    if (k + 3 < bw) {
-      *reinterpret_cast<uint32_t*>(crow + k) = cw[ci];
-    } else {
-#pragma unroll
-      for (int u = 0; u < 4; ++u)
-        if (k + u < bw) crow[k + u] = (uint8_t)(cw[ci] >> (8 * u));
-    }
-  }
   // per-row totals (all lanes of a row hold the same e2 / bnd)
   if (t == 0) {
     if (j0 == 0) { a.row_e2[row] = e2; a.row_bnd[row] = bnd; a.overflow[row] = ovf_row; }
