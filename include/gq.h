@@ -114,6 +114,30 @@ gq_status gq_prepare_hinv(const double* d_H, int64_t n, double damp, int reverse
                           uint8_t* d_dead, double* d_delta, void* d_ws, size_t ws_bytes,
                           gq_stream_t stream);
 
+/*
+ * gq_prepare_hinv without a workspace, for callers that cannot allocate device memory at call
+ * time (a plugin whose memory plan is fixed in advance, code recorded into a CUDA graph under
+ * a capture mode that forbids cudaMalloc, a host that hands this library only its inputs and
+ * outputs).  The papers have no counterpart of this call; it exists for such callers.
+ *
+ * Same arguments and results as gq_prepare_hinv, minus the workspace: the scratch is a static
+ * device array inside the library (about 11 MB per device that loads the library, held until
+ * the process exits), so n is limited to 1 <= n <= 1024; larger n returns GQ_ERR_INVALID_ARG
+ * and enqueues nothing.  No device memory is allocated or freed.
+ *
+ *   d_status   optional (may be NULL) device int, written on `stream` with the device-side
+ *              status of this call (GQ_OK, or GQ_ERR_NOT_PD for a non-positive pivot).
+ *
+ * The first call on a device looks up the scratch array's device address (once per device);
+ * make that first call outside any stream capture.  Every call on a device shares the one
+ * scratch array and leaves its contents behind; each call clears what it needs cleared.  Two
+ * calls whose work overlaps on the GPU (different streams, no ordering between them) race on
+ * the scratch and give undefined results: order them on one stream or with events.
+ */
+gq_status gq_prepare_hinv_static(const double* d_H, int64_t n, double damp, int reverse,
+                                 float* d_U, uint8_t* d_dead, double* d_delta, int* d_status,
+                                 gq_stream_t stream);
+
 /* Workspace bytes gq_quantize_layer needs for an m x n layer under cfg. */
 size_t gq_quantize_workspace_size(int64_t m, int64_t n, const gq_quant_cfg* cfg);
 

@@ -53,6 +53,8 @@ def _load():
     lib.gq_quantize_layer.restype = I
     lib.gq_quantize_layer.argtypes = [P, I, I64, I64, P, P, P, ctypes.POINTER(_Cfg), P, P, P, P,
                                       P, SZ, P]
+    lib.gq_prepare_hinv_static.restype = I
+    lib.gq_prepare_hinv_static.argtypes = [P, I64, ctypes.c_double, I, P, P, P, P, P]
     lib.gq_workspace_status.restype = I
     lib.gq_workspace_status.argtypes = [P, ctypes.POINTER(ctypes.c_int), P]
     return lib
@@ -61,7 +63,7 @@ def _load():
 LIB = _load()
 EXPORTED = ("gq_version", "gq_status_string", "gq_hessian_accumulate", "gq_prepare_workspace_size",
             "gq_prepare_hinv", "gq_quantize_workspace_size", "gq_quantize_layer",
-            "gq_workspace_status")
+            "gq_workspace_status", "gq_prepare_hinv_static")
 
 
 def _ptr(t):
@@ -132,6 +134,24 @@ def gq_prepare_hinv(H: torch.Tensor, damp: float = 0.01, reverse: bool = False, 
                                _ptr(delta), _ptr(ws), ws.numel(), _stream(stream)),
            "gq_prepare_hinv")
     return U, dead, delta, ws
+
+
+def gq_prepare_hinv_static(H: torch.Tensor, damp: float = 0.01, reverse: bool = False, U=None,
+                           dead=None, delta=None, status=None, stream=None):
+    """gq_prepare_hinv on the library's built-in scratch (n <= 1024; no device allocation by
+    the library).  Returns (U, dead, delta, status) with status a device int32 [1]."""
+    n = H.shape[0]
+    _need(H, torch.float64, (n, n), "H")
+    dev = H.device
+    U = torch.empty((n, n), dtype=torch.float32, device=dev) if U is None else U
+    dead = torch.empty(n, dtype=torch.uint8, device=dev) if dead is None else dead
+    delta = torch.empty(1, dtype=torch.float64, device=dev) if delta is None else delta
+    status = torch.empty(1, dtype=torch.int32, device=dev) if status is None else status
+    _need(U, torch.float32, (n, n), "U")
+    _check(LIB.gq_prepare_hinv_static(_ptr(H), n, float(damp), int(bool(reverse)), _ptr(U),
+                                      _ptr(dead), _ptr(delta), _ptr(status), _stream(stream)),
+           "gq_prepare_hinv_static")
+    return U, dead, delta, status
 
 
 @dataclass
