@@ -29,6 +29,7 @@ gq_status ensure_device_setup() {
   if (g_init_done[dev]) return GQ_OK;
   if (factor_init_attributes() != cudaSuccess) return GQ_ERR_CUDA;
   if (quant_init_attributes() != cudaSuccess) return GQ_ERR_CUDA;
+  if (lazy_tc_init_attributes() != cudaSuccess) return GQ_ERR_CUDA;
   g_init_done[dev] = true;
   return GQ_OK;
 }

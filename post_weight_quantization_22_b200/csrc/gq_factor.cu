@@ -68,6 +68,19 @@ __global__ void build_m_kernel(const double* H, int64_t n, int reverse, const Ws
   M[i * n + j] = v;
 }
 
+// 1/p for p > 0: the hardware reciprocal estimate (rcp.approx.ftz.f64, about 2^-22 relative)
+// refined by two Newton-Raphson steps r <- r + r (1 - p r), each squaring the relative error,
+// to fp64 precision.  It replaces an IEEE division on the leaf's per-pivot critical path; the
+// result may differ from 1.0/p in the last bit, far inside the factor's tolerance.
+__device__ __forceinline__ double recip_newton(double p) {
+  double r;
+  asm("rcp.approx.ftz.f64 %0, %1;" : "=d"(r) : "d"(p));
+  double e = fma(-p, r, 1.0);
+  r = fma(r, e, r);
+  e = fma(-p, r, 1.0);
+  return fma(r, e, r);
+}
+
 // ---------------------------------------------------------------------------------------
 // Diagonal block (w <= 64): inverse of its Cholesky factor, in place, in one elimination pass.
 // Unnormalised elimination of [S | I] (S the block, symmetric, lower part used): at pivot c,
@@ -99,17 +112,26 @@ __global__ void __launch_bounds__(256) potrf_diag_kernel(double* M, int64_t n, i
     if (r > c) {
       double p = S[c * ld + c];
       if (!(p > 0.0)) p = 1.0;  // recorded below; keeps the arithmetic finite
-      const double f = S[r * ld + c] / p;
-      // fixed trip counts with predicates: all loads of a pivot step issue back to back
+      const double f = S[r * ld + c] * recip_newton(p);
+      // All loads of a pivot step first, then the updates, then the stores: the stores could
+      // alias later loads of the same array, so interleaving them would serialise every
+      // round trip through shared memory.
+      double cv[kNB / 4], rv[kNB / 4], av[kNB / 4], pv[kNB / 4];
 #pragma unroll
       for (int i = 0; i < kNB / 4; ++i) {
         const int q = c + 1 + part + 4 * i;
-        if (q <= r) S[r * ld + q] = fma(-f, S[q * ld + c], S[r * ld + q]);
+        const int j = part + 4 * i;
+        cv[i] = (q <= r) ? S[q * ld + c] : 0.0;
+        rv[i] = (q <= r) ? S[r * ld + q] : 0.0;
+        pv[i] = (j <= c) ? A[c * ld + j] : 0.0;
+        av[i] = (j <= c) ? A[r * ld + j] : 0.0;
       }
 #pragma unroll
       for (int i = 0; i < kNB / 4; ++i) {
+        const int q = c + 1 + part + 4 * i;
         const int j = part + 4 * i;
-        if (j <= c) A[r * ld + j] = fma(-f, A[c * ld + j], A[r * ld + j]);
+        if (q <= r) S[r * ld + q] = fma(-f, cv[i], rv[i]);
+        if (j <= c) A[r * ld + j] = fma(-f, pv[i], av[i]);
       }
     }
     __syncthreads();

@@ -1,6 +1,7 @@
 // Internal declarations shared by the libgq translation units (not part of the C ABI).
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 #include <stdint.h>
@@ -76,5 +77,17 @@ void count_launches(long k);
 // one-time per-device kernel attribute setup (dynamic shared memory above 48 KB)
 cudaError_t factor_init_attributes();
 cudaError_t quant_init_attributes();
+cudaError_t lazy_tc_init_attributes();
+
+// ---- lazy block update on tensor cores (gq_lazy_tc.cu) ----
+struct LazyTcMaps {
+  CUtensorMap ahi, alo, bhi, blo;
+};
+// E_hi / E_lo: rows x 128 fp32; U_hi / U_lo: n x n fp32 with leading dimension ldu (mult. of 4)
+cudaError_t lazy_tc_make_maps(LazyTcMaps* maps, const float* Ehi, const float* Elo, int64_t rows,
+                              const float* Uhi, const float* Ulo, int64_t n, int64_t ldu);
+// Wf[:, j1:] -= (E_hi + E_lo) (U_hi + U_lo)[j0:j0+128, j1:]  (3xTF32), rows < k_rows
+cudaError_t launch_lazy_tc(const LazyTcMaps& maps, float* Wf, int64_t n, int64_t k_rows,
+                           int64_t j0, int64_t j1, WsHeader* hdr, cudaStream_t s);
 
 }  // namespace gq

@@ -1,0 +1,197 @@
+// Lazy block update on the tensor cores: W[:, j1:] -= E U[j0:j0+128, j1:] in fp32 accuracy.
+//
+// GPTQ defers the trailing update of the columns after a 128-column block to one rank-128 GEMM
+// (the lazy batch); here it runs as tcgen05.mma kind::tf32 with the 3xTF32 split: each fp32
+// operand is carried as hi + lo (hi = tf32 rounding, lo = the fp32 remainder), and
+// acc += A_hi B_hi + A_hi B_lo + A_lo B_hi, accumulated in fp32 in tensor memory.  The column
+// loop writes E as E_hi / E_lo; U is split once per quantize call.
+//
+// CTA tile 128 (rows) x 128 (columns), K = 128 in 4 stages of 32 (3-deep ring), operands by
+// TMA (no multicast): A = E (K-major, rows of 32 fp32 = 128 B, 128-byte swizzle), B = U rows
+// j0.. (MN-major, 4 runs of 32 columns, 128-byte swizzle with 32-byte chunks: the layout the
+// tensor cores require for 32-bit MN-major operands).  Warp 0 lane 0 issues the loads, warp 1 lane 0 the MMAs, all four
+// warps read the accumulator (lane = row) and subtract it from the fp32 work matrix.
+#include "gq_internal.cuh"
+#include "gq_tc.cuh"
+
+#include <cudaTypedefs.h>
+#include <mutex>
+
+namespace gq {
+
+namespace {
+constexpr int kLBK = 32;                                  // K per stage
+constexpr int kLStages = 3;
+constexpr uint32_t kLTile = 128 * kLBK * 4;               // 16 KB per operand tile
+constexpr uint32_t kLStage = 4 * kLTile;                  // A_hi, A_lo, B_hi, B_lo
+constexpr size_t kLSmem = kLStages * kLStage + 1024 + 256;
+constexpr uint32_t kLIdesc = tc::idesc_f32acc(2, 2, 0, 1, 128, 128);  // tf32, A K-major, B MN-major
+}  // namespace
+
+__global__ void __launch_bounds__(128, 1)
+    lazy_tc_kernel(const __grid_constant__ CUtensorMap m_ahi, const __grid_constant__ CUtensorMap m_alo,
+                   const __grid_constant__ CUtensorMap m_bhi, const __grid_constant__ CUtensorMap m_blo,
+                   float* Wf, int64_t n, int64_t k_rows, int j0, int j1, WsHeader* hdr) {
+  extern __shared__ uint8_t lz_smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(lz_smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(base + kLStages * kLStage);
+  uint64_t* empty = full + kLStages;
+  uint64_t* accum = empty + kLStages;
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(accum + 1);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int tile_n = blockIdx.x, tile_m = blockIdx.y;
+
+  if (tid == 0) {
+    for (int s = 0; s < kLStages; ++s) { tc::mbar_init(&full[s], 1); tc::mbar_init(&empty[s], 1); }
+    tc::mbar_init(accum, 1);
+    tc::fence_barrier_init();
+    tc::prefetch_tmap(&m_ahi); tc::prefetch_tmap(&m_alo);
+    tc::prefetch_tmap(&m_bhi); tc::prefetch_tmap(&m_blo);
+  }
+  if (warp == 1) tc::tmem_alloc(tslot, 128);
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = *tslot;
+  constexpr int NK = 128 / kLBK;
+
+  if (warp == 0 && lane == 0) {
+    // producer
+    for (int kc = 0; kc < NK; ++kc) {
+      const int s = kc % kLStages;
+      if (kc >= kLStages && !tc::mbar_wait(&empty[s], ((kc / kLStages) - 1) & 1)) {
+        record_status(hdr, GQ_ERR_TIMEOUT);
+        break;
+      }
+      uint8_t* st = base + s * kLStage;
+      tc::mbar_arrive_expect_tx(&full[s], kLStage);
+      tc::tma_load_2d(st, &m_ahi, &full[s], kc * kLBK, tile_m * 128);
+      tc::tma_load_2d(st + kLTile, &m_alo, &full[s], kc * kLBK, tile_m * 128);
+#pragma unroll
+      for (int g = 0; g < 4; ++g) {
+        const int x = j1 + tile_n * 128 + g * 32, y = j0 + kc * kLBK;
+        tc::tma_load_2d(st + 2 * kLTile + g * 4096, &m_bhi, &full[s], x, y);
+        tc::tma_load_2d(st + 3 * kLTile + g * 4096, &m_blo, &full[s], x, y);
+      }
+    }
+  } else if (warp == 1 && lane == 0) {
+    // MMA issuer
+    for (int kc = 0; kc < NK; ++kc) {
+      const int s = kc % kLStages;
+      if (!tc::mbar_wait(&full[s], (kc / kLStages) & 1)) {
+        record_status(hdr, GQ_ERR_TIMEOUT);
+        break;
+      }
+      tc::fence_after_sync();
+      const uint32_t a_hi = tc::smem_u32(base + s * kLStage);
+      const uint32_t a_lo = a_hi + kLTile, b_hi = a_hi + 2 * kLTile, b_lo = a_hi + 3 * kLTile;
+#pragma unroll
+      for (int k = 0; k < kLBK / 8; ++k) {
+        const uint64_t dah = tc::sdesc(a_hi + k * 32, 16, 1024, tc::kLayoutSW128);
+        const uint64_t dal = tc::sdesc(a_lo + k * 32, 16, 1024, tc::kLayoutSW128);
+        const uint64_t dbh = tc::sdesc(b_hi + k * 1024, 4096, 512, tc::kLayoutSW128Base32B);
+        const uint64_t dbl = tc::sdesc(b_lo + k * 1024, 4096, 512, tc::kLayoutSW128Base32B);
+        tc::mma_tf32(tmem, dah, dbh, kLIdesc, (kc | k) != 0);
+        tc::mma_tf32(tmem, dah, dbl, kLIdesc, 1);
+        tc::mma_tf32(tmem, dal, dbh, kLIdesc, 1);
+      }
+      tc::mma_commit(&empty[s]);
+    }
+    tc::mma_commit(accum);
+  }
+  __syncwarp();
+
+  // epilogue: TMEM lane = tile row, 4 x 32 columns
+  bool ok = tc::mbar_wait(accum, 0);
+  if (!ok && lane == 0) record_status(hdr, GQ_ERR_TIMEOUT);
+  tc::fence_after_sync();
+  const int64_t row = (int64_t)tile_m * 128 + warp * 32 + lane;
+  if (ok) {
+#pragma unroll 1
+    for (int cc = 0; cc < 4; ++cc) {
+      float v[32];
+      tc::tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + cc * 32, v);
+      const int64_t col0 = (int64_t)j1 + tile_n * 128 + cc * 32;
+      if (row < k_rows && col0 < n) {
+        float* dst = Wf + row * n + col0;
+        if (col0 + 32 <= n && ((reinterpret_cast<uintptr_t>(dst) & 15) == 0)) {
+#pragma unroll
+          for (int i = 0; i < 32; i += 4) {
+            float4 w = *reinterpret_cast<float4*>(dst + i);
+            w.x -= v[i]; w.y -= v[i + 1]; w.z -= v[i + 2]; w.w -= v[i + 3];
+            *reinterpret_cast<float4*>(dst + i) = w;
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            if (col0 + i < n) dst[i] -= v[i];
+        }
+      }
+    }
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  if (warp == 1) tc::tmem_dealloc(tmem, 128);
+}
+
+// ---- host side ----
+namespace {
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::mutex g_encode_mu;
+
+cudaError_t get_encode() {
+  std::lock_guard<std::mutex> lk(g_encode_mu);
+  if (g_encode) return cudaSuccess;
+  void* fn = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q);
+  if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || !fn) return cudaErrorNotSupported;
+  g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  return cudaSuccess;
+}
+
+// fp32 row-major matrix (rows x cols, leading dimension ld elements) as a 2-D tensor map with a
+// box of 32 columns x box_rows rows, zero fill outside; swizzle as the operand's layout needs.
+cudaError_t encode_f32(CUtensorMap* map, const float* p, int64_t rows, int64_t cols, int64_t ld,
+                       uint32_t box_rows, CUtensorMapSwizzle swz) {
+  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)ld * sizeof(float)};
+  cuuint32_t box[2] = {32, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(p), dims,
+                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+}  // namespace
+
+cudaError_t lazy_tc_init_attributes() {
+  return cudaFuncSetAttribute(lazy_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              (int)kLSmem);
+}
+
+cudaError_t lazy_tc_make_maps(LazyTcMaps* maps, const float* Ehi, const float* Elo, int64_t rows,
+                              const float* Uhi, const float* Ulo, int64_t n, int64_t ldu) {
+  cudaError_t e = get_encode();
+  if (e != cudaSuccess) return e;
+  const CUtensorMapSwizzle ka = CU_TENSOR_MAP_SWIZZLE_128B;            // K-major A
+  const CUtensorMapSwizzle mb = CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B;    // MN-major 32-bit B
+  if ((e = encode_f32(&maps->ahi, Ehi, rows, kBlock, kBlock, 128, ka))) return e;
+  if ((e = encode_f32(&maps->alo, Elo, rows, kBlock, kBlock, 128, ka))) return e;
+  if ((e = encode_f32(&maps->bhi, Uhi, n, n, ldu, kLBK, mb))) return e;
+  return encode_f32(&maps->blo, Ulo, n, n, ldu, kLBK, mb);
+}
+
+cudaError_t launch_lazy_tc(const LazyTcMaps& maps, float* Wf, int64_t n, int64_t k_rows,
+                           int64_t j0, int64_t j1, WsHeader* hdr, cudaStream_t s) {
+  if (j1 >= n || k_rows <= 0) return cudaSuccess;
+  dim3 grid((unsigned)((n - j1 + 127) / 128), (unsigned)((k_rows + 127) / 128));
+  lazy_tc_kernel<<<grid, 128, kLSmem, s>>>(maps.ahi, maps.alo, maps.bhi, maps.blo, Wf, n, k_rows,
+                                           (int)j0, (int)j1, hdr);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+}  // namespace gq

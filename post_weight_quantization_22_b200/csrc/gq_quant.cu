@@ -9,8 +9,8 @@
 // processing order (columns reversed for the last-to-first variant, dead columns zeroed).  Per
 // 128-column block: `colloop` runs the sequential column recursion for 32 rows per CTA (4
 // lanes per row, each lane owning 32 of the block's columns in 4-wide chunks), keeping the
-// block's part of U in shared memory; `lazy_update` then applies W[:, j+128:] -= E U[j:j+128,
-// j+128:] to the rest of the work matrix.
+// block's part of U in shared memory; the tensor-core lazy update (gq_lazy_tc.cu) then applies
+// W[:, j+128:] -= E U[j:j+128, j+128:] to the rest of the work matrix.
 #include "gq_internal.cuh"
 
 #include <algorithm>
@@ -25,7 +25,11 @@ constexpr int kRowsPerCta = 4 * 32 / kP;  // 32 rows per 128-thread CTA
 struct QLayout {
   WsHeader* hdr;
   float* Wf;        // k x n work matrix (compact rows)
-  float* E;         // k x 128 scaled errors of the current block
+  float* Ehi;       // k x 128 scaled errors of the current block, tf32 part
+  float* Elo;       // k x 128 fp32 remainder (E = Ehi + Elo)
+  float* Uhi;       // n x ldu tf32 part of U (columns >= n zero)
+  float* Ulo;       // n x ldu fp32 remainder
+  int64_t ldu;
   uint8_t* codes8;  // m x ldc8 codes in processing order
   int64_t ldc8;
   double* row_s;    // per-row step (group_size 0)
@@ -45,7 +49,11 @@ static QLayout q_layout(void* ws, int64_t m, int64_t n) {
   QLayout L;
   L.hdr = c.take<WsHeader>(1);
   L.Wf = c.take<float>((size_t)m * n);
-  L.E = c.take<float>((size_t)m * kBlock);
+  L.Ehi = c.take<float>((size_t)m * kBlock);
+  L.Elo = c.take<float>((size_t)m * kBlock);
+  L.ldu = (n + 31) / 32 * 32;
+  L.Uhi = c.take<float>((size_t)n * L.ldu);
+  L.Ulo = c.take<float>((size_t)n * L.ldu);
   L.ldc8 = (n + 15) / 16 * 16;
   L.codes8 = c.take<uint8_t>((size_t)m * L.ldc8);
   L.row_s = c.take<double>(m);
@@ -126,6 +134,26 @@ __global__ void q_row_grid_kernel(const float* Wf, int64_t n, int64_t k_rows, co
   }
 }
 
+// tf32 rounding (to nearest, ties away) of an fp32 value, kept in an fp32 container
+__device__ __forceinline__ float tf32_rna(float x) {
+  uint32_t r;
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+  return __uint_as_float(r);
+}
+
+// U -> (Uhi, Ulo) with Uhi = tf32(U), Ulo = U - Uhi; columns n..ldu-1 zero
+__global__ void split_u_kernel(const float* U, int64_t n, int64_t ldu, float* Uhi, float* Ulo) {
+  const int64_t total = n * ldu;
+  for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < total;
+       e += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t i = e / ldu, j = e % ldu;
+    const float u = j < n ? U[i * n + j] : 0.f;
+    const float h = tf32_rna(u);
+    Uhi[e] = h;
+    Ulo[e] = u - h;
+  }
+}
+
 // ------------------------------------------------------------------------------------------
 // the column loop of one 128-column block
 // ------------------------------------------------------------------------------------------
@@ -139,7 +167,8 @@ struct ColArgs {
   const float* U;
   int bits;
   int clip;
-  float* E;
+  float* Ehi;
+  float* Elo;
   uint8_t* codes8;
   int64_t ldc8;
   float* scales;
@@ -218,7 +247,8 @@ __global__ void __launch_bounds__(128, 1) colloop_kernel(ColArgs a) {
   int ovf = 0;
   const unsigned full = 0xffffffffu;
   const int gbase = lane & ~(kP - 1);
-  float* Erow = a.E + rr * kBlock;
+  float* Ehrow = a.Ehi + rr * kBlock;
+  float* Elrow = a.Elo + rr * kBlock;
   uint8_t* crow = a.codes8 + row * a.ldc8 + j0;
 
   for (int seg = 0; seg < kBlock / 16; ++seg) {
@@ -297,7 +327,11 @@ __global__ void __launch_bounds__(128, 1) colloop_kernel(ColArgs a) {
     // this segment's errors and codes
     if (active) {
       const int k = 16 * seg + 4 * t;
-      *reinterpret_cast<float4*>(Erow + k) = make_float4(eo[0], eo[1], eo[2], eo[3]);
+      float4 hi, lo;
+      hi.x = tf32_rna(eo[0]); hi.y = tf32_rna(eo[1]); hi.z = tf32_rna(eo[2]); hi.w = tf32_rna(eo[3]);
+      lo.x = eo[0] - hi.x; lo.y = eo[1] - hi.y; lo.z = eo[2] - hi.z; lo.w = eo[3] - hi.w;
+      *reinterpret_cast<float4*>(Ehrow + k) = hi;
+      *reinterpret_cast<float4*>(Elrow + k) = lo;
       if (k + 3 < bw) {
         *reinterpret_cast<uint32_t*>(crow + k) = cw;
       } else {
@@ -319,53 +353,6 @@ __global__ void __launch_bounds__(128, 1) colloop_kernel(ColArgs a) {
   if (t == 0) {
     if (j0 == 0) { a.row_e2[row] = e2; a.row_bnd[row] = bnd; a.overflow[row] = ovf_row; }
     else { a.row_e2[row] += e2; a.row_bnd[row] += bnd; a.overflow[row] |= ovf_row; }
-  }
-}
-
-// ------------------------------------------------------------------------------------------
-// lazy rank-<=128 update: Wf[:, j1:] -= E[:, :bw] U[j0:j0+bw, j1:]   (fp32 SIMT, v1)
-// ------------------------------------------------------------------------------------------
-__global__ void __launch_bounds__(256) lazy_update_kernel(float* Wf, int64_t n, int64_t k_rows,
-                                                          int64_t j0, int bw, int64_t j1,
-                                                          const float* E, const float* U) {
-  __shared__ float As[16][64 + 4];
-  __shared__ float Bs[16][64 + 4];
-  const int64_t r0 = (int64_t)blockIdx.y * 64, c0 = j1 + (int64_t)blockIdx.x * 64;
-  const int tid = threadIdx.x, tx = tid % 16, ty = tid / 16;
-  float acc[4][4] = {};
-  for (int k0 = 0; k0 < bw; k0 += 16) {
-#pragma unroll
-    for (int r = 0; r < 4; ++r) {
-      int e = tid + 256 * r;
-      int ii = e / 16, kk = e % 16;
-      int64_t gr = r0 + ii;
-      As[kk][ii] = (gr < k_rows && k0 + kk < bw) ? E[gr * kBlock + k0 + kk] : 0.f;
-      int kb = e / 64, jj = e % 64;
-      int64_t gc = c0 + jj;
-      Bs[kb][jj] = (gc < n && k0 + kb < bw) ? U[(j0 + k0 + kb) * n + gc] : 0.f;
-    }
-    __syncthreads();
-#pragma unroll
-    for (int kk = 0; kk < 16; ++kk) {
-      float av[4], bv[4];
-#pragma unroll
-      for (int q = 0; q < 4; ++q) { av[q] = As[kk][ty + 16 * q]; bv[q] = Bs[kk][tx + 16 * q]; }
-#pragma unroll
-      for (int p = 0; p < 4; ++p)
-#pragma unroll
-        for (int q = 0; q < 4; ++q) acc[p][q] = fmaf(av[p], bv[q], acc[p][q]);
-    }
-    __syncthreads();
-  }
-#pragma unroll
-  for (int p = 0; p < 4; ++p) {
-    int64_t gr = r0 + ty + 16 * p;
-    if (gr >= k_rows) continue;
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      int64_t gc = c0 + tx + 16 * q;
-      if (gc < n) Wf[gr * n + gc] -= acc[p][q];
-    }
   }
 }
 
@@ -512,6 +499,13 @@ gq_status run_quantize(const QuantArgs& a, cudaStream_t s) {
   q_reset_kernel<<<(unsigned)((m + 255) / 256), 256, 0, s>>>(m, L.alpha, L.overflow, a.loss);
   count_launches(1);
   Q_TRY(cudaGetLastError());
+  {
+    const int64_t total = n * L.ldu;
+    unsigned grid = (unsigned)std::min<int64_t>((total + 255) / 256, 148 * 32);
+    split_u_kernel<<<grid, 256, 0, s>>>(a.U, n, L.ldu, L.Uhi, L.Ulo);
+    count_launches(1);
+    Q_TRY(cudaGetLastError());
+  }
   int64_t k_rows = m;
   const int* rowlist = nullptr;
   const int nblocks = (int)((n + kBlock - 1) / kBlock);
@@ -538,23 +532,21 @@ gq_status run_quantize(const QuantArgs& a, cudaStream_t s) {
       count_launches(1);
       Q_TRY(cudaGetLastError());
     }
+    LazyTcMaps maps;
+    Q_TRY(lazy_tc_make_maps(&maps, L.Ehi, L.Elo, k_rows, L.Uhi, L.Ulo, n, L.ldu));
     for (int b = 0; b < nblocks; ++b) {
       const int64_t j0 = (int64_t)b * kBlock;
       const int bw = (int)std::min<int64_t>(kBlock, n - j0);
       ColArgs ca{};
       ca.Wf = L.Wf; ca.n = n; ca.k_rows = k_rows; ca.rowlist = rowlist; ca.j0 = j0; ca.bw = bw;
-      ca.U = a.U; ca.bits = cfg.bits; ca.clip = cfg.clip; ca.E = L.E; ca.codes8 = L.codes8;
+      ca.U = a.U; ca.bits = cfg.bits; ca.clip = cfg.clip; ca.Ehi = L.Ehi; ca.Elo = L.Elo;
+      ca.codes8 = L.codes8;
       ca.ldc8 = L.ldc8; ca.scales = a.scales; ca.zeros = a.zeros; ca.ngroups = ngroups;
       ca.row_s = L.row_s; ca.row_z = L.row_z; ca.row_e2 = L.row_e2; ca.row_bnd = L.row_bnd;
       ca.overflow = L.overflow;
       Q_TRY(colloop_dispatch(G, ca, s));
       const int64_t j1 = j0 + bw;
-      if (j1 < n) {
-        dim3 grid((unsigned)((n - j1 + 63) / 64), (unsigned)((k_rows + 63) / 64));
-        lazy_update_kernel<<<grid, 256, 0, s>>>(L.Wf, n, k_rows, j0, bw, j1, L.E, a.U);
-        count_launches(1);
-        Q_TRY(cudaGetLastError());
-      }
+      if (j1 < n) Q_TRY(launch_lazy_tc(maps, L.Wf, n, k_rows, j0, j1, L.hdr, s));
     }
     if (cfg.clip) break;
     // clip-free: collect rows whose codes left [0, 2^b - 1] and rerun them on a wider step
