@@ -82,70 +82,73 @@ __device__ __forceinline__ double recip_newton(double p) {
 }
 
 // ---------------------------------------------------------------------------------------
-// Diagonal block (w <= 64): inverse of its Cholesky factor, in place, in one elimination pass.
-// Unnormalised elimination of [S | I] (S the block, symmetric, lower part used): at pivot c,
-// rows r > c take S[r][s] -= f_r S[s][c] (s in (c, r]) and A[r][j] -= f_r A[c][j] (j <= c),
-// f_r = S[r][c] / S[c][c].  Then A = L_unit^-1, the pivots are D of S = L_unit D L_unit^T, and
-// L^-1 = D^-1/2 A.  One barrier per pivot; 4 threads per row.
+// Diagonal block (w <= 64): the inverse of its Cholesky factor, in place (lower part).
+// Unnormalised elimination of [S | I] (S the block, rows >= w padded with the identity): at
+// pivot c, rows r > c take S[r][q] -= f_r S[q][c] (q in (c, r]) and A[r][j] -= f_r A[c][j]
+// (j <= c), f_r = S[r][c] / S[c][c].  Then A = L_unit^-1, the pivots are D of
+// S = L_unit D L_unit^T, and L^-1 = D^-1/2 A.
+// 256 threads, 4 per row; thread (r, part) keeps S[r][4i+part] and A[r][4i+part] (i < 16) in
+// registers.  Per pivot only column c of S and row c of A travel, through double-buffered
+// shared memory, with one barrier; the pivot loop is unrolled so every register index is fixed.
 // ---------------------------------------------------------------------------------------
-__global__ void __launch_bounds__(256) potrf_diag_kernel(double* M, int64_t n, int64_t c0, int w,
-                                                         WsHeader* hdr) {
-  extern __shared__ double sm[];
-  const int ld = kNB + 1;
-  double* S = sm;                 // [64][65] Schur complement (lower)
-  double* A = sm + kNB * ld;      // [64][65] eliminated identity (lower)
+__global__ void __launch_bounds__(256, 1) potrf_diag_kernel(double* M, int64_t n, int64_t c0,
+                                                            int w, WsHeader* hdr) {
+  __shared__ double colbuf[2][kNB];
+  __shared__ double rowbuf[2][kNB];
   const int tid = threadIdx.x;
-  for (int e = tid; e < kNB * kNB; e += 256) {
-    int i = e / kNB, j = e % kNB;
+  const int r = tid >> 2, part = tid & 3;
+  double sv[16], av[16];
+  // all loads of the block issue before any use
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const int q = 4 * i + part;
     double v = 0.0;
-    if (i < w && j < w) {
-      if (j <= i) v = M[(c0 + i) * n + c0 + j];
-    } else if (i == j) {
+    if (r < w && q < w) {
+      if (q <= r) v = M[(c0 + r) * n + c0 + q];
+    } else if (q == r) {
       v = 1.0;
     }
-    S[i * ld + j] = v;
-    A[i * ld + j] = (i == j) ? 1.0 : 0.0;
+    sv[i] = v;
+    av[i] = (q == r) ? 1.0 : 0.0;
   }
-  __syncthreads();
-  const int r = tid >> 2, part = tid & 3;
+#pragma unroll
   for (int c = 0; c < kNB - 1; ++c) {
-    if (r > c) {
-      double p = S[c * ld + c];
-      if (!(p > 0.0)) p = 1.0;  // recorded below; keeps the arithmetic finite
-      const double f = S[r * ld + c] * recip_newton(p);
-      // All loads of a pivot step first, then the updates, then the stores: the stores could
-      // alias later loads of the same array, so interleaving them would serialise every
-      // round trip through shared memory.
-      double cv[kNB / 4], rv[kNB / 4], av[kNB / 4], pv[kNB / 4];
+    const int buf = c & 1;
+    if (part == (c & 3)) colbuf[buf][r] = sv[c >> 2];  // S[r][c]
+    if (r == c) {
 #pragma unroll
-      for (int i = 0; i < kNB / 4; ++i) {
-        const int q = c + 1 + part + 4 * i;
-        const int j = part + 4 * i;
-        cv[i] = (q <= r) ? S[q * ld + c] : 0.0;
-        rv[i] = (q <= r) ? S[r * ld + q] : 0.0;
-        pv[i] = (j <= c) ? A[c * ld + j] : 0.0;
-        av[i] = (j <= c) ? A[r * ld + j] : 0.0;
-      }
-#pragma unroll
-      for (int i = 0; i < kNB / 4; ++i) {
-        const int q = c + 1 + part + 4 * i;
-        const int j = part + 4 * i;
-        if (q <= r) S[r * ld + q] = fma(-f, cv[i], rv[i]);
-        if (j <= c) A[r * ld + j] = fma(-f, pv[i], av[i]);
-      }
+      for (int i = 0; i < 16; ++i)
+        if (4 * i + part <= c) rowbuf[buf][4 * i + part] = av[i];  // A[c][j]
     }
     __syncthreads();
-  }
-  // L^-1[r][j] = A[r][j] / sqrt(D_r)
-  for (int e = tid; e < kNB * kNB; e += 256) {
-    int i = e / kNB, j = e % kNB;
-    if (i < w && j <= i) {
-      double p = S[i * ld + i];
-      if (!(p > 0.0)) {
-        if (j == 0) record_status(hdr, GQ_ERR_NOT_PD);
-        p = 1.0;
+    if (r > c) {
+      double p = colbuf[buf][c];
+      if (!(p > 0.0)) p = 1.0;  // reported below from the final pivots
+      const double f = colbuf[buf][r] * recip_newton(p);
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const int q = 4 * i + part;
+        if (q > c && q <= r) sv[i] = fma(-f, colbuf[buf][q], sv[i]);
+        if (q <= c) av[i] = fma(-f, rowbuf[buf][q], av[i]);
       }
-      M[(c0 + i) * n + c0 + j] = A[i * ld + j] / sqrt(p);
+    }
+  }
+  // pivot D_r = S[r][r], held by part r % 4
+  double d = 0.0;
+#pragma unroll
+  for (int i = 0; i < 16; ++i)
+    if (4 * i + part == r) d = sv[i];
+  d = __shfl_sync(0xffffffffu, d, (tid & 31 & ~3) | (r & 3));
+  if (!(d > 0.0)) {
+    if (r < w && part == 0) record_status(hdr, GQ_ERR_NOT_PD);
+    d = 1.0;
+  }
+  const double rs = 1.0 / sqrt(d);
+  if (r < w) {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const int q = 4 * i + part;
+      if (q <= r) M[(c0 + r) * n + c0 + q] = av[i] * rs;
     }
   }
 }
@@ -192,10 +195,7 @@ static PrepLayout prep_layout(void* ws, int64_t n) {
 
 size_t prepare_ws_bytes(int64_t n) { return prep_layout(nullptr, n).bytes; }
 
-cudaError_t factor_init_attributes() {
-  return cudaFuncSetAttribute(potrf_diag_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              2 * kNB * (kNB + 1) * (int)sizeof(double));
-}
+cudaError_t factor_init_attributes() { return cudaSuccess; }
 
 #define GQ_TRY(x)                               \
   do {                                          \
@@ -220,11 +220,10 @@ cudaError_t launch_prepare(const double* H, int64_t n, double damp, int reverse,
   // is replaced by the inverse of its factor; the panel below becomes L21 = A21 L11^-T; the
   // trailing matrix takes A22 -= L21 L21^T.
   const int64_t nb = (n + kNB - 1) / kNB;
-  const size_t psmem = 2 * kNB * (kNB + 1) * sizeof(double);
   for (int64_t k = 0; k < nb; ++k) {
     const int64_t c0 = k * kNB;
     const int w = (int)std::min<int64_t>(kNB, n - c0);
-    potrf_diag_kernel<<<1, 256, psmem, s>>>(L.M, n, c0, w, L.hdr);
+    potrf_diag_kernel<<<1, 256, 0, s>>>(L.M, n, c0, w, L.hdr);
     count_launches(1);
     GQ_TRY(cudaGetLastError());
     const int64_t rem = n - c0 - w;

@@ -134,6 +134,15 @@ __global__ void q_row_grid_kernel(const float* Wf, int64_t n, int64_t k_rows, co
   }
 }
 
+// Round to nearest integer, ties to even, for |x| < 2^51: adding and subtracting 1.5 * 2^52
+// leaves no fraction bits, so the fp64 addition itself rounds x (in the default
+// round-to-nearest-even mode).  Two fixed-latency adds instead of a conversion instruction on
+// the column loop's critical path.  The grid values here are far below 2^51.
+__device__ __forceinline__ double rint_small(double x) {
+  const double magic = 6755399441055744.0;  // 1.5 * 2^52
+  return __dsub_rn(__dadd_rn(x, magic), magic);
+}
+
 // tf32 rounding (to nearest, ties away) of an fp32 value, kept in an fp32 container
 __device__ __forceinline__ float tf32_rna(float x) {
   uint32_t r;
@@ -289,7 +298,7 @@ __global__ void __launch_bounds__(128, 1) colloop_kernel(ColArgs a) {
         const double sd = s * id;
         const double x = __shfl_sync(full, v[slot], gbase + owner);
         const double xi = x * id;
-        double c = rint(x * inv_s);
+        double c = rint_small(x * inv_s);
         if (a.clip) {
           c = fmin(fmax(c, cmin), cmax);
         } else if (c < cmin || c > cmax) {
