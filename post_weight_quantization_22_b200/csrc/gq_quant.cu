@@ -12,6 +12,7 @@
 // block's part of U in shared memory; the tensor-core lazy update (gq_lazy_tc.cu) then applies
 // W[:, j+128:] -= E U[j:j+128, j+128:] to the rest of the work matrix.
 #include "gq_internal.cuh"
+#include "gq_tc.cuh"
 
 #include <algorithm>
 #include <math.h>
@@ -21,6 +22,10 @@ namespace gq {
 constexpr int kP = 4;                     // lanes per row in the column loop
 constexpr int kVPL = kBlock / kP;          // values per lane (32)
 constexpr int kRowsPerCta = 4 * 32 / kP;  // 32 rows per 128-thread CTA
+// Per-block prepared U for the column loop (see ublk_kernel): 128 x 128 doubles + 2 x 128.
+constexpr int64_t kUBlkDoubles = (int64_t)kBlock * kBlock + 2 * kBlock;
+constexpr uint32_t kUBlkBytes = (uint32_t)(kUBlkDoubles * sizeof(double));
+constexpr uint32_t kBulkChunk = 32768;
 
 struct QLayout {
   WsHeader* hdr;
@@ -30,6 +35,7 @@ struct QLayout {
   float* Uhi;       // n x ldu tf32 part of U (columns >= n zero)
   float* Ulo;       // n x ldu fp32 remainder
   int64_t ldu;
+  double* Ublk;     // per-block prepared U for the column loop
   uint8_t* codes8;  // m x ldc8 codes in processing order
   int64_t ldc8;
   double* row_s;    // per-row step (group_size 0)
@@ -54,6 +60,7 @@ static QLayout q_layout(void* ws, int64_t m, int64_t n) {
   L.ldu = (n + 31) / 32 * 32;
   L.Uhi = c.take<float>((size_t)n * L.ldu);
   L.Ulo = c.take<float>((size_t)n * L.ldu);
+  L.Ublk = c.take<double>((size_t)((n + kBlock - 1) / kBlock) * kUBlkDoubles);
   L.ldc8 = (n + 15) / 16 * 16;
   L.codes8 = c.take<uint8_t>((size_t)m * L.ldc8);
   L.row_s = c.take<double>(m);
@@ -163,10 +170,35 @@ __global__ void split_u_kernel(const float* U, int64_t n, int64_t ldu, float* Uh
   }
 }
 
+// Per-block prepared U, built once per call: the block's 128 x 128 part of U in fp64 with the
+// strict lower triangle and the columns past the block's width zeroed, then 1/U_jj and
+// 1/U_jj^2 (1 past the width).  The column loop copies it into shared memory in one go.
+
+__global__ void ublk_kernel(const float* U, int64_t n, double* Ublk) {
+  const int64_t b = blockIdx.y;
+  const int64_t j0 = b * kBlock;
+  const int bw = (int)((n - j0) < kBlock ? (n - j0) : kBlock);
+  double* dst = Ublk + b * kUBlkDoubles;
+  for (int e = blockIdx.x * blockDim.x + threadIdx.x; e < kBlock * kBlock + kBlock;
+       e += gridDim.x * blockDim.x) {
+    if (e < kBlock * kBlock) {
+      const int jj = e / kBlock, kk = e % kBlock;
+      dst[e] = (jj < bw && kk >= jj && kk < bw) ? (double)U[(j0 + jj) * n + j0 + kk] : 0.0;
+    } else {
+      const int jj = e - kBlock * kBlock;
+      const double d = jj < bw ? (double)U[(j0 + jj) * n + j0 + jj] : 1.0;
+      dst[kBlock * kBlock + jj] = 1.0 / d;
+      dst[kBlock * kBlock + kBlock + jj] = 1.0 / (d * d);
+    }
+  }
+}
+
 // ------------------------------------------------------------------------------------------
 // the column loop of one 128-column block
 // ------------------------------------------------------------------------------------------
 struct ColArgs {
+  const double* Ublk;  // per-block prepared U (kUBlkDoubles each)
+  WsHeader* hdr;
   const float* Wf;
   int64_t n;
   int64_t k_rows;
@@ -203,29 +235,25 @@ struct ColArgs {
 template <int G>
 __global__ void __launch_bounds__(128, 1) colloop_kernel(ColArgs a) {
   extern __shared__ __align__(16) double q_smem[];
-  double* Us = q_smem;                       // [128][128]
+  double* Us = q_smem;                       // [128][128] this block's part of U (fp64, masked)
   double* invd = q_smem + kBlock * kBlock;   // [128]  1/U_jj
   double* invd2 = invd + kBlock;             // [128]  1/U_jj^2
+  uint64_t* bar = reinterpret_cast<uint64_t*>(invd2 + kBlock);
   const int tid = threadIdx.x;
   const int bw = a.bw;
   const int64_t n = a.n, j0 = a.j0;
-  for (int e = tid * 2; e < kBlock * kBlock; e += 128 * 2) {
-    int jj = e / kBlock, kk = e % kBlock;
-    double2 v = make_double2(0.0, 0.0);
-    if (jj < bw) {
-      const float* src = a.U + (j0 + jj) * n + j0 + kk;
-      if (kk >= jj && kk < bw) v.x = (double)src[0];
-      if (kk + 1 >= jj && kk + 1 < bw) v.y = (double)src[1];
+  // the prepared block (kUBlkBytes) arrives by bulk async copies while the rows load below
+  if (tid == 0) {
+    tc::mbar_init(bar, 1);
+    tc::fence_barrier_init();
+    tc::mbar_arrive_expect_tx(bar, (uint32_t)kUBlkBytes);
+    const char* src = reinterpret_cast<const char*>(a.Ublk + (j0 / kBlock) * kUBlkDoubles);
+    char* dst = reinterpret_cast<char*>(q_smem);
+    for (uint32_t off = 0; off < kUBlkBytes; off += kBulkChunk) {
+      const uint32_t len = kUBlkBytes - off < kBulkChunk ? kUBlkBytes - off : kBulkChunk;
+      tc::bulk_copy_g2s(dst + off, src + off, len, bar);
     }
-    *reinterpret_cast<double2*>(&Us[e]) = v;
   }
-  if (tid < kBlock) {
-    double d = (tid < bw) ? (double)a.U[(j0 + tid) * n + j0 + tid] : 1.0;
-    invd[tid] = 1.0 / d;
-    invd2[tid] = 1.0 / (d * d);
-  }
-  __syncthreads();
-
   const int lane = tid & 31, warp = tid >> 5;
   const int t = lane % kP;
   const int64_t rr = (int64_t)blockIdx.x * kRowsPerCta + warp * (32 / kP) + lane / kP;
@@ -249,6 +277,11 @@ __global__ void __launch_bounds__(128, 1) colloop_kernel(ColArgs a) {
       }
     }
     v[4 * c + 0] = x.x; v[4 * c + 1] = x.y; v[4 * c + 2] = x.z; v[4 * c + 3] = x.w;
+  }
+  __syncthreads();  // the barrier's initialisation is visible to every waiting thread
+  if (!tc::mbar_wait(bar, 0)) {
+    if (tid == 0) record_status(a.hdr, GQ_ERR_TIMEOUT);
+    return;  // nothing was computed; the bulk copy has been waited for the full bound
   }
   double s = 1.0, inv_s = 1.0, z = 0.0;
   if (G == 0 && active) { s = a.row_s[row]; z = a.row_z[row]; inv_s = 1.0 / s; }
@@ -466,7 +499,7 @@ __global__ void q_ladder_kernel(int64_t m, int* overflow, float* alpha, float la
     if (_e != cudaSuccess) return GQ_ERR_CUDA;      \
   } while (0)
 
-constexpr size_t kColSmem = (size_t)(kBlock * kBlock + 2 * kBlock) * sizeof(double);
+constexpr size_t kColSmem = (size_t)kUBlkBytes + 16;  // + the mbarrier
 
 cudaError_t quant_init_attributes() {
   const int smem = (int)kColSmem;
@@ -514,6 +547,10 @@ gq_status run_quantize(const QuantArgs& a, cudaStream_t s) {
     split_u_kernel<<<grid, 256, 0, s>>>(a.U, n, L.ldu, L.Uhi, L.Ulo);
     count_launches(1);
     Q_TRY(cudaGetLastError());
+    dim3 g2(16, (unsigned)((n + kBlock - 1) / kBlock));
+    ublk_kernel<<<g2, 256, 0, s>>>(a.U, n, L.Ublk);
+    count_launches(1);
+    Q_TRY(cudaGetLastError());
   }
   int64_t k_rows = m;
   const int* rowlist = nullptr;
@@ -547,6 +584,7 @@ gq_status run_quantize(const QuantArgs& a, cudaStream_t s) {
       const int64_t j0 = (int64_t)b * kBlock;
       const int bw = (int)std::min<int64_t>(kBlock, n - j0);
       ColArgs ca{};
+      ca.Ublk = L.Ublk; ca.hdr = L.hdr;
       ca.Wf = L.Wf; ca.n = n; ca.k_rows = k_rows; ca.rowlist = rowlist; ca.j0 = j0; ca.bw = bw;
       ca.U = a.U; ca.bits = cfg.bits; ca.clip = cfg.clip; ca.Ehi = L.Ehi; ca.Elo = L.Elo;
       ca.codes8 = L.codes8;
