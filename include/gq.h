@@ -70,22 +70,30 @@ unsigned long long gq_kernel_launches(void);
 /* Human-readable text of a status code (static storage). */
 const char* gq_status_string(gq_status s);
 
+/* Workspace bytes gq_hessian_accumulate needs for T tokens of width n. */
+size_t gq_hessian_workspace_size(int64_t T, int64_t n);
+
 /*
- * H += 2 X^T X  ("The Geometry of LLM Quantization", section 2.1: the lattice basis comes from
- * the calibration inputs and the CVP's Gram matrix is X^T X).
+ * H = 2 X^T X, or H += 2 X^T X  ("The Geometry of LLM Quantization", section 2.1: the lattice
+ * basis comes from the calibration inputs and the CVP's Gram matrix is X^T X).
  *
- *   d_H     n x n, fp64, device, read-modify-write; the caller zeroes it before the first
- *           chunk and may call again with further token chunks (streaming accumulation).
- *           Both triangles are written (H stays exactly symmetric).
+ *   d_H        n x n, fp64, device.  accumulate = 0 overwrites it with 2 X^T X; accumulate = 1
+ *              adds 2 X^T X (streaming over token chunks).  Both triangles are written (H stays
+ *              exactly symmetric).
  *   d_X     T x n, row-major (tokens x features), dtype x_dtype (bf16 or fp32), device.
- *   T, n    T >= 0 (T = 0 is a no-op), 1 <= n <= 65536.
+ *   T, n    T >= 0 (T = 0 is a no-op), 1 <= n <= 32768.
+ *   d_ws    workspace of at least gq_hessian_workspace_size(T, n) bytes (256-byte aligned).
  *
- * Precision: every product of two inputs is formed exactly and the token sums are kept to
- * fp64 accuracy; H is fp64 because the column loop's codes depend on H to about 1e-9
- * relative for the ill-conditioned Hessians of LLM layers.
+ * Precision: the products are formed exactly (each value as four 7-bit digits against a
+ * power-of-two scale per input column, int8 tensor-core products with int32 sums) and
+ * combined in fp64; the only error besides fp64 rounding is the rounding of entries smaller
+ * than 2^-21 of their column's largest, at 2^-29 of that largest.  H is fp64 because the
+ * column loop's codes depend on H to about 1e-9 relative for the ill-conditioned Hessians of
+ * LLM layers.
  */
 gq_status gq_hessian_accumulate(double* d_H, const void* d_X, gq_dtype x_dtype, int64_t T,
-                                int64_t n, gq_stream_t stream);
+                                int64_t n, int accumulate, void* d_ws, size_t ws_bytes,
+                                gq_stream_t stream);
 
 /* Workspace bytes gq_prepare_hinv needs for width n (256-byte aligned base required). */
 size_t gq_prepare_workspace_size(int64_t n);
@@ -100,7 +108,7 @@ size_t gq_prepare_workspace_size(int64_t n);
  * from the last pivot) and U = R^-1, in fp64; U is stored rounded to fp32.
  *
  *   d_H        n x n fp64 (from gq_hessian_accumulate), device, read only.
- *   n          1 <= n <= 65536.
+ *   n          1 <= n <= 32768.
  *   damp       >= 0 (0.01 in the usual setting).
  *   reverse    0 or 1, as above; pass the same value to gq_quantize_layer.
  *   d_U        n x n fp32, device, written in full (strict lower triangle set to 0).
@@ -166,7 +174,7 @@ size_t gq_quantize_workspace_size(int64_t m, int64_t n, const gq_quant_cfg* cfg)
  *             (W0 = W with dead columns zeroed), [1] tr(D H_d D^T) = sum of e^2,
  *             [2] Theorem 5 bound sum_r sum_j s_rj^2 / (4 U_jj^2) (a guarantee for clip = 0).
  *   d_ws      workspace of at least gq_quantize_workspace_size(m, n, cfg) bytes.
- * Limits: 1 <= m <= 2^24, 1 <= n <= 65536, 2 <= bits <= 8; reverse = 1 needs group_size 0.
+ * Limits: 1 <= m <= 2^24, 1 <= n <= 32768, 2 <= bits <= 8; reverse = 1 needs group_size 0.
  * Device-detected error: GQ_ERR_NO_FIT.
  */
 gq_status gq_quantize_layer(const void* d_W, gq_dtype w_dtype, int64_t m, int64_t n,

@@ -30,6 +30,7 @@ gq_status ensure_device_setup() {
   if (factor_init_attributes() != cudaSuccess) return GQ_ERR_CUDA;
   if (quant_init_attributes() != cudaSuccess) return GQ_ERR_CUDA;
   if (lazy_tc_init_attributes() != cudaSuccess) return GQ_ERR_CUDA;
+  if (hessian_init_attributes() != cudaSuccess) return GQ_ERR_CUDA;
   g_init_done[dev] = true;
   return GQ_OK;
 }
@@ -131,16 +132,29 @@ const char* gq_status_string(gq_status s) {
   return "unknown status";
 }
 
+size_t gq_hessian_workspace_size(int64_t T, int64_t n) {
+  if (T < 0 || n < 1 || n > kMaxN || T > (int64_t(1) << 31) - 1) return 0;
+  return hessian_ws_bytes(T, n);
+}
+
 gq_status gq_hessian_accumulate(double* d_H, const void* d_X, gq_dtype x_dtype, int64_t T,
-                                int64_t n, gq_stream_t stream) {
+                                int64_t n, int accumulate, void* d_ws, size_t ws_bytes,
+                                gq_stream_t stream) {
   if (T < 0 || n < 1 || n > kMaxN || T > (int64_t(1) << 31) - 1) return GQ_ERR_INVALID_ARG;
   if (x_dtype != GQ_BF16 && x_dtype != GQ_FP32) return GQ_ERR_INVALID_ARG;
-  if (!d_H || (T > 0 && !d_X)) return GQ_ERR_INVALID_ARG;
-  if (T == 0) return GQ_OK;
+  if (!d_H || (T > 0 && !d_X) || !d_ws) return GQ_ERR_INVALID_ARG;
+  if (accumulate != 0 && accumulate != 1) return GQ_ERR_INVALID_ARG;
+  if (!aligned256(d_ws) || ws_bytes < hessian_ws_bytes(T, n)) return GQ_ERR_WORKSPACE;
+  if (T == 0 && accumulate) return GQ_OK;
   gq_status st = ensure_device_setup();
   if (st != GQ_OK) return st;
-  cudaError_t e = launch_hessian(d_H, d_X, x_dtype, T, n, (cudaStream_t)stream);
-  return e == cudaSuccess ? GQ_OK : GQ_ERR_CUDA;
+  auto enqueue = [&](cudaStream_t s) {
+    return launch_hessian(d_H, d_X, x_dtype, T, n, accumulate, d_ws, s) == cudaSuccess
+               ? GQ_OK : GQ_ERR_CUDA;
+  };
+  return run_graphed({3, P(d_H), P(d_X), (uint64_t)x_dtype, (uint64_t)T, (uint64_t)n,
+                      (uint64_t)accumulate, P(d_ws)},
+                     (cudaStream_t)stream, enqueue);
 }
 
 size_t gq_prepare_workspace_size(int64_t n) {

@@ -42,8 +42,10 @@ __device__ __forceinline__ void record_status(WsHeader* h, int code) {
 }
 
 // ---- Hessian (H += 2 X^T X, fp64-accurate) ----
+size_t hessian_ws_bytes(int64_t T, int64_t n);
+cudaError_t hessian_init_attributes();
 cudaError_t launch_hessian(double* H, const void* X, gq_dtype xt, int64_t T, int64_t n,
-                           cudaStream_t s);
+                           int accumulate, void* ws, cudaStream_t s);
 
 // ---- factor preparation ----
 size_t prepare_ws_bytes(int64_t n);

@@ -96,6 +96,16 @@ __device__ __forceinline__ void mma_tf32(uint32_t tmem_d, uint64_t adesc, uint64
       "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
+// D[tmem] (+)= A[smem] * B[smem], kind::i8 (signed int8 operands, int32 accumulator).
+__device__ __forceinline__ void mma_i8(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc,
+                                       uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n.reg .pred p;\n"
+      "setp.ne.b32 p, %4, 0;\n"
+      "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n}\n" ::"r"(tmem_d),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
 // The mbarrier gets one arrival when every MMA this thread issued before has completed.
 __device__ __forceinline__ void mma_commit(uint64_t* bar) {
   asm volatile(
@@ -126,9 +136,10 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
 //   offset >> 4, 46-47 version (1), 61-63 layout type.
 // Layout 2, 128-byte swizzle (16-byte chunks, 8-row period): K-major operands, rows of
 //   128 bytes, 8-row groups SBO = 1024 apart (LBO unused, 16).
+// Layout 4, 64-byte swizzle: K-major operands with 64-byte rows, 8-row groups SBO = 512 apart.
 // Layout 1, 128-byte swizzle with 32-byte chunks (4-row period): the only layout for 32-bit
 //   MN-major operands; 128-byte runs along M/N with LBO between runs, 4-row K groups SBO apart.
-constexpr uint32_t kLayoutSW128 = 2, kLayoutSW128Base32B = 1;
+constexpr uint32_t kLayoutSW128 = 2, kLayoutSW128Base32B = 1, kLayoutSW64 = 4;
 __device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo, uint32_t sbo,
                                           uint32_t layout) {
   uint64_t d = 0;

@@ -43,7 +43,9 @@ def _load():
     lib.gq_status_string.restype = ctypes.c_char_p
     lib.gq_status_string.argtypes = [I]
     lib.gq_hessian_accumulate.restype = I
-    lib.gq_hessian_accumulate.argtypes = [P, P, I, I64, I64, P]
+    lib.gq_hessian_accumulate.argtypes = [P, P, I, I64, I64, I, P, SZ, P]
+    lib.gq_hessian_workspace_size.restype = SZ
+    lib.gq_hessian_workspace_size.argtypes = [I64, I64]
     lib.gq_prepare_workspace_size.restype = SZ
     lib.gq_prepare_workspace_size.argtypes = [I64]
     lib.gq_prepare_hinv.restype = I
@@ -61,7 +63,8 @@ def _load():
 
 
 LIB = _load()
-EXPORTED = ("gq_version", "gq_status_string", "gq_hessian_accumulate", "gq_prepare_workspace_size",
+EXPORTED = ("gq_version", "gq_status_string", "gq_hessian_accumulate", "gq_hessian_workspace_size",
+            "gq_prepare_workspace_size",
             "gq_prepare_hinv", "gq_quantize_workspace_size", "gq_quantize_layer",
             "gq_workspace_status", "gq_prepare_hinv_static")
 
@@ -103,13 +106,20 @@ def gq_version() -> str:
     return LIB.gq_version().decode()
 
 
-def gq_hessian_accumulate(H: torch.Tensor, X: torch.Tensor, stream=None) -> torch.Tensor:
-    """H += 2 X^T X on the GPU (H fp64 n x n, X bf16/fp32 T x n, both on the same device)."""
+def gq_hessian_workspace_size(T: int, n: int) -> int:
+    return int(LIB.gq_hessian_workspace_size(T, n))
+
+
+def gq_hessian_accumulate(H: torch.Tensor, X: torch.Tensor, accumulate: bool = True, ws=None,
+                          stream=None) -> torch.Tensor:
+    """H (+)= 2 X^T X on the GPU (H fp64 n x n, X bf16/fp32 T x n, same device)."""
     T, n = X.shape
     _need(H, torch.float64, (n, n), "H")
     if not X.is_cuda or not X.is_contiguous():
         raise ValueError("X must be a contiguous cuda tensor")
-    _check(LIB.gq_hessian_accumulate(_ptr(H), _ptr(X), _dtype_code(X), T, n, _stream(stream)),
+    ws = workspace(gq_hessian_workspace_size(T, n), X.device) if ws is None else ws
+    _check(LIB.gq_hessian_accumulate(_ptr(H), _ptr(X), _dtype_code(X), T, n, int(bool(accumulate)),
+                                     _ptr(ws), ws.numel(), _stream(stream)),
            "gq_hessian_accumulate")
     return H
 

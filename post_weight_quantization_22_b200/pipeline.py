@@ -25,13 +25,16 @@ class LayerResult:
 
 
 class LayerQuantizer:
-    def __init__(self, m: int, n: int, cfg: G.QuantCfg, device="cuda", damp: float = 0.01):
+    def __init__(self, m: int, n: int, cfg: G.QuantCfg, device="cuda", damp: float = 0.01,
+                 max_tokens: int = 65536):
         self.m, self.n, self.cfg, self.damp = m, n, cfg, damp
+        self.max_tokens = max_tokens
         dev = torch.device(device)
         self.H = torch.zeros((n, n), dtype=torch.float64, device=dev)
         self.U = torch.empty((n, n), dtype=torch.float32, device=dev)
         self.dead = torch.empty(n, dtype=torch.uint8, device=dev)
         self.delta = torch.empty(1, dtype=torch.float64, device=dev)
+        self.ws_hess = G.workspace(G.gq_hessian_workspace_size(max_tokens, n), dev)
         self.ws_prep = G.workspace(G.gq_prepare_workspace_size(n), dev)
         self.ws_quant = G.workspace(G.gq_quantize_workspace_size(m, n, cfg), dev)
         ng = 1 if cfg.group_size == 0 else -(-n // cfg.group_size)
@@ -41,9 +44,9 @@ class LayerQuantizer:
         self.loss = torch.empty(3, dtype=torch.float64, device=dev)
 
     def hessian(self, X: torch.Tensor, reset: bool = True, stream=None):
-        if reset:
-            self.H.zero_()
-        G.gq_hessian_accumulate(self.H, X, stream=stream)
+        if X.shape[0] > self.max_tokens:
+            raise ValueError(f"{X.shape[0]} tokens exceed this quantizer's {self.max_tokens}")
+        G.gq_hessian_accumulate(self.H, X, accumulate=not reset, ws=self.ws_hess, stream=stream)
 
     def prepare(self, stream=None):
         G.gq_prepare_hinv(self.H, self.damp, self.cfg.reverse, self.U, self.dead, self.delta,

@@ -19,7 +19,7 @@ pytestmark = pytest.mark.gpu
 CODE_MATCH = 0.999
 LOSS_REL = 1e-3
 H_REL = 1e-5
-H_REL_DESIGN = 1e-12
+H_REL_DESIGN = 1e-9   # digit rounding of entries below 2^-21 of their column's largest
 U_REL_DESIGN = 1e-6
 
 
@@ -35,7 +35,7 @@ def _compare(g, o, W, bits, group, rows=None, check_loss=True):
     if "U" in o:
         assert rel_fro(np.triu(g["U"]), o["U"]) <= U_REL_DESIGN
     assert np.array_equal(g["dead"], o["dead"])
-    assert abs(g["delta"] - o["delta"]) <= 1e-12 * abs(o["delta"])
+    assert abs(g["delta"] - o["delta"]) <= H_REL_DESIGN * abs(o["delta"])  # a mean of diag(H)
     gc = g["codes"] if rows is None else g["codes"][rows]
     match = float(np.mean(gc == o["codes"]))
     assert match >= CODE_MATCH, f"code match {match:.6f}"
