@@ -22,7 +22,8 @@
 
 namespace gq {
 
-constexpr int kNB = 64;  // Cholesky panel width
+constexpr int kNB = 64;      // Cholesky panel width (the leaf)
+constexpr int kSuper = 256;  // super-panel width (trailing-update depth)
 
 // ---------------------------------------------------------------------------------------
 // dead fix + damping statistics (one CTA)
@@ -216,13 +217,18 @@ cudaError_t launch_prepare(const double* H, int64_t n, double damp, int reverse,
     count_launches(1);
     GQ_TRY(cudaGetLastError());
   }
-  // Blocked right-looking Cholesky of M (lower, in place, 64-wide panels).  Each diagonal block
-  // is replaced by the inverse of its factor; the panel below becomes L21 = A21 L11^-T; the
-  // trailing matrix takes A22 -= L21 L21^T.
+  // Blocked right-looking Cholesky of M (lower, in place), 64-wide panels grouped into
+  // 256-wide super-panels.  For each 64-wide panel: the diagonal block is replaced by the
+  // inverse of its factor (leaf), the rows below become L21 = A21 L11^-T, and only the rest of
+  // the super-panel takes the update A -= L21 L21^T.  The columns after the super-panel take
+  // one K = 256 update per super-panel (fewer, larger fp64 tensor-core GEMMs, 4x less
+  // read-modify-write traffic on the trailing matrix than 64-wide steps).
   const int64_t nb = (n + kNB - 1) / kNB;
   for (int64_t k = 0; k < nb; ++k) {
     const int64_t c0 = k * kNB;
     const int w = (int)std::min<int64_t>(kNB, n - c0);
+    const int64_t sp0 = (c0 / kSuper) * kSuper;                 // super-panel start
+    const int64_t sp1 = std::min<int64_t>(sp0 + kSuper, n);     // super-panel end
     potrf_diag_kernel<<<1, 256, 0, s>>>(L.M, n, c0, w, L.hdr);
     count_launches(1);
     GQ_TRY(cudaGetLastError());
@@ -236,11 +242,21 @@ cudaError_t launch_prepare(const double* H, int64_t n, double damp, int reverse,
       g.C = P; g.ldc = n;
       GQ_TRY((f64_gemm<double, double, false, true>(g, 1, s)));
     }
-    {  // trailing: C -= P P^T, lower tiles
+    const int64_t inw = sp1 - (c0 + w);  // columns of the super-panel after this panel
+    if (inw > 0) {  // A[:, c0+w : sp1] -= L21 L21[c0+w : sp1]^T for every row below
       F64GemmArgs g{};
-      g.M = (int)rem; g.N = (int)rem; g.K = w; g.alpha = -1.0; g.beta_one = 1;
+      g.M = (int)rem; g.N = (int)inw; g.K = w; g.alpha = -1.0; g.beta_one = 1;
       g.A = P; g.lda = n; g.B = P; g.ldb = n;
       g.C = L.M + (c0 + w) * n + (c0 + w); g.ldc = n; g.lower_tiles = 1;
+      GQ_TRY((f64_gemm<double, double, false, true>(g, 1, s)));
+    }
+    if (c0 + w == sp1 && sp1 < n) {  // super-panel done: trailing update with K = its width
+      const int64_t trem = n - sp1, kw = sp1 - sp0;
+      double* PS = L.M + sp1 * n + sp0;  // L of the super-panel, rows sp1..n-1
+      F64GemmArgs g{};
+      g.M = (int)trem; g.N = (int)trem; g.K = (int)kw; g.alpha = -1.0; g.beta_one = 1;
+      g.A = PS; g.lda = n; g.B = PS; g.ldb = n;
+      g.C = L.M + sp1 * n + sp1; g.ldc = n; g.lower_tiles = 1;
       GQ_TRY((f64_gemm<double, double, false, true>(g, 1, s)));
     }
   }

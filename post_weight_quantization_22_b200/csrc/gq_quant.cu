@@ -19,9 +19,11 @@
 
 namespace gq {
 
-constexpr int kP = 4;                     // lanes per row in the column loop
+constexpr int kP = 4;                      // lanes per row in the column loop
 constexpr int kVPL = kBlock / kP;          // values per lane (32)
-constexpr int kRowsPerCta = 4 * 32 / kP;  // 32 rows per 128-thread CTA
+constexpr int kSW = 4 * kP;                // segment width: one 4-column chunk per lane
+constexpr int kColThreads = 128;
+constexpr int kRowsPerCta = kColThreads / kP;  // 32 rows per CTA
 // Per-block prepared U for the column loop (see ublk_kernel): 128 x 128 doubles + 2 x 128.
 constexpr int64_t kUBlkDoubles = (int64_t)kBlock * kBlock + 2 * kBlock;
 constexpr uint32_t kUBlkBytes = (uint32_t)(kUBlkDoubles * sizeof(double));
@@ -222,18 +224,19 @@ struct ColArgs {
   int* overflow;
 };
 
-// Lane ownership: the block's 128 columns form 8 segments of 16; in each segment lane t of a
-// row owns the 4-column chunk [16 seg + 4t, 16 seg + 4t + 4).  Each lane keeps its 8 chunks in
-// registers, v[4c + u] = chunk (seg + c); after a segment the array is rotated by one chunk,
-// so the unrolled 16-step body refers to fixed registers and the segment loop stays a small
-// runtime loop (a fully unrolled 128-step body does not fit the instruction cache).
+// Lane ownership: each row is handled by kP = 4 lanes; the block's 128 columns form 8 segments
+// of 16, and in each segment lane t owns the 4-column chunk [16 seg + 4t, 16 seg + 4t + 4).
+// Each lane keeps its 8 chunks in registers, v[4c + u] = chunk (seg + c); after a segment the
+// array is rotated by one chunk, so the unrolled 16-step body refers to fixed registers and the
+// segment loop stays a small runtime loop (a fully unrolled 128-step body does not fit the
+// instruction cache).  128-thread CTAs of 32 rows.
 //
 // The recursion runs in fp64: the in-block feedback sums cancel strongly when the grid is
 // coarse, and an fp32 recursion flips ~1-3 % of the codes on ill-conditioned layers (measured
 // against the fp64 oracle), while fp64 here with fp32 storage of W, E and U between blocks
 // reproduces the oracle's codes.
 template <int G>
-__global__ void __launch_bounds__(128, 1) colloop_kernel(ColArgs a) {
+__global__ void __launch_bounds__(kColThreads, 1) colloop_kernel(ColArgs a) {
   extern __shared__ __align__(16) double q_smem[];
   double* Us = q_smem;                       // [128][128] this block's part of U (fp64, masked)
   double* invd = q_smem + kBlock * kBlock;   // [128]  1/U_jj
@@ -264,7 +267,7 @@ __global__ void __launch_bounds__(128, 1) colloop_kernel(ColArgs a) {
   double v[kVPL];
 #pragma unroll
   for (int c = 0; c < kVPL / 4; ++c) {
-    int k = 16 * c + 4 * t;
+    int k = kSW * c + 4 * t;
     float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
     if (active) {
       const float* src = a.Wf + rr * n + j0 + k;
@@ -292,40 +295,44 @@ __global__ void __launch_bounds__(128, 1) colloop_kernel(ColArgs a) {
   float* Ehrow = a.Ehi + rr * kBlock;
   float* Elrow = a.Elo + rr * kBlock;
   uint8_t* crow = a.codes8 + row * a.ldc8 + j0;
+  constexpr int kGStep = (G > 0 && G < kSW) ? G : kSW;  // distance between possible group starts
 
-  for (int seg = 0; seg < kBlock / 16; ++seg) {
-    if (16 * seg >= bw) break;
-    if constexpr (G > 0) {
-      if ((16 * seg) % G == 0) {
-        double lo = 0.0, hi = 0.0;
-#pragma unroll
-        for (int c = 0; c < (G / 16 < 8 ? G / 16 : 8); ++c)
-#pragma unroll
-          for (int u = 0; u < 4; ++u)
-            if (16 * (seg + c) + 4 * t + u < bw) { lo = fmin(lo, v[4 * c + u]); hi = fmax(hi, v[4 * c + u]); }
-#pragma unroll
-        for (int o = kP / 2; o > 0; o >>= 1) {
-          lo = fmin(lo, __shfl_xor_sync(full, lo, o));
-          hi = fmax(hi, __shfl_xor_sync(full, hi, o));
-        }
-        if (lo == 0.0 && hi == 0.0) { lo = -1.0; hi = 1.0; }
-        s = (hi - lo) / maxq;
-        z = rint(-lo / s);
-        inv_s = 1.0 / s;
-        if (active && t == 0) {
-          int64_t g = (j0 + 16 * seg) / G;
-          a.scales[row * a.ngroups + g] = (float)s;
-          a.zeros[row * a.ngroups + g] = (uint8_t)z;
-        }
-      }
-    }
-    const double cmin = -z, cmax = maxq - z;  // code range in the shifted domain c - z
+  for (int seg = 0; seg < kBlock / kSW; ++seg) {
+    if (kSW * seg >= bw) break;
     float eo[4] = {0.f, 0.f, 0.f, 0.f};
     uint32_t cw = 0u;
 #pragma unroll
-    for (int jl = 0; jl < 16; ++jl) {
-      const int jj = 16 * seg + jl;
+    for (int jl = 0; jl < kSW; ++jl) {
+      const int jj = kSW * seg + jl;
       if (jj < bw) {
+        if constexpr (G > 0) {
+          if (jl % kGStep == 0 && (jj % G) == 0) {
+            // group grid from the current (error-fed) weights of columns [jj, jj + G)
+            double lo = 0.0, hi = 0.0;
+#pragma unroll
+            for (int c = 0; c < kVPL / 4; ++c)
+#pragma unroll
+              for (int u = 0; u < 4; ++u) {
+                const int k = kSW * (seg + c) + 4 * t + u;
+                if (k >= jj && k < jj + G && k < bw) { lo = fmin(lo, v[4 * c + u]); hi = fmax(hi, v[4 * c + u]); }
+              }
+#pragma unroll
+            for (int o = kP / 2; o > 0; o >>= 1) {
+              lo = fmin(lo, __shfl_xor_sync(full, lo, o));
+              hi = fmax(hi, __shfl_xor_sync(full, hi, o));
+            }
+            if (lo == 0.0 && hi == 0.0) { lo = -1.0; hi = 1.0; }
+            s = (hi - lo) / maxq;
+            z = rint(-lo / s);
+            inv_s = 1.0 / s;
+            if (active && t == 0) {
+              const int64_t g = (j0 + jj) / G;
+              a.scales[row * a.ngroups + g] = (float)s;
+              a.zeros[row * a.ngroups + g] = (uint8_t)z;
+            }
+          }
+        }
+        const double cmin = -z, cmax = maxq - z;  // code range in the shifted domain c - z
         const int owner = jl / 4, slot = jl % 4;
         const double id = invd[jj];
         const double sd = s * id;
@@ -344,7 +351,7 @@ __global__ void __launch_bounds__(128, 1) colloop_kernel(ColArgs a) {
         }
         e2 = fma(e, e, e2);
         bnd = fma(s * s, invd2[jj], bnd);
-        const double* urow = Us + jj * kBlock + 16 * seg + 4 * t;
+        const double* urow = Us + jj * kBlock + kSW * seg + 4 * t;
         if (t >= owner) {  // the chunk that holds column jj: only its later columns
           const double2 u01 = *reinterpret_cast<const double2*>(urow);
           const double2 u23 = *reinterpret_cast<const double2*>(urow + 2);
@@ -355,9 +362,9 @@ __global__ void __launch_bounds__(128, 1) colloop_kernel(ColArgs a) {
         }
 #pragma unroll
         for (int c2 = 1; c2 < kVPL / 4; ++c2) {
-          if (c2 < kBlock / 16 - seg) {
-            const double2 u01 = *reinterpret_cast<const double2*>(urow + 16 * c2);
-            const double2 u23 = *reinterpret_cast<const double2*>(urow + 16 * c2 + 2);
+          if (c2 < kBlock / kSW - seg) {
+            const double2 u01 = *reinterpret_cast<const double2*>(urow + kSW * c2);
+            const double2 u23 = *reinterpret_cast<const double2*>(urow + kSW * c2 + 2);
             v[4 * c2 + 0] = fma(-e, u01.x, v[4 * c2 + 0]);
             v[4 * c2 + 1] = fma(-e, u01.y, v[4 * c2 + 1]);
             v[4 * c2 + 2] = fma(-e, u23.x, v[4 * c2 + 2]);
@@ -368,7 +375,7 @@ __global__ void __launch_bounds__(128, 1) colloop_kernel(ColArgs a) {
     }
     // this segment's errors and codes
     if (active) {
-      const int k = 16 * seg + 4 * t;
+      const int k = kSW * seg + 4 * t;
       float4 hi, lo;
       hi.x = tf32_rna(eo[0]); hi.y = tf32_rna(eo[1]); hi.z = tf32_rna(eo[2]); hi.w = tf32_rna(eo[3]);
       lo.x = eo[0] - hi.x; lo.y = eo[1] - hi.y; lo.z = eo[2] - hi.z; lo.w = eo[3] - hi.w;
@@ -515,7 +522,7 @@ template <int G>
 static cudaError_t launch_colloop(const ColArgs& ca, cudaStream_t s) {
   const size_t smem = kColSmem;
   unsigned grid = (unsigned)((ca.k_rows + kRowsPerCta - 1) / kRowsPerCta);
-  colloop_kernel<G><<<grid, 128, smem, s>>>(ca);
+  colloop_kernel<G><<<grid, kColThreads, smem, s>>>(ca);
   count_launches(1);
   return cudaGetLastError();
 }
