@@ -374,6 +374,31 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def run_case(args):
+    """One untimed invocation for profilers: `layer` (the q_proj recipe at --case-n) or `factor`
+    (gq_prepare_hinv on a seeded SPD fp64 H of width --case-n)."""
+    from post_weight_quantization_22_b200 import gq as G
+    from post_weight_quantization_22_b200 import synth
+    from post_weight_quantization_22_b200.pipeline import LayerQuantizer
+
+    torch.cuda.set_device(0)
+    n = args.case_n
+    if args.case == "layer":
+        W, X, spec = synth.workload(DEFAULT_WORKLOAD, m=n, n=n, T=n)
+        cfg = G.QuantCfg(bits=spec["bits"], group_size=spec["group"])
+        lq = LayerQuantizer(n, n, cfg, device="cuda")
+        lq.run(W.cuda(), X.cuda())
+        torch.cuda.synchronize()
+        print("status", lq.status())
+    else:
+        g = torch.Generator(device="cuda").manual_seed(0)
+        X = torch.randn(n + 64, n, dtype=torch.float64, device="cuda", generator=g)
+        H = 2 * (X.T @ X)
+        U, dead, delta, ws = G.gq_prepare_hinv(H, 0.01)
+        torch.cuda.synchronize()
+        print("status", G.gq_workspace_status(ws))
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -384,7 +409,12 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-rows", type=int, default=256)
     ap.add_argument("--ref-rows", type=int, default=32)
+    ap.add_argument("--case", choices=["layer", "factor"], default=None,
+                    help="run one untimed invocation (for profilers) and exit")
+    ap.add_argument("--case-n", type=int, default=2048)
     args = ap.parse_args(argv)
+    if args.case:
+        return run_case(args)
     if args.warmup < 3 and args.impl == "gq":
         print("note: warm-up raised to 3 steps", file=sys.stderr)
         args.warmup = 3
