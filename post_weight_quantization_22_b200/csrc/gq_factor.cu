@@ -14,7 +14,6 @@
 // Everything is fp64: the damped Hessians of LLM layers have condition numbers ~1e5 and the
 // codes downstream change when U carries fp32-level errors.
 #include "gq_internal.cuh"
-#include "gq_f64gemm.cuh"
 
 #include <math.h>
 #include <vector>
@@ -54,8 +53,8 @@ __global__ void __launch_bounds__(1024) diag_stats_kernel(const double* H, int64
 }
 
 // M[i][j] (j <= i) = Hfix[pi(i)][pi(j)] + (i == j) * delta, pi(i) = n-1-i (forward) or i.
-__global__ void build_m_kernel(const double* H, int64_t n, int reverse, const WsHeader* hdr,
-                               double* M) {
+__global__ void build_m_kernel(const double* H, int64_t n, int64_t ldm, int reverse,
+                               const WsHeader* hdr, double* M) {
   int64_t j = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
   int64_t i = blockIdx.y;
   if (j > i || i >= n) return;
@@ -66,7 +65,7 @@ __global__ void build_m_kernel(const double* H, int64_t n, int reverse, const Ws
     if (v == 0.0) v = 1.0;
     v += hdr->scratch[0];
   }
-  M[i * n + j] = v;
+  M[i * ldm + j] = v;
 }
 
 // 1/p for p > 0: the hardware reciprocal estimate (rcp.approx.ftz.f64, about 2^-22 relative)
@@ -88,88 +87,124 @@ __device__ __forceinline__ double recip_newton(double p) {
 // pivot c, rows r > c take S[r][q] -= f_r S[q][c] (q in (c, r]) and A[r][j] -= f_r A[c][j]
 // (j <= c), f_r = S[r][c] / S[c][c].  Then A = L_unit^-1, the pivots are D of
 // S = L_unit D L_unit^T, and L^-1 = D^-1/2 A.
-// 256 threads, 4 per row; thread (r, part) keeps S[r][4i+part] and A[r][4i+part] (i < 16) in
-// registers.  Per pivot only column c of S and row c of A travel, through double-buffered
-// shared memory, with one barrier; the pivot loop is unrolled so every register index is fixed.
+// 256 threads; thread (a, b) = (tid / 16, tid % 16) keeps the 4 x 4 blocks S[4a..4a+3][4b..4b+3]
+// and A[4a..4a+3][4b..4b+3] in registers.  Per pivot, column c of S and row c of A travel
+// through double-buffered shared memory (one barrier); a thread reads 4 multipliers, 4 column
+// values and 4 row values there with 16-byte loads.  The pivot loop is unrolled 4 deep (register
+// indices fixed, the body small enough to stay in the instruction cache).
 // ---------------------------------------------------------------------------------------
-__global__ void __launch_bounds__(256, 1) potrf_diag_kernel(double* M, int64_t n, int64_t c0,
+__global__ void __launch_bounds__(256, 1) potrf_diag_kernel(double* M, int64_t ldm, int64_t c0,
                                                             int w, WsHeader* hdr) {
-  __shared__ double colbuf[2][kNB];
-  __shared__ double rowbuf[2][kNB];
+  __shared__ __align__(16) double colbuf[2][kNB];
+  __shared__ __align__(16) double rowbuf[2][kNB];
+  __shared__ double dbuf[kNB];
   const int tid = threadIdx.x;
-  const int r = tid >> 2, part = tid & 3;
-  double sv[16], av[16];
-  // all loads of the block issue before any use
+  const int a = tid >> 4, b = tid & 15;
+  double sv[4][4], av[4][4];
 #pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    const int q = 4 * i + part;
-    double v = 0.0;
-    if (r < w && q < w) {
-      if (q <= r) v = M[(c0 + r) * n + c0 + q];
-    } else if (q == r) {
-      v = 1.0;
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int r = 4 * a + i, q = 4 * b + j;
+      double v = 0.0;
+      if (r < w && q < w) {
+        if (q <= r) v = M[(c0 + r) * ldm + c0 + q];
+      } else if (q == r) {
+        v = 1.0;
+      }
+      sv[i][j] = v;
+      av[i][j] = (q == r) ? 1.0 : 0.0;
     }
-    sv[i] = v;
-    av[i] = (q == r) ? 1.0 : 0.0;
-  }
+#pragma unroll 1
+  for (int c4 = 0; c4 < kNB / 4; ++c4) {
 #pragma unroll
-  for (int c = 0; c < kNB - 1; ++c) {
-    const int buf = c & 1;
-    if (part == (c & 3)) colbuf[buf][r] = sv[c >> 2];  // S[r][c]
-    if (r == c) {
+    for (int cc = 0; cc < 4; ++cc) {
+      const int c = 4 * c4 + cc;
+      const int buf = cc & 1;
+      if (b == c4) {
 #pragma unroll
-      for (int i = 0; i < 16; ++i)
-        if (4 * i + part <= c) rowbuf[buf][4 * i + part] = av[i];  // A[c][j]
-    }
-    __syncthreads();
-    if (r > c) {
-      double p = colbuf[buf][c];
-      if (!(p > 0.0)) p = 1.0;  // reported below from the final pivots
-      const double f = colbuf[buf][r] * recip_newton(p);
+        for (int i = 0; i < 4; ++i) colbuf[buf][4 * a + i] = sv[i][cc];  // S[.][c]
+      }
+      if (a == c4) {
 #pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        const int q = 4 * i + part;
-        if (q > c && q <= r) sv[i] = fma(-f, colbuf[buf][q], sv[i]);
-        if (q <= c) av[i] = fma(-f, rowbuf[buf][q], av[i]);
+        for (int j = 0; j < 4; ++j) rowbuf[buf][4 * b + j] = av[cc][j];  // A[c][.]
+      }
+      __syncthreads();
+      if (4 * a + 3 > c) {
+        double p = colbuf[buf][c];
+        if (!(p > 0.0)) p = 1.0;  // reported below from the final pivots
+        const double rp = recip_newton(p);
+        const double2 f01 = *reinterpret_cast<const double2*>(&colbuf[buf][4 * a]);
+        const double2 f23 = *reinterpret_cast<const double2*>(&colbuf[buf][4 * a + 2]);
+        const double fr[4] = {f01.x * rp, f01.y * rp, f23.x * rp, f23.y * rp};
+        if (4 * b + 3 > c) {  // S: entries with c < q <= r
+          const double2 q01 = *reinterpret_cast<const double2*>(&colbuf[buf][4 * b]);
+          const double2 q23 = *reinterpret_cast<const double2*>(&colbuf[buf][4 * b + 2]);
+          const double cq[4] = {q01.x, q01.y, q23.x, q23.y};
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+              if (4 * b + j > c && 4 * b + j <= 4 * a + i) sv[i][j] = fma(-fr[i], cq[j], sv[i][j]);
+        }
+        if (4 * b <= c) {  // A: entries with q <= c < r
+          const double2 r01 = *reinterpret_cast<const double2*>(&rowbuf[buf][4 * b]);
+          const double2 r23 = *reinterpret_cast<const double2*>(&rowbuf[buf][4 * b + 2]);
+          const double rq[4] = {r01.x, r01.y, r23.x, r23.y};
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+              if (4 * b + j <= c && 4 * a + i > c) av[i][j] = fma(-fr[i], rq[j], av[i][j]);
+        }
       }
     }
   }
-  // pivot D_r = S[r][r], held by part r % 4
-  double d = 0.0;
+  // pivots D_r = S[r][r], held by the diagonal threads
+  if (a == b) {
 #pragma unroll
-  for (int i = 0; i < 16; ++i)
-    if (4 * i + part == r) d = sv[i];
-  d = __shfl_sync(0xffffffffu, d, (tid & 31 & ~3) | (r & 3));
-  if (!(d > 0.0)) {
-    if (r < w && part == 0) record_status(hdr, GQ_ERR_NOT_PD);
-    d = 1.0;
+    for (int i = 0; i < 4; ++i) dbuf[4 * a + i] = sv[i][i];
   }
-  const double rs = 1.0 / sqrt(d);
-  if (r < w) {
+  __syncthreads();
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      const int q = 4 * i + part;
-      if (q <= r) M[(c0 + r) * n + c0 + q] = av[i] * rs;
+  for (int i = 0; i < 4; ++i) {
+    const int r = 4 * a + i;
+    double d = dbuf[r];
+    if (!(d > 0.0)) {
+      if (r < w && b == 0) record_status(hdr, GQ_ERR_NOT_PD);
+      d = 1.0;
+    }
+    const double rs = 1.0 / sqrt(d);
+    if (r < w) {
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int q = 4 * b + j;
+        if (q <= r) M[(c0 + r) * ldm + c0 + q] = av[i][j] * rs;
+      }
     }
   }
 }
 
 // U[i][j] = (i <= j) ? (float) Linv[n-1-i][n-1-j] : 0
-__global__ void flip_to_u_kernel(const double* M, int64_t n, float* U) {
+__global__ void flip_to_u_kernel(const double* M, int64_t n, int64_t ldm, float* U) {
   int64_t j = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
   int64_t i = blockIdx.y;
   if (j >= n) return;
   float v = 0.f;
-  if (i <= j) v = (float)M[(n - 1 - i) * n + (n - 1 - j)];
+  if (i <= j) v = (float)M[(n - 1 - i) * ldm + (n - 1 - j)];
   U[i * n + j] = v;
 }
 
 // ---------------------------------------------------------------------------------------
 // host orchestration
 // ---------------------------------------------------------------------------------------
+// Leading dimension of the factor's work matrix: rows start on 128-byte boundaries (TMA needs
+// 16-byte multiples).
+static int64_t m_ld(int64_t n) { return (n + 15) / 16 * 16; }
+
 struct PrepLayout {
   WsHeader* hdr;
-  double* M;     // n x n: lower triangle = J P H_d P J, then the inverse of its Cholesky factor
+  double* M;     // n x ldm: lower triangle = J P H_d P J, then the inverse of its Cholesky factor
   double* tbuf;  // doubling scratch of the triangular inverse
   size_t bytes;
 };
@@ -188,7 +223,7 @@ static PrepLayout prep_layout(void* ws, int64_t n) {
   Carver c(ws);
   PrepLayout L;
   L.hdr = c.take<WsHeader>(1);
-  L.M = c.take<double>((size_t)n * n);
+  L.M = c.take<double>((size_t)n * m_ld(n));
   L.tbuf = c.take<double>(trtri_tbuf_elems(n) + 1);
   L.bytes = c.off;
   return L;
@@ -196,7 +231,7 @@ static PrepLayout prep_layout(void* ws, int64_t n) {
 
 size_t prepare_ws_bytes(int64_t n) { return prep_layout(nullptr, n).bytes; }
 
-cudaError_t factor_init_attributes() { return cudaSuccess; }
+cudaError_t factor_init_attributes() { return dgemm_init_attributes(); }
 
 #define GQ_TRY(x)                               \
   do {                                          \
@@ -207,16 +242,22 @@ cudaError_t factor_init_attributes() { return cudaSuccess; }
 cudaError_t launch_prepare(const double* H, int64_t n, double damp, int reverse, float* U,
                            uint8_t* dead, double* delta, void* ws, cudaStream_t s) {
   PrepLayout L = prep_layout(ws, n);
+  const int64_t ldm = m_ld(n);
   GQ_TRY(cudaMemsetAsync(L.hdr, 0, sizeof(WsHeader), s));
   diag_stats_kernel<<<1, 1024, 0, s>>>(H, n, damp, dead, delta, L.hdr);
   count_launches(1);
   GQ_TRY(cudaGetLastError());
   {
     dim3 grid((unsigned)((n + 255) / 256), (unsigned)n);
-    build_m_kernel<<<grid, 256, 0, s>>>(H, n, reverse, L.hdr, L.M);
+    build_m_kernel<<<grid, 256, 0, s>>>(H, n, ldm, reverse, L.hdr, L.M);
     count_launches(1);
     GQ_TRY(cudaGetLastError());
   }
+  // The work matrix as a GEMM operand (its upper triangle is scratch: the GEMM never multiplies
+  // entries outside an operand's triangle).
+  auto Mop = [&](int64_t row0, int64_t col0, int64_t zrow = 0, int64_t zcol = 0) {
+    return DgemmOperand{L.M, n, n, ldm, row0, col0, zrow, zcol};
+  };
   // Blocked right-looking Cholesky of M (lower, in place), 64-wide panels grouped into
   // 256-wide super-panels.  For each 64-wide panel: the diagonal block is replaced by the
   // inverse of its factor (leaf), the rows below become L21 = A21 L11^-T, and only the rest of
@@ -229,35 +270,37 @@ cudaError_t launch_prepare(const double* H, int64_t n, double damp, int reverse,
     const int w = (int)std::min<int64_t>(kNB, n - c0);
     const int64_t sp0 = (c0 / kSuper) * kSuper;                 // super-panel start
     const int64_t sp1 = std::min<int64_t>(sp0 + kSuper, n);     // super-panel end
-    potrf_diag_kernel<<<1, 256, 0, s>>>(L.M, n, c0, w, L.hdr);
+    potrf_diag_kernel<<<1, 256, 0, s>>>(L.M, ldm, c0, w, L.hdr);
     count_launches(1);
     GQ_TRY(cudaGetLastError());
     const int64_t rem = n - c0 - w;
     if (rem <= 0) continue;
-    double* P = L.M + (c0 + w) * n + c0;
-    {  // P <- P (L11^-1)^T  (in place: one output tile column, each CTA owns its rows)
-      F64GemmArgs g{};
-      g.M = (int)rem; g.N = w; g.K = w; g.alpha = 1.0; g.beta_one = 0;
-      g.A = P; g.lda = n; g.B = L.M + c0 * n + c0; g.ldb = n; g.b_upper = 1;
-      g.C = P; g.ldc = n;
-      GQ_TRY((f64_gemm<double, double, false, true>(g, 1, s)));
+    {  // P <- P (L11^-1)^T, in place: each CTA owns whole rows of P (N = w = one tile)
+      DgemmCall g{};
+      g.M = (int)rem; g.N = w; g.K = w; g.batch = 1; g.alpha = 1.0; g.beta_one = 0;
+      g.A = Mop(c0 + w, c0);
+      g.B = Mop(c0, c0); g.b_nmajor = 0; g.b_upper = 1;  // opB[k][j] = L11^-1[j][k]
+      g.C = L.M + (c0 + w) * ldm + c0; g.ldc = ldm; g.hdr = L.hdr;
+      GQ_TRY(launch_dgemm(g, s));
     }
     const int64_t inw = sp1 - (c0 + w);  // columns of the super-panel after this panel
     if (inw > 0) {  // A[:, c0+w : sp1] -= L21 L21[c0+w : sp1]^T for every row below
-      F64GemmArgs g{};
-      g.M = (int)rem; g.N = (int)inw; g.K = w; g.alpha = -1.0; g.beta_one = 1;
-      g.A = P; g.lda = n; g.B = P; g.ldb = n;
-      g.C = L.M + (c0 + w) * n + (c0 + w); g.ldc = n; g.lower_tiles = 1;
-      GQ_TRY((f64_gemm<double, double, false, true>(g, 1, s)));
+      DgemmCall g{};
+      g.M = (int)rem; g.N = (int)inw; g.K = w; g.batch = 1; g.alpha = -1.0; g.beta_one = 1;
+      g.A = Mop(c0 + w, c0);
+      g.B = Mop(c0 + w, c0); g.b_nmajor = 0;
+      g.C = L.M + (c0 + w) * ldm + (c0 + w); g.ldc = ldm; g.lower_tiles = 1; g.hdr = L.hdr;
+      GQ_TRY(launch_dgemm(g, s));
     }
     if (c0 + w == sp1 && sp1 < n) {  // super-panel done: trailing update with K = its width
       const int64_t trem = n - sp1, kw = sp1 - sp0;
-      double* PS = L.M + sp1 * n + sp0;  // L of the super-panel, rows sp1..n-1
-      F64GemmArgs g{};
-      g.M = (int)trem; g.N = (int)trem; g.K = (int)kw; g.alpha = -1.0; g.beta_one = 1;
-      g.A = PS; g.lda = n; g.B = PS; g.ldb = n;
-      g.C = L.M + sp1 * n + sp1; g.ldc = n; g.lower_tiles = 1;
-      GQ_TRY((f64_gemm<double, double, false, true>(g, 1, s)));
+      DgemmCall g{};
+      g.M = (int)trem; g.N = (int)trem; g.K = (int)kw; g.batch = 1; g.alpha = -1.0;
+      g.beta_one = 1;
+      g.A = Mop(sp1, sp0);
+      g.B = Mop(sp1, sp0); g.b_nmajor = 0;
+      g.C = L.M + sp1 * ldm + sp1; g.ldc = ldm; g.lower_tiles = 1; g.hdr = L.hdr;
+      GQ_TRY(launch_dgemm(g, s));
     }
   }
   // Triangular inverse by doubling over the diagonal blocks (already inverted):
@@ -273,27 +316,29 @@ cudaError_t launch_prepare(const double* H, int64_t n, double damp, int reverse,
       if (batch <= 0 || cw <= 0) continue;
       double* tb = L.tbuf + (pass == 0 ? 0 : npairs_full * bs * bs);
       {  // T = B A^-1
-        F64GemmArgs g{};
-        g.M = (int)cw; g.N = (int)bs; g.K = (int)bs; g.alpha = 1.0; g.beta_one = 0;
-        g.A = L.M + (r + bs) * n + r; g.lda = n; g.strideA = 2 * bs * n + 2 * bs;
-        g.B = L.M + r * n + r; g.ldb = n; g.strideB = 2 * bs * n + 2 * bs; g.b_lower = 1;
-        g.C = tb; g.ldc = bs; g.strideC = bs * bs;
-        GQ_TRY((f64_gemm<double, double, false, false>(g, (int)batch, s)));
+        DgemmCall g{};
+        g.M = (int)cw; g.N = (int)bs; g.K = (int)bs; g.batch = (int)batch; g.alpha = 1.0;
+        g.beta_one = 0;
+        g.A = Mop(r + bs, r, 2 * bs, 2 * bs);
+        g.B = Mop(r, r, 2 * bs, 2 * bs); g.b_nmajor = 1; g.b_lower = 1;
+        g.C = tb; g.ldc = bs; g.strideC = bs * bs; g.hdr = L.hdr;
+        GQ_TRY(launch_dgemm(g, s));
       }
       {  // B <- -C^-1 T
-        F64GemmArgs g{};
-        g.M = (int)cw; g.N = (int)bs; g.K = (int)cw; g.alpha = -1.0; g.beta_one = 0;
-        g.A = L.M + (r + bs) * n + (r + bs); g.lda = n; g.strideA = 2 * bs * n + 2 * bs;
-        g.a_lower = 1;
-        g.B = tb; g.ldb = bs; g.strideB = bs * bs;
-        g.C = L.M + (r + bs) * n + r; g.ldc = n; g.strideC = 2 * bs * n + 2 * bs;
-        GQ_TRY((f64_gemm<double, double, false, false>(g, (int)batch, s)));
+        DgemmCall g{};
+        g.M = (int)cw; g.N = (int)bs; g.K = (int)cw; g.batch = (int)batch; g.alpha = -1.0;
+        g.beta_one = 0;
+        g.A = Mop(r + bs, r + bs, 2 * bs, 2 * bs); g.a_lower = 1;
+        g.B = DgemmOperand{tb, batch * bs, bs, bs, 0, 0, bs, 0}; g.b_nmajor = 1;
+        g.C = L.M + (r + bs) * ldm + r; g.ldc = ldm; g.strideC = 2 * bs * ldm + 2 * bs;
+        g.hdr = L.hdr;
+        GQ_TRY(launch_dgemm(g, s));
       }
     }
   }
   {
     dim3 grid((unsigned)((n + 255) / 256), (unsigned)n);
-    flip_to_u_kernel<<<grid, 256, 0, s>>>(L.M, n, U);
+    flip_to_u_kernel<<<grid, 256, 0, s>>>(L.M, n, ldm, U);
     count_launches(1);
     GQ_TRY(cudaGetLastError());
   }

@@ -81,6 +81,43 @@ cudaError_t factor_init_attributes();
 cudaError_t quant_init_attributes();
 cudaError_t lazy_tc_init_attributes();
 
+// ---- TMA tensor maps (gq_lazy_tc.cu) ----
+// Row-major matrix (rows x cols elements of elem_bytes, leading dimension ld elements) as a 2-D
+// tensor map with a box of box_cols x box_rows elements, zero fill outside the matrix.
+cudaError_t encode_tmap_2d(CUtensorMap* map, CUtensorMapDataType dt, size_t elem_bytes,
+                           const void* p, int64_t rows, int64_t cols, int64_t ld,
+                           uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle swz);
+
+// ---- fp64 GEMM on the fp64 tensor cores (gq_dgemm.cu) ----
+// A matrix operand: a row-major fp64 matrix (rows x cols, leading dimension ld, 16-byte aligned
+// base, ld even) and the position of the GEMM's operand block inside it; batch z adds
+// (zrow, zcol) to the position.
+struct DgemmOperand {
+  const double* base;
+  int64_t rows, cols, ld;
+  int64_t row0, col0, zrow, zcol;
+};
+// C[i][j] = (beta_one ? C[i][j] : 0) + alpha * sum_k opA[i][k] opB[k][j], i < M, j < N, k < K.
+//   opA[i][k] = A(row0 + i, col0 + k)                      (contraction index contiguous)
+//   opB[k][j] = B(row0 + j, col0 + k)  if !b_nmajor         ("NT": contraction contiguous)
+//             = B(row0 + k, col0 + j)  if  b_nmajor         ("NN": output index contiguous)
+// Structure: a_lower (opA[i][k] = 0 for k > i), b_lower (opB[k][j] = 0 for k < j), b_upper
+// (opB[k][j] = 0 for k > j): the zero parts are never multiplied, whatever memory holds there.
+// lower_tiles: only output tiles that reach the diagonal i >= j are computed.
+struct DgemmCall {
+  int M, N, K, batch;
+  double alpha;
+  int beta_one;
+  DgemmOperand A, B;
+  int b_nmajor;
+  double* C;
+  int64_t ldc, strideC;
+  int a_lower, b_lower, b_upper, lower_tiles;
+  WsHeader* hdr;
+};
+cudaError_t dgemm_init_attributes();
+cudaError_t launch_dgemm(const DgemmCall& c, cudaStream_t s);
+
 // ---- lazy block update on tensor cores (gq_lazy_tc.cu) ----
 struct LazyTcMaps {
   CUtensorMap ahi, alo, bhi, blo;

@@ -155,17 +155,25 @@ cudaError_t get_encode() {
 // box of 32 columns x box_rows rows, zero fill outside; swizzle as the operand's layout needs.
 cudaError_t encode_f32(CUtensorMap* map, const float* p, int64_t rows, int64_t cols, int64_t ld,
                        uint32_t box_rows, CUtensorMapSwizzle swz) {
+  return encode_tmap_2d(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, sizeof(float), p, rows, cols, ld,
+                        32, box_rows, swz);
+}
+}  // namespace
+
+cudaError_t encode_tmap_2d(CUtensorMap* map, CUtensorMapDataType dt, size_t elem_bytes,
+                           const void* p, int64_t rows, int64_t cols, int64_t ld,
+                           uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle swz) {
+  cudaError_t e = get_encode();
+  if (e != cudaSuccess) return e;
   cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
-  cuuint64_t strides[1] = {(cuuint64_t)ld * sizeof(float)};
-  cuuint32_t box[2] = {32, box_rows};
+  cuuint64_t strides[1] = {(cuuint64_t)ld * elem_bytes};
+  cuuint32_t box[2] = {box_cols, box_rows};
   cuuint32_t estr[2] = {1, 1};
-  CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(p), dims,
-                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
-                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+  CUresult r = g_encode(map, dt, 2, const_cast<void*>(p), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
-}  // namespace
 
 cudaError_t lazy_tc_init_attributes() {
   return cudaFuncSetAttribute(lazy_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
