@@ -95,7 +95,9 @@ gq_status gq_hessian_accumulate(double* d_H, const void* d_X, gq_dtype x_dtype, 
                                 int64_t n, int accumulate, void* d_ws, size_t ws_bytes,
                                 gq_stream_t stream);
 
-/* Workspace bytes gq_prepare_hinv needs for width n (256-byte aligned base required). */
+/* Workspace bytes gq_prepare_hinv needs for width n (256-byte aligned base required): two fp64
+ * n x n work matrices (the factor and its inverse in place, and the inverse's accumulated block
+ * products), about 16 n^2 bytes. */
 size_t gq_prepare_workspace_size(int64_t n);
 
 /*
@@ -129,7 +131,7 @@ gq_status gq_prepare_hinv(const double* d_H, int64_t n, double damp, int reverse
  * outputs).  The papers have no counterpart of this call; it exists for such callers.
  *
  * Same arguments and results as gq_prepare_hinv, minus the workspace: the scratch is a static
- * device array inside the library (about 11 MB per device that loads the library, held until
+ * device array inside the library (about 17 MB per device that loads the library, held until
  * the process exits), so n is limited to 1 <= n <= 1024; larger n returns GQ_ERR_INVALID_ARG
  * and enqueues nothing.  No device memory is allocated or freed.
  *

@@ -87,7 +87,7 @@ gq_status run_graphed(std::vector<uint64_t> key, cudaStream_t user, Enqueue enqu
     return st != GQ_OK ? st : GQ_ERR_CUDA;
   }
   cudaGraphExec_t exec = nullptr;
-  ec = cudaGraphInstantiate(&exec, graph, 0);
+  ec = cudaGraphInstantiateWithFlags(&exec, graph, cudaGraphInstantiateFlagUseNodePriority);
   cudaGraphDestroy(graph);
   if (ec != cudaSuccess) {
     (void)cudaGetLastError();

@@ -55,13 +55,6 @@ struct DgemmArgs {
   WsHeader* hdr;
 };
 
-__device__ __forceinline__ void dmma16x8x8(double (&c)[4], const double (&a)[4],
-                                           const double (&b)[2]) {
-  asm("mma.sync.aligned.m16n8k8.row.col.f64.f64.f64.f64 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
-      "{%8,%9}, {%0,%1,%2,%3};"
-      : "+d"(c[0]), "+d"(c[1]), "+d"(c[2]), "+d"(c[3])
-      : "d"(a[0]), "d"(a[1]), "d"(a[2]), "d"(a[3]), "d"(b[0]), "d"(b[1]));
-}
 }  // namespace
 
 template <bool kNN, int kWM>
@@ -143,12 +136,24 @@ __device__ __forceinline__ void dgemm_body(const CUtensorMap& ma, const CUtensor
         }
         issued = kc + 1;
       }
+      // The epilogue reads this C tile: bring it into L2 while the last slices are consumed.
+      if (g.beta_one && g.c_vec && j0 + kBN <= g.N) {
+        const double* c0p = g.C + (int64_t)z * g.strideC + (int64_t)i0 * g.ldc + j0;
+        const int rows = min(kBM, g.M - i0);
+        for (int r = 0; r < rows; ++r) tc::bulk_prefetch_l2(c0p + (int64_t)r * g.ldc, kBN * 8);
+      }
     }
   } else {
     const int wm = warp >> 1, wn = warp & 1;  // warp grid kWM x 2
     const int gq4 = lane >> 2, t = lane & 3;
     const int rowA = wm * 32 + gq4;   // + mi * 16 (+ 8)
     const int colB = wn * 32 + gq4;   // + nj * 8
+    // Slices that need the zero structure applied: kc >= mask_from (ragged K end, a_lower,
+    // b_upper) or kc < mask_below (b_lower), for this warp's rows and columns.
+    int mask_from = (k_hi - k_lo) / kBK;  // the ragged last slice, if any
+    if (g.a_lower) mask_from = min(mask_from, max(0, (i0 + wm * 32 - k_lo - kBK + 1 + kBK) / kBK));
+    if (g.b_upper) mask_from = min(mask_from, max(0, (j0 + wn * 32 - k_lo - kBK + 1 + kBK) / kBK));
+    const int mask_below = g.b_lower ? (j0 + wn * 32 + 31 - k_lo + kBK - 1) / kBK : 0;
     for (int kc = 0; kc < nk; ++kc) {
       const int s = kc % kStages;
       if (!tc::mbar_wait(&full[s], (kc / kStages) & 1)) {
@@ -157,10 +162,7 @@ __device__ __forceinline__ void dgemm_body(const CUtensorMap& ma, const CUtensor
       }
       const uint8_t* sA = base + s * kStageBytes;
       const uint8_t* sB = sA + kTileA;
-      const int kb = k_lo + kc * kBK;
-      const bool mask = (kb + kBK > k_hi) || (g.a_lower && kb + kBK - 1 > i0 + wm * 32) ||
-                        (g.b_upper && kb + kBK - 1 > j0 + wn * 32) ||
-                        (g.b_lower && kb < j0 + wn * 32 + 31);
+      const bool mask = kc >= mask_from || kc < mask_below;
 #pragma unroll
       for (int kk = 0; kk < 2; ++kk) {
         const int c = (t + 4 * (t & 1)) ^ kk;
@@ -200,7 +202,7 @@ __device__ __forceinline__ void dgemm_body(const CUtensorMap& ma, const CUtensor
           if (lane == 0) tc::mbar_arrive(&empty[s]);
         }
         if (mask) {
-          const int ka = kb + 2 * c, kb1 = ka + 1;
+          const int ka = k_lo + kc * kBK + 2 * c, kb1 = ka + 1;
 #pragma unroll
           for (int mi = 0; mi < 2; ++mi) {
             const int i = i0 + rowA + mi * 16;
@@ -220,7 +222,7 @@ __device__ __forceinline__ void dgemm_body(const CUtensorMap& ma, const CUtensor
 #pragma unroll
         for (int mi = 0; mi < 2; ++mi)
 #pragma unroll
-          for (int nj = 0; nj < 4; ++nj) dmma16x8x8(acc[mi][nj], a[mi], b[nj]);
+          for (int nj = 0; nj < 4; ++nj) tc::dmma_m16n8k8(acc[mi][nj], a[mi], b[nj]);
       }
     }
 
@@ -242,24 +244,36 @@ __device__ __forceinline__ void dgemm_body(const CUtensorMap& ma, const CUtensor
     asm volatile("bar.sync 1, %0;" ::"r"(kCWarps * 32) : "memory");
     double* C = g.C + (int64_t)z * g.strideC;
     const int j = j0 + 2 * lane;
-    for (int r = warp; r < kBM; r += kCWarps) {
-      const int i = i0 + r;
-      if (i >= g.M) break;
-      const double2 a2 = *reinterpret_cast<const double2*>(sC + r * kCPitch + 2 * lane);
-      double* crow = C + (int64_t)i * g.ldc;
-      const double v0 = g.alpha * a2.x, v1 = g.alpha * a2.y;
-      if (g.c_vec && j + 1 < g.N) {
-        double2* p = reinterpret_cast<double2*>(crow + j);
-        double2 o = make_double2(v0, v1);
-        if (g.beta_one) {
-          const double2 c = *p;
-          o.x += c.x;
-          o.y += c.y;
+    constexpr int kRows = kBM / kCWarps;  // rows per warp, all loads in flight together
+    const bool vec = g.c_vec && j + 1 < g.N;
+    double2 cv[kRows];
+#pragma unroll
+    for (int t = 0; t < kRows; ++t) {
+      const int i = i0 + warp + t * kCWarps;
+      cv[t] = make_double2(0.0, 0.0);
+      if (g.beta_one && i < g.M) {
+        const double* crow = C + (int64_t)i * g.ldc;
+        if (vec) {
+          cv[t] = *reinterpret_cast<const double2*>(crow + j);
+        } else {
+          if (j < g.N) cv[t].x = crow[j];
+          if (j + 1 < g.N) cv[t].y = crow[j + 1];
         }
-        *p = o;
-      } else {
-        if (j < g.N) crow[j] = g.beta_one ? crow[j] + v0 : v0;
-        if (j + 1 < g.N) crow[j + 1] = g.beta_one ? crow[j + 1] + v1 : v1;
+      }
+    }
+#pragma unroll
+    for (int t = 0; t < kRows; ++t) {
+      const int r = warp + t * kCWarps, i = i0 + r;
+      if (i < g.M) {
+        const double2 a2 = *reinterpret_cast<const double2*>(sC + r * kCPitch + 2 * lane);
+        double* crow = C + (int64_t)i * g.ldc;
+        const double2 o = make_double2(cv[t].x + g.alpha * a2.x, cv[t].y + g.alpha * a2.y);
+        if (vec) {
+          *reinterpret_cast<double2*>(crow + j) = o;
+        } else {
+          if (j < g.N) crow[j] = o.x;
+          if (j + 1 < g.N) crow[j + 1] = o.y;
+        }
       }
     }
   }

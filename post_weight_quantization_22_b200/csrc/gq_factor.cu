@@ -14,6 +14,7 @@
 // Everything is fp64: the damped Hessians of LLM layers have condition numbers ~1e5 and the
 // codes downstream change when U carries fp32-level errors.
 #include "gq_internal.cuh"
+#include "gq_tc.cuh"
 
 #include <math.h>
 #include <vector>
@@ -23,6 +24,8 @@ namespace gq {
 
 constexpr int kNB = 64;      // Cholesky panel width (the leaf)
 constexpr int kSuper = 256;  // super-panel width (trailing-update depth)
+constexpr int kPnPitch = 68;  // shared-memory pitch (doubles) of the panel kernel's tiles
+constexpr size_t kPnSmem = (size_t)(kNB + 32) * kPnPitch * sizeof(double);
 
 // ---------------------------------------------------------------------------------------
 // dead fix + damping statistics (one CTA)
@@ -88,16 +91,30 @@ __device__ __forceinline__ double recip_newton(double p) {
 // (j <= c), f_r = S[r][c] / S[c][c].  Then A = L_unit^-1, the pivots are D of
 // S = L_unit D L_unit^T, and L^-1 = D^-1/2 A.
 // 256 threads; thread (a, b) = (tid / 16, tid % 16) keeps the 4 x 4 blocks S[4a..4a+3][4b..4b+3]
-// and A[4a..4a+3][4b..4b+3] in registers.  Per pivot, column c of S and row c of A travel
-// through double-buffered shared memory (one barrier); a thread reads 4 multipliers, 4 column
-// values and 4 row values there with 16-byte loads.  The pivot loop is unrolled 4 deep (register
-// indices fixed, the body small enough to stay in the instruction cache).
+// and A[4a..4a+3][4b..4b+3] in registers.  Column c of S and row c of A travel through
+// double-buffered shared memory; a thread reads 4 multipliers, 4 column values and 4 row values
+// there with 16-byte loads.
+// The updates run on whole 4 x 4 blocks without per-entry conditions: after pivot c only the
+// trailing lower triangle S[r][q], c < q <= r, the pivots S[r][r] and A[r][j], j <= c < r, are
+// read again, and every entry outside them (columns <= c, the upper part) only ever feeds other
+// such entries, so whatever they hold does not matter.  Rows r <= c must stay fixed (their
+// pivots are final), so their multipliers are set to 0; A[c][j] is exactly 0 for j > c.
+// Synchronisation is one mbarrier phase per pivot, split into arrive and wait: at pivot c the
+// owners of column c+1 of S and row c+1 of A update those entries first, publish them and
+// arrive; every thread then does the rest of its block update while the phase completes, and
+// waits for it only when it needs pivot c+1.  The per-pivot critical path is load, reciprocal,
+// one FMA and a store.  A row block whose rows are all eliminated leaves with arrive_drop.
+// The pivot loop is unrolled 4 deep (register indices fixed, the body small enough to stay in
+// the instruction cache).  Waits are bounded: a timeout is recorded and the kernel finishes.
 // ---------------------------------------------------------------------------------------
-__global__ void __launch_bounds__(256, 1) potrf_diag_kernel(double* M, int64_t ldm, int64_t c0,
-                                                            int w, WsHeader* hdr) {
+__global__ void __launch_bounds__(256, 1) potrf_panel_kernel(double* M, int64_t ldm, int64_t n,
+                                                             int64_t c0, int w, double* Dinv,
+                                                             WsHeader* hdr) {
+  extern __shared__ __align__(16) double pn_smem[];
   __shared__ __align__(16) double colbuf[2][kNB];
   __shared__ __align__(16) double rowbuf[2][kNB];
   __shared__ double dbuf[kNB];
+  __shared__ __align__(8) uint64_t bar;
   const int tid = threadIdx.x;
   const int a = tid >> 4, b = tid & 15;
   double sv[4][4], av[4][4];
@@ -115,74 +132,158 @@ __global__ void __launch_bounds__(256, 1) potrf_diag_kernel(double* M, int64_t l
       sv[i][j] = v;
       av[i][j] = (q == r) ? 1.0 : 0.0;
     }
+  if (tid == 0) tc::mbar_init(&bar, 256);
+  __syncthreads();
+  // pivot 0's column and row, then phase 0
+  if (b == 0) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) colbuf[0][4 * a + i] = sv[i][0];
+  }
+  if (a == 0) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) rowbuf[0][4 * b + j] = av[0][j];
+  }
+  tc::mbar_arrive(&bar);
+  bool live = true;
 #pragma unroll 1
-  for (int c4 = 0; c4 < kNB / 4; ++c4) {
+  for (int c4 = 0; c4 < kNB / 4 && live; ++c4) {
 #pragma unroll
     for (int cc = 0; cc < 4; ++cc) {
       const int c = 4 * c4 + cc;
-      const int buf = cc & 1;
-      if (b == c4) {
-#pragma unroll
-        for (int i = 0; i < 4; ++i) colbuf[buf][4 * a + i] = sv[i][cc];  // S[.][c]
+      if (!live || c == kNB - 1) break;
+      if (!tc::mbar_wait(&bar, c & 1)) {  // pivot c published
+        record_status(hdr, GQ_ERR_TIMEOUT);
+        live = false;
+        break;
       }
-      if (a == c4) {
-#pragma unroll
-        for (int j = 0; j < 4; ++j) rowbuf[buf][4 * b + j] = av[cc][j];  // A[c][.]
+      if (4 * a + 3 == c) {  // every row of this block is eliminated: leave the protocol
+        tc::mbar_arrive_drop(&bar);
+        live = false;
+        break;
       }
-      __syncthreads();
-      if (4 * a + 3 > c) {
-        double p = colbuf[buf][c];
-        if (!(p > 0.0)) p = 1.0;  // reported below from the final pivots
-        const double rp = recip_newton(p);
-        const double2 f01 = *reinterpret_cast<const double2*>(&colbuf[buf][4 * a]);
-        const double2 f23 = *reinterpret_cast<const double2*>(&colbuf[buf][4 * a + 2]);
-        const double fr[4] = {f01.x * rp, f01.y * rp, f23.x * rp, f23.y * rp};
-        if (4 * b + 3 > c) {  // S: entries with c < q <= r
-          const double2 q01 = *reinterpret_cast<const double2*>(&colbuf[buf][4 * b]);
-          const double2 q23 = *reinterpret_cast<const double2*>(&colbuf[buf][4 * b + 2]);
-          const double cq[4] = {q01.x, q01.y, q23.x, q23.y};
+      const int buf = cc & 1, nbuf = buf ^ 1;
+      const int cn = (cc + 1) & 3;  // column / row index of pivot c+1 inside its 4-block
+      double p = colbuf[buf][c];
+      if (!(p > 0.0)) p = 1.0;  // reported below from the final pivots
+      const double rp = recip_newton(p);
+      const double2 f01 = *reinterpret_cast<const double2*>(&colbuf[buf][4 * a]);
+      const double2 f23 = *reinterpret_cast<const double2*>(&colbuf[buf][4 * a + 2]);
+      const double2 q01 = *reinterpret_cast<const double2*>(&colbuf[buf][4 * b]);
+      const double2 q23 = *reinterpret_cast<const double2*>(&colbuf[buf][4 * b + 2]);
+      const double2 r01 = *reinterpret_cast<const double2*>(&rowbuf[buf][4 * b]);
+      const double2 r23 = *reinterpret_cast<const double2*>(&rowbuf[buf][4 * b + 2]);
+      const double fr[4] = {4 * a + 0 > c ? f01.x * rp : 0.0, 4 * a + 1 > c ? f01.y * rp : 0.0,
+                            4 * a + 2 > c ? f23.x * rp : 0.0, 4 * a + 3 > c ? f23.y * rp : 0.0};
+      const double cq[4] = {q01.x, q01.y, q23.x, q23.y};
+      const double rq[4] = {r01.x, r01.y, r23.x, r23.y};
+      // critical: column c+1 of S and row c+1 of A, published before the rest
+      const bool own_col = (b == ((c + 1) >> 2)), own_row = (a == ((c + 1) >> 2));
+      if (own_col) {
 #pragma unroll
-          for (int i = 0; i < 4; ++i)
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-              if (4 * b + j > c && 4 * b + j <= 4 * a + i) sv[i][j] = fma(-fr[i], cq[j], sv[i][j]);
-        }
-        if (4 * b <= c) {  // A: entries with q <= c < r
-          const double2 r01 = *reinterpret_cast<const double2*>(&rowbuf[buf][4 * b]);
-          const double2 r23 = *reinterpret_cast<const double2*>(&rowbuf[buf][4 * b + 2]);
-          const double rq[4] = {r01.x, r01.y, r23.x, r23.y};
-#pragma unroll
-          for (int i = 0; i < 4; ++i)
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-              if (4 * b + j <= c && 4 * a + i > c) av[i][j] = fma(-fr[i], rq[j], av[i][j]);
+        for (int i = 0; i < 4; ++i) {
+          sv[i][cn] = fma(-fr[i], cq[cn], sv[i][cn]);
+          colbuf[nbuf][4 * a + i] = sv[i][cn];
         }
       }
+      if (own_row) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          av[cn][j] = fma(-fr[cn], rq[j], av[cn][j]);
+          rowbuf[nbuf][4 * b + j] = av[cn][j];
+        }
+      }
+      tc::mbar_arrive(&bar);
+      // the rest of the block update, overlapped with the next phase
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          if (!(own_col && j == cn)) sv[i][j] = fma(-fr[i], cq[j], sv[i][j]);
+          if (!(own_row && i == cn)) av[i][j] = fma(-fr[i], rq[j], av[i][j]);
+        }
     }
   }
+  __syncthreads();
   // pivots D_r = S[r][r], held by the diagonal threads
   if (a == b) {
 #pragma unroll
     for (int i = 0; i < 4; ++i) dbuf[4 * a + i] = sv[i][i];
   }
   __syncthreads();
+  // L11^-1 = D^-1/2 A (lower; zero above) into shared memory, and by CTA 0 into the leaf
+  // buffer (not into the diagonal block itself: other CTAs may still be reading that block for
+  // their own copy of the leaf)
+  double* sL = pn_smem;                   // 64 x kPnPitch
+  double* sP = pn_smem + kNB * kPnPitch;  // 32 x kPnPitch: a chunk of the panel below
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     const int r = 4 * a + i;
     double d = dbuf[r];
     if (!(d > 0.0)) {
-      if (r < w && b == 0) record_status(hdr, GQ_ERR_NOT_PD);
+      if (r < w && b == 0 && blockIdx.x == 0) record_status(hdr, GQ_ERR_NOT_PD);
       d = 1.0;
     }
     const double rs = 1.0 / sqrt(d);
-    if (r < w) {
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int q = 4 * b + j;
-        if (q <= r) M[(c0 + r) * ldm + c0 + q] = av[i][j] * rs;
-      }
+    for (int j = 0; j < 4; ++j) {
+      const int q = 4 * b + j;
+      const double v = q <= r ? av[i][j] * rs : 0.0;
+      sL[r * kPnPitch + q] = v;
+      if (blockIdx.x == 0) Dinv[r * kNB + q] = v;
     }
   }
+  // Panel below (w == 64 whenever rows remain): P <- P L11^-T, in place, in chunks of 32 rows
+  // spread over the CTAs.  Each warp computes one m16 x (2 x n8) part of the 32 x 64 chunk with
+  // fp64 MMAs; the padded pitch makes the fragment loads conflict-free.
+  const int64_t rem = n - c0 - w;
+  if (rem <= 0) return;
+  const int warp = tid >> 5, lane = tid & 31, g = lane >> 2, t = lane & 3;
+  const int mi = warp & 1, np = warp >> 1;
+  const int64_t nch = (rem + 31) / 32;
+  for (int64_t ch = blockIdx.x; ch < nch; ch += gridDim.x) {
+    const int64_t r0 = c0 + w + ch * 32;
+    __syncthreads();  // sL written / the previous chunk consumed
+    for (int e = tid; e < 32 * 32; e += 256) {
+      const int rr = e >> 5, cc2 = (e & 31) * 2;
+      double2 v = make_double2(0.0, 0.0);
+      if (r0 + rr < n) v = *reinterpret_cast<const double2*>(M + (r0 + rr) * ldm + c0 + cc2);
+      *reinterpret_cast<double2*>(sP + rr * kPnPitch + cc2) = v;
+    }
+    __syncthreads();
+    double acc[2][4] = {{0.0, 0.0, 0.0, 0.0}, {0.0, 0.0, 0.0, 0.0}};
+#pragma unroll
+    for (int kb = 0; kb < kNB; kb += 8) {
+      const double* pa = sP + (mi * 16 + g) * kPnPitch + kb + t;
+      const double af[4] = {pa[0], pa[8 * kPnPitch], pa[4], pa[8 * kPnPitch + 4]};
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const double* pb = sL + ((2 * np + u) * 8 + g) * kPnPitch + kb + t;
+        const double bf[2] = {pb[0], pb[4]};
+        tc::dmma_m16n8k8(acc[u], af, bf);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 2; ++u)
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int64_t row = r0 + mi * 16 + g + 8 * h;
+        if (row < n)
+          *reinterpret_cast<double2*>(M + row * ldm + c0 + (2 * np + u) * 8 + 2 * t) =
+              make_double2(acc[u][2 * h], acc[u][2 * h + 1]);
+      }
+  }
+}
+
+// Diagonal 64-blocks of [r0, r0 + w) <- the inverted leaves (lower parts), once every panel
+// kernel of the range has finished.
+__global__ void place_leaves_kernel(double* M, int64_t ldm, const double* Dinv, int64_t r0,
+                                    int64_t w) {
+  const int64_t r = blockIdx.x;  // row inside the range
+  const int q = threadIdx.x;     // column inside the row's 64-block
+  if (r >= w) return;
+  const int64_t b0 = (r / kNB) * kNB;  // block start inside the range
+  const int64_t rr = r - b0;
+  if (q <= rr) M[(r0 + r) * ldm + r0 + b0 + q] = Dinv[((r0 + b0) / kNB) * kNB * kNB + rr * kNB + q];
 }
 
 // U[i][j] = (i <= j) ? (float) Linv[n-1-i][n-1-j] : 0
@@ -205,15 +306,18 @@ static int64_t m_ld(int64_t n) { return (n + 15) / 16 * 16; }
 struct PrepLayout {
   WsHeader* hdr;
   double* M;     // n x ldm: lower triangle = J P H_d P J, then the inverse of its Cholesky factor
-  double* tbuf;  // doubling scratch of the triangular inverse
+  double* T;     // n x ldm: block rows of L X accumulated for the inverse (lower blocks)
+  double* Dinv;  // ceil(n / 64) x 64 x 64: the inverted 64-wide leaves
+  double* tbuf;  // doubling scratch of the diagonal super-block inverses
   size_t bytes;
 };
 
-static size_t trtri_tbuf_elems(int64_t n) {
+// doubling scratch for one diagonal block of width w (<= kSuper)
+static size_t trtri_tbuf_elems(int64_t w) {
   size_t best = 0;
-  for (int64_t bs = kNB; bs < n; bs *= 2) {
+  for (int64_t bs = kNB; bs < w; bs *= 2) {
     size_t tot = 0;
-    for (int64_t r = 0; r + bs < n; r += 2 * bs) tot += (size_t)bs * bs;
+    for (int64_t r = 0; r + bs < w; r += 2 * bs) tot += (size_t)bs * bs;
     best = std::max(best, tot);
   }
   return best;
@@ -224,14 +328,21 @@ static PrepLayout prep_layout(void* ws, int64_t n) {
   PrepLayout L;
   L.hdr = c.take<WsHeader>(1);
   L.M = c.take<double>((size_t)n * m_ld(n));
-  L.tbuf = c.take<double>(trtri_tbuf_elems(n) + 1);
+  L.T = c.take<double>((size_t)n * m_ld(n));
+  L.Dinv = c.take<double>((size_t)((n + kNB - 1) / kNB) * kNB * kNB);
+  L.tbuf = c.take<double>(trtri_tbuf_elems(kSuper) + 1);
   L.bytes = c.off;
   return L;
 }
 
 size_t prepare_ws_bytes(int64_t n) { return prep_layout(nullptr, n).bytes; }
 
-cudaError_t factor_init_attributes() { return dgemm_init_attributes(); }
+cudaError_t factor_init_attributes() {
+  cudaError_t e = cudaFuncSetAttribute(potrf_panel_kernel,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kPnSmem);
+  if (e != cudaSuccess) return e;
+  return dgemm_init_attributes();
+}
 
 #define GQ_TRY(x)                               \
   do {                                          \
@@ -239,10 +350,102 @@ cudaError_t factor_init_attributes() { return dgemm_init_attributes(); }
     if (_e != cudaSuccess) return _e;           \
   } while (0)
 
+// Inverse of the diagonal block [r0, r0 + w) of L (w <= kSuper) from its inverted 64-wide
+// leaves, by doubling: inv([[A, 0], [B, C]]) = [[A^-1, 0], [-C^-1 B A^-1, C^-1]], all pairs of
+// a level batched.
+static cudaError_t invert_diag_block(double* M, int64_t n, int64_t ldm, int64_t r0, int64_t w,
+                                     const double* Dinv, double* tbuf, WsHeader* hdr,
+                                     cudaStream_t s) {
+  place_leaves_kernel<<<(unsigned)w, kNB, 0, s>>>(M, ldm, Dinv, r0, w);
+  count_launches(1);
+  {
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  for (int64_t bs = kNB; bs < w; bs *= 2) {
+    const int64_t npairs_full = w / (2 * bs);
+    const int64_t rtail = npairs_full * 2 * bs;
+    const int64_t cw_tail = w - rtail - bs;
+    for (int pass = 0; pass < 2; ++pass) {
+      const int64_t r = r0 + (pass == 0 ? 0 : rtail);
+      const int64_t cw = pass == 0 ? bs : cw_tail;
+      const int64_t batch = pass == 0 ? npairs_full : (cw_tail > 0 ? 1 : 0);
+      if (batch <= 0 || cw <= 0) continue;
+      double* tb = tbuf + (pass == 0 ? 0 : npairs_full * bs * bs);
+      {  // T = B A^-1
+        DgemmCall g{};
+        g.M = (int)cw; g.N = (int)bs; g.K = (int)bs; g.batch = (int)batch; g.alpha = 1.0;
+        g.beta_one = 0;
+        g.A = DgemmOperand{M, n, n, ldm, r + bs, r, 2 * bs, 2 * bs};
+        g.B = DgemmOperand{M, n, n, ldm, r, r, 2 * bs, 2 * bs}; g.b_nmajor = 1; g.b_lower = 1;
+        g.C = tb; g.ldc = bs; g.strideC = bs * bs; g.hdr = hdr;
+        cudaError_t e = launch_dgemm(g, s);
+        if (e != cudaSuccess) return e;
+      }
+      {  // B <- -C^-1 T
+        DgemmCall g{};
+        g.M = (int)cw; g.N = (int)bs; g.K = (int)cw; g.batch = (int)batch; g.alpha = -1.0;
+        g.beta_one = 0;
+        g.A = DgemmOperand{M, n, n, ldm, r + bs, r + bs, 2 * bs, 2 * bs}; g.a_lower = 1;
+        g.B = DgemmOperand{tb, batch * bs, bs, bs, 0, 0, bs, 0}; g.b_nmajor = 1;
+        g.C = M + (r + bs) * ldm + r; g.ldc = ldm; g.strideC = 2 * bs * ldm + 2 * bs;
+        g.hdr = hdr;
+        cudaError_t e = launch_dgemm(g, s);
+        if (e != cudaSuccess) return e;
+      }
+    }
+  }
+  return cudaSuccess;
+}
+
+// Three streams per call, forked from and joined back into the caller's stream:
+//   A (highest priority): the latency-bound chain (leaf + panel solve kernels, the in-panel
+//     updates, and the trailing update of the next super-panel's columns);
+//   B: the trailing update of all later columns, overlapped with the next super-panel's chain;
+//   C (lowest priority): the block rows of the triangular inverse, each started as soon as
+//     its super-panel is factored.
+// One set per host thread and device, created on first use and kept.
+struct PrepStreams {
+  bool ready = false;
+  cudaStream_t a = nullptr, b = nullptr, c = nullptr;
+  cudaEvent_t fork = nullptr, panel[2] = {}, far[2] = {}, join[3] = {};
+};
+thread_local PrepStreams t_prep_streams[128];
+
+static cudaError_t prep_streams(PrepStreams** out) {
+  int dev = 0;
+  GQ_TRY(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= 128) return cudaErrorInvalidDevice;
+  PrepStreams& p = t_prep_streams[dev];
+  if (!p.ready) {
+    int least = 0, greatest = 0;
+    GQ_TRY(cudaDeviceGetStreamPriorityRange(&least, &greatest));
+    GQ_TRY(cudaStreamCreateWithPriority(&p.a, cudaStreamNonBlocking, greatest));
+    GQ_TRY(cudaStreamCreateWithPriority(&p.b, cudaStreamNonBlocking, (least + greatest) / 2));
+    GQ_TRY(cudaStreamCreateWithPriority(&p.c, cudaStreamNonBlocking, least));
+    cudaEvent_t* evs[] = {&p.fork, &p.panel[0], &p.panel[1], &p.far[0], &p.far[1],
+                          &p.join[0], &p.join[1], &p.join[2]};
+    for (cudaEvent_t* e : evs) GQ_TRY(cudaEventCreateWithFlags(e, cudaEventDisableTiming));
+    p.ready = true;
+  }
+  *out = &p;
+  return cudaSuccess;
+}
+
 cudaError_t launch_prepare(const double* H, int64_t n, double damp, int reverse, float* U,
-                           uint8_t* dead, double* delta, void* ws, cudaStream_t s) {
+                           uint8_t* dead, double* delta, void* ws, cudaStream_t s0) {
   PrepLayout L = prep_layout(ws, n);
   const int64_t ldm = m_ld(n);
+  int dev = 0, sms = 148;
+  GQ_TRY(cudaGetDevice(&dev));
+  GQ_TRY(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
+  PrepStreams* ps = nullptr;
+  GQ_TRY(prep_streams(&ps));
+  cudaStream_t s = ps->a, sb = ps->b, sc = ps->c;
+  GQ_TRY(cudaEventRecord(ps->fork, s0));
+  GQ_TRY(cudaStreamWaitEvent(s, ps->fork, 0));
+  GQ_TRY(cudaStreamWaitEvent(sb, ps->fork, 0));
+  GQ_TRY(cudaStreamWaitEvent(sc, ps->fork, 0));
   GQ_TRY(cudaMemsetAsync(L.hdr, 0, sizeof(WsHeader), s));
   diag_stats_kernel<<<1, 1024, 0, s>>>(H, n, damp, dead, delta, L.hdr);
   count_launches(1);
@@ -258,33 +461,73 @@ cudaError_t launch_prepare(const double* H, int64_t n, double damp, int reverse,
   auto Mop = [&](int64_t row0, int64_t col0, int64_t zrow = 0, int64_t zcol = 0) {
     return DgemmOperand{L.M, n, n, ldm, row0, col0, zrow, zcol};
   };
+  auto Top = [&](int64_t row0, int64_t col0) {
+    return DgemmOperand{L.T, n, n, ldm, row0, col0, 0, 0};
+  };
+  // Block row [k0, k1) of the triangular inverse X = L^-1 (stream C):
+  //   X_KK = L_KK^-1 (doubling over the inverted 64-wide leaves inside the block),
+  //   X[K, :k0] = -X_KK T[K, :k0],   T[K, J] = sum_{J <= I < K} L[K, I] X[I, J],
+  // with T accumulated right-looking once X's block row K is known:
+  //   T[i >= k1, K] = L[i, K] X_KK,   T[i >= k1, :k0] += L[i, K] X[K, :k0]   (K = 256 GEMMs).
+  // X overwrites L in place: block row K of L is not read by the Cholesky after block K.
+  auto inverse_block_row = [&](int64_t k0, int64_t k1) -> cudaError_t {
+    const int64_t kw = k1 - k0;
+    GQ_TRY(invert_diag_block(L.M, n, ldm, k0, kw, L.Dinv, L.tbuf, L.hdr, sc));
+    if (k0 > 0) {  // X[K, :k0] = -X_KK T[K, :k0]
+      DgemmCall g{};
+      g.M = (int)kw; g.N = (int)k0; g.K = (int)kw; g.batch = 1; g.alpha = -1.0; g.beta_one = 0;
+      g.A = Mop(k0, k0); g.a_lower = 1;
+      g.B = Top(k0, 0); g.b_nmajor = 1;
+      g.C = L.M + k0 * ldm; g.ldc = ldm; g.hdr = L.hdr;
+      GQ_TRY(launch_dgemm(g, sc));
+    }
+    if (k1 < n) {
+      {  // T[k1:, K] = L[k1:, K] X_KK
+        DgemmCall g{};
+        g.M = (int)(n - k1); g.N = (int)kw; g.K = (int)kw; g.batch = 1; g.alpha = 1.0;
+        g.beta_one = 0;
+        g.A = Mop(k1, k0);
+        g.B = Mop(k0, k0); g.b_nmajor = 1; g.b_lower = 1;
+        g.C = L.T + k1 * ldm + k0; g.ldc = ldm; g.hdr = L.hdr;
+        GQ_TRY(launch_dgemm(g, sc));
+      }
+      if (k0 > 0) {  // T[k1:, :k0] += L[k1:, K] X[K, :k0]
+        DgemmCall g{};
+        g.M = (int)(n - k1); g.N = (int)k0; g.K = (int)kw; g.batch = 1; g.alpha = 1.0;
+        g.beta_one = 1;
+        g.A = Mop(k1, k0);
+        g.B = Mop(k0, 0); g.b_nmajor = 1;
+        g.C = L.T + k1 * ldm; g.ldc = ldm; g.hdr = L.hdr;
+        GQ_TRY(launch_dgemm(g, sc));
+      }
+    }
+    return cudaSuccess;
+  };
   // Blocked right-looking Cholesky of M (lower, in place), 64-wide panels grouped into
-  // 256-wide super-panels.  For each 64-wide panel: the diagonal block is replaced by the
-  // inverse of its factor (leaf), the rows below become L21 = A21 L11^-T, and only the rest of
-  // the super-panel takes the update A -= L21 L21^T.  The columns after the super-panel take
-  // one K = 256 update per super-panel (fewer, larger fp64 tensor-core GEMMs, 4x less
-  // read-modify-write traffic on the trailing matrix than 64-wide steps).
+  // 256-wide super-panels (stream A).  For each 64-wide panel one kernel replaces the diagonal
+  // block by the inverse of its factor (leaf) and the rows below by L21 = A21 L11^-T; then only
+  // the rest of the super-panel takes the update A -= L21 L21^T.  After a super-panel, the
+  // trailing matrix takes one K = 256 update: the next super-panel's columns on A, all later
+  // columns on B, overlapped with the next super-panel's chain (look-ahead of one).
   const int64_t nb = (n + kNB - 1) / kNB;
+  int sidx = 0;
+  bool far_pending = false;
   for (int64_t k = 0; k < nb; ++k) {
     const int64_t c0 = k * kNB;
     const int w = (int)std::min<int64_t>(kNB, n - c0);
     const int64_t sp0 = (c0 / kSuper) * kSuper;                 // super-panel start
     const int64_t sp1 = std::min<int64_t>(sp0 + kSuper, n);     // super-panel end
-    potrf_diag_kernel<<<1, 256, 0, s>>>(L.M, ldm, c0, w, L.hdr);
-    count_launches(1);
-    GQ_TRY(cudaGetLastError());
     const int64_t rem = n - c0 - w;
-    if (rem <= 0) continue;
-    {  // P <- P (L11^-1)^T, in place: each CTA owns whole rows of P (N = w = one tile)
-      DgemmCall g{};
-      g.M = (int)rem; g.N = w; g.K = w; g.batch = 1; g.alpha = 1.0; g.beta_one = 0;
-      g.A = Mop(c0 + w, c0);
-      g.B = Mop(c0, c0); g.b_nmajor = 0; g.b_upper = 1;  // opB[k][j] = L11^-1[j][k]
-      g.C = L.M + (c0 + w) * ldm + c0; g.ldc = ldm; g.hdr = L.hdr;
-      GQ_TRY(launch_dgemm(g, s));
+    {  // leaf (every CTA) + P <- P L11^-T for the rows below, one wave of CTAs
+      const int64_t nch = rem > 0 ? (rem + 31) / 32 : 1;
+      const int grid = (int)std::min<int64_t>(nch, sms);
+      potrf_panel_kernel<<<grid, 256, kPnSmem, s>>>(L.M, ldm, n, c0, w,
+                                                    L.Dinv + (c0 / kNB) * kNB * kNB, L.hdr);
+      count_launches(1);
+      GQ_TRY(cudaGetLastError());
     }
     const int64_t inw = sp1 - (c0 + w);  // columns of the super-panel after this panel
-    if (inw > 0) {  // A[:, c0+w : sp1] -= L21 L21[c0+w : sp1]^T for every row below
+    if (rem > 0 && inw > 0) {  // A[:, c0+w : sp1] -= L21 L21[c0+w : sp1]^T for every row below
       DgemmCall g{};
       g.M = (int)rem; g.N = (int)inw; g.K = w; g.batch = 1; g.alpha = -1.0; g.beta_one = 1;
       g.A = Mop(c0 + w, c0);
@@ -292,56 +535,52 @@ cudaError_t launch_prepare(const double* H, int64_t n, double damp, int reverse,
       g.C = L.M + (c0 + w) * ldm + (c0 + w); g.ldc = ldm; g.lower_tiles = 1; g.hdr = L.hdr;
       GQ_TRY(launch_dgemm(g, s));
     }
-    if (c0 + w == sp1 && sp1 < n) {  // super-panel done: trailing update with K = its width
-      const int64_t trem = n - sp1, kw = sp1 - sp0;
-      DgemmCall g{};
-      g.M = (int)trem; g.N = (int)trem; g.K = (int)kw; g.batch = 1; g.alpha = -1.0;
-      g.beta_one = 1;
-      g.A = Mop(sp1, sp0);
-      g.B = Mop(sp1, sp0); g.b_nmajor = 0;
-      g.C = L.M + sp1 * ldm + sp1; g.ldc = ldm; g.lower_tiles = 1; g.hdr = L.hdr;
-      GQ_TRY(launch_dgemm(g, s));
-    }
-  }
-  // Triangular inverse by doubling over the diagonal blocks (already inverted):
-  //   inv([[A, 0], [B, C]]) = [[A^-1, 0], [-C^-1 B A^-1, C^-1]], all pairs of a level batched.
-  for (int64_t bs = kNB; bs < n; bs *= 2) {
-    const int64_t npairs_full = n / (2 * bs);
-    const int64_t rtail = npairs_full * 2 * bs;
-    const int64_t cw_tail = n - rtail - bs;
-    for (int pass = 0; pass < 2; ++pass) {
-      int64_t r = pass == 0 ? 0 : rtail;
-      int64_t cw = pass == 0 ? bs : cw_tail;
-      int64_t batch = pass == 0 ? npairs_full : (cw_tail > 0 ? 1 : 0);
-      if (batch <= 0 || cw <= 0) continue;
-      double* tb = L.tbuf + (pass == 0 ? 0 : npairs_full * bs * bs);
-      {  // T = B A^-1
+    if (c0 + w != sp1) continue;
+    // super-panel [sp0, sp1) factored
+    cudaEvent_t ev_panel = ps->panel[sidx & 1];
+    GQ_TRY(cudaEventRecord(ev_panel, s));
+    GQ_TRY(cudaStreamWaitEvent(sc, ev_panel, 0));
+    GQ_TRY(inverse_block_row(sp0, sp1));
+    if (sp1 < n) {
+      const int64_t sp2 = std::min<int64_t>(sp1 + kSuper, n), kw = sp1 - sp0;
+      if (far_pending) GQ_TRY(cudaStreamWaitEvent(s, ps->far[(sidx - 1) & 1], 0));
+      {  // next super-panel's columns: A[sp1:, sp1:sp2] -= L[sp1:, SP] L[sp1:sp2, SP]^T
         DgemmCall g{};
-        g.M = (int)cw; g.N = (int)bs; g.K = (int)bs; g.batch = (int)batch; g.alpha = 1.0;
-        g.beta_one = 0;
-        g.A = Mop(r + bs, r, 2 * bs, 2 * bs);
-        g.B = Mop(r, r, 2 * bs, 2 * bs); g.b_nmajor = 1; g.b_lower = 1;
-        g.C = tb; g.ldc = bs; g.strideC = bs * bs; g.hdr = L.hdr;
+        g.M = (int)(n - sp1); g.N = (int)(sp2 - sp1); g.K = (int)kw; g.batch = 1;
+        g.alpha = -1.0; g.beta_one = 1;
+        g.A = Mop(sp1, sp0);
+        g.B = Mop(sp1, sp0); g.b_nmajor = 0;
+        g.C = L.M + sp1 * ldm + sp1; g.ldc = ldm; g.lower_tiles = 1; g.hdr = L.hdr;
         GQ_TRY(launch_dgemm(g, s));
       }
-      {  // B <- -C^-1 T
+      far_pending = false;
+      if (sp2 < n) {  // later columns, stream B: A[sp2:, sp2:] -= L[sp2:, SP] L[sp2:, SP]^T
+        GQ_TRY(cudaStreamWaitEvent(sb, ev_panel, 0));
         DgemmCall g{};
-        g.M = (int)cw; g.N = (int)bs; g.K = (int)cw; g.batch = (int)batch; g.alpha = -1.0;
-        g.beta_one = 0;
-        g.A = Mop(r + bs, r + bs, 2 * bs, 2 * bs); g.a_lower = 1;
-        g.B = DgemmOperand{tb, batch * bs, bs, bs, 0, 0, bs, 0}; g.b_nmajor = 1;
-        g.C = L.M + (r + bs) * ldm + r; g.ldc = ldm; g.strideC = 2 * bs * ldm + 2 * bs;
-        g.hdr = L.hdr;
-        GQ_TRY(launch_dgemm(g, s));
+        g.M = (int)(n - sp2); g.N = (int)(n - sp2); g.K = (int)kw; g.batch = 1;
+        g.alpha = -1.0; g.beta_one = 1;
+        g.A = Mop(sp2, sp0);
+        g.B = Mop(sp2, sp0); g.b_nmajor = 0;
+        g.C = L.M + sp2 * ldm + sp2; g.ldc = ldm; g.lower_tiles = 1; g.hdr = L.hdr;
+        GQ_TRY(launch_dgemm(g, sb));
+        GQ_TRY(cudaEventRecord(ps->far[sidx & 1], sb));
+        far_pending = true;
       }
     }
+    ++sidx;
   }
+  GQ_TRY(cudaEventRecord(ps->join[1], sb));
+  GQ_TRY(cudaEventRecord(ps->join[2], sc));
+  GQ_TRY(cudaStreamWaitEvent(s, ps->join[1], 0));
+  GQ_TRY(cudaStreamWaitEvent(s, ps->join[2], 0));
   {
     dim3 grid((unsigned)((n + 255) / 256), (unsigned)n);
     flip_to_u_kernel<<<grid, 256, 0, s>>>(L.M, n, ldm, U);
     count_launches(1);
     GQ_TRY(cudaGetLastError());
   }
+  GQ_TRY(cudaEventRecord(ps->join[0], s));
+  GQ_TRY(cudaStreamWaitEvent(s0, ps->join[0], 0));
   return cudaSuccess;
 }
 

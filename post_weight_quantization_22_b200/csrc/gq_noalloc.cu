@@ -8,7 +8,7 @@
 // buffers.  Such a caller cannot provide the n x n fp64 workspace gq_prepare_hinv needs.  This
 // entry point uses a scratch area compiled into the library instead: a file-scope static
 // device array, sized for layers up to kStaticMaxN input features.  Every GPU that loads the
-// library holds that array (about 11 MB) until the process exits.
+// library holds that array (about 17 MB) until the process exits.
 //
 // The same kernels run as in gq_prepare_hinv, in the same order, on the caller's stream; only
 // the scratch address differs.
@@ -19,7 +19,7 @@
 namespace {
 
 constexpr int64_t kStaticMaxN = 1024;
-constexpr size_t kStaticBytes = size_t(11) << 20;  // >= the workspace of width kStaticMaxN
+constexpr size_t kStaticBytes = size_t(17) << 20;  // >= the workspace of width kStaticMaxN
 
 // One scratch area per device that loads the library, shared by every call on that device.
 static __device__ __align__(256) unsigned char g_prepare_scratch[kStaticBytes];

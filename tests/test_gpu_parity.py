@@ -183,3 +183,32 @@ def test_qproj_full_size_sampled_rows():
     h = torch.from_numpy(o["H"]).cuda()
     proxy = 0.5 * float(torch.sum((d @ h) * d))
     assert abs(g["loss"][0] - proxy) <= LOSS_REL * proxy
+
+
+@pytest.mark.parametrize("n", [1000, 2304])
+def test_prepare_replays_identical_under_load(n):
+    """The factorisation runs on three streams; repeated calls (graph replays) of the same
+    prepare, each while another stream keeps the SMs busy with unrelated GEMMs, must give
+    bit-identical U with a clean status, and U must match the oracle."""
+    from post_weight_quantization_22_b200 import gq as G
+    _, X, _ = synth.workload("q_proj_4096x4096", m=8, n=n, T=n + 512)
+    H = torch.zeros((n, n), dtype=torch.float64, device="cuda")
+    G.gq_hessian_accumulate(H, X.cuda())
+    busy = torch.cuda.Stream()
+    a = torch.randn(4096, 4096, device="cuda")
+    U0, dead, delta, ws = G.gq_prepare_hinv(H, 0.01)
+    torch.cuda.synchronize()
+    assert G.gq_workspace_status(ws)[0] == 0
+    U0 = U0.clone()
+    for it in range(4):
+        with torch.cuda.stream(busy):
+            for _ in range(8):
+                a = torch.tanh(a @ a.T * 1e-3)
+        U, _, _, _ = G.gq_prepare_hinv(H, 0.01, ws=ws)
+        torch.cuda.synchronize()
+        assert G.gq_workspace_status(ws)[0] == 0, it
+        assert torch.equal(U, U0), it
+    Hn = H.cpu().numpy()
+    hfix, _, _ = O.fix_dead_features(Hn, np.zeros((1, n)))
+    hd, _ = O.dampen(hfix, 0.01)
+    assert rel_fro(np.triu(U0.cpu().numpy()), O.hinv_upper_factor(hd)) <= U_REL_DESIGN
