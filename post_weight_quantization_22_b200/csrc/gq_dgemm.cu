@@ -96,7 +96,7 @@ __device__ __forceinline__ void dgemm_body(const CUtensorMap& ma, const CUtensor
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) {
       tc::mbar_init(&full[s], 1);
-      tc::mbar_init(&empty[s], kCWarps);
+      tc::mbar_init(&empty[s], kCWarps * 32);
     }
     tc::fence_barrier_init();
   }
@@ -197,9 +197,13 @@ __device__ __forceinline__ void dgemm_body(const CUtensorMap& ma, const CUtensor
                 p + kb1 * 128 + ((((nn >> 1) ^ (kb1 & 7))) << 4));
           }
         }
-        if (kk == 1) {  // the whole slice is in registers: release the stage
-          __syncwarp();
-          if (lane == 0) tc::mbar_arrive(&empty[s]);
+        if (kk == 1) {
+          // The whole slice is in registers: release the stage.  Every lane arrives for its own
+          // shared-memory reads, after a proxy fence, so the producer's next TMA write into the
+          // stage (async proxy) cannot overtake any lane's fragment loads (generic proxy).  A
+          // single arrive per warp after __syncwarp let that write land early under load.
+          tc::fence_proxy_async_smem();
+          tc::mbar_arrive(&empty[s]);
         }
         if (mask) {
           const int ka = k_lo + kc * kBK + 2 * c, kb1 = ka + 1;

@@ -56,6 +56,10 @@ __global__ void __launch_bounds__(128, 1)
   const uint32_t tmem = *tslot;
   constexpr int NK = 128 / kLBK;
 
+  const int64_t row = (int64_t)tile_m * 128 + warp * 32 + lane;
+  const int64_t colt = (int64_t)j1 + tile_n * 128;  // first column of this tile
+  float* wrow = Wf + row * n + colt;
+  const bool vec = ((reinterpret_cast<uintptr_t>(Wf) & 15) == 0) && (n % 4 == 0);
   if (warp == 0 && lane == 0) {
     // producer
     for (int kc = 0; kc < NK; ++kc) {
@@ -74,6 +78,12 @@ __global__ void __launch_bounds__(128, 1)
         tc::tma_load_2d(st + 2 * kLTile + g * 4096, &m_bhi, &full[s], x, y);
         tc::tma_load_2d(st + 3 * kLTile + g * 4096, &m_blo, &full[s], x, y);
       }
+    }
+    // the epilogue's read-modify-write tile: into L2 while the MMAs run
+    if (vec && colt + 128 <= n) {
+      const int64_t r0 = (int64_t)tile_m * 128;
+      const int rows = (int)min((int64_t)128, k_rows - r0);
+      for (int r = 0; r < rows; ++r) tc::bulk_prefetch_l2(Wf + (r0 + r) * n + colt, 512);
     }
   } else if (warp == 1 && lane == 0) {
     // MMA issuer
@@ -102,31 +112,43 @@ __global__ void __launch_bounds__(128, 1)
   }
   __syncwarp();
 
-  // epilogue: TMEM lane = tile row, 4 x 32 columns
+  // Epilogue: TMEM lane = tile row, 4 chunks of 32 columns; row = this thread's row.  The work
+  // matrix values of the first two chunks are loaded before the accumulator is waited for, so
+  // their latency overlaps the MMAs; each later chunk's load is issued two chunks ahead.
+  const bool full_row = row < k_rows && colt + 128 <= n && vec;
+  float4 wv[2][8];
+  if (full_row) {
+#pragma unroll
+    for (int c = 0; c < 2; ++c)
+#pragma unroll
+      for (int i = 0; i < 8; ++i) wv[c][i] = *reinterpret_cast<const float4*>(wrow + c * 32 + 4 * i);
+  }
   bool ok = tc::mbar_wait(accum, 0);
   if (!ok && lane == 0) record_status(hdr, GQ_ERR_TIMEOUT);
   tc::fence_after_sync();
-  const int64_t row = (int64_t)tile_m * 128 + warp * 32 + lane;
   if (ok) {
-#pragma unroll 1
+#pragma unroll
     for (int cc = 0; cc < 4; ++cc) {
       float v[32];
       tc::tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + cc * 32, v);
-      const int64_t col0 = (int64_t)j1 + tile_n * 128 + cc * 32;
-      if (row < k_rows && col0 < n) {
-        float* dst = Wf + row * n + col0;
-        if (col0 + 32 <= n && ((reinterpret_cast<uintptr_t>(dst) & 15) == 0)) {
+      const int64_t col0 = colt + cc * 32;
+      if (full_row) {
 #pragma unroll
-          for (int i = 0; i < 32; i += 4) {
-            float4 w = *reinterpret_cast<float4*>(dst + i);
-            w.x -= v[i]; w.y -= v[i + 1]; w.z -= v[i + 2]; w.w -= v[i + 3];
-            *reinterpret_cast<float4*>(dst + i) = w;
-          }
-        } else {
-#pragma unroll
-          for (int i = 0; i < 32; ++i)
-            if (col0 + i < n) dst[i] -= v[i];
+        for (int i = 0; i < 8; ++i) {
+          float4 w = wv[cc & 1][i];
+          w.x -= v[4 * i]; w.y -= v[4 * i + 1]; w.z -= v[4 * i + 2]; w.w -= v[4 * i + 3];
+          *reinterpret_cast<float4*>(wrow + cc * 32 + 4 * i) = w;
         }
+        if (cc + 2 < 4) {
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            wv[cc & 1][i] = *reinterpret_cast<const float4*>(wrow + (cc + 2) * 32 + 4 * i);
+        }
+      } else if (row < k_rows && col0 < n) {
+        float* dst = Wf + row * n + col0;
+#pragma unroll
+        for (int i = 0; i < 32; ++i)
+          if (col0 + i < n) dst[i] -= v[i];
       }
     }
   }
@@ -193,9 +215,10 @@ cudaError_t lazy_tc_make_maps(LazyTcMaps* maps, const float* Ehi, const float* E
 }
 
 cudaError_t launch_lazy_tc(const LazyTcMaps& maps, float* Wf, int64_t n, int64_t k_rows,
-                           int64_t j0, int64_t j1, WsHeader* hdr, cudaStream_t s) {
-  if (j1 >= n || k_rows <= 0) return cudaSuccess;
-  dim3 grid((unsigned)((n - j1 + 127) / 128), (unsigned)((k_rows + 127) / 128));
+                           int64_t j0, int64_t j1, int64_t jend, WsHeader* hdr, cudaStream_t s) {
+  if (jend > n) jend = n;
+  if (j1 >= jend || k_rows <= 0) return cudaSuccess;
+  dim3 grid((unsigned)((jend - j1 + 127) / 128), (unsigned)((k_rows + 127) / 128));
   lazy_tc_kernel<<<grid, 128, kLSmem, s>>>(maps.ahi, maps.alo, maps.bhi, maps.blo, Wf, n, k_rows,
                                            (int)j0, (int)j1, hdr);
   count_launches(1);

@@ -32,8 +32,8 @@ constexpr uint32_t kBulkChunk = 32768;
 struct QLayout {
   WsHeader* hdr;
   float* Wf;        // k x n work matrix (compact rows)
-  float* Ehi;       // k x 128 scaled errors of the current block, tf32 part
-  float* Elo;       // k x 128 fp32 remainder (E = Ehi + Elo)
+  float* Ehi[2];    // k x 128 scaled errors of a block, tf32 part (blocks alternate buffers)
+  float* Elo[2];    // k x 128 fp32 remainder (E = Ehi + Elo)
   float* Uhi;       // n x ldu tf32 part of U (columns >= n zero)
   float* Ulo;       // n x ldu fp32 remainder
   int64_t ldu;
@@ -57,8 +57,10 @@ static QLayout q_layout(void* ws, int64_t m, int64_t n) {
   QLayout L;
   L.hdr = c.take<WsHeader>(1);
   L.Wf = c.take<float>((size_t)m * n);
-  L.Ehi = c.take<float>((size_t)m * kBlock);
-  L.Elo = c.take<float>((size_t)m * kBlock);
+  for (int i = 0; i < 2; ++i) {
+    L.Ehi[i] = c.take<float>((size_t)m * kBlock);
+    L.Elo[i] = c.take<float>((size_t)m * kBlock);
+  }
   L.ldu = (n + 31) / 32 * 32;
   L.Uhi = c.take<float>((size_t)n * L.ldu);
   L.Ulo = c.take<float>((size_t)n * L.ldu);
@@ -538,6 +540,38 @@ static cudaError_t colloop_dispatch(int group, const ColArgs& ca, cudaStream_t s
   }
 }
 
+// Two streams per call, forked from and joined back into the caller's stream: A (higher
+// priority) runs the column loop of each block and the lazy update of the next block's 128
+// columns; B runs the lazy update of all later columns, overlapped with the next block's
+// column loop (look-ahead of one block).  One set per host thread and device, kept.
+struct QuantStreams {
+  bool ready = false;
+  cudaStream_t a = nullptr, b = nullptr;
+  cudaEvent_t fork = nullptr, col[2] = {}, rest[2] = {}, join[2] = {};
+};
+thread_local QuantStreams t_quant_streams[128];
+
+static cudaError_t quant_streams(QuantStreams** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 128) return cudaErrorInvalidDevice;
+  QuantStreams& q = t_quant_streams[dev];
+  if (!q.ready) {
+    int least = 0, greatest = 0;
+    if ((e = cudaDeviceGetStreamPriorityRange(&least, &greatest))) return e;
+    if ((e = cudaStreamCreateWithPriority(&q.a, cudaStreamNonBlocking, greatest))) return e;
+    if ((e = cudaStreamCreateWithPriority(&q.b, cudaStreamNonBlocking, least))) return e;
+    cudaEvent_t* evs[] = {&q.fork, &q.col[0], &q.col[1], &q.rest[0], &q.rest[1], &q.join[0],
+                          &q.join[1]};
+    for (cudaEvent_t* ev : evs)
+      if ((e = cudaEventCreateWithFlags(ev, cudaEventDisableTiming))) return e;
+    q.ready = true;
+  }
+  *out = &q;
+  return cudaSuccess;
+}
+
 gq_status run_quantize(const QuantArgs& a, cudaStream_t s) {
   const int64_t m = a.m, n = a.n;
   QLayout L = q_layout(a.ws, m, n);
@@ -585,23 +619,51 @@ gq_status run_quantize(const QuantArgs& a, cudaStream_t s) {
       count_launches(1);
       Q_TRY(cudaGetLastError());
     }
-    LazyTcMaps maps;
-    Q_TRY(lazy_tc_make_maps(&maps, L.Ehi, L.Elo, k_rows, L.Uhi, L.Ulo, n, L.ldu));
+    LazyTcMaps maps[2];
+    for (int i = 0; i < 2; ++i)
+      Q_TRY(lazy_tc_make_maps(&maps[i], L.Ehi[i], L.Elo[i], k_rows, L.Uhi, L.Ulo, n, L.ldu));
+    // Blocks on stream A; the lazy update after block b is split: the next block's 128 columns
+    // on A (the next column loop needs them), all later columns on B.  Block b's errors live in
+    // buffer b & 1 until its later-column update is done (the column loop of block b + 2, which
+    // reuses the buffer, waits for it through the next-block update of block b + 1).
+    QuantStreams* qs = nullptr;
+    Q_TRY(quant_streams(&qs));
+    cudaStream_t sa = qs->a, sb = qs->b;
+    Q_TRY(cudaEventRecord(qs->fork, s));
+    Q_TRY(cudaStreamWaitEvent(sa, qs->fork, 0));
+    Q_TRY(cudaStreamWaitEvent(sb, qs->fork, 0));
+    bool rest_pending = false;
     for (int b = 0; b < nblocks; ++b) {
       const int64_t j0 = (int64_t)b * kBlock;
       const int bw = (int)std::min<int64_t>(kBlock, n - j0);
       ColArgs ca{};
       ca.Ublk = L.Ublk; ca.hdr = L.hdr;
       ca.Wf = L.Wf; ca.n = n; ca.k_rows = k_rows; ca.rowlist = rowlist; ca.j0 = j0; ca.bw = bw;
-      ca.U = a.U; ca.bits = cfg.bits; ca.clip = cfg.clip; ca.Ehi = L.Ehi; ca.Elo = L.Elo;
+      ca.U = a.U; ca.bits = cfg.bits; ca.clip = cfg.clip; ca.Ehi = L.Ehi[b & 1];
+      ca.Elo = L.Elo[b & 1];
       ca.codes8 = L.codes8;
       ca.ldc8 = L.ldc8; ca.scales = a.scales; ca.zeros = a.zeros; ca.ngroups = ngroups;
       ca.row_s = L.row_s; ca.row_z = L.row_z; ca.row_e2 = L.row_e2; ca.row_bnd = L.row_bnd;
       ca.overflow = L.overflow;
-      Q_TRY(colloop_dispatch(G, ca, s));
+      Q_TRY(colloop_dispatch(G, ca, sa));
       const int64_t j1 = j0 + bw;
-      if (j1 < n) Q_TRY(launch_lazy_tc(maps, L.Wf, n, k_rows, j0, j1, L.hdr, s));
+      if (j1 >= n) continue;
+      const int64_t jn = std::min<int64_t>(j1 + kBlock, n);
+      Q_TRY(cudaEventRecord(qs->col[b & 1], sa));
+      if (rest_pending) Q_TRY(cudaStreamWaitEvent(sa, qs->rest[(b - 1) & 1], 0));
+      Q_TRY(launch_lazy_tc(maps[b & 1], L.Wf, n, k_rows, j0, j1, jn, L.hdr, sa));
+      rest_pending = false;
+      if (jn < n) {
+        Q_TRY(cudaStreamWaitEvent(sb, qs->col[b & 1], 0));
+        Q_TRY(launch_lazy_tc(maps[b & 1], L.Wf, n, k_rows, j0, jn, n, L.hdr, sb));
+        Q_TRY(cudaEventRecord(qs->rest[b & 1], sb));
+        rest_pending = true;
+      }
     }
+    Q_TRY(cudaEventRecord(qs->join[1], sb));
+    Q_TRY(cudaStreamWaitEvent(sa, qs->join[1], 0));
+    Q_TRY(cudaEventRecord(qs->join[0], sa));
+    Q_TRY(cudaStreamWaitEvent(s, qs->join[0], 0));
     if (cfg.clip) break;
     // clip-free: collect rows whose codes left [0, 2^b - 1] and rerun them on a wider step
     Q_TRY(cudaMemsetAsync(L.counter, 0, sizeof(int), s));
