@@ -6,11 +6,14 @@
 // acc += A_hi B_hi + A_hi B_lo + A_lo B_hi, accumulated in fp32 in tensor memory.  The column
 // loop writes E as E_hi / E_lo; U is split once per quantize call.
 //
-// CTA tile 128 (rows) x 128 (columns), K = 128 in 4 stages of 32 (3-deep ring), operands by
-// TMA (no multicast): A = E (K-major, rows of 32 fp32 = 128 B, 128-byte swizzle), B = U rows
+// CTA tile 128 (rows) x 128 (columns), K = 128 in 8 slices of 16 (3-deep ring, 32 KB a
+// stage, so two CTAs share an SM and one's epilogue overlaps the other's MMAs), operands by
+// TMA (no multicast): A = E (K-major, rows of 16 fp32 = 64 B, 64-byte swizzle), B = U rows
 // j0.. (MN-major, 4 runs of 32 columns, 128-byte swizzle with 32-byte chunks: the layout the
-// tensor cores require for 32-bit MN-major operands).  Warp 0 lane 0 issues the loads, warp 1 lane 0 the MMAs, all four
-// warps read the accumulator (lane = row) and subtract it from the fp32 work matrix.
+// tensor cores require for 32-bit MN-major operands).  Warp 0 lane 0 issues the loads, warp 1
+// lane 0 the MMAs; all eight warps read the accumulator (warps w and w + 4 share TMEM lanes
+// 32 (w % 4) ..; they take the left and right 64 columns) and subtract it from the fp32 work
+// matrix, with their work-matrix loads issued before the accumulator is ready.
 #include "gq_internal.cuh"
 #include "gq_tc.cuh"
 
@@ -20,15 +23,17 @@
 namespace gq {
 
 namespace {
-constexpr int kLBK = 32;                                  // K per stage
+constexpr int kLBK = 16;                                  // K per stage
 constexpr int kLStages = 3;
-constexpr uint32_t kLTile = 128 * kLBK * 4;               // 16 KB per operand tile
+constexpr int kLThreads = 256;
+constexpr uint32_t kLTile = 128 * kLBK * 4;               // 8 KB per operand tile
+constexpr uint32_t kLRun = 32 * kLBK * 4;                 // one 32-column run of a B tile
 constexpr uint32_t kLStage = 4 * kLTile;                  // A_hi, A_lo, B_hi, B_lo
 constexpr size_t kLSmem = kLStages * kLStage + 1024 + 256;
 constexpr uint32_t kLIdesc = tc::idesc_f32acc(2, 2, 0, 1, 128, 128);  // tf32, A K-major, B MN-major
 }  // namespace
 
-__global__ void __launch_bounds__(128, 1)
+__global__ void __launch_bounds__(kLThreads, 2)
     lazy_tc_kernel(const __grid_constant__ CUtensorMap m_ahi, const __grid_constant__ CUtensorMap m_alo,
                    const __grid_constant__ CUtensorMap m_bhi, const __grid_constant__ CUtensorMap m_blo,
                    float* Wf, int64_t n, int64_t k_rows, int j0, int j1, WsHeader* hdr) {
@@ -56,9 +61,10 @@ __global__ void __launch_bounds__(128, 1)
   const uint32_t tmem = *tslot;
   constexpr int NK = 128 / kLBK;
 
-  const int64_t row = (int64_t)tile_m * 128 + warp * 32 + lane;
+  const int64_t row = (int64_t)tile_m * 128 + (warp & 3) * 32 + lane;
   const int64_t colt = (int64_t)j1 + tile_n * 128;  // first column of this tile
-  float* wrow = Wf + row * n + colt;
+  const int chalf = (warp >> 2) * 64;                // this warp's 64 columns of the tile
+  float* wrow = Wf + row * n + colt + chalf;
   const bool vec = ((reinterpret_cast<uintptr_t>(Wf) & 15) == 0) && (n % 4 == 0);
   if (warp == 0 && lane == 0) {
     // producer
@@ -75,8 +81,8 @@ __global__ void __launch_bounds__(128, 1)
 #pragma unroll
       for (int g = 0; g < 4; ++g) {
         const int x = j1 + tile_n * 128 + g * 32, y = j0 + kc * kLBK;
-        tc::tma_load_2d(st + 2 * kLTile + g * 4096, &m_bhi, &full[s], x, y);
-        tc::tma_load_2d(st + 3 * kLTile + g * 4096, &m_blo, &full[s], x, y);
+        tc::tma_load_2d(st + 2 * kLTile + g * kLRun, &m_bhi, &full[s], x, y);
+        tc::tma_load_2d(st + 3 * kLTile + g * kLRun, &m_blo, &full[s], x, y);
       }
     }
     // the epilogue's read-modify-write tile: into L2 while the MMAs run
@@ -98,10 +104,10 @@ __global__ void __launch_bounds__(128, 1)
       const uint32_t a_lo = a_hi + kLTile, b_hi = a_hi + 2 * kLTile, b_lo = a_hi + 3 * kLTile;
 #pragma unroll
       for (int k = 0; k < kLBK / 8; ++k) {
-        const uint64_t dah = tc::sdesc(a_hi + k * 32, 16, 1024, tc::kLayoutSW128);
-        const uint64_t dal = tc::sdesc(a_lo + k * 32, 16, 1024, tc::kLayoutSW128);
-        const uint64_t dbh = tc::sdesc(b_hi + k * 1024, 4096, 512, tc::kLayoutSW128Base32B);
-        const uint64_t dbl = tc::sdesc(b_lo + k * 1024, 4096, 512, tc::kLayoutSW128Base32B);
+        const uint64_t dah = tc::sdesc(a_hi + k * 32, 16, 512, tc::kLayoutSW64);
+        const uint64_t dal = tc::sdesc(a_lo + k * 32, 16, 512, tc::kLayoutSW64);
+        const uint64_t dbh = tc::sdesc(b_hi + k * 1024, kLRun, 512, tc::kLayoutSW128Base32B);
+        const uint64_t dbl = tc::sdesc(b_lo + k * 1024, kLRun, 512, tc::kLayoutSW128Base32B);
         tc::mma_tf32(tmem, dah, dbh, kLIdesc, (kc | k) != 0);
         tc::mma_tf32(tmem, dah, dbl, kLIdesc, 1);
         tc::mma_tf32(tmem, dal, dbh, kLIdesc, 1);
@@ -112,9 +118,9 @@ __global__ void __launch_bounds__(128, 1)
   }
   __syncwarp();
 
-  // Epilogue: TMEM lane = tile row, 4 chunks of 32 columns; row = this thread's row.  The work
-  // matrix values of the first two chunks are loaded before the accumulator is waited for, so
-  // their latency overlaps the MMAs; each later chunk's load is issued two chunks ahead.
+  // Epilogue: TMEM lane = tile row; this warp's two chunks of 32 columns.  Both chunks of the
+  // work matrix are loaded before the accumulator is waited for, so the load latency overlaps
+  // the MMAs (and the other CTA on the SM).
   const bool full_row = row < k_rows && colt + 128 <= n && vec;
   float4 wv[2][8];
   if (full_row) {
@@ -128,21 +134,16 @@ __global__ void __launch_bounds__(128, 1)
   tc::fence_after_sync();
   if (ok) {
 #pragma unroll
-    for (int cc = 0; cc < 4; ++cc) {
+    for (int cc = 0; cc < 2; ++cc) {
       float v[32];
-      tc::tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + cc * 32, v);
-      const int64_t col0 = colt + cc * 32;
+      tc::tmem_ld32(tmem + ((uint32_t)((warp & 3) * 32) << 16) + chalf + cc * 32, v);
+      const int64_t col0 = colt + chalf + cc * 32;
       if (full_row) {
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-          float4 w = wv[cc & 1][i];
+          float4 w = wv[cc][i];
           w.x -= v[4 * i]; w.y -= v[4 * i + 1]; w.z -= v[4 * i + 2]; w.w -= v[4 * i + 3];
           *reinterpret_cast<float4*>(wrow + cc * 32 + 4 * i) = w;
-        }
-        if (cc + 2 < 4) {
-#pragma unroll
-          for (int i = 0; i < 8; ++i)
-            wv[cc & 1][i] = *reinterpret_cast<const float4*>(wrow + (cc + 2) * 32 + 4 * i);
         }
       } else if (row < k_rows && col0 < n) {
         float* dst = Wf + row * n + col0;
@@ -206,10 +207,11 @@ cudaError_t lazy_tc_make_maps(LazyTcMaps* maps, const float* Ehi, const float* E
                               const float* Uhi, const float* Ulo, int64_t n, int64_t ldu) {
   cudaError_t e = get_encode();
   if (e != cudaSuccess) return e;
-  const CUtensorMapSwizzle ka = CU_TENSOR_MAP_SWIZZLE_128B;            // K-major A
+  const CUtensorMapSwizzle ka = CU_TENSOR_MAP_SWIZZLE_64B;             // K-major A, 64-byte rows
   const CUtensorMapSwizzle mb = CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B;    // MN-major 32-bit B
-  if ((e = encode_f32(&maps->ahi, Ehi, rows, kBlock, kBlock, 128, ka))) return e;
-  if ((e = encode_f32(&maps->alo, Elo, rows, kBlock, kBlock, 128, ka))) return e;
+  const CUtensorMapDataType f32 = CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+  if ((e = encode_tmap_2d(&maps->ahi, f32, 4, Ehi, rows, kBlock, kBlock, kLBK, 128, ka))) return e;
+  if ((e = encode_tmap_2d(&maps->alo, f32, 4, Elo, rows, kBlock, kBlock, kLBK, 128, ka))) return e;
   if ((e = encode_f32(&maps->bhi, Uhi, n, n, ldu, kLBK, mb))) return e;
   return encode_f32(&maps->blo, Ulo, n, n, ldu, kLBK, mb);
 }
@@ -219,7 +221,7 @@ cudaError_t launch_lazy_tc(const LazyTcMaps& maps, float* Wf, int64_t n, int64_t
   if (jend > n) jend = n;
   if (j1 >= jend || k_rows <= 0) return cudaSuccess;
   dim3 grid((unsigned)((jend - j1 + 127) / 128), (unsigned)((k_rows + 127) / 128));
-  lazy_tc_kernel<<<grid, 128, kLSmem, s>>>(maps.ahi, maps.alo, maps.bhi, maps.blo, Wf, n, k_rows,
+  lazy_tc_kernel<<<grid, kLThreads, kLSmem, s>>>(maps.ahi, maps.alo, maps.bhi, maps.blo, Wf, n, k_rows,
                                            (int)j0, (int)j1, hdr);
   count_launches(1);
   return cudaGetLastError();

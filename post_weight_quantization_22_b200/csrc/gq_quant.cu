@@ -7,9 +7,9 @@
 //
 // Work layout: the weights are copied once into an fp32 work matrix Wf (rows x n) in the
 // processing order (columns reversed for the last-to-first variant, dead columns zeroed).  Per
-// 128-column block: `colloop` runs the sequential column recursion for 32 rows per CTA (4
-// lanes per row, each lane owning 32 of the block's columns in 4-wide chunks), keeping the
-// block's part of U in shared memory; the tensor-core lazy update (gq_lazy_tc.cu) then applies
+// 128-column block: `colloop` runs the column recursion for 64 rows per CTA (16 per warp, in
+// 8-column tiles with fp64 tensor-core updates between tiles), keeping the block's part of U
+// in shared memory; the tensor-core lazy update (gq_lazy_tc.cu) then applies
 // W[:, j+128:] -= E U[j:j+128, j+128:] to the rest of the work matrix.
 #include "gq_internal.cuh"
 #include "gq_tc.cuh"
@@ -19,14 +19,17 @@
 
 namespace gq {
 
-constexpr int kP = 4;                      // lanes per row in the column loop
-constexpr int kVPL = kBlock / kP;          // values per lane (32)
-constexpr int kSW = 4 * kP;                // segment width: one 4-column chunk per lane
-constexpr int kColThreads = 128;
-constexpr int kRowsPerCta = kColThreads / kP;  // 32 rows per CTA
-// Per-block prepared U for the column loop (see ublk_kernel): 128 x 128 doubles + 2 x 128.
-constexpr int64_t kUBlkDoubles = (int64_t)kBlock * kBlock + 2 * kBlock;
-constexpr uint32_t kUBlkBytes = (uint32_t)(kUBlkDoubles * sizeof(double));
+constexpr int kColWarps = 4;                    // warps per column-loop CTA, 8 rows each
+constexpr int kColThreads = 32 * kColWarps;
+constexpr int kRowsPerCta = 8 * kColWarps;      // 32 rows per CTA
+constexpr int kTiles = kBlock / 8;              // 8-column tiles of a block
+constexpr int kUtPitch = 136;                   // floats per row of the transposed U block
+// Per-block prepared U for the column loop (see ublk_kernel): the transposed block in fp32
+// (128 rows of kUtPitch floats), then 1/U_jj and 1/U_jj^2 in fp64.
+constexpr uint32_t kUtBytes = (uint32_t)(kBlock * kUtPitch * sizeof(float));
+constexpr uint32_t kUBlkBytes = kUtBytes + 2 * kBlock * (uint32_t)sizeof(double);
+constexpr int64_t kUBlkDoubles = kUBlkBytes / sizeof(double);
+static_assert(kUBlkBytes % 16 == 0, "bulk copies move multiples of 16 bytes");
 constexpr uint32_t kBulkChunk = 32768;
 
 struct QLayout {
@@ -174,25 +177,26 @@ __global__ void split_u_kernel(const float* U, int64_t n, int64_t ldu, float* Uh
   }
 }
 
-// Per-block prepared U, built once per call: the block's 128 x 128 part of U in fp64 with the
-// strict lower triangle and the columns past the block's width zeroed, then 1/U_jj and
-// 1/U_jj^2 (1 past the width).  The column loop copies it into shared memory in one go.
-
+// Per-block prepared U, built once per call: the block's 128 x 128 part of U transposed,
+// Ut[c][k] = U[j0 + k][j0 + c] for k <= c < width (0 elsewhere), in fp32 (U is fp32, so this
+// is exact) with row pitch kUtPitch, then 1/U_jj and 1/U_jj^2 in fp64 (1 past the width).  The
+// column loop copies it into shared memory in one go.
 __global__ void ublk_kernel(const float* U, int64_t n, double* Ublk) {
   const int64_t b = blockIdx.y;
   const int64_t j0 = b * kBlock;
   const int bw = (int)((n - j0) < kBlock ? (n - j0) : kBlock);
-  double* dst = Ublk + b * kUBlkDoubles;
-  for (int e = blockIdx.x * blockDim.x + threadIdx.x; e < kBlock * kBlock + kBlock;
+  float* ut = reinterpret_cast<float*>(Ublk + b * kUBlkDoubles);
+  double* dinv = reinterpret_cast<double*>(reinterpret_cast<char*>(ut) + kUtBytes);
+  for (int e = blockIdx.x * blockDim.x + threadIdx.x; e < kBlock * kUtPitch + kBlock;
        e += gridDim.x * blockDim.x) {
-    if (e < kBlock * kBlock) {
-      const int jj = e / kBlock, kk = e % kBlock;
-      dst[e] = (jj < bw && kk >= jj && kk < bw) ? (double)U[(j0 + jj) * n + j0 + kk] : 0.0;
+    if (e < kBlock * kUtPitch) {
+      const int c = e / kUtPitch, k = e % kUtPitch;
+      ut[e] = (c < bw && k <= c) ? U[(j0 + k) * n + j0 + c] : 0.f;
     } else {
-      const int jj = e - kBlock * kBlock;
+      const int jj = e - kBlock * kUtPitch;
       const double d = jj < bw ? (double)U[(j0 + jj) * n + j0 + jj] : 1.0;
-      dst[kBlock * kBlock + jj] = 1.0 / d;
-      dst[kBlock * kBlock + kBlock + jj] = 1.0 / (d * d);
+      dinv[jj] = 1.0 / d;
+      dinv[kBlock + jj] = 1.0 / (d * d);
     }
   }
 }
@@ -226,12 +230,19 @@ struct ColArgs {
   int* overflow;
 };
 
-// Lane ownership: each row is handled by kP = 4 lanes; the block's 128 columns form 8 segments
-// of 16, and in each segment lane t owns the 4-column chunk [16 seg + 4t, 16 seg + 4t + 4).
-// Each lane keeps its 8 chunks in registers, v[4c + u] = chunk (seg + c); after a segment the
-// array is rotated by one chunk, so the unrolled 16-step body refers to fixed registers and the
-// segment loop stays a small runtime loop (a fully unrolled 128-step body does not fit the
-// instruction cache).  128-thread CTAs of 32 rows.
+// Thread layout: a warp owns 8 rows; lane (g, t) = (lane / 4, lane % 4) holds row g and, of
+// every 8-column tile, columns 2t and 2t + 1: w[tile][p] (p = column 2t + p).  That is the
+// accumulator layout of the fp64 mma.sync m16n8k8 for its first 8 rows (the other 8 are zero
+// padding: 8 rows a warp keep twice as many warps busy as 16, and the loop is latency-bound).
+// Per tile of 8 columns the recursion is sequential only inside the tile (each column needs the
+// errors of the earlier ones): the owner's value is shared in the quad, every lane of the quad
+// computes the code and error of its row, and a lane updates its own later columns of the tile.
+// The tile's 8 error columns then update every later tile of the block at once, one fp64
+// tensor-core MMA per tile (the errors already sit in the A-operand layout when the k slots of
+// lane t are taken as columns 2t and 2t + 1).  This is GPTQ's lazy batch applied again inside
+// the block; the group grid, taken at a group's first column, sees the same error-fed values
+// as the column-by-column recursion.  The register array is rotated by one tile after each
+// tile so that the unrolled body refers to fixed registers.
 //
 // The recursion runs in fp64: the in-block feedback sums cancel strongly when the grid is
 // coarse, and an fp32 recursion flips ~1-3 % of the codes on ill-conditioned layers (measured
@@ -240,18 +251,18 @@ struct ColArgs {
 template <int G>
 __global__ void __launch_bounds__(kColThreads, 1) colloop_kernel(ColArgs a) {
   extern __shared__ __align__(16) double q_smem[];
-  double* Us = q_smem;                       // [128][128] this block's part of U (fp64, masked)
-  double* invd = q_smem + kBlock * kBlock;   // [128]  1/U_jj
-  double* invd2 = invd + kBlock;             // [128]  1/U_jj^2
-  uint64_t* bar = reinterpret_cast<uint64_t*>(invd2 + kBlock);
+  const float* Ut = reinterpret_cast<const float*>(q_smem);
+  const double* invd = reinterpret_cast<const double*>(reinterpret_cast<const char*>(q_smem) + kUtBytes);
+  const double* invd2 = invd + kBlock;
+  uint64_t* bar = reinterpret_cast<uint64_t*>(reinterpret_cast<char*>(q_smem) + kUBlkBytes);
   const int tid = threadIdx.x;
   const int bw = a.bw;
   const int64_t n = a.n, j0 = a.j0;
-  // the prepared block (kUBlkBytes) arrives by bulk async copies while the rows load below
+  // the prepared block arrives by bulk async copies while the rows load below
   if (tid == 0) {
     tc::mbar_init(bar, 1);
     tc::fence_barrier_init();
-    tc::mbar_arrive_expect_tx(bar, (uint32_t)kUBlkBytes);
+    tc::mbar_arrive_expect_tx(bar, kUBlkBytes);
     const char* src = reinterpret_cast<const char*>(a.Ublk + (j0 / kBlock) * kUBlkDoubles);
     char* dst = reinterpret_cast<char*>(q_smem);
     for (uint32_t off = 0; off < kUBlkBytes; off += kBulkChunk) {
@@ -260,28 +271,30 @@ __global__ void __launch_bounds__(kColThreads, 1) colloop_kernel(ColArgs a) {
     }
   }
   const int lane = tid & 31, warp = tid >> 5;
-  const int t = lane % kP;
-  const int64_t rr = (int64_t)blockIdx.x * kRowsPerCta + warp * (32 / kP) + lane / kP;
-  const bool active = rr < a.k_rows;
-  const int64_t row = active ? (a.rowlist ? a.rowlist[rr] : rr) : 0;
+  const int g = lane >> 2, t = lane & 3;
+  const unsigned full = 0xffffffffu;
+  const int qbase = lane & ~3;
+  const int64_t rr = (int64_t)blockIdx.x * kRowsPerCta + warp * 8 + g;
+  const bool act = rr < a.k_rows;
+  const int64_t row = act ? (a.rowlist ? a.rowlist[rr] : rr) : 0;
   const double maxq = (double)((1 << a.bits) - 1);
 
-  double v[kVPL];
+  double w[kTiles][2];
 #pragma unroll
-  for (int c = 0; c < kVPL / 4; ++c) {
-    int k = kSW * c + 4 * t;
-    float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (active) {
-      const float* src = a.Wf + rr * n + j0 + k;
-      if (k + 3 < bw && ((j0 + k + rr * n) & 3) == 0) {
-        x = *reinterpret_cast<const float4*>(src);
+  for (int k = 0; k < kTiles; ++k) {
+    const int col = 8 * k + 2 * t;
+    float2 x = make_float2(0.f, 0.f);
+    if (act) {
+      const float* src = a.Wf + rr * n + j0 + col;
+      if (col + 1 < bw && ((j0 + col + rr * n) & 1) == 0) {
+        x = *reinterpret_cast<const float2*>(src);
       } else {
-        float* dx = &x.x;
-#pragma unroll
-        for (int u = 0; u < 4; ++u) dx[u] = (k + u < bw) ? src[u] : 0.f;
+        if (col < bw) x.x = src[0];
+        if (col + 1 < bw) x.y = src[1];
       }
     }
-    v[4 * c + 0] = x.x; v[4 * c + 1] = x.y; v[4 * c + 2] = x.z; v[4 * c + 3] = x.w;
+    w[k][0] = x.x;
+    w[k][1] = x.y;
   }
   __syncthreads();  // the barrier's initialisation is visible to every waiting thread
   if (!tc::mbar_wait(bar, 0)) {
@@ -289,121 +302,111 @@ __global__ void __launch_bounds__(kColThreads, 1) colloop_kernel(ColArgs a) {
     return;  // nothing was computed; the bulk copy has been waited for the full bound
   }
   double s = 1.0, inv_s = 1.0, z = 0.0;
-  if (G == 0 && active) { s = a.row_s[row]; z = a.row_z[row]; inv_s = 1.0 / s; }
+  if (G == 0 && act) { s = a.row_s[row]; z = a.row_z[row]; inv_s = 1.0 / s; }
   double e2 = 0.0, bnd = 0.0;
   int ovf = 0;
-  const unsigned full = 0xffffffffu;
-  const int gbase = lane & ~(kP - 1);
-  float* Ehrow = a.Ehi + rr * kBlock;
-  float* Elrow = a.Elo + rr * kBlock;
-  uint8_t* crow = a.codes8 + row * a.ldc8 + j0;
-  constexpr int kGStep = (G > 0 && G < kSW) ? G : kSW;  // distance between possible group starts
+  const bool clip = a.clip != 0;
 
-  for (int seg = 0; seg < kBlock / kSW; ++seg) {
-    if (kSW * seg >= bw) break;
-    float eo[4] = {0.f, 0.f, 0.f, 0.f};
-    uint32_t cw = 0u;
+#pragma unroll 1
+  for (int T = 0; T < kTiles; ++T) {
+    if (8 * T >= bw) break;
+    if constexpr (G > 0) {
+      if ((8 * T) % G == 0) {
+        // group grid from the current (error-fed) weights of columns [8T, 8T + G)
+        double lo = 0.0, hi = 0.0;
 #pragma unroll
-    for (int jl = 0; jl < kSW; ++jl) {
-      const int jj = kSW * seg + jl;
+        for (int k = 0; k < G / 8 && k < kTiles; ++k)
+#pragma unroll
+          for (int p = 0; p < 2; ++p)
+            if (8 * (T + k) + 2 * t + p < bw) { lo = fmin(lo, w[k][p]); hi = fmax(hi, w[k][p]); }
+        lo = fmin(lo, __shfl_xor_sync(full, lo, 1));
+        hi = fmax(hi, __shfl_xor_sync(full, hi, 1));
+        lo = fmin(lo, __shfl_xor_sync(full, lo, 2));
+        hi = fmax(hi, __shfl_xor_sync(full, hi, 2));
+        if (lo == 0.0 && hi == 0.0) { lo = -1.0; hi = 1.0; }
+        s = (hi - lo) / maxq;
+        z = rint(-lo / s);
+        inv_s = 1.0 / s;
+        if (act && t == 0) {
+          const int64_t gi = (j0 + 8 * T) / G;
+          a.scales[row * a.ngroups + gi] = (float)s;
+          a.zeros[row * a.ngroups + gi] = (uint8_t)z;
+        }
+      }
+    }
+    // U entries of this tile's recursion: ut[p][i] = U[8T + i][8T + 2t + p]
+    double ut[2][8];
+#pragma unroll
+    for (int p = 0; p < 2; ++p) {
+      const float* up = Ut + (8 * T + 2 * t + p) * kUtPitch + 8 * T;
+      const float4 lo4 = *reinterpret_cast<const float4*>(up);
+      const float4 hi4 = *reinterpret_cast<const float4*>(up + 4);
+      ut[p][0] = lo4.x; ut[p][1] = lo4.y; ut[p][2] = lo4.z; ut[p][3] = lo4.w;
+      ut[p][4] = hi4.x; ut[p][5] = hi4.y; ut[p][6] = hi4.z; ut[p][7] = hi4.w;
+    }
+    const double cmin = -z, cmax = maxq - z;  // code range in the domain c - z
+    double ea[2] = {0.0, 0.0}, ca[2] = {0.0, 0.0};  // this lane's errors / codes (cols 2t, 2t+1)
+    double d2sum = 0.0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int jj = 8 * T + i;
       if (jj < bw) {
-        if constexpr (G > 0) {
-          if (jl % kGStep == 0 && (jj % G) == 0) {
-            // group grid from the current (error-fed) weights of columns [jj, jj + G)
-            double lo = 0.0, hi = 0.0;
-#pragma unroll
-            for (int c = 0; c < kVPL / 4; ++c)
-#pragma unroll
-              for (int u = 0; u < 4; ++u) {
-                const int k = kSW * (seg + c) + 4 * t + u;
-                if (k >= jj && k < jj + G && k < bw) { lo = fmin(lo, v[4 * c + u]); hi = fmax(hi, v[4 * c + u]); }
-              }
-#pragma unroll
-            for (int o = kP / 2; o > 0; o >>= 1) {
-              lo = fmin(lo, __shfl_xor_sync(full, lo, o));
-              hi = fmax(hi, __shfl_xor_sync(full, hi, o));
-            }
-            if (lo == 0.0 && hi == 0.0) { lo = -1.0; hi = 1.0; }
-            s = (hi - lo) / maxq;
-            z = rint(-lo / s);
-            inv_s = 1.0 / s;
-            if (active && t == 0) {
-              const int64_t g = (j0 + jj) / G;
-              a.scales[row * a.ngroups + g] = (float)s;
-              a.zeros[row * a.ngroups + g] = (uint8_t)z;
-            }
-          }
-        }
-        const double cmin = -z, cmax = maxq - z;  // code range in the shifted domain c - z
-        const int owner = jl / 4, slot = jl % 4;
+        const int town = i >> 1, pown = i & 1;
         const double id = invd[jj];
-        const double sd = s * id;
-        const double x = __shfl_sync(full, v[slot], gbase + owner);
-        const double xi = x * id;
+        d2sum += invd2[jj];
+        const double x = __shfl_sync(full, w[0][pown], qbase | town);
         double c = rint_small(x * inv_s);
-        if (a.clip) {
-          c = fmin(fmax(c, cmin), cmax);
-        } else if (c < cmin || c > cmax) {
-          ovf = 1;
-        }
-        const double e = fma(-c, sd, xi);  // (x - s c) / U_jj
-        if (t == owner) {
-          eo[slot] = (float)e;
-          cw |= (uint32_t)(int)fmin(fmax(c + z, 0.0), maxq) << (8 * slot);
-        }
+        if (clip) c = fmin(fmax(c, cmin), cmax);
+        else if (c < cmin || c > cmax) ovf = 1;
+        const double e = fma(-s, c, x) * id;  // (x - s c) / U_jj
+        if (t == town) { ea[pown] = e; ca[pown] = c; }
         e2 = fma(e, e, e2);
-        bnd = fma(s * s, invd2[jj], bnd);
-        const double* urow = Us + jj * kBlock + kSW * seg + 4 * t;
-        if (t >= owner) {  // the chunk that holds column jj: only its later columns
-          const double2 u01 = *reinterpret_cast<const double2*>(urow);
-          const double2 u23 = *reinterpret_cast<const double2*>(urow + 2);
-          if (t > owner || 0 > slot) v[0] = fma(-e, u01.x, v[0]);
-          if (t > owner || 1 > slot) v[1] = fma(-e, u01.y, v[1]);
-          if (t > owner || 2 > slot) v[2] = fma(-e, u23.x, v[2]);
-          if (t > owner || 3 > slot) v[3] = fma(-e, u23.y, v[3]);
-        }
 #pragma unroll
-        for (int c2 = 1; c2 < kVPL / 4; ++c2) {
-          if (c2 < kBlock / kSW - seg) {
-            const double2 u01 = *reinterpret_cast<const double2*>(urow + kSW * c2);
-            const double2 u23 = *reinterpret_cast<const double2*>(urow + kSW * c2 + 2);
-            v[4 * c2 + 0] = fma(-e, u01.x, v[4 * c2 + 0]);
-            v[4 * c2 + 1] = fma(-e, u01.y, v[4 * c2 + 1]);
-            v[4 * c2 + 2] = fma(-e, u23.x, v[4 * c2 + 2]);
-            v[4 * c2 + 3] = fma(-e, u23.y, v[4 * c2 + 3]);
-          }
-        }
+        for (int p = 0; p < 2; ++p)
+          if (2 * t + p > i) w[0][p] = fma(-e, ut[p][i], w[0][p]);
       }
     }
-    // this segment's errors and codes
-    if (active) {
-      const int k = kSW * seg + 4 * t;
-      float4 hi, lo;
-      hi.x = tf32_rna(eo[0]); hi.y = tf32_rna(eo[1]); hi.z = tf32_rna(eo[2]); hi.w = tf32_rna(eo[3]);
-      lo.x = eo[0] - hi.x; lo.y = eo[1] - hi.y; lo.z = eo[2] - hi.z; lo.w = eo[3] - hi.w;
-      *reinterpret_cast<float4*>(Ehrow + k) = hi;
-      *reinterpret_cast<float4*>(Elrow + k) = lo;
-      if (k + 3 < bw) {
-        *reinterpret_cast<uint32_t*>(crow + k) = cw;
-      } else {
-#pragma unroll
-        for (int u = 0; u < 4; ++u)
-          if (k + u < bw) crow[k + u] = (uint8_t)(cw >> (8 * u));
+    bnd = fma(s * s, d2sum, bnd);
+    // this tile's errors (E = E_hi + E_lo for the lazy update) and codes
+    {
+      const int col = 8 * T + 2 * t;
+      if (act && col < bw) {
+        const float f0 = (float)ea[0], f1 = (float)ea[1];
+        float2 hi2, lo2;
+        hi2.x = tf32_rna(f0); hi2.y = tf32_rna(f1);
+        lo2.x = f0 - hi2.x; lo2.y = f1 - hi2.y;
+        *reinterpret_cast<float2*>(a.Ehi + rr * kBlock + col) = hi2;
+        *reinterpret_cast<float2*>(a.Elo + rr * kBlock + col) = lo2;
+        uint8_t* cp = a.codes8 + row * a.ldc8 + j0 + col;
+        cp[0] = (uint8_t)(int)fmin(fmax(ca[0] + z, 0.0), maxq);
+        if (col + 1 < bw) cp[1] = (uint8_t)(int)fmin(fmax(ca[1] + z, 0.0), maxq);
       }
     }
-    // rotate: chunk seg + 1 moves to registers 0..3
+    // the later tiles of the block take this tile's errors: w[k] -= E_T U[T rows][tile k]
+    const double an[4] = {-ea[0], 0.0, -ea[1], 0.0};
 #pragma unroll
-    for (int i = 0; i < kVPL - 4; ++i) v[i] = v[i + 4];
+    for (int k = 1; k < kTiles; ++k) {
+      if (T + k < kTiles && 8 * (T + k) < bw) {
+        const float2 bv =
+            *reinterpret_cast<const float2*>(Ut + (8 * (T + k) + g) * kUtPitch + 8 * T + 2 * t);
+        const double b2[2] = {(double)bv.x, (double)bv.y};
+        double c4[4] = {w[k][0], w[k][1], 0.0, 0.0};
+        tc::dmma_m16n8k8(c4, an, b2);
+        w[k][0] = c4[0]; w[k][1] = c4[1];
+      }
+    }
+    // rotate: tile T + 1 moves to position 0
+#pragma unroll
+    for (int k = 0; k < kTiles - 1; ++k) { w[k][0] = w[k + 1][0]; w[k][1] = w[k + 1][1]; }
   }
-  // per-row overflow flag (all lanes of the warp take part in the shuffle)
-  int ovf_row = ovf;
-#pragma unroll
-  for (int o = kP / 2; o > 0; o >>= 1) ovf_row |= __shfl_xor_sync(0xffffffffu, ovf_row, o);
-  if (!active) return;
-  // per-row totals (all lanes of a row hold the same e2 / bnd)
-  if (t == 0) {
-    if (j0 == 0) { a.row_e2[row] = e2; a.row_bnd[row] = bnd; a.overflow[row] = ovf_row; }
-    else { a.row_e2[row] += e2; a.row_bnd[row] += bnd; a.overflow[row] |= ovf_row; }
+  // per-row overflow flag (all lanes of the warp take part in the shuffles)
+  int ovf_q = ovf;
+  ovf_q |= __shfl_xor_sync(full, ovf_q, 1);
+  ovf_q |= __shfl_xor_sync(full, ovf_q, 2);
+  // per-row totals (all lanes of a quad hold the same e2 / bnd)
+  if (act && t == 0) {
+    if (j0 == 0) { a.row_e2[row] = e2; a.row_bnd[row] = bnd; a.overflow[row] = ovf_q; }
+    else { a.row_e2[row] += e2; a.row_bnd[row] += bnd; a.overflow[row] |= ovf_q; }
   }
 }
 
