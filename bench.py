@@ -323,7 +323,7 @@ def run_gq(args):
                    "parallelism": f"{ws} independent layers (one per GPU)"},
         "stages": stages,
         "roofline": roof,
-        "roofline_peak_kind": peak_kind,
+        "roofline_peak_kind": "derived: fp64 unit counts x measured max SM clock",
         "cpu_baseline": cpu,
         "e2e": {"value": job_throughput(m * n, ws, args.steps, e2e_ms), "unit": UNIT,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
