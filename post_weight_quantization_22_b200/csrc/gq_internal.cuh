@@ -127,9 +127,7 @@ cudaError_t lazy_tc_make_maps(LazyTcMaps* maps, const float* Ehi, const float* E
                               const float* Uhi, const float* Ulo, int64_t n, int64_t ldu);
 // Wf[:, j1:jend] -= (E_hi + E_lo) (U_hi + U_lo)[j0:j0+128, j1:jend]  (3xTF32), rows < k_rows;
 // jend is n or j1 + 128k.
-// background: one CTA an SM, leaving room for the concurrent column loop.
 cudaError_t launch_lazy_tc(const LazyTcMaps& maps, float* Wf, int64_t n, int64_t k_rows,
-                           int64_t j0, int64_t j1, int64_t jend, WsHeader* hdr, cudaStream_t s,
-                           bool background);
+                           int64_t j0, int64_t j1, int64_t jend, WsHeader* hdr, cudaStream_t s);
 
 }  // namespace gq

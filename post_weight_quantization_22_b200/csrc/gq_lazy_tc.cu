@@ -30,10 +30,6 @@ constexpr uint32_t kLTile = 128 * kLBK * 4;               // 8 KB per operand ti
 constexpr uint32_t kLRun = 32 * kLBK * 4;                 // one 32-column run of a B tile
 constexpr uint32_t kLStage = 4 * kLTile;                  // A_hi, A_lo, B_hi, B_lo
 constexpr size_t kLSmem = kLStages * kLStage + 1024 + 256;
-// A background launch (the later columns, overlapped with the next block's column loop) asks
-// for this much shared memory so that only one of its CTAs fits an SM and the column loop's CTA
-// (72 KB) still finds room next to it.
-constexpr size_t kLSmemBackground = 140 * 1024;
 constexpr uint32_t kLIdesc = tc::idesc_f32acc(2, 2, 0, 1, 128, 128);  // tf32, A K-major, B MN-major
 }  // namespace
 
@@ -204,7 +200,7 @@ cudaError_t encode_tmap_2d(CUtensorMap* map, CUtensorMapDataType dt, size_t elem
 
 cudaError_t lazy_tc_init_attributes() {
   return cudaFuncSetAttribute(lazy_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              (int)kLSmemBackground);
+                              (int)kLSmem);
 }
 
 cudaError_t lazy_tc_make_maps(LazyTcMaps* maps, const float* Ehi, const float* Elo, int64_t rows,
@@ -221,13 +217,11 @@ cudaError_t lazy_tc_make_maps(LazyTcMaps* maps, const float* Ehi, const float* E
 }
 
 cudaError_t launch_lazy_tc(const LazyTcMaps& maps, float* Wf, int64_t n, int64_t k_rows,
-                           int64_t j0, int64_t j1, int64_t jend, WsHeader* hdr, cudaStream_t s,
-                           bool background) {
+                           int64_t j0, int64_t j1, int64_t jend, WsHeader* hdr, cudaStream_t s) {
   if (jend > n) jend = n;
   if (j1 >= jend || k_rows <= 0) return cudaSuccess;
   dim3 grid((unsigned)((jend - j1 + 127) / 128), (unsigned)((k_rows + 127) / 128));
-  lazy_tc_kernel<<<grid, kLThreads, background ? kLSmemBackground : kLSmem, s>>>(
-      maps.ahi, maps.alo, maps.bhi, maps.blo, Wf, n, k_rows,
+  lazy_tc_kernel<<<grid, kLThreads, kLSmem, s>>>(maps.ahi, maps.alo, maps.bhi, maps.blo, Wf, n, k_rows,
                                            (int)j0, (int)j1, hdr);
   count_launches(1);
   return cudaGetLastError();

@@ -654,11 +654,11 @@ gq_status run_quantize(const QuantArgs& a, cudaStream_t s) {
       const int64_t jn = std::min<int64_t>(j1 + kBlock, n);
       Q_TRY(cudaEventRecord(qs->col[b & 1], sa));
       if (rest_pending) Q_TRY(cudaStreamWaitEvent(sa, qs->rest[(b - 1) & 1], 0));
-      Q_TRY(launch_lazy_tc(maps[b & 1], L.Wf, n, k_rows, j0, j1, jn, L.hdr, sa, false));
+      Q_TRY(launch_lazy_tc(maps[b & 1], L.Wf, n, k_rows, j0, j1, jn, L.hdr, sa));
       rest_pending = false;
       if (jn < n) {
         Q_TRY(cudaStreamWaitEvent(sb, qs->col[b & 1], 0));
-        Q_TRY(launch_lazy_tc(maps[b & 1], L.Wf, n, k_rows, j0, jn, n, L.hdr, sb, true));
+        Q_TRY(launch_lazy_tc(maps[b & 1], L.Wf, n, k_rows, j0, jn, n, L.hdr, sb));
         Q_TRY(cudaEventRecord(qs->rest[b & 1], sb));
         rest_pending = true;
       }
