@@ -12,7 +12,7 @@ import torch
 
 from oracle import gptq_oracle as O
 from post_weight_quantization_22_b200 import synth
-from tests.gpu_helpers import rel_fro, run_gpu
+from tests.gpu_helpers import rel_fro, run_gpu, unpack_np
 
 pytestmark = pytest.mark.gpu
 
@@ -42,7 +42,17 @@ def _compare(g, o, W, bits, group, rows=None, check_loss=True):
     gz = g["zeros"] if rows is None else g["zeros"][rows]
     assert float(np.mean(gz == o["zeros"])) >= CODE_MATCH
     gs = g["scales"] if rows is None else g["scales"][rows]
-    np.testing.assert_allclose(gs, o["scales"], rtol=1e-4 if group else 1e-6)
+    if group:
+        # A group's grid comes from the error-fed weights at its first column, so it is fixed by
+        # the codes before that column: compare it wherever the row's earlier codes agree (a
+        # permitted code difference changes every later group of its row).
+        ng = gs.shape[1]
+        same_before = np.ones((gc.shape[0], ng), dtype=bool)
+        for k in range(1, ng):
+            same_before[:, k] = np.all(gc[:, : k * group] == o["codes"][:, : k * group], axis=1)
+        np.testing.assert_allclose(gs[same_before], o["scales"][same_before], rtol=1e-4)
+    else:
+        np.testing.assert_allclose(gs, o["scales"], rtol=1e-6)
     # packed words: identical wherever a row's codes are identical
     same = np.all(gc == o["codes"], axis=1)
     gp = g["packed"] if rows is None else g["packed"][rows]
@@ -212,3 +222,59 @@ def test_prepare_replays_identical_under_load(n):
     hfix, _, _ = O.fix_dead_features(Hn, np.zeros((1, n)))
     hd, _ = O.dampen(hfix, 0.01)
     assert rel_fro(np.triu(U0.cpu().numpy()), O.hinv_upper_factor(hd)) <= U_REL_DESIGN
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("name", ["mlp_up_14336x4096", "mlp_down_4096x14336"])
+def test_mlp_pair_full_size_sampled_rows(name):
+    """The MLP pair at full size (8192 tokens, 3-bit g128; the down projection needs a
+    14336-wide factor), in the bench's launch configuration: H and U in full against the oracle,
+    codes / grids on sampled rows."""
+    W, X, spec = synth.workload(name)
+    g = run_gpu(W, X, bits=spec["bits"], group=spec["group"])
+    assert g["status"] == (0, 0)
+    rows = np.random.default_rng(11).choice(spec["m"], size=32, replace=False)
+    o = _oracle(W, X, spec["bits"], spec["group"], False, True, rows=rows)
+    _compare(g, o, W, spec["bits"], spec["group"], rows=rows)
+
+
+@pytest.mark.slow
+def test_clipfree_babai_full_size_sampled_rows():
+    """The clip-free last-to-first variant at full size (4096 x 4096, 3-bit, per-row step chosen
+    so that no entry clips): codes, ladder rounds per row and the Theorem-5 bound on sampled
+    rows."""
+    W, X, spec = synth.workload("clipfree_babai_4096x4096")
+    g = run_gpu(W, X, bits=3, group=0, reverse=True, clip=False)
+    assert g["status"][0] == 0 and g["status"][1] == 0
+    rows = np.random.default_rng(5).choice(4096, size=48, replace=False)
+    o = _oracle(W, X, 3, 0, True, False, rows=rows)
+    _compare(g, o, W, 3, 0, rows=rows)
+
+
+@pytest.mark.slow
+def test_sweep_block_shared_hessian_2bit_g64():
+    """One block of the 8B-shaped sweep: q, k and v share their input, so one H and one factor
+    serve three layers of different heights (2-bit, group 64, 8192 tokens)."""
+    from post_weight_quantization_22_b200 import gq as G
+    T, n = synth.SWEEP_T, 4096
+    x_seed = synth.sweep_seeds(0, 0, "attn")[1]
+    X = synth.to_bf16(synth.make_x("calib", T, n, x_seed))
+    H = torch.zeros((n, n), dtype=torch.float64, device="cuda")
+    G.gq_hessian_accumulate(H, X.cuda())
+    U, dead, delta, _ = G.gq_prepare_hinv(H, 0.01)
+    cfg = G.QuantCfg(bits=2, group_size=64)
+    for li, (name, m, _, kind) in enumerate(synth.SWEEP_LAYERS[:3]):
+        w_seed = synth.sweep_seeds(0, li, kind)[0]
+        W = synth.to_bf16(synth.make_w("layer", m, n, w_seed))
+        codes, scales, zeros, loss, ws = G.gq_quantize_layer(W.cuda(), U, dead, delta, cfg)
+        torch.cuda.synchronize()
+        assert G.gq_workspace_status(ws)[0] == 0
+        packed = codes.cpu().numpy().view(np.uint32)
+        gres = dict(H=H.cpu().numpy(), U=U.cpu().numpy(), packed=packed,
+                    codes=unpack_np(packed, n, 2),
+                    scales=scales.cpu().numpy(), zeros=zeros.cpu().numpy().astype(np.int64),
+                    loss=loss.cpu().numpy(), dead=dead.cpu().numpy().astype(bool),
+                    delta=float(delta.item()))
+        rows = np.random.default_rng(20 + li).choice(m, size=32, replace=False)
+        o = _oracle(W, X, 2, 64, False, True, rows=rows)
+        _compare(gres, o, W, 2, 64, rows=rows)
