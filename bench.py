@@ -258,19 +258,15 @@ def run_gq(args):
              "loss": torch.empty_like(lq.loss, device="cpu").pin_memory()}
     e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
               for _ in range(args.steps)]
+    for _ in range(args.warmup):  # untimed: the host-input path's graphs are captured here
+        lq.run_host(Wh, Xh, out=out_h)
     barrier(device)
     torch.cuda.synchronize(device)
     for k in range(args.steps):
         flush.zero_()
         a, b = e2e_ev[k]
         a.record(stream)
-        Wd.copy_(Wh, non_blocking=True)
-        Xd.copy_(Xh, non_blocking=True)
-        res = lq.run(Wd, Xd)
-        out_h["codes"].copy_(res.codes, non_blocking=True)
-        out_h["scales"].copy_(res.scales, non_blocking=True)
-        out_h["zeros"].copy_(res.zeros, non_blocking=True)
-        out_h["loss"].copy_(res.loss, non_blocking=True)
+        lq.run_host(Wh, Xh, out=out_h)  # pinned host in, pinned host out, copies overlapped
         b.record(stream)
     torch.cuda.synchronize(device)
     barrier(device)
@@ -292,7 +288,7 @@ def run_gq(args):
     dom = int(np.argmax(mean_stage))
     dname = names[dom]
     achieved = work[dname] / (mean_stage[dom] / 1e3) / 1e12
-    roof = {"kernel": {"hessian": "f64_gemm_kernel (H += 2 X^T X)",
+    roof = {"kernel": {"hessian": "hessian_tc_kernel (H += 2 X^T X, int8 digit products)",
                        "factor": "blocked fp64 Cholesky + triangular inverse",
                        "column_loop": "colloop + lazy_update"}[dname],
             "bound": "alu", "achieved": round(achieved, 3), "peak": round(fp64_tf, 2),

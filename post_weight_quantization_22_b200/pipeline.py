@@ -68,6 +68,54 @@ class LayerQuantizer:
         sq, rounds = G.gq_workspace_status(self.ws_quant)
         return sp, sq, rounds
 
+    def run_host(self, W_host: torch.Tensor, X_host: torch.Tensor, out: dict | None = None,
+                 x_chunks: int = 2, stream=None) -> LayerResult:
+        """The whole layer from pinned host tensors, transfers overlapped with the kernels.
+
+        X goes to the device in ``x_chunks`` token slices on a copy stream while H accumulates
+        slice by slice; W goes on the copy stream after X and is waited for only by the column
+        loop; the results are copied into ``out`` (pinned host tensors named codes / scales /
+        zeros / loss) on the compute stream.  Device copies of W and X are kept between calls.
+        """
+        dev = self.H.device
+        cur = torch.cuda.current_stream(dev) if stream is None else stream
+        if not hasattr(self, "_copy_stream"):
+            self._copy_stream = torch.cuda.Stream(device=dev)
+        if getattr(self, "_Wd", None) is None or self._Wd.shape != W_host.shape or self._Wd.dtype != W_host.dtype:
+            self._Wd = torch.empty(W_host.shape, dtype=W_host.dtype, device=dev)
+        if getattr(self, "_Xd", None) is None or self._Xd.shape != X_host.shape or self._Xd.dtype != X_host.dtype:
+            self._Xd = torch.empty(X_host.shape, dtype=X_host.dtype, device=dev)
+        cs = self._copy_stream
+        T = X_host.shape[0]
+        k = max(1, min(int(x_chunks), T))
+        bounds = [(T * i) // k for i in range(k + 1)]
+        cs.wait_stream(cur)  # the previous call's readers of the device copies are done
+        evs = []
+        with torch.cuda.stream(cs):
+            for a, b in zip(bounds[:-1], bounds[1:]):
+                self._Xd[a:b].copy_(X_host[a:b], non_blocking=True)
+                e = torch.cuda.Event()
+                e.record(cs)
+                evs.append(e)
+            self._Wd.copy_(W_host, non_blocking=True)
+            ew = torch.cuda.Event()
+            ew.record(cs)
+        for i, ((a, b), e) in enumerate(zip(zip(bounds[:-1], bounds[1:]), evs)):
+            cur.wait_event(e)
+            if b > a:
+                G.gq_hessian_accumulate(self.H, self._Xd[a:b], accumulate=i > 0,
+                                        ws=self.ws_hess, stream=cur)
+        self.prepare(stream=cur)
+        cur.wait_event(ew)
+        self.quantize(self._Wd, stream=cur)
+        if out is not None:
+            with torch.cuda.stream(cur):
+                out["codes"].copy_(self.codes, non_blocking=True)
+                out["scales"].copy_(self.scales, non_blocking=True)
+                out["zeros"].copy_(self.zeros, non_blocking=True)
+                out["loss"].copy_(self.loss, non_blocking=True)
+        return self.result()
+
     def result(self) -> LayerResult:
         return LayerResult(self.codes, self.scales, self.zeros, self.loss, self.H, self.U,
                            self.dead, self.delta)

@@ -38,6 +38,7 @@ def _compare(g, o, W, bits, group, rows=None, check_loss=True):
     assert abs(g["delta"] - o["delta"]) <= H_REL_DESIGN * abs(o["delta"])  # a mean of diag(H)
     gc = g["codes"] if rows is None else g["codes"][rows]
     match = float(np.mean(gc == o["codes"]))
+    print(f"code match {match:.6f}")
     assert match >= CODE_MATCH, f"code match {match:.6f}"
     gz = g["zeros"] if rows is None else g["zeros"][rows]
     assert float(np.mean(gz == o["zeros"])) >= CODE_MATCH
@@ -278,3 +279,29 @@ def test_sweep_block_shared_hessian_2bit_g64():
         rows = np.random.default_rng(20 + li).choice(m, size=32, replace=False)
         o = _oracle(W, X, 2, 64, False, True, rows=rows)
         _compare(gres, o, W, 2, 64, rows=rows)
+
+
+def test_run_host_overlapped_copies_match_device_run():
+    """LayerQuantizer.run_host (pinned host inputs, transfers overlapped with the kernels) gives
+    the device-input results: bit for bit with X in one slice, and within the parity bar with X
+    in two slices (H's exact digit products are then summed in another order)."""
+    from post_weight_quantization_22_b200 import gq as G
+    from post_weight_quantization_22_b200.pipeline import LayerQuantizer
+    W, X, spec = synth.workload("q_proj_4096x4096", m=512, n=1024, T=1536)
+    cfg = G.QuantCfg(bits=4, group_size=128)
+    ref = LayerQuantizer(512, 1024, cfg, device="cuda")
+    r = ref.run(W.cuda(), X.cuda())
+    codes0, scales0 = r.codes.clone(), r.scales.clone()
+    Wh, Xh = W.pin_memory(), X.pin_memory()
+    lq = LayerQuantizer(512, 1024, cfg, device="cuda")
+    out = {k: torch.empty_like(getattr(lq, k), device="cpu").pin_memory()
+           for k in ("codes", "scales", "zeros", "loss")}
+    lq.run_host(Wh, Xh, out=out, x_chunks=1)
+    torch.cuda.synchronize()
+    assert torch.equal(out["codes"], codes0.cpu()) and torch.equal(out["scales"], scales0.cpu())
+    lq.run_host(Wh, Xh, out=out, x_chunks=2)
+    torch.cuda.synchronize()
+    c1 = unpack_np(out["codes"].numpy().view(np.uint32), 1024, 4)
+    c0 = unpack_np(codes0.cpu().numpy().view(np.uint32), 1024, 4)
+    assert np.mean(c1 == c0) >= CODE_MATCH
+    assert lq.status()[:2] == (0, 0)
