@@ -41,6 +41,8 @@ __all__ = [
     "fix_dead_features",
     "dampen",
     "hinv_upper_factor",
+    "act_order",
+    "min_pivot_order",
     "minmax_grid",
     "clipfree_grid",
     "gptq_columns",
@@ -110,6 +112,49 @@ def hinv_upper_factor(Hd) -> np.ndarray:
     hinv = Linv.T @ Linv
     hinv = 0.5 * (hinv + hinv.T)
     return np.linalg.cholesky(hinv).T
+
+
+# ---------------------------------------------------------------------------------------------
+# Quantization order
+# ---------------------------------------------------------------------------------------------
+
+def act_order(H) -> np.ndarray:
+    """Columns by descending Hessian diagonal ([GEOM] 2.3, the role of the order: "act-order",
+    named there as the cheap approximation of the min-pivot order).
+
+    reading: the diagonal of H after the dead-feature fix (damping adds the same amount to every
+    entry and changes nothing); equal values keep ascending column index.  Returns perm with
+    perm[k] = the original column processed k-th.
+    """
+    d = np.diag(_f64(H))
+    return np.array(sorted(range(d.shape[0]), key=lambda i: (-d[i], i)), dtype=np.int64)
+
+
+def min_pivot_order(Hd) -> np.ndarray:
+    """Greedy min-pivot order ([GEOM] 2.3: Theorem 5's D is the LDL diagonal of the permuted
+    Hessian; the bound is tightened by taking, at each LDL step, the smallest diagonal entry).
+
+    The LDL factorisation eliminates columns one at a time; a column's pivot is its variance
+    given the columns eliminated before it.  Babai decides them in the opposite order (the
+    column eliminated last, conditioned on all others, is decided first), so the processing
+    order is the elimination order reversed.  At each step the remaining column with the
+    smallest current Schur-complement diagonal is eliminated (ties: lowest column index); a
+    non-positive pivot raises LinAlgError.  Returns perm, perm[k] = column processed k-th.
+    """
+    S = _f64(Hd).copy()
+    n = S.shape[0]
+    remaining = list(range(n))
+    elim = []
+    for _ in range(n):
+        k = int(np.argmin([S[i, i] for i in remaining]))  # first minimum = lowest index
+        i = remaining.pop(k)
+        p = S[i, i]
+        if not p > 0.0:
+            raise np.linalg.LinAlgError("non-positive pivot")
+        col = S[:, i].copy()
+        S -= np.outer(col, col) / p  # Schur complement; eliminated rows/columns stay zero
+        elim.append(i)
+    return np.array(elim[::-1], dtype=np.int64)
 
 
 # ---------------------------------------------------------------------------------------------
@@ -294,7 +339,7 @@ def babai_bound(scales_per_col, pivots) -> float:
 
 def quantize_layer(W, X, bits: int, group: int = 0, reverse: bool = False, clip: bool = True,
                    damp: float = 0.01, ladder: float = 1.25, ladder_max: int = 8,
-                   rows=None, H=None):
+                   rows=None, H=None, order=None):
     """Quantize one linear layer: H, dead fix, damping, factor, column loop, losses.
 
     ``W`` is m x n (output rows x input features), ``X`` is T x n.  ``rows`` restricts the
@@ -303,6 +348,10 @@ def quantize_layer(W, X, bits: int, group: int = 0, reverse: bool = False, clip:
 
     Forward order uses the GPTQ form with U (``gptq_columns``).  Reverse order uses the SIC
     form with the lower Cholesky factor of H_d (``babai_sic_reverse``); per-row grids only.
+    ``order`` = "act", "min_pivot" or an explicit permutation (perm[k] = column processed
+    k-th) runs the GPTQ form on the columns in that order, with U the factor of the permuted
+    H_d; group grids then cover consecutive columns of the processing order (reading: the pages
+    do not combine groups with an order), so scales / zeros are indexed by processing group.
 
     clip=False (reading of "per-row step set so that no entry needs clipping"): run unclamped;
     a row whose codes leave [0, 2^b - 1] is rerun with alpha multiplied by ``ladder``, at most
@@ -321,8 +370,31 @@ def quantize_layer(W, X, bits: int, group: int = 0, reverse: bool = False, clip:
     maxq = 2 ** bits - 1
     if reverse and group:
         raise ValueError("the last-to-first variant uses a per-row grid")
+    perm = None
+    if order is not None:
+        if reverse:
+            raise ValueError("an order replaces the reverse flag")
+        if isinstance(order, str):
+            perm = act_order(h_fix) if order == "act" else min_pivot_order(hd) if order == "min_pivot" else None
+            if perm is None:
+                raise ValueError(f"unknown order {order!r}")
+        else:
+            perm = np.asarray(order, dtype=np.int64)
+            if sorted(perm.tolist()) != list(range(n)):
+                raise ValueError("order is not a permutation of the columns")
 
-    if reverse:
+    if perm is not None:
+        U = hinv_upper_factor(hd[np.ix_(perm, perm)])
+        pivots = 1.0 / np.diag(U) ** 2  # in processing order
+
+        def run(rows_w, alpha):
+            r = gptq_columns(rows_w[:, perm], U, bits, group=group, clip=clip, alpha=alpha)
+            for key in ("codes", "Q"):
+                back = np.empty_like(r[key])
+                back[:, perm] = r[key]
+                r[key] = back
+            return r
+    elif reverse:
         L = np.linalg.cholesky(hd)
         pivots = np.diag(L) ** 2
 
@@ -354,9 +426,9 @@ def quantize_layer(W, X, bits: int, group: int = 0, reverse: bool = False, clip:
 
     Q = res["Q"]
     g = group if group else n
-    s_cols = np.repeat(res["scales"], g, axis=1)[:, :n]
+    s_cols = np.repeat(res["scales"], g, axis=1)[:, :n]  # processing order
     out = dict(H=H, dead=dead, delta=delta, Hd=hd, codes=res["codes"], scales=res["scales"],
-               zeros=res["zeros"], Q=Q, alpha=alpha, ladder_rounds=retries)
+               zeros=res["zeros"], Q=Q, alpha=alpha, ladder_rounds=retries, perm=perm)
     if reverse:
         out["L"] = L
     else:
@@ -367,7 +439,8 @@ def quantize_layer(W, X, bits: int, group: int = 0, reverse: bool = False, clip:
     if X is not None:
         out["loss_proxy"] = proxy_loss(w0_sel, Q, X)
     out["loss_proxy_h"] = 0.5 * quadratic_loss(w0_sel, Q, h_fix)
-    # pivots are indexed by original column in both orders: 1/U_jj^2 (forward), L_jj^2 (reverse)
+    # pivots: 1/U_jj^2 in processing order (forward, or an explicit order), L_jj^2 (reverse,
+    # per-row grid, so the column order of s_cols does not matter)
     out["bound"] = babai_bound(s_cols, pivots)
     out["packed"] = pack_codes(np.clip(res["codes"], 0, maxq), bits)
     return out

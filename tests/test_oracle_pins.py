@@ -385,3 +385,122 @@ def test_quantize_layer_sampled_rows_match_full():
     part = O.quantize_layer(w, x, bits=3, group=8, rows=rows)
     assert np.array_equal(part["codes"], full["codes"][rows])
     np.testing.assert_allclose(part["scales"], full["scales"][rows])
+
+
+# --------------------------------------------------------------------------------------------
+# quantization order (GEOM 2.3: the bound depends on the order; min-pivot and act-order)
+# --------------------------------------------------------------------------------------------
+
+def test_act_order_hand_values_and_dead_fix():
+    """act-order = descending Hessian diagonal; equal values keep column order; a dead column
+    counts with its fixed diagonal 1."""
+    assert O.act_order(np.diag([2.0, 5.0, 5.0, 1.0])).tolist() == [1, 2, 0, 3]
+    h = np.diag([0.0, 3.0, 1.0, 0.5])
+    hf, _, dead = O.fix_dead_features(h, np.zeros((1, 4)))
+    assert dead.tolist() == [True, False, False, False]
+    assert O.act_order(hf).tolist() == [1, 0, 2, 3]
+    res = O.quantize_layer(np.ones((1, 4)) * 0.1, None, 4, H=h, order="act")
+    assert res["perm"].tolist() == [1, 0, 2, 3]
+
+
+def test_min_pivot_two_by_two_closed_form():
+    """H = [[a, b], [b, c]], a < c: eliminating column 0 first gives D = (a, c - b^2/a), whose
+    sum is below the other order's a + c - b^2/c; column 0 is then decided last, and in the
+    processing order (1, 0) the pivots are var(x1 | x0) = c - b^2/a and a."""
+    a, b, c = 2.0, 1.5, 5.0
+    h = np.array([[a, b], [b, c]])
+    perm = O.min_pivot_order(h)
+    assert perm.tolist() == [1, 0]
+    U = O.hinv_upper_factor(h[np.ix_(perm, perm)])
+    np.testing.assert_allclose(1.0 / np.diag(U) ** 2, [c - b * b / a, a], rtol=1e-14)
+    assert (c - b * b / a) + a < (a - b * b / c) + c
+
+
+def test_min_pivot_greedy_by_conditional_variances():
+    """Each elimination step takes the remaining column of smallest variance given the columns
+    eliminated before it, computed here from inverses of principal submatrices (no Schur
+    updates); the factor of the permuted Hessian has exactly those pivots, last first."""
+    w, x = _rand_problem(30, 7, 1, seed=91)
+    hd, _ = O.dampen(O.hessian(x), 0.01)
+    perm = O.min_pivot_order(hd)
+    elim = perm[::-1].tolist()
+    chosen = []
+    for k in range(7):
+        E = elim[:k]
+        var = {}
+        for i in range(7):
+            if i in E:
+                continue
+            idx = E + [i]
+            var[i] = 1.0 / np.linalg.inv(hd[np.ix_(idx, idx)])[-1, -1]
+        best = min(var, key=lambda i: (var[i], i))
+        assert elim[k] == best
+        chosen.append(var[best])
+    U = O.hinv_upper_factor(hd[np.ix_(perm, perm)])
+    np.testing.assert_allclose(1.0 / np.diag(U) ** 2, chosen[::-1], rtol=1e-10)
+    # the pivots' product is det(H_d) in every order
+    np.testing.assert_allclose(np.sum(np.log(chosen)), np.linalg.slogdet(hd)[1], rtol=1e-12)
+
+
+@pytest.mark.parametrize("kind", ["act", "min_pivot", "random"])
+def test_ordered_gptq_is_babai_in_that_order(kind):
+    """GEOM 2.2 Theorem 4 with an order T: GPTQ over the columns in processing order equals
+    textbook Babai on the tall basis [sqrt2 X; sqrt(delta) I] diag(s) with the basis columns in
+    the reverse of that order; codes come back in the original column positions."""
+    n, T, m = 10, 40, 40
+    w, x = _rand_problem(T, n, m, seed=95)
+    order = np.random.default_rng(3).permutation(n) if kind == "random" else kind
+    res = O.quantize_layer(w, x, 3, clip=False, order=order)
+    perm = res["perm"]
+    if kind != "random":
+        assert sorted(perm.tolist()) != perm.tolist() or kind == "act"
+    F = np.vstack([np.sqrt(2.0) * x, np.sqrt(res["delta"]) * np.eye(n)])
+    for r in range(m):
+        s = res["scales"][r, 0]
+        u = _babai_gram_schmidt((F * s)[:, perm[::-1]], F @ w[r])
+        expect = np.empty(n, dtype=np.int64)
+        expect[perm[::-1]] = u.astype(np.int64)
+        assert np.array_equal(res["codes"][r] - int(res["zeros"][r, 0]), expect)
+
+
+def test_ordered_groups_cover_processing_order_on_diagonal_hessian():
+    """Diagonal H: no feedback, so GPTQ in any order is round-to-nearest; with groups the grid
+    of group g comes from the original weights of the columns processed g-th (reading: groups
+    follow the processing order)."""
+    rng = np.random.default_rng(97)
+    n, m, g = 12, 9, 4
+    d = rng.uniform(0.5, 3.0, n)
+    w = 0.02 * rng.standard_normal((m, n))
+    res = O.quantize_layer(w, None, 3, group=g, H=np.diag(d), order="act")
+    perm = np.argsort(-d, kind="stable")
+    assert np.array_equal(res["perm"], perm)
+    for k in range(n // g):
+        cols = perm[k * g:(k + 1) * g]
+        lo = np.minimum(w[:, cols].min(axis=1), 0.0)
+        hi = np.maximum(w[:, cols].max(axis=1), 0.0)
+        s = (hi - lo) / 7.0
+        z = np.rint(-lo / s)
+        np.testing.assert_array_equal(res["scales"][:, k], s)
+        code = np.clip(np.rint(w[:, cols] / s[:, None]) + z[:, None], 0, 7)
+        np.testing.assert_array_equal(res["codes"][:, cols], code)
+
+
+@pytest.mark.parametrize("order", ["act", "min_pivot"])
+def test_clipfree_bound_holds_in_every_order(order):
+    """GEOM 2.3 Theorem 5 for the permuted Hessian: the clip-free damped loss of the whole layer
+    stays below (1/4) sum s^2 D in that order's pivots."""
+    w, x = _rand_problem(200, 32, 48, seed=99)
+    res = O.quantize_layer(w, x, 3, clip=False, order=order)
+    assert res["loss_damped"] <= res["bound"] * (1 + 1e-12)
+
+
+def test_identity_and_reversal_orders_match_the_flags():
+    """order = identity is the forward path; order = reversed columns (per-row grid) gives the
+    codes of the last-to-first SIC form."""
+    w, x = _rand_problem(80, 16, 20, seed=101)
+    nat = O.quantize_layer(w, x, 4, group=8)
+    idn = O.quantize_layer(w, x, 4, group=8, order=np.arange(16))
+    assert np.array_equal(nat["codes"], idn["codes"])
+    rev = O.quantize_layer(w, x, 3, reverse=True)
+    prm = O.quantize_layer(w, x, 3, order=np.arange(16)[::-1])
+    assert np.array_equal(rev["codes"], prm["codes"])
