@@ -50,6 +50,21 @@ typedef enum {
 
 typedef enum { GQ_BF16 = 0, GQ_FP32 = 1 } gq_dtype;
 
+/* Column processing order ("The Geometry of LLM Quantization", section 2.3: Theorem 5's bound
+ * is (1/4) sum s^2 D over the LDL pivots D of the Hessian permuted into the quantization
+ * order, so the order changes the bound; the min-pivot order takes the smallest pivot at each
+ * LDL step and "act-order" (descending Hessian diagonal) is its cheap approximation).  A
+ * permutation perm lists the original columns in processing order: perm[k] = the column
+ * processed k-th. */
+typedef enum {
+  GQ_ORDER_NATURAL = 0,   /* columns 0, 1, ..., n-1 (GPTQ order) */
+  GQ_ORDER_REVERSE = 1,   /* columns n-1, ..., 0 (Babai order) */
+  GQ_ORDER_ACT = 2,       /* descending diagonal of H after the dead fix; ties by column index */
+  GQ_ORDER_MIN_PIVOT = 3, /* greedy min-pivot: the reverse of the elimination order of a
+                             pivoted LDL of H_d that always eliminates the smallest pivot */
+  GQ_ORDER_GIVEN = 4      /* the caller's permutation */
+} gq_order;
+
 /* Quantization settings of one call of gq_quantize_layer. */
 typedef struct {
   int bits;       /* code width b, 2..8 */
@@ -148,6 +163,22 @@ gq_status gq_prepare_hinv_static(const double* d_H, int64_t n, double damp, int 
                                  float* d_U, uint8_t* d_dead, double* d_delta, int* d_status,
                                  gq_stream_t stream);
 
+/*
+ * gq_prepare_hinv in a chosen column order: U = the upper Cholesky factor of (P H_d P^T)^-1,
+ * P the permutation matrix of the processing order (row k of P H_d P^T is column perm[k] of
+ * H_d).  Same arguments, results and workspace as gq_prepare_hinv, plus:
+ *
+ *   order    a gq_order.  NATURAL and REVERSE give exactly gq_prepare_hinv's U with
+ *            reverse = 0 / 1 (d_perm is then not touched and may be NULL).
+ *   d_perm   n int32, device.  ACT and MIN_PIVOT write the order computed on the device from
+ *            H; GIVEN reads it.  Pass the same array to gq_quantize_layer_ordered.
+ * Device-detected errors: GQ_ERR_INVALID_ARG (GIVEN: d_perm is not a permutation of 0..n-1;
+ * every access stays in bounds and U is then undefined), GQ_ERR_NOT_PD.
+ */
+gq_status gq_prepare_hinv_ordered(const double* d_H, int64_t n, double damp, gq_order order,
+                                  int32_t* d_perm, float* d_U, uint8_t* d_dead, double* d_delta,
+                                  void* d_ws, size_t ws_bytes, gq_stream_t stream);
+
 /* Workspace bytes gq_quantize_layer needs for an m x n layer under cfg. */
 size_t gq_quantize_workspace_size(int64_t m, int64_t n, const gq_quant_cfg* cfg);
 
@@ -184,6 +215,24 @@ gq_status gq_quantize_layer(const void* d_W, gq_dtype w_dtype, int64_t m, int64_
                             const gq_quant_cfg* cfg, uint32_t* d_codes, float* d_scales,
                             uint8_t* d_zeros, double* d_loss, void* d_ws, size_t ws_bytes,
                             gq_stream_t stream);
+
+/*
+ * gq_quantize_layer with the columns processed in the order d_perm (n int32, device, from
+ * gq_prepare_hinv_ordered; d_U must be the factor of that order).  cfg->reverse must be 0.
+ * The packed codes are still indexed by ORIGINAL column.  Group grids cover consecutive
+ * columns of the processing order: group g of a row covers original columns
+ * d_perm[g*group_size .. (g+1)*group_size - 1] (the usual act-order convention; for a
+ * dequantizer, the group of original column c is (position of c in d_perm) / group_size).
+ * The Theorem 5 bound uses the pivots of the processing order.
+ * Device-detected errors: GQ_ERR_INVALID_ARG (d_perm is not a permutation; every access stays
+ * in bounds and the outputs are then undefined), GQ_ERR_NO_FIT.
+ */
+gq_status gq_quantize_layer_ordered(const void* d_W, gq_dtype w_dtype, int64_t m, int64_t n,
+                                    const float* d_U, const uint8_t* d_dead,
+                                    const double* d_delta, const gq_quant_cfg* cfg,
+                                    const int32_t* d_perm, uint32_t* d_codes, float* d_scales,
+                                    uint8_t* d_zeros, double* d_loss, void* d_ws,
+                                    size_t ws_bytes, gq_stream_t stream);
 
 /*
  * Synchronize `stream` and return the device-side status recorded in a workspace by the last

@@ -172,10 +172,33 @@ gq_status gq_prepare_hinv(const double* d_H, int64_t n, double damp, int reverse
   gq_status st = ensure_device_setup();
   if (st != GQ_OK) return st;
   auto enqueue = [&](cudaStream_t s) {
-    return launch_prepare(d_H, n, damp, reverse, d_U, d_dead, d_delta, d_ws, s) == cudaSuccess
+    return launch_prepare(d_H, n, damp, reverse, nullptr, d_U, d_dead, d_delta, d_ws, s) ==
+                   cudaSuccess
                ? GQ_OK : GQ_ERR_CUDA;
   };
   return run_graphed({1, P(d_H), (uint64_t)n, bits_of(damp), (uint64_t)reverse, P(d_U),
+                      P(d_dead), P(d_delta), P(d_ws)},
+                     (cudaStream_t)stream, enqueue);
+}
+
+gq_status gq_prepare_hinv_ordered(const double* d_H, int64_t n, double damp, gq_order order,
+                                  int32_t* d_perm, float* d_U, uint8_t* d_dead, double* d_delta,
+                                  void* d_ws, size_t ws_bytes, gq_stream_t stream) {
+  const int o = (int)order;
+  if (o < GQ_ORDER_NATURAL || o > GQ_ORDER_GIVEN) return GQ_ERR_INVALID_ARG;
+  if (o == GQ_ORDER_NATURAL || o == GQ_ORDER_REVERSE)
+    return gq_prepare_hinv(d_H, n, damp, o, d_U, d_dead, d_delta, d_ws, ws_bytes, stream);
+  if (n < 1 || n > kMaxN || !(damp >= 0.0)) return GQ_ERR_INVALID_ARG;
+  if (!d_H || !d_U || !d_dead || !d_delta || !d_ws || !d_perm) return GQ_ERR_INVALID_ARG;
+  if (o == GQ_ORDER_MIN_PIVOT) return GQ_ERR_UNSUPPORTED;
+  if (!aligned256(d_ws) || ws_bytes < prepare_ws_bytes(n)) return GQ_ERR_WORKSPACE;
+  gq_status st = ensure_device_setup();
+  if (st != GQ_OK) return st;
+  auto enqueue = [&](cudaStream_t s) {
+    return launch_prepare(d_H, n, damp, o, d_perm, d_U, d_dead, d_delta, d_ws, s) == cudaSuccess
+               ? GQ_OK : GQ_ERR_CUDA;
+  };
+  return run_graphed({4, P(d_H), (uint64_t)n, bits_of(damp), (uint64_t)o, P(d_perm), P(d_U),
                       P(d_dead), P(d_delta), P(d_ws)},
                      (cudaStream_t)stream, enqueue);
 }
@@ -202,11 +225,12 @@ size_t gq_quantize_workspace_size(int64_t m, int64_t n, const gq_quant_cfg* cfg)
   return quantize_ws_bytes(m, n, *cfg);
 }
 
-gq_status gq_quantize_layer(const void* d_W, gq_dtype w_dtype, int64_t m, int64_t n,
-                            const float* d_U, const uint8_t* d_dead, const double* d_delta,
-                            const gq_quant_cfg* cfg, uint32_t* d_codes, float* d_scales,
-                            uint8_t* d_zeros, double* d_loss, void* d_ws, size_t ws_bytes,
-                            gq_stream_t stream) {
+static gq_status quantize_common(const void* d_W, gq_dtype w_dtype, int64_t m, int64_t n,
+                                 const float* d_U, const uint8_t* d_dead, const double* d_delta,
+                                 const gq_quant_cfg* cfg, const int32_t* d_perm,
+                                 uint32_t* d_codes, float* d_scales, uint8_t* d_zeros,
+                                 double* d_loss, void* d_ws, size_t ws_bytes,
+                                 gq_stream_t stream) {
   if (m < 1 || m > kMaxM || n < 1 || n > kMaxN) return GQ_ERR_INVALID_ARG;
   if (w_dtype != GQ_BF16 && w_dtype != GQ_FP32) return GQ_ERR_INVALID_ARG;
   gq_status st = check_cfg(cfg);
@@ -220,14 +244,34 @@ gq_status gq_quantize_layer(const void* d_W, gq_dtype w_dtype, int64_t m, int64_
   QuantArgs a{};
   a.W = d_W; a.wt = w_dtype; a.m = m; a.n = n; a.U = d_U; a.dead = d_dead; a.delta = d_delta;
   a.cfg = *cfg; a.codes = d_codes; a.scales = d_scales; a.zeros = d_zeros; a.loss = d_loss;
-  a.ws = d_ws;
+  a.ws = d_ws; a.perm = d_perm;
   if (!cfg->clip) return run_quantize(a, (cudaStream_t)stream);  // the ladder reads back counts
   auto enqueue = [&](cudaStream_t s) { return run_quantize(a, s); };
   return run_graphed({2, P(d_W), (uint64_t)w_dtype, (uint64_t)m, (uint64_t)n, P(d_U), P(d_dead),
                       P(d_delta), (uint64_t)cfg->bits, (uint64_t)cfg->group_size,
-                      (uint64_t)cfg->reverse, (uint64_t)cfg->clip, P(d_codes), P(d_scales),
-                      P(d_zeros), P(d_loss), P(d_ws)},
+                      (uint64_t)cfg->reverse, (uint64_t)cfg->clip, P(d_perm), P(d_codes),
+                      P(d_scales), P(d_zeros), P(d_loss), P(d_ws)},
                      (cudaStream_t)stream, enqueue);
+}
+
+gq_status gq_quantize_layer(const void* d_W, gq_dtype w_dtype, int64_t m, int64_t n,
+                            const float* d_U, const uint8_t* d_dead, const double* d_delta,
+                            const gq_quant_cfg* cfg, uint32_t* d_codes, float* d_scales,
+                            uint8_t* d_zeros, double* d_loss, void* d_ws, size_t ws_bytes,
+                            gq_stream_t stream) {
+  return quantize_common(d_W, w_dtype, m, n, d_U, d_dead, d_delta, cfg, nullptr, d_codes,
+                         d_scales, d_zeros, d_loss, d_ws, ws_bytes, stream);
+}
+
+gq_status gq_quantize_layer_ordered(const void* d_W, gq_dtype w_dtype, int64_t m, int64_t n,
+                                    const float* d_U, const uint8_t* d_dead,
+                                    const double* d_delta, const gq_quant_cfg* cfg,
+                                    const int32_t* d_perm, uint32_t* d_codes, float* d_scales,
+                                    uint8_t* d_zeros, double* d_loss, void* d_ws,
+                                    size_t ws_bytes, gq_stream_t stream) {
+  if (!d_perm || !cfg || cfg->reverse) return GQ_ERR_INVALID_ARG;
+  return quantize_common(d_W, w_dtype, m, n, d_U, d_dead, d_delta, cfg, d_perm, d_codes,
+                         d_scales, d_zeros, d_loss, d_ws, ws_bytes, stream);
 }
 
 gq_status gq_workspace_status(void* d_ws, int* h_ladder_rounds, gq_stream_t stream) {

@@ -71,6 +71,83 @@ __global__ void build_m_kernel(const double* H, int64_t n, int64_t ldm, int reve
   M[i * ldm + j] = v;
 }
 
+// ---------------------------------------------------------------------------------------
+// Column orders ("The Geometry of LLM Quantization", section 2.3, the role of the order)
+// ---------------------------------------------------------------------------------------
+// act-order sort key: the diagonal after the dead fix (0 -> 1); NaN sorts last, so the keys
+// are totally ordered and the ranks below always form a permutation.
+__device__ __forceinline__ double act_key(double v) {
+  if (v == 0.0) return 1.0;
+  return (v == v) ? v : -INFINITY;
+}
+
+constexpr int kActCols = 128;  // columns ranked per CTA (8 threads each)
+
+// perm[rank(i)] = i, rank(i) = #{j : key_j > key_i} + #{j < i : key_j == key_i}: the columns
+// by descending Hessian diagonal, ties in column order.  O(n^2) comparisons, each CTA ranking
+// 128 columns against all n keys staged through shared memory.
+__global__ void __launch_bounds__(1024) act_order_kernel(const double* H, int64_t n, int* perm) {
+  __shared__ double keys[1024];
+  const int sub = threadIdx.x & 7;
+  const int64_t i = blockIdx.x * (int64_t)kActCols + (threadIdx.x >> 3);
+  const double ki = (i < n) ? act_key(H[i * n + i]) : 0.0;
+  int rank = 0;
+  for (int64_t j0 = 0; j0 < n; j0 += 1024) {
+    __syncthreads();
+    const int64_t jj = j0 + threadIdx.x;
+    keys[threadIdx.x] = (jj < n) ? act_key(H[jj * n + jj]) : 0.0;
+    __syncthreads();
+    const int lim = (int)((n - j0) < 1024 ? (n - j0) : 1024);
+    for (int k = sub; k < lim; k += 8) {
+      const double kj = keys[k];
+      rank += (kj > ki) || (kj == ki && j0 + k < i);
+    }
+  }
+  rank += __shfl_xor_sync(0xffffffffu, rank, 1);
+  rank += __shfl_xor_sync(0xffffffffu, rank, 2);
+  rank += __shfl_xor_sync(0xffffffffu, rank, 4);
+  if (sub == 0 && i < n) perm[rank] = (int)i;
+}
+
+// A caller's permutation: every entry in [0, n) and none repeated (mark zeroed beforehand);
+// otherwise GQ_ERR_INVALID_ARG is recorded.
+__global__ void perm_check_kernel(const int* perm, int64_t n, int* mark, WsHeader* hdr) {
+  for (int64_t k = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; k < n;
+       k += (int64_t)gridDim.x * blockDim.x) {
+    const unsigned p = (unsigned)perm[k];
+    if (p >= (unsigned long long)n || atomicExch(&mark[p], 1) != 0)
+      record_status(hdr, GQ_ERR_INVALID_ARG);
+  }
+}
+
+// M[i][j] (j <= i) = Hfix[pi(i)][pi(j)] + (i == j) * delta with pi(i) = perm[n-1-i]: M is the
+// permuted Hessian in the reverse of the processing order.  One CTA per row of M; the row
+// pi(i) of H is staged in shared memory (coalesced) when `stage`, so the gather of its
+// columns reads shared memory.
+constexpr int64_t kStageMaxN = 25600;  // 200 KB of shared memory per staged row
+__global__ void __launch_bounds__(256) build_m_perm_kernel(const double* H, int64_t n,
+                                                           int64_t ldm, const int* perm,
+                                                           int stage, const WsHeader* hdr,
+                                                           double* M) {
+  extern __shared__ double srow[];
+  const int64_t i = blockIdx.x;
+  const double* hrow = H + perm_at(perm, n - 1 - i, n) * n;
+  if (stage) {
+    for (int64_t c = threadIdx.x; c < n; c += blockDim.x) srow[c] = hrow[c];
+    __syncthreads();
+  }
+  const double delta = hdr->scratch[0];
+  for (int64_t j = threadIdx.x; j <= i; j += blockDim.x) {
+    const int64_t pj = perm_at(perm, n - 1 - j, n);
+    double v = stage ? srow[pj] : hrow[pj];
+    if (i == j) {
+      if (v == 0.0) v = 1.0;
+      v += delta;
+    }
+    M[i * ldm + j] = v;
+  }
+}
+
 // 1/p for p > 0: the hardware reciprocal estimate (rcp.approx.ftz.f64, about 2^-22 relative)
 // refined by two Newton-Raphson steps r <- r + r (1 - p r), each squaring the relative error,
 // to fp64 precision.  It replaces an IEEE division on the leaf's per-pivot critical path; the
@@ -309,6 +386,7 @@ struct PrepLayout {
   double* T;     // n x ldm: block rows of L X accumulated for the inverse (lower blocks)
   double* Dinv;  // ceil(n / 64) x 64 x 64: the inverted 64-wide leaves
   double* tbuf;  // doubling scratch of the diagonal super-block inverses
+  int* pmark;    // n ints: occurrence marks when checking a caller's permutation
   size_t bytes;
 };
 
@@ -331,6 +409,7 @@ static PrepLayout prep_layout(void* ws, int64_t n) {
   L.T = c.take<double>((size_t)n * m_ld(n));
   L.Dinv = c.take<double>((size_t)((n + kNB - 1) / kNB) * kNB * kNB);
   L.tbuf = c.take<double>(trtri_tbuf_elems(kSuper) + 1);
+  L.pmark = c.take<int>((size_t)n);
   L.bytes = c.off;
   return L;
 }
@@ -340,6 +419,9 @@ size_t prepare_ws_bytes(int64_t n) { return prep_layout(nullptr, n).bytes; }
 cudaError_t factor_init_attributes() {
   cudaError_t e = cudaFuncSetAttribute(potrf_panel_kernel,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kPnSmem);
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(build_m_perm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)(kStageMaxN * sizeof(double)));
   if (e != cudaSuccess) return e;
   return dgemm_init_attributes();
 }
@@ -432,8 +514,9 @@ static cudaError_t prep_streams(PrepStreams** out) {
   return cudaSuccess;
 }
 
-cudaError_t launch_prepare(const double* H, int64_t n, double damp, int reverse, float* U,
-                           uint8_t* dead, double* delta, void* ws, cudaStream_t s0) {
+cudaError_t launch_prepare(const double* H, int64_t n, double damp, int order, int* perm,
+                           float* U, uint8_t* dead, double* delta, void* ws, cudaStream_t s0) {
+  if (order == GQ_ORDER_MIN_PIVOT) return cudaErrorNotSupported;
   PrepLayout L = prep_layout(ws, n);
   const int64_t ldm = m_ld(n);
   int dev = 0, sms = 148;
@@ -450,9 +533,26 @@ cudaError_t launch_prepare(const double* H, int64_t n, double damp, int reverse,
   diag_stats_kernel<<<1, 1024, 0, s>>>(H, n, damp, dead, delta, L.hdr);
   count_launches(1);
   GQ_TRY(cudaGetLastError());
-  {
+  if (order == GQ_ORDER_ACT) {
+    act_order_kernel<<<(unsigned)((n + kActCols - 1) / kActCols), 1024, 0, s>>>(H, n, perm);
+    count_launches(1);
+    GQ_TRY(cudaGetLastError());
+  } else if (order == GQ_ORDER_GIVEN) {
+    GQ_TRY(cudaMemsetAsync(L.pmark, 0, (size_t)n * sizeof(int), s));
+    perm_check_kernel<<<(unsigned)std::min<int64_t>((n + 255) / 256, 1024), 256, 0, s>>>(
+        perm, n, L.pmark, L.hdr);
+    count_launches(1);
+    GQ_TRY(cudaGetLastError());
+  }
+  if (order == GQ_ORDER_NATURAL || order == GQ_ORDER_REVERSE) {
     dim3 grid((unsigned)((n + 255) / 256), (unsigned)n);
-    build_m_kernel<<<grid, 256, 0, s>>>(H, n, ldm, reverse, L.hdr, L.M);
+    build_m_kernel<<<grid, 256, 0, s>>>(H, n, ldm, order == GQ_ORDER_REVERSE, L.hdr, L.M);
+    count_launches(1);
+    GQ_TRY(cudaGetLastError());
+  } else {
+    const int stage = n <= kStageMaxN;
+    build_m_perm_kernel<<<(unsigned)n, 256, stage ? (size_t)n * sizeof(double) : 0, s>>>(
+        H, n, ldm, perm, stage, L.hdr, L.M);
     count_launches(1);
     GQ_TRY(cudaGetLastError());
   }

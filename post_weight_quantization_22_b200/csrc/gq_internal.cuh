@@ -49,8 +49,17 @@ cudaError_t launch_hessian(double* H, const void* X, gq_dtype xt, int64_t T, int
 
 // ---- factor preparation ----
 size_t prepare_ws_bytes(int64_t n);
-cudaError_t launch_prepare(const double* H, int64_t n, double damp, int reverse, float* U,
-                           uint8_t* dead, double* delta, void* ws, cudaStream_t s);
+// order: a gq_order value; perm (n ints) is written for ACT / MIN_PIVOT, read for GIVEN and
+// not used for NATURAL / REVERSE (may be null there).
+cudaError_t launch_prepare(const double* H, int64_t n, double damp, int order, int* perm,
+                           float* U, uint8_t* dead, double* delta, void* ws, cudaStream_t s);
+
+// perm[k] as an index that is always in [0, n) (0 for an out-of-range entry; a caller-given
+// permutation is validated separately and reported through the workspace status).
+__device__ __forceinline__ int64_t perm_at(const int* perm, int64_t k, int64_t n) {
+  unsigned p = (unsigned)perm[k];
+  return p < (unsigned long long)n ? (int64_t)p : 0;
+}
 
 // ---- quantization ----
 struct QuantArgs {
@@ -66,6 +75,7 @@ struct QuantArgs {
   uint8_t* zeros;
   double* loss;
   void* ws;
+  const int* perm;  // processing order (null: natural, or reversed when cfg.reverse)
 };
 size_t quantize_ws_bytes(int64_t m, int64_t n, const gq_quant_cfg& cfg);
 // Returns GQ_OK or an error; the clip-free ladder synchronizes the stream per round.

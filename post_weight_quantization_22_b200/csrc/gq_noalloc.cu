@@ -62,7 +62,7 @@ extern "C" gq_status gq_prepare_hinv_static(const double* d_H, int64_t n, double
   cudaStream_t s = (cudaStream_t)stream;
   // launch_prepare clears the scratch's status word first and writes every other scratch
   // element it reads before reading it, so the previous call's contents do not leak in.
-  if (gq::launch_prepare(d_H, n, damp, reverse, d_U, d_dead, d_delta, scratch, s) != cudaSuccess)
+  if (gq::launch_prepare(d_H, n, damp, reverse, nullptr, d_U, d_dead, d_delta, scratch, s) != cudaSuccess)
     return GQ_ERR_CUDA;
   if (d_status &&
       cudaMemcpyAsync(d_status, scratch, sizeof(int), cudaMemcpyDeviceToDevice, s) != cudaSuccess)

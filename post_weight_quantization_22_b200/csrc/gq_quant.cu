@@ -52,6 +52,7 @@ struct QLayout {
   int* overflow;    // per-row clip-free overflow flag
   int* rowlist;     // compact row -> original row
   int* counter;
+  int* iperm;       // n: processing position of each original column (ordered calls)
   size_t bytes;
 };
 
@@ -79,6 +80,7 @@ static QLayout q_layout(void* ws, int64_t m, int64_t n) {
   L.overflow = c.take<int>(m);
   L.rowlist = c.take<int>(m);
   L.counter = c.take<int>(4);
+  L.iperm = c.take<int>((size_t)n);
   L.bytes = c.off;
   return L;
 }
@@ -111,6 +113,40 @@ __global__ void q_load_kernel(const TW* W, int64_t n, int64_t k_rows, const int*
     else v = (float)W[row * n + c];
     if (dead && dead[c]) v = 0.f;
     Wf[e] = v;
+  }
+}
+
+// Ordered calls: Wf[r'][p] = dead[perm[p]] ? 0 : W[row][perm[p]].  One CTA per row; the row
+// is staged in shared memory (coalesced reads) and gathered from there.
+template <class TW>
+__global__ void __launch_bounds__(256) q_load_perm_kernel(const TW* W, int64_t n,
+                                                          const int* rowlist,
+                                                          const uint8_t* dead, const int* perm,
+                                                          float* Wf) {
+  extern __shared__ float srow[];
+  const int64_t rr = blockIdx.x;
+  const int64_t row = rowlist ? rowlist[rr] : rr;
+  const TW* wrow = W + row * n;
+  for (int64_t c = threadIdx.x; c < n; c += blockDim.x) {
+    float v;
+    if constexpr (sizeof(TW) == 2) v = __bfloat162float(wrow[c]);
+    else v = (float)wrow[c];
+    if (dead && dead[c]) v = 0.f;
+    srow[c] = v;
+  }
+  __syncthreads();
+  float* out = Wf + rr * n;
+  for (int64_t p = threadIdx.x; p < n; p += blockDim.x) out[p] = srow[perm_at(perm, p, n)];
+}
+
+// iperm[perm[k]] = k (iperm preset to -1); a repeated or out-of-range entry records
+// GQ_ERR_INVALID_ARG.
+__global__ void perm_invert_kernel(const int* perm, int64_t n, int* iperm, WsHeader* hdr) {
+  for (int64_t k = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; k < n;
+       k += (int64_t)gridDim.x * blockDim.x) {
+    const unsigned p = (unsigned)perm[k];
+    if (p >= (unsigned long long)n || atomicExch(&iperm[p], (int)k) != -1)
+      record_status(hdr, GQ_ERR_INVALID_ARG);
   }
 }
 
@@ -416,19 +452,30 @@ __global__ void __launch_bounds__(kColThreads, 1) colloop_kernel(ColArgs a) {
 template <class TW>
 __global__ void __launch_bounds__(128) pack_kernel(const TW* W, const uint8_t* dead, int64_t n,
                                                    const uint8_t* codes8, int64_t ldc8,
-                                                   int reverse, int bits, int group,
+                                                   const int* iperm, int reverse, int bits,
+                                                   int group,
                                                    int64_t ngroups, const float* scales,
                                                    const uint8_t* zeros, uint32_t* codes,
                                                    double* row_d2) {
   const int64_t r = blockIdx.x;
   const uint8_t* crow = codes8 + r * ldc8;
+  if (iperm) {  // ordered call: gather the codes from a shared-memory copy of the row
+    extern __shared__ uint8_t scodes[];
+    for (int64_t p = threadIdx.x; p < n; p += blockDim.x) scodes[p] = crow[p];
+    __syncthreads();
+    crow = scodes;
+  }
+  // processing position of original column c
+  auto pos = [&](int64_t c) -> int64_t {
+    return iperm ? perm_at(iperm, c, n) : (reverse ? n - 1 - c : c);
+  };
   const int64_t nwords = (n * bits + 31) / 32;
   for (int64_t w = threadIdx.x; w < nwords; w += blockDim.x) {
     uint32_t word = 0u;
     int64_t cf = (32 * w) / bits, cl = (32 * w + 31) / bits;
     if (cl > n - 1) cl = n - 1;
     for (int64_t c = cf; c <= cl; ++c) {
-      uint32_t code = crow[reverse ? n - 1 - c : c];
+      uint32_t code = crow[pos(c)];
       int64_t pos = (int64_t)bits * c - 32 * w;
       if (pos >= 0) word |= code << pos;
       else word |= code >> (-pos);
@@ -441,9 +488,10 @@ __global__ void __launch_bounds__(128) pack_kernel(const TW* W, const uint8_t* d
     if constexpr (sizeof(TW) == 2) w0 = __bfloat162float(W[r * n + c]);
     else w0 = (float)W[r * n + c];
     if (dead && dead[c]) w0 = 0.f;
-    int64_t g = group ? c / group : 0;
+    const int64_t pc = pos(c);
+    int64_t g = group ? pc / group : 0;  // groups follow the processing order
     float s = scales[r * ngroups + g], z = (float)zeros[r * ngroups + g];
-    float code = (float)crow[reverse ? n - 1 - c : c];
+    float code = (float)crow[pc];
     double d = (double)w0 - (double)s * (double)(code - z);
     acc += d * d;
   }
@@ -520,7 +568,10 @@ cudaError_t quant_init_attributes() {
   if ((e = cudaFuncSetAttribute(colloop_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem))) return e;
   if ((e = cudaFuncSetAttribute(colloop_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem))) return e;
   if ((e = cudaFuncSetAttribute(colloop_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem))) return e;
-  return cudaFuncSetAttribute(colloop_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if ((e = cudaFuncSetAttribute(colloop_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem))) return e;
+  const int row_smem = 32768 * (int)sizeof(float);  // a staged row of the widest layer
+  if ((e = cudaFuncSetAttribute(q_load_perm_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, row_smem))) return e;
+  return cudaFuncSetAttribute(q_load_perm_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, row_smem);
 }
 
 template <int G>
@@ -596,6 +647,13 @@ gq_status run_quantize(const QuantArgs& a, cudaStream_t s) {
     count_launches(1);
     Q_TRY(cudaGetLastError());
   }
+  if (a.perm) {
+    Q_TRY(cudaMemsetAsync(L.iperm, 0xff, (size_t)n * sizeof(int), s));
+    perm_invert_kernel<<<(unsigned)std::min<int64_t>((n + 255) / 256, 1024), 256, 0, s>>>(
+        a.perm, n, L.iperm, L.hdr);
+    count_launches(1);
+    Q_TRY(cudaGetLastError());
+  }
   int64_t k_rows = m;
   const int* rowlist = nullptr;
   const int nblocks = (int)((n + kBlock - 1) / kBlock);
@@ -603,7 +661,17 @@ gq_status run_quantize(const QuantArgs& a, cudaStream_t s) {
   int rounds_run = 0;
   for (int round = 0; round < max_rounds; ++round) {
     rounds_run = round;
-    {
+    if (a.perm) {
+      const size_t sm = (size_t)n * sizeof(float);
+      if (a.wt == GQ_BF16)
+        q_load_perm_kernel<__nv_bfloat16><<<(unsigned)k_rows, 256, sm, s>>>(
+            static_cast<const __nv_bfloat16*>(a.W), n, rowlist, a.dead, a.perm, L.Wf);
+      else
+        q_load_perm_kernel<float><<<(unsigned)k_rows, 256, sm, s>>>(
+            static_cast<const float*>(a.W), n, rowlist, a.dead, a.perm, L.Wf);
+      count_launches(1);
+      Q_TRY(cudaGetLastError());
+    } else {
       int64_t total = k_rows * n;
       unsigned grid = (unsigned)std::min<int64_t>((total + 255) / 256, 148 * 64);
       if (a.wt == GQ_BF16)
@@ -697,14 +765,16 @@ gq_status run_quantize(const QuantArgs& a, cudaStream_t s) {
     Q_TRY(cudaMemcpyAsync(&L.hdr->ladder_rounds, &rr, sizeof(int), cudaMemcpyHostToDevice, s));
     Q_TRY(cudaStreamSynchronize(s));
   }
+  const int* iperm = a.perm ? L.iperm : nullptr;
+  const size_t pack_smem = a.perm ? (size_t)n : 0;
   if (a.wt == GQ_BF16)
-    pack_kernel<__nv_bfloat16><<<(unsigned)m, 128, 0, s>>>(
-        static_cast<const __nv_bfloat16*>(a.W), a.dead, n, L.codes8, L.ldc8, cfg.reverse,
-        cfg.bits, G, ngroups, a.scales, a.zeros, a.codes, L.row_d2);
+    pack_kernel<__nv_bfloat16><<<(unsigned)m, 128, pack_smem, s>>>(
+        static_cast<const __nv_bfloat16*>(a.W), a.dead, n, L.codes8, L.ldc8, iperm,
+        cfg.reverse, cfg.bits, G, ngroups, a.scales, a.zeros, a.codes, L.row_d2);
   else
-    pack_kernel<float><<<(unsigned)m, 128, 0, s>>>(static_cast<const float*>(a.W), a.dead, n,
-                                                   L.codes8, L.ldc8, cfg.reverse, cfg.bits, G,
-                                                   ngroups, a.scales, a.zeros, a.codes, L.row_d2);
+    pack_kernel<float><<<(unsigned)m, 128, pack_smem, s>>>(
+        static_cast<const float*>(a.W), a.dead, n, L.codes8, L.ldc8, iperm, cfg.reverse,
+        cfg.bits, G, ngroups, a.scales, a.zeros, a.codes, L.row_d2);
   count_launches(1);
   Q_TRY(cudaGetLastError());
   q_reduce_kernel<<<1, 1024, 0, s>>>(m, L.row_e2, L.row_bnd, L.row_d2, a.delta, a.loss);

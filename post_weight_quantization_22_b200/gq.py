@@ -18,6 +18,7 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libgq.so")
 
 GQ_BF16, GQ_FP32 = 0, 1
+ORDERS = {"natural": 0, "reverse": 1, "act": 2, "min_pivot": 3, "given": 4}  # gq_order
 STATUS = {0: "ok", 1: "invalid argument", 2: "not positive definite", 3: "CUDA error",
           4: "unsupported", 5: "timeout", 6: "no fit", 7: "workspace"}
 
@@ -55,6 +56,11 @@ def _load():
     lib.gq_quantize_layer.restype = I
     lib.gq_quantize_layer.argtypes = [P, I, I64, I64, P, P, P, ctypes.POINTER(_Cfg), P, P, P, P,
                                       P, SZ, P]
+    lib.gq_prepare_hinv_ordered.restype = I
+    lib.gq_prepare_hinv_ordered.argtypes = [P, I64, ctypes.c_double, I, P, P, P, P, P, SZ, P]
+    lib.gq_quantize_layer_ordered.restype = I
+    lib.gq_quantize_layer_ordered.argtypes = [P, I, I64, I64, P, P, P, ctypes.POINTER(_Cfg), P,
+                                              P, P, P, P, P, SZ, P]
     lib.gq_prepare_hinv_static.restype = I
     lib.gq_prepare_hinv_static.argtypes = [P, I64, ctypes.c_double, I, P, P, P, P, P]
     lib.gq_workspace_status.restype = I
@@ -66,7 +72,8 @@ LIB = _load()
 EXPORTED = ("gq_version", "gq_status_string", "gq_hessian_accumulate", "gq_hessian_workspace_size",
             "gq_prepare_workspace_size",
             "gq_prepare_hinv", "gq_quantize_workspace_size", "gq_quantize_layer",
-            "gq_workspace_status", "gq_prepare_hinv_static")
+            "gq_workspace_status", "gq_prepare_hinv_static", "gq_prepare_hinv_ordered",
+            "gq_quantize_layer_ordered")
 
 
 def _ptr(t):
@@ -146,6 +153,32 @@ def gq_prepare_hinv(H: torch.Tensor, damp: float = 0.01, reverse: bool = False, 
     return U, dead, delta, ws
 
 
+def gq_prepare_hinv_ordered(H: torch.Tensor, damp: float = 0.01, order: str = "act", perm=None,
+                            U=None, dead=None, delta=None, ws=None, stream=None):
+    """gq_prepare_hinv in a column order ("natural", "reverse", "act", "min_pivot", "given").
+    Returns (perm int32 n, U, dead, delta, ws); for "given" pass perm, else it is written."""
+    n = H.shape[0]
+    _need(H, torch.float64, (n, n), "H")
+    if order not in ORDERS:
+        raise ValueError(f"unknown order {order!r}")
+    dev = H.device
+    if perm is None:
+        if order == "given":
+            raise ValueError("order 'given' needs perm")
+        perm = torch.empty(n, dtype=torch.int32, device=dev)
+    _need(perm, torch.int32, (n,), "perm")
+    U = torch.empty((n, n), dtype=torch.float32, device=dev) if U is None else U
+    dead = torch.empty(n, dtype=torch.uint8, device=dev) if dead is None else dead
+    delta = torch.empty(1, dtype=torch.float64, device=dev) if delta is None else delta
+    ws = workspace(gq_prepare_workspace_size(n), dev) if ws is None else ws
+    _need(U, torch.float32, (n, n), "U")
+    _check(LIB.gq_prepare_hinv_ordered(_ptr(H), n, float(damp), ORDERS[order], _ptr(perm),
+                                       _ptr(U), _ptr(dead), _ptr(delta), _ptr(ws), ws.numel(),
+                                       _stream(stream)),
+           "gq_prepare_hinv_ordered")
+    return perm, U, dead, delta, ws
+
+
 def gq_prepare_hinv_static(H: torch.Tensor, damp: float = 0.01, reverse: bool = False, U=None,
                            dead=None, delta=None, status=None, stream=None):
     """gq_prepare_hinv on the library's built-in scratch (n <= 1024; no device allocation by
@@ -207,6 +240,32 @@ def gq_quantize_layer(W: torch.Tensor, U: torch.Tensor, dead, delta, cfg: QuantC
                                  ctypes.byref(c), _ptr(codes), _ptr(scales), _ptr(zeros),
                                  _ptr(loss), _ptr(ws), ws.numel(), _stream(stream)),
            "gq_quantize_layer")
+    return codes, scales, zeros, loss, ws
+
+
+def gq_quantize_layer_ordered(W: torch.Tensor, U: torch.Tensor, dead, delta, cfg: QuantCfg,
+                              perm: torch.Tensor, codes=None, scales=None, zeros=None, loss=None,
+                              ws=None, stream=None):
+    """gq_quantize_layer with the columns in the order perm (from gq_prepare_hinv_ordered);
+    codes stay indexed by original column, groups follow the processing order."""
+    m, n = W.shape
+    if not W.is_cuda or not W.is_contiguous():
+        raise ValueError("W must be a contiguous cuda tensor")
+    dev = W.device
+    _need(U, torch.float32, (n, n), "U")
+    _need(perm, torch.int32, (n,), "perm")
+    G = 1 if cfg.group_size == 0 else -(-n // cfg.group_size)
+    codes = torch.empty((m, n_words(n, cfg.bits)), dtype=torch.int32, device=dev) if codes is None else codes
+    scales = torch.empty((m, G), dtype=torch.float32, device=dev) if scales is None else scales
+    zeros = torch.empty((m, G), dtype=torch.uint8, device=dev) if zeros is None else zeros
+    loss = torch.empty(3, dtype=torch.float64, device=dev) if loss is None else loss
+    ws = workspace(gq_quantize_workspace_size(m, n, cfg), dev) if ws is None else ws
+    c = cfg.c()
+    _check(LIB.gq_quantize_layer_ordered(_ptr(W), _dtype_code(W), m, n, _ptr(U), _ptr(dead),
+                                         _ptr(delta), ctypes.byref(c), _ptr(perm), _ptr(codes),
+                                         _ptr(scales), _ptr(zeros), _ptr(loss), _ptr(ws),
+                                         ws.numel(), _stream(stream)),
+           "gq_quantize_layer_ordered")
     return codes, scales, zeros, loss, ws
 
 

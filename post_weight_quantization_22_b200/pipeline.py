@@ -26,8 +26,14 @@ class LayerResult:
 
 class LayerQuantizer:
     def __init__(self, m: int, n: int, cfg: G.QuantCfg, device="cuda", damp: float = 0.01,
-                 max_tokens: int = 65536):
-        self.m, self.n, self.cfg, self.damp = m, n, cfg, damp
+                 max_tokens: int = 65536, order: str | None = None):
+        """``order``: None (natural, or reversed when ``cfg.reverse``), or a column order of
+        gq_prepare_hinv_ordered: "act", "min_pivot", or "given" (fill ``self.perm`` first)."""
+        if order is not None and order not in ("act", "min_pivot", "given"):
+            raise ValueError(f"unknown order {order!r}")
+        if order is not None and cfg.reverse:
+            raise ValueError("an order replaces cfg.reverse")
+        self.m, self.n, self.cfg, self.damp, self.order = m, n, cfg, damp, order
         self.max_tokens = max_tokens
         dev = torch.device(device)
         self.H = torch.zeros((n, n), dtype=torch.float64, device=dev)
@@ -42,6 +48,7 @@ class LayerQuantizer:
         self.scales = torch.empty((m, ng), dtype=torch.float32, device=dev)
         self.zeros = torch.empty((m, ng), dtype=torch.uint8, device=dev)
         self.loss = torch.empty(3, dtype=torch.float64, device=dev)
+        self.perm = torch.arange(n, dtype=torch.int32, device=dev) if order else None
 
     def hessian(self, X: torch.Tensor, reset: bool = True, stream=None):
         if X.shape[0] > self.max_tokens:
@@ -49,12 +56,21 @@ class LayerQuantizer:
         G.gq_hessian_accumulate(self.H, X, accumulate=not reset, ws=self.ws_hess, stream=stream)
 
     def prepare(self, stream=None):
-        G.gq_prepare_hinv(self.H, self.damp, self.cfg.reverse, self.U, self.dead, self.delta,
-                          self.ws_prep, stream=stream)
+        if self.order:
+            G.gq_prepare_hinv_ordered(self.H, self.damp, self.order, self.perm, self.U, self.dead,
+                                      self.delta, self.ws_prep, stream=stream)
+        else:
+            G.gq_prepare_hinv(self.H, self.damp, self.cfg.reverse, self.U, self.dead,
+                              self.delta, self.ws_prep, stream=stream)
 
     def quantize(self, W: torch.Tensor, stream=None):
-        G.gq_quantize_layer(W, self.U, self.dead, self.delta, self.cfg, self.codes, self.scales,
-                            self.zeros, self.loss, self.ws_quant, stream=stream)
+        if self.order:
+            G.gq_quantize_layer_ordered(W, self.U, self.dead, self.delta, self.cfg, self.perm,
+                                        self.codes, self.scales, self.zeros, self.loss,
+                                        self.ws_quant, stream=stream)
+        else:
+            G.gq_quantize_layer(W, self.U, self.dead, self.delta, self.cfg, self.codes,
+                                self.scales, self.zeros, self.loss, self.ws_quant, stream=stream)
 
     def run(self, W: torch.Tensor, X: torch.Tensor, stream=None) -> LayerResult:
         self.hessian(X, stream=stream)

@@ -17,13 +17,15 @@ def unpack_np(packed: np.ndarray, n: int, bits: int) -> np.ndarray:
 
 
 def run_gpu(W: torch.Tensor, X: torch.Tensor, bits: int, group: int = 0, reverse: bool = False,
-            clip: bool = True, damp: float = 0.01):
+            clip: bool = True, damp: float = 0.01, order=None, perm=None):
     from post_weight_quantization_22_b200 import gq as G
     from post_weight_quantization_22_b200.pipeline import LayerQuantizer
 
     m, n = W.shape
     cfg = G.QuantCfg(bits=bits, group_size=group, reverse=reverse, clip=clip)
-    lq = LayerQuantizer(m, n, cfg, device="cuda", damp=damp)
+    lq = LayerQuantizer(m, n, cfg, device="cuda", damp=damp, order=order)
+    if perm is not None:
+        lq.perm.copy_(torch.as_tensor(np.asarray(perm), dtype=torch.int32))
     res = lq.run(W.cuda().contiguous(), X.cuda().contiguous())
     torch.cuda.synchronize()
     sp, sq, rounds = lq.status()
@@ -32,7 +34,8 @@ def run_gpu(W: torch.Tensor, X: torch.Tensor, bits: int, group: int = 0, reverse
                 codes=unpack_np(packed, n, bits), scales=res.scales.cpu().numpy(),
                 zeros=res.zeros.cpu().numpy().astype(np.int64), loss=res.loss.cpu().numpy(),
                 dead=res.dead.cpu().numpy().astype(bool), delta=float(res.delta.item()),
-                status=(sp, sq), rounds=rounds)
+                status=(sp, sq), rounds=rounds,
+                perm=None if lq.perm is None else lq.perm.cpu().numpy().astype(np.int64))
 
 
 def rel_fro(a, b) -> float:

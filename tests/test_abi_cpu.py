@@ -52,3 +52,24 @@ def test_package_has_no_cpu_fallback():
                 src = open(os.path.join(dirpath, f)).read()
                 assert not re.search(r"^\s*(from|import)\s+oracle", src, flags=re.M), f
                 assert "gptq_oracle" not in src, f
+
+
+def test_ordered_entry_points_reject_bad_arguments_without_gpu():
+    """Argument checks of the ordered calls return before any device work."""
+    from post_weight_quantization_22_b200 import gq as G
+    L = G.LIB
+    fake = ctypes.c_void_p(4096)
+    # unknown order value
+    assert L.gq_prepare_hinv_ordered(fake, 16, 0.01, 9, fake, fake, fake, fake, fake, 1 << 20,
+                                     None) == 1
+    # ACT without a perm array
+    assert L.gq_prepare_hinv_ordered(fake, 16, 0.01, 2, None, fake, fake, fake, fake, 1 << 20,
+                                     None) == 1
+    cfg = G.QuantCfg(bits=4)
+    c = cfg.c()
+    # no perm, and reverse together with a perm
+    assert L.gq_quantize_layer_ordered(fake, 0, 4, 16, fake, None, None, ctypes.byref(c), None,
+                                       fake, fake, fake, fake, fake, 1 << 20, None) == 1
+    c2 = G.QuantCfg(bits=4, reverse=True).c()
+    assert L.gq_quantize_layer_ordered(fake, 0, 4, 16, fake, None, None, ctypes.byref(c2), fake,
+                                       fake, fake, fake, fake, fake, 1 << 20, None) == 1

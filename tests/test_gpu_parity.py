@@ -23,11 +23,12 @@ H_REL_DESIGN = 1e-9   # digit rounding of entries below 2^-21 of their column's 
 U_REL_DESIGN = 1e-6
 
 
-def _oracle(W, X, bits, group, reverse, clip, rows=None):
-    return O.quantize_layer(W, X, bits=bits, group=group, reverse=reverse, clip=clip, rows=rows)
+def _oracle(W, X, bits, group, reverse, clip, rows=None, order=None):
+    return O.quantize_layer(W, X, bits=bits, group=group, reverse=reverse, clip=clip, rows=rows,
+                            order=order)
 
 
-def _compare(g, o, W, bits, group, rows=None, check_loss=True):
+def _compare(g, o, W, bits, group, rows=None, check_loss=True, perm=None):
     W = W.double().numpy() if hasattr(W, "double") else W
     n = W.shape[1]
     Hrel = rel_fro(g["H"], o["H"])
@@ -49,8 +50,9 @@ def _compare(g, o, W, bits, group, rows=None, check_loss=True):
         # permitted code difference changes every later group of its row).
         ng = gs.shape[1]
         same_before = np.ones((gc.shape[0], ng), dtype=bool)
-        for k in range(1, ng):
-            same_before[:, k] = np.all(gc[:, : k * group] == o["codes"][:, : k * group], axis=1)
+        pc, po = (gc, o["codes"]) if perm is None else (gc[:, perm], o["codes"][:, perm])
+        for k in range(1, ng):  # "earlier" = earlier in the processing order
+            same_before[:, k] = np.all(pc[:, : k * group] == po[:, : k * group], axis=1)
         np.testing.assert_allclose(gs[same_before], o["scales"][same_before], rtol=1e-4)
     else:
         np.testing.assert_allclose(gs, o["scales"], rtol=1e-6)
@@ -172,6 +174,81 @@ def test_argument_errors_enqueue_nothing():
     with pytest.raises(G.GQError) as e:
         G.gq_quantize_layer(W, U, None, None, G.QuantCfg(bits=4), ws=G.workspace(256, "cuda"))
     assert e.value.code == 7
+
+
+def _check_act_perm(g_perm, o):
+    """The device's act-order against the oracle's: identical, except that columns whose fixed
+    diagonals agree to the Hessian's accuracy may be exchanged (a near-tie that the fp64 sums
+    of the two sides may order differently)."""
+    d = np.diag(o["H"]).copy()
+    d[d == 0.0] = 1.0
+    ref = O.act_order(np.diag(d))
+    assert sorted(g_perm.tolist()) == list(range(len(d)))
+    assert np.all(np.diff(d[g_perm]) <= H_REL_DESIGN * np.abs(d[g_perm][1:]))
+    diff = np.nonzero(g_perm != ref)[0]
+    for k in diff:
+        assert abs(d[g_perm[k]] - d[ref[k]]) <= H_REL_DESIGN * abs(d[ref[k]])
+    return len(diff)
+
+
+def test_act_order_ragged_group128():
+    """act-order (descending diag H) on the q_proj recipe at a ragged size, 4-bit g128: the
+    device's order against the oracle's; then codes / grids (per processing-order group) / U /
+    losses against the oracle run in the device's order."""
+    W, X, spec = synth.workload("q_proj_4096x4096", m=320, n=1000, T=1200)
+    g = run_gpu(W, X, bits=4, group=128, order="act")
+    assert g["status"] == (0, 0)
+    o = _oracle(W, X, 4, 128, False, True, order=g["perm"])
+    assert _check_act_perm(g["perm"], o) == 0
+    _compare(g, o, W, 4, 128, perm=g["perm"])
+
+
+def test_act_order_tiny_fp32_per_row_and_dead_columns():
+    W, X, spec = synth.workload("tiny_256x512")
+    X = X.clone()
+    X[:, [5, 300]] = 0  # two dead columns: fixed diagonal 1, weights zeroed
+    g = run_gpu(W, X, bits=4, order="act")
+    assert g["status"] == (0, 0)
+    o = _oracle(W, X, 4, 0, False, True, order=g["perm"])
+    _check_act_perm(g["perm"], o)
+    assert g["dead"].sum() == 2
+    _compare(g, o, W, 4, 0, perm=g["perm"])
+
+
+def test_given_order_clipfree_ladder():
+    """A caller's random order, clip-free 3-bit per-row ladder."""
+    W, X, spec = synth.workload("clipfree_babai_4096x4096", m=160, n=520, T=700)
+    perm = np.random.default_rng(11).permutation(520)
+    g = run_gpu(W, X, bits=3, clip=False, order="given", perm=perm)
+    assert g["status"] == (0, 0)
+    assert np.array_equal(g["perm"], perm)
+    o = _oracle(W, X, 3, 0, False, False, order=perm)
+    assert g["rounds"] == o["ladder_rounds"]
+    _compare(g, o, W, 3, 0, perm=perm)
+    assert g["loss"][1] <= g["loss"][2]
+
+
+def test_given_order_that_is_not_a_permutation_is_reported():
+    """A repeated entry and an out-of-range entry: both calls record GQ_ERR_INVALID_ARG (every
+    access is clamped in bounds; duplicated columns keep the damped matrix definite)."""
+    from post_weight_quantization_22_b200 import gq as G
+    W, X, spec = synth.workload("q_proj_4096x4096", m=64, n=200, T=300)
+    H = torch.zeros((200, 200), dtype=torch.float64, device="cuda")
+    G.gq_hessian_accumulate(H, X.cuda())
+    for bad_entry in (3, 200 + 7):
+        perm = torch.arange(200, dtype=torch.int32, device="cuda")
+        perm[10] = bad_entry
+        _, U, dead, delta, ws = G.gq_prepare_hinv_ordered(H, 0.01, "given", perm)
+        assert G.gq_workspace_status(ws)[0] == 1
+        U0, dead0, delta0, ws0 = G.gq_prepare_hinv(H, 0.01)
+        assert G.gq_workspace_status(ws0)[0] == 0
+        *_, wsq = G.gq_quantize_layer_ordered(W.cuda(), U0, dead0, delta0,
+                                               G.QuantCfg(bits=4), perm)
+        assert G.gq_workspace_status(wsq)[0] == 1
+    with pytest.raises(G.GQError) as e:
+        G.gq_quantize_layer_ordered(W.cuda(), U0, dead0, delta0,
+                                    G.QuantCfg(bits=4, reverse=True), perm)
+    assert e.value.code == 1
 
 
 @pytest.mark.slow
