@@ -210,7 +210,7 @@ def run_gq(args):
                      clip=bool(spec["clip"]))
     Wd, Xd = W.to(device), X.to(device)
     Wh, Xh = W.pin_memory(), X.pin_memory()
-    lq = LayerQuantizer(m, n, cfg, device=device)
+    lq = LayerQuantizer(m, n, cfg, device=device, order=args.order)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
     stream = torch.cuda.current_stream(device)
 
@@ -315,6 +315,7 @@ def run_gq(args):
                 "N(0,0.02^2) weights with Student-t outlier rows)",
         "config": {"workload": args.workload, "m": m, "n": n, "tokens": T, "bits": spec["bits"],
                    "group": spec["group"], "reverse": spec["reverse"], "clip": spec["clip"],
+                   **({"order": args.order} if args.order else {}),
                    "l2": "flushed between steps (256 MiB write, untimed)",
                    "parallelism": f"{ws} independent layers (one per GPU)"},
         "stages": stages,
@@ -403,6 +404,8 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["gq", "reference"], default="gq")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--order", choices=["act"], default=None,
+                    help="process the columns in act-order (descending Hessian diagonal)")
     ap.add_argument("--cpu-rows", type=int, default=256)
     ap.add_argument("--ref-rows", type=int, default=32)
     ap.add_argument("--case", choices=["layer", "factor"], default=None,

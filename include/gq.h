@@ -61,7 +61,8 @@ typedef enum {
   GQ_ORDER_REVERSE = 1,   /* columns n-1, ..., 0 (Babai order) */
   GQ_ORDER_ACT = 2,       /* descending diagonal of H after the dead fix; ties by column index */
   GQ_ORDER_MIN_PIVOT = 3, /* greedy min-pivot: the reverse of the elimination order of a
-                             pivoted LDL of H_d that always eliminates the smallest pivot */
+                             pivoted LDL of H_d that always eliminates the smallest pivot.
+                             Reserved: gq_prepare_hinv_ordered returns GQ_ERR_UNSUPPORTED */
   GQ_ORDER_GIVEN = 4      /* the caller's permutation */
 } gq_order;
 
@@ -170,8 +171,9 @@ gq_status gq_prepare_hinv_static(const double* d_H, int64_t n, double damp, int 
  *
  *   order    a gq_order.  NATURAL and REVERSE give exactly gq_prepare_hinv's U with
  *            reverse = 0 / 1 (d_perm is then not touched and may be NULL).
- *   d_perm   n int32, device.  ACT and MIN_PIVOT write the order computed on the device from
- *            H; GIVEN reads it.  Pass the same array to gq_quantize_layer_ordered.
+ *   d_perm   n int32, device.  ACT writes the order computed on the device from H; GIVEN
+ *            reads it.  Pass the same array to gq_quantize_layer_ordered.  MIN_PIVOT is
+ *            rejected with GQ_ERR_UNSUPPORTED (no device implementation).
  * Device-detected errors: GQ_ERR_INVALID_ARG (GIVEN: d_perm is not a permutation of 0..n-1;
  * every access stays in bounds and U is then undefined), GQ_ERR_NOT_PD.
  */

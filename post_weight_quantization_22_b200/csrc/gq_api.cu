@@ -190,7 +190,7 @@ gq_status gq_prepare_hinv_ordered(const double* d_H, int64_t n, double damp, gq_
     return gq_prepare_hinv(d_H, n, damp, o, d_U, d_dead, d_delta, d_ws, ws_bytes, stream);
   if (n < 1 || n > kMaxN || !(damp >= 0.0)) return GQ_ERR_INVALID_ARG;
   if (!d_H || !d_U || !d_dead || !d_delta || !d_ws || !d_perm) return GQ_ERR_INVALID_ARG;
-  if (o == GQ_ORDER_MIN_PIVOT) return GQ_ERR_UNSUPPORTED;
+  if (o == GQ_ORDER_MIN_PIVOT) return GQ_ERR_UNSUPPORTED;  // no device implementation yet
   if (!aligned256(d_ws) || ws_bytes < prepare_ws_bytes(n)) return GQ_ERR_WORKSPACE;
   gq_status st = ensure_device_setup();
   if (st != GQ_OK) return st;

@@ -49,8 +49,8 @@ cudaError_t launch_hessian(double* H, const void* X, gq_dtype xt, int64_t T, int
 
 // ---- factor preparation ----
 size_t prepare_ws_bytes(int64_t n);
-// order: a gq_order value; perm (n ints) is written for ACT / MIN_PIVOT, read for GIVEN and
-// not used for NATURAL / REVERSE (may be null there).
+// order: a gq_order value other than MIN_PIVOT; perm (n ints) is written for ACT, read for
+// GIVEN and not used for NATURAL / REVERSE (may be null there).
 cudaError_t launch_prepare(const double* H, int64_t n, double damp, int order, int* perm,
                            float* U, uint8_t* dead, double* delta, void* ws, cudaStream_t s);
 

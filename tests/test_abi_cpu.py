@@ -62,6 +62,9 @@ def test_ordered_entry_points_reject_bad_arguments_without_gpu():
     # unknown order value
     assert L.gq_prepare_hinv_ordered(fake, 16, 0.01, 9, fake, fake, fake, fake, fake, 1 << 20,
                                      None) == 1
+    # the min-pivot order has no device implementation: rejected before any device work
+    assert L.gq_prepare_hinv_ordered(fake, 16, 0.01, 3, fake, fake, fake, fake, fake, 1 << 20,
+                                     None) == 4
     # ACT without a perm array
     assert L.gq_prepare_hinv_ordered(fake, 16, 0.01, 2, None, fake, fake, fake, fake, 1 << 20,
                                      None) == 1
