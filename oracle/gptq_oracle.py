@@ -47,6 +47,7 @@ __all__ = [
     "clipfree_grid",
     "gptq_columns",
     "babai_sic_reverse",
+    "zsic_spacing",
     "pack_codes",
     "proxy_loss",
     "quadratic_loss",
@@ -199,11 +200,25 @@ def clipfree_grid(w, bits: int, alpha):
     return s, z
 
 
+def zsic_spacing(pivots) -> np.ndarray:
+    """Per-column grid spacing of ZSIC ([WSIC] 2: alpha_i proportional to 1 / |l_ii|).
+
+    ``pivots`` are the LDL pivots D_jj = l_jj^2 of the Hessian in the processing order.
+    reading: the factors are normalised to geometric mean 1, kappa_j = g / |l_jj| with g the
+    geometric mean of |l_jj|, so that a row's steps s kappa_j have the same geometric mean (the
+    same log-volume of the lattice cell, i.e. the same entropy-coded rate) as the uniform step s.
+    """
+    l = np.sqrt(_f64(pivots))
+    g = float(np.exp(np.mean(np.log(l))))
+    return g / l
+
+
 # ---------------------------------------------------------------------------------------------
 # Column loops
 # ---------------------------------------------------------------------------------------------
 
-def gptq_columns(W, U, bits: int, group: int = 0, clip: bool = True, alpha=None, grid=None):
+def gptq_columns(W, U, bits: int, group: int = 0, clip: bool = True, alpha=None, grid=None,
+                 col_scale=None):
     """GPTQ error-feedback loop, columns 0..n-1 in order ([GEOM] 2.2).
 
     For each column j: quantize the current column on the row's grid, error
@@ -214,7 +229,8 @@ def gptq_columns(W, U, bits: int, group: int = 0, clip: bool = True, alpha=None,
     recomputed at the group's first column from the current, error-fed weights of the group.
     clip=False: codes are unconstrained integers (no clamp) on the ``clipfree_grid`` with the
     per-row factor ``alpha`` (group must be 0).  ``grid`` = (s, z) fixes the per-row grid
-    instead (a fixed lattice).
+    instead (a fixed lattice).  ``col_scale`` (per-row grids only) multiplies the step of
+    column j by col_scale[j]: the grid of column j is s col_scale[j] (c - z).
 
     Returns dict(codes, scales, zeros, Q, e) in processing order; e is the m x n matrix of
     scaled errors, whose squares sum to tr(D H_d D^T).
@@ -225,6 +241,9 @@ def gptq_columns(W, U, bits: int, group: int = 0, clip: bool = True, alpha=None,
     maxq = 2 ** bits - 1
     if not clip and group:
         raise ValueError("the clip-free variant uses a per-row grid")
+    if col_scale is not None and group:
+        raise ValueError("per-column spacing uses a per-row grid")
+    kap = np.ones(n) if col_scale is None else _f64(col_scale)
     ngroups = 1 if group == 0 else -(-n // group)
     scales = np.zeros((m, ngroups))
     zeros = np.zeros((m, ngroups))
@@ -243,10 +262,11 @@ def gptq_columns(W, U, bits: int, group: int = 0, clip: bool = True, alpha=None,
         if group and j % group == 0:
             s, z = minmax_grid(w[:, j:j + group], bits)
             scales[:, j // group], zeros[:, j // group] = s, z
-        c = np.rint(w[:, j] / s) + z
+        sj = s * kap[j]
+        c = np.rint(w[:, j] / sj) + z
         if clip:
             c = np.clip(c, 0, maxq)
-        q = s * (c - z)
+        q = sj * (c - z)
         e = (w[:, j] - q) / u[j, j]
         w[:, j + 1:] -= np.outer(e, u[j, j + 1:])
         codes[:, j] = c.astype(np.int64)
@@ -339,7 +359,7 @@ def babai_bound(scales_per_col, pivots) -> float:
 
 def quantize_layer(W, X, bits: int, group: int = 0, reverse: bool = False, clip: bool = True,
                    damp: float = 0.01, ladder: float = 1.25, ladder_max: int = 8,
-                   rows=None, H=None, order=None):
+                   rows=None, H=None, order=None, spacing: str = "uniform"):
     """Quantize one linear layer: H, dead fix, damping, factor, column loop, losses.
 
     ``W`` is m x n (output rows x input features), ``X`` is T x n.  ``rows`` restricts the
@@ -352,6 +372,9 @@ def quantize_layer(W, X, bits: int, group: int = 0, reverse: bool = False, clip:
     k-th) runs the GPTQ form on the columns in that order, with U the factor of the permuted
     H_d; group grids then cover consecutive columns of the processing order (reading: the pages
     do not combine groups with an order), so scales / zeros are indexed by processing group.
+
+    spacing="zsic" (per-row grids, forward or an explicit order): column j's step is the row
+    step times ``zsic_spacing`` of the processing order's pivots.
 
     clip=False (reading of "per-row step set so that no entry needs clipping"): run unclamped;
     a row whose codes leave [0, 2^b - 1] is rerun with alpha multiplied by ``ladder``, at most
@@ -383,12 +406,20 @@ def quantize_layer(W, X, bits: int, group: int = 0, reverse: bool = False, clip:
             if sorted(perm.tolist()) != list(range(n)):
                 raise ValueError("order is not a permutation of the columns")
 
+    if spacing not in ("uniform", "zsic"):
+        raise ValueError(f"unknown spacing {spacing!r}")
+    if spacing == "zsic" and (reverse or group):
+        raise ValueError("ZSIC spacing here takes a per-row grid and the forward / ordered form")
+    kap = None
     if perm is not None:
         U = hinv_upper_factor(hd[np.ix_(perm, perm)])
         pivots = 1.0 / np.diag(U) ** 2  # in processing order
+        if spacing == "zsic":
+            kap = zsic_spacing(pivots)
 
         def run(rows_w, alpha):
-            r = gptq_columns(rows_w[:, perm], U, bits, group=group, clip=clip, alpha=alpha)
+            r = gptq_columns(rows_w[:, perm], U, bits, group=group, clip=clip, alpha=alpha,
+                             col_scale=kap)
             for key in ("codes", "Q"):
                 back = np.empty_like(r[key])
                 back[:, perm] = r[key]
@@ -403,9 +434,12 @@ def quantize_layer(W, X, bits: int, group: int = 0, reverse: bool = False, clip:
     else:
         U = hinv_upper_factor(hd)
         pivots = 1.0 / np.diag(U) ** 2
+        if spacing == "zsic":
+            kap = zsic_spacing(pivots)
 
         def run(rows_w, alpha):
-            return gptq_columns(rows_w, U, bits, group=group, clip=clip, alpha=alpha)
+            return gptq_columns(rows_w, U, bits, group=group, clip=clip, alpha=alpha,
+                                col_scale=kap)
 
     alpha = np.ones(len(sel))
     res = run(w_sel, alpha)
@@ -427,8 +461,11 @@ def quantize_layer(W, X, bits: int, group: int = 0, reverse: bool = False, clip:
     Q = res["Q"]
     g = group if group else n
     s_cols = np.repeat(res["scales"], g, axis=1)[:, :n]  # processing order
+    if kap is not None:
+        s_cols = s_cols * kap[None, :]
     out = dict(H=H, dead=dead, delta=delta, Hd=hd, codes=res["codes"], scales=res["scales"],
-               zeros=res["zeros"], Q=Q, alpha=alpha, ladder_rounds=retries, perm=perm)
+               zeros=res["zeros"], Q=Q, alpha=alpha, ladder_rounds=retries, perm=perm,
+               col_scale=kap)
     if reverse:
         out["L"] = L
     else:

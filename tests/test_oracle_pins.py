@@ -504,3 +504,62 @@ def test_identity_and_reversal_orders_match_the_flags():
     rev = O.quantize_layer(w, x, 3, reverse=True)
     prm = O.quantize_layer(w, x, 3, order=np.arange(16)[::-1])
     assert np.array_equal(rev["codes"], prm["codes"])
+
+
+# --------------------------------------------------------------------------------------------
+# ZSIC per-column spacing (WaterSIC section 2: alpha_i proportional to 1 / |l_ii|)
+# --------------------------------------------------------------------------------------------
+
+def test_zsic_spacing_hand_values():
+    """pivots (1, 4, 16): |l| = (1, 2, 4), geometric mean 2, so kappa = (2, 1, 1/2)."""
+    np.testing.assert_allclose(O.zsic_spacing([1.0, 4.0, 16.0]), [2.0, 1.0, 0.5], rtol=1e-15)
+
+
+def test_zsic_on_diagonal_hessian_is_rtn_with_column_steps():
+    """Diagonal H: no feedback; column j is rounded on the step s sqrt(g2 / H_d,jj) with g2 the
+    geometric mean of the damped diagonal (closed form of alpha_j proportional to 1/|l_jj|)."""
+    rng = np.random.default_rng(111)
+    n, m = 10, 7
+    d = rng.uniform(0.5, 4.0, n)
+    w = 0.02 * rng.standard_normal((m, n))
+    res = O.quantize_layer(w, None, 4, H=np.diag(d), spacing="zsic")
+    dd = d + 0.01 * d.mean()
+    kap = np.sqrt(np.exp(np.mean(np.log(dd))) / dd)
+    s, z = res["scales"][:, 0], res["zeros"][:, 0]
+    code = np.clip(np.rint(w / (s[:, None] * kap[None, :])) + z[:, None], 0, 15)
+    np.testing.assert_array_equal(res["codes"], code)
+
+
+@pytest.mark.parametrize("seed", range(3))
+def test_zsic_is_babai_on_column_scaled_basis(seed):
+    """Clip-free ZSIC = textbook Babai on the tall basis [sqrt2 X; sqrt(delta) I] diag(s kappa)
+    with the basis order reversed."""
+    n, T, m = 10, 40, 30
+    w, x = _rand_problem(T, n, m, seed=113 + seed)
+    res = O.quantize_layer(w, x, 3, clip=False, spacing="zsic")
+    F = np.vstack([np.sqrt(2.0) * x, np.sqrt(res["delta"]) * np.eye(n)])
+    kap = res["col_scale"]
+    for r in range(m):
+        s = res["scales"][r, 0]
+        u = _babai_gram_schmidt((F * (s * kap))[:, ::-1], F @ w[r])[::-1]
+        assert np.array_equal(res["codes"][r] - int(res["zeros"][r, 0]), u.astype(np.int64))
+
+
+def test_zsic_bound_and_am_gm_against_uniform():
+    """Theorem 5 with per-column steps: the clip-free damped loss of each row is at most
+    (1/4) sum_j (s kappa_j)^2 D_jj = (n/4) s^2 g^2; and at the same row step this is at most the
+    uniform grid's (1/4) s^2 sum_j D_jj (arithmetic vs geometric mean of the pivots)."""
+    w, x = _rand_problem(200, 32, 40, seed=117)
+    hd, _ = O.dampen(O.hessian(x), 0.01)
+    U = O.hinv_upper_factor(hd)
+    D = 1.0 / np.diag(U) ** 2
+    kap = O.zsic_spacing(D)
+    s, z = O.clipfree_grid(w, 3, np.ones(40))
+    zs = O.gptq_columns(w, U, 3, clip=False, grid=(s, z), col_scale=kap)
+    g2 = np.exp(np.mean(np.log(D)))
+    for r in range(40):
+        d = w[r] - zs["Q"][r]
+        b_z = 0.25 * s[r] ** 2 * np.sum(kap ** 2 * D)
+        np.testing.assert_allclose(b_z, 0.25 * 32 * s[r] ** 2 * g2, rtol=1e-12)
+        assert d @ hd @ d <= b_z * (1 + 1e-12)
+        assert b_z <= 0.25 * s[r] ** 2 * D.sum()
