@@ -74,6 +74,10 @@ typedef struct {
   int clip;       /* 1: codes clamped to [0, 2^b-1] (GPTQ); 0: clip-free with a scale ladder */
   float ladder;   /* clip-free: factor applied to a row's step when its codes overflow (1.25) */
   int ladder_max; /* clip-free: at most this many widenings per row (8) */
+  int spacing;    /* 0: one step per row or group; 1: ZSIC ("WaterSIC", section 2: grid spacing
+                     proportional to 1/|l_jj|): column j's step is the row step times
+                     kappa_j = U_jj / geomean(U_kk), U in the processing order.  Needs
+                     group_size 0 and reverse 0 (use an order for last-to-first). */
 } gq_quant_cfg;
 
 /* Library version string, e.g. "gq 0.1 sm_100a". */
@@ -209,7 +213,9 @@ size_t gq_quantize_workspace_size(int64_t m, int64_t n, const gq_quant_cfg* cfg)
  *             (W0 = W with dead columns zeroed), [1] tr(D H_d D^T) = sum of e^2,
  *             [2] Theorem 5 bound sum_r sum_j s_rj^2 / (4 U_jj^2) (a guarantee for clip = 0).
  *   d_ws      workspace of at least gq_quantize_workspace_size(m, n, cfg) bytes.
- * Limits: 1 <= m <= 2^24, 1 <= n <= 32768, 2 <= bits <= 8; reverse = 1 needs group_size 0.
+ * Limits: 1 <= m <= 2^24, 1 <= n <= 32768, 2 <= bits <= 8; reverse = 1 needs group_size 0;
+ * spacing = 1 needs group_size 0 and reverse 0.  With spacing = 1 the Theorem 5 bound and the
+ * losses use the per-column steps.
  * Device-detected error: GQ_ERR_NO_FIT.
  */
 gq_status gq_quantize_layer(const void* d_W, gq_dtype w_dtype, int64_t m, int64_t n,
@@ -235,6 +241,15 @@ gq_status gq_quantize_layer_ordered(const void* d_W, gq_dtype w_dtype, int64_t m
                                     const int32_t* d_perm, uint32_t* d_codes, float* d_scales,
                                     uint8_t* d_zeros, double* d_loss, void* d_ws,
                                     size_t ws_bytes, gq_stream_t stream);
+
+/*
+ * The ZSIC column factors kappa_j = U_jj / geomean(U_kk) ("WaterSIC", section 2) of a factor
+ * from gq_prepare_hinv(_ordered), exactly as gq_quantize_layer uses them with spacing = 1; a
+ * dequantizer takes column j's step as (row step) x kappa_j, j in the processing order.
+ *
+ *   d_U      n x n fp32, device.   d_kappa  n fp64, device, written.   1 <= n <= 32768.
+ */
+gq_status gq_zsic_spacing(const float* d_U, int64_t n, double* d_kappa, gq_stream_t stream);
 
 /*
  * Synchronize `stream` and return the device-side status recorded in a workspace by the last

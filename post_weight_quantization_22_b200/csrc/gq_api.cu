@@ -213,6 +213,8 @@ static gq_status check_cfg(const gq_quant_cfg* cfg) {
     return (g > 0 && g <= 128 && kBlock % g == 0) ? GQ_ERR_UNSUPPORTED : GQ_ERR_INVALID_ARG;
   }
   if (g != 0 && (cfg->reverse || !cfg->clip)) return GQ_ERR_UNSUPPORTED;
+  if (cfg->spacing != 0 && cfg->spacing != 1) return GQ_ERR_INVALID_ARG;
+  if (cfg->spacing && (g != 0 || cfg->reverse)) return GQ_ERR_UNSUPPORTED;
   if (!cfg->clip) {
     if (!(cfg->ladder > 1.f) || cfg->ladder_max < 0 || cfg->ladder_max > 64)
       return GQ_ERR_INVALID_ARG;
@@ -249,7 +251,8 @@ static gq_status quantize_common(const void* d_W, gq_dtype w_dtype, int64_t m, i
   auto enqueue = [&](cudaStream_t s) { return run_quantize(a, s); };
   return run_graphed({2, P(d_W), (uint64_t)w_dtype, (uint64_t)m, (uint64_t)n, P(d_U), P(d_dead),
                       P(d_delta), (uint64_t)cfg->bits, (uint64_t)cfg->group_size,
-                      (uint64_t)cfg->reverse, (uint64_t)cfg->clip, P(d_perm), P(d_codes),
+                      (uint64_t)cfg->reverse, (uint64_t)cfg->clip, (uint64_t)cfg->spacing,
+                      P(d_perm), P(d_codes),
                       P(d_scales), P(d_zeros), P(d_loss), P(d_ws)},
                      (cudaStream_t)stream, enqueue);
 }
@@ -272,6 +275,14 @@ gq_status gq_quantize_layer_ordered(const void* d_W, gq_dtype w_dtype, int64_t m
   if (!d_perm || !cfg || cfg->reverse) return GQ_ERR_INVALID_ARG;
   return quantize_common(d_W, w_dtype, m, n, d_U, d_dead, d_delta, cfg, d_perm, d_codes,
                          d_scales, d_zeros, d_loss, d_ws, ws_bytes, stream);
+}
+
+gq_status gq_zsic_spacing(const float* d_U, int64_t n, double* d_kappa, gq_stream_t stream) {
+  if (n < 1 || n > kMaxN || !d_U || !d_kappa) return GQ_ERR_INVALID_ARG;
+  gq_status st = ensure_device_setup();
+  if (st != GQ_OK) return st;
+  return launch_zsic_spacing(d_U, n, d_kappa, (cudaStream_t)stream) == cudaSuccess ? GQ_OK
+                                                                                   : GQ_ERR_CUDA;
 }
 
 gq_status gq_workspace_status(void* d_ws, int* h_ladder_rounds, gq_stream_t stream) {

@@ -78,6 +78,7 @@ struct QuantArgs {
   const int* perm;  // processing order (null: natural, or reversed when cfg.reverse)
 };
 size_t quantize_ws_bytes(int64_t m, int64_t n, const gq_quant_cfg& cfg);
+cudaError_t launch_zsic_spacing(const float* U, int64_t n, double* kappa, cudaStream_t s);
 // Returns GQ_OK or an error; the clip-free ladder synchronizes the stream per round.
 gq_status run_quantize(const QuantArgs& a, cudaStream_t s);
 

@@ -25,11 +25,14 @@ constexpr int kRowsPerCta = 8 * kColWarps;      // 32 rows per CTA
 constexpr int kTiles = kBlock / 8;              // 8-column tiles of a block
 constexpr int kUtPitch = 136;                   // floats per row of the transposed U block
 // Per-block prepared U for the column loop (see ublk_kernel): the transposed block in fp32
-// (128 rows of kUtPitch floats), then 1/U_jj and 1/U_jj^2 in fp64.
+// (128 rows of kUtPitch floats), then 1/U_jj and kappa_j^2 / U_jj^2 in fp64, then the ZSIC
+// column factors kappa_j and 1/kappa_j (all 1 for one step per row).  The column loop copies the
+// first kUBlkBytes, or all kUBlkBytesZ bytes when the columns have their own spacing.
 constexpr uint32_t kUtBytes = (uint32_t)(kBlock * kUtPitch * sizeof(float));
 constexpr uint32_t kUBlkBytes = kUtBytes + 2 * kBlock * (uint32_t)sizeof(double);
-constexpr int64_t kUBlkDoubles = kUBlkBytes / sizeof(double);
-static_assert(kUBlkBytes % 16 == 0, "bulk copies move multiples of 16 bytes");
+constexpr uint32_t kUBlkBytesZ = kUtBytes + 4 * kBlock * (uint32_t)sizeof(double);
+constexpr int64_t kUBlkDoubles = kUBlkBytesZ / sizeof(double);  // stride between blocks
+static_assert(kUBlkBytes % 16 == 0 && kUBlkBytesZ % 16 == 0, "bulk copies move multiples of 16 bytes");
 constexpr uint32_t kBulkChunk = 32768;
 
 struct QLayout {
@@ -53,6 +56,7 @@ struct QLayout {
   int* rowlist;     // compact row -> original row
   int* counter;
   int* iperm;       // n: processing position of each original column (ordered calls)
+  double* kappa;    // n: ZSIC column factors in processing order
   size_t bytes;
 };
 
@@ -81,6 +85,7 @@ static QLayout q_layout(void* ws, int64_t m, int64_t n) {
   L.rowlist = c.take<int>(m);
   L.counter = c.take<int>(4);
   L.iperm = c.take<int>((size_t)n);
+  L.kappa = c.take<double>((size_t)n);
   L.bytes = c.off;
   return L;
 }
@@ -217,7 +222,27 @@ __global__ void split_u_kernel(const float* U, int64_t n, int64_t ldu, float* Uh
 // Ut[c][k] = U[j0 + k][j0 + c] for k <= c < width (0 elsewhere), in fp32 (U is fp32, so this
 // is exact) with row pitch kUtPitch, then 1/U_jj and 1/U_jj^2 in fp64 (1 past the width).  The
 // column loop copies it into shared memory in one go.
-__global__ void ublk_kernel(const float* U, int64_t n, double* Ublk) {
+// ZSIC ("WaterSIC", section 2: grid spacing proportional to 1/|l_jj|): in the processing order
+// the LDL pivot of column j is 1/U_jj^2, so |l_jj| = 1/U_jj and kappa_j = U_jj / geomean(U_kk)
+// (normalised to geometric mean 1: the row's steps keep the geometric mean of its step).  One CTA.
+__global__ void __launch_bounds__(1024) q_zsic_kernel(const float* U, int64_t n, double* kappa) {
+  __shared__ double red[32];
+  double acc = 0.0;
+  for (int64_t j = threadIdx.x; j < n; j += blockDim.x) acc += log((double)U[j * n + j]);
+  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = acc;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    acc = threadIdx.x < (blockDim.x >> 5) ? red[threadIdx.x] : 0.0;
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    if (threadIdx.x == 0) red[0] = exp(-acc / (double)n);  // 1 / geometric mean
+  }
+  __syncthreads();
+  const double inv_gm = red[0];
+  for (int64_t j = threadIdx.x; j < n; j += blockDim.x) kappa[j] = (double)U[j * n + j] * inv_gm;
+}
+
+__global__ void ublk_kernel(const float* U, int64_t n, double* Ublk, const double* kappa) {
   const int64_t b = blockIdx.y;
   const int64_t j0 = b * kBlock;
   const int bw = (int)((n - j0) < kBlock ? (n - j0) : kBlock);
@@ -231,8 +256,11 @@ __global__ void ublk_kernel(const float* U, int64_t n, double* Ublk) {
     } else {
       const int jj = e - kBlock * kUtPitch;
       const double d = jj < bw ? (double)U[(j0 + jj) * n + j0 + jj] : 1.0;
+      const double k = (kappa && jj < bw) ? kappa[j0 + jj] : 1.0;
       dinv[jj] = 1.0 / d;
-      dinv[kBlock + jj] = 1.0 / (d * d);
+      dinv[kBlock + jj] = kappa ? (k * k) / (d * d) : 1.0 / (d * d);
+      dinv[2 * kBlock + jj] = k;
+      dinv[3 * kBlock + jj] = 1.0 / k;
     }
   }
 }
@@ -284,13 +312,18 @@ struct ColArgs {
 // coarse, and an fp32 recursion flips ~1-3 % of the codes on ill-conditioned layers (measured
 // against the fp64 oracle), while fp64 here with fp32 storage of W, E and U between blocks
 // reproduces the oracle's codes.
-template <int G>
+// Z: ZSIC spacing (per-row grid only): column j's step is the row step times kappa_j.
+template <int G, bool Z = false>
 __global__ void __launch_bounds__(kColThreads, 1) colloop_kernel(ColArgs a) {
+  static_assert(!Z || G == 0, "per-column spacing takes a per-row grid");
+  constexpr uint32_t kCopy = Z ? kUBlkBytesZ : kUBlkBytes;
   extern __shared__ __align__(16) double q_smem[];
   const float* Ut = reinterpret_cast<const float*>(q_smem);
   const double* invd = reinterpret_cast<const double*>(reinterpret_cast<const char*>(q_smem) + kUtBytes);
-  const double* invd2 = invd + kBlock;
-  uint64_t* bar = reinterpret_cast<uint64_t*>(reinterpret_cast<char*>(q_smem) + kUBlkBytes);
+  const double* invd2 = invd + kBlock;  // kappa_j^2 / U_jj^2
+  const double* kap = invd + 2 * kBlock;
+  const double* kinv = invd + 3 * kBlock;
+  uint64_t* bar = reinterpret_cast<uint64_t*>(reinterpret_cast<char*>(q_smem) + kCopy);
   const int tid = threadIdx.x;
   const int bw = a.bw;
   const int64_t n = a.n, j0 = a.j0;
@@ -298,11 +331,11 @@ __global__ void __launch_bounds__(kColThreads, 1) colloop_kernel(ColArgs a) {
   if (tid == 0) {
     tc::mbar_init(bar, 1);
     tc::fence_barrier_init();
-    tc::mbar_arrive_expect_tx(bar, kUBlkBytes);
+    tc::mbar_arrive_expect_tx(bar, kCopy);
     const char* src = reinterpret_cast<const char*>(a.Ublk + (j0 / kBlock) * kUBlkDoubles);
     char* dst = reinterpret_cast<char*>(q_smem);
-    for (uint32_t off = 0; off < kUBlkBytes; off += kBulkChunk) {
-      const uint32_t len = kUBlkBytes - off < kBulkChunk ? kUBlkBytes - off : kBulkChunk;
+    for (uint32_t off = 0; off < kCopy; off += kBulkChunk) {
+      const uint32_t len = kCopy - off < kBulkChunk ? kCopy - off : kBulkChunk;
       tc::bulk_copy_g2s(dst + off, src + off, len, bar);
     }
   }
@@ -391,10 +424,12 @@ __global__ void __launch_bounds__(kColThreads, 1) colloop_kernel(ColArgs a) {
         const double id = invd[jj];
         d2sum += invd2[jj];
         const double x = __shfl_sync(full, w[0][pown], qbase | town);
-        double c = rint_small(x * inv_s);
+        double sj = s, isj = inv_s;
+        if constexpr (Z) { sj = s * kap[jj]; isj = inv_s * kinv[jj]; }
+        double c = rint_small(x * isj);
         if (clip) c = fmin(fmax(c, cmin), cmax);
         else if (c < cmin || c > cmax) ovf = 1;
-        const double e = fma(-s, c, x) * id;  // (x - s c) / U_jj
+        const double e = fma(-sj, c, x) * id;  // (x - s_j c) / U_jj
         if (t == town) { ea[pown] = e; ca[pown] = c; }
         e2 = fma(e, e, e2);
 #pragma unroll
@@ -452,8 +487,8 @@ __global__ void __launch_bounds__(kColThreads, 1) colloop_kernel(ColArgs a) {
 template <class TW>
 __global__ void __launch_bounds__(128) pack_kernel(const TW* W, const uint8_t* dead, int64_t n,
                                                    const uint8_t* codes8, int64_t ldc8,
-                                                   const int* iperm, int reverse, int bits,
-                                                   int group,
+                                                   const int* iperm, const double* kappa,
+                                                   int reverse, int bits, int group,
                                                    int64_t ngroups, const float* scales,
                                                    const uint8_t* zeros, uint32_t* codes,
                                                    double* row_d2) {
@@ -492,7 +527,8 @@ __global__ void __launch_bounds__(128) pack_kernel(const TW* W, const uint8_t* d
     int64_t g = group ? pc / group : 0;  // groups follow the processing order
     float s = scales[r * ngroups + g], z = (float)zeros[r * ngroups + g];
     float code = (float)crow[pc];
-    double d = (double)w0 - (double)s * (double)(code - z);
+    const double sk = kappa ? (double)s * kappa[pc] : (double)s;
+    double d = (double)w0 - sk * (double)(code - z);
     acc += d * d;
   }
   __shared__ double red[4];
@@ -560,6 +596,7 @@ __global__ void q_ladder_kernel(int64_t m, int* overflow, float* alpha, float la
   } while (0)
 
 constexpr size_t kColSmem = (size_t)kUBlkBytes + 16;  // + the mbarrier
+constexpr size_t kColSmemZ = (size_t)kUBlkBytesZ + 16;
 
 cudaError_t quant_init_attributes() {
   const int smem = (int)kColSmem;
@@ -569,21 +606,23 @@ cudaError_t quant_init_attributes() {
   if ((e = cudaFuncSetAttribute(colloop_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem))) return e;
   if ((e = cudaFuncSetAttribute(colloop_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem))) return e;
   if ((e = cudaFuncSetAttribute(colloop_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem))) return e;
+  if ((e = cudaFuncSetAttribute(colloop_kernel<0, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kColSmemZ))) return e;
   const int row_smem = 32768 * (int)sizeof(float);  // a staged row of the widest layer
   if ((e = cudaFuncSetAttribute(q_load_perm_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, row_smem))) return e;
   return cudaFuncSetAttribute(q_load_perm_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, row_smem);
 }
 
-template <int G>
+template <int G, bool Z = false>
 static cudaError_t launch_colloop(const ColArgs& ca, cudaStream_t s) {
-  const size_t smem = kColSmem;
+  const size_t smem = Z ? kColSmemZ : kColSmem;
   unsigned grid = (unsigned)((ca.k_rows + kRowsPerCta - 1) / kRowsPerCta);
-  colloop_kernel<G><<<grid, kColThreads, smem, s>>>(ca);
+  colloop_kernel<G, Z><<<grid, kColThreads, smem, s>>>(ca);
   count_launches(1);
   return cudaGetLastError();
 }
 
-static cudaError_t colloop_dispatch(int group, const ColArgs& ca, cudaStream_t s) {
+static cudaError_t colloop_dispatch(int group, int spacing, const ColArgs& ca, cudaStream_t s) {
+  if (spacing) return group == 0 ? launch_colloop<0, true>(ca, s) : cudaErrorInvalidValue;
   switch (group) {
     case 0: return launch_colloop<0>(ca, s);
     case 16: return launch_colloop<16>(ca, s);
@@ -642,8 +681,13 @@ gq_status run_quantize(const QuantArgs& a, cudaStream_t s) {
     split_u_kernel<<<grid, 256, 0, s>>>(a.U, n, L.ldu, L.Uhi, L.Ulo);
     count_launches(1);
     Q_TRY(cudaGetLastError());
+    if (cfg.spacing) {
+      q_zsic_kernel<<<1, 1024, 0, s>>>(a.U, n, L.kappa);
+      count_launches(1);
+      Q_TRY(cudaGetLastError());
+    }
     dim3 g2(16, (unsigned)((n + kBlock - 1) / kBlock));
-    ublk_kernel<<<g2, 256, 0, s>>>(a.U, n, L.Ublk);
+    ublk_kernel<<<g2, 256, 0, s>>>(a.U, n, L.Ublk, cfg.spacing ? L.kappa : nullptr);
     count_launches(1);
     Q_TRY(cudaGetLastError());
   }
@@ -716,7 +760,7 @@ gq_status run_quantize(const QuantArgs& a, cudaStream_t s) {
       ca.ldc8 = L.ldc8; ca.scales = a.scales; ca.zeros = a.zeros; ca.ngroups = ngroups;
       ca.row_s = L.row_s; ca.row_z = L.row_z; ca.row_e2 = L.row_e2; ca.row_bnd = L.row_bnd;
       ca.overflow = L.overflow;
-      Q_TRY(colloop_dispatch(G, ca, sa));
+      Q_TRY(colloop_dispatch(G, cfg.spacing, ca, sa));
       const int64_t j1 = j0 + bw;
       if (j1 >= n) continue;
       const int64_t jn = std::min<int64_t>(j1 + kBlock, n);
@@ -766,14 +810,15 @@ gq_status run_quantize(const QuantArgs& a, cudaStream_t s) {
     Q_TRY(cudaStreamSynchronize(s));
   }
   const int* iperm = a.perm ? L.iperm : nullptr;
+  const double* kappa = cfg.spacing ? L.kappa : nullptr;
   const size_t pack_smem = a.perm ? (size_t)n : 0;
   if (a.wt == GQ_BF16)
     pack_kernel<__nv_bfloat16><<<(unsigned)m, 128, pack_smem, s>>>(
-        static_cast<const __nv_bfloat16*>(a.W), a.dead, n, L.codes8, L.ldc8, iperm,
+        static_cast<const __nv_bfloat16*>(a.W), a.dead, n, L.codes8, L.ldc8, iperm, kappa,
         cfg.reverse, cfg.bits, G, ngroups, a.scales, a.zeros, a.codes, L.row_d2);
   else
     pack_kernel<float><<<(unsigned)m, 128, pack_smem, s>>>(
-        static_cast<const float*>(a.W), a.dead, n, L.codes8, L.ldc8, iperm, cfg.reverse,
+        static_cast<const float*>(a.W), a.dead, n, L.codes8, L.ldc8, iperm, kappa, cfg.reverse,
         cfg.bits, G, ngroups, a.scales, a.zeros, a.codes, L.row_d2);
   count_launches(1);
   Q_TRY(cudaGetLastError());
@@ -783,4 +828,12 @@ gq_status run_quantize(const QuantArgs& a, cudaStream_t s) {
   return GQ_OK;
 }
 
+}  // namespace gq
+
+namespace gq {
+cudaError_t launch_zsic_spacing(const float* U, int64_t n, double* kappa, cudaStream_t s) {
+  q_zsic_kernel<<<1, 1024, 0, s>>>(U, n, kappa);
+  count_launches(1);
+  return cudaGetLastError();
+}
 }  // namespace gq

@@ -31,7 +31,8 @@ class GQError(RuntimeError):
 
 class _Cfg(ctypes.Structure):
     _fields_ = [("bits", ctypes.c_int), ("group_size", ctypes.c_int), ("reverse", ctypes.c_int),
-                ("clip", ctypes.c_int), ("ladder", ctypes.c_float), ("ladder_max", ctypes.c_int)]
+                ("clip", ctypes.c_int), ("ladder", ctypes.c_float), ("ladder_max", ctypes.c_int),
+                ("spacing", ctypes.c_int)]
 
 
 def _load():
@@ -63,6 +64,8 @@ def _load():
                                               P, P, P, P, P, SZ, P]
     lib.gq_prepare_hinv_static.restype = I
     lib.gq_prepare_hinv_static.argtypes = [P, I64, ctypes.c_double, I, P, P, P, P, P]
+    lib.gq_zsic_spacing.restype = I
+    lib.gq_zsic_spacing.argtypes = [P, I64, P, P]
     lib.gq_workspace_status.restype = I
     lib.gq_workspace_status.argtypes = [P, ctypes.POINTER(ctypes.c_int), P]
     return lib
@@ -73,7 +76,7 @@ EXPORTED = ("gq_version", "gq_status_string", "gq_hessian_accumulate", "gq_hessi
             "gq_prepare_workspace_size",
             "gq_prepare_hinv", "gq_quantize_workspace_size", "gq_quantize_layer",
             "gq_workspace_status", "gq_prepare_hinv_static", "gq_prepare_hinv_ordered",
-            "gq_quantize_layer_ordered")
+            "gq_quantize_layer_ordered", "gq_zsic_spacing")
 
 
 def _ptr(t):
@@ -205,10 +208,14 @@ class QuantCfg:
     clip: bool = True
     ladder: float = 1.25
     ladder_max: int = 8
+    spacing: str = "uniform"  # or "zsic": per-column steps, kappa_j = U_jj / geomean(U)
 
     def c(self) -> _Cfg:
+        if self.spacing not in ("uniform", "zsic"):
+            raise ValueError(f"unknown spacing {self.spacing!r}")
         return _Cfg(int(self.bits), int(self.group_size), int(bool(self.reverse)),
-                    int(bool(self.clip)), float(self.ladder), int(self.ladder_max))
+                    int(bool(self.clip)), float(self.ladder), int(self.ladder_max),
+                    1 if self.spacing == "zsic" else 0)
 
 
 def gq_quantize_workspace_size(m: int, n: int, cfg: QuantCfg) -> int:
@@ -267,6 +274,16 @@ def gq_quantize_layer_ordered(W: torch.Tensor, U: torch.Tensor, dead, delta, cfg
                                          ws.numel(), _stream(stream)),
            "gq_quantize_layer_ordered")
     return codes, scales, zeros, loss, ws
+
+
+def gq_zsic_spacing(U: torch.Tensor, kappa=None, stream=None) -> torch.Tensor:
+    """ZSIC column factors kappa_j = U_jj / geomean(U_kk) (fp64, processing order)."""
+    n = U.shape[0]
+    _need(U, torch.float32, (n, n), "U")
+    kappa = torch.empty(n, dtype=torch.float64, device=U.device) if kappa is None else kappa
+    _need(kappa, torch.float64, (n,), "kappa")
+    _check(LIB.gq_zsic_spacing(_ptr(U), n, _ptr(kappa), _stream(stream)), "gq_zsic_spacing")
+    return kappa
 
 
 def gq_workspace_status(ws: torch.Tensor, stream=None):

@@ -17,12 +17,14 @@ def unpack_np(packed: np.ndarray, n: int, bits: int) -> np.ndarray:
 
 
 def run_gpu(W: torch.Tensor, X: torch.Tensor, bits: int, group: int = 0, reverse: bool = False,
-            clip: bool = True, damp: float = 0.01, order=None, perm=None):
+            clip: bool = True, damp: float = 0.01, order=None, perm=None, spacing="uniform",
+            ladder_max: int = 8):
     from post_weight_quantization_22_b200 import gq as G
     from post_weight_quantization_22_b200.pipeline import LayerQuantizer
 
     m, n = W.shape
-    cfg = G.QuantCfg(bits=bits, group_size=group, reverse=reverse, clip=clip)
+    cfg = G.QuantCfg(bits=bits, group_size=group, reverse=reverse, clip=clip, spacing=spacing,
+                     ladder_max=ladder_max)
     lq = LayerQuantizer(m, n, cfg, device="cuda", damp=damp, order=order)
     if perm is not None:
         lq.perm.copy_(torch.as_tensor(np.asarray(perm), dtype=torch.int32))
@@ -35,7 +37,8 @@ def run_gpu(W: torch.Tensor, X: torch.Tensor, bits: int, group: int = 0, reverse
                 zeros=res.zeros.cpu().numpy().astype(np.int64), loss=res.loss.cpu().numpy(),
                 dead=res.dead.cpu().numpy().astype(bool), delta=float(res.delta.item()),
                 status=(sp, sq), rounds=rounds,
-                perm=None if lq.perm is None else lq.perm.cpu().numpy().astype(np.int64))
+                perm=None if lq.perm is None else lq.perm.cpu().numpy().astype(np.int64),
+                kappa=G.gq_zsic_spacing(res.U).cpu().numpy() if spacing == "zsic" else None)
 
 
 def rel_fro(a, b) -> float:

@@ -40,6 +40,10 @@ def test_size_queries_and_strings_without_gpu():
     assert G.gq_prepare_workspace_size(0) == 0
     assert G.gq_quantize_workspace_size(4096, 4096, G.QuantCfg(bits=9)) == 0
     assert G.gq_quantize_workspace_size(16, 16, G.QuantCfg(bits=3, group_size=64, reverse=True)) == 0
+    # ZSIC spacing takes a per-row grid and the forward (or ordered) form
+    assert G.gq_quantize_workspace_size(16, 16, G.QuantCfg(bits=3, group_size=16, spacing="zsic")) == 0
+    assert G.gq_quantize_workspace_size(16, 16, G.QuantCfg(bits=3, reverse=True, spacing="zsic")) == 0
+    assert G.gq_quantize_workspace_size(16, 16, G.QuantCfg(bits=3, spacing="zsic")) > 0
     assert G.LIB.gq_kernel_launches() == 0
 
 

@@ -23,9 +23,10 @@ H_REL_DESIGN = 1e-9   # digit rounding of entries below 2^-21 of their column's 
 U_REL_DESIGN = 1e-6
 
 
-def _oracle(W, X, bits, group, reverse, clip, rows=None, order=None):
+def _oracle(W, X, bits, group, reverse, clip, rows=None, order=None, spacing="uniform",
+            ladder_max=8):
     return O.quantize_layer(W, X, bits=bits, group=group, reverse=reverse, clip=clip, rows=rows,
-                            order=order)
+                            order=order, spacing=spacing, ladder_max=ladder_max)
 
 
 def _compare(g, o, W, bits, group, rows=None, check_loss=True, perm=None):
@@ -213,6 +214,36 @@ def test_act_order_tiny_fp32_per_row_and_dead_columns():
     _check_act_perm(g["perm"], o)
     assert g["dead"].sum() == 2
     _compare(g, o, W, 4, 0, perm=g["perm"])
+
+
+def test_zsic_spacing_clipfree_ladder():
+    """ZSIC per-column spacing (kappa_j = U_jj / geomean U) with the clip-free ladder: the
+    device's kappa, codes, steps, ladder rounds, losses and the per-column Theorem 5 bound
+    against the oracle.  8-bit codes and up to 16 widenings: the spacing spans ~20x on this
+    recipe, so the few finely spaced outlier columns need a wide code range."""
+    W, X, spec = synth.workload("q_proj_4096x4096", m=200, n=520, T=700)
+    g = run_gpu(W, X, bits=8, clip=False, spacing="zsic", ladder_max=16)
+    assert g["status"] == (0, 0)
+    o = _oracle(W, X, 8, 0, False, False, spacing="zsic", ladder_max=16)
+    np.testing.assert_allclose(g["kappa"], o["col_scale"], rtol=1e-6)
+    assert g["rounds"] == o["ladder_rounds"]
+    _compare(g, o, W, 8, 0)
+    assert g["loss"][1] <= g["loss"][2]
+
+
+def test_zsic_spacing_with_act_order_4bit_and_am_gm_bound():
+    """ZSIC spacing in act-order, 4-bit clamped, against the oracle; and on the device's own
+    outputs the AM-GM comparison: at the same row steps the ZSIC bound (n/4) s^2 g^2 is below
+    the uniform grid's (1/4) s^2 sum D."""
+    W, X, spec = synth.workload("q_proj_4096x4096", m=96, n=384, T=500)
+    g = run_gpu(W, X, bits=4, order="act", spacing="zsic")
+    assert g["status"] == (0, 0)
+    o = _oracle(W, X, 4, 0, False, True, order=g["perm"], spacing="zsic")
+    np.testing.assert_allclose(g["kappa"], o["col_scale"], rtol=1e-6)
+    _compare(g, o, W, 4, 0, perm=g["perm"])
+    u = run_gpu(W, X, bits=4, order="act")
+    np.testing.assert_allclose(g["scales"], u["scales"], rtol=0, atol=0)
+    assert g["loss"][2] <= u["loss"][2]
 
 
 def test_given_order_clipfree_ladder():
