@@ -49,6 +49,10 @@ __all__ = [
     "babai_sic_reverse",
     "zsic_spacing",
     "pack_codes",
+    "huffman_lengths",
+    "canonical_codewords",
+    "huffman_encode",
+    "huffman_decode",
     "proxy_loss",
     "quadratic_loss",
     "babai_bound",
@@ -228,7 +232,9 @@ def gptq_columns(W, U, bits: int, group: int = 0, clip: bool = True, alpha=None,
     Grid (reading): per row (group == 0) from the row as given; per group of ``group`` columns,
     recomputed at the group's first column from the current, error-fed weights of the group.
     clip=False: codes are unconstrained integers (no clamp) on the ``clipfree_grid`` with the
-    per-row factor ``alpha`` (group must be 0).  ``grid`` = (s, z) fixes the per-row grid
+    per-row factor ``alpha`` (group must be 0).  clip="unbounded" (HPTQ reading, [GEOM]
+    section 3: one unconstrained integer grid for normal and outlier weights): the lattice
+    s Z with the min-max step of the row, zero point 0, no clamp.  ``grid`` = (s, z) fixes the per-row grid
     instead (a fixed lattice).  ``col_scale`` (per-row grids only) multiplies the step of
     column j by col_scale[j]: the grid of column j is s col_scale[j] (c - z).
 
@@ -239,8 +245,8 @@ def gptq_columns(W, U, bits: int, group: int = 0, clip: bool = True, alpha=None,
     u = _f64(U)
     m, n = w.shape
     maxq = 2 ** bits - 1
-    if not clip and group:
-        raise ValueError("the clip-free variant uses a per-row grid")
+    if (not clip or clip == "unbounded") and group:
+        raise ValueError("the clip-free and unbounded variants use a per-row grid")
     if col_scale is not None and group:
         raise ValueError("per-column spacing uses a per-row grid")
     kap = np.ones(n) if col_scale is None else _f64(col_scale)
@@ -250,9 +256,15 @@ def gptq_columns(W, U, bits: int, group: int = 0, clip: bool = True, alpha=None,
     codes = np.zeros((m, n), dtype=np.int64)
     Q = np.zeros((m, n))
     E = np.zeros((m, n))
+    unbounded = clip == "unbounded"
+    if unbounded:
+        clip = False
     if group == 0:
         if grid is not None:
             s, z = (np.asarray(g, dtype=np.float64).copy() for g in grid)
+        elif unbounded:
+            s, _ = minmax_grid(w, bits)
+            z = np.zeros(m)
         elif clip:
             s, z = minmax_grid(w, bits)
         else:
@@ -329,6 +341,85 @@ def pack_codes(codes, bits: int) -> np.ndarray:
     return out.astype(np.uint32)
 
 
+# ---------------------------------------------------------------------------------------------
+# Entropy coding of unconstrained integer codes
+# ---------------------------------------------------------------------------------------------
+
+def huffman_lengths(counts) -> np.ndarray:
+    """Huffman code lengths for symbol counts ([GEOM] section 3, HPTQ: the integers of a single
+    unconstrained grid are Huffman-coded).  Textbook construction: repeatedly merge the two
+    least frequent trees; a symbol's length is its depth.  Symbols with count 0 get length 0;
+    a lone symbol gets length 1.  Ties may be broken either way: every optimal code has the same
+    total length sum(count * length), the quantity the tests compare.
+    """
+    import heapq
+    counts = [int(c) for c in counts]
+    live = [i for i, c in enumerate(counts) if c > 0]
+    lengths = np.zeros(len(counts), dtype=np.int64)
+    if len(live) == 1:
+        lengths[live[0]] = 1
+        return lengths
+    heap = [(counts[i], k, [i]) for k, i in enumerate(live)]
+    heapq.heapify(heap)
+    uid = len(live)
+    while len(heap) > 1:
+        c1, _, s1 = heapq.heappop(heap)
+        c2, _, s2 = heapq.heappop(heap)
+        for i in s1 + s2:
+            lengths[i] += 1
+        heapq.heappush(heap, (c1 + c2, uid, s1 + s2))
+        uid += 1
+    return lengths
+
+
+def canonical_codewords(lengths) -> np.ndarray:
+    """Canonical prefix code for given lengths: symbols ordered by (length, symbol) receive
+    consecutive codewords, shifted left by one at each increase of the length."""
+    lengths = [int(x) for x in lengths]
+    words = np.zeros(len(lengths), dtype=np.uint64)
+    code, prev = 0, 0
+    for ln, sym in sorted((ln, i) for i, ln in enumerate(lengths) if ln > 0):
+        code <<= ln - prev
+        words[sym] = code
+        code += 1
+        prev = ln
+    return words
+
+
+def huffman_encode(symbols, lengths) -> tuple[np.ndarray, int]:
+    """Concatenate the canonical codewords of ``symbols`` MSB first into 64-bit words (stream
+    bit i is bit 63 - i % 64 of word i // 64).  Returns (words, total bits)."""
+    words = canonical_codewords(lengths)
+    out = []
+    for sym in np.asarray(symbols).ravel():
+        ln = int(lengths[sym])
+        out.append(format(int(words[sym]), f"0{ln}b"))
+    bits = "".join(out)
+    nw = -(-len(bits) // 64)
+    padded = bits.ljust(64 * max(nw, 1), "0")
+    arr = np.array([int(padded[64 * k:64 * k + 64], 2) for k in range(max(nw, 1))],
+                   dtype=np.uint64)
+    return arr, len(bits)
+
+
+def huffman_decode(words, total_bits: int, lengths, count: int) -> np.ndarray:
+    """Inverse of ``huffman_encode``: read ``count`` symbols of the canonical code."""
+    cw = canonical_codewords(lengths)
+    table = {(int(lengths[i]), int(cw[i])): i for i in range(len(lengths)) if lengths[i] > 0}
+    bits = "".join(format(int(w), "064b") for w in np.asarray(words, dtype=np.uint64))[:total_bits]
+    out, pos = [], 0
+    for _ in range(count):
+        ln, val = 0, 0
+        while True:
+            val = (val << 1) | (bits[pos] == "1")
+            pos += 1
+            ln += 1
+            if (ln, val) in table:
+                out.append(table[(ln, val)])
+                break
+    return np.array(out, dtype=np.int64)
+
+
 def proxy_loss(W0, Q, X) -> float:
     """||(W0 - Q) X^T||_F^2: squared output error over the calibration tokens ([GEOM] 2.1)."""
     d = _f64(W0) - _f64(Q)
@@ -376,6 +467,9 @@ def quantize_layer(W, X, bits: int, group: int = 0, reverse: bool = False, clip:
     spacing="zsic" (per-row grids, forward or an explicit order): column j's step is the row
     step times ``zsic_spacing`` of the processing order's pivots.
 
+    clip="unbounded": codes are any integers on the per-row lattice s Z (see gptq_columns), no
+    ladder; they are meant for entropy coding (``huffman_lengths``).
+
     clip=False (reading of "per-row step set so that no entry needs clipping"): run unclamped;
     a row whose codes leave [0, 2^b - 1] is rerun with alpha multiplied by ``ladder``, at most
     ``ladder_max`` times; rows still outside raise ValueError.
@@ -393,6 +487,8 @@ def quantize_layer(W, X, bits: int, group: int = 0, reverse: bool = False, clip:
     maxq = 2 ** bits - 1
     if reverse and group:
         raise ValueError("the last-to-first variant uses a per-row grid")
+    if reverse and clip == "unbounded":
+        raise ValueError("the unbounded lattice takes the forward or ordered form")
     perm = None
     if order is not None:
         if reverse:
@@ -444,7 +540,7 @@ def quantize_layer(W, X, bits: int, group: int = 0, reverse: bool = False, clip:
     alpha = np.ones(len(sel))
     res = run(w_sel, alpha)
     retries = 0
-    if not clip:
+    if clip is False:
         for _ in range(ladder_max):
             bad = np.nonzero((res["codes"] < 0).any(axis=1) | (res["codes"] > maxq).any(axis=1))[0]
             if bad.size == 0:
@@ -480,4 +576,9 @@ def quantize_layer(W, X, bits: int, group: int = 0, reverse: bool = False, clip:
     # per-row grid, so the column order of s_cols does not matter)
     out["bound"] = babai_bound(s_cols, pivots)
     out["packed"] = pack_codes(np.clip(res["codes"], 0, maxq), bits)
+    if clip == "unbounded":
+        sym = res["codes"] - res["codes"].min()
+        ln = huffman_lengths(np.bincount(sym.ravel()))
+        out["huffman_bits"] = int(np.sum(np.bincount(sym.ravel()) * ln[:sym.max() + 1]))
+        out["rate"] = out["huffman_bits"] / sym.size
     return out

@@ -563,3 +563,52 @@ def test_zsic_bound_and_am_gm_against_uniform():
         np.testing.assert_allclose(b_z, 0.25 * 32 * s[r] ** 2 * g2, rtol=1e-12)
         assert d @ hd @ d <= b_z * (1 + 1e-12)
         assert b_z <= 0.25 * s[r] ** 2 * D.sum()
+
+
+# --------------------------------------------------------------------------------------------
+# Huffman coding of unconstrained integer codes (GEOM section 3, HPTQ)
+# --------------------------------------------------------------------------------------------
+
+def test_huffman_textbook_example():
+    """The classic six-symbol example (counts 45, 13, 12, 16, 9, 5): optimal total length 224,
+    lengths (1, 3, 3, 3, 4, 4)."""
+    ln = O.huffman_lengths([45, 13, 12, 16, 9, 5])
+    assert int(np.dot(ln, [45, 13, 12, 16, 9, 5])) == 224
+    assert sorted(ln.tolist()) == [1, 3, 3, 3, 4, 4]
+
+
+@pytest.mark.parametrize("seed", range(3))
+def test_huffman_kraft_entropy_and_roundtrip(seed):
+    """Kraft equality sum 2^-l = 1 (a full prefix code), N H <= total < N (H + 1), the canonical
+    codewords are prefix-free, and decoding the stream gives the symbols back."""
+    rng = np.random.default_rng(200 + seed)
+    sym = np.clip(np.rint(rng.standard_t(3, 3000) * 3).astype(np.int64) + 40, 0, 80)
+    counts = np.bincount(sym, minlength=81)
+    ln = O.huffman_lengths(counts)
+    used = counts > 0
+    assert abs(np.sum(2.0 ** -ln[used]) - 1.0) < 1e-12
+    p = counts[used] / counts.sum()
+    H = -np.sum(p * np.log2(p))
+    total = int(np.dot(counts, ln))
+    assert sym.size * H <= total < sym.size * (H + 1)
+    cw = O.canonical_codewords(ln)
+    words = [format(int(cw[i]), f"0{ln[i]}b") for i in np.nonzero(used)[0]]
+    for a in words:
+        for b in words:
+            assert a == b or not b.startswith(a)
+    stream, nbits = O.huffman_encode(sym, ln)
+    assert nbits == total
+    assert np.array_equal(O.huffman_decode(stream, nbits, ln, sym.size), sym)
+
+
+def test_unbounded_lattice_on_diagonal_hessian_is_rounding():
+    """Unconstrained lattice, diagonal H: no feedback, codes = rint(w / s) with zero point 0 and
+    s the min-max step of the row (values far outside the b-bit range stay unclamped)."""
+    rng = np.random.default_rng(211)
+    w = 0.02 * rng.standard_normal((6, 12))
+    w[0, 3] = 0.5  # an outlier
+    res = O.quantize_layer(w, None, 3, H=np.diag(rng.uniform(1, 2, 12)), clip="unbounded")
+    s = (np.maximum(w.max(1), 0) - np.minimum(w.min(1), 0)) / 7.0
+    np.testing.assert_array_equal(res["codes"], np.rint(w / s[:, None]))
+    assert (res["zeros"] == 0).all()
+    assert res["rate"] > 0
