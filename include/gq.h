@@ -71,7 +71,11 @@ typedef struct {
   int bits;       /* code width b, 2..8 */
   int group_size; /* 0: one grid per row; else the group width, which must divide 128 */
   int reverse;    /* 0: columns first to last (GPTQ order); 1: last to first (Babai order) */
-  int clip;       /* 1: codes clamped to [0, 2^b-1] (GPTQ); 0: clip-free with a scale ladder */
+  int clip;       /* 1: codes clamped to [0, 2^b-1] (GPTQ); 0: clip-free with a scale ladder;
+                     2: unconstrained integer lattice ("The Geometry of LLM Quantization",
+                     section 3, HPTQ): step s = (hi - lo) / (2^b - 1) of the row, zero point 0,
+                     codes any int32 (for entropy coding, gq_huffman_encode); needs
+                     group_size 0 and reverse 0 */
   float ladder;   /* clip-free: factor applied to a row's step when its codes overflow (1.25) */
   int ladder_max; /* clip-free: at most this many widenings per row (8) */
   int spacing;    /* 0: one step per row or group; 1: ZSIC ("WaterSIC", section 2: grid spacing
@@ -206,6 +210,8 @@ size_t gq_quantize_workspace_size(int64_t m, int64_t n, const gq_quant_cfg* cfg)
  *   d_delta   1 double from gq_prepare_hinv (may be NULL: loss[0] is then not computed).
  *   d_codes   m x ceil(n*b/32) uint32, written: per row an LSB-first bitstream of b-bit
  *             codes, the code of ORIGINAL column c at bits [b*c, b*c+b); unused bits are 0.
+ *             With clip = 2: m x n int32, the code of original column c at [row][c]
+ *             (dequantized weight = scale * code).
  *   d_scales  m x G fp32, written, G = 1 (group_size 0) or ceil(n / group_size); group g
  *             covers original columns [g*group_size, (g+1)*group_size).
  *   d_zeros   m x G uint8, written; dequantized weight = scale * (code - zero).
@@ -250,6 +256,34 @@ gq_status gq_quantize_layer_ordered(const void* d_W, gq_dtype w_dtype, int64_t m
  *   d_U      n x n fp32, device.   d_kappa  n fp64, device, written.   1 <= n <= 32768.
  */
 gq_status gq_zsic_spacing(const float* d_U, int64_t n, double* d_kappa, gq_stream_t stream);
+
+/* Workspace bytes gq_huffman_encode needs for `count` codes (0 if count is out of range). */
+size_t gq_huffman_workspace_size(int64_t count);
+
+/*
+ * Canonical Huffman coding of integer codes ("The Geometry of LLM Quantization", section 3,
+ * HPTQ: the integers of one unconstrained grid are Huffman-coded, so the bit width follows the
+ * weight distribution; "WaterSIC", section 2: entropy coding of the ZSIC integers).  Typical
+ * input: the int32 codes of gq_quantize_layer with clip = 2; rate = total bits / count.
+ *
+ *   d_codes      count int32, device, read.  1 <= count <= 2^31 - 1.  The values may span at
+ *                most 4096 consecutive integers (symbol k is the value min + k).
+ *   d_stream     stream_words uint64, device, written (zeroed first): the codewords of d_codes
+ *                in order, MSB first (stream bit i is bit 63 - i % 64 of word i / 64).  Room
+ *                for count words (64 bits a code) always suffices.
+ *   d_lengths    4096 uint8, device, written: the codeword length of symbol k (0 = unused).
+ *   d_codewords  4096 uint64, device, written: the canonical codeword of symbol k (symbols in
+ *                order of (length, k) take consecutive values, shifted left at each new length).
+ *   d_info       4 int64, device, written: [min value, number of symbols spanned, total bits,
+ *                longest codeword].
+ *   d_ws         workspace of at least gq_huffman_workspace_size(count) bytes.
+ * Device-detected errors (nothing is encoded): GQ_ERR_UNSUPPORTED (more than 4096 values
+ * spanned, or a codeword longer than 63 bits), GQ_ERR_WORKSPACE (the total exceeds
+ * 64 * stream_words bits).
+ */
+gq_status gq_huffman_encode(const int32_t* d_codes, int64_t count, uint64_t* d_stream,
+                            int64_t stream_words, uint8_t* d_lengths, uint64_t* d_codewords,
+                            int64_t* d_info, void* d_ws, size_t ws_bytes, gq_stream_t stream);
 
 /*
  * Synchronize `stream` and return the device-side status recorded in a workspace by the last

@@ -31,6 +31,7 @@ gq_status ensure_device_setup() {
   if (quant_init_attributes() != cudaSuccess) return GQ_ERR_CUDA;
   if (lazy_tc_init_attributes() != cudaSuccess) return GQ_ERR_CUDA;
   if (hessian_init_attributes() != cudaSuccess) return GQ_ERR_CUDA;
+  if (huffman_init_attributes() != cudaSuccess) return GQ_ERR_CUDA;
   g_init_done[dev] = true;
   return GQ_OK;
 }
@@ -207,12 +208,13 @@ static gq_status check_cfg(const gq_quant_cfg* cfg) {
   if (!cfg) return GQ_ERR_INVALID_ARG;
   if (cfg->bits < 2 || cfg->bits > 8) return GQ_ERR_INVALID_ARG;
   if (cfg->reverse != 0 && cfg->reverse != 1) return GQ_ERR_INVALID_ARG;
-  if (cfg->clip != 0 && cfg->clip != 1) return GQ_ERR_INVALID_ARG;
+  if (cfg->clip < 0 || cfg->clip > 2) return GQ_ERR_INVALID_ARG;
   const int g = cfg->group_size;
   if (g != 0 && g != 16 && g != 32 && g != 64 && g != 128) {
     return (g > 0 && g <= 128 && kBlock % g == 0) ? GQ_ERR_UNSUPPORTED : GQ_ERR_INVALID_ARG;
   }
-  if (g != 0 && (cfg->reverse || !cfg->clip)) return GQ_ERR_UNSUPPORTED;
+  if (g != 0 && (cfg->reverse || cfg->clip != 1)) return GQ_ERR_UNSUPPORTED;
+  if (cfg->clip == 2 && cfg->reverse) return GQ_ERR_UNSUPPORTED;
   if (cfg->spacing != 0 && cfg->spacing != 1) return GQ_ERR_INVALID_ARG;
   if (cfg->spacing && (g != 0 || cfg->reverse)) return GQ_ERR_UNSUPPORTED;
   if (!cfg->clip) {
@@ -283,6 +285,35 @@ gq_status gq_zsic_spacing(const float* d_U, int64_t n, double* d_kappa, gq_strea
   if (st != GQ_OK) return st;
   return launch_zsic_spacing(d_U, n, d_kappa, (cudaStream_t)stream) == cudaSuccess ? GQ_OK
                                                                                    : GQ_ERR_CUDA;
+}
+
+size_t gq_huffman_workspace_size(int64_t count) {
+  if (count < 1 || count > (int64_t(1) << 31) - 1) return 0;
+  return huffman_ws_bytes(count);
+}
+
+gq_status gq_huffman_encode(const int32_t* d_codes, int64_t count, uint64_t* d_stream,
+                            int64_t stream_words, uint8_t* d_lengths, uint64_t* d_codewords,
+                            int64_t* d_info, void* d_ws, size_t ws_bytes, gq_stream_t stream) {
+  if (count < 1 || count > (int64_t(1) << 31) - 1 || stream_words < 1) return GQ_ERR_INVALID_ARG;
+  if (!d_codes || !d_stream || !d_lengths || !d_codewords || !d_info || !d_ws)
+    return GQ_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(d_stream) & 7u) || (reinterpret_cast<uintptr_t>(d_codewords) & 7u) ||
+      (reinterpret_cast<uintptr_t>(d_info) & 7u) || (reinterpret_cast<uintptr_t>(d_codes) & 3u))
+    return GQ_ERR_INVALID_ARG;
+  if (!aligned256(d_ws) || ws_bytes < huffman_ws_bytes(count)) return GQ_ERR_WORKSPACE;
+  gq_status st = ensure_device_setup();
+  if (st != GQ_OK) return st;
+  auto enqueue = [&](cudaStream_t s) {
+    return launch_huffman(d_codes, count, reinterpret_cast<unsigned long long*>(d_stream),
+                          stream_words, d_lengths,
+                          reinterpret_cast<unsigned long long*>(d_codewords),
+                          reinterpret_cast<long long*>(d_info), d_ws, s) == cudaSuccess
+               ? GQ_OK : GQ_ERR_CUDA;
+  };
+  return run_graphed({5, P(d_codes), (uint64_t)count, P(d_stream), (uint64_t)stream_words,
+                      P(d_lengths), P(d_codewords), P(d_info), P(d_ws)},
+                     (cudaStream_t)stream, enqueue);
 }
 
 gq_status gq_workspace_status(void* d_ws, int* h_ladder_rounds, gq_stream_t stream) {

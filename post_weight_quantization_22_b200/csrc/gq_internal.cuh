@@ -79,6 +79,13 @@ struct QuantArgs {
 };
 size_t quantize_ws_bytes(int64_t m, int64_t n, const gq_quant_cfg& cfg);
 cudaError_t launch_zsic_spacing(const float* U, int64_t n, double* kappa, cudaStream_t s);
+
+// ---- canonical Huffman coding of int32 codes ----
+size_t huffman_ws_bytes(int64_t count);
+cudaError_t huffman_init_attributes();
+cudaError_t launch_huffman(const int* codes, int64_t count, unsigned long long* stream_words,
+                           int64_t nwords, uint8_t* lengths, unsigned long long* words,
+                           long long* info, void* ws, cudaStream_t s);
 // Returns GQ_OK or an error; the clip-free ladder synchronizes the stream per round.
 gq_status run_quantize(const QuantArgs& a, cudaStream_t s);
 

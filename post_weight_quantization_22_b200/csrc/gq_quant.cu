@@ -57,10 +57,11 @@ struct QLayout {
   int* counter;
   int* iperm;       // n: processing position of each original column (ordered calls)
   double* kappa;    // n: ZSIC column factors in processing order
+  int* codes32;     // m x n int32 codes in processing order (unconstrained lattice only)
   size_t bytes;
 };
 
-static QLayout q_layout(void* ws, int64_t m, int64_t n) {
+static QLayout q_layout(void* ws, int64_t m, int64_t n, bool unbounded) {
   Carver c(ws);
   QLayout L;
   L.hdr = c.take<WsHeader>(1);
@@ -86,12 +87,13 @@ static QLayout q_layout(void* ws, int64_t m, int64_t n) {
   L.counter = c.take<int>(4);
   L.iperm = c.take<int>((size_t)n);
   L.kappa = c.take<double>((size_t)n);
+  L.codes32 = unbounded ? c.take<int>((size_t)m * n) : nullptr;
   L.bytes = c.off;
   return L;
 }
 
-size_t quantize_ws_bytes(int64_t m, int64_t n, const gq_quant_cfg&) {
-  return q_layout(nullptr, m, n).bytes;
+size_t quantize_ws_bytes(int64_t m, int64_t n, const gq_quant_cfg& cfg) {
+  return q_layout(nullptr, m, n, cfg.clip == 2).bytes;
 }
 
 // ------------------------------------------------------------------------------------------
@@ -175,9 +177,12 @@ __global__ void q_row_grid_kernel(const float* Wf, int64_t n, int64_t k_rows, co
     if (dlo == 0.0 && dhi == 0.0) { dlo = -1.0; dhi = 1.0; }
     double maxq = (double)((1 << bits) - 1);
     double s, z;
-    if (clip) {
+    if (clip == 1) {
       s = (dhi - dlo) / maxq;
       z = rint(-dlo / s);
+    } else if (clip == 2) {  // unconstrained lattice s Z: the min-max step, zero point 0
+      s = (dhi - dlo) / maxq;
+      z = 0.0;
     } else {
       s = (double)alpha[row] * (dhi - dlo) / maxq;
       z = rint(maxq * 0.5 - (dhi + dlo) / (2.0 * s));
@@ -284,6 +289,7 @@ struct ColArgs {
   float* Elo;
   uint8_t* codes8;
   int64_t ldc8;
+  int* codes32;  // unconstrained lattice: int32 codes (processing order, row stride n), or null
   float* scales;
   uint8_t* zeros;
   int64_t ngroups;
@@ -374,7 +380,8 @@ __global__ void __launch_bounds__(kColThreads, 1) colloop_kernel(ColArgs a) {
   if (G == 0 && act) { s = a.row_s[row]; z = a.row_z[row]; inv_s = 1.0 / s; }
   double e2 = 0.0, bnd = 0.0;
   int ovf = 0;
-  const bool clip = a.clip != 0;
+  const bool clip = a.clip == 1;      // clamp to [0, 2^b - 1]
+  const bool track = a.clip == 0;     // clip-free: flag codes outside the range for the ladder
 
 #pragma unroll 1
   for (int T = 0; T < kTiles; ++T) {
@@ -428,7 +435,7 @@ __global__ void __launch_bounds__(kColThreads, 1) colloop_kernel(ColArgs a) {
         if constexpr (Z) { sj = s * kap[jj]; isj = inv_s * kinv[jj]; }
         double c = rint_small(x * isj);
         if (clip) c = fmin(fmax(c, cmin), cmax);
-        else if (c < cmin || c > cmax) ovf = 1;
+        else if (track && (c < cmin || c > cmax)) ovf = 1;
         const double e = fma(-sj, c, x) * id;  // (x - s_j c) / U_jj
         if (t == town) { ea[pown] = e; ca[pown] = c; }
         e2 = fma(e, e, e2);
@@ -448,9 +455,15 @@ __global__ void __launch_bounds__(kColThreads, 1) colloop_kernel(ColArgs a) {
         lo2.x = f0 - hi2.x; lo2.y = f1 - hi2.y;
         *reinterpret_cast<float2*>(a.Ehi + rr * kBlock + col) = hi2;
         *reinterpret_cast<float2*>(a.Elo + rr * kBlock + col) = lo2;
-        uint8_t* cp = a.codes8 + row * a.ldc8 + j0 + col;
-        cp[0] = (uint8_t)(int)fmin(fmax(ca[0] + z, 0.0), maxq);
-        if (col + 1 < bw) cp[1] = (uint8_t)(int)fmin(fmax(ca[1] + z, 0.0), maxq);
+        if (a.codes32) {  // unconstrained lattice: z = 0, any integer
+          int* cp = a.codes32 + row * n + j0 + col;
+          cp[0] = (int)ca[0];
+          if (col + 1 < bw) cp[1] = (int)ca[1];
+        } else {
+          uint8_t* cp = a.codes8 + row * a.ldc8 + j0 + col;
+          cp[0] = (uint8_t)(int)fmin(fmax(ca[0] + z, 0.0), maxq);
+          if (col + 1 < bw) cp[1] = (uint8_t)(int)fmin(fmax(ca[1] + z, 0.0), maxq);
+        }
       }
     }
     // the later tiles of the block take this tile's errors: w[k] -= E_T U[T rows][tile k]
@@ -488,13 +501,14 @@ template <class TW>
 __global__ void __launch_bounds__(128) pack_kernel(const TW* W, const uint8_t* dead, int64_t n,
                                                    const uint8_t* codes8, int64_t ldc8,
                                                    const int* iperm, const double* kappa,
-                                                   int reverse, int bits, int group,
+                                                   const int* codes32, int reverse, int bits,
+                                                   int group,
                                                    int64_t ngroups, const float* scales,
                                                    const uint8_t* zeros, uint32_t* codes,
                                                    double* row_d2) {
   const int64_t r = blockIdx.x;
   const uint8_t* crow = codes8 + r * ldc8;
-  if (iperm) {  // ordered call: gather the codes from a shared-memory copy of the row
+  if (!codes32 && iperm) {  // ordered call: gather the codes from a shared-memory copy of the row
     extern __shared__ uint8_t scodes[];
     for (int64_t p = threadIdx.x; p < n; p += blockDim.x) scodes[p] = crow[p];
     __syncthreads();
@@ -504,7 +518,12 @@ __global__ void __launch_bounds__(128) pack_kernel(const TW* W, const uint8_t* d
   auto pos = [&](int64_t c) -> int64_t {
     return iperm ? perm_at(iperm, c, n) : (reverse ? n - 1 - c : c);
   };
-  const int64_t nwords = (n * bits + 31) / 32;
+  const int* crow32 = codes32 ? codes32 + r * n : nullptr;
+  if (codes32) {  // unconstrained lattice: the output is int32 codes in original column order
+    int* out = reinterpret_cast<int*>(codes) + r * n;
+    for (int64_t c = threadIdx.x; c < n; c += blockDim.x) out[c] = crow32[pos(c)];
+  }
+  const int64_t nwords = codes32 ? 0 : (n * bits + 31) / 32;
   for (int64_t w = threadIdx.x; w < nwords; w += blockDim.x) {
     uint32_t word = 0u;
     int64_t cf = (32 * w) / bits, cl = (32 * w + 31) / bits;
@@ -526,7 +545,7 @@ __global__ void __launch_bounds__(128) pack_kernel(const TW* W, const uint8_t* d
     const int64_t pc = pos(c);
     int64_t g = group ? pc / group : 0;  // groups follow the processing order
     float s = scales[r * ngroups + g], z = (float)zeros[r * ngroups + g];
-    float code = (float)crow[pc];
+    float code = codes32 ? (float)crow32[pc] : (float)crow[pc];
     const double sk = kappa ? (double)s * kappa[pc] : (double)s;
     double d = (double)w0 - sk * (double)(code - z);
     acc += d * d;
@@ -667,7 +686,7 @@ static cudaError_t quant_streams(QuantStreams** out) {
 
 gq_status run_quantize(const QuantArgs& a, cudaStream_t s) {
   const int64_t m = a.m, n = a.n;
-  QLayout L = q_layout(a.ws, m, n);
+  QLayout L = q_layout(a.ws, m, n, a.cfg.clip == 2);
   const gq_quant_cfg& cfg = a.cfg;
   const int G = cfg.group_size;
   const int64_t ngroups = G ? (n + G - 1) / G : 1;
@@ -757,6 +776,7 @@ gq_status run_quantize(const QuantArgs& a, cudaStream_t s) {
       ca.U = a.U; ca.bits = cfg.bits; ca.clip = cfg.clip; ca.Ehi = L.Ehi[b & 1];
       ca.Elo = L.Elo[b & 1];
       ca.codes8 = L.codes8;
+      ca.codes32 = L.codes32;
       ca.ldc8 = L.ldc8; ca.scales = a.scales; ca.zeros = a.zeros; ca.ngroups = ngroups;
       ca.row_s = L.row_s; ca.row_z = L.row_z; ca.row_e2 = L.row_e2; ca.row_bnd = L.row_bnd;
       ca.overflow = L.overflow;
@@ -811,15 +831,15 @@ gq_status run_quantize(const QuantArgs& a, cudaStream_t s) {
   }
   const int* iperm = a.perm ? L.iperm : nullptr;
   const double* kappa = cfg.spacing ? L.kappa : nullptr;
-  const size_t pack_smem = a.perm ? (size_t)n : 0;
+  const size_t pack_smem = (a.perm && !L.codes32) ? (size_t)n : 0;
   if (a.wt == GQ_BF16)
     pack_kernel<__nv_bfloat16><<<(unsigned)m, 128, pack_smem, s>>>(
         static_cast<const __nv_bfloat16*>(a.W), a.dead, n, L.codes8, L.ldc8, iperm, kappa,
-        cfg.reverse, cfg.bits, G, ngroups, a.scales, a.zeros, a.codes, L.row_d2);
+        L.codes32, cfg.reverse, cfg.bits, G, ngroups, a.scales, a.zeros, a.codes, L.row_d2);
   else
     pack_kernel<float><<<(unsigned)m, 128, pack_smem, s>>>(
-        static_cast<const float*>(a.W), a.dead, n, L.codes8, L.ldc8, iperm, kappa, cfg.reverse,
-        cfg.bits, G, ngroups, a.scales, a.zeros, a.codes, L.row_d2);
+        static_cast<const float*>(a.W), a.dead, n, L.codes8, L.ldc8, iperm, kappa, L.codes32,
+        cfg.reverse, cfg.bits, G, ngroups, a.scales, a.zeros, a.codes, L.row_d2);
   count_launches(1);
   Q_TRY(cudaGetLastError());
   q_reduce_kernel<<<1, 1024, 0, s>>>(m, L.row_e2, L.row_bnd, L.row_d2, a.delta, a.loss);

@@ -64,6 +64,10 @@ def _load():
                                               P, P, P, P, P, SZ, P]
     lib.gq_prepare_hinv_static.restype = I
     lib.gq_prepare_hinv_static.argtypes = [P, I64, ctypes.c_double, I, P, P, P, P, P]
+    lib.gq_huffman_workspace_size.restype = SZ
+    lib.gq_huffman_workspace_size.argtypes = [I64]
+    lib.gq_huffman_encode.restype = I
+    lib.gq_huffman_encode.argtypes = [P, I64, P, I64, P, P, P, P, SZ, P]
     lib.gq_zsic_spacing.restype = I
     lib.gq_zsic_spacing.argtypes = [P, I64, P, P]
     lib.gq_workspace_status.restype = I
@@ -76,7 +80,8 @@ EXPORTED = ("gq_version", "gq_status_string", "gq_hessian_accumulate", "gq_hessi
             "gq_prepare_workspace_size",
             "gq_prepare_hinv", "gq_quantize_workspace_size", "gq_quantize_layer",
             "gq_workspace_status", "gq_prepare_hinv_static", "gq_prepare_hinv_ordered",
-            "gq_quantize_layer_ordered", "gq_zsic_spacing")
+            "gq_quantize_layer_ordered", "gq_zsic_spacing", "gq_huffman_workspace_size",
+            "gq_huffman_encode")
 
 
 def _ptr(t):
@@ -205,7 +210,7 @@ class QuantCfg:
     bits: int = 4
     group_size: int = 0
     reverse: bool = False
-    clip: bool = True
+    clip: bool | str = True  # True clamp, False clip-free ladder, "unbounded" lattice s Z
     ladder: float = 1.25
     ladder_max: int = 8
     spacing: str = "uniform"  # or "zsic": per-column steps, kappa_j = U_jj / geomean(U)
@@ -213,9 +218,9 @@ class QuantCfg:
     def c(self) -> _Cfg:
         if self.spacing not in ("uniform", "zsic"):
             raise ValueError(f"unknown spacing {self.spacing!r}")
-        return _Cfg(int(self.bits), int(self.group_size), int(bool(self.reverse)),
-                    int(bool(self.clip)), float(self.ladder), int(self.ladder_max),
-                    1 if self.spacing == "zsic" else 0)
+        clip = 2 if self.clip == "unbounded" else int(bool(self.clip))
+        return _Cfg(int(self.bits), int(self.group_size), int(bool(self.reverse)), clip,
+                    float(self.ladder), int(self.ladder_max), 1 if self.spacing == "zsic" else 0)
 
 
 def gq_quantize_workspace_size(m: int, n: int, cfg: QuantCfg) -> int:
@@ -236,7 +241,8 @@ def gq_quantize_layer(W: torch.Tensor, U: torch.Tensor, dead, delta, cfg: QuantC
     dev = W.device
     _need(U, torch.float32, (n, n), "U")
     G = 1 if cfg.group_size == 0 else -(-n // cfg.group_size)
-    codes = torch.empty((m, n_words(n, cfg.bits)), dtype=torch.int32, device=dev) if codes is None else codes
+    ncols = n if cfg.clip == "unbounded" else n_words(n, cfg.bits)
+    codes = torch.empty((m, ncols), dtype=torch.int32, device=dev) if codes is None else codes
     scales = torch.empty((m, G), dtype=torch.float32, device=dev) if scales is None else scales
     zeros = torch.empty((m, G), dtype=torch.uint8, device=dev) if zeros is None else zeros
     loss = torch.empty(3, dtype=torch.float64, device=dev) if loss is None else loss
@@ -262,7 +268,8 @@ def gq_quantize_layer_ordered(W: torch.Tensor, U: torch.Tensor, dead, delta, cfg
     _need(U, torch.float32, (n, n), "U")
     _need(perm, torch.int32, (n,), "perm")
     G = 1 if cfg.group_size == 0 else -(-n // cfg.group_size)
-    codes = torch.empty((m, n_words(n, cfg.bits)), dtype=torch.int32, device=dev) if codes is None else codes
+    ncols = n if cfg.clip == "unbounded" else n_words(n, cfg.bits)
+    codes = torch.empty((m, ncols), dtype=torch.int32, device=dev) if codes is None else codes
     scales = torch.empty((m, G), dtype=torch.float32, device=dev) if scales is None else scales
     zeros = torch.empty((m, G), dtype=torch.uint8, device=dev) if zeros is None else zeros
     loss = torch.empty(3, dtype=torch.float64, device=dev) if loss is None else loss
@@ -284,6 +291,27 @@ def gq_zsic_spacing(U: torch.Tensor, kappa=None, stream=None) -> torch.Tensor:
     _need(kappa, torch.float64, (n,), "kappa")
     _check(LIB.gq_zsic_spacing(_ptr(U), n, _ptr(kappa), _stream(stream)), "gq_zsic_spacing")
     return kappa
+
+
+def gq_huffman_encode(codes: torch.Tensor, stream_words: int | None = None, ws=None,
+                      stream=None):
+    """Canonical Huffman coding of int32 codes on the device.  Returns (stream uint64 words as
+    an int64 tensor, lengths uint8[4096], codewords int64[4096], info int64[4]
+    = [min value, symbols spanned, total bits, longest codeword], workspace)."""
+    if not codes.is_cuda or codes.dtype != torch.int32 or not codes.is_contiguous():
+        raise ValueError("codes: expected a contiguous cuda int32 tensor")
+    count = codes.numel()
+    dev = codes.device
+    words = count if stream_words is None else int(stream_words)
+    out = torch.empty(max(words, 1), dtype=torch.int64, device=dev)
+    lengths = torch.empty(4096, dtype=torch.uint8, device=dev)
+    cw = torch.empty(4096, dtype=torch.int64, device=dev)
+    info = torch.empty(4, dtype=torch.int64, device=dev)
+    ws = workspace(int(LIB.gq_huffman_workspace_size(count)), dev) if ws is None else ws
+    _check(LIB.gq_huffman_encode(_ptr(codes), count, _ptr(out), out.numel(), _ptr(lengths),
+                                 _ptr(cw), _ptr(info), _ptr(ws), ws.numel(), _stream(stream)),
+           "gq_huffman_encode")
+    return out, lengths, cw, info, ws
 
 
 def gq_workspace_status(ws: torch.Tensor, stream=None):

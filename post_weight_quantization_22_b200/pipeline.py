@@ -44,7 +44,8 @@ class LayerQuantizer:
         self.ws_prep = G.workspace(G.gq_prepare_workspace_size(n), dev)
         self.ws_quant = G.workspace(G.gq_quantize_workspace_size(m, n, cfg), dev)
         ng = 1 if cfg.group_size == 0 else -(-n // cfg.group_size)
-        self.codes = torch.empty((m, G.n_words(n, cfg.bits)), dtype=torch.int32, device=dev)
+        ncols = n if cfg.clip == "unbounded" else G.n_words(n, cfg.bits)
+        self.codes = torch.empty((m, ncols), dtype=torch.int32, device=dev)
         self.scales = torch.empty((m, ng), dtype=torch.float32, device=dev)
         self.zeros = torch.empty((m, ng), dtype=torch.uint8, device=dev)
         self.loss = torch.empty(3, dtype=torch.float64, device=dev)

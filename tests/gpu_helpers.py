@@ -31,9 +31,14 @@ def run_gpu(W: torch.Tensor, X: torch.Tensor, bits: int, group: int = 0, reverse
     res = lq.run(W.cuda().contiguous(), X.cuda().contiguous())
     torch.cuda.synchronize()
     sp, sq, rounds = lq.status()
-    packed = res.codes.cpu().numpy().view(np.uint32)
+    if clip == "unbounded":  # int32 codes, original column order
+        packed = None
+        codes = res.codes.cpu().numpy().astype(np.int64)
+    else:
+        packed = res.codes.cpu().numpy().view(np.uint32)
+        codes = unpack_np(packed, n, bits)
     return dict(H=res.H.cpu().numpy(), U=res.U.cpu().numpy(), packed=packed,
-                codes=unpack_np(packed, n, bits), scales=res.scales.cpu().numpy(),
+                codes=codes, scales=res.scales.cpu().numpy(), codes_dev=res.codes,
                 zeros=res.zeros.cpu().numpy().astype(np.int64), loss=res.loss.cpu().numpy(),
                 dead=res.dead.cpu().numpy().astype(bool), delta=float(res.delta.item()),
                 status=(sp, sq), rounds=rounds,

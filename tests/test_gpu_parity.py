@@ -59,8 +59,9 @@ def _compare(g, o, W, bits, group, rows=None, check_loss=True, perm=None):
         np.testing.assert_allclose(gs, o["scales"], rtol=1e-6)
     # packed words: identical wherever a row's codes are identical
     same = np.all(gc == o["codes"], axis=1)
-    gp = g["packed"] if rows is None else g["packed"][rows]
-    assert np.array_equal(gp[same], o["packed"][same])
+    if g["packed"] is not None:
+        gp = g["packed"] if rows is None else g["packed"][rows]
+        assert np.array_equal(gp[same], o["packed"][same])
     if check_loss and rows is None:
         # absolute floor for exactly-representable rows (zero loss): fp rounding of one unit
         # of error energy, ||W0||^2 mean(diag H) * 1e-12
@@ -244,6 +245,85 @@ def test_zsic_spacing_with_act_order_4bit_and_am_gm_bound():
     u = run_gpu(W, X, bits=4, order="act")
     np.testing.assert_allclose(g["scales"], u["scales"], rtol=0, atol=0)
     assert g["loss"][2] <= u["loss"][2]
+
+
+def _huffman_check(codes_dev, stream_words=None):
+    """The device's Huffman coding of int32 codes against the oracle: the total is the optimal
+    total of the codes' histogram (unique over all optimal codes), the lengths form a complete
+    prefix code, and the stream equals the oracle's encoding with the device's lengths, bit for
+    bit (canonical codewords are fixed by the lengths)."""
+    from post_weight_quantization_22_b200 import gq as G
+    out, ln, cw, info, ws = G.gq_huffman_encode(codes_dev, stream_words)
+    assert G.gq_workspace_status(ws)[0] == 0
+    codes = codes_dev.cpu().numpy().astype(np.int64).ravel()
+    lo, K, total, maxlen = (int(v) for v in info.cpu().numpy())
+    assert lo == codes.min() and K == codes.max() - lo + 1
+    sym = codes - lo
+    counts = np.bincount(sym, minlength=K)
+    ln = ln.cpu().numpy().astype(np.int64)[:K]
+    assert total == int(np.dot(counts, O.huffman_lengths(counts)))
+    assert total == int(np.dot(counts, ln)) and maxlen == ln.max()
+    used = counts > 0
+    assert np.all((ln > 0) == used)
+    if used.sum() > 1:
+        assert abs(np.sum(2.0 ** -ln[used]) - 1.0) < 1e-12
+    assert np.array_equal(cw.cpu().numpy().view(np.uint64)[:K], O.canonical_codewords(ln))
+    ref, nbits = O.huffman_encode(sym, ln)
+    got = out.cpu().numpy().view(np.uint64)
+    assert nbits == total
+    assert np.array_equal(got[:len(ref)], ref) and not got[len(ref):].any()
+    return total
+
+
+@pytest.mark.parametrize("count,spread", [(100003, 3.0), (1, 1.0), (5000, 0.0), (70000, 15.0)])
+def test_huffman_encoder_against_oracle(count, spread):
+    """Ragged tiles (100003 codes), a single code, a single symbol (5000 equal codes), a wide
+    heavy-tailed alphabet with negative values."""
+    rng = np.random.default_rng(count)
+    vals = np.rint(rng.standard_t(3, count) * spread).astype(np.int32) - 7
+    _huffman_check(torch.from_numpy(vals).cuda())
+
+
+def test_huffman_encoder_reports_span_and_stream_errors():
+    """More than 4096 values spanned -> GQ_ERR_UNSUPPORTED; a stream too small for the total ->
+    GQ_ERR_WORKSPACE; nothing is encoded (the stream stays zero)."""
+    from post_weight_quantization_22_b200 import gq as G
+    wide = torch.tensor([0, 5000, 3, 3], dtype=torch.int32, device="cuda")
+    out, *_, info, ws = G.gq_huffman_encode(wide)
+    assert G.gq_workspace_status(ws)[0] == 4
+    codes = torch.from_numpy(np.arange(100000, dtype=np.int32) % 64).cuda()
+    out, *_, info, ws = G.gq_huffman_encode(codes, stream_words=10)
+    assert G.gq_workspace_status(ws)[0] == 7
+    assert int(info[2]) == 600000 and not out.any()
+
+
+def test_unbounded_lattice_codes_and_huffman_rate():
+    """Unconstrained lattice (HPTQ reading): per-row min-max step, zero point 0, int32 codes
+    without a range; codes / steps / losses against the oracle, then the device's Huffman rate
+    of those codes (bits per weight) against the oracle's on its own codes."""
+    W, X, spec = synth.workload("q_proj_4096x4096", m=128, n=520, T=700)
+    g = run_gpu(W, X, bits=4, clip="unbounded")
+    assert g["status"] == (0, 0)
+    o = _oracle(W, X, 4, 0, False, "unbounded")
+    assert (g["zeros"] == 0).all()
+    _compare(g, o, W, 4, 0)
+    total = _huffman_check(g["codes_dev"])
+    rate = total / g["codes"].size
+    assert abs(rate - o["rate"]) <= 0.01 * o["rate"]
+    assert g["loss"][1] <= g["loss"][2]
+
+
+def test_zsic_unbounded_lattice_with_huffman():
+    """ZSIC as the pages state it: per-column spacing kappa_j on an unconstrained lattice,
+    entropy-coded; against the oracle."""
+    W, X, spec = synth.workload("q_proj_4096x4096", m=128, n=520, T=700)
+    g = run_gpu(W, X, bits=4, clip="unbounded", spacing="zsic")
+    assert g["status"] == (0, 0)
+    o = _oracle(W, X, 4, 0, False, "unbounded", spacing="zsic")
+    _compare(g, o, W, 4, 0)
+    total = _huffman_check(g["codes_dev"])
+    assert abs(total / g["codes"].size - o["rate"]) <= 0.01 * o["rate"]
+    assert g["loss"][1] <= g["loss"][2]
 
 
 def test_given_order_clipfree_ladder():
