@@ -2,15 +2,18 @@
 //
 // Sources: "The Geometry of LLM Quantization: GPTQ as Babai's Nearest Plane Algorithm",
 // section 2.2 (GPTQ's error propagation is the nearest-plane step; back to front it is Babai),
-// section 2.3 (no-clipping setting; Theorem 5 bound (1/4) sum s^2 D_jj); "RDQ: Residual
-// Distribution Quantization", setup (group-128 asymmetric integer format).
+// section 2.3 (no-clipping setting; Theorem 5 bound (1/4) sum s^2 D_jj; the order's role),
+// section 3 (HPTQ: one unconstrained integer grid); "WaterSIC", section 2 (ZSIC spacing);
+// "RDQ: Residual Distribution Quantization", setup (group-128 asymmetric integer format).
 //
 // Work layout: the weights are copied once into an fp32 work matrix Wf (rows x n) in the
-// processing order (columns reversed for the last-to-first variant, dead columns zeroed).  Per
-// 128-column block: `colloop` runs the column recursion for 64 rows per CTA (16 per warp, in
-// 8-column tiles with fp64 tensor-core updates between tiles), keeping the block's part of U
-// in shared memory; the tensor-core lazy update (gq_lazy_tc.cu) then applies
-// W[:, j+128:] -= E U[j:j+128, j+128:] to the rest of the work matrix.
+// processing order (natural, reversed, or a permutation; dead columns zeroed).  Per 128-column
+// block: `colloop` runs the column recursion for 32 rows per CTA (8 per warp, in 8-column
+// tiles with fp64 tensor-core updates between tiles), keeping the block's part of U in shared
+// memory; the tensor-core lazy update (gq_lazy_tc.cu) then applies
+// W[:, j+128:] -= E U[j:j+128, j+128:] to the rest of the work matrix.  Grids: per row or per
+// group (min-max), clip-free with a per-row ladder, the unconstrained lattice s Z (int32 codes),
+// and ZSIC per-column spacing on a per-row grid.
 #include "gq_internal.cuh"
 #include "gq_tc.cuh"
 
