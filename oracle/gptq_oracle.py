@@ -47,6 +47,8 @@ __all__ = [
     "clipfree_grid",
     "gptq_columns",
     "babai_sic_reverse",
+    "ssqr_columns",
+    "ssqr_search",
     "zsic_spacing",
     "pack_codes",
     "huffman_lengths",
@@ -285,6 +287,72 @@ def gptq_columns(W, U, bits: int, group: int = 0, clip: bool = True, alpha=None,
         Q[:, j] = q
         E[:, j] = e
     return dict(codes=codes, scales=scales, zeros=zeros, Q=Q, e=E)
+
+
+def ssqr_columns(W, U, bits: int, alpha):
+    """GPTQ with SSQR outliers ([GEOM] section 3, SSQR: weights that do not fit the low-bit
+    grid are kept in full precision as sparse floating-point values).
+
+    reading: the clip-free centred grid of ``clipfree_grid`` with the per-row factor ``alpha``;
+    an entry whose code falls outside [0, 2^b - 1] is an outlier: it keeps its current
+    (error-fed) value exactly, q = w, so its error e is 0 and nothing is fed forward.
+    Returns dict(codes (outliers 0), outlier (bool mask), Q, e, scales, zeros).
+    """
+    w = _f64(W).copy()
+    u = _f64(U)
+    m, n = w.shape
+    maxq = 2 ** bits - 1
+    s, z = clipfree_grid(w, bits, alpha)
+    codes = np.zeros((m, n), dtype=np.int64)
+    mask = np.zeros((m, n), dtype=bool)
+    Q = np.zeros((m, n))
+    E = np.zeros((m, n))
+    for j in range(n):
+        c = np.rint(w[:, j] / s) + z
+        out = (c < 0) | (c > maxq)
+        q = np.where(out, w[:, j], s * (c - z))
+        e = (w[:, j] - q) / u[j, j]
+        w[:, j + 1:] -= np.outer(e, u[j, j + 1:])
+        codes[:, j] = np.where(out, 0, c).astype(np.int64)
+        mask[:, j] = out
+        Q[:, j] = q
+        E[:, j] = e
+    return dict(codes=codes, outlier=mask, Q=Q, e=E, scales=s[:, None], zeros=z[:, None])
+
+
+def ssqr_search(W, U, bits: int, density: float, steps: int = 20, max_doublings: int = 12):
+    """Per-row scale search of SSQR ([GEOM] section 3: a binary search adjusts the scale to
+    meet a target outlier density).
+
+    reading: the smallest factor alpha (finest grid) whose outlier count is at most
+    density * n.  alpha starts at 1 and doubles until the row is feasible (at most
+    ``max_doublings`` times); then ``steps`` bisection steps in log2(alpha) between the last
+    infeasible value (alpha / 2, or 2^-8 when alpha = 1 is already feasible) and the feasible
+    one.  The result is always a feasible alpha.  Returns (result of ``ssqr_columns`` at the
+    chosen alphas, alphas, the last infeasible log2 alphas).
+    """
+    w = _f64(W)
+    m, n = w.shape
+    limit = np.floor(density * n + 1e-9)
+    hi = np.zeros(m)                       # log2 alpha, feasible once the doubling stops
+    feas = ssqr_columns(w, U, bits, 2.0 ** hi)["outlier"].sum(axis=1) <= limit
+    lo = np.where(feas, -8.0, np.nan)
+    for _ in range(max_doublings):
+        if feas.all():
+            break
+        bad = ~feas
+        lo[bad] = hi[bad]
+        hi[bad] += 1.0
+        feas = ssqr_columns(w, U, bits, 2.0 ** hi)["outlier"].sum(axis=1) <= limit
+    if not feas.all():
+        raise ValueError("some rows exceed the outlier density even at the widest grid")
+    for _ in range(steps):
+        mid = 0.5 * (lo + hi)
+        ok = ssqr_columns(w, U, bits, 2.0 ** mid)["outlier"].sum(axis=1) <= limit
+        hi = np.where(ok, mid, hi)
+        lo = np.where(ok, lo, mid)
+    alpha = 2.0 ** hi
+    return ssqr_columns(w, U, bits, alpha), alpha, lo
 
 
 def babai_sic_reverse(W, L, bits: int, clip: bool = False, alpha=None):

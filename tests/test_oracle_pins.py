@@ -612,3 +612,46 @@ def test_unbounded_lattice_on_diagonal_hessian_is_rounding():
     np.testing.assert_array_equal(res["codes"], np.rint(w / s[:, None]))
     assert (res["zeros"] == 0).all()
     assert res["rate"] > 0
+
+
+# --------------------------------------------------------------------------------------------
+# SSQR: full-precision outliers and the scale search (GEOM section 3)
+# --------------------------------------------------------------------------------------------
+
+def test_ssqr_outliers_are_exact_and_feed_nothing_forward():
+    """An outlier keeps its error-fed value exactly (e = 0); the normals' codes are in range and
+    their dequantized values lie on the row grid; with a tiny alpha almost every entry is an
+    outlier and Q equals W (no error anywhere)."""
+    w, x = _rand_problem(80, 16, 12, seed=221)
+    hd, _ = O.dampen(O.hessian(x), 0.01)
+    U = O.hinv_upper_factor(hd)
+    r = O.ssqr_columns(w, U, 3, np.full(12, 0.3))
+    assert r["outlier"].any() and (~r["outlier"]).any()
+    assert np.all(r["e"][r["outlier"]] == 0.0)
+    c = r["codes"]
+    assert c[~r["outlier"]].min() >= 0 and c[~r["outlier"]].max() <= 7
+    s, z = r["scales"][:, 0], r["zeros"][:, 0]
+    grid = s[:, None] * (c - z[:, None])
+    np.testing.assert_allclose(r["Q"][~r["outlier"]], grid[~r["outlier"]], rtol=0, atol=1e-15)
+    tiny = O.ssqr_columns(w, U, 3, np.full(12, 1e-9))
+    assert tiny["outlier"].all() and np.array_equal(tiny["Q"], w)
+
+
+@pytest.mark.parametrize("density", [0.0, 0.05, 0.2])
+def test_ssqr_search_is_a_bisection_of_feasibility(density):
+    """The chosen alpha is feasible (at most density * n outliers per row) and the last
+    infeasible probe lies within the bisection resolution below it, so no finer grid within
+    that resolution meets the density; with density 0 no row has an outlier."""
+    w, x = _rand_problem(100, 20, 10, seed=223)
+    hd, _ = O.dampen(O.hessian(x), 0.01)
+    U = O.hinv_upper_factor(hd)
+    steps = 16
+    r, alpha, lo = O.ssqr_search(w, U, 3, density, steps=steps)
+    limit = np.floor(density * 20 + 1e-9)
+    assert np.all(r["outlier"].sum(axis=1) <= limit)
+    hi = np.log2(alpha)
+    assert np.all(hi - lo <= 9.0 / 2 ** steps + 1e-12)
+    probe = O.ssqr_columns(w, U, 3, 2.0 ** lo)["outlier"].sum(axis=1)
+    assert np.all(probe > limit)
+    if density == 0.0:
+        assert not r["outlier"].any()
