@@ -80,3 +80,21 @@ def test_ordered_entry_points_reject_bad_arguments_without_gpu():
     c2 = G.QuantCfg(bits=4, reverse=True).c()
     assert L.gq_quantize_layer_ordered(fake, 0, 4, 16, fake, None, None, ctypes.byref(c2), fake,
                                        fake, fake, fake, fake, fake, 1 << 20, None) == 1
+
+
+def test_quant_cfg_binding_matches_the_header_struct():
+    """The ctypes mirror of gq_quant_cfg has the header's fields, in order, with matching types;
+    the Python settings map to the C values (clip: clamp 1 / clip-free 0 / lattice 2;
+    spacing: uniform 0 / ZSIC 1)."""
+    from post_weight_quantization_22_b200 import gq as G
+    text = open(os.path.join(ROOT, "include", "gq.h")).read()
+    body = re.search(r"typedef struct \{(.*?)\} gq_quant_cfg;", text, flags=re.S).group(1)
+    body = re.sub(r"/\*.*?\*/", "", body, flags=re.S)
+    fields = re.findall(r"\b(int|float)\s+(\w+)\s*;", body)
+    assert [n for _, n in fields] == [n for n, _ in G._Cfg._fields_]
+    ctype = {"int": ctypes.c_int, "float": ctypes.c_float}
+    assert [ctype[t] for t, _ in fields] == [t for _, t in G._Cfg._fields_]
+    c = G.QuantCfg(bits=3, clip="unbounded", spacing="zsic").c()
+    assert (c.bits, c.clip, c.spacing) == (3, 2, 1)
+    c = G.QuantCfg(bits=4, clip=False).c()
+    assert (c.clip, c.spacing) == (0, 0)
