@@ -372,8 +372,10 @@ def run_reference(args):
 
 
 def run_case(args):
-    """One untimed invocation for profilers: `layer` (the q_proj recipe at --case-n) or `factor`
-    (gq_prepare_hinv on a seeded SPD fp64 H of width --case-n)."""
+    """One invocation for profilers: `layer` (the q_proj recipe at --case-n), `factor`
+    (gq_prepare_hinv on a seeded SPD fp64 H of width --case-n), or `huffman` (the Huffman
+    encoder on the unconstrained-lattice codes of that layer, event-timed, one JSON line with
+    its HBM roofline)."""
     from post_weight_quantization_22_b200 import gq as G
     from post_weight_quantization_22_b200 import synth
     from post_weight_quantization_22_b200.pipeline import LayerQuantizer
@@ -387,13 +389,42 @@ def run_case(args):
         lq.run(W.cuda(), X.cuda())
         torch.cuda.synchronize()
         print("status", lq.status())
-    else:
+    elif args.case == "factor":
         g = torch.Generator(device="cuda").manual_seed(0)
         X = torch.randn(n + 64, n, dtype=torch.float64, device="cuda", generator=g)
         H = 2 * (X.T @ X)
         U, dead, delta, ws = G.gq_prepare_hinv(H, 0.01)
         torch.cuda.synchronize()
         print("status", G.gq_workspace_status(ws))
+    else:  # huffman: encode the unconstrained-lattice codes of the q_proj recipe, timed
+        W, X, spec = synth.workload(DEFAULT_WORKLOAD, m=n, n=n, T=n)
+        cfg = G.QuantCfg(bits=spec["bits"], clip="unbounded")
+        lq = LayerQuantizer(n, n, cfg, device="cuda")
+        lq.run(W.cuda(), X.cuda())
+        codes = lq.codes
+        out, ln, cw, info, ws = G.gq_huffman_encode(codes)
+        bufs = dict(ws=ws, out=out, lengths=ln, cw=cw, info=info)
+        for _ in range(3):
+            G.gq_huffman_encode(codes, **bufs)
+        torch.cuda.synchronize()
+        reps = 20
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(reps):
+            G.gq_huffman_encode(codes, **bufs)
+        b.record()
+        torch.cuda.synchronize()
+        ms = a.elapsed_time(b) / reps
+        total_bits = int(info[2])
+        # algorithmic bytes: the codes read twice (histogram, encode; the range and tile-sum
+        # passes read them again but a plain encoder needs two) and the stream written once
+        nbytes = 2 * 4 * codes.numel() + total_bits / 8
+        peaks, kind = measured_peaks()
+        gbs = nbytes / (ms * 1e-3) / 1e9
+        print(json.dumps({"case": "huffman", "codes": codes.numel(), "bits_per_weight":
+                          total_bits / codes.numel(), "ms": ms, "achieved_gbs": gbs,
+                          "peak_gbs": peaks["hbm_gbs"], "frac": gbs / peaks["hbm_gbs"],
+                          "peak_kind": kind, "status": G.gq_workspace_status(ws)[0]}))
 
 
 def main(argv=None):
@@ -408,7 +439,7 @@ def main(argv=None):
                     help="process the columns in act-order (descending Hessian diagonal)")
     ap.add_argument("--cpu-rows", type=int, default=256)
     ap.add_argument("--ref-rows", type=int, default=32)
-    ap.add_argument("--case", choices=["layer", "factor"], default=None,
+    ap.add_argument("--case", choices=["layer", "factor", "huffman"], default=None,
                     help="run one untimed invocation (for profilers) and exit")
     ap.add_argument("--case-n", type=int, default=2048)
     args = ap.parse_args(argv)

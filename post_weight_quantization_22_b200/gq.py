@@ -294,19 +294,24 @@ def gq_zsic_spacing(U: torch.Tensor, kappa=None, stream=None) -> torch.Tensor:
 
 
 def gq_huffman_encode(codes: torch.Tensor, stream_words: int | None = None, ws=None,
-                      stream=None):
+                      stream=None, out=None, lengths=None, cw=None, info=None):
     """Canonical Huffman coding of int32 codes on the device.  Returns (stream uint64 words as
     an int64 tensor, lengths uint8[4096], codewords int64[4096], info int64[4]
-    = [min value, symbols spanned, total bits, longest codeword], workspace)."""
+    = [min value, symbols spanned, total bits, longest codeword], workspace); pass the
+    returned buffers back in to reuse them."""
     if not codes.is_cuda or codes.dtype != torch.int32 or not codes.is_contiguous():
         raise ValueError("codes: expected a contiguous cuda int32 tensor")
     count = codes.numel()
     dev = codes.device
-    words = count if stream_words is None else int(stream_words)
-    out = torch.empty(max(words, 1), dtype=torch.int64, device=dev)
-    lengths = torch.empty(4096, dtype=torch.uint8, device=dev)
-    cw = torch.empty(4096, dtype=torch.int64, device=dev)
-    info = torch.empty(4, dtype=torch.int64, device=dev)
+    words = (count if stream_words is None else int(stream_words)) if out is None else out.numel()
+    out = torch.empty(max(words, 1), dtype=torch.int64, device=dev) if out is None else out
+    lengths = torch.empty(4096, dtype=torch.uint8, device=dev) if lengths is None else lengths
+    cw = torch.empty(4096, dtype=torch.int64, device=dev) if cw is None else cw
+    info = torch.empty(4, dtype=torch.int64, device=dev) if info is None else info
+    _need(out, torch.int64, (out.numel(),), "out")
+    _need(lengths, torch.uint8, (4096,), "lengths")
+    _need(cw, torch.int64, (4096,), "cw")
+    _need(info, torch.int64, (4,), "info")
     ws = workspace(int(LIB.gq_huffman_workspace_size(count)), dev) if ws is None else ws
     _check(LIB.gq_huffman_encode(_ptr(codes), count, _ptr(out), out.numel(), _ptr(lengths),
                                  _ptr(cw), _ptr(info), _ptr(ws), ws.numel(), _stream(stream)),
