@@ -28,9 +28,9 @@ Sources, by page title and section:
 The pages do not print GPTQ's update, its min-max quantizer or its Cholesky trick; where they
 are silent the plainest reading is taken and flagged ``reading:`` below.
 
-Pins (tests/test_oracle_pins.py, tests/test_oracle_golden.py): every public function here is
-pinned against a closed form, a hand-derived example, an independent textbook construction
-(Gram-Schmidt Babai, brute-force CVP) or an invariant.  No function is "parity unpinned".
+Pins (tests/test_oracle_pins.py, with tests/golden/gptq_two_column_hand.json): every public
+function here is pinned against a closed form, a hand-derived example, an independent textbook
+construction (Gram-Schmidt Babai, brute-force CVP) or an invariant.  No function is "parity unpinned".
 """
 from __future__ import annotations
 

@@ -134,6 +134,30 @@ def test_clipfree_grid_reduces_to_minmax_at_alpha_one_and_widens():
     assert np.all(np.rint(lo / s3) + z3 >= 0) and np.all(np.rint(hi / s3) + z3 <= 7)
 
 
+def test_clipfree_grid_centred_zero_point_hand_values():
+    """The clip-free grid centres the row's range [lo, hi] on the code range: with the widened
+    step s = alpha (hi - lo) / (2^b - 1), z = rint((2^b - 1)/2 - (hi + lo)/(2 s)) ("The Geometry
+    of LLM Quantization", section 2.3, no-clipping setting: one uniform grid per row, wide
+    enough that nothing clips).  Rows a, b and e are chosen so that the uncentred zero point
+    rint(-lo / s) differs from the centred one."""
+    w2 = np.array([[0.25, 1.0],     # a: lo 0,  hi 1
+                   [-1.0, -0.5],    # b: lo -1, hi 0
+                   [-0.3, 0.5],     # c: lo -0.3, hi 0.5
+                   [0.0, 0.0]])     # d: flat row -> [lo, hi] = [-1, 1]
+    alpha = np.array([2.0, 1.25, 2.0, 1.25])
+    s, z = O.clipfree_grid(w2, 2, alpha)
+    # a: s = 2 * 1 / 3;       z = rint(1.5 - 1 / (4/3))       = rint(0.75)   = 1  (rint(-lo/s) = 0)
+    # b: s = 1.25 * 1 / 3;    z = rint(1.5 + 1 / (2.5/3))     = rint(2.7)    = 3  (rint(2.4) = 2)
+    # c: s = 2 * 0.8 / 3;     z = rint(1.5 - 0.2 / (3.2/3))   = rint(1.3125) = 1
+    # d: s = 1.25 * 2 / 3;    z = rint(1.5 - 0)               = 2 (half to even)
+    np.testing.assert_allclose(s, [2.0 / 3, 1.25 / 3, 1.6 / 3, 2.5 / 3], rtol=1e-15)
+    assert z.tolist() == [1.0, 3.0, 1.0, 2.0]
+    # e: 3 bits, lo 0, hi 0.7, alpha 2: s = 1.4 / 7 = 0.2; z = rint(3.5 - 0.7 / 0.4) = rint(1.75) = 2
+    s3, z3 = O.clipfree_grid(np.array([[0.1, 0.7]]), 3, np.array([2.0]))
+    np.testing.assert_allclose(s3, [0.2], rtol=1e-15)
+    assert z3.tolist() == [2.0]
+
+
 # --------------------------------------------------------------------------------------------
 # column loop: special cases, independent Babai, brute force, invariants
 # --------------------------------------------------------------------------------------------
@@ -360,6 +384,43 @@ def test_quantize_layer_clipfree_ladder_fits_every_row():
     assert out["ladder_rounds"] >= 1          # 2-bit unclamped rounding overflows at alpha = 1
     assert np.all(out["alpha"] >= 1.0)
     assert out["loss_damped"] <= out["bound"]
+
+
+def test_quantize_layer_clipfree_ladder_hand_trace():
+    """The scale ladder of the clip-free variant, traced by hand (reading of "per-row step s set
+    so that no entry needs clipping", with the scale search of "The Geometry of LLM
+    Quantization", section 3, SSQR, as the mechanism): only the rows whose codes leave
+    [0, 2^b - 1] are rerun, each time with alpha multiplied by 1.25; a row that fits keeps
+    alpha = 1.
+
+    H = [[5, 2], [2, 1]] (det 1, no damping) gives H^-1 = [[1, -2], [-2, 5]] and the upper
+    factor U = [[1, -2], [0, 1]]: column 1 receives w1 - e0 U01 = w1 + 2 e0.  2 bits, maxq 3.
+
+    row 0, w = [0.45, 1.0], lo 0, hi 1:
+      alpha 1:    s = 1/3,  z = rint(1.5 - 1.5) = 0; c0 = rint(1.35) = 1, e0 = 0.45 - 1/3
+                  = 0.11667; w1' = 1.23333, 3.7 -> c1 = 4 > 3: overflow
+      alpha 1.25: s = 5/12, z = rint(1.5 - 1.2) = 0; c0 = rint(1.08) = 1, e0 = 0.03333;
+                  w1' = 1.06667, 2.56 -> c1 = 3: fits
+    row 1, w = [-0.3, 0.1], lo -0.3, hi 0.1:
+      alpha 1:    s = 0.4/3, z = rint(1.5 + 0.75) = 2; c0 = rint(-2.25) + 2 = 0, e0 = -0.03333;
+                  w1' = 0.03333, 0.25 -> c1 = 0 + 2 = 2: fits
+    row 2, w = [-0.35, 1.0], lo -0.35, hi 1, range 1.35:
+      alpha 1:      s = 0.45,     z = rint(1.5 - 0.72222) = 1; c0 = rint(-0.77778) + 1 = 0,
+                    e0 = 0.1;   w1' = 1.2,   rint(2.66667) + 1 = 4: overflow
+      alpha 1.25:   s = 0.5625,   z = rint(1.5 - 0.57778) = 1; c0 = rint(-0.62222) + 1 = 0,
+                    e0 = 0.2125; w1' = 1.425, rint(2.53333) + 1 = 4: overflow
+      alpha 1.5625: s = 0.703125, z = rint(1.5 - 0.46222) = 1; c0 = rint(-0.49778) + 1 = 1,
+                    q0 = 0, e0 = -0.35; w1' = 0.3, rint(0.42667) + 1 = 1: fits
+    """
+    H = np.array([[5.0, 2.0], [2.0, 1.0]])
+    W = np.array([[0.45, 1.0], [-0.3, 0.1], [-0.35, 1.0]])
+    np.testing.assert_allclose(O.hinv_upper_factor(H), [[1.0, -2.0], [0.0, 1.0]], atol=1e-14)
+    out = O.quantize_layer(W, None, bits=2, clip=False, damp=0.0, H=H)
+    np.testing.assert_allclose(out["alpha"], [1.25, 1.0, 1.5625], rtol=1e-15)
+    assert out["ladder_rounds"] == 2
+    assert out["codes"].tolist() == [[1, 3], [0, 2], [1, 1]]
+    assert out["zeros"][:, 0].tolist() == [0.0, 2.0, 1.0]
+    np.testing.assert_allclose(out["scales"][:, 0], [1.25 / 3, 0.4 / 3, 0.703125], rtol=1e-14)
 
 
 def test_quantize_layer_dead_feature_and_loss_bookkeeping():
