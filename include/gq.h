@@ -105,7 +105,8 @@ size_t gq_hessian_workspace_size(int64_t T, int64_t n);
  *              adds 2 X^T X (streaming over token chunks).  Both triangles are written (H stays
  *              exactly symmetric).
  *   d_X     T x n, row-major (tokens x features), dtype x_dtype (bf16 or fp32), device.
- *   T, n    T >= 0 (T = 0 is a no-op), 1 <= n <= 32768.
+ *   T, n    T >= 0 (T = 0: H = 0 when accumulate = 0, H unchanged when accumulate = 1),
+ *           1 <= n <= 32768.
  *   d_ws    workspace of at least gq_hessian_workspace_size(T, n) bytes (256-byte aligned).
  *
  * Precision: the products are formed exactly (each value as four 7-bit digits against a
@@ -162,8 +163,12 @@ gq_status gq_prepare_hinv(const double* d_H, int64_t n, double damp, int reverse
  *   d_status   optional (may be NULL) device int, written on `stream` with the device-side
  *              status of this call (GQ_OK, or GQ_ERR_NOT_PD for a non-positive pivot).
  *
- * The first call on a device looks up the scratch array's device address (once per device);
- * make that first call outside any stream capture.  Every call on a device shares the one
+ * The first call on a device looks up the scratch array's device address (once per device).
+ * With CUDA's lazy module loading (the default) that lookup is also when the driver loads this
+ * part of the library and reserves the ~17 MB array on that device; and the first call from
+ * each host thread creates the library's private streams and events for that thread and
+ * device.  So make the first call per device, and per calling thread, outside any stream
+ * capture and at a point where that one-time setup is acceptable.  Every call on a device shares the one
  * scratch array and leaves its contents behind; each call clears what it needs cleared.  Two
  * calls whose work overlaps on the GPU (different streams, no ordering between them) race on
  * the scratch and give undefined results: order them on one stream or with events.

@@ -199,6 +199,12 @@ def gq_prepare_hinv_static(H: torch.Tensor, damp: float = 0.01, reverse: bool = 
     delta = torch.empty(1, dtype=torch.float64, device=dev) if delta is None else delta
     status = torch.empty(1, dtype=torch.int32, device=dev) if status is None else status
     _need(U, torch.float32, (n, n), "U")
+    _need(dead, torch.uint8, (n,), "dead")
+    _need(delta, torch.float64, (1,), "delta")
+    _need(status, torch.int32, (1,), "status")
+    for t, name in ((U, "U"), (dead, "dead"), (delta, "delta"), (status, "status")):
+        if t.device != dev:
+            raise ValueError(f"{name}: on {t.device}, H is on {dev}")
     _check(LIB.gq_prepare_hinv_static(_ptr(H), n, float(damp), int(bool(reverse)), _ptr(U),
                                       _ptr(dead), _ptr(delta), _ptr(status), _stream(stream)),
            "gq_prepare_hinv_static")

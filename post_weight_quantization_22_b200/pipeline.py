@@ -52,6 +52,8 @@ class LayerQuantizer:
         self.perm = torch.arange(n, dtype=torch.int32, device=dev) if order else None
 
     def hessian(self, X: torch.Tensor, reset: bool = True, stream=None):
+        if X.shape[0] < 1 and not reset:
+            return
         if X.shape[0] > self.max_tokens:
             raise ValueError(f"{X.shape[0]} tokens exceed this quantizer's {self.max_tokens}")
         G.gq_hessian_accumulate(self.H, X, accumulate=not reset, ws=self.ws_hess, stream=stream)
@@ -104,6 +106,8 @@ class LayerQuantizer:
             self._Xd = torch.empty(X_host.shape, dtype=X_host.dtype, device=dev)
         cs = self._copy_stream
         T = X_host.shape[0]
+        if T < 1:
+            raise ValueError("run_host needs at least one calibration token")
         k = max(1, min(int(x_chunks), T))
         bounds = [(T * i) // k for i in range(k + 1)]
         cs.wait_stream(cur)  # the previous call's readers of the device copies are done

@@ -10,6 +10,7 @@ import numpy as np
 import pytest
 import torch
 
+from oracle import gptq_oracle as O
 from post_weight_quantization_22_b200 import synth
 from tests.gpu_helpers import rel_fro
 
@@ -39,6 +40,13 @@ def test_static_scratch_matches_workspace_call_twice_in_a_row():
         assert rel_fro(np.triu(U2.cpu().numpy()), np.triu(U1.cpu().numpy())) <= U_REL
         assert torch.equal(dead1, dead2)
         assert abs(float(delta2.item()) - float(delta1.item())) <= 1e-12 * abs(float(delta1.item()))
+        # and against the fp64 oracle's factor of the damped Hessian in the processing order
+        # (last to first when reverse: the factor of the column-reversed matrix)
+        hfix, _, _ = O.fix_dead_features(H.cpu().numpy(), np.zeros((1, n)))
+        hd, _ = O.dampen(hfix, 0.01)
+        if reverse:
+            hd = hd[::-1, ::-1]
+        assert rel_fro(np.triu(U2.cpu().numpy()), O.hinv_upper_factor(hd)) <= U_REL
 
 
 def test_static_scratch_reports_status_and_rejects_large_n():
