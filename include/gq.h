@@ -291,6 +291,19 @@ gq_status gq_huffman_encode(const int32_t* d_codes, int64_t count, uint64_t* d_s
                             int64_t* d_info, void* d_ws, size_t ws_bytes, gq_stream_t stream);
 
 /*
+ * Test setting of the bounded device waits, for tests of the timeout path (process-wide, read
+ * when a call is enqueued; default off).  poll_limit > 0 replaces the poll budget of the
+ * factor's per-pivot waits in gq_prepare_hinv(_ordered) (0 restores the default of about 2^26
+ * polls, well over a second); withhold_arrival = 1 makes the factor's leaf kernel withhold one
+ * thread's first barrier arrival, so that every wait of that phase runs out: the kernel records
+ * GQ_ERR_TIMEOUT in the workspace and returns (no copy or tensor-core operation is in flight in
+ * that kernel), and the call's U is undefined.  withhold_arrival must be 0 or 1.  The setting is
+ * part of the key under which a call's launch sequence is cached, so calls made under it never
+ * replay as clean calls.
+ */
+gq_status gq_debug_wait_test(uint32_t poll_limit, int withhold_arrival);
+
+/*
  * Synchronize `stream` and return the device-side status recorded in a workspace by the last
  * gq_prepare_hinv / gq_quantize_layer that used it (GQ_OK if none), then clear it.
  * For gq_quantize_layer's clip-free ladder, h_ladder_rounds (may be NULL) receives the number

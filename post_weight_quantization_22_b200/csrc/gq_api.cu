@@ -1,5 +1,6 @@
 // C ABI entry points of libgq: argument validation, per-device setup, dispatch.
 #include "gq_internal.cuh"
+#include "gq_tc.cuh"
 
 #include <atomic>
 #include <cstring>
@@ -12,6 +13,13 @@ using namespace gq;
 namespace gq {
 static std::atomic<unsigned long long> g_launches{0};
 void count_launches(long k) { g_launches.fetch_add((unsigned long long)k, std::memory_order_relaxed); }
+
+static std::atomic<uint32_t> g_wait_polls{0};  // 0: the default budget
+static std::atomic<int> g_wait_withhold{0};
+WaitTest wait_test() {
+  const uint32_t p = g_wait_polls.load();
+  return WaitTest{p ? p : tc::kDefaultPolls, g_wait_withhold.load()};
+}
 }  // namespace gq
 
 namespace {
@@ -177,8 +185,9 @@ gq_status gq_prepare_hinv(const double* d_H, int64_t n, double damp, int reverse
                    cudaSuccess
                ? GQ_OK : GQ_ERR_CUDA;
   };
+  const WaitTest wt = wait_test();
   return run_graphed({1, P(d_H), (uint64_t)n, bits_of(damp), (uint64_t)reverse, P(d_U),
-                      P(d_dead), P(d_delta), P(d_ws)},
+                      P(d_dead), P(d_delta), P(d_ws), wt.polls, (uint64_t)wt.withhold},
                      (cudaStream_t)stream, enqueue);
 }
 
@@ -199,8 +208,9 @@ gq_status gq_prepare_hinv_ordered(const double* d_H, int64_t n, double damp, gq_
     return launch_prepare(d_H, n, damp, o, d_perm, d_U, d_dead, d_delta, d_ws, s) == cudaSuccess
                ? GQ_OK : GQ_ERR_CUDA;
   };
+  const WaitTest wt = wait_test();
   return run_graphed({4, P(d_H), (uint64_t)n, bits_of(damp), (uint64_t)o, P(d_perm), P(d_U),
-                      P(d_dead), P(d_delta), P(d_ws)},
+                      P(d_dead), P(d_delta), P(d_ws), wt.polls, (uint64_t)wt.withhold},
                      (cudaStream_t)stream, enqueue);
 }
 
@@ -314,6 +324,13 @@ gq_status gq_huffman_encode(const int32_t* d_codes, int64_t count, uint64_t* d_s
   return run_graphed({5, P(d_codes), (uint64_t)count, P(d_stream), (uint64_t)stream_words,
                       P(d_lengths), P(d_codewords), P(d_info), P(d_ws)},
                      (cudaStream_t)stream, enqueue);
+}
+
+gq_status gq_debug_wait_test(uint32_t poll_limit, int withhold_arrival) {
+  if (withhold_arrival != 0 && withhold_arrival != 1) return GQ_ERR_INVALID_ARG;
+  gq::g_wait_polls.store(poll_limit);
+  gq::g_wait_withhold.store(withhold_arrival);
+  return GQ_OK;
 }
 
 gq_status gq_workspace_status(void* d_ws, int* h_ladder_rounds, gq_stream_t stream) {

@@ -186,7 +186,8 @@ __device__ __forceinline__ double recip_newton(double p) {
 // ---------------------------------------------------------------------------------------
 __global__ void __launch_bounds__(256, 1) potrf_panel_kernel(double* M, int64_t ldm, int64_t n,
                                                              int64_t c0, int w, double* Dinv,
-                                                             WsHeader* hdr) {
+                                                             WsHeader* hdr, uint32_t polls,
+                                                             int withhold) {
   extern __shared__ __align__(16) double pn_smem[];
   __shared__ __align__(16) double colbuf[2][kNB];
   __shared__ __align__(16) double rowbuf[2][kNB];
@@ -220,7 +221,9 @@ __global__ void __launch_bounds__(256, 1) potrf_panel_kernel(double* M, int64_t 
 #pragma unroll
     for (int j = 0; j < 4; ++j) rowbuf[0][4 * b + j] = av[0][j];
   }
-  tc::mbar_arrive(&bar);
+  // (test setting: thread 0 withholds this arrival, so phase 0 never completes and every wait
+  // below runs out after `polls` polls)
+  if (!(withhold && tid == 0)) tc::mbar_arrive(&bar);
   bool live = true;
 #pragma unroll 1
   for (int c4 = 0; c4 < kNB / 4 && live; ++c4) {
@@ -228,7 +231,7 @@ __global__ void __launch_bounds__(256, 1) potrf_panel_kernel(double* M, int64_t 
     for (int cc = 0; cc < 4; ++cc) {
       const int c = 4 * c4 + cc;
       if (!live || c == kNB - 1) break;
-      if (!tc::mbar_wait(&bar, c & 1)) {  // pivot c published
+      if (!tc::mbar_wait_polls(&bar, c & 1, polls)) {  // pivot c published
         record_status(hdr, GQ_ERR_TIMEOUT);
         live = false;
         break;
@@ -524,6 +527,7 @@ cudaError_t launch_prepare(const double* H, int64_t n, double damp, int order, i
   GQ_TRY(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
   PrepStreams* ps = nullptr;
   GQ_TRY(prep_streams(&ps));
+  const WaitTest wt = wait_test();
   cudaStream_t s = ps->a, sb = ps->b, sc = ps->c;
   GQ_TRY(cudaEventRecord(ps->fork, s0));
   GQ_TRY(cudaStreamWaitEvent(s, ps->fork, 0));
@@ -622,7 +626,8 @@ cudaError_t launch_prepare(const double* H, int64_t n, double damp, int order, i
       const int64_t nch = rem > 0 ? (rem + 31) / 32 : 1;
       const int grid = (int)std::min<int64_t>(nch, sms);
       potrf_panel_kernel<<<grid, 256, kPnSmem, s>>>(L.M, ldm, n, c0, w,
-                                                    L.Dinv + (c0 / kNB) * kNB * kNB, L.hdr);
+                                                    L.Dinv + (c0 / kNB) * kNB * kNB, L.hdr,
+                                                    wt.polls, wt.withhold);
       count_launches(1);
       GQ_TRY(cudaGetLastError());
     }

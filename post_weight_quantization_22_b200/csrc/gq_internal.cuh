@@ -94,6 +94,14 @@ constexpr int kBlock = 128;  // columns per GPTQ block (lazy-update rank)
 // Kernel launches issued by this library since load (instrumentation; see gq_kernel_launches).
 void count_launches(long k);
 
+// Test setting of the bounded waits (gq_debug_wait_test): the poll budget of the factor leaf
+// kernel's per-pivot waits and whether that kernel withholds one thread's first arrival.
+struct WaitTest {
+  uint32_t polls;
+  int withhold;
+};
+WaitTest wait_test();
+
 // one-time per-device kernel attribute setup (dynamic shared memory above 48 KB)
 cudaError_t factor_init_attributes();
 cudaError_t quant_init_attributes();

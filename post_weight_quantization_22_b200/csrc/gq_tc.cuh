@@ -50,12 +50,16 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
-// Wait for the phase with the given parity; gives up after ~2^26 polls (well over a second)
-// and returns false so the caller can record an error instead of hanging the GPU.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
-  for (uint32_t i = 0; i < (1u << 26); ++i)
+// Wait for the phase with the given parity; gives up after `polls` polls and returns false so
+// the caller can record an error instead of hanging the GPU.
+constexpr uint32_t kDefaultPolls = 1u << 26;  // well over a second
+__device__ __forceinline__ bool mbar_wait_polls(uint64_t* bar, uint32_t parity, uint32_t polls) {
+  for (uint32_t i = 0; i < polls; ++i)
     if (mbar_try_wait(bar, parity)) return true;
   return false;
+}
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+  return mbar_wait_polls(bar, parity, kDefaultPolls);
 }
 
 // ---- TMA (2-D tile load into shared memory, completion counted on an mbarrier) ----

@@ -70,6 +70,8 @@ def _load():
     lib.gq_huffman_encode.argtypes = [P, I64, P, I64, P, P, P, P, SZ, P]
     lib.gq_zsic_spacing.restype = I
     lib.gq_zsic_spacing.argtypes = [P, I64, P, P]
+    lib.gq_debug_wait_test.restype = I
+    lib.gq_debug_wait_test.argtypes = [ctypes.c_uint32, I]
     lib.gq_workspace_status.restype = I
     lib.gq_workspace_status.argtypes = [P, ctypes.POINTER(ctypes.c_int), P]
     return lib
@@ -81,7 +83,7 @@ EXPORTED = ("gq_version", "gq_status_string", "gq_hessian_accumulate", "gq_hessi
             "gq_prepare_hinv", "gq_quantize_workspace_size", "gq_quantize_layer",
             "gq_workspace_status", "gq_prepare_hinv_static", "gq_prepare_hinv_ordered",
             "gq_quantize_layer_ordered", "gq_zsic_spacing", "gq_huffman_workspace_size",
-            "gq_huffman_encode")
+            "gq_huffman_encode", "gq_debug_wait_test", "gq_kernel_launches")
 
 
 def _ptr(t):
@@ -323,6 +325,13 @@ def gq_huffman_encode(codes: torch.Tensor, stream_words: int | None = None, ws=N
                                  _ptr(cw), _ptr(info), _ptr(ws), ws.numel(), _stream(stream)),
            "gq_huffman_encode")
     return out, lengths, cw, info, ws
+
+
+def gq_debug_wait_test(poll_limit: int = 0, withhold_arrival: bool = False) -> None:
+    """Test setting of the bounded waits (see gq.h); gq_debug_wait_test() restores the
+    defaults."""
+    _check(LIB.gq_debug_wait_test(int(poll_limit), int(bool(withhold_arrival))),
+           "gq_debug_wait_test")
 
 
 def gq_workspace_status(ws: torch.Tensor, stream=None):

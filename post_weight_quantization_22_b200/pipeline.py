@@ -141,3 +141,157 @@ class LayerQuantizer:
         return LayerResult(self.codes, self.scales, self.zeros, self.loss, self.H, self.U,
                            self.dead, self.delta)
 
+
+
+# ---------------------------------------------------------------------------------------------
+# Several layers that share an input: one Hessian and one factor per input
+# ---------------------------------------------------------------------------------------------
+
+class BlockQuantizer:
+    """Quantize a group of layers whose inputs are shared: the layers that read the same
+    activations (q/k/v, gate/up) share one Hessian H = 2 X^T X and one factor U, so each input
+    runs gq_hessian_accumulate and gq_prepare_hinv once and each layer runs gq_quantize_layer.
+
+    ``layers``: sequence of (name, m, n, input_key); layers with the same input_key must have
+    the same n.  Device buffers are allocated here, once; ``run`` allocates nothing.
+    """
+
+    def __init__(self, layers, cfg: G.QuantCfg, device="cuda", damp: float = 0.01,
+                 max_tokens: int = 65536):
+        self.layers = [tuple(l) for l in layers]
+        self.cfg, self.damp, self.max_tokens = cfg, damp, max_tokens
+        dev = torch.device(device)
+        self.inputs = {}
+        for name, m, n, key in self.layers:
+            if key in self.inputs:
+                if self.inputs[key]["n"] != n:
+                    raise ValueError(f"layers of input {key!r} disagree on n")
+                continue
+            self.inputs[key] = dict(
+                n=n, H=torch.zeros((n, n), dtype=torch.float64, device=dev),
+                U=torch.empty((n, n), dtype=torch.float32, device=dev),
+                dead=torch.empty(n, dtype=torch.uint8, device=dev),
+                delta=torch.empty(1, dtype=torch.float64, device=dev),
+                ws_hess=G.workspace(G.gq_hessian_workspace_size(max_tokens, n), dev),
+                ws_prep=G.workspace(G.gq_prepare_workspace_size(n), dev))
+        # one quantize workspace per layer shape (layers run one after another on one stream)
+        self._ws_quant = {}
+        self.out = {}
+        for name, m, n, key in self.layers:
+            if (m, n) not in self._ws_quant:
+                self._ws_quant[(m, n)] = G.workspace(G.gq_quantize_workspace_size(m, n, cfg), dev)
+            ng = 1 if cfg.group_size == 0 else -(-n // cfg.group_size)
+            ncols = n if cfg.clip == "unbounded" else G.n_words(n, cfg.bits)
+            self.out[name] = dict(
+                codes=torch.empty((m, ncols), dtype=torch.int32, device=dev),
+                scales=torch.empty((m, ng), dtype=torch.float32, device=dev),
+                zeros=torch.empty((m, ng), dtype=torch.uint8, device=dev),
+                loss=torch.empty(3, dtype=torch.float64, device=dev))
+
+    def weights(self) -> int:
+        return sum(m * n for _, m, n, _ in self.layers)
+
+    def hessian(self, key: str, X: torch.Tensor, stream=None):
+        """H = 2 X^T X of one input."""
+        d = self.inputs[key]
+        if X.shape[0] > self.max_tokens:
+            raise ValueError(f"{X.shape[0]} tokens exceed {self.max_tokens}")
+        G.gq_hessian_accumulate(d["H"], X, accumulate=False, ws=d["ws_hess"], stream=stream)
+
+    def prepare(self, key: str, stream=None):
+        """U (and the dead mask, the damping) of one input from its H."""
+        d = self.inputs[key]
+        G.gq_prepare_hinv(d["H"], self.damp, self.cfg.reverse, d["U"], d["dead"], d["delta"],
+                          d["ws_prep"], stream=stream)
+
+    def factor(self, key: str, X: torch.Tensor, stream=None):
+        """H and U of one input."""
+        self.hessian(key, X, stream=stream)
+        self.prepare(key, stream=stream)
+
+    def quantize(self, name: str, W: torch.Tensor, stream=None):
+        _, m, n, key = next(l for l in self.layers if l[0] == name)
+        d, o = self.inputs[key], self.out[name]
+        G.gq_quantize_layer(W, d["U"], d["dead"], d["delta"], self.cfg, o["codes"], o["scales"],
+                            o["zeros"], o["loss"], self._ws_quant[(m, n)], stream=stream)
+
+    def run(self, Ws: dict, Xs: dict, names=None, stream=None) -> dict:
+        """The factor of every input that the layers ``names`` (default: all) read, then those
+        layers; returns {name: out buffers}."""
+        names = [l[0] for l in self.layers] if names is None else list(names)
+        keys = []
+        for name, _, _, key in self.layers:
+            if name in names and key not in keys:
+                keys.append(key)
+        for key in keys:
+            self.factor(key, Xs[key], stream=stream)
+        for name in names:
+            self.quantize(name, Ws[name], stream=stream)
+        return {name: self.out[name] for name in names}
+
+    def status(self):
+        """Worst device status over every workspace (0 if all are clean); synchronizes."""
+        codes = []
+        for d in self.inputs.values():
+            codes.append(G.gq_workspace_status(d["ws_prep"])[0])
+        for ws in self._ws_quant.values():
+            codes.append(G.gq_workspace_status(ws)[0])
+        bad = [c for c in codes if c != 0]
+        return bad[0] if bad else 0
+
+
+# ---------------------------------------------------------------------------------------------
+# A sweep over many blocks with per-layer checkpoints
+# ---------------------------------------------------------------------------------------------
+
+class SweepCheckpoint:
+    """Per-layer results of a long sweep on disk, so that an interrupted sweep resumes at the
+    first layer without a result.  One file per (tag, block, layer): the layer's codes, scales,
+    zeros and losses as host tensors (``torch.save``), written to a temporary name and renamed,
+    so a file that exists is complete."""
+
+    def __init__(self, directory: str, tag: str):
+        import os
+        self.dir, self.tag = directory, tag
+        os.makedirs(directory, exist_ok=True)
+
+    def path(self, block: int, layer: str) -> str:
+        import os
+        return os.path.join(self.dir, f"{self.tag}.b{block:03d}.{layer}.pt")
+
+    def done(self, block: int, layer: str) -> bool:
+        import os
+        return os.path.exists(self.path(block, layer))
+
+    def save(self, block: int, layer: str, tensors: dict):
+        import os
+        p = self.path(block, layer)
+        host = {k: v.detach().to("cpu").clone() for k, v in tensors.items()}
+        torch.save(host, p + ".tmp")
+        os.replace(p + ".tmp", p)
+
+    def load(self, block: int, layer: str) -> dict:
+        return torch.load(self.path(block, layer))
+
+
+def run_sweep(blocks, layers, make_inputs, quantize_block, ckpt: SweepCheckpoint,
+              on_layer=None) -> int:
+    """Quantize ``blocks`` (an iterable of block indices) of ``layers`` ((name, m, n,
+    input_key) tuples), skipping every layer that ``ckpt`` already holds.
+
+    ``make_inputs(block)`` returns (Ws, Xs) for one block; ``quantize_block(Ws, Xs, names)``
+    quantizes the named layers (and the inputs they need) and returns {name: tensors}.  A block
+    whose layers are all checkpointed is not regenerated.  Returns the number of layers run."""
+    ran = 0
+    for b in blocks:
+        todo = [l[0] for l in layers if not ckpt.done(b, l[0])]
+        if not todo:
+            continue
+        Ws, Xs = make_inputs(b)
+        res = quantize_block(Ws, Xs, todo)
+        for name in todo:
+            ckpt.save(b, name, res[name])
+            ran += 1
+            if on_layer is not None:
+                on_layer(b, name)
+    return ran

@@ -120,6 +120,21 @@ def sweep_seeds(block: int, layer_index: int, input_kind: str):
     return 1000 + 10 * block + layer_index, 5000 + 10 * block + SWEEP_INPUT_INDEX[input_kind]
 
 
+def sweep_block(block: int, T: int = SWEEP_T, scale: int = 1):
+    """Inputs of one block of the sweep: ({layer name: W}, {input key: X}), bf16 torch CPU
+    tensors.  The attention, o_proj and MLP inputs use the decaying-spectrum generator, the
+    down_proj input its post-SiLU-like transform.  ``scale`` divides every dimension (reduced
+    cases for tests)."""
+    Ws, Xs = {}, {}
+    for li, (name, m, n, kind) in enumerate(SWEEP_LAYERS):
+        w_seed, x_seed = sweep_seeds(block, li, kind)
+        Ws[name] = to_bf16(make_w("layer", m // scale, n // scale, w_seed))
+        if kind not in Xs:
+            x_kind = "post_silu" if kind == "down" else "calib"
+            Xs[kind] = to_bf16(make_x(x_kind, T // scale, n // scale, x_seed))
+    return Ws, Xs
+
+
 def make_x(x_kind: str, T: int, n: int, seed: int) -> np.ndarray:
     if x_kind == "calib":
         return calib_activations(T, n, seed)

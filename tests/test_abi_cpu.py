@@ -98,3 +98,10 @@ def test_quant_cfg_binding_matches_the_header_struct():
     assert (c.bits, c.clip, c.spacing) == (3, 2, 1)
     c = G.QuantCfg(bits=4, clip=False).c()
     assert (c.clip, c.spacing) == (0, 0)
+
+
+def test_wait_test_setting_is_host_only_and_checked():
+    from post_weight_quantization_22_b200 import gq as G
+    assert G.LIB.gq_debug_wait_test(0, 2) == 1          # withhold must be 0 or 1
+    assert G.LIB.gq_debug_wait_test(4096, 1) == 0       # a host-side setting: no GPU needed
+    assert G.LIB.gq_debug_wait_test(0, 0) == 0          # back to the defaults

@@ -440,33 +440,43 @@ def test_clipfree_babai_full_size_sampled_rows():
     _compare(g, o, W, 3, 0, rows=rows)
 
 
+@pytest.fixture(scope="module")
+def sweep_block0():
+    """Block 0 of the 8B-shaped sweep (bf16 weights and its four inputs, 8192 tokens each)."""
+    return synth.sweep_block(0)
+
+
 @pytest.mark.slow
-def test_sweep_block_shared_hessian_2bit_g64():
-    """One block of the 8B-shaped sweep: q, k and v share their input, so one H and one factor
-    serve three layers of different heights (2-bit, group 64, 8192 tokens)."""
+@pytest.mark.parametrize("key", ["attn", "o", "mlp", "down"])
+def test_sweep_block_layers_2bit_g64(sweep_block0, key):
+    """Every layer of one block of the 8B-shaped sweep at 2-bit, group 64, in the bench's launch
+    configuration (BlockQuantizer: one H and one factor per input, shared by the layers that
+    read it): q/k/v share the attention input, gate/up the MLP input (14336 rows each), o and
+    down have their own (down's factor is 14336 wide).  H and U in full against the oracle,
+    codes / grids on sampled rows of every layer."""
     from post_weight_quantization_22_b200 import gq as G
-    T, n = synth.SWEEP_T, 4096
-    x_seed = synth.sweep_seeds(0, 0, "attn")[1]
-    X = synth.to_bf16(synth.make_x("calib", T, n, x_seed))
-    H = torch.zeros((n, n), dtype=torch.float64, device="cuda")
-    G.gq_hessian_accumulate(H, X.cuda())
-    U, dead, delta, _ = G.gq_prepare_hinv(H, 0.01)
-    cfg = G.QuantCfg(bits=2, group_size=64)
-    for li, (name, m, _, kind) in enumerate(synth.SWEEP_LAYERS[:3]):
-        w_seed = synth.sweep_seeds(0, li, kind)[0]
-        W = synth.to_bf16(synth.make_w("layer", m, n, w_seed))
-        codes, scales, zeros, loss, ws = G.gq_quantize_layer(W.cuda(), U, dead, delta, cfg)
-        torch.cuda.synchronize()
-        assert G.gq_workspace_status(ws)[0] == 0
-        packed = codes.cpu().numpy().view(np.uint32)
-        gres = dict(H=H.cpu().numpy(), U=U.cpu().numpy(), packed=packed,
-                    codes=unpack_np(packed, n, 2),
-                    scales=scales.cpu().numpy(), zeros=zeros.cpu().numpy().astype(np.int64),
-                    loss=loss.cpu().numpy(), dead=dead.cpu().numpy().astype(bool),
-                    delta=float(delta.item()))
+    from post_weight_quantization_22_b200.pipeline import BlockQuantizer
+    Ws, Xs = sweep_block0
+    layers = [l for l in synth.SWEEP_LAYERS if l[3] == key]
+    bq = BlockQuantizer(layers, G.QuantCfg(bits=2, group_size=64), device="cuda",
+                        max_tokens=synth.SWEEP_T)
+    out = bq.run({n: Ws[n].cuda() for n, _, _, _ in layers}, {key: Xs[key].cuda()})
+    torch.cuda.synchronize()
+    assert bq.status() == 0
+    d = bq.inputs[key]
+    X = Xs[key]
+    H = O.hessian(X)
+    for li, (name, m, n, _) in enumerate(layers):
+        o_ = out[name]
+        packed = o_["codes"].cpu().numpy().view(np.uint32)
+        gres = dict(H=d["H"].cpu().numpy(), U=d["U"].cpu().numpy(), packed=packed,
+                    codes=unpack_np(packed, n, 2), scales=o_["scales"].cpu().numpy(),
+                    zeros=o_["zeros"].cpu().numpy().astype(np.int64),
+                    loss=o_["loss"].cpu().numpy(), dead=d["dead"].cpu().numpy().astype(bool),
+                    delta=float(d["delta"].item()))
         rows = np.random.default_rng(20 + li).choice(m, size=32, replace=False)
-        o = _oracle(W, X, 2, 64, False, True, rows=rows)
-        _compare(gres, o, W, 2, 64, rows=rows)
+        o = O.quantize_layer(Ws[name], X, bits=2, group=64, rows=rows, H=H)
+        _compare(gres, o, Ws[name], 2, 64, rows=rows)
 
 
 def test_run_host_overlapped_copies_match_device_run():
@@ -493,3 +503,32 @@ def test_run_host_overlapped_copies_match_device_run():
     c0 = unpack_np(codes0.cpu().numpy().view(np.uint32), 1024, 4)
     assert np.mean(c1 == c0) >= CODE_MATCH
     assert lq.status()[:2] == (0, 0)
+
+
+def test_bounded_wait_runs_out_and_the_next_call_is_clean():
+    """Failure detection of the bounded waits: with the test setting, the factor's leaf kernel
+    withholds one barrier arrival, every wait of that phase gives up after 4096 polls, the call
+    reports GQ_ERR_TIMEOUT through its workspace, and the context stays usable: the next call on
+    the same buffers, without the setting, is clean and matches the oracle."""
+    import time
+    from post_weight_quantization_22_b200 import gq as G
+    _, X, _ = synth.workload("q_proj_4096x4096", m=8, n=200, T=300)
+    H = torch.zeros((200, 200), dtype=torch.float64, device="cuda")
+    G.gq_hessian_accumulate(H, X.cuda())
+    torch.cuda.synchronize()
+    G.gq_debug_wait_test(4096, True)
+    try:
+        t0 = time.perf_counter()
+        U, dead, delta, ws = G.gq_prepare_hinv(H, 0.01)
+        torch.cuda.synchronize()
+        elapsed = time.perf_counter() - t0
+    finally:
+        G.gq_debug_wait_test()
+    assert G.gq_workspace_status(ws)[0] == 5           # GQ_ERR_TIMEOUT
+    assert elapsed < 30.0
+    U2, _, _, _ = G.gq_prepare_hinv(H, 0.01, U=U, dead=dead, delta=delta, ws=ws)
+    torch.cuda.synchronize()
+    assert G.gq_workspace_status(ws)[0] == 0
+    hfix, _, _ = O.fix_dead_features(H.cpu().numpy(), np.zeros((1, 200)))
+    hd, _ = O.dampen(hfix, 0.01)
+    assert rel_fro(np.triu(U2.cpu().numpy()), O.hinv_upper_factor(hd)) <= U_REL_DESIGN

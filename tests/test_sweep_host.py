@@ -1,0 +1,112 @@
+"""Host logic without a GPU: the sweep's per-layer checkpoint / resume, the shared-input block
+layout, and the bench's roofline arithmetic and bounded oracle sample."""
+import os
+import sys
+
+import numpy as np
+import pytest
+import torch
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+LAYERS = (("q", 8, 4, "attn"), ("k", 4, 4, "attn"), ("o", 8, 4, "o"), ("down", 4, 12, "down"))
+
+
+def _inputs(block):
+    g = torch.Generator().manual_seed(block)
+    Ws = {name: torch.randn(m, n, generator=g) for name, m, n, _ in LAYERS}
+    Xs = {"attn": torch.randn(5, 4, generator=g), "o": torch.randn(5, 4, generator=g),
+          "down": torch.randn(5, 12, generator=g)}
+    return Ws, Xs
+
+
+def _fake_block(calls):
+    """A stand-in for BlockQuantizer.run: deterministic outputs from the inputs."""
+    def q(Ws, Xs, names):
+        calls.append(tuple(names))
+        out = {}
+        for name, _, _, key in LAYERS:
+            if name in names:
+                out[name] = {"codes": (Ws[name] * 7).round().to(torch.int32),
+                             "loss": (Ws[name] @ Xs[key].T).pow(2).sum().reshape(1)}
+        return out
+    return q
+
+
+def test_sweep_resumes_at_the_first_missing_layer(tmp_path):
+    from post_weight_quantization_22_b200.pipeline import SweepCheckpoint, run_sweep
+    full = SweepCheckpoint(str(tmp_path / "full"), "cfg5")
+    calls = []
+    assert run_sweep(range(3), LAYERS, _inputs, _fake_block(calls), full) == 12
+    assert len(calls) == 3
+
+    part = SweepCheckpoint(str(tmp_path / "part"), "cfg5")
+    seen = []
+
+    class Stop(Exception):
+        pass
+
+    def stop_after_six(b, name):
+        seen.append((b, name))
+        if len(seen) == 6:
+            raise Stop()
+    calls2 = []
+    with pytest.raises(Stop):
+        run_sweep(range(3), LAYERS, _inputs, _fake_block(calls2), part, on_layer=stop_after_six)
+    # a half-written file from a crash is not a result
+    open(part.path(2, "q") + ".tmp", "wb").write(b"partial")
+    calls3 = []
+    assert run_sweep(range(3), LAYERS, _inputs, _fake_block(calls3), part) == 6
+    assert calls3 == [("o", "down"), ("q", "k", "o", "down")]  # block 0 skipped entirely
+    for b in range(3):
+        for name, _, _, _ in LAYERS:
+            a, c = full.load(b, name), part.load(b, name)
+            assert torch.equal(a["codes"], c["codes"]) and torch.equal(a["loss"], c["loss"])
+    # nothing left to do: no inputs are generated
+    def no_inputs(b):
+        raise AssertionError("regenerated a finished block")
+    assert run_sweep(range(3), LAYERS, no_inputs, _fake_block([]), part) == 0
+
+
+def test_sweep_block_inputs_share_one_input_per_kind():
+    from post_weight_quantization_22_b200 import synth
+    Ws, Xs = synth.sweep_block(0, scale=16)
+    assert set(Xs) == {"attn", "o", "mlp", "down"}
+    for name, m, n, kind in synth.SWEEP_LAYERS:
+        assert tuple(Ws[name].shape) == (m // 16, n // 16)
+        assert Xs[kind].shape[1] == n // 16 and Ws[name].dtype == torch.bfloat16
+    # the attention input of block 0 is the one the q/k/v parity test builds by hand
+    x_seed = synth.sweep_seeds(0, 0, "attn")[1]
+    ref = synth.to_bf16(synth.make_x("calib", synth.SWEEP_T // 16, 4096 // 16, x_seed))
+    assert torch.equal(ref, Xs["attn"])
+
+
+def test_stage_model_fractions_are_floor_over_measured():
+    sys.path.insert(0, ROOT)
+    import bench
+    peaks = dict(hbm_gbs=6000.0, bf16_tflops=1500.0, fp64_tflops=36.0, tf32_tflops=750.0,
+                 fp32_tflops=70.0, int8_tops=3000.0)
+    inputs, layers = [("x", 4096, 4096)], [("w", 4096, 4096, "x")]
+    ms = {"hessian": 0.8, "factor": 3.0, "column_loop": 2.0}
+    st, ov = bench.stage_model(inputs, layers, 4, 128, 2, peaks, ms)
+    n, T, m = 4096, 4096, 4096
+    h_floor = 2 * n * (n + 1) / 2 * T * bench.HESSIAN_DIGIT_PRODUCTS / 3000e12
+    assert st["hessian"]["t_roof_ms"] == pytest.approx(h_floor * 1e3, rel=1e-3)
+    assert st["factor"]["t_roof_ms"] == pytest.approx(2 * n ** 3 / 3 / 36e12 * 1e3, rel=1e-3)
+    assert st["column_loop"]["t_roof_ms"] == pytest.approx(3 * m * n * n / 750e12 * 1e3, rel=1e-3)
+    for k in ms:
+        assert st[k]["frac"] == pytest.approx(st[k]["t_roof_ms"] / ms[k], rel=1e-3)
+    assert ov["t_ms"] == pytest.approx(5.8)
+    assert ov["frac_as_built"] == pytest.approx(
+        sum(st[k]["t_roof_ms"] for k in ms) / 5.8, rel=1e-3)
+
+
+def test_oracle_sample_scales_each_part_by_its_cost():
+    sys.path.insert(0, ROOT)
+    import bench
+    rng = np.random.default_rng(0)
+    X = rng.standard_normal((64, 48))
+    W = 0.02 * rng.standard_normal((40, 48))
+    t, det = bench.oracle_layer_sample([(X, [(W, 3, 0)])], tokens=32, n_sub=24, rows=8)
+    assert t == pytest.approx(det["hessian_s"] + det["factor_s"] + det["loop_s"])
+    assert 0 < det["measured_s"] < t       # every part is scaled up from a smaller sample
