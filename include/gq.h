@@ -122,7 +122,9 @@ gq_status gq_hessian_accumulate(double* d_H, const void* d_X, gq_dtype x_dtype, 
 
 /* Workspace bytes gq_prepare_hinv needs for width n (256-byte aligned base required): two fp64
  * n x n work matrices (the factor and its inverse in place, and the inverse's accumulated block
- * products), about 16 n^2 bytes. */
+ * products), about 16 n^2 bytes, and from n = 1536 about 3 n^2 bytes more of int8 digit planes
+ * (the large products of the factorisation run as exact int8 digit products on the tensor
+ * cores, combined in fp64). */
 size_t gq_prepare_workspace_size(int64_t n);
 
 /*

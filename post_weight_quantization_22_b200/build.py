@@ -16,7 +16,7 @@ CSRC = os.path.join(PKG, "csrc")
 OUT = os.path.join(PKG, "libgq.so")
 BUILD_DIR = os.path.join(ROOT, "_build", "libgq")
 SOURCES = ["gq_api.cu", "gq_hessian.cu", "gq_factor.cu", "gq_dgemm.cu", "gq_quant.cu", "gq_lazy_tc.cu",
-           "gq_noalloc.cu", "gq_huffman.cu"]
+           "gq_noalloc.cu", "gq_huffman.cu", "gq_split.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-Xcompiler", "-O3",
          "--expt-relaxed-constexpr", "-I", os.path.join(ROOT, "include")]

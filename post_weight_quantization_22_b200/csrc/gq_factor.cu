@@ -383,6 +383,11 @@ __global__ void flip_to_u_kernel(const double* M, int64_t n, int64_t ldm, float*
 // 16-byte multiples).
 static int64_t m_ld(int64_t n) { return (n + 15) / 16 * 16; }
 
+// Widths from which the large products run on the int8 tensor cores (gq_split.cu); below it
+// every product stays on the fp64 units (the products are small and the chain dominates).
+constexpr int64_t kSplitMinN = 1536;
+static bool use_split(int64_t n) { return n >= kSplitMinN; }
+
 struct PrepLayout {
   WsHeader* hdr;
   double* M;     // n x ldm: lower triangle = J P H_d P J, then the inverse of its Cholesky factor
@@ -390,8 +395,22 @@ struct PrepLayout {
   double* Dinv;  // ceil(n / 64) x 64 x 64: the inverted 64-wide leaves
   double* tbuf;  // doubling scratch of the diagonal super-block inverses
   int* pmark;    // n ints: occurrence marks when checking a caller's permutation
+  // int8 digit planes (split path only): for every super-panel K with rows below it, the rows
+  // sp1..n-1 of its columns of L (kept until the call ends, read by three streams), and one
+  // block row of the inverse as the second operand of the inverse's products
+  int8_t* ldig;
+  int* lex;
+  int8_t* xdig;
+  int* xex;
   size_t bytes;
 };
+
+// rows of the L digit planes of the super-panels before super-panel K
+static int64_t lrow_offset(int64_t n, int64_t K) {
+  int64_t off = 0;
+  for (int64_t k = 0; k < K; ++k) off += std::max<int64_t>(n - (k + 1) * kSuper, 0);
+  return off;
+}
 
 // doubling scratch for one diagonal block of width w (<= kSuper)
 static size_t trtri_tbuf_elems(int64_t w) {
@@ -413,6 +432,14 @@ static PrepLayout prep_layout(void* ws, int64_t n) {
   L.Dinv = c.take<double>((size_t)((n + kNB - 1) / kNB) * kNB * kNB);
   L.tbuf = c.take<double>(trtri_tbuf_elems(kSuper) + 1);
   L.pmark = c.take<int>((size_t)n);
+  L.ldig = nullptr; L.lex = nullptr; L.xdig = nullptr; L.xex = nullptr;
+  if (use_split(n)) {
+    const int64_t lrows = lrow_offset(n, (n + kSuper - 1) / kSuper);
+    L.ldig = c.take<int8_t>((size_t)kSplitDigits * kSplitK * (size_t)lrows);
+    L.lex = c.take<int>((size_t)lrows);
+    L.xdig = c.take<int8_t>((size_t)kSplitDigits * kSplitK * (size_t)n);
+    L.xex = c.take<int>((size_t)n);
+  }
   L.bytes = c.off;
   return L;
 }
@@ -426,6 +453,7 @@ cudaError_t factor_init_attributes() {
   e = cudaFuncSetAttribute(build_m_perm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)(kStageMaxN * sizeof(double)));
   if (e != cudaSuccess) return e;
+  if ((e = split_init_attributes()) != cudaSuccess) return e;
   return dgemm_init_attributes();
 }
 
@@ -574,6 +602,13 @@ cudaError_t launch_prepare(const double* H, int64_t n, double damp, int order, i
   // with T accumulated right-looking once X's block row K is known:
   //   T[i >= k1, K] = L[i, K] X_KK,   T[i >= k1, :k0] += L[i, K] X[K, :k0]   (K = 256 GEMMs).
   // X overwrites L in place: block row K of L is not read by the Cholesky after block K.
+  const bool split = use_split(n);
+  // digit planes of super-panel K's columns of L, rows sp1 .. n-1 (plane row r = row sp1 + r)
+  auto l_operand = [&](int64_t K) {
+    const int64_t off = lrow_offset(n, K);
+    return SplitOperand{L.ldig + off * kSplitDigits * kSplitK, L.lex + off,
+                        n - std::min<int64_t>((K + 1) * kSuper, n)};
+  };
   auto inverse_block_row = [&](int64_t k0, int64_t k1) -> cudaError_t {
     const int64_t kw = k1 - k0;
     GQ_TRY(invert_diag_block(L.M, n, ldm, k0, kw, L.Dinv, L.tbuf, L.hdr, sc));
@@ -595,7 +630,12 @@ cudaError_t launch_prepare(const double* H, int64_t n, double damp, int order, i
         g.C = L.T + k1 * ldm + k0; g.ldc = ldm; g.hdr = L.hdr;
         GQ_TRY(launch_dgemm(g, sc));
       }
-      if (k0 > 0) {  // T[k1:, :k0] += L[k1:, K] X[K, :k0]
+      if (k0 > 0 && split) {  // T[k1:, :k0] += L[k1:, K] X[K, :k0] on the int8 tensor cores
+        const SplitOperand xop{L.xdig, L.xex, k0};
+        GQ_TRY(launch_split_cols(L.M + k0 * ldm, ldm, (int)k0, xop, sc));
+        GQ_TRY(launch_split_gemm(L.T + k1 * ldm, ldm, (int)(n - k1), (int)k0, l_operand(k0 / kSuper),
+                                 0, xop, 0, 1.0, 0, L.hdr, sc));
+      } else if (k0 > 0) {  // T[k1:, :k0] += L[k1:, K] X[K, :k0]
         DgemmCall g{};
         g.M = (int)(n - k1); g.N = (int)k0; g.K = (int)kw; g.batch = 1; g.alpha = 1.0;
         g.beta_one = 1;
@@ -641,7 +681,11 @@ cudaError_t launch_prepare(const double* H, int64_t n, double damp, int order, i
       GQ_TRY(launch_dgemm(g, s));
     }
     if (c0 + w != sp1) continue;
-    // super-panel [sp0, sp1) factored
+    // super-panel [sp0, sp1) factored; on the split path its columns of L below it become
+    // digit planes once, for the two trailing updates and the inverse's block product
+    const bool sp_split = split && sp1 < n;
+    const SplitOperand lop = sp_split ? l_operand(sp0 / kSuper) : SplitOperand{};
+    if (sp_split) GQ_TRY(launch_split_rows(L.M + sp1 * ldm + sp0, ldm, (int)(n - sp1), lop, s));
     cudaEvent_t ev_panel = ps->panel[sidx & 1];
     GQ_TRY(cudaEventRecord(ev_panel, s));
     GQ_TRY(cudaStreamWaitEvent(sc, ev_panel, 0));
@@ -649,7 +693,10 @@ cudaError_t launch_prepare(const double* H, int64_t n, double damp, int order, i
     if (sp1 < n) {
       const int64_t sp2 = std::min<int64_t>(sp1 + kSuper, n), kw = sp1 - sp0;
       if (far_pending) GQ_TRY(cudaStreamWaitEvent(s, ps->far[(sidx - 1) & 1], 0));
-      {  // next super-panel's columns: A[sp1:, sp1:sp2] -= L[sp1:, SP] L[sp1:sp2, SP]^T
+      if (sp_split) {  // next super-panel's columns: A[sp1:, sp1:sp2] -= L[sp1:, SP] L[sp1:sp2, SP]^T
+        GQ_TRY(launch_split_gemm(L.M + sp1 * ldm + sp1, ldm, (int)(n - sp1), (int)(sp2 - sp1),
+                                 lop, 0, lop, 0, -1.0, 1, L.hdr, s));
+      } else {  // next super-panel's columns: A[sp1:, sp1:sp2] -= L[sp1:, SP] L[sp1:sp2, SP]^T
         DgemmCall g{};
         g.M = (int)(n - sp1); g.N = (int)(sp2 - sp1); g.K = (int)kw; g.batch = 1;
         g.alpha = -1.0; g.beta_one = 1;
@@ -661,13 +708,19 @@ cudaError_t launch_prepare(const double* H, int64_t n, double damp, int order, i
       far_pending = false;
       if (sp2 < n) {  // later columns, stream B: A[sp2:, sp2:] -= L[sp2:, SP] L[sp2:, SP]^T
         GQ_TRY(cudaStreamWaitEvent(sb, ev_panel, 0));
-        DgemmCall g{};
-        g.M = (int)(n - sp2); g.N = (int)(n - sp2); g.K = (int)kw; g.batch = 1;
-        g.alpha = -1.0; g.beta_one = 1;
-        g.A = Mop(sp2, sp0);
-        g.B = Mop(sp2, sp0); g.b_nmajor = 0;
-        g.C = L.M + sp2 * ldm + sp2; g.ldc = ldm; g.lower_tiles = 1; g.hdr = L.hdr;
-        GQ_TRY(launch_dgemm(g, sb));
+        if (sp_split) {
+          GQ_TRY(launch_split_gemm(L.M + sp2 * ldm + sp2, ldm, (int)(n - sp2), (int)(n - sp2),
+                                   lop, (int)(sp2 - sp1), lop, (int)(sp2 - sp1), -1.0, 1, L.hdr,
+                                   sb));
+        } else {
+          DgemmCall g{};
+          g.M = (int)(n - sp2); g.N = (int)(n - sp2); g.K = (int)kw; g.batch = 1;
+          g.alpha = -1.0; g.beta_one = 1;
+          g.A = Mop(sp2, sp0);
+          g.B = Mop(sp2, sp0); g.b_nmajor = 0;
+          g.C = L.M + sp2 * ldm + sp2; g.ldc = ldm; g.lower_tiles = 1; g.hdr = L.hdr;
+          GQ_TRY(launch_dgemm(g, sb));
+        }
         GQ_TRY(cudaEventRecord(ps->far[sidx & 1], sb));
         far_pending = true;
       }

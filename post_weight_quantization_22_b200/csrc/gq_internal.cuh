@@ -144,6 +144,29 @@ struct DgemmCall {
 cudaError_t dgemm_init_attributes();
 cudaError_t launch_dgemm(const DgemmCall& c, cudaStream_t s);
 
+// ---- fp64-accurate products from int8 digit products (gq_split.cu) ----
+constexpr int kSplitDigits = 6;  // signed 7-bit digits per value
+constexpr int kSplitK = 256;     // depth of every split product (one super-panel)
+// Digit planes of an operand: plane s is plane_rows x kSplitK int8 (K-major rows), planes
+// stacked at plane_rows x kSplitK bytes; ex[r] is the power-of-two scale exponent of row r.
+struct SplitOperand {
+  int8_t* digits;
+  int* ex;
+  int64_t plane_rows;
+};
+cudaError_t split_init_attributes();
+// digits of the rows of A (rows x kSplitK fp64, leading dimension lda, 16-byte aligned)
+cudaError_t launch_split_rows(const double* A, int64_t lda, int rows, SplitOperand op,
+                              cudaStream_t s);
+// digits of the columns of X (kSplitK rows x cols fp64, leading dimension ldx) as operand rows
+cudaError_t launch_split_cols(const double* X, int64_t ldx, int cols, SplitOperand op,
+                              cudaStream_t s);
+// C[i][j] += alpha sum_k A(a_row0 + i, k) B(b_row0 + j, k), i < M, j < N (only j <= i when
+// lower), C fp64 row-major with leading dimension ldc.
+cudaError_t launch_split_gemm(double* C, int64_t ldc, int M, int N, const SplitOperand& A,
+                              int a_row0, const SplitOperand& B, int b_row0, double alpha,
+                              int lower, WsHeader* hdr, cudaStream_t s);
+
 // ---- lazy block update on tensor cores (gq_lazy_tc.cu) ----
 struct LazyTcMaps {
   CUtensorMap ahi, alo, bhi, blo;

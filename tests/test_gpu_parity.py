@@ -91,6 +91,24 @@ def test_qproj_recipe_ragged_group128():
     _compare(g, o, W, 4, 128)
 
 
+def test_ragged_split_factor_group128():
+    """n = 1700 takes the factor's split path (the large products as exact int8 digit products
+    on the tensor cores, from n = 1536): the last super-panel is 164 wide and the last panel 36,
+    so the digit planes, the lower-tile enumeration and the masked epilogue all meet ragged
+    edges; U and the codes against the oracle."""
+    W, X, spec = synth.workload("q_proj_4096x4096", m=300, n=1700, T=2000)
+    g = run_gpu(W, X, bits=4, group=128)
+    assert g["status"] == (0, 0)
+    o = _oracle(W, X, 4, 128, False, True)
+    _compare(g, o, W, 4, 128)
+    gr = run_gpu(W, X, bits=3, reverse=True, clip=False)
+    assert gr["status"] == (0, 0)
+    orr = _oracle(W, X, 3, 0, True, False)
+    hd = orr["Hd"][::-1, ::-1]
+    assert rel_fro(np.triu(gr["U"]), O.hinv_upper_factor(hd)) <= U_REL_DESIGN
+    _compare(gr, orr, W, 3, 0)
+
+
 def test_clipfree_reverse_ladder_and_bound():
     """clip-free Babai, last to first, 3-bit per-row step widened until no code overflows."""
     W, X, spec = synth.workload("clipfree_babai_4096x4096", m=256, n=640, T=900)
