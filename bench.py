@@ -44,8 +44,8 @@ SWEEP_WORKLOAD = "sweep_block"
 L2_FLUSH_BYTES = 256 << 20
 
 # int8 digit products the Hessian kernel issues per multiply-add of X^T X (four 7-bit digits a
-# value, every pair of digits kept)
-HESSIAN_DIGIT_PRODUCTS = 16
+# value, the 13 pairs of digits with a + b <= 4)
+HESSIAN_DIGIT_PRODUCTS = 13
 
 
 # ---------------------------------------------------------------------------------------------
@@ -242,6 +242,32 @@ def complete_peaks(peaks: dict) -> dict:
 # the work of a step and its floor on each pipe
 # ---------------------------------------------------------------------------------------------
 
+# The factor's schedule (gq_factor.cu): 256-wide super-panels; from n = 1536 the trailing
+# update of every super-panel that has rows below it (next super-panel's columns and all later
+# ones: the lower triangle of the remaining (n - sp1) x (n - sp1) block, depth 256) and the
+# inverse's block product T[sp1:, :sp0] += L[sp1:, K] X[K, :sp0] run as int8 digit products,
+# 21 per multiply-add (six 7-bit digits a value, the pairs with p + q <= 5).
+FACTOR_SUPER = 256
+FACTOR_SPLIT_MIN_N = 1536
+FACTOR_DIGIT_PRODUCTS = 21
+
+
+def factor_work(n: int):
+    """(multiply-adds done as int8 digit products, remaining fp64 flops) of one factor of
+    width n; the two add up to the algorithmic 2 n^3 / 3 flops."""
+    total = 2.0 * n ** 3 / 3.0
+    if n < FACTOR_SPLIT_MIN_N:
+        return 0.0, total
+    macs = 0.0
+    for sp0 in range(0, n, FACTOR_SUPER):
+        sp1 = sp0 + FACTOR_SUPER
+        if sp1 >= n:
+            break
+        r = n - sp1
+        macs += (r * (r + 1) / 2.0 + r * sp0) * FACTOR_SUPER
+    return macs, max(total - 2.0 * macs, 0.0)
+
+
 def step_shapes(workload: str, spec: dict):
     """(inputs [(key, n, T)], layers [(name, m, n, key)]) of one step."""
     if workload == SWEEP_WORKLOAD:
@@ -269,6 +295,9 @@ def stage_model(inputs, layers, bits: int, group: int, w_bytes: int, peaks: dict
     bf16 = peaks["bf16_tflops"] * 1e12
     h_macs = sum(n * (n + 1) / 2 * T for _, n, T in inputs)
     f_flops = sum(2.0 * n ** 3 / 3 for _, n, _ in inputs)
+    f_split = [factor_work(n) for _, n, _ in inputs]
+    f_int8_ops = sum(2.0 * macs * FACTOR_DIGIT_PRODUCTS for macs, _ in f_split)
+    f_fp64 = sum(fp for _, fp in f_split)
     lazy_flops = sum(float(m) * n * n for _, m, n, _ in layers)
     loop_bytes = 0.0
     for _, m, n, _ in layers:
@@ -276,16 +305,19 @@ def stage_model(inputs, layers, bits: int, group: int, w_bytes: int, peaks: dict
         loop_bytes += m * n * w_bytes + n * n / 2 * 4 + m * n * bits / 8 + m * G * 5
     t = {
         "hessian": 2 * h_macs * HESSIAN_DIGIT_PRODUCTS / int8,
-        "factor": f_flops / fp64,
+        "factor": f_int8_ops / int8 + f_fp64 / fp64,
         "column_loop": max(3 * lazy_flops / tf32, loop_bytes / hbm),
     }
     stages = {
         "hessian": dict(work=2 * h_macs, unit="flop", pipe="int8 tensor cores",
                         issued=f"{HESSIAN_DIGIT_PRODUCTS} int8 digit products per multiply-add",
                         peak=f"{peaks['int8_tops']:.0f} TOPS int8 (cuBLAS, measured here)"),
-        "factor": dict(work=f_flops, unit="flop", pipe="fp64 tensor cores",
-                       issued="fp64 (DMMA m16n8k8 and DFMA)",
-                       peak=f"{peaks['fp64_tflops']:.1f} TFLOP/s fp64 (cuBLAS, measured here)"),
+        "factor": dict(work=f_flops, unit="flop", pipe="int8 tensor cores + fp64 tensor cores",
+                       issued=(f"{f_int8_ops / 2 / FACTOR_DIGIT_PRODUCTS / (f_flops / 2):.3f} of "
+                               f"the multiply-adds as {FACTOR_DIGIT_PRODUCTS} int8 digit products "
+                               f"each, the rest fp64 (DMMA m16n8k8 and DFMA)"),
+                       peak=(f"{peaks['int8_tops']:.0f} TOPS int8 and {peaks['fp64_tflops']:.1f} "
+                             f"TFLOP/s fp64 (cuBLAS, measured here)")),
         "column_loop": dict(work=lazy_flops, unit="flop", pipe="tf32 tensor cores / HBM",
                             issued="3xTF32 lazy updates; floor also >= algorithmic HBM bytes",
                             bytes=loop_bytes,
@@ -557,7 +589,8 @@ def run_gq(args):
     d = stages[dname]
     roof = {"kernel": {"hessian": "gq_hessian_accumulate (hessian_tc_kernel: int8 digit "
                                   "products on tcgen05)",
-                       "factor": "gq_prepare_hinv (blocked fp64 Cholesky + triangular inverse)",
+                       "factor": "gq_prepare_hinv (blocked Cholesky + triangular inverse: "
+                                 "split_gemm_kernel int8 digit products, fp64 leaves and panels)",
                        "column_loop": "gq_quantize_layer (colloop_kernel + lazy_tc_kernel)"}[dname],
             "bound": "tensor",
             "achieved": d["achieved_tflops"],

@@ -61,8 +61,8 @@ typedef enum {
   GQ_ORDER_REVERSE = 1,   /* columns n-1, ..., 0 (Babai order) */
   GQ_ORDER_ACT = 2,       /* descending diagonal of H after the dead fix; ties by column index */
   GQ_ORDER_MIN_PIVOT = 3, /* greedy min-pivot: the reverse of the elimination order of a
-                             pivoted LDL of H_d that always eliminates the smallest pivot.
-                             Reserved: gq_prepare_hinv_ordered returns GQ_ERR_UNSUPPORTED */
+                             pivoted LDL of H_d that always eliminates the smallest remaining
+                             Schur-complement pivot (ties: lowest column index) */
   GQ_ORDER_GIVEN = 4      /* the caller's permutation */
 } gq_order;
 
@@ -109,10 +109,12 @@ size_t gq_hessian_workspace_size(int64_t T, int64_t n);
  *           1 <= n <= 32768.
  *   d_ws    workspace of at least gq_hessian_workspace_size(T, n) bytes (256-byte aligned).
  *
- * Precision: the products are formed exactly (each value as four 7-bit digits against a
- * power-of-two scale per input column, int8 tensor-core products with int32 sums) and
- * combined in fp64; the only error besides fp64 rounding is the rounding of entries smaller
- * than 2^-21 of their column's largest, at 2^-29 of that largest.  H is fp64 because the
+ * Precision: the products are formed from exact pieces (each value as four 7-bit digits
+ * against a power-of-two scale per input column, int8 tensor-core products of the 13 digit
+ * pairs that weigh at least 2^-42 of the scales, int32 sums) and combined in fp64; besides fp64
+ * rounding, the errors are the rounding of entries smaller than 2^-21 of their column's
+ * largest, at 2^-29 of that largest, and the three dropped digit pairs, below 2^-35 of a
+ * product's scale (H within about 1e-12 relative of the exact 2 X^T X on the layer recipes).  H is fp64 because the
  * column loop's codes depend on H to about 1e-9 relative for the ill-conditioned Hessians of
  * LLM layers.
  */
@@ -186,9 +188,10 @@ gq_status gq_prepare_hinv_static(const double* d_H, int64_t n, double damp, int 
  *
  *   order    a gq_order.  NATURAL and REVERSE give exactly gq_prepare_hinv's U with
  *            reverse = 0 / 1 (d_perm is then not touched and may be NULL).
- *   d_perm   n int32, device.  ACT writes the order computed on the device from H; GIVEN
- *            reads it.  Pass the same array to gq_quantize_layer_ordered.  MIN_PIVOT is
- *            rejected with GQ_ERR_UNSUPPORTED (no device implementation).
+ *   d_perm   n int32, device.  ACT and MIN_PIVOT write the order computed on the device from
+ *            H; GIVEN reads it.  Pass the same array to gq_quantize_layer_ordered.  MIN_PIVOT
+ *            runs a pivoted elimination of H_d before the factor (about n/32 one-CTA panel
+ *            launches and as many n x n fp64 rank-32 updates).
  * Device-detected errors: GQ_ERR_INVALID_ARG (GIVEN: d_perm is not a permutation of 0..n-1;
  * every access stays in bounds and U is then undefined), GQ_ERR_NOT_PD.
  */
@@ -255,6 +258,46 @@ gq_status gq_quantize_layer_ordered(const void* d_W, gq_dtype w_dtype, int64_t m
                                     uint8_t* d_zeros, double* d_loss, void* d_ws,
                                     size_t ws_bytes, gq_stream_t stream);
 
+/* Workspace bytes gq_ssqr_quantize_layer needs for an m x n layer (0 if out of range). */
+size_t gq_ssqr_workspace_size(int64_t m, int64_t n);
+
+/*
+ * SSQR ("The Geometry of LLM Quantization", section 3, scale-adjusted SpQR): the layer is
+ * quantized with the GPTQ column loop on one clip-free grid per row, centred on the row's range
+ * [lo, hi] (lo <= 0 <= hi) with step s = alpha (hi - lo) / (2^b - 1); an entry whose code would
+ * leave [0, 2^b - 1] is an outlier: it keeps its current (error-fed) value in full precision,
+ * feeds no error forward, and gets code 0 in the packed stream.  Each row's alpha is found by a
+ * search for the target outlier density: the smallest alpha (finest grid) with at most
+ * floor(density n) outliers, by doubling alpha from 1 until the row is feasible (at most
+ * max_doublings times) and then `steps` bisection steps in log2 alpha between the last
+ * infeasible value (2^-8 when alpha = 1 is already feasible) and the feasible one; the result
+ * is always a feasible alpha.  Natural column order, one grid per row.  SYNCHRONIZES `stream`
+ * once per doubling round.
+ *
+ *   d_W, w_dtype, m, n, d_U, d_dead, d_delta   as gq_quantize_layer (reverse = 0).
+ *   bits          2..8.   density  0..1.   steps  0..60 (20 usual).   max_doublings  0..30.
+ *   d_codes       m x ceil(n*b/32) uint32, written (outliers have code 0).
+ *   d_scales      m fp32, written (the step s of each row).   d_zeros  m uint8, written.
+ *   d_alpha       m doubles, written: the chosen alpha of each row.
+ *   d_row_ptr     m + 1 int64, written: CSR row offsets of the outliers.
+ *   d_col_idx     nnz_capacity int32, written: column of each outlier (ascending in a row).
+ *   d_values      nnz_capacity fp32, written: the kept value of each outlier (dequantized
+ *                 weight = value there, scale * (code - zero) elsewhere).
+ *   nnz_capacity  room in d_col_idx / d_values; m * floor(density n) always suffices.
+ *   d_loss        3 doubles, written as by gq_quantize_layer ([2], the Theorem 5 sum over all
+ *                 columns, is not a bound here).
+ *   d_ws          workspace of at least gq_ssqr_workspace_size(m, n) bytes.
+ * Device-detected errors: GQ_ERR_NO_FIT (some row is still infeasible after max_doublings),
+ * GQ_ERR_WORKSPACE (more outliers than nnz_capacity; the CSR arrays then hold the first ones).
+ */
+gq_status gq_ssqr_quantize_layer(const void* d_W, gq_dtype w_dtype, int64_t m, int64_t n,
+                                 const float* d_U, const uint8_t* d_dead, const double* d_delta,
+                                 int bits, double density, int steps, int max_doublings,
+                                 uint32_t* d_codes, float* d_scales, uint8_t* d_zeros,
+                                 double* d_alpha, int64_t* d_row_ptr, int32_t* d_col_idx,
+                                 float* d_values, int64_t nnz_capacity, double* d_loss,
+                                 void* d_ws, size_t ws_bytes, gq_stream_t stream);
+
 /*
  * The ZSIC column factors kappa_j = U_jj / geomean(U_kk) ("WaterSIC", section 2) of a factor
  * from gq_prepare_hinv(_ordered), exactly as gq_quantize_layer uses them with spacing = 1; a
@@ -275,9 +318,10 @@ size_t gq_huffman_workspace_size(int64_t count);
  *
  *   d_codes      count int32, device, read.  1 <= count <= 2^31 - 1.  The values may span at
  *                most 4096 consecutive integers (symbol k is the value min + k).
- *   d_stream     stream_words uint64, device, written (zeroed first): the codewords of d_codes
- *                in order, MSB first (stream bit i is bit 63 - i % 64 of word i / 64).  Room
- *                for count words (64 bits a code) always suffices.
+ *   d_stream     stream_words uint64, device: the codewords of d_codes in order, MSB first
+ *                (stream bit i is bit 63 - i % 64 of word i / 64), in the first
+ *                ceil(total bits / 64) words (zeroed, then written); later words are not
+ *                touched.  Room for count words (64 bits a code) always suffices.
  *   d_lengths    4096 uint8, device, written: the codeword length of symbol k (0 = unused).
  *   d_codewords  4096 uint64, device, written: the canonical codeword of symbol k (symbols in
  *                order of (length, k) take consecutive values, shifted left at each new length).

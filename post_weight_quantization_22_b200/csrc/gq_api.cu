@@ -200,7 +200,6 @@ gq_status gq_prepare_hinv_ordered(const double* d_H, int64_t n, double damp, gq_
     return gq_prepare_hinv(d_H, n, damp, o, d_U, d_dead, d_delta, d_ws, ws_bytes, stream);
   if (n < 1 || n > kMaxN || !(damp >= 0.0)) return GQ_ERR_INVALID_ARG;
   if (!d_H || !d_U || !d_dead || !d_delta || !d_ws || !d_perm) return GQ_ERR_INVALID_ARG;
-  if (o == GQ_ORDER_MIN_PIVOT) return GQ_ERR_UNSUPPORTED;  // no device implementation yet
   if (!aligned256(d_ws) || ws_bytes < prepare_ws_bytes(n)) return GQ_ERR_WORKSPACE;
   gq_status st = ensure_device_setup();
   if (st != GQ_OK) return st;
@@ -287,6 +286,46 @@ gq_status gq_quantize_layer_ordered(const void* d_W, gq_dtype w_dtype, int64_t m
   if (!d_perm || !cfg || cfg->reverse) return GQ_ERR_INVALID_ARG;
   return quantize_common(d_W, w_dtype, m, n, d_U, d_dead, d_delta, cfg, d_perm, d_codes,
                          d_scales, d_zeros, d_loss, d_ws, ws_bytes, stream);
+}
+
+size_t gq_ssqr_workspace_size(int64_t m, int64_t n) {
+  if (m < 1 || m > kMaxM || n < 1 || n > kMaxN) return 0;
+  return ssqr_ws_bytes(m, n);
+}
+
+gq_status gq_ssqr_quantize_layer(const void* d_W, gq_dtype w_dtype, int64_t m, int64_t n,
+                                 const float* d_U, const uint8_t* d_dead, const double* d_delta,
+                                 int bits, double density, int steps, int max_doublings,
+                                 uint32_t* d_codes, float* d_scales, uint8_t* d_zeros,
+                                 double* d_alpha, int64_t* d_row_ptr, int32_t* d_col_idx,
+                                 float* d_values, int64_t nnz_capacity, double* d_loss,
+                                 void* d_ws, size_t ws_bytes, gq_stream_t stream) {
+  if (m < 1 || m > kMaxM || n < 1 || n > kMaxN) return GQ_ERR_INVALID_ARG;
+  if (w_dtype != GQ_BF16 && w_dtype != GQ_FP32) return GQ_ERR_INVALID_ARG;
+  if (bits < 2 || bits > 8 || !(density >= 0.0 && density <= 1.0)) return GQ_ERR_INVALID_ARG;
+  if (steps < 0 || steps > 60 || max_doublings < 0 || max_doublings > 30 || nnz_capacity < 0)
+    return GQ_ERR_INVALID_ARG;
+  if (!d_W || !d_U || !d_codes || !d_scales || !d_zeros || !d_alpha || !d_row_ptr || !d_loss ||
+      !d_ws)
+    return GQ_ERR_INVALID_ARG;
+  if (nnz_capacity > 0 && (!d_col_idx || !d_values)) return GQ_ERR_INVALID_ARG;
+  if (!aligned256(d_ws) || ws_bytes < ssqr_ws_bytes(m, n)) return GQ_ERR_WORKSPACE;
+  if ((reinterpret_cast<uintptr_t>(d_U) & 15u) != 0 ||
+      (reinterpret_cast<uintptr_t>(d_row_ptr) & 7u) != 0 ||
+      (reinterpret_cast<uintptr_t>(d_alpha) & 7u) != 0)
+    return GQ_ERR_INVALID_ARG;
+  gq_status st = ensure_device_setup();
+  if (st != GQ_OK) return st;
+  QuantArgs a{};
+  a.W = d_W; a.wt = w_dtype; a.m = m; a.n = n; a.U = d_U; a.dead = d_dead; a.delta = d_delta;
+  a.cfg = gq_quant_cfg{bits, 0, 0, 3, 1.25f, 0, 0};
+  a.codes = d_codes; a.scales = d_scales; a.zeros = d_zeros; a.loss = d_loss; a.ws = d_ws;
+  a.perm = nullptr;
+  SsqrArgs o{};
+  o.density = density; o.steps = steps; o.max_doublings = max_doublings; o.alpha = d_alpha;
+  o.row_ptr = reinterpret_cast<long long*>(d_row_ptr); o.col_idx = d_col_idx;
+  o.values = d_values; o.capacity = nnz_capacity;
+  return run_ssqr(a, o, (cudaStream_t)stream);  // synchronizes per doubling round
 }
 
 gq_status gq_zsic_spacing(const float* d_U, int64_t n, double* d_kappa, gq_stream_t stream) {

@@ -148,6 +148,123 @@ __global__ void __launch_bounds__(256) build_m_perm_kernel(const double* H, int6
   }
 }
 
+// ---------------------------------------------------------------------------------------
+// Greedy min-pivot order ("The Geometry of LLM Quantization", section 2.3: Theorem 5's bound is
+// (1/4) sum s^2 D over the LDL pivots D of the Hessian in the quantization order, so taking
+// the smallest remaining Schur-complement pivot at every elimination step tightens it).  The
+// elimination runs in panels of kMpW pivots on the full symmetric H_d in original indexing:
+// one CTA per panel does the pivot steps (argmin of the current Schur diagonal over the
+// remaining columns, ties to the lowest index; the Schur column at the pivot from the panel's
+// earlier columns; the diagonal updated in place), then one fp64 GEMM applies the panel's
+// rank-kMpW update to the whole matrix.  Eliminated rows and columns become zero, as in the
+// rank-one form.  Babai decides the columns in the reverse of the elimination order, so that
+// reversal is the processing order.  No kernel waits on another: the CTAs of one launch never
+// depend on each other, and consecutive launches are ordered by the stream.
+// ---------------------------------------------------------------------------------------
+constexpr int kMpW = 32;  // pivots per panel
+
+// A (full symmetric, n x lda) = H with the dead fix and the damping, both triangles
+__global__ void build_full_kernel(const double* H, int64_t n, int64_t lda, const WsHeader* hdr,
+                                  double* A) {
+  const int64_t j = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+  const int64_t i = blockIdx.y;
+  if (j >= n) return;
+  double v = H[i * n + j];
+  if (i == j) {
+    if (v == 0.0) v = 1.0;
+    v += hdr->scratch[0];
+  }
+  A[i * lda + j] = v;
+}
+
+// The w pivot steps of one panel.  Lp[i][kk] holds the Schur column of the kk-th pivot of the
+// panel (row i; 0 for rows eliminated before it, the pivot itself on the pivot's row), Dp[kk]
+// the pivot; d[i] the current Schur diagonal, elim[i] whether column i is eliminated.
+__global__ void __launch_bounds__(1024, 1) minpivot_panel_kernel(const double* A, int64_t lda,
+                                                                 int64_t n, int64_t k0, int w,
+                                                                 double* d, int* elim,
+                                                                 double* Lp, double* Dp,
+                                                                 int* order, WsHeader* hdr) {
+  __shared__ double s_v[32];
+  __shared__ int s_i[32];
+  __shared__ int s_p;
+  __shared__ double s_d;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  for (int64_t i = tid; i < n; i += 1024)
+    if (!elim[i]) d[i] = A[i * lda + i];
+  __syncthreads();
+  for (int kk = 0; kk < w; ++kk) {
+    double best = INFINITY;
+    int bi = 0x7fffffff;
+    for (int64_t i = tid; i < n; i += 1024) {
+      if (elim[i]) continue;
+      // NaN compares as +inf, so every remaining column is a candidate and the winner is
+      // always a remaining index (at least one remains at every step)
+      const double v = d[i] == d[i] ? d[i] : INFINITY;
+      if (v < best || (v == best && (int)i < bi)) { best = v; bi = (int)i; }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const double ov = __shfl_xor_sync(0xffffffffu, best, o);
+      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+      if (ov < best || (ov == best && oi < bi)) { best = ov; bi = oi; }
+    }
+    if (lane == 0) { s_v[warp] = best; s_i[warp] = bi; }
+    __syncthreads();
+    if (warp == 0) {
+      best = s_v[lane];
+      bi = s_i[lane];
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const double ov = __shfl_xor_sync(0xffffffffu, best, o);
+        const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+        if (ov < best || (ov == best && oi < bi)) { best = ov; bi = oi; }
+      }
+      if (lane == 0) { s_p = bi; s_d = best; }
+    }
+    __syncthreads();
+    const int p = s_p;
+    double D = s_d;
+    if (!(D > 0.0) || !(D < INFINITY)) {  // reported; the rest of the order is then undefined
+      if (tid == 0) record_status(hdr, GQ_ERR_NOT_PD);
+      D = 1.0;
+    }
+    const double rD = 1.0 / D;
+    for (int64_t i = tid; i < n; i += 1024) {
+      double c = 0.0;
+      if (!elim[i]) {
+        c = A[(int64_t)p * lda + i];  // = A[i][p] (both triangles are kept)
+        for (int j = 0; j < kk; ++j) c -= Lp[i * kMpW + j] * Lp[(int64_t)p * kMpW + j] / Dp[j];
+        if (i != p) d[i] -= c * c * rD;
+      }
+      Lp[i * kMpW + kk] = c;
+    }
+    __syncthreads();
+    if (tid == 0) {
+      Lp[(int64_t)p * kMpW + kk] = D;
+      Dp[kk] = D;
+      elim[p] = 1;
+      order[k0 + kk] = p;
+    }
+    __syncthreads();
+  }
+}
+
+// Ls[i][j] = Lp[i][j] / Dp[j] (the left factor of the panel's update A -= Ls Lp^T)
+__global__ void minpivot_scale_kernel(const double* Lp, const double* Dp, int64_t n, int w,
+                                      double* Ls) {
+  const int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+  if (e >= n * kMpW) return;
+  const int j = (int)(e % kMpW);
+  Ls[e] = j < w ? Lp[e] / Dp[j] : 0.0;
+}
+
+// processing order = elimination order reversed
+__global__ void reverse_order_kernel(const int* order, int64_t n, int* perm) {
+  const int64_t k = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+  if (k < n) perm[k] = order[n - 1 - k];
+}
+
 // 1/p for p > 0: the hardware reciprocal estimate (rcp.approx.ftz.f64, about 2^-22 relative)
 // refined by two Newton-Raphson steps r <- r + r (1 - p r), each squaring the relative error,
 // to fp64 precision.  It replaces an IEEE division on the leaf's per-pivot critical path; the
@@ -395,6 +512,14 @@ struct PrepLayout {
   double* Dinv;  // ceil(n / 64) x 64 x 64: the inverted 64-wide leaves
   double* tbuf;  // doubling scratch of the diagonal super-block inverses
   int* pmark;    // n ints: occurrence marks when checking a caller's permutation
+  // min-pivot elimination (before M is built; A lives in T): panel columns Lp and Ls (n x 32),
+  // Schur diagonal d, elimination flags, panel pivots, elimination order
+  double* mpL;
+  double* mpLs;
+  double* mpd;
+  double* mpD;
+  int* mpelim;
+  int* mporder;
   // int8 digit planes (split path only): for every super-panel K with rows below it, the rows
   // sp1..n-1 of its columns of L (kept until the call ends, read by three streams), and one
   // block row of the inverse as the second operand of the inverse's products
@@ -432,6 +557,23 @@ static PrepLayout prep_layout(void* ws, int64_t n) {
   L.Dinv = c.take<double>((size_t)((n + kNB - 1) / kNB) * kNB * kNB);
   L.tbuf = c.take<double>(trtri_tbuf_elems(kSuper) + 1);
   L.pmark = c.take<int>((size_t)n);
+  {
+    const size_t need = (size_t)n * kMpW * 2 + (size_t)n + kMpW + (size_t)n;  // doubles
+    if ((size_t)n * m_ld(n) >= need) {  // inside M
+      double* b = L.M;
+      L.mpL = b; L.mpLs = b + (size_t)n * kMpW; L.mpd = L.mpLs + (size_t)n * kMpW;
+      L.mpD = L.mpd + n;
+      L.mpelim = reinterpret_cast<int*>(L.mpD + kMpW);
+      L.mporder = L.mpelim + n;
+    } else {
+      L.mpL = c.take<double>((size_t)n * kMpW);
+      L.mpLs = c.take<double>((size_t)n * kMpW);
+      L.mpd = c.take<double>((size_t)n);
+      L.mpD = c.take<double>(kMpW);
+      L.mpelim = c.take<int>((size_t)n);
+      L.mporder = c.take<int>((size_t)n);
+    }
+  }
   L.ldig = nullptr; L.lex = nullptr; L.xdig = nullptr; L.xex = nullptr;
   if (use_split(n)) {
     const int64_t lrows = lrow_offset(n, (n + kSuper - 1) / kSuper);
@@ -547,7 +689,6 @@ static cudaError_t prep_streams(PrepStreams** out) {
 
 cudaError_t launch_prepare(const double* H, int64_t n, double damp, int order, int* perm,
                            float* U, uint8_t* dead, double* delta, void* ws, cudaStream_t s0) {
-  if (order == GQ_ORDER_MIN_PIVOT) return cudaErrorNotSupported;
   PrepLayout L = prep_layout(ws, n);
   const int64_t ldm = m_ld(n);
   int dev = 0, sms = 148;
@@ -567,6 +708,37 @@ cudaError_t launch_prepare(const double* H, int64_t n, double damp, int order, i
   GQ_TRY(cudaGetLastError());
   if (order == GQ_ORDER_ACT) {
     act_order_kernel<<<(unsigned)((n + kActCols - 1) / kActCols), 1024, 0, s>>>(H, n, perm);
+    count_launches(1);
+    GQ_TRY(cudaGetLastError());
+  } else if (order == GQ_ORDER_MIN_PIVOT) {
+    const int64_t ldm = m_ld(n);
+    double* A = L.T;  // full symmetric H_d (T is not used before the inverse writes it)
+    {
+      dim3 grid((unsigned)((n + 255) / 256), (unsigned)n);
+      build_full_kernel<<<grid, 256, 0, s>>>(H, n, ldm, L.hdr, A);
+      count_launches(1);
+      GQ_TRY(cudaGetLastError());
+    }
+    GQ_TRY(cudaMemsetAsync(L.mpelim, 0, (size_t)n * sizeof(int), s));
+    for (int64_t k0 = 0; k0 < n; k0 += kMpW) {
+      const int w = (int)std::min<int64_t>(kMpW, n - k0);
+      minpivot_panel_kernel<<<1, 1024, 0, s>>>(A, ldm, n, k0, w, L.mpd, L.mpelim, L.mpL, L.mpD,
+                                               L.mporder, L.hdr);
+      count_launches(1);
+      GQ_TRY(cudaGetLastError());
+      if (k0 + w >= n) break;
+      minpivot_scale_kernel<<<(unsigned)((n * kMpW + 255) / 256), 256, 0, s>>>(L.mpL, L.mpD, n,
+                                                                               w, L.mpLs);
+      count_launches(1);
+      GQ_TRY(cudaGetLastError());
+      DgemmCall g{};  // A -= Ls Lp^T over the whole matrix
+      g.M = (int)n; g.N = (int)n; g.K = w; g.batch = 1; g.alpha = -1.0; g.beta_one = 1;
+      g.A = DgemmOperand{L.mpLs, n, kMpW, kMpW, 0, 0, 0, 0};
+      g.B = DgemmOperand{L.mpL, n, kMpW, kMpW, 0, 0, 0, 0}; g.b_nmajor = 0;
+      g.C = A; g.ldc = ldm; g.hdr = L.hdr;
+      GQ_TRY(launch_dgemm(g, s));
+    }
+    reverse_order_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(L.mporder, n, perm);
     count_launches(1);
     GQ_TRY(cudaGetLastError());
   } else if (order == GQ_ORDER_GIVEN) {

@@ -7,16 +7,19 @@
 //
 // One stream of kernels:
 //   range      min / max code (atomics);
-//   histogram  counts of the spanned values (at most kHuffMaxSym; per-CTA shared-memory bins);
+//   histogram  counts of the spanned values (at most kHuffMaxSym; per-CTA shared-memory bins,
+//              the lanes of a warp holding the same value adding with one atomic);
 //   build      one CTA: the used symbols sorted by (count, symbol) with a bitonic sort, the
 //              two-queue Huffman merge (ties take the leaf), depths from the root down, then the
 //              canonical codewords (consecutive within a length, shifted left at each new
 //              length) and the total length;
 //   tile sums  the code lengths of each 4096-code tile;
 //   scan       exclusive scan of the tile sums (one CTA);
-//   encode     each CTA scans its tile's lengths in shared memory and ORs every codeword into
-//              the stream, MSB first in 64-bit words (stream bit i = bit 63 - i % 64 of word
-//              i / 64; a codeword may straddle two words).
+//   zero       the stream words that will receive bits (the total is known now);
+//   encode     each CTA scans its tile's lengths in shared memory; each thread assembles its
+//              codewords word by word in a register and ORs the words into the stream, MSB
+//              first in 64-bit words (stream bit i = bit 63 - i % 64 of word i / 64; a
+//              codeword may straddle two words).
 // Device-detected failures (more than kHuffMaxSym values spanned, a codeword longer than 63
 // bits, a stream too small for the total) are recorded in the workspace status and skip the
 // encoding.
@@ -93,9 +96,16 @@ __global__ void huff_hist_kernel(const int* codes, int64_t count, const int* sta
   if (K > kHuffMaxSym) return;  // the same for every CTA; the build kernel reports it
   for (int i = threadIdx.x; i < K; i += blockDim.x) bins[i] = 0ull;
   __syncthreads();
-  for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < count;
-       e += (int64_t)gridDim.x * blockDim.x)
-    atomicAdd(&bins[codes[e] - lo], 1ull);
+  // the lanes of a warp that hold the same symbol add their count with one atomic (low-bit
+  // codes have a handful of distinct values, so per-code atomics would serialise on them)
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  const int64_t e_end = (count + stride - 1) / stride * stride;  // every lane runs each round
+  for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < e_end; e += stride) {
+    const int sym = e < count ? codes[e] - lo : -1;
+    const unsigned peers = __match_any_sync(0xffffffffu, sym);
+    if (sym >= 0 && (threadIdx.x & 31) == __ffs(peers) - 1)
+      atomicAdd(&bins[sym], (unsigned long long)__popc(peers));
+  }
   __syncthreads();
   for (int i = threadIdx.x; i < K; i += blockDim.x)
     if (bins[i]) atomicAdd(&hist[i], bins[i]);
@@ -304,22 +314,45 @@ __global__ void __launch_bounds__(kHuffThreads) huff_encode_kernel(
     if (sym[i] >= 0) mine += sl[sym[i]];
   }
   unsigned long long pos = tile_off[blockIdx.x] + block_exclusive_scan(mine, wsum, nullptr);
+  // this thread's codewords are assembled word by word in a register; a word is ORed into the
+  // stream when the bits move on (its first and last words may be shared with the neighbours,
+  // hence the atomics; the count drops from one per code to about one per word)
+  unsigned long long buf = 0ull, bw = pos >> 6;
 #pragma unroll
   for (int i = 0; i < kHuffPer; ++i) {
     if (sym[i] < 0) continue;
     const int ln = sl[sym[i]];
     const unsigned long long cw = sw[sym[i]];
-    const unsigned long long wi = pos >> 6;
+    if ((pos >> 6) != bw) {
+      if (buf) atomicOr(&stream[bw], buf);
+      bw = pos >> 6;
+      buf = 0ull;
+    }
     const int o = (int)(pos & 63ull);
     if (o + ln <= 64) {
-      atomicOr(&stream[wi], cw << (64 - o - ln));
+      buf |= cw << (64 - o - ln);
     } else {
       const int h = o + ln - 64;  // bits that spill into the next word
-      atomicOr(&stream[wi], cw >> h);
-      atomicOr(&stream[wi + 1], cw << (64 - h));
+      buf |= cw >> h;
+      atomicOr(&stream[bw], buf);
+      ++bw;
+      buf = cw << (64 - h);
     }
     pos += (unsigned long long)ln;
   }
+  if (buf) atomicOr(&stream[bw], buf);
+}
+
+// Zero the stream words that will receive bits (the total is known once the code is built).
+__global__ void huff_zero_kernel(const int* state, const long long* info, int64_t nwords,
+                                 unsigned long long* stream) {
+  if (state[2]) return;
+  const long long total = info[2];
+  int64_t used = (total + 63) / 64;
+  if (used > nwords) used = nwords;
+  for (int64_t w = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; w < used;
+       w += (int64_t)gridDim.x * blockDim.x)
+    stream[w] = 0ull;
 }
 
 cudaError_t huffman_init_attributes() {
@@ -334,8 +367,6 @@ cudaError_t launch_huffman(const int* codes, int64_t count, unsigned long long* 
   const int64_t ntiles = (count + kHuffTile - 1) / kHuffTile;
   cudaError_t e;
   if ((e = cudaMemsetAsync(L.hdr, 0, sizeof(WsHeader), s))) return e;
-  if ((e = cudaMemsetAsync(stream_words, 0, (size_t)nwords * sizeof(unsigned long long), s)))
-    return e;
   huff_init_kernel<<<1, 1024, 0, s>>>(L.state, L.hist);
   const unsigned grid = (unsigned)std::min<int64_t>((count + 255) / 256, 148 * 8);
   huff_range_kernel<<<grid, 256, 0, s>>>(codes, count, L.state);
@@ -345,9 +376,11 @@ cudaError_t launch_huffman(const int* codes, int64_t count, unsigned long long* 
   huff_tile_sum_kernel<<<(unsigned)ntiles, kHuffThreads, 0, s>>>(codes, count, L.state, lengths,
                                                                  L.tile_sum);
   huff_scan_kernel<<<1, 1024, 0, s>>>(L.state, L.tile_sum, ntiles, L.tile_off);
+  huff_zero_kernel<<<(unsigned)std::min<int64_t>((nwords + 255) / 256, 148 * 8), 256, 0, s>>>(
+      L.state, info, nwords, stream_words);
   huff_encode_kernel<<<(unsigned)ntiles, kHuffThreads, 0, s>>>(codes, count, L.state, lengths,
                                                                words, L.tile_off, stream_words);
-  count_launches(7);
+  count_launches(8);
   return cudaGetLastError();
 }
 

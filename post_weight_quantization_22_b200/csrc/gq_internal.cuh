@@ -78,6 +78,18 @@ struct QuantArgs {
   const int* perm;  // processing order (null: natural, or reversed when cfg.reverse)
 };
 size_t quantize_ws_bytes(int64_t m, int64_t n, const gq_quant_cfg& cfg);
+// SSQR outlier search (cfg.clip = 3, one grid per row, natural order): its workspace, and the
+// search + final pass with the outliers written as CSR.
+size_t ssqr_ws_bytes(int64_t m, int64_t n);
+struct SsqrArgs {
+  double density;
+  int steps, max_doublings;
+  double* alpha;        // m, out
+  long long* row_ptr;   // m + 1, out
+  int* col_idx;         // capacity, out
+  float* values;        // capacity, out
+  int64_t capacity;
+};
 cudaError_t launch_zsic_spacing(const float* U, int64_t n, double* kappa, cudaStream_t s);
 
 // ---- canonical Huffman coding of int32 codes ----
@@ -88,6 +100,8 @@ cudaError_t launch_huffman(const int* codes, int64_t count, unsigned long long* 
                            long long* info, void* ws, cudaStream_t s);
 // Returns GQ_OK or an error; the clip-free ladder synchronizes the stream per round.
 gq_status run_quantize(const QuantArgs& a, cudaStream_t s);
+// Synchronizes the stream once per doubling round of the search.
+gq_status run_ssqr(const QuantArgs& a, const SsqrArgs& o, cudaStream_t s);
 
 constexpr int kBlock = 128;  // columns per GPTQ block (lazy-update rank)
 
@@ -171,12 +185,15 @@ cudaError_t launch_split_gemm(double* C, int64_t ldc, int M, int N, const SplitO
 struct LazyTcMaps {
   CUtensorMap ahi, alo, bhi, blo;
 };
-// E_hi / E_lo: rows x 128 fp32; U_hi / U_lo: n x n fp32 with leading dimension ldu (mult. of 4)
+// E_hi / E_lo: rows x n fp32 with leading dimension ldE (multiple of 4); U_hi / U_lo: n x n
+// fp32 with leading dimension ldu (multiple of 4)
 cudaError_t lazy_tc_make_maps(LazyTcMaps* maps, const float* Ehi, const float* Elo, int64_t rows,
-                              const float* Uhi, const float* Ulo, int64_t n, int64_t ldu);
-// Wf[:, j1:jend] -= (E_hi + E_lo) (U_hi + U_lo)[j0:j0+128, j1:jend]  (3xTF32), rows < k_rows;
-// jend is n or j1 + 128k.
+                              int64_t ldE, const float* Uhi, const float* Ulo, int64_t n,
+                              int64_t ldu);
+// Wf[:, j1:jend] -= (E_hi + E_lo)[:, k0:k0+K] (U_hi + U_lo)[k0:k0+K, j1:jend]  (3xTF32),
+// rows < k_rows; K and k0 multiples of 16, k0 + K <= n.
 cudaError_t launch_lazy_tc(const LazyTcMaps& maps, float* Wf, int64_t n, int64_t k_rows,
-                           int64_t j0, int64_t j1, int64_t jend, WsHeader* hdr, cudaStream_t s);
+                           int64_t k0, int K, int64_t j1, int64_t jend, WsHeader* hdr,
+                           cudaStream_t s);
 
 }  // namespace gq

@@ -41,8 +41,9 @@ constexpr uint32_t kBulkChunk = 32768;
 struct QLayout {
   WsHeader* hdr;
   float* Wf;        // k x n work matrix (compact rows)
-  float* Ehi[2];    // k x 128 scaled errors of a block, tf32 part (blocks alternate buffers)
-  float* Elo[2];    // k x 128 fp32 remainder (E = Ehi + Elo)
+  float* Ehi;       // k x ldE scaled errors of every column, tf32 part (processing order)
+  float* Elo;       // k x ldE fp32 remainder (E = Ehi + Elo)
+  int64_t ldE;
   float* Uhi;       // n x ldu tf32 part of U (columns >= n zero)
   float* Ulo;       // n x ldu fp32 remainder
   int64_t ldu;
@@ -61,18 +62,26 @@ struct QLayout {
   int* iperm;       // n: processing position of each original column (ordered calls)
   double* kappa;    // n: ZSIC column factors in processing order
   int* codes32;     // m x n int32 codes in processing order (unconstrained lattice only)
+  // outlier search (SSQR) only
+  double* alpha_d;  // per-row grid factor 2^t of the current pass
+  uint8_t* omask;   // m x ldc8: 1 where the entry is an outlier (processing order)
+  float* oval;      // m x ldE: the kept value of each outlier
+  int* ocount;      // per-row outlier count of the last pass
+  double* s_lo;     // per-row search bracket in log2 alpha: lo infeasible (or -8), hi feasible
+  double* s_hi;
+  double* s_mid;
+  int* s_feas;
   size_t bytes;
 };
 
-static QLayout q_layout(void* ws, int64_t m, int64_t n, bool unbounded) {
+static QLayout q_layout(void* ws, int64_t m, int64_t n, bool unbounded, bool outliers) {
   Carver c(ws);
   QLayout L;
   L.hdr = c.take<WsHeader>(1);
   L.Wf = c.take<float>((size_t)m * n);
-  for (int i = 0; i < 2; ++i) {
-    L.Ehi[i] = c.take<float>((size_t)m * kBlock);
-    L.Elo[i] = c.take<float>((size_t)m * kBlock);
-  }
+  L.ldE = (n + 31) / 32 * 32;  // rows start on 16-byte boundaries for TMA
+  L.Ehi = c.take<float>((size_t)m * L.ldE);
+  L.Elo = c.take<float>((size_t)m * L.ldE);
   L.ldu = (n + 31) / 32 * 32;
   L.Uhi = c.take<float>((size_t)n * L.ldu);
   L.Ulo = c.take<float>((size_t)n * L.ldu);
@@ -91,13 +100,27 @@ static QLayout q_layout(void* ws, int64_t m, int64_t n, bool unbounded) {
   L.iperm = c.take<int>((size_t)n);
   L.kappa = c.take<double>((size_t)n);
   L.codes32 = unbounded ? c.take<int>((size_t)m * n) : nullptr;
+  L.alpha_d = nullptr; L.omask = nullptr; L.oval = nullptr; L.ocount = nullptr;
+  L.s_lo = nullptr; L.s_hi = nullptr; L.s_mid = nullptr; L.s_feas = nullptr;
+  if (outliers) {
+    L.alpha_d = c.take<double>(m);
+    L.omask = c.take<uint8_t>((size_t)m * L.ldc8);
+    L.oval = c.take<float>((size_t)m * L.ldE);
+    L.ocount = c.take<int>(m);
+    L.s_lo = c.take<double>(m);
+    L.s_hi = c.take<double>(m);
+    L.s_mid = c.take<double>(m);
+    L.s_feas = c.take<int>(m);
+  }
   L.bytes = c.off;
   return L;
 }
 
 size_t quantize_ws_bytes(int64_t m, int64_t n, const gq_quant_cfg& cfg) {
-  return q_layout(nullptr, m, n, cfg.clip == 2).bytes;
+  return q_layout(nullptr, m, n, cfg.clip == 2, false).bytes;
 }
+
+size_t ssqr_ws_bytes(int64_t m, int64_t n) { return q_layout(nullptr, m, n, false, true).bytes; }
 
 // ------------------------------------------------------------------------------------------
 // setup kernels
@@ -161,9 +184,11 @@ __global__ void perm_invert_kernel(const int* perm, int64_t n, int* iperm, WsHea
 }
 
 // per-row grid from the (dead-zeroed) row: one warp per row
+// clip: 1 min-max grid; 0 clip-free (centred, step widened by the ladder factor alpha);
+// 2 unconstrained lattice; 3 outliers (centred, step widened by the fp64 factor alpha_d).
 __global__ void q_row_grid_kernel(const float* Wf, int64_t n, int64_t k_rows, const int* rowlist,
-                                  int bits, int clip, const float* alpha, double* row_s,
-                                  double* row_z, float* scales, uint8_t* zeros) {
+                                  int bits, int clip, const float* alpha, const double* alpha_d,
+                                  double* row_s, double* row_z, float* scales, uint8_t* zeros) {
   int64_t rr = blockIdx.x * (int64_t)(blockDim.x / 32) + threadIdx.x / 32;
   int lane = threadIdx.x & 31;
   if (rr >= k_rows) return;
@@ -187,7 +212,8 @@ __global__ void q_row_grid_kernel(const float* Wf, int64_t n, int64_t k_rows, co
       s = (dhi - dlo) / maxq;
       z = 0.0;
     } else {
-      s = (double)alpha[row] * (dhi - dlo) / maxq;
+      const double al = clip == 3 ? alpha_d[row] : (double)alpha[row];
+      s = al * (dhi - dlo) / maxq;
       z = rint(maxq * 0.5 - (dhi + dlo) / (2.0 * s));
     }
     row_s[row] = s;
@@ -288,8 +314,9 @@ struct ColArgs {
   const float* U;
   int bits;
   int clip;
-  float* Ehi;
+  float* Ehi;       // k x ldE, column j0 + c of the block at [row][j0 + c]
   float* Elo;
+  int64_t ldE;
   uint8_t* codes8;
   int64_t ldc8;
   int* codes32;  // unconstrained lattice: int32 codes (processing order, row stride n), or null
@@ -301,6 +328,9 @@ struct ColArgs {
   double* row_e2;
   double* row_bnd;
   int* overflow;
+  uint8_t* omask;  // clip 3: outlier flags (row stride ldc8), kept values (row stride ldE), counts
+  float* oval;
+  int* ocount;
 };
 
 // Thread layout: a warp owns 8 rows; lane (g, t) = (lane / 4, lane % 4) holds row g and, of
@@ -385,6 +415,11 @@ __global__ void __launch_bounds__(kColThreads, 1) colloop_kernel(ColArgs a) {
   int ovf = 0;
   const bool clip = a.clip == 1;      // clamp to [0, 2^b - 1]
   const bool track = a.clip == 0;     // clip-free: flag codes outside the range for the ladder
+  // outliers ("The Geometry of LLM Quantization", section 3, SSQR): an entry whose code leaves
+  // [0, 2^b - 1] keeps its current (error-fed) value in full precision: error 0, nothing fed
+  // forward, code 0 in the packed stream
+  const bool outl = a.clip == 3;
+  int nout = 0;
 
 #pragma unroll 1
   for (int T = 0; T < kTiles; ++T) {
@@ -425,6 +460,8 @@ __global__ void __launch_bounds__(kColThreads, 1) colloop_kernel(ColArgs a) {
     }
     const double cmin = -z, cmax = maxq - z;  // code range in the domain c - z
     double ea[2] = {0.0, 0.0}, ca[2] = {0.0, 0.0};  // this lane's errors / codes (cols 2t, 2t+1)
+    double xa[2] = {0.0, 0.0};                      // this lane's values before rounding
+    bool oa[2] = {false, false};                    // ... and whether they are outliers
     double d2sum = 0.0;
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
@@ -437,10 +474,14 @@ __global__ void __launch_bounds__(kColThreads, 1) colloop_kernel(ColArgs a) {
         double sj = s, isj = inv_s;
         if constexpr (Z) { sj = s * kap[jj]; isj = inv_s * kinv[jj]; }
         double c = rint_small(x * isj);
+        bool out = false;
         if (clip) c = fmin(fmax(c, cmin), cmax);
-        else if (track && (c < cmin || c > cmax)) ovf = 1;
-        const double e = fma(-sj, c, x) * id;  // (x - s_j c) / U_jj
-        if (t == town) { ea[pown] = e; ca[pown] = c; }
+        else if (track || outl) out = c < cmin || c > cmax;
+        if (track && out) ovf = 1;
+        out = out && outl;
+        nout += out ? 1 : 0;
+        const double e = out ? 0.0 : fma(-sj, c, x) * id;  // (x - s_j c) / U_jj
+        if (t == town) { ea[pown] = e; ca[pown] = c; xa[pown] = x; oa[pown] = out; }
         e2 = fma(e, e, e2);
 #pragma unroll
         for (int p = 0; p < 2; ++p)
@@ -456,16 +497,26 @@ __global__ void __launch_bounds__(kColThreads, 1) colloop_kernel(ColArgs a) {
         float2 hi2, lo2;
         hi2.x = tf32_rna(f0); hi2.y = tf32_rna(f1);
         lo2.x = f0 - hi2.x; lo2.y = f1 - hi2.y;
-        *reinterpret_cast<float2*>(a.Ehi + rr * kBlock + col) = hi2;
-        *reinterpret_cast<float2*>(a.Elo + rr * kBlock + col) = lo2;
+        *reinterpret_cast<float2*>(a.Ehi + rr * a.ldE + j0 + col) = hi2;
+        *reinterpret_cast<float2*>(a.Elo + rr * a.ldE + j0 + col) = lo2;
         if (a.codes32) {  // unconstrained lattice: z = 0, any integer
           int* cp = a.codes32 + row * n + j0 + col;
           cp[0] = (int)ca[0];
           if (col + 1 < bw) cp[1] = (int)ca[1];
         } else {
           uint8_t* cp = a.codes8 + row * a.ldc8 + j0 + col;
-          cp[0] = (uint8_t)(int)fmin(fmax(ca[0] + z, 0.0), maxq);
-          if (col + 1 < bw) cp[1] = (uint8_t)(int)fmin(fmax(ca[1] + z, 0.0), maxq);
+          cp[0] = oa[0] ? (uint8_t)0 : (uint8_t)(int)fmin(fmax(ca[0] + z, 0.0), maxq);
+          if (col + 1 < bw) cp[1] = oa[1] ? (uint8_t)0 : (uint8_t)(int)fmin(fmax(ca[1] + z, 0.0), maxq);
+          if (outl) {
+            uint8_t* mp = a.omask + row * a.ldc8 + j0 + col;
+            float* vp = a.oval + row * a.ldE + j0 + col;
+            mp[0] = oa[0] ? 1 : 0;
+            if (oa[0]) vp[0] = (float)xa[0];
+            if (col + 1 < bw) {
+              mp[1] = oa[1] ? 1 : 0;
+              if (oa[1]) vp[1] = (float)xa[1];
+            }
+          }
         }
       }
     }
@@ -494,6 +545,10 @@ __global__ void __launch_bounds__(kColThreads, 1) colloop_kernel(ColArgs a) {
   if (act && t == 0) {
     if (j0 == 0) { a.row_e2[row] = e2; a.row_bnd[row] = bnd; a.overflow[row] = ovf_q; }
     else { a.row_e2[row] += e2; a.row_bnd[row] += bnd; a.overflow[row] |= ovf_q; }
+    if (outl) {  // every lane of the quad counted the row's outliers
+      if (j0 == 0) a.ocount[row] = nout;
+      else a.ocount[row] += nout;
+    }
   }
 }
 
@@ -507,7 +562,8 @@ __global__ void __launch_bounds__(128) pack_kernel(const TW* W, const uint8_t* d
                                                    const int* codes32, int reverse, int bits,
                                                    int group,
                                                    int64_t ngroups, const float* scales,
-                                                   const uint8_t* zeros, uint32_t* codes,
+                                                   const uint8_t* zeros, const uint8_t* omask,
+                                                   const float* oval, int64_t ldE, uint32_t* codes,
                                                    double* row_d2) {
   const int64_t r = blockIdx.x;
   const uint8_t* crow = codes8 + r * ldc8;
@@ -551,6 +607,7 @@ __global__ void __launch_bounds__(128) pack_kernel(const TW* W, const uint8_t* d
     float code = codes32 ? (float)crow32[pc] : (float)crow[pc];
     const double sk = kappa ? (double)s * kappa[pc] : (double)s;
     double d = (double)w0 - sk * (double)(code - z);
+    if (omask && omask[r * ldc8 + pc]) d = (double)w0 - (double)oval[r * ldE + pc];
     acc += d * d;
   }
   __shared__ double red[4];
@@ -655,14 +712,17 @@ static cudaError_t colloop_dispatch(int group, int spacing, const ColArgs& ca, c
   }
 }
 
-// Two streams per call, forked from and joined back into the caller's stream: A (higher
-// priority) runs the column loop of each block and the lazy update of the next block's 128
-// columns; B runs the lazy update of all later columns, overlapped with the next block's
-// column loop (look-ahead of one block).  One set per host thread and device, kept.
+// Three streams per call, forked from and joined back into the caller's stream (priority
+// high to low): A runs the column loop of each block, the update of the next block's columns
+// and, at the end of a super-block, the update of the next super-block; B runs the update of
+// the rest of the current super-block after each block; C runs the update of all columns after
+// the next super-block once a super-block is done.  One set per host thread and device, kept.
+constexpr int kSuperBlocks = 8;  // blocks per super-block (1024 columns)
 struct QuantStreams {
   bool ready = false;
-  cudaStream_t a = nullptr, b = nullptr;
-  cudaEvent_t fork = nullptr, col[2] = {}, rest[2] = {}, join[2] = {};
+  cudaStream_t a = nullptr, b = nullptr, c = nullptr;
+  cudaEvent_t fork = nullptr, col[4] = {}, mid[4] = {}, sbdone = nullptr, far[2] = {},
+              join[3] = {};
 };
 thread_local QuantStreams t_quant_streams[128];
 
@@ -676,9 +736,12 @@ static cudaError_t quant_streams(QuantStreams** out) {
     int least = 0, greatest = 0;
     if ((e = cudaDeviceGetStreamPriorityRange(&least, &greatest))) return e;
     if ((e = cudaStreamCreateWithPriority(&q.a, cudaStreamNonBlocking, greatest))) return e;
-    if ((e = cudaStreamCreateWithPriority(&q.b, cudaStreamNonBlocking, least))) return e;
-    cudaEvent_t* evs[] = {&q.fork, &q.col[0], &q.col[1], &q.rest[0], &q.rest[1], &q.join[0],
-                          &q.join[1]};
+    if ((e = cudaStreamCreateWithPriority(&q.b, cudaStreamNonBlocking, (least + greatest) / 2)))
+      return e;
+    if ((e = cudaStreamCreateWithPriority(&q.c, cudaStreamNonBlocking, least))) return e;
+    cudaEvent_t* evs[] = {&q.fork,   &q.col[0], &q.col[1], &q.col[2],  &q.col[3],  &q.mid[0],
+                          &q.mid[1], &q.mid[2], &q.mid[3], &q.sbdone, &q.far[0], &q.far[1],
+                          &q.join[0], &q.join[1], &q.join[2]};
     for (cudaEvent_t* ev : evs)
       if ((e = cudaEventCreateWithFlags(ev, cudaEventDisableTiming))) return e;
     q.ready = true;
@@ -687,12 +750,11 @@ static cudaError_t quant_streams(QuantStreams** out) {
   return cudaSuccess;
 }
 
-gq_status run_quantize(const QuantArgs& a, cudaStream_t s) {
+// Per-call set-up shared by every pass: status cleared, ladder factors 1, U split into tf32
+// parts, the per-block prepared U (and the ZSIC factors), the inverse permutation.
+static gq_status quant_setup(const QuantArgs& a, const QLayout& L, cudaStream_t s) {
   const int64_t m = a.m, n = a.n;
-  QLayout L = q_layout(a.ws, m, n, a.cfg.clip == 2);
   const gq_quant_cfg& cfg = a.cfg;
-  const int G = cfg.group_size;
-  const int64_t ngroups = G ? (n + G - 1) / G : 1;
   Q_TRY(cudaMemsetAsync(L.hdr, 0, sizeof(WsHeader), s));
   q_reset_kernel<<<(unsigned)((m + 255) / 256), 256, 0, s>>>(m, L.alpha, L.overflow, a.loss);
   count_launches(1);
@@ -720,88 +782,182 @@ gq_status run_quantize(const QuantArgs& a, cudaStream_t s) {
     count_launches(1);
     Q_TRY(cudaGetLastError());
   }
+  return GQ_OK;
+}
+
+// One pass of the column loop over k_rows rows (all rows, or the rows listed in rowlist): the
+// fp32 work matrix loaded, the per-row grids, then the blocks with their lazy updates.
+static gq_status quant_pass(const QuantArgs& a, const QLayout& L, int64_t k_rows,
+                            const int* rowlist, cudaStream_t s) {
+  const int64_t n = a.n;
+  const gq_quant_cfg& cfg = a.cfg;
+  const int G = cfg.group_size;
+  const int64_t ngroups = G ? (n + G - 1) / G : 1;
+  const int nblocks = (int)((n + kBlock - 1) / kBlock);
+  if (a.perm) {
+    const size_t sm = (size_t)n * sizeof(float);
+    if (a.wt == GQ_BF16)
+      q_load_perm_kernel<__nv_bfloat16><<<(unsigned)k_rows, 256, sm, s>>>(
+          static_cast<const __nv_bfloat16*>(a.W), n, rowlist, a.dead, a.perm, L.Wf);
+    else
+      q_load_perm_kernel<float><<<(unsigned)k_rows, 256, sm, s>>>(
+          static_cast<const float*>(a.W), n, rowlist, a.dead, a.perm, L.Wf);
+    count_launches(1);
+    Q_TRY(cudaGetLastError());
+  } else {
+    int64_t total = k_rows * n;
+    unsigned grid = (unsigned)std::min<int64_t>((total + 255) / 256, 148 * 64);
+    if (a.wt == GQ_BF16)
+      q_load_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(
+          static_cast<const __nv_bfloat16*>(a.W), n, k_rows, rowlist, a.dead, cfg.reverse, L.Wf);
+    else
+      q_load_kernel<float><<<grid, 256, 0, s>>>(static_cast<const float*>(a.W), n, k_rows,
+                                                rowlist, a.dead, cfg.reverse, L.Wf);
+    count_launches(1);
+    Q_TRY(cudaGetLastError());
+  }
+  if (G == 0) {
+    unsigned grid = (unsigned)((k_rows + 7) / 8);
+    q_row_grid_kernel<<<grid, 256, 0, s>>>(L.Wf, n, k_rows, rowlist, cfg.bits, cfg.clip,
+                                           L.alpha, L.alpha_d, L.row_s, L.row_z, a.scales,
+                                           a.zeros);
+    count_launches(1);
+    Q_TRY(cudaGetLastError());
+  }
+  LazyTcMaps maps;
+  Q_TRY(lazy_tc_make_maps(&maps, L.Ehi, L.Elo, k_rows, L.ldE, L.Uhi, L.Ulo, n, L.ldu));
+  // Two-level lazy updates (GPTQ's lazy batch, applied twice): the columns are grouped into
+  // super-blocks of kSuperBlocks blocks.  After block b (columns [j0, j1)) of super-block S:
+  //   A: W[:, next block] -= E_b U[b, next block]         (if the next block is in S)
+  //   B: W[:, rest of S]  -= E_b U[b, rest of S]
+  // and once S is done:
+  //   A: W[:, next super-block]      -= E_S U[S, next super-block]   (depth 1024)
+  //   C: W[:, everything after that] -= E_S U[S, ...]               (depth 1024)
+  // so the fp32 work matrix beyond the current super-block is read and written once per
+  // super-block instead of once per block.  E of every column is kept (no buffer reuse).
+  // Waits (two streams never read-modify-write the same columns at once): A's update after
+  // block b (which writes block b + 1) waits for B's update after block b - 1 (which writes
+  // blocks b + 1 .. the end of S), so the column loop of a block always sees every earlier
+  // block's contribution; A's next-super-block update waits for C's update after the previous
+  // super-block (both write those columns).
+  QuantStreams* qs = nullptr;
+  Q_TRY(quant_streams(&qs));
+  cudaStream_t sa = qs->a, sb = qs->b, sc = qs->c;
+  Q_TRY(cudaEventRecord(qs->fork, s));
+  Q_TRY(cudaStreamWaitEvent(sa, qs->fork, 0));
+  Q_TRY(cudaStreamWaitEvent(sb, qs->fork, 0));
+  Q_TRY(cudaStreamWaitEvent(sc, qs->fork, 0));
+  bool far_pending = false;
+  int far_idx = 0;
+  for (int b = 0; b < nblocks; ++b) {
+    const int64_t j0 = (int64_t)b * kBlock;
+    const int bw = (int)std::min<int64_t>(kBlock, n - j0);
+    const int64_t j1 = j0 + bw;
+    const int bi = b % kSuperBlocks;
+    const int64_t sb0 = (int64_t)(b - bi) * kBlock;
+    const int64_t sb1 = std::min<int64_t>(sb0 + (int64_t)kSuperBlocks * kBlock, n);
+    ColArgs ca{};
+    ca.Ublk = L.Ublk; ca.hdr = L.hdr;
+    ca.Wf = L.Wf; ca.n = n; ca.k_rows = k_rows; ca.rowlist = rowlist; ca.j0 = j0; ca.bw = bw;
+    ca.U = a.U; ca.bits = cfg.bits; ca.clip = cfg.clip; ca.Ehi = L.Ehi; ca.Elo = L.Elo;
+    ca.ldE = L.ldE;
+    ca.codes8 = L.codes8;
+    ca.codes32 = L.codes32;
+    ca.ldc8 = L.ldc8; ca.scales = a.scales; ca.zeros = a.zeros; ca.ngroups = ngroups;
+    ca.row_s = L.row_s; ca.row_z = L.row_z; ca.row_e2 = L.row_e2; ca.row_bnd = L.row_bnd;
+    ca.overflow = L.overflow;
+    ca.omask = L.omask; ca.oval = L.oval; ca.ocount = L.ocount;
+    Q_TRY(colloop_dispatch(G, cfg.spacing, ca, sa));
+    if (j1 < sb1) {  // the rest of this super-block takes block b's errors (depth 128)
+      const int64_t jn = std::min<int64_t>(j1 + kBlock, sb1);
+      if (jn < sb1) {
+        Q_TRY(cudaEventRecord(qs->col[b & 3], sa));
+        Q_TRY(cudaStreamWaitEvent(sb, qs->col[b & 3], 0));
+        Q_TRY(launch_lazy_tc(maps, L.Wf, n, k_rows, j0, bw, jn, sb1, L.hdr, sb));
+        Q_TRY(cudaEventRecord(qs->mid[b & 3], sb));
+      }
+      // B's update after block b - 1 also writes the next block: finish it first
+      if (bi >= 1) Q_TRY(cudaStreamWaitEvent(sa, qs->mid[(b - 1) & 3], 0));
+      Q_TRY(launch_lazy_tc(maps, L.Wf, n, k_rows, j0, bw, j1, jn, L.hdr, sa));
+    } else if (sb1 < n) {  // super-block [sb0, sb1) done: everything after it (depth 1024)
+      const int64_t sb2 = std::min<int64_t>(sb1 + (int64_t)kSuperBlocks * kBlock, n);
+      const int depth = (int)(sb1 - sb0);
+      if (sb2 < n) {
+        Q_TRY(cudaEventRecord(qs->sbdone, sa));
+        Q_TRY(cudaStreamWaitEvent(sc, qs->sbdone, 0));
+      }
+      if (far_pending) Q_TRY(cudaStreamWaitEvent(sa, qs->far[(far_idx - 1) & 1], 0));
+      Q_TRY(launch_lazy_tc(maps, L.Wf, n, k_rows, sb0, depth, sb1, sb2, L.hdr, sa));
+      far_pending = false;
+      if (sb2 < n) {
+        Q_TRY(launch_lazy_tc(maps, L.Wf, n, k_rows, sb0, depth, sb2, n, L.hdr, sc));
+        Q_TRY(cudaEventRecord(qs->far[far_idx & 1], sc));
+        far_pending = true;
+        ++far_idx;
+      }
+    }
+  }
+  Q_TRY(cudaEventRecord(qs->join[1], sb));
+  Q_TRY(cudaEventRecord(qs->join[2], sc));
+  Q_TRY(cudaStreamWaitEvent(sa, qs->join[1], 0));
+  Q_TRY(cudaStreamWaitEvent(sa, qs->join[2], 0));
+  Q_TRY(cudaEventRecord(qs->join[0], sa));
+  Q_TRY(cudaStreamWaitEvent(s, qs->join[0], 0));
+  return GQ_OK;
+}
+
+// Packing (codes by original column; an outlier's kept value in the error norm), per-row
+// ||w0 - q||^2, and the three loss numbers.
+static gq_status quant_finish(const QuantArgs& a, const QLayout& L, cudaStream_t s) {
+  const int64_t m = a.m, n = a.n;
+  const gq_quant_cfg& cfg = a.cfg;
+  const int G = cfg.group_size;
+  const int64_t ngroups = G ? (n + G - 1) / G : 1;
+  const int* iperm = a.perm ? L.iperm : nullptr;
+  const double* kappa = cfg.spacing ? L.kappa : nullptr;
+  const size_t pack_smem = (a.perm && !L.codes32) ? (size_t)n : 0;
+  if (a.wt == GQ_BF16)
+    pack_kernel<__nv_bfloat16><<<(unsigned)m, 128, pack_smem, s>>>(
+        static_cast<const __nv_bfloat16*>(a.W), a.dead, n, L.codes8, L.ldc8, iperm, kappa,
+        L.codes32, cfg.reverse, cfg.bits, G, ngroups, a.scales, a.zeros, L.omask, L.oval,
+        L.ldE, a.codes, L.row_d2);
+  else
+    pack_kernel<float><<<(unsigned)m, 128, pack_smem, s>>>(
+        static_cast<const float*>(a.W), a.dead, n, L.codes8, L.ldc8, iperm, kappa, L.codes32,
+        cfg.reverse, cfg.bits, G, ngroups, a.scales, a.zeros, L.omask, L.oval, L.ldE, a.codes,
+        L.row_d2);
+  count_launches(1);
+  Q_TRY(cudaGetLastError());
+  q_reduce_kernel<<<1, 1024, 0, s>>>(m, L.row_e2, L.row_bnd, L.row_d2, a.delta, a.loss);
+  count_launches(1);
+  Q_TRY(cudaGetLastError());
+  return GQ_OK;
+}
+
+// Writes GQ_ERR_NO_FIT into the status word unless an earlier error is there (synchronizes).
+static gq_status record_no_fit(const QLayout& L, cudaStream_t s) {
+  int code = GQ_ERR_NO_FIT, cur = 0;
+  Q_TRY(cudaMemcpyAsync(&cur, &L.hdr->status, sizeof(int), cudaMemcpyDeviceToHost, s));
+  Q_TRY(cudaStreamSynchronize(s));
+  if (cur == 0)
+    Q_TRY(cudaMemcpyAsync(&L.hdr->status, &code, sizeof(int), cudaMemcpyHostToDevice, s));
+  Q_TRY(cudaStreamSynchronize(s));
+  return GQ_OK;
+}
+
+gq_status run_quantize(const QuantArgs& a, cudaStream_t s) {
+  const int64_t m = a.m;
+  const gq_quant_cfg& cfg = a.cfg;
+  QLayout L = q_layout(a.ws, m, a.n, cfg.clip == 2, false);
+  gq_status st = quant_setup(a, L, s);
+  if (st != GQ_OK) return st;
   int64_t k_rows = m;
   const int* rowlist = nullptr;
-  const int nblocks = (int)((n + kBlock - 1) / kBlock);
   const int max_rounds = cfg.clip ? 1 : cfg.ladder_max + 1;
   int rounds_run = 0;
   for (int round = 0; round < max_rounds; ++round) {
     rounds_run = round;
-    if (a.perm) {
-      const size_t sm = (size_t)n * sizeof(float);
-      if (a.wt == GQ_BF16)
-        q_load_perm_kernel<__nv_bfloat16><<<(unsigned)k_rows, 256, sm, s>>>(
-            static_cast<const __nv_bfloat16*>(a.W), n, rowlist, a.dead, a.perm, L.Wf);
-      else
-        q_load_perm_kernel<float><<<(unsigned)k_rows, 256, sm, s>>>(
-            static_cast<const float*>(a.W), n, rowlist, a.dead, a.perm, L.Wf);
-      count_launches(1);
-      Q_TRY(cudaGetLastError());
-    } else {
-      int64_t total = k_rows * n;
-      unsigned grid = (unsigned)std::min<int64_t>((total + 255) / 256, 148 * 64);
-      if (a.wt == GQ_BF16)
-        q_load_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(
-            static_cast<const __nv_bfloat16*>(a.W), n, k_rows, rowlist, a.dead, cfg.reverse, L.Wf);
-      else
-        q_load_kernel<float><<<grid, 256, 0, s>>>(static_cast<const float*>(a.W), n, k_rows,
-                                                  rowlist, a.dead, cfg.reverse, L.Wf);
-      count_launches(1);
-      Q_TRY(cudaGetLastError());
-    }
-    if (G == 0) {
-      unsigned grid = (unsigned)((k_rows + 7) / 8);
-      q_row_grid_kernel<<<grid, 256, 0, s>>>(L.Wf, n, k_rows, rowlist, cfg.bits, cfg.clip,
-                                             L.alpha, L.row_s, L.row_z, a.scales, a.zeros);
-      count_launches(1);
-      Q_TRY(cudaGetLastError());
-    }
-    LazyTcMaps maps[2];
-    for (int i = 0; i < 2; ++i)
-      Q_TRY(lazy_tc_make_maps(&maps[i], L.Ehi[i], L.Elo[i], k_rows, L.Uhi, L.Ulo, n, L.ldu));
-    // Blocks on stream A; the lazy update after block b is split: the next block's 128 columns
-    // on A (the next column loop needs them), all later columns on B.  Block b's errors live in
-    // buffer b & 1 until its later-column update is done (the column loop of block b + 2, which
-    // reuses the buffer, waits for it through the next-block update of block b + 1).
-    QuantStreams* qs = nullptr;
-    Q_TRY(quant_streams(&qs));
-    cudaStream_t sa = qs->a, sb = qs->b;
-    Q_TRY(cudaEventRecord(qs->fork, s));
-    Q_TRY(cudaStreamWaitEvent(sa, qs->fork, 0));
-    Q_TRY(cudaStreamWaitEvent(sb, qs->fork, 0));
-    bool rest_pending = false;
-    for (int b = 0; b < nblocks; ++b) {
-      const int64_t j0 = (int64_t)b * kBlock;
-      const int bw = (int)std::min<int64_t>(kBlock, n - j0);
-      ColArgs ca{};
-      ca.Ublk = L.Ublk; ca.hdr = L.hdr;
-      ca.Wf = L.Wf; ca.n = n; ca.k_rows = k_rows; ca.rowlist = rowlist; ca.j0 = j0; ca.bw = bw;
-      ca.U = a.U; ca.bits = cfg.bits; ca.clip = cfg.clip; ca.Ehi = L.Ehi[b & 1];
-      ca.Elo = L.Elo[b & 1];
-      ca.codes8 = L.codes8;
-      ca.codes32 = L.codes32;
-      ca.ldc8 = L.ldc8; ca.scales = a.scales; ca.zeros = a.zeros; ca.ngroups = ngroups;
-      ca.row_s = L.row_s; ca.row_z = L.row_z; ca.row_e2 = L.row_e2; ca.row_bnd = L.row_bnd;
-      ca.overflow = L.overflow;
-      Q_TRY(colloop_dispatch(G, cfg.spacing, ca, sa));
-      const int64_t j1 = j0 + bw;
-      if (j1 >= n) continue;
-      const int64_t jn = std::min<int64_t>(j1 + kBlock, n);
-      Q_TRY(cudaEventRecord(qs->col[b & 1], sa));
-      if (rest_pending) Q_TRY(cudaStreamWaitEvent(sa, qs->rest[(b - 1) & 1], 0));
-      Q_TRY(launch_lazy_tc(maps[b & 1], L.Wf, n, k_rows, j0, j1, jn, L.hdr, sa));
-      rest_pending = false;
-      if (jn < n) {
-        Q_TRY(cudaStreamWaitEvent(sb, qs->col[b & 1], 0));
-        Q_TRY(launch_lazy_tc(maps[b & 1], L.Wf, n, k_rows, j0, jn, n, L.hdr, sb));
-        Q_TRY(cudaEventRecord(qs->rest[b & 1], sb));
-        rest_pending = true;
-      }
-    }
-    Q_TRY(cudaEventRecord(qs->join[1], sb));
-    Q_TRY(cudaStreamWaitEvent(sa, qs->join[1], 0));
-    Q_TRY(cudaEventRecord(qs->join[0], sa));
-    Q_TRY(cudaStreamWaitEvent(s, qs->join[0], 0));
+    if ((st = quant_pass(a, L, k_rows, rowlist, s)) != GQ_OK) return st;
     if (cfg.clip) break;
     // clip-free: collect rows whose codes left [0, 2^b - 1] and rerun them on a wider step
     Q_TRY(cudaMemsetAsync(L.counter, 0, sizeof(int), s));
@@ -814,14 +970,7 @@ gq_status run_quantize(const QuantArgs& a, cudaStream_t s) {
     Q_TRY(cudaStreamSynchronize(s));
     if (cnt == 0) break;
     if (round == max_rounds - 1) {
-      int code = GQ_ERR_NO_FIT;
-      // first error wins: write only if the status word is still clear
-      int cur = 0;
-      Q_TRY(cudaMemcpyAsync(&cur, &L.hdr->status, sizeof(int), cudaMemcpyDeviceToHost, s));
-      Q_TRY(cudaStreamSynchronize(s));
-      if (cur == 0) Q_TRY(cudaMemcpyAsync(&L.hdr->status, &code, sizeof(int),
-                                          cudaMemcpyHostToDevice, s));
-      Q_TRY(cudaStreamSynchronize(s));
+      if ((st = record_no_fit(L, s)) != GQ_OK) return st;
       break;
     }
     k_rows = cnt;
@@ -832,20 +981,198 @@ gq_status run_quantize(const QuantArgs& a, cudaStream_t s) {
     Q_TRY(cudaMemcpyAsync(&L.hdr->ladder_rounds, &rr, sizeof(int), cudaMemcpyHostToDevice, s));
     Q_TRY(cudaStreamSynchronize(s));
   }
-  const int* iperm = a.perm ? L.iperm : nullptr;
-  const double* kappa = cfg.spacing ? L.kappa : nullptr;
-  const size_t pack_smem = (a.perm && !L.codes32) ? (size_t)n : 0;
-  if (a.wt == GQ_BF16)
-    pack_kernel<__nv_bfloat16><<<(unsigned)m, 128, pack_smem, s>>>(
-        static_cast<const __nv_bfloat16*>(a.W), a.dead, n, L.codes8, L.ldc8, iperm, kappa,
-        L.codes32, cfg.reverse, cfg.bits, G, ngroups, a.scales, a.zeros, a.codes, L.row_d2);
-  else
-    pack_kernel<float><<<(unsigned)m, 128, pack_smem, s>>>(
-        static_cast<const float*>(a.W), a.dead, n, L.codes8, L.ldc8, iperm, kappa, L.codes32,
-        cfg.reverse, cfg.bits, G, ngroups, a.scales, a.zeros, a.codes, L.row_d2);
+  return quant_finish(a, L, s);
+}
+
+// ---------------------------------------------------------------------------------------------
+// SSQR ("The Geometry of LLM Quantization", section 3: a few weights are kept in full precision
+// as sparse floats, the rest quantized on a low-bit grid, the scale set by a binary search for
+// a target outlier density).  Reading: the clip-free centred grid of each row widened by alpha;
+// alpha is the smallest factor (finest grid) with at most limit = floor(density n) outliers,
+// found in log2 alpha by doubling from 1 until feasible and then a fixed number of bisection
+// steps between the last infeasible value (or -8 when 1 is feasible) and the feasible one.
+// ---------------------------------------------------------------------------------------------
+// 2^x; exact for integer x, the correctly rounded-or-close exp2 otherwise
+__device__ __forceinline__ double pow2_real(double x) {
+  if (x == floor(x) && fabs(x) < 1000.0) return ldexp(1.0, (int)x);
+  return exp2(x);
+}
+
+enum SsqrMode {
+  kSsqrInit = 0,      // hi = 0 (alpha 1), every row still to be checked
+  kSsqrCheck = 1,     // after a pass of the listed / unchecked rows: feasibility, new list
+  kSsqrDouble = 2,    // before a doubling pass: infeasible rows lo = hi, hi += 1
+  kSsqrMid = 3,       // before a bisection pass: mid = (lo + hi) / 2, alpha = 2^mid
+  kSsqrBisect = 4,    // after a bisection pass: feasible -> hi = mid, else lo = mid
+  kSsqrFinal = 5      // alpha = 2^hi for the final pass, copied out
+};
+
+__global__ void ssqr_state_kernel(int64_t m, int mode, int limit, const int* ocount, double* lo,
+                                  double* hi, double* mid, int* feas, double* alpha_d,
+                                  int* rowlist, int* counter, double* alpha_out) {
+  const int64_t r = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+  if (r >= m) return;
+  switch (mode) {
+    case kSsqrInit:
+      hi[r] = 0.0;
+      lo[r] = -8.0;
+      feas[r] = 0;
+      alpha_d[r] = 1.0;
+      break;
+    case kSsqrCheck:
+      if (!feas[r]) {
+        if (ocount[r] <= limit) {
+          feas[r] = 1;
+        } else {
+          rowlist[atomicAdd(counter, 1)] = (int)r;
+        }
+      }
+      break;
+    case kSsqrDouble:
+      if (!feas[r]) {
+        lo[r] = hi[r];
+        hi[r] += 1.0;
+        alpha_d[r] = pow2_real(hi[r]);
+      }
+      break;
+    case kSsqrMid:
+      mid[r] = 0.5 * (lo[r] + hi[r]);
+      alpha_d[r] = pow2_real(mid[r]);
+      break;
+    case kSsqrBisect:
+      if (ocount[r] <= limit) hi[r] = mid[r];
+      else lo[r] = mid[r];
+      break;
+    case kSsqrFinal:
+      alpha_d[r] = pow2_real(hi[r]);
+      alpha_out[r] = alpha_d[r];
+      break;
+  }
+}
+
+// row_ptr = exclusive scan of the per-row outlier counts (one CTA); a total beyond the caller's
+// capacity records GQ_ERR_WORKSPACE (the fill below then writes nothing past the capacity).
+__global__ void __launch_bounds__(1024) csr_rowptr_kernel(int64_t m, const int* ocount,
+                                                          int64_t capacity, long long* row_ptr,
+                                                          WsHeader* hdr) {
+  __shared__ long long warp_tot[32];
+  __shared__ long long carry;
+  if (threadIdx.x == 0) carry = 0;
+  __syncthreads();
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  for (int64_t base = 0; base < m; base += 1024) {
+    const int64_t r = base + threadIdx.x;
+    long long v = r < m ? (long long)ocount[r] : 0;
+    long long x = v;  // inclusive warp scan
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const long long y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
+    }
+    if (lane == 31) warp_tot[warp] = x;
+    __syncthreads();
+    if (warp == 0) {
+      long long t = warp_tot[lane];
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const long long y = __shfl_up_sync(0xffffffffu, t, o);
+        if (lane >= o) t += y;
+      }
+      warp_tot[lane] = t;  // inclusive over warps
+    }
+    __syncthreads();
+    const long long before = carry + (warp > 0 ? warp_tot[warp - 1] : 0) + x - v;
+    if (r < m) row_ptr[r] = before;
+    __syncthreads();
+    if (threadIdx.x == 1023) carry = before + v;
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) {
+    row_ptr[m] = carry;
+    if (carry > capacity) record_status(hdr, GQ_ERR_WORKSPACE);
+  }
+}
+
+// Column indices (ascending) and kept values of each row's outliers; one CTA of 128 threads per
+// row, columns in chunks of 128 with a block-wide prefix of the flags.
+__global__ void __launch_bounds__(128) csr_fill_kernel(int64_t n, const uint8_t* omask,
+                                                       int64_t ldc8, const float* oval,
+                                                       int64_t ldE, const long long* row_ptr,
+                                                       int64_t capacity, int* col_idx,
+                                                       float* values) {
+  __shared__ int warp_cnt[4];
+  const int64_t r = blockIdx.x;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  long long pos = row_ptr[r];
+  for (int64_t c0 = 0; c0 < n; c0 += 128) {
+    const int64_t c = c0 + threadIdx.x;
+    const bool f = c < n && omask[r * ldc8 + c];
+    const unsigned bal = __ballot_sync(0xffffffffu, f);
+    if (lane == 0) warp_cnt[warp] = __popc(bal);
+    __syncthreads();
+    int off = 0;
+    for (int w = 0; w < warp; ++w) off += warp_cnt[w];
+    const int total = warp_cnt[0] + warp_cnt[1] + warp_cnt[2] + warp_cnt[3];
+    if (f) {
+      const long long idx = pos + off + __popc(bal & ((1u << lane) - 1u));
+      if (idx < capacity) {
+        col_idx[idx] = (int)c;
+        values[idx] = oval[r * ldE + c];
+      }
+    }
+    pos += total;
+    __syncthreads();
+  }
+}
+
+gq_status run_ssqr(const QuantArgs& a, const SsqrArgs& o, cudaStream_t s) {
+  const int64_t m = a.m, n = a.n;
+  QLayout L = q_layout(a.ws, m, n, false, true);
+  gq_status st = quant_setup(a, L, s);
+  if (st != GQ_OK) return st;
+  const int limit = (int)floor(o.density * (double)n + 1e-9);
+  const unsigned rgrid = (unsigned)((m + 255) / 256);
+  auto state = [&](int mode) -> gq_status {
+    ssqr_state_kernel<<<rgrid, 256, 0, s>>>(m, mode, limit, L.ocount, L.s_lo, L.s_hi, L.s_mid,
+                                            L.s_feas, L.alpha_d, L.rowlist, L.counter, o.alpha);
+    count_launches(1);
+    Q_TRY(cudaGetLastError());
+    return GQ_OK;
+  };
+  auto check = [&](int* cnt) -> gq_status {
+    Q_TRY(cudaMemsetAsync(L.counter, 0, sizeof(int), s));
+    gq_status e = state(kSsqrCheck);
+    if (e != GQ_OK) return e;
+    Q_TRY(cudaMemcpyAsync(cnt, L.counter, sizeof(int), cudaMemcpyDeviceToHost, s));
+    Q_TRY(cudaStreamSynchronize(s));
+    return GQ_OK;
+  };
+  // doubling from alpha = 1 until every row is feasible
+  if ((st = state(kSsqrInit)) != GQ_OK) return st;
+  if ((st = quant_pass(a, L, m, nullptr, s)) != GQ_OK) return st;
+  int cnt = 0;
+  if ((st = check(&cnt)) != GQ_OK) return st;
+  for (int d = 0; d < o.max_doublings && cnt > 0; ++d) {
+    if ((st = state(kSsqrDouble)) != GQ_OK) return st;
+    if ((st = quant_pass(a, L, cnt, L.rowlist, s)) != GQ_OK) return st;
+    if ((st = check(&cnt)) != GQ_OK) return st;
+  }
+  if (cnt > 0 && (st = record_no_fit(L, s)) != GQ_OK) return st;
+  // bisection in log2 alpha, every row at once
+  for (int k = 0; k < o.steps; ++k) {
+    if ((st = state(kSsqrMid)) != GQ_OK) return st;
+    if ((st = quant_pass(a, L, m, nullptr, s)) != GQ_OK) return st;
+    if ((st = state(kSsqrBisect)) != GQ_OK) return st;
+  }
+  // the result: every row at its feasible alpha, packed, losses, outliers as CSR
+  if ((st = state(kSsqrFinal)) != GQ_OK) return st;
+  if ((st = quant_pass(a, L, m, nullptr, s)) != GQ_OK) return st;
+  if ((st = quant_finish(a, L, s)) != GQ_OK) return st;
+  csr_rowptr_kernel<<<1, 1024, 0, s>>>(m, L.ocount, o.capacity, o.row_ptr, L.hdr);
   count_launches(1);
   Q_TRY(cudaGetLastError());
-  q_reduce_kernel<<<1, 1024, 0, s>>>(m, L.row_e2, L.row_bnd, L.row_d2, a.delta, a.loss);
+  csr_fill_kernel<<<(unsigned)m, 128, 0, s>>>(n, L.omask, L.ldc8, L.oval, L.ldE, o.row_ptr,
+                                             o.capacity, o.col_idx, o.values);
   count_launches(1);
   Q_TRY(cudaGetLastError());
   return GQ_OK;

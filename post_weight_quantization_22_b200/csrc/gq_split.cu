@@ -301,6 +301,11 @@ __global__ void __launch_bounds__(kSThreads, 1)
           tc::fence_after_sync();
           const uint32_t a0 = tc::smem_u32(base + s * kSStage);
           const uint32_t b0 = a0 + kSplitDigits * kSATile;
+          // the stage's descriptors once; an operand at a constant byte offset from the stage
+          // is the same descriptor with offset / 16 added to its start-address field (the
+          // field holds address / 16 in 14 bits, and no address here reaches 2^18)
+          const uint64_t ad0 = tc::sdesc(a0, 16, 512, tc::kLayoutSW64);
+          const uint64_t bd0 = tc::sdesc(b0, 16, 512, tc::kLayoutSW64);
 #pragma unroll
           for (int k = 0; k < kSBK / 32; ++k) {
 #pragma unroll
@@ -309,9 +314,8 @@ __global__ void __launch_bounds__(kSThreads, 1)
               for (int q = 0; p + q < kSplitDigits; ++q) {  // digit pairs of weight >= 2^-7(S+1)
                 // p = 0 is the first pair of class q: it opens the accumulator of the tile
                 const uint32_t acc = (kc == 0 && k == 0 && p == 0) ? 0u : 1u;
-                const uint64_t ad = tc::sdesc(a0 + p * kSATile + k * 32, 16, 512, tc::kLayoutSW64);
-                const uint64_t bd = tc::sdesc(b0 + q * kSBTile + k * 32, 16, 512, tc::kLayoutSW64);
-                tc::mma_i8(tmem + (p + q) * kSBN, ad, bd, kSIdesc, acc);
+                tc::mma_i8(tmem + (p + q) * kSBN, ad0 + (uint64_t)((p * kSATile + k * 32) >> 4),
+                           bd0 + (uint64_t)((q * kSBTile + k * 32) >> 4), kSIdesc, acc);
               }
             }
           }
@@ -352,16 +356,17 @@ __global__ void __launch_bounds__(kSThreads, 1)
 #pragma unroll
       for (int j = 0; j < 32; ++j) acc[j] = 0.0;
       const uint32_t tbase = tmem + ((uint32_t)(quad * 32) << 16) + half * 32;
+      // Classes c and c + 1 weigh 2^-7 apart and every class sum is below 2^23 in magnitude,
+      // so 128 acc_c + acc_(c+1) is exact in int32: one conversion to fp64 per pair (the fp64
+      // conversions, not the loads, are the slow part of this phase).
 #pragma unroll
       for (int c = kSplitDigits - 2; c >= 0; c -= 2) {  // smallest classes first, two per wait
         uint32_t va[32], vb[32];
         tc::tmem_ld32x2(tbase + (c + 1) * kSBN, tbase + c * kSBN, va, vb);
-        const double wa = pow2(-7 * (c + 3)), wb = pow2(-7 * (c + 2));
+        const double w = pow2(-7 * (c + 3));
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          acc[j] = fma((double)(int)va[j], wa, acc[j]);
-          acc[j] = fma((double)(int)vb[j], wb, acc[j]);
-        }
+        for (int j = 0; j < 32; ++j)
+          acc[j] = fma((double)((int)vb[j] * 128 + (int)va[j]), w, acc[j]);
       }
       // the accumulators are in registers: the MMA warp may start the next tile
       tc::fence_before_sync();

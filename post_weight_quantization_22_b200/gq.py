@@ -68,6 +68,11 @@ def _load():
     lib.gq_huffman_workspace_size.argtypes = [I64]
     lib.gq_huffman_encode.restype = I
     lib.gq_huffman_encode.argtypes = [P, I64, P, I64, P, P, P, P, SZ, P]
+    lib.gq_ssqr_workspace_size.restype = SZ
+    lib.gq_ssqr_workspace_size.argtypes = [I64, I64]
+    lib.gq_ssqr_quantize_layer.restype = I
+    lib.gq_ssqr_quantize_layer.argtypes = [P, I, I64, I64, P, P, P, I, ctypes.c_double, I, I, P,
+                                           P, P, P, P, P, P, I64, P, P, SZ, P]
     lib.gq_zsic_spacing.restype = I
     lib.gq_zsic_spacing.argtypes = [P, I64, P, P]
     lib.gq_debug_wait_test.restype = I
@@ -83,7 +88,8 @@ EXPORTED = ("gq_version", "gq_status_string", "gq_hessian_accumulate", "gq_hessi
             "gq_prepare_hinv", "gq_quantize_workspace_size", "gq_quantize_layer",
             "gq_workspace_status", "gq_prepare_hinv_static", "gq_prepare_hinv_ordered",
             "gq_quantize_layer_ordered", "gq_zsic_spacing", "gq_huffman_workspace_size",
-            "gq_huffman_encode", "gq_debug_wait_test", "gq_kernel_launches")
+            "gq_huffman_encode", "gq_debug_wait_test", "gq_kernel_launches",
+            "gq_ssqr_workspace_size", "gq_ssqr_quantize_layer")
 
 
 def _ptr(t):
@@ -289,6 +295,43 @@ def gq_quantize_layer_ordered(W: torch.Tensor, U: torch.Tensor, dead, delta, cfg
                                          ws.numel(), _stream(stream)),
            "gq_quantize_layer_ordered")
     return codes, scales, zeros, loss, ws
+
+
+def gq_ssqr_quantize_layer(W: torch.Tensor, U: torch.Tensor, dead, delta, bits: int,
+                           density: float, steps: int = 20, max_doublings: int = 12,
+                           capacity: int | None = None, ws=None, stream=None):
+    """SSQR on the device: per-row scale search for a target outlier density, outliers kept
+    in full precision.  Returns dict(codes (packed, outliers 0), scales [m], zeros [m],
+    alpha [m] fp64, row_ptr [m+1] int64, col_idx, values (CSR of the outliers), loss, ws)."""
+    m, n = W.shape
+    if not W.is_cuda or not W.is_contiguous():
+        raise ValueError("W must be a contiguous cuda tensor")
+    dev = W.device
+    _need(U, torch.float32, (n, n), "U")
+    if dead is not None:
+        _need(dead, torch.uint8, (n,), "dead")
+    if delta is not None:
+        _need(delta, torch.float64, (1,), "delta")
+    limit = int(density * n + 1e-9)
+    cap = m * max(limit, 0) if capacity is None else int(capacity)
+    codes = torch.empty((m, n_words(n, bits)), dtype=torch.int32, device=dev)
+    scales = torch.empty(m, dtype=torch.float32, device=dev)
+    zeros = torch.empty(m, dtype=torch.uint8, device=dev)
+    alpha = torch.empty(m, dtype=torch.float64, device=dev)
+    row_ptr = torch.empty(m + 1, dtype=torch.int64, device=dev)
+    col_idx = torch.empty(max(cap, 1), dtype=torch.int32, device=dev)
+    values = torch.empty(max(cap, 1), dtype=torch.float32, device=dev)
+    loss = torch.empty(3, dtype=torch.float64, device=dev)
+    ws = workspace(int(LIB.gq_ssqr_workspace_size(m, n)), dev) if ws is None else ws
+    _check(LIB.gq_ssqr_quantize_layer(_ptr(W), _dtype_code(W), m, n, _ptr(U), _ptr(dead),
+                                      _ptr(delta), int(bits), float(density), int(steps),
+                                      int(max_doublings), _ptr(codes), _ptr(scales),
+                                      _ptr(zeros), _ptr(alpha), _ptr(row_ptr), _ptr(col_idx),
+                                      _ptr(values), cap, _ptr(loss), _ptr(ws), ws.numel(),
+                                      _stream(stream)),
+           "gq_ssqr_quantize_layer")
+    return dict(codes=codes, scales=scales, zeros=zeros, alpha=alpha, row_ptr=row_ptr,
+                col_idx=col_idx, values=values, loss=loss, ws=ws)
 
 
 def gq_zsic_spacing(U: torch.Tensor, kappa=None, stream=None) -> torch.Tensor:

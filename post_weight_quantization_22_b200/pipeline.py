@@ -28,8 +28,8 @@ class LayerQuantizer:
     def __init__(self, m: int, n: int, cfg: G.QuantCfg, device="cuda", damp: float = 0.01,
                  max_tokens: int = 65536, order: str | None = None):
         """``order``: None (natural, or reversed when ``cfg.reverse``), or a column order of
-        gq_prepare_hinv_ordered: "act" or "given" (fill ``self.perm`` first)."""
-        if order is not None and order not in ("act", "given"):
+        gq_prepare_hinv_ordered: "act", "min_pivot" or "given" (fill ``self.perm`` first)."""
+        if order is not None and order not in ("act", "min_pivot", "given"):
             raise ValueError(f"unknown order {order!r}")
         if order is not None and cfg.reverse:
             raise ValueError("an order replaces cfg.reverse")

@@ -66,9 +66,9 @@ def test_ordered_entry_points_reject_bad_arguments_without_gpu():
     # unknown order value
     assert L.gq_prepare_hinv_ordered(fake, 16, 0.01, 9, fake, fake, fake, fake, fake, 1 << 20,
                                      None) == 1
-    # the min-pivot order has no device implementation: rejected before any device work
-    assert L.gq_prepare_hinv_ordered(fake, 16, 0.01, 3, fake, fake, fake, fake, fake, 1 << 20,
-                                     None) == 4
+    # the min-pivot order writes the order: without a perm array it is rejected
+    assert L.gq_prepare_hinv_ordered(fake, 16, 0.01, 3, None, fake, fake, fake, fake, 1 << 20,
+                                     None) == 1
     # ACT without a perm array
     assert L.gq_prepare_hinv_ordered(fake, 16, 0.01, 2, None, fake, fake, fake, fake, 1 << 20,
                                      None) == 1
@@ -105,3 +105,15 @@ def test_wait_test_setting_is_host_only_and_checked():
     assert G.LIB.gq_debug_wait_test(0, 2) == 1          # withhold must be 0 or 1
     assert G.LIB.gq_debug_wait_test(4096, 1) == 0       # a host-side setting: no GPU needed
     assert G.LIB.gq_debug_wait_test(0, 0) == 0          # back to the defaults
+
+
+def test_ssqr_entry_rejects_bad_arguments_without_gpu():
+    from post_weight_quantization_22_b200 import gq as G
+    assert G.LIB.gq_ssqr_workspace_size(0, 16) == 0
+    assert G.LIB.gq_ssqr_workspace_size(16, 16) > 0
+    # density outside [0, 1], bits outside 2..8: rejected before any device work
+    args = [None, 0, 16, 16, None, None, None]
+    for bits, density in ((3, -0.1), (3, 1.5), (1, 0.1), (9, 0.1)):
+        rc = G.LIB.gq_ssqr_quantize_layer(*args, bits, density, 20, 12, None, None, None, None,
+                                          None, None, None, 0, None, None, 0, None)
+        assert rc == 1, (bits, density, rc)

@@ -68,7 +68,10 @@ def _compare(g, o, W, bits, group, rows=None, check_loss=True, perm=None):
         floor = 1e-12 * float(np.sum(np.asarray(W, dtype=np.float64) ** 2)) * float(np.mean(np.diag(o["H"])))
         assert abs(g["loss"][0] - o["loss_proxy"]) <= LOSS_REL * o["loss_proxy"] + floor
         assert abs(g["loss"][1] - o["loss_damped"]) <= LOSS_REL * o["loss_damped"] + floor
-        assert abs(g["loss"][2] - o["bound"]) <= 1e-5 * o["bound"]
+        # the bound's steps are fixed by the codes (a group grid comes from the error-fed
+        # weights), so it is held to 1e-5 when every code agrees, else to the loss tolerance
+        bound_tol = 1e-5 if match == 1.0 or not group else LOSS_REL
+        assert abs(g["loss"][2] - o["bound"]) <= bound_tol * o["bound"]
     return match
 
 
@@ -271,7 +274,10 @@ def _huffman_check(codes_dev, stream_words=None):
     prefix code, and the stream equals the oracle's encoding with the device's lengths, bit for
     bit (canonical codewords are fixed by the lengths)."""
     from post_weight_quantization_22_b200 import gq as G
-    out, ln, cw, info, ws = G.gq_huffman_encode(codes_dev, stream_words)
+    words = codes_dev.numel() if stream_words is None else stream_words
+    sentinel = 0x5A5A5A5A5A5A5A5A
+    out = torch.full((max(words, 1),), sentinel, dtype=torch.int64, device="cuda")
+    out, ln, cw, info, ws = G.gq_huffman_encode(codes_dev, out=out)
     assert G.gq_workspace_status(ws)[0] == 0
     codes = codes_dev.cpu().numpy().astype(np.int64).ravel()
     lo, K, total, maxlen = (int(v) for v in info.cpu().numpy())
@@ -289,7 +295,8 @@ def _huffman_check(codes_dev, stream_words=None):
     ref, nbits = O.huffman_encode(sym, ln)
     got = out.cpu().numpy().view(np.uint64)
     assert nbits == total
-    assert np.array_equal(got[:len(ref)], ref) and not got[len(ref):].any()
+    assert np.array_equal(got[:len(ref)], ref)
+    assert np.all(got[len(ref):] == np.uint64(sentinel))  # words past the stream untouched
     return total
 
 
@@ -304,15 +311,16 @@ def test_huffman_encoder_against_oracle(count, spread):
 
 def test_huffman_encoder_reports_span_and_stream_errors():
     """More than 4096 values spanned -> GQ_ERR_UNSUPPORTED; a stream too small for the total ->
-    GQ_ERR_WORKSPACE; nothing is encoded (the stream stays zero)."""
+    GQ_ERR_WORKSPACE; nothing is encoded (the stream buffer is not touched)."""
     from post_weight_quantization_22_b200 import gq as G
     wide = torch.tensor([0, 5000, 3, 3], dtype=torch.int32, device="cuda")
     out, *_, info, ws = G.gq_huffman_encode(wide)
     assert G.gq_workspace_status(ws)[0] == 4
     codes = torch.from_numpy(np.arange(100000, dtype=np.int32) % 64).cuda()
-    out, *_, info, ws = G.gq_huffman_encode(codes, stream_words=10)
+    out = torch.full((10,), 7, dtype=torch.int64, device="cuda")
+    out, *_, info, ws = G.gq_huffman_encode(codes, out=out)
     assert G.gq_workspace_status(ws)[0] == 7
-    assert int(info[2]) == 600000 and not out.any()
+    assert int(info[2]) == 600000 and bool((out == 7).all())
 
 
 def test_unbounded_lattice_codes_and_huffman_rate():
@@ -550,3 +558,129 @@ def test_bounded_wait_runs_out_and_the_next_call_is_clean():
     hfix, _, _ = O.fix_dead_features(H.cpu().numpy(), np.zeros((1, 200)))
     hd, _ = O.dampen(hfix, 0.01)
     assert rel_fro(np.triu(U2.cpu().numpy()), O.hinv_upper_factor(hd)) <= U_REL_DESIGN
+
+
+def _ssqr_compare(gres, o_res, o_alpha, rows, bits, density, n, w0, U):
+    """SSQR parity.  The search: most rows end at the oracle's alpha exactly; a row whose
+    outlier count sits at the limit at some trial alpha can take the other branch when one
+    near-tie code differs (the lazy updates are not bit-identical to the oracle), so for the
+    others the device's alpha must be feasible by the oracle's own count (one entry of slack).
+    Then, at the device's alphas, outlier masks, codes, kept values and steps against the
+    oracle's column loop at those same alphas."""
+    alpha = gres["alpha"].cpu().numpy()[rows]
+    same = np.isclose(alpha, o_alpha, rtol=1e-12, atol=0.0)
+    print(f"ssqr alpha identical on {same.mean():.4f} of rows")
+    assert same.mean() >= 0.75
+    limit = int(np.floor(density * n + 1e-9))
+    at_dev = O.ssqr_columns(w0[rows], U, bits, alpha)
+    assert np.all(at_dev["outlier"].sum(axis=1) <= limit + 1)
+    # CSR -> dense mask / values (original column order == processing order here)
+    rp = gres["row_ptr"].cpu().numpy()
+    ci = gres["col_idx"].cpu().numpy()
+    vv = gres["values"].cpu().numpy()
+    assert rp[0] == 0 and np.all(np.diff(rp) >= 0) and np.all(np.diff(rp) <= limit)
+    mask = np.zeros((len(rows), n), dtype=bool)
+    vals = np.zeros((len(rows), n))
+    for k, r in enumerate(rows):
+        cols = ci[rp[r]:rp[r + 1]]
+        assert np.all(np.diff(cols) > 0)
+        mask[k, cols] = True
+        vals[k, cols] = vv[rp[r]:rp[r + 1]]
+    codes = unpack_np(gres["codes"].cpu().numpy().view(np.uint32), n, bits)[rows]
+    assert float(np.mean(mask == at_dev["outlier"])) >= CODE_MATCH
+    assert float(np.mean(codes == at_dev["codes"])) >= CODE_MATCH
+    # a kept value is the error-fed weight, so it is fixed only where the row's codes and
+    # outlier flags all agree (a permitted code difference moves the row's later values)
+    row_same = np.all(codes == at_dev["codes"], axis=1) & np.all(mask == at_dev["outlier"], axis=1)
+    assert row_same.mean() >= 0.9
+    both = mask & at_dev["outlier"] & row_same[:, None]
+    np.testing.assert_allclose(vals[both], at_dev["Q"][both], rtol=1e-6, atol=1e-7)
+    np.testing.assert_allclose(gres["scales"].cpu().numpy()[rows], at_dev["scales"][:, 0],
+                               rtol=1e-6)
+    return same, at_dev
+
+
+def _ssqr_gpu(W, X, bits, density, steps=20):
+    from post_weight_quantization_22_b200 import gq as G
+    m, n = W.shape
+    H = torch.zeros((n, n), dtype=torch.float64, device="cuda")
+    G.gq_hessian_accumulate(H, X.cuda())
+    U, dead, delta, ws_p = G.gq_prepare_hinv(H, 0.01)
+    res = G.gq_ssqr_quantize_layer(W.cuda(), U, dead, delta, bits, density, steps=steps)
+    torch.cuda.synchronize()
+    assert G.gq_workspace_status(ws_p)[0] == 0
+    assert G.gq_workspace_status(res["ws"])[0] == 0
+    res["U"] = U
+    return res
+
+
+def test_ssqr_search_ragged_against_oracle():
+    """SSQR on the device ("The Geometry of LLM Quantization", section 3): per-row scale search
+    for at most 2 % outliers, outliers kept at their error-fed values, CSR output; 3-bit, a
+    ragged 200 x 700 layer (700 not a multiple of the 128-column block)."""
+    W, X, spec = synth.workload("q_proj_4096x4096", m=200, n=700, T=900)
+    bits, density = 3, 0.02
+    g = _ssqr_gpu(W, X, bits, density)
+    H = O.hessian(X)
+    hfix, w0, _ = O.fix_dead_features(H, W)
+    hd, delta = O.dampen(hfix, 0.01)
+    U = O.hinv_upper_factor(hd)
+    o_res, o_alpha, _ = O.ssqr_search(w0, U, bits, density)
+    rows = np.arange(200)
+    same, at_dev = _ssqr_compare(g, o_res, o_alpha, rows, bits, density, 700, w0, U)
+    # scaled errors' energy (tr(D H_d D^T)) and the proxy loss over the whole layer, against
+    # the oracle's column loop at the device's alphas
+    e2 = float(np.sum(at_dev["e"] ** 2))
+    assert abs(g["loss"].cpu().numpy()[1] - e2) <= LOSS_REL * e2
+    Q = at_dev["Q"]
+    proxy = O.proxy_loss(w0, Q, X)
+    assert abs(g["loss"].cpu().numpy()[0] - proxy) <= LOSS_REL * proxy
+
+
+@pytest.mark.slow
+def test_ssqr_search_full_size_sampled_rows():
+    """SSQR at the q_proj size (4096 x 4096, 4096 tokens), 3-bit, 1 % outliers: the search on
+    every row on the device, compared with the oracle's search on 16 sampled rows."""
+    W, X, spec = synth.workload("q_proj_4096x4096")
+    bits, density = 3, 0.01
+    g = _ssqr_gpu(W, X, bits, density)
+    H = O.hessian(X)
+    hfix, w0, _ = O.fix_dead_features(H, W)
+    hd, _ = O.dampen(hfix, 0.01)
+    U = O.hinv_upper_factor(hd)
+    rows = np.random.default_rng(31).choice(4096, size=16, replace=False)
+    o_res, o_alpha, _ = O.ssqr_search(w0[rows], U, bits, density)
+    _ssqr_compare(g, o_res, o_alpha, rows, bits, density, 4096, w0, U)
+
+
+def test_min_pivot_order_ragged():
+    """Greedy min-pivot order on the device ("The Geometry of LLM Quantization", section 2.3:
+    at every LDL step the smallest remaining Schur-complement pivot; Babai decides the columns in
+    the reverse of that elimination order): the order equals the oracle's on a ragged width
+    (300 = 9 panels of 32 + 12), then U, codes and losses in that order, per-row and group 64."""
+    W, X, spec = synth.workload("q_proj_4096x4096", m=96, n=300, T=400)
+    for group in (0, 64):
+        g = run_gpu(W, X, bits=4, group=group, order="min_pivot")
+        assert g["status"] == (0, 0)
+        o = _oracle(W, X, 4, group, False, True, order="min_pivot")
+        assert np.array_equal(g["perm"], o["perm"])
+        _compare(g, o, W, 4, group, perm=o["perm"])
+
+
+@pytest.mark.slow
+def test_min_pivot_order_full_size_sampled_rows():
+    """The min-pivot order at the q_proj width (4096): the device order against the oracle's,
+    then the 4-bit group-128 codes of sampled rows in that order."""
+    W, X, spec = synth.workload("q_proj_4096x4096")
+    g = run_gpu(W, X, bits=4, group=128, order="min_pivot")
+    assert g["status"] == (0, 0)
+    H = O.hessian(X)
+    hfix, _, _ = O.fix_dead_features(H, np.zeros((1, 4096)))
+    hd, _ = O.dampen(hfix, 0.01)
+    perm = O.min_pivot_order(hd)
+    same = float(np.mean(g["perm"] == perm))
+    print(f"min-pivot order identical at {same:.5f} of positions")
+    assert np.array_equal(g["perm"], perm)
+    rows = np.random.default_rng(41).choice(4096, size=24, replace=False)
+    o = O.quantize_layer(W, X, bits=4, group=128, rows=rows, H=H, order=perm)
+    _compare(g, o, W, 4, 128, rows=rows, perm=perm)

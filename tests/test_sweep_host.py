@@ -92,7 +92,9 @@ def test_stage_model_fractions_are_floor_over_measured():
     n, T, m = 4096, 4096, 4096
     h_floor = 2 * n * (n + 1) / 2 * T * bench.HESSIAN_DIGIT_PRODUCTS / 3000e12
     assert st["hessian"]["t_roof_ms"] == pytest.approx(h_floor * 1e3, rel=1e-3)
-    assert st["factor"]["t_roof_ms"] == pytest.approx(2 * n ** 3 / 3 / 36e12 * 1e3, rel=1e-3)
+    macs, fp64 = bench.factor_work(n)
+    f_floor = 2 * macs * bench.FACTOR_DIGIT_PRODUCTS / 3000e12 + fp64 / 36e12
+    assert st["factor"]["t_roof_ms"] == pytest.approx(f_floor * 1e3, rel=1e-3)
     assert st["column_loop"]["t_roof_ms"] == pytest.approx(3 * m * n * n / 750e12 * 1e3, rel=1e-3)
     for k in ms:
         assert st[k]["frac"] == pytest.approx(st[k]["t_roof_ms"] / ms[k], rel=1e-3)
@@ -110,3 +112,20 @@ def test_oracle_sample_scales_each_part_by_its_cost():
     t, det = bench.oracle_layer_sample([(X, [(W, 3, 0)])], tokens=32, n_sub=24, rows=8)
     assert t == pytest.approx(det["hessian_s"] + det["factor_s"] + det["loop_s"])
     assert 0 < det["measured_s"] < t       # every part is scaled up from a smaller sample
+
+
+def test_factor_work_model_matches_the_library_split_policy():
+    """bench.factor_work follows the factor's schedule: the split products start at the width
+    where the factor's workspace gains its digit planes, and the two parts add up to 2 n^3 / 3."""
+    sys.path.insert(0, ROOT)
+    import bench
+    from post_weight_quantization_22_b200 import gq as G
+    n0 = bench.FACTOR_SPLIT_MIN_N
+    jump = G.gq_prepare_workspace_size(n0) / n0 ** 2 - G.gq_prepare_workspace_size(n0 - 1) / (n0 - 1) ** 2
+    assert jump > 2.0                        # ~3 n^2 bytes of digit planes appear at n0
+    assert bench.factor_work(n0 - 1)[0] == 0.0
+    for n in (n0, 4096, 14336):
+        macs, fp64 = bench.factor_work(n)
+        assert 2 * macs + fp64 == pytest.approx(2 * n ** 3 / 3, rel=1e-12)
+    macs, fp64 = bench.factor_work(14336)
+    assert 2 * macs / (2 * 14336 ** 3 / 3) > 0.9   # nearly all of the factor at that width
