@@ -175,6 +175,12 @@ def minmax_grid(w, bits: int):
     range becomes [-1, 1]; scale s = (hi - lo) / (2^b - 1); zero point z = rint(-lo / s), so
     z lies in [0, 2^b - 1].  rint is round-half-to-even.  Returns (s, z) as fp64 vectors.
     """
+    s, zt = _minmax_unrounded(w, bits)
+    return s, np.rint(zt)
+
+
+def _minmax_unrounded(w, bits: int):
+    """``minmax_grid``'s scale and its zero point before rounding, -lo / s."""
     w = _f64(w)
     maxq = float(2 ** bits - 1)
     lo = np.minimum(w.min(axis=1), 0.0)
@@ -183,8 +189,7 @@ def minmax_grid(w, bits: int):
     lo = np.where(flat, -1.0, lo)
     hi = np.where(flat, 1.0, hi)
     s = (hi - lo) / maxq
-    z = np.rint(-lo / s)
-    return s, z
+    return s, -lo / s
 
 
 def clipfree_grid(w, bits: int, alpha):
@@ -224,7 +229,7 @@ def zsic_spacing(pivots) -> np.ndarray:
 # ---------------------------------------------------------------------------------------------
 
 def gptq_columns(W, U, bits: int, group: int = 0, clip: bool = True, alpha=None, grid=None,
-                 col_scale=None):
+                 col_scale=None, follow=None, tie_tol: float = 1e-3):
     """GPTQ error-feedback loop, columns 0..n-1 in order ([GEOM] 2.2).
 
     For each column j: quantize the current column on the row's grid, error
@@ -239,6 +244,15 @@ def gptq_columns(W, U, bits: int, group: int = 0, clip: bool = True, alpha=None,
     s Z with the min-max step of the row, zero point 0, no clamp.  ``grid`` = (s, z) fixes the per-row grid
     instead (a fixed lattice).  ``col_scale`` (per-row grids only) multiplies the step of
     column j by col_scale[j]: the grid of column j is s col_scale[j] (c - z).
+
+    ``follow`` is a harness for comparing an implementation that carries the weights in
+    lower precision: dict(codes = m x n, zeros = m x ngroups for group grids) of its decisions
+    in processing order.  Where its code (or group zero point) differs from this loop's by one
+    and this loop's unrounded value lies within ``tie_tol`` grid steps of the rounding boundary
+    between the two, the loop takes the other decision and carries on from it, so that one
+    near-tie does not change every later decision of the row; any other difference is counted
+    and the loop keeps its own.  The result then also holds ``followed`` (decisions taken over)
+    and ``disagree`` (differences beyond the tolerance).  The arithmetic is unchanged.
 
     Returns dict(codes, scales, zeros, Q, e) in processing order; e is the m x n matrix of
     scaled errors, whose squares sum to tr(D H_d D^T).
@@ -261,6 +275,17 @@ def gptq_columns(W, U, bits: int, group: int = 0, clip: bool = True, alpha=None,
     unbounded = clip == "unbounded"
     if unbounded:
         clip = False
+    followed = disagree = 0
+
+    def take(own, unrounded, other):
+        """own decision, or the followed one where the two sit on either side of a near-tie
+        (unrounded: this loop's value in the units the decision rounds)"""
+        nonlocal followed, disagree
+        diff = other != own
+        tie = diff & (np.abs(other - own) == 1) & (np.abs(unrounded - (own + other) / 2) <= tie_tol)
+        followed += int(np.count_nonzero(tie))
+        disagree += int(np.count_nonzero(diff & ~tie))
+        return np.where(tie, other, own)
     if group == 0:
         if grid is not None:
             s, z = (np.asarray(g, dtype=np.float64).copy() for g in grid)
@@ -274,19 +299,28 @@ def gptq_columns(W, U, bits: int, group: int = 0, clip: bool = True, alpha=None,
         scales[:, 0], zeros[:, 0] = s, z
     for j in range(n):
         if group and j % group == 0:
-            s, z = minmax_grid(w[:, j:j + group], bits)
+            s, zt = _minmax_unrounded(w[:, j:j + group], bits)
+            z = np.rint(zt)
+            if follow is not None and follow.get("zeros") is not None:
+                z = take(z, zt, np.asarray(follow["zeros"], dtype=np.float64)[:, j // group])
             scales[:, j // group], zeros[:, j // group] = s, z
         sj = s * kap[j]
         c = np.rint(w[:, j] / sj) + z
         if clip:
             c = np.clip(c, 0, maxq)
+        if follow is not None:
+            # boundary between codes c and c' in units of w / sj: (c + c') / 2 - z
+            c = take(c, w[:, j] / sj + z, np.asarray(follow["codes"], dtype=np.float64)[:, j])
         q = sj * (c - z)
         e = (w[:, j] - q) / u[j, j]
         w[:, j + 1:] -= np.outer(e, u[j, j + 1:])
         codes[:, j] = c.astype(np.int64)
         Q[:, j] = q
         E[:, j] = e
-    return dict(codes=codes, scales=scales, zeros=zeros, Q=Q, e=E)
+    out = dict(codes=codes, scales=scales, zeros=zeros, Q=Q, e=E)
+    if follow is not None:
+        out.update(followed=followed, disagree=disagree)
+    return out
 
 
 def ssqr_columns(W, U, bits: int, alpha):
@@ -518,7 +552,8 @@ def babai_bound(scales_per_col, pivots) -> float:
 
 def quantize_layer(W, X, bits: int, group: int = 0, reverse: bool = False, clip: bool = True,
                    damp: float = 0.01, ladder: float = 1.25, ladder_max: int = 8,
-                   rows=None, H=None, order=None, spacing: str = "uniform"):
+                   rows=None, H=None, order=None, spacing: str = "uniform", follow=None,
+                   tie_tol: float = 1e-3):
     """Quantize one linear layer: H, dead fix, damping, factor, column loop, losses.
 
     ``W`` is m x n (output rows x input features), ``X`` is T x n.  ``rows`` restricts the
@@ -541,6 +576,11 @@ def quantize_layer(W, X, bits: int, group: int = 0, reverse: bool = False, clip:
     clip=False (reading of "per-row step set so that no entry needs clipping"): run unclamped;
     a row whose codes leave [0, 2^b - 1] is rerun with alpha multiplied by ``ladder``, at most
     ``ladder_max`` times; rows still outside raise ValueError.
+
+    ``follow`` (GPTQ form, clipped or unbounded grids): another implementation's decisions for
+    the selected rows, dict(codes in the original column order, zeros by processing group),
+    taken over at near-ties as ``gptq_columns`` describes; the result adds ``followed`` and
+    ``disagree``.
 
     Returns a dict; codes / scales / zeros / Q are in the original column order.
     """
@@ -570,6 +610,8 @@ def quantize_layer(W, X, bits: int, group: int = 0, reverse: bool = False, clip:
             if sorted(perm.tolist()) != list(range(n)):
                 raise ValueError("order is not a permutation of the columns")
 
+    if follow is not None and (reverse or clip is False):
+        raise ValueError("follow takes the GPTQ form without the scale ladder")
     if spacing not in ("uniform", "zsic"):
         raise ValueError(f"unknown spacing {spacing!r}")
     if spacing == "zsic" and (reverse or group):
@@ -581,9 +623,12 @@ def quantize_layer(W, X, bits: int, group: int = 0, reverse: bool = False, clip:
         if spacing == "zsic":
             kap = zsic_spacing(pivots)
 
+        fol = None if follow is None else dict(codes=np.asarray(follow["codes"])[:, perm],
+                                               zeros=follow.get("zeros"))
+
         def run(rows_w, alpha):
             r = gptq_columns(rows_w[:, perm], U, bits, group=group, clip=clip, alpha=alpha,
-                             col_scale=kap)
+                             col_scale=kap, follow=fol, tie_tol=tie_tol)
             for key in ("codes", "Q"):
                 back = np.empty_like(r[key])
                 back[:, perm] = r[key]
@@ -603,7 +648,7 @@ def quantize_layer(W, X, bits: int, group: int = 0, reverse: bool = False, clip:
 
         def run(rows_w, alpha):
             return gptq_columns(rows_w, U, bits, group=group, clip=clip, alpha=alpha,
-                                col_scale=kap)
+                                col_scale=kap, follow=follow, tie_tol=tie_tol)
 
     alpha = np.ones(len(sel))
     res = run(w_sel, alpha)
@@ -630,6 +675,8 @@ def quantize_layer(W, X, bits: int, group: int = 0, reverse: bool = False, clip:
     out = dict(H=H, dead=dead, delta=delta, Hd=hd, codes=res["codes"], scales=res["scales"],
                zeros=res["zeros"], Q=Q, alpha=alpha, ladder_rounds=retries, perm=perm,
                col_scale=kap)
+    if follow is not None:
+        out["followed"], out["disagree"] = res["followed"], res["disagree"]
     if reverse:
         out["L"] = L
     else:

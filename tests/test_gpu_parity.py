@@ -1,7 +1,13 @@
 """Parity of the CUDA path (through the C ABI) with the fp64 oracle on seeded inputs.
 
 Tolerances: codes >= 99.9 % identical, proxy loss within 1e-3 relative, H within 1e-5 relative
-Frobenius (the layer-quantization contract).  Tighter design checks are added where the
+Frobenius (the layer-quantization contract).  The library carries the error-fed weights in fp32,
+the oracle in fp64, so a weight within rounding of a code boundary may land on either side, and
+GPTQ feeds that one difference into every later column of its row.  Where the library's
+decision and the oracle's differ by one step at a value within TIE_TOL grid steps of the
+boundary between them, the oracle takes the library's decision and carries on (its ``follow``
+harness); every other difference fails the test, and the near-ties taken over are held to a
+small count.  Tighter design checks are added where the
 arithmetic fixes them: H is accumulated from exact products in fp64 (<= 1e-12), U is an fp64
 factor stored in fp32 (<= 1e-6 relative Frobenius), per-row grids come from the input row
 (scales within fp32 rounding).
@@ -21,12 +27,21 @@ LOSS_REL = 1e-3
 H_REL = 1e-5
 H_REL_DESIGN = 1e-9   # digit rounding of entries below 2^-21 of their column's largest
 U_REL_DESIGN = 1e-6
+TIE_TOL = 1e-3          # grid steps: fp32 carries the weights to ~1e-6 of a step here
+FOLLOW_FRAC = 1e-4      # near-ties taken over, per decision (plus two)
 
 
 def _oracle(W, X, bits, group, reverse, clip, rows=None, order=None, spacing="uniform",
-            ladder_max=8):
+            ladder_max=8, g=None):
+    """The oracle on the same input; with the library's result ``g`` (GPTQ form without the
+    scale ladder) it follows the library's decisions at near-ties (see the module docstring)."""
+    follow = None
+    if g is not None and not reverse and clip is not False:
+        sel = slice(None) if rows is None else rows
+        follow = dict(codes=g["codes"][sel], zeros=g["zeros"][sel] if group else None)
     return O.quantize_layer(W, X, bits=bits, group=group, reverse=reverse, clip=clip, rows=rows,
-                            order=order, spacing=spacing, ladder_max=ladder_max)
+                            order=order, spacing=spacing, ladder_max=ladder_max, follow=follow,
+                            tie_tol=TIE_TOL)
 
 
 def _compare(g, o, W, bits, group, rows=None, check_loss=True, perm=None):
@@ -39,6 +54,10 @@ def _compare(g, o, W, bits, group, rows=None, check_loss=True, perm=None):
     assert np.array_equal(g["dead"], o["dead"])
     assert abs(g["delta"] - o["delta"]) <= H_REL_DESIGN * abs(o["delta"])  # a mean of diag(H)
     gc = g["codes"] if rows is None else g["codes"][rows]
+    if "disagree" in o:  # the oracle followed the library at near-ties
+        print(f"near-ties followed {o['followed']} of {gc.size}")
+        assert o["disagree"] == 0, f"{o['disagree']} decisions differ beyond a near-tie"
+        assert o["followed"] <= FOLLOW_FRAC * gc.size + 2, o["followed"]
     match = float(np.mean(gc == o["codes"]))
     print(f"code match {match:.6f}")
     assert match >= CODE_MATCH, f"code match {match:.6f}"
@@ -80,7 +99,7 @@ def test_tiny_fp32_per_row_4bit():
     W, X, spec = synth.workload("tiny_256x512")
     g = run_gpu(W, X, bits=4)
     assert g["status"] == (0, 0)
-    o = _oracle(W, X, 4, 0, False, True)
+    o = _oracle(W, X, 4, 0, False, True, g=g)
     _compare(g, o, W, 4, 0)
 
 
@@ -90,7 +109,7 @@ def test_qproj_recipe_ragged_group128():
     W, X, spec = synth.workload("q_proj_4096x4096", m=320, n=1000, T=1200)
     g = run_gpu(W, X, bits=4, group=128)
     assert g["status"] == (0, 0)
-    o = _oracle(W, X, 4, 128, False, True)
+    o = _oracle(W, X, 4, 128, False, True, g=g)
     _compare(g, o, W, 4, 128)
 
 
@@ -102,7 +121,7 @@ def test_ragged_split_factor_group128():
     W, X, spec = synth.workload("q_proj_4096x4096", m=300, n=1700, T=2000)
     g = run_gpu(W, X, bits=4, group=128)
     assert g["status"] == (0, 0)
-    o = _oracle(W, X, 4, 128, False, True)
+    o = _oracle(W, X, 4, 128, False, True, g=g)
     _compare(g, o, W, 4, 128)
     gr = run_gpu(W, X, bits=3, reverse=True, clip=False)
     assert gr["status"] == (0, 0)
@@ -117,7 +136,7 @@ def test_clipfree_reverse_ladder_and_bound():
     W, X, spec = synth.workload("clipfree_babai_4096x4096", m=256, n=640, T=900)
     g = run_gpu(W, X, bits=3, reverse=True, clip=False)
     assert g["status"] == (0, 0)
-    o = _oracle(W, X, 3, 0, True, False)
+    o = _oracle(W, X, 3, 0, True, False, g=g)
     assert g["rounds"] == o["ladder_rounds"]
     _compare(g, o, W, 3, 0)
     assert g["codes"].min() >= 0 and g["codes"].max() <= 7
@@ -127,7 +146,7 @@ def test_clipfree_reverse_ladder_and_bound():
 def test_group64_2bit_forward():
     W, X, spec = synth.workload("q_proj_4096x4096", m=200, n=512, T=700)
     g = run_gpu(W, X, bits=2, group=64)
-    o = _oracle(W, X, 2, 64, False, True)
+    o = _oracle(W, X, 2, 64, False, True, g=g)
     _compare(g, o, W, 2, 64)
 
 
@@ -135,7 +154,7 @@ def test_reverse_with_clip_and_forward_clipfree():
     W, X, spec = synth.workload("q_proj_4096x4096", m=96, n=384, T=500)
     for reverse, clip in ((True, True), (False, False)):
         g = run_gpu(W, X, bits=3, reverse=reverse, clip=clip)
-        o = _oracle(W, X, 3, 0, reverse, clip)
+        o = _oracle(W, X, 3, 0, reverse, clip, g=g)
         _compare(g, o, W, 3, 0)
 
 
@@ -144,7 +163,7 @@ def test_dead_feature():
     X = X.clone()
     X[:, [3, 77, 200]] = 0
     g = run_gpu(W, X, bits=4, group=32)
-    o = _oracle(W, X, 4, 32, False, True)
+    o = _oracle(W, X, 4, 32, False, True, g=g)
     assert g["dead"].sum() == 3
     _compare(g, o, W, 4, 32)
 
@@ -153,7 +172,7 @@ def test_dead_feature():
 def test_edge_shapes(m, n, T):
     W, X, spec = synth.workload("q_proj_4096x4096", m=m, n=n, T=T)
     g = run_gpu(W, X, bits=4)
-    o = _oracle(W, X, 4, 0, False, True)
+    o = _oracle(W, X, 4, 0, False, True, g=g)
     _compare(g, o, W, 4, 0)
 
 
@@ -221,7 +240,7 @@ def test_act_order_ragged_group128():
     W, X, spec = synth.workload("q_proj_4096x4096", m=320, n=1000, T=1200)
     g = run_gpu(W, X, bits=4, group=128, order="act")
     assert g["status"] == (0, 0)
-    o = _oracle(W, X, 4, 128, False, True, order=g["perm"])
+    o = _oracle(W, X, 4, 128, False, True, order=g["perm"], g=g)
     assert _check_act_perm(g["perm"], o) == 0
     _compare(g, o, W, 4, 128, perm=g["perm"])
 
@@ -232,7 +251,7 @@ def test_act_order_tiny_fp32_per_row_and_dead_columns():
     X[:, [5, 300]] = 0  # two dead columns: fixed diagonal 1, weights zeroed
     g = run_gpu(W, X, bits=4, order="act")
     assert g["status"] == (0, 0)
-    o = _oracle(W, X, 4, 0, False, True, order=g["perm"])
+    o = _oracle(W, X, 4, 0, False, True, order=g["perm"], g=g)
     _check_act_perm(g["perm"], o)
     assert g["dead"].sum() == 2
     _compare(g, o, W, 4, 0, perm=g["perm"])
@@ -246,7 +265,7 @@ def test_zsic_spacing_clipfree_ladder():
     W, X, spec = synth.workload("q_proj_4096x4096", m=200, n=520, T=700)
     g = run_gpu(W, X, bits=8, clip=False, spacing="zsic", ladder_max=16)
     assert g["status"] == (0, 0)
-    o = _oracle(W, X, 8, 0, False, False, spacing="zsic", ladder_max=16)
+    o = _oracle(W, X, 8, 0, False, False, spacing="zsic", ladder_max=16, g=g)
     np.testing.assert_allclose(g["kappa"], o["col_scale"], rtol=1e-6)
     assert g["rounds"] == o["ladder_rounds"]
     _compare(g, o, W, 8, 0)
@@ -260,7 +279,7 @@ def test_zsic_spacing_with_act_order_4bit_and_am_gm_bound():
     W, X, spec = synth.workload("q_proj_4096x4096", m=96, n=384, T=500)
     g = run_gpu(W, X, bits=4, order="act", spacing="zsic")
     assert g["status"] == (0, 0)
-    o = _oracle(W, X, 4, 0, False, True, order=g["perm"], spacing="zsic")
+    o = _oracle(W, X, 4, 0, False, True, order=g["perm"], spacing="zsic", g=g)
     np.testing.assert_allclose(g["kappa"], o["col_scale"], rtol=1e-6)
     _compare(g, o, W, 4, 0, perm=g["perm"])
     u = run_gpu(W, X, bits=4, order="act")
@@ -330,7 +349,7 @@ def test_unbounded_lattice_codes_and_huffman_rate():
     W, X, spec = synth.workload("q_proj_4096x4096", m=128, n=520, T=700)
     g = run_gpu(W, X, bits=4, clip="unbounded")
     assert g["status"] == (0, 0)
-    o = _oracle(W, X, 4, 0, False, "unbounded")
+    o = _oracle(W, X, 4, 0, False, "unbounded", g=g)
     assert (g["zeros"] == 0).all()
     _compare(g, o, W, 4, 0)
     total = _huffman_check(g["codes_dev"])
@@ -345,7 +364,7 @@ def test_zsic_unbounded_lattice_with_huffman():
     W, X, spec = synth.workload("q_proj_4096x4096", m=128, n=520, T=700)
     g = run_gpu(W, X, bits=4, clip="unbounded", spacing="zsic")
     assert g["status"] == (0, 0)
-    o = _oracle(W, X, 4, 0, False, "unbounded", spacing="zsic")
+    o = _oracle(W, X, 4, 0, False, "unbounded", spacing="zsic", g=g)
     _compare(g, o, W, 4, 0)
     total = _huffman_check(g["codes_dev"])
     assert abs(total / g["codes"].size - o["rate"]) <= 0.01 * o["rate"]
@@ -359,7 +378,7 @@ def test_given_order_clipfree_ladder():
     g = run_gpu(W, X, bits=3, clip=False, order="given", perm=perm)
     assert g["status"] == (0, 0)
     assert np.array_equal(g["perm"], perm)
-    o = _oracle(W, X, 3, 0, False, False, order=perm)
+    o = _oracle(W, X, 3, 0, False, False, order=perm, g=g)
     assert g["rounds"] == o["ladder_rounds"]
     _compare(g, o, W, 3, 0, perm=perm)
     assert g["loss"][1] <= g["loss"][2]
@@ -397,7 +416,7 @@ def test_qproj_full_size_sampled_rows():
     g = run_gpu(W, X, bits=4, group=128)
     assert g["status"] == (0, 0)
     rows = np.random.default_rng(7).choice(4096, size=64, replace=False)
-    o = _oracle(W, X, 4, 128, False, True, rows=rows)
+    o = _oracle(W, X, 4, 128, False, True, rows=rows, g=g)
     _compare(g, o, W, 4, 128, rows=rows)
     # loss bookkeeping at full size: sum of e^2 == tr(D H_d D^T) of the GPU's Q
     q = g["scales"].repeat(128, axis=1)[:, :4096] * (g["codes"] - g["zeros"].repeat(128, axis=1)[:, :4096])
@@ -449,7 +468,7 @@ def test_mlp_pair_full_size_sampled_rows(name):
     g = run_gpu(W, X, bits=spec["bits"], group=spec["group"])
     assert g["status"] == (0, 0)
     rows = np.random.default_rng(11).choice(spec["m"], size=32, replace=False)
-    o = _oracle(W, X, spec["bits"], spec["group"], False, True, rows=rows)
+    o = _oracle(W, X, spec["bits"], spec["group"], False, True, rows=rows, g=g)
     _compare(g, o, W, spec["bits"], spec["group"], rows=rows)
 
 
@@ -462,7 +481,7 @@ def test_clipfree_babai_full_size_sampled_rows():
     g = run_gpu(W, X, bits=3, group=0, reverse=True, clip=False)
     assert g["status"][0] == 0 and g["status"][1] == 0
     rows = np.random.default_rng(5).choice(4096, size=48, replace=False)
-    o = _oracle(W, X, 3, 0, True, False, rows=rows)
+    o = _oracle(W, X, 3, 0, True, False, rows=rows, g=g)
     _compare(g, o, W, 3, 0, rows=rows)
 
 
@@ -501,7 +520,8 @@ def test_sweep_block_layers_2bit_g64(sweep_block0, key):
                     loss=o_["loss"].cpu().numpy(), dead=d["dead"].cpu().numpy().astype(bool),
                     delta=float(d["delta"].item()))
         rows = np.random.default_rng(20 + li).choice(m, size=32, replace=False)
-        o = O.quantize_layer(Ws[name], X, bits=2, group=64, rows=rows, H=H)
+        o = O.quantize_layer(Ws[name], X, bits=2, group=64, rows=rows, H=H, tie_tol=TIE_TOL,
+                             follow=dict(codes=gres["codes"][rows], zeros=gres["zeros"][rows]))
         _compare(gres, o, Ws[name], 2, 64, rows=rows)
 
 
@@ -662,7 +682,7 @@ def test_min_pivot_order_ragged():
     for group in (0, 64):
         g = run_gpu(W, X, bits=4, group=group, order="min_pivot")
         assert g["status"] == (0, 0)
-        o = _oracle(W, X, 4, group, False, True, order="min_pivot")
+        o = _oracle(W, X, 4, group, False, True, order="min_pivot", g=g)
         assert np.array_equal(g["perm"], o["perm"])
         _compare(g, o, W, 4, group, perm=o["perm"])
 
@@ -682,5 +702,6 @@ def test_min_pivot_order_full_size_sampled_rows():
     print(f"min-pivot order identical at {same:.5f} of positions")
     assert np.array_equal(g["perm"], perm)
     rows = np.random.default_rng(41).choice(4096, size=24, replace=False)
-    o = O.quantize_layer(W, X, bits=4, group=128, rows=rows, H=H, order=perm)
+    o = O.quantize_layer(W, X, bits=4, group=128, rows=rows, H=H, order=perm, tie_tol=TIE_TOL,
+                         follow=dict(codes=g["codes"][rows], zeros=g["zeros"][rows]))
     _compare(g, o, W, 4, 128, rows=rows, perm=perm)

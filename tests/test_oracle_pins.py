@@ -716,3 +716,71 @@ def test_ssqr_search_is_a_bisection_of_feasibility(density):
     assert np.all(probe > limit)
     if density == 0.0:
         assert not r["outlier"].any()
+
+
+# ---------------------------------------------------------------------------------------------
+# The follow harness of gptq_columns: near-ties taken over, everything else counted
+# ---------------------------------------------------------------------------------------------
+
+def test_follow_own_decisions_changes_nothing():
+    rng = np.random.default_rng(5)
+    W = rng.standard_normal((6, 40))
+    X = rng.standard_normal((200, 40))
+    plain = O.quantize_layer(W, X, bits=3, group=8)
+    fol = O.quantize_layer(W, X, bits=3, group=8,
+                           follow=dict(codes=plain["codes"], zeros=plain["zeros"]))
+    assert fol["followed"] == 0 and fol["disagree"] == 0
+    assert np.array_equal(fol["codes"], plain["codes"])
+    assert np.array_equal(fol["Q"], plain["Q"])
+
+
+def test_follow_takes_a_tie_and_counts_a_real_difference():
+    """U = I (nothing fed forward), 2-bit, row [0, 1.75, 3.5]: s = 7/6, z = 0, so column 1 sits
+    on the boundary between codes 1 and 2 (own choice 2, round half to even) and column 2 is
+    3 with no tie."""
+    U = np.eye(3)
+    w = np.array([[0.0, 1.75, 3.5]])
+    own = O.gptq_columns(w, U, 2)
+    assert own["codes"].tolist() == [[0, 2, 3]]
+    tie = O.gptq_columns(w, U, 2, follow=dict(codes=[[0, 1, 3]]))
+    assert tie["codes"].tolist() == [[0, 1, 3]] and (tie["followed"], tie["disagree"]) == (1, 0)
+    far = O.gptq_columns(w, U, 2, follow=dict(codes=[[0, 2, 1]]))
+    assert far["codes"].tolist() == [[0, 2, 3]] and (far["followed"], far["disagree"]) == (0, 1)
+    off_by_one = O.gptq_columns(w, U, 2, follow=dict(codes=[[1, 2, 3]]))  # t = 0: no tie
+    assert off_by_one["codes"].tolist() == [[0, 2, 3]] and off_by_one["disagree"] == 1
+
+
+def test_follow_carries_on_from_the_followed_code():
+    """U = [[1, 1], [0, 1]], 2-bit, row [0.75, 1.5]: s = 0.5, z = 0.  Own: t0 = 1.5 -> 2,
+    e0 = -0.25, w1 = 1.75, t1 = 3.5 -> 4 -> clamp 3.  Followed code 1: e0 = 0.25, w1 = 1.25,
+    t1 = 2.5 -> 2 (half to even)."""
+    U = np.array([[1.0, 1.0], [0.0, 1.0]])
+    w = np.array([[0.75, 1.5]])
+    assert O.gptq_columns(w, U, 2)["codes"].tolist() == [[2, 3]]
+    r = O.gptq_columns(w, U, 2, follow=dict(codes=[[1, 2]]))
+    assert r["codes"].tolist() == [[1, 2]] and (r["followed"], r["disagree"]) == (1, 0)
+    np.testing.assert_allclose(r["e"], [[0.25, 1.25 - 1.0]])
+
+
+def test_follow_takes_a_tied_zero_point():
+    """group 2, 2-bit, row [-0.75, 0.75]: s = 0.5, -lo/s = 1.5, own zero 2 (half to even);
+    followed zero 1.  Codes: rint(-1.5) + 1 = -1 -> 0 and rint(1.5) + 1 = 3."""
+    U = np.eye(2)
+    w = np.array([[-0.75, 0.75]])
+    own = O.gptq_columns(w, U, 2, group=2)
+    assert own["zeros"].tolist() == [[2.0]] and own["codes"].tolist() == [[0, 3]]
+    r = O.gptq_columns(w, U, 2, group=2, follow=dict(codes=[[0, 3]], zeros=[[1]]))
+    assert r["zeros"].tolist() == [[1.0]] and r["codes"].tolist() == [[0, 3]]
+    assert (r["followed"], r["disagree"]) == (1, 0)
+    np.testing.assert_allclose(r["Q"], [[-0.5, 1.0]])
+
+
+def test_follow_is_refused_where_it_has_no_meaning():
+    rng = np.random.default_rng(1)
+    W = rng.standard_normal((2, 8))
+    X = rng.standard_normal((40, 8))
+    f = dict(codes=np.zeros((2, 8), dtype=np.int64))
+    with pytest.raises(ValueError):
+        O.quantize_layer(W, X, bits=3, reverse=True, follow=f)
+    with pytest.raises(ValueError):
+        O.quantize_layer(W, X, bits=3, clip=False, follow=f)
