@@ -242,12 +242,12 @@ def complete_peaks(peaks: dict) -> dict:
 # the work of a step and its floor on each pipe
 # ---------------------------------------------------------------------------------------------
 
-# The factor's schedule (gq_factor.cu): 256-wide super-panels; from n = 1536 the trailing
+# The factor's schedule (gq_factor.cu): from n = 1536, 512-wide super-panels; the trailing
 # update of every super-panel that has rows below it (next super-panel's columns and all later
-# ones: the lower triangle of the remaining (n - sp1) x (n - sp1) block, depth 256) and the
+# ones: the lower triangle of the remaining (n - sp1) x (n - sp1) block, depth 512) and the
 # inverse's block product T[sp1:, :sp0] += L[sp1:, K] X[K, :sp0] run as int8 digit products,
 # 21 per multiply-add (six 7-bit digits a value, the pairs with p + q <= 5).
-FACTOR_SUPER = 256
+FACTOR_SUPER = 512  # the split path's super-panel width (products of depth 512)
 FACTOR_SPLIT_MIN_N = 1536
 FACTOR_DIGIT_PRODUCTS = 21
 
@@ -717,7 +717,8 @@ def run_reference(args):
 
 
 def run_case(args):
-    """One invocation for profilers: `layer` (the q_proj recipe at --case-n), `factor`
+    """One invocation for profilers: `layer` (the q_proj recipe at --case-n, or --workload
+    at its full size when --case-n is not given, two calls so a profiler can skip the first), `factor`
     (gq_prepare_hinv on a seeded SPD fp64 H of width --case-n), or `huffman` (the Huffman
     encoder on the unconstrained-lattice codes of that layer, event-timed, one JSON line with
     its HBM roofline)."""
@@ -726,12 +727,18 @@ def run_case(args):
     from post_weight_quantization_22_b200.pipeline import LayerQuantizer
 
     torch.cuda.set_device(0)
-    n = args.case_n
+    n = args.case_n if args.case_n is not None else 2048
     if args.case == "layer":
-        W, X, spec = synth.workload("q_proj_4096x4096", m=n, n=n, T=n)
+        if args.case_n is None:
+            W, X, spec = synth.workload(args.workload)
+        else:
+            W, X, spec = synth.workload("q_proj_4096x4096", m=n, n=n, T=n)
+        m, n = W.shape
         cfg = G.QuantCfg(bits=spec["bits"], group_size=spec["group"])
-        lq = LayerQuantizer(n, n, cfg, device="cuda")
-        lq.run(W.cuda(), X.cuda())
+        lq = LayerQuantizer(m, n, cfg, device="cuda", max_tokens=X.shape[0])
+        Wd, Xd = W.cuda(), X.cuda()
+        for _ in range(1 if args.case_n is not None else 2):
+            lq.run(Wd, Xd)
         torch.cuda.synchronize()
         print("status", lq.status())
     elif args.case == "factor":
@@ -789,7 +796,8 @@ def main(argv=None):
     ap.add_argument("--ref-rows", type=int, default=8)
     ap.add_argument("--case", choices=["layer", "factor", "huffman"], default=None,
                     help="run one untimed invocation (for profilers) and exit")
-    ap.add_argument("--case-n", type=int, default=2048)
+    ap.add_argument("--case-n", type=int, default=None,
+                    help="size of the case (default: 2048; `layer`: --workload at full size)")
     args = ap.parse_args(argv)
     if args.case:
         return run_case(args)

@@ -23,7 +23,7 @@
 namespace gq {
 
 constexpr int kNB = 64;      // Cholesky panel width (the leaf)
-constexpr int kSuper = 256;  // super-panel width (trailing-update depth)
+constexpr int kSuper = 256;  // super-panel width (trailing-update depth) of the fp64 path
 constexpr int kPnPitch = 68;  // shared-memory pitch (doubles) of the panel kernel's tiles
 constexpr size_t kPnSmem = (size_t)(kNB + 32) * kPnPitch * sizeof(double);
 
@@ -504,6 +504,10 @@ static int64_t m_ld(int64_t n) { return (n + 15) / 16 * 16; }
 // every product stays on the fp64 units (the products are small and the chain dominates).
 constexpr int64_t kSplitMinN = 1536;
 static bool use_split(int64_t n) { return n >= kSplitMinN; }
+// Super-panel width: the split path's products are as deep as a super-panel (kSplitK = 512,
+// which keeps the fp64 read-modify-write of each output tile under its products); the fp64
+// path keeps 256 (a shorter chain of in-panel updates).
+static int64_t super_width(int64_t n) { return use_split(n) ? kSplitK : kSuper; }
 
 struct PrepLayout {
   WsHeader* hdr;
@@ -527,17 +531,20 @@ struct PrepLayout {
   int* lex;
   int8_t* xdig;
   int* xex;
+  int8_t* kdig;  // the diagonal block X_KK of the inverse: its rows, then its columns
+  int* kex;
   size_t bytes;
 };
 
 // rows of the L digit planes of the super-panels before super-panel K
 static int64_t lrow_offset(int64_t n, int64_t K) {
   int64_t off = 0;
-  for (int64_t k = 0; k < K; ++k) off += std::max<int64_t>(n - (k + 1) * kSuper, 0);
+  const int64_t sw = super_width(n);
+  for (int64_t k = 0; k < K; ++k) off += std::max<int64_t>(n - (k + 1) * sw, 0);
   return off;
 }
 
-// doubling scratch for one diagonal block of width w (<= kSuper)
+// doubling scratch for one diagonal block of width w (<= 512)
 static size_t trtri_tbuf_elems(int64_t w) {
   size_t best = 0;
   for (int64_t bs = kNB; bs < w; bs *= 2) {
@@ -555,7 +562,7 @@ static PrepLayout prep_layout(void* ws, int64_t n) {
   L.M = c.take<double>((size_t)n * m_ld(n));
   L.T = c.take<double>((size_t)n * m_ld(n));
   L.Dinv = c.take<double>((size_t)((n + kNB - 1) / kNB) * kNB * kNB);
-  L.tbuf = c.take<double>(trtri_tbuf_elems(kSuper) + 1);
+  L.tbuf = c.take<double>(trtri_tbuf_elems(super_width(n)) + 1);
   L.pmark = c.take<int>((size_t)n);
   {
     const size_t need = (size_t)n * kMpW * 2 + (size_t)n + kMpW + (size_t)n;  // doubles
@@ -575,12 +582,15 @@ static PrepLayout prep_layout(void* ws, int64_t n) {
     }
   }
   L.ldig = nullptr; L.lex = nullptr; L.xdig = nullptr; L.xex = nullptr;
+  L.kdig = nullptr; L.kex = nullptr;
   if (use_split(n)) {
-    const int64_t lrows = lrow_offset(n, (n + kSuper - 1) / kSuper);
+    const int64_t lrows = lrow_offset(n, (n + kSplitK - 1) / kSplitK);
     L.ldig = c.take<int8_t>((size_t)kSplitDigits * kSplitK * (size_t)lrows);
     L.lex = c.take<int>((size_t)lrows);
     L.xdig = c.take<int8_t>((size_t)kSplitDigits * kSplitK * (size_t)n);
     L.xex = c.take<int>((size_t)n);
+    L.kdig = c.take<int8_t>((size_t)2 * kSplitDigits * kSplitK * kSplitK);
+    L.kex = c.take<int>((size_t)2 * kSplitK);
   }
   L.bytes = c.off;
   return L;
@@ -605,7 +615,7 @@ cudaError_t factor_init_attributes() {
     if (_e != cudaSuccess) return _e;           \
   } while (0)
 
-// Inverse of the diagonal block [r0, r0 + w) of L (w <= kSuper) from its inverted 64-wide
+// Inverse of the diagonal block [r0, r0 + w) of L (w <= 512) from its inverted 64-wide
 // leaves, by doubling: inv([[A, 0], [B, C]]) = [[A^-1, 0], [-C^-1 B A^-1, C^-1]], all pairs of
 // a level batched.
 static cudaError_t invert_diag_block(double* M, int64_t n, int64_t ldm, int64_t r0, int64_t w,
@@ -772,19 +782,35 @@ cudaError_t launch_prepare(const double* H, int64_t n, double damp, int order, i
   //   X_KK = L_KK^-1 (doubling over the inverted 64-wide leaves inside the block),
   //   X[K, :k0] = -X_KK T[K, :k0],   T[K, J] = sum_{J <= I < K} L[K, I] X[I, J],
   // with T accumulated right-looking once X's block row K is known:
-  //   T[i >= k1, K] = L[i, K] X_KK,   T[i >= k1, :k0] += L[i, K] X[K, :k0]   (K = 256 GEMMs).
+  //   T[i >= k1, K] = L[i, K] X_KK,   T[i >= k1, :k0] += L[i, K] X[K, :k0].
   // X overwrites L in place: block row K of L is not read by the Cholesky after block K.
+  // On the split path a full-width block row (512) takes its three products on the int8
+  // tensor cores; X_KK's rows and columns are split with its upper triangle counted as zero,
+  // and the two products that assign (rather than add) write into zeroed blocks.
   const bool split = use_split(n);
+  const int64_t sup = super_width(n);
   // digit planes of super-panel K's columns of L, rows sp1 .. n-1 (plane row r = row sp1 + r)
   auto l_operand = [&](int64_t K) {
     const int64_t off = lrow_offset(n, K);
     return SplitOperand{L.ldig + off * kSplitDigits * kSplitK, L.lex + off,
-                        n - std::min<int64_t>((K + 1) * kSuper, n)};
+                        n - std::min<int64_t>((K + 1) * sup, n)};
   };
   auto inverse_block_row = [&](int64_t k0, int64_t k1) -> cudaError_t {
     const int64_t kw = k1 - k0;
     GQ_TRY(invert_diag_block(L.M, n, ldm, k0, kw, L.Dinv, L.tbuf, L.hdr, sc));
-    if (k0 > 0) {  // X[K, :k0] = -X_KK T[K, :k0]
+    const bool ksplit = split && kw == kSplitK;
+    const SplitOperand krows{L.kdig, L.kex, kSplitK};  // rows of X_KK
+    const SplitOperand kcols{L.kdig + (size_t)kSplitDigits * kSplitK * kSplitK, L.kex + kSplitK,
+                             kSplitK};                  // columns of X_KK
+    if (k0 > 0 && ksplit) {  // X[K, :k0] = -X_KK T[K, :k0] (block row K of L is not needed)
+      const SplitOperand top{L.xdig, L.xex, k0};
+      GQ_TRY(launch_split_rows(L.M + k0 * ldm + k0, ldm, (int)kw, krows, sc, 1));
+      GQ_TRY(launch_split_cols(L.T + k0 * ldm, ldm, (int)k0, top, sc));
+      GQ_TRY(cudaMemset2DAsync(L.M + k0 * ldm, ldm * sizeof(double), 0, k0 * sizeof(double),
+                               kw, sc));
+      GQ_TRY(launch_split_gemm(L.M + k0 * ldm, ldm, (int)kw, (int)k0, krows, 0, top, 0, -1.0, 0,
+                               L.hdr, sc));
+    } else if (k0 > 0) {  // X[K, :k0] = -X_KK T[K, :k0]
       DgemmCall g{};
       g.M = (int)kw; g.N = (int)k0; g.K = (int)kw; g.batch = 1; g.alpha = -1.0; g.beta_one = 0;
       g.A = Mop(k0, k0); g.a_lower = 1;
@@ -793,7 +819,13 @@ cudaError_t launch_prepare(const double* H, int64_t n, double damp, int order, i
       GQ_TRY(launch_dgemm(g, sc));
     }
     if (k1 < n) {
-      {  // T[k1:, K] = L[k1:, K] X_KK
+      if (ksplit) {  // T[k1:, K] = L[k1:, K] X_KK
+        GQ_TRY(launch_split_cols(L.M + k0 * ldm + k0, ldm, (int)kw, kcols, sc, 1));
+        GQ_TRY(cudaMemset2DAsync(L.T + k1 * ldm + k0, ldm * sizeof(double), 0,
+                                 kw * sizeof(double), n - k1, sc));
+        GQ_TRY(launch_split_gemm(L.T + k1 * ldm + k0, ldm, (int)(n - k1), (int)kw,
+                                 l_operand(k0 / sup), 0, kcols, 0, 1.0, 0, L.hdr, sc));
+      } else {  // T[k1:, K] = L[k1:, K] X_KK
         DgemmCall g{};
         g.M = (int)(n - k1); g.N = (int)kw; g.K = (int)kw; g.batch = 1; g.alpha = 1.0;
         g.beta_one = 0;
@@ -805,7 +837,7 @@ cudaError_t launch_prepare(const double* H, int64_t n, double damp, int order, i
       if (k0 > 0 && split) {  // T[k1:, :k0] += L[k1:, K] X[K, :k0] on the int8 tensor cores
         const SplitOperand xop{L.xdig, L.xex, k0};
         GQ_TRY(launch_split_cols(L.M + k0 * ldm, ldm, (int)k0, xop, sc));
-        GQ_TRY(launch_split_gemm(L.T + k1 * ldm, ldm, (int)(n - k1), (int)k0, l_operand(k0 / kSuper),
+        GQ_TRY(launch_split_gemm(L.T + k1 * ldm, ldm, (int)(n - k1), (int)k0, l_operand(k0 / sup),
                                  0, xop, 0, 1.0, 0, L.hdr, sc));
       } else if (k0 > 0) {  // T[k1:, :k0] += L[k1:, K] X[K, :k0]
         DgemmCall g{};
@@ -831,8 +863,8 @@ cudaError_t launch_prepare(const double* H, int64_t n, double damp, int order, i
   for (int64_t k = 0; k < nb; ++k) {
     const int64_t c0 = k * kNB;
     const int w = (int)std::min<int64_t>(kNB, n - c0);
-    const int64_t sp0 = (c0 / kSuper) * kSuper;                 // super-panel start
-    const int64_t sp1 = std::min<int64_t>(sp0 + kSuper, n);     // super-panel end
+    const int64_t sp0 = (c0 / sup) * sup;                       // super-panel start
+    const int64_t sp1 = std::min<int64_t>(sp0 + sup, n);        // super-panel end
     const int64_t rem = n - c0 - w;
     {  // leaf (every CTA) + P <- P L11^-T for the rows below, one wave of CTAs
       const int64_t nch = rem > 0 ? (rem + 31) / 32 : 1;
@@ -856,14 +888,14 @@ cudaError_t launch_prepare(const double* H, int64_t n, double damp, int order, i
     // super-panel [sp0, sp1) factored; on the split path its columns of L below it become
     // digit planes once, for the two trailing updates and the inverse's block product
     const bool sp_split = split && sp1 < n;
-    const SplitOperand lop = sp_split ? l_operand(sp0 / kSuper) : SplitOperand{};
+    const SplitOperand lop = sp_split ? l_operand(sp0 / sup) : SplitOperand{};
     if (sp_split) GQ_TRY(launch_split_rows(L.M + sp1 * ldm + sp0, ldm, (int)(n - sp1), lop, s));
     cudaEvent_t ev_panel = ps->panel[sidx & 1];
     GQ_TRY(cudaEventRecord(ev_panel, s));
     GQ_TRY(cudaStreamWaitEvent(sc, ev_panel, 0));
     GQ_TRY(inverse_block_row(sp0, sp1));
     if (sp1 < n) {
-      const int64_t sp2 = std::min<int64_t>(sp1 + kSuper, n), kw = sp1 - sp0;
+      const int64_t sp2 = std::min<int64_t>(sp1 + sup, n), kw = sp1 - sp0;
       if (far_pending) GQ_TRY(cudaStreamWaitEvent(s, ps->far[(sidx - 1) & 1], 0));
       if (sp_split) {  // next super-panel's columns: A[sp1:, sp1:sp2] -= L[sp1:, SP] L[sp1:sp2, SP]^T
         GQ_TRY(launch_split_gemm(L.M + sp1 * ldm + sp1, ldm, (int)(n - sp1), (int)(sp2 - sp1),

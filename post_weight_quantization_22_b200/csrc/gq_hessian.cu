@@ -42,9 +42,10 @@ constexpr uint32_t kHStage = kHS * (kHATile + kHBTile);  // 48 KB
 constexpr size_t kHSmem = kHStages * kHStage + 1024 + 256;
 constexpr int kHClasses = 5;                           // a + b in [0, 4] (13 digit pairs)
 constexpr int64_t kHChunk = 65536;                     // tokens per pass (int32 headroom)
-// int8 x int8 -> s32, A and B K-major, M 128, N 64
-constexpr uint32_t kHIdesc = (2u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(kHBN >> 3) << 17) |
-                             ((uint32_t)(kHBM >> 4) << 24);
+// int8 x int8 -> s32, A and B K-major, M 128, N columns (a multiple of 16, at most 256)
+__host__ __device__ constexpr uint32_t hess_idesc(uint32_t N) {
+  return (2u << 4) | (1u << 7) | (1u << 10) | ((N >> 3) << 17) | ((uint32_t)(kHBM >> 4) << 24);
+}
 }  // namespace
 
 // ---------------------------------------------------------------------------------------
@@ -172,19 +173,24 @@ __global__ void __launch_bounds__(128, 1)
       // start-address field (address / 16 in 14 bits; no address here reaches 2^18)
       const uint64_t ad0 = tc::sdesc(a0, 16, 512, tc::kLayoutSW64);
       const uint64_t bd0 = tc::sdesc(b0, 16, 512, tc::kLayoutSW64);
+      // Digit pairs (da, db) with da + db < 5 (pairs below 2^-35 of the leading one are
+      // dropped).  For one da the products with consecutive db go to consecutive classes,
+      // side by side in TMEM, and the B planes sit back to back in shared memory (64 rows
+      // each, the same swizzle phase): one product A_da [B_db0; B_db0+1; ..] covers them.
+      // One instruction has one accumulate flag, so the pair that opens class 4, (1, 3), is
+      // issued on its own: 5 instructions per k-step instead of 13.
+      struct Run { int da, db0, nb, open; };
+      constexpr Run kRuns[5] = {{0, 0, 4, 1}, {1, 0, 3, 0}, {1, 3, 1, 1}, {2, 0, 3, 0}, {3, 0, 2, 0}};
+      static_assert(kHS == 4 && kHClasses == 5, "the runs list the 13 pairs of 4 digits");
 #pragma unroll
       for (int k = 0; k < kHBK / 32; ++k) {
 #pragma unroll
-        for (int da = 0; da < kHS; ++da) {
-#pragma unroll
-          for (int db = 0; db < kHS; ++db) {
-            const int c = da + db;
-            if (c >= kHClasses) continue;  // pairs below 2^-35 of the leading one
-            const int first_a = c > kHS - 1 ? c - (kHS - 1) : 0;  // first pair of class c
-            const uint32_t acc = (kc == 0 && k == 0 && da == first_a) ? 0u : 1u;
-            tc::mma_i8(tmem + c * kHBN, ad0 + (uint64_t)((da * kHATile + k * 32) >> 4),
-                       bd0 + (uint64_t)((db * kHBTile + k * 32) >> 4), kHIdesc, acc);
-          }
+        for (int r = 0; r < 5; ++r) {
+          const Run u = kRuns[r];
+          const uint32_t acc = (kc == 0 && k == 0 && u.open) ? 0u : 1u;
+          tc::mma_i8(tmem + (u.da + u.db0) * kHBN, ad0 + (uint64_t)((u.da * kHATile + k * 32) >> 4),
+                     bd0 + (uint64_t)((u.db0 * kHBTile + k * 32) >> 4),
+                     hess_idesc((uint32_t)(u.nb * kHBN)), acc);
         }
       }
       tc::mma_commit(&empty[s]);

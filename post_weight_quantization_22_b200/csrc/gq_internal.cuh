@@ -160,7 +160,7 @@ cudaError_t launch_dgemm(const DgemmCall& c, cudaStream_t s);
 
 // ---- fp64-accurate products from int8 digit products (gq_split.cu) ----
 constexpr int kSplitDigits = 6;  // signed 7-bit digits per value
-constexpr int kSplitK = 256;     // depth of every split product (one super-panel)
+constexpr int kSplitK = 512;     // depth of every split product (one super-panel of the split path)
 // Digit planes of an operand: plane s is plane_rows x kSplitK int8 (K-major rows), planes
 // stacked at plane_rows x kSplitK bytes; ex[r] is the power-of-two scale exponent of row r.
 struct SplitOperand {
@@ -169,12 +169,14 @@ struct SplitOperand {
   int64_t plane_rows;
 };
 cudaError_t split_init_attributes();
-// digits of the rows of A (rows x kSplitK fp64, leading dimension lda, 16-byte aligned)
+// digits of the rows of A (rows x kSplitK fp64, leading dimension lda, 16-byte aligned);
+// tri: A is lower triangular from (0, 0), entries right of the diagonal count as zero
 cudaError_t launch_split_rows(const double* A, int64_t lda, int rows, SplitOperand op,
-                              cudaStream_t s);
-// digits of the columns of X (kSplitK rows x cols fp64, leading dimension ldx) as operand rows
+                              cudaStream_t s, int tri = 0);
+// digits of the columns of X (kSplitK rows x cols fp64, leading dimension ldx) as operand rows;
+// tri: X is lower triangular from (0, 0), entries above the diagonal count as zero
 cudaError_t launch_split_cols(const double* X, int64_t ldx, int cols, SplitOperand op,
-                              cudaStream_t s);
+                              cudaStream_t s, int tri = 0);
 // C[i][j] += alpha sum_k A(a_row0 + i, k) B(b_row0 + j, k), i < M, j < N (only j <= i when
 // lower), C fp64 row-major with leading dimension ldc.
 cudaError_t launch_split_gemm(double* C, int64_t ldc, int M, int N, const SplitOperand& A,

@@ -1,7 +1,7 @@
 // fp64-accurate GEMMs of the factorisation on the int8 tensor cores (exact digit products).
 //
-// The factor's time is in two families of large products, both of depth K = 256 (one
-// super-panel): the trailing Cholesky updates M[i][j] -= sum_k L[i][k] L[j][k] (lower part) and
+// The factor's time is in two families of large products, both of depth K = 512 (one
+// super-panel of the split path): the trailing Cholesky updates M[i][j] -= sum_k L[i][k] L[j][k] (lower part) and
 // the triangular inverse's block products T[i][j] += sum_k L[i][k] X[k][j].  On sm_100a the fp64
 // units cap them at ~37 TFLOP/s; the int8 tensor cores run ~100x faster per product, so each
 // fp64 operand is cut into exact int8 pieces (the splitting idea of Ozaki et al., "Error-free
@@ -13,7 +13,7 @@
 //   7-bit digits d_s in [-64, 64] (round to nearest at every step, so the first S digits carry
 //   7S = 42 bits of the row's scale; the remainder below 2^-(7S+1) is dropped).  Then
 //     sum_k a_ik b_jk = 2^(e_i + e_j) sum_{p + q <= S - 1} 2^-7(p+q+2) sum_k dA_p,ik dB_q,jk,
-//   each inner sum an exact int8 x int8 -> int32 tensor-core product (|sum| < 2^23 for K = 256),
+//   each inner sum an exact int8 x int8 -> int32 tensor-core product (|sum| < 2^24 for K = 512),
 //   grouped by class c = p + q into S int32 accumulators in tensor memory and combined in fp64
 //   in the epilogue.  The dropped pairs p + q >= S weigh below 2^-7(S+1) of the kept ones.
 //
@@ -24,12 +24,14 @@
 // Kernels: split_rows_kernel (digits of row-major rows, K contiguous: the panel's rows of L),
 // split_cols_kernel (digits of the columns of a row-major block, transposed through shared
 // memory: a block row of the inverse), and split_gemm_kernel (tcgen05 kind::i8, 128 x 64 tiles,
-// TMA-fed 3-stage ring, warp-specialised: a producer warp, an MMA warp and four epilogue warps;
-// a CTA runs a few tiles and hands the accumulator back to the MMA warp as soon as the epilogue
-// has read it, so the fp64 read-modify-write of C overlaps the next tile's products).  Eight
-// epilogue warps, two per TMEM lane quadrant, each read 32 columns of all classes, two classes
-// per load-and-wait, and each thread prefetches its own row of the C tile into L2 while the
-// products run.
+// TMA-fed 2-stage ring of 72 KB stages, warp-specialised: a producer warp, an MMA warp and
+// eight epilogue warps; a CTA runs a few tiles and hands the accumulator back to the MMA warp
+// as soon as the epilogue has read it, so the update of C overlaps the next tile's products).
+// For one A digit the products with consecutive B digits are one instruction of N up to 256
+// (their B planes sit back to back in shared memory, their classes side by side in TMEM).
+// The epilogue warps, two per TMEM lane quadrant, each read 32 columns of all classes, two
+// classes per load-and-wait; each thread stages its row's 32 scaled values in shared memory
+// and adds them to C with one bulk fp64 reduce-add, done at L2 (C is never loaded into the SM).
 #include "gq_internal.cuh"
 #include "gq_tc.cuh"
 
@@ -38,20 +40,24 @@ namespace gq {
 namespace {
 constexpr int kSBM = 128, kSBN = 64;  // output tile
 constexpr int kSBK = 64;              // K bytes per stage (two MMA k-steps of 32)
-constexpr int kSStages = 3;
+constexpr int kSStages = 2;
 constexpr uint32_t kSATile = kSBM * kSBK;                  // 8 KB per digit plane
 constexpr uint32_t kSBTile = kSBN * kSBK;                  // 4 KB per digit plane
 constexpr uint32_t kSStage = kSplitDigits * (kSATile + kSBTile);  // 72 KB
-constexpr size_t kSSmem = kSStages * kSStage + 1024 + 256;
+constexpr int kSEpiPitch = 32 * 8 + 16;  // bytes per staged row of 32 doubles (padded: the
+                                         // 16-byte stores of a warp spread over the banks)
+constexpr uint32_t kSEpiBytes = 8 * 32 * kSEpiPitch;  // eight epilogue warps x 32 rows
+constexpr size_t kSSmem = kSStages * kSStage + 1024 + 256 + kSEpiBytes;
 constexpr int kSEpiWarps = 8;        // two per TMEM lane quadrant, 32 columns each
 constexpr int kSThreads = 32 * (2 + kSEpiWarps);  // warp 0 producer, warp 1 MMA, then epilogue
 constexpr int kSTilesPerCta = 4;     // CTAs retire regularly, so other streams' kernels get SMs
 constexpr uint32_t kSTmemCols = 512; // kSplitDigits x 64 columns, rounded up to a power of two
 static_assert(kSplitDigits * kSBN <= (int)kSTmemCols, "class accumulators must fit in TMEM");
 static_assert(kSplitDigits % 2 == 0, "the epilogue reads the classes two at a time");
-// int8 x int8 -> s32, A and B K-major, M 128, N 64
-constexpr uint32_t kSIdesc = (2u << 4) | (1u << 7) | (1u << 10) |
-                             ((uint32_t)(kSBN >> 3) << 17) | ((uint32_t)(kSBM >> 4) << 24);
+// int8 x int8 -> s32, A and B K-major, M 128, N columns (a multiple of 16, at most 256)
+__host__ __device__ constexpr uint32_t split_idesc(uint32_t N) {
+  return (2u << 4) | (1u << 7) | (1u << 10) | ((N >> 3) << 17) | ((uint32_t)(kSBM >> 4) << 24);
+}
 
 struct SplitArgs {
   double* C;
@@ -106,88 +112,50 @@ __device__ __forceinline__ void tile_of(const SplitArgs& g, int t, int& bi, int&
 }  // namespace
 
 // ---------------------------------------------------------------------------------------------
-// digit splits (K = kSplitK = 256 values per operand row)
+// digit splits (K = kSplitK values per operand row)
 // ---------------------------------------------------------------------------------------------
-// Row r of A (rows x 256, leading dimension lda): exponent ex[r] and digit planes
-// D[s][r][k] (plane stride plane_rows x 256 bytes).  One warp per row; lane l takes k = 8l..8l+7.
+// Row r of A (rows x kSplitK, leading dimension lda): exponent ex[r] and digit planes
+// D[s][r][k] (plane stride plane_rows x kSplitK bytes).  One warp per row; lane l takes the 8
+// consecutive values k = 256 g + 8 l .. + 7 of each 256-wide group g.  tri: A is a lower
+// triangular block whose diagonal starts at (0, 0); entries k > r count as zero (whatever
+// the memory holds there).
+constexpr int kRowGroups = kSplitK / 256;
 __global__ void __launch_bounds__(256) split_rows_kernel(const double* A, int64_t lda, int rows,
-                                                         int64_t plane_rows, int8_t* D, int* ex) {
+                                                         int64_t plane_rows, int8_t* D, int* ex,
+                                                         int tri) {
   const int r = blockIdx.x * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (r >= rows) return;
-  const double* src = A + (int64_t)r * lda + 8 * lane;
-  double v[8];
+  double v[kRowGroups][8];
 #pragma unroll
-  for (int i = 0; i < 8; i += 2) {
-    const double2 x = *reinterpret_cast<const double2*>(src + i);
-    v[i] = x.x;
-    v[i + 1] = x.y;
+  for (int g = 0; g < kRowGroups; ++g) {
+    const double* src = A + (int64_t)r * lda + 256 * g + 8 * lane;
+#pragma unroll
+    for (int i = 0; i < 8; i += 2) {
+      const double2 x = *reinterpret_cast<const double2*>(src + i);
+      const int k = 256 * g + 8 * lane + i;
+      v[g][i] = (tri && k > r) ? 0.0 : x.x;
+      v[g][i + 1] = (tri && k + 1 > r) ? 0.0 : x.y;
+    }
   }
   double mx = 0.0;
 #pragma unroll
-  for (int i = 0; i < 8; ++i) mx = fmax(mx, fabs(v[i]));
+  for (int g = 0; g < kRowGroups; ++g)
+#pragma unroll
+    for (int i = 0; i < 8; ++i) mx = fmax(mx, fabs(v[g][i]));
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) mx = fmax(mx, __shfl_xor_sync(0xffffffffu, mx, o));
   const int e = split_exponent(mx);
   if (lane == 0) ex[r] = e;
   const double sc = pow2(-e);
-  uint64_t packed[kSplitDigits];
 #pragma unroll
-  for (int s = 0; s < kSplitDigits; ++s) packed[s] = 0;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    double x = v[i] * sc;
-#pragma unroll
-    for (int s = 0; s < kSplitDigits; ++s) {
-      x *= 128.0;
-      const double q = rint(x);
-      x -= q;
-      packed[s] |= (uint64_t)(uint8_t)(int8_t)(int)q << (8 * i);
-    }
-  }
-#pragma unroll
-  for (int s = 0; s < kSplitDigits; ++s)
-    *reinterpret_cast<uint64_t*>(D + (int64_t)s * plane_rows * kSplitK + (int64_t)r * kSplitK +
-                                 8 * lane) = packed[s];
-}
-
-// Column j of X (256 rows x cols, leading dimension ldx) as an operand row: exponent ex[j] and
-// digit planes D[s][j][k] = digit s of X[k][j] 2^-ex[j].  A CTA takes 32 columns; thread
-// (ty, tx) = (tid / 32, tid % 32) reads X[32 ty .. 32 ty + 31][j0 + tx] (coalesced along tx),
-// packs the digits of 8 consecutive k into one 8-byte shared-memory store per plane, and the CTA
-// writes the 32 rows of each plane out with coalesced 8-byte stores.
-constexpr int kColPitch = kSplitK + 8;  // bytes per staged row (8-byte stores at distinct banks)
-constexpr size_t kSplitColsSmem = (size_t)kSplitDigits * 32 * kColPitch + 8 * 32 * sizeof(double);
-__global__ void __launch_bounds__(256) split_cols_kernel(const double* X, int64_t ldx, int cols,
-                                                         int64_t plane_rows, int8_t* D, int* ex) {
-  extern __shared__ __align__(16) uint8_t sc_smem[];
-  uint8_t* sD = sc_smem;  // [s][32 columns][kColPitch]
-  double* red = reinterpret_cast<double*>(sc_smem + (size_t)kSplitDigits * 32 * kColPitch);
-  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
-  const int j0 = blockIdx.x * 32, j = j0 + tx;
-  const bool act = j < cols;
-  double v[32];
-#pragma unroll
-  for (int i = 0; i < 32; ++i) v[i] = act ? X[(int64_t)(32 * ty + i) * ldx + j] : 0.0;
-  double mx = 0.0;
-#pragma unroll
-  for (int i = 0; i < 32; ++i) mx = fmax(mx, fabs(v[i]));
-  red[ty * 32 + tx] = mx;
-  __syncthreads();
-  mx = 0.0;
-#pragma unroll
-  for (int y = 0; y < 8; ++y) mx = fmax(mx, red[y * 32 + tx]);
-  const int e = split_exponent(mx);
-  if (ty == 0 && act) ex[j] = e;
-  const double sc = pow2(-e);
-#pragma unroll
-  for (int g8 = 0; g8 < 4; ++g8) {
+  for (int g = 0; g < kRowGroups; ++g) {
     uint64_t packed[kSplitDigits];
 #pragma unroll
     for (int s = 0; s < kSplitDigits; ++s) packed[s] = 0;
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-      double x = v[8 * g8 + i] * sc;
+      double x = v[g][i] * sc;
 #pragma unroll
       for (int s = 0; s < kSplitDigits; ++s) {
         x *= 128.0;
@@ -198,19 +166,76 @@ __global__ void __launch_bounds__(256) split_cols_kernel(const double* X, int64_
     }
 #pragma unroll
     for (int s = 0; s < kSplitDigits; ++s)
-      *reinterpret_cast<uint64_t*>(sD + ((size_t)s * 32 + tx) * kColPitch + 32 * ty + 8 * g8) =
+      *reinterpret_cast<uint64_t*>(D + (int64_t)s * plane_rows * kSplitK + (int64_t)r * kSplitK +
+                                   256 * g + 8 * lane) = packed[s];
+  }
+}
+
+// Column j of X (kSplitK rows x cols, leading dimension ldx) as an operand row: exponent ex[j]
+// and digit planes D[s][j][k] = digit s of X[k][j] 2^-ex[j].  A CTA takes 32 columns; thread
+// (ty, tx) = (tid / 32, tid % 32) owns rows kPerTy ty .. + kPerTy - 1 of column j0 + tx (reads
+// coalesced along tx): a max pass, then per 8 consecutive rows the digits packed into one 8-byte
+// shared-memory store per plane; the CTA writes the 32 rows of each plane out with coalesced
+// 8-byte stores.  tri: X is a lower triangular block whose diagonal starts at (0, 0); entries
+// with row k < column j count as zero.
+constexpr int kPerTy = kSplitK / 8;
+constexpr int kColPitch = kSplitK + 8;  // bytes per staged row (8-byte stores at distinct banks)
+constexpr size_t kSplitColsSmem = (size_t)kSplitDigits * 32 * kColPitch + 8 * 32 * sizeof(double);
+__global__ void __launch_bounds__(256) split_cols_kernel(const double* X, int64_t ldx, int cols,
+                                                         int64_t plane_rows, int8_t* D, int* ex,
+                                                         int tri) {
+  extern __shared__ __align__(16) uint8_t sc_smem[];
+  uint8_t* sD = sc_smem;  // [s][32 columns][kColPitch]
+  double* red = reinterpret_cast<double*>(sc_smem + (size_t)kSplitDigits * 32 * kColPitch);
+  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
+  const int j0 = blockIdx.x * 32, j = j0 + tx;
+  const bool act = j < cols;
+  const double* xcol = X + (int64_t)(kPerTy * ty) * ldx + j;
+  const int kmin = tri ? j : 0;  // rows below kmin of this column count as zero
+  double mx = 0.0;
+  if (act)
+    for (int i = 0; i < kPerTy; ++i)
+      if (kPerTy * ty + i >= kmin) mx = fmax(mx, fabs(xcol[(int64_t)i * ldx]));
+  red[ty * 32 + tx] = mx;
+  __syncthreads();
+  mx = 0.0;
+#pragma unroll
+  for (int y = 0; y < 8; ++y) mx = fmax(mx, red[y * 32 + tx]);
+  const int e = split_exponent(mx);
+  if (ty == 0 && act) ex[j] = e;
+  const double sc = pow2(-e);
+#pragma unroll 1
+  for (int g8 = 0; g8 < kPerTy / 8; ++g8) {
+    uint64_t packed[kSplitDigits];
+#pragma unroll
+    for (int s = 0; s < kSplitDigits; ++s) packed[s] = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int k = kPerTy * ty + 8 * g8 + i;
+      double x = (act && k >= kmin) ? xcol[(int64_t)(8 * g8 + i) * ldx] * sc : 0.0;
+#pragma unroll
+      for (int s = 0; s < kSplitDigits; ++s) {
+        x *= 128.0;
+        const double q = rint(x);
+        x -= q;
+        packed[s] |= (uint64_t)(uint8_t)(int8_t)(int)q << (8 * i);
+      }
+    }
+#pragma unroll
+    for (int s = 0; s < kSplitDigits; ++s)
+      *reinterpret_cast<uint64_t*>(sD + ((size_t)s * 32 + tx) * kColPitch + kPerTy * ty + 8 * g8) =
           packed[s];
   }
   __syncthreads();
-  // plane s, row j0 + rr: 256 bytes = 32 words; 256 threads write 8 rows per pass
+  // plane s, rows j0 .. j0 + 31: kSplitK / 8 words each, written in order by consecutive threads
+  constexpr int kWords = kSplitK / 8;
   for (int s = 0; s < kSplitDigits; ++s) {
-#pragma unroll
-    for (int pass = 0; pass < 4; ++pass) {
-      const int rr = pass * 8 + ty;
+    for (int idx = threadIdx.x; idx < 32 * kWords; idx += 256) {
+      const int rr = idx / kWords, w = idx % kWords;
       if (j0 + rr < cols)
         *reinterpret_cast<uint64_t*>(D + (int64_t)s * plane_rows * kSplitK +
-                                     (int64_t)(j0 + rr) * kSplitK + 8 * tx) =
-            *reinterpret_cast<const uint64_t*>(sD + ((size_t)s * 32 + rr) * kColPitch + 8 * tx);
+                                     (int64_t)(j0 + rr) * kSplitK + 8 * w) =
+            *reinterpret_cast<const uint64_t*>(sD + ((size_t)s * 32 + rr) * kColPitch + 8 * w);
     }
   }
 }
@@ -306,16 +331,23 @@ __global__ void __launch_bounds__(kSThreads, 1)
           // field holds address / 16 in 14 bits, and no address here reaches 2^18)
           const uint64_t ad0 = tc::sdesc(a0, 16, 512, tc::kLayoutSW64);
           const uint64_t bd0 = tc::sdesc(b0, 16, 512, tc::kLayoutSW64);
+          // Digit pairs (p, q) with p + q < S (weight >= 2^-7(S+1)).  For one p the products
+          // with q = 0 .. S-1-p go to classes p .. S-1, which sit side by side in TMEM, and the
+          // B planes q = 0 .. sit back to back in shared memory (64 rows each, the same swizzle
+          // phase), so they are one product A_p [B_0; B_1; ..] with N = 64 (S - p), cut at
+          // N = 256: 8 instructions per k-step instead of 21, and each A plane read once.
 #pragma unroll
           for (int k = 0; k < kSBK / 32; ++k) {
 #pragma unroll
             for (int p = 0; p < kSplitDigits; ++p) {
 #pragma unroll
-              for (int q = 0; p + q < kSplitDigits; ++q) {  // digit pairs of weight >= 2^-7(S+1)
-                // p = 0 is the first pair of class q: it opens the accumulator of the tile
+              for (int q0 = 0; p + q0 < kSplitDigits; q0 += 256 / kSBN) {
+                const int nq = min(kSplitDigits - p - q0, 256 / kSBN);
+                // p = 0 opens every class accumulator of the tile
                 const uint32_t acc = (kc == 0 && k == 0 && p == 0) ? 0u : 1u;
-                tc::mma_i8(tmem + (p + q) * kSBN, ad0 + (uint64_t)((p * kSATile + k * 32) >> 4),
-                           bd0 + (uint64_t)((q * kSBTile + k * 32) >> 4), kSIdesc, acc);
+                tc::mma_i8(tmem + (p + q0) * kSBN, ad0 + (uint64_t)((p * kSATile + k * 32) >> 4),
+                           bd0 + (uint64_t)((q0 * kSBTile + k * 32) >> 4),
+                           split_idesc((uint32_t)(nq * kSBN)), acc);
               }
             }
           }
@@ -329,6 +361,9 @@ __global__ void __launch_bounds__(kSThreads, 1)
   } else {  // epilogue: warp w reads TMEM lanes 32 (w % 4) .., columns 32 ((w - 2) / 4) ..
     const int quad = warp & 3, half = (warp - 2) >> 2;
     double* colscale = s_colscale[warp - 2];
+    // this thread's staging row (a 32-bit shared-memory address)
+    const uint32_t srow = tc::smem_u32(base + kSStages * kSStage + 256) +
+                          (uint32_t)(((warp - 2) * 32 + lane) * kSEpiPitch);
     int done = 0;
     for (int t = t_begin; t < t_end; ++t, ++done) {
       int bi, bj;
@@ -339,7 +374,6 @@ __global__ void __launch_bounds__(kSThreads, 1)
       const bool rowok = i < g.M && jt < g.N;
       const bool vec = rowok && jt + 32 <= g.N && (!g.lower || jt + 31 <= i) &&
                        ((reinterpret_cast<uintptr_t>(crow) & 15) == 0);
-      if (vec) tc::bulk_prefetch_l2(crow, 32 * sizeof(double));  // this row's part of the tile
       // the columns' scales into this warp's slice of shared memory, one load per column (read
       // inside the store loop, they would be reloaded after every store to C: the compiler
       // cannot rule out that C aliases the exponents).  Warp-private: no barrier beyond the
@@ -373,21 +407,19 @@ __global__ void __launch_bounds__(kSThreads, 1)
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(tempty);
       if (vec) {
+        // The row's 32 scaled values into its staging row, then one bulk reduce-add of 256
+        // bytes into C at L2: no load of C into the SM.  si cs acc is exact (a power-of-two
+        // scaling of acc), so C + si cs acc rounds once, as fma(si cs, acc, C) would.
         const double si = g.alpha * pow2(g.ea[g.a0 + i]);
+        tc::bulk_wait_group_read0();  // the previous tile's reduce has read this staging row
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {  // 16 columns at a time, every load in flight together
-          double2 cv[8];
-#pragma unroll
-          for (int u = 0; u < 8; ++u) cv[u] = *reinterpret_cast<const double2*>(crow + 16 * h + 2 * u);
-#pragma unroll
-          for (int u = 0; u < 8; ++u) {
-            const int j = 16 * h + 2 * u;
-            const double2 cs = *reinterpret_cast<const double2*>(colscale + j);
-            cv[u].x = fma(si * cs.x, acc[j], cv[u].x);
-            cv[u].y = fma(si * cs.y, acc[j + 1], cv[u].y);
-            *reinterpret_cast<double2*>(crow + j) = cv[u];
-          }
+        for (int j = 0; j < 32; j += 2) {
+          const double2 cs = *reinterpret_cast<const double2*>(colscale + j);
+          tc::st_shared_f64x2(srow + 8 * j, (si * cs.x) * acc[j], (si * cs.y) * acc[j + 1]);
         }
+        tc::fence_proxy_async_smem();  // the stores above, visible to the bulk copy
+        tc::bulk_reduce_add_f64(crow, srow, 32 * sizeof(double));
+        tc::bulk_commit_group();
       } else if (rowok) {
         const double si = g.alpha * pow2(g.ea[g.a0 + i]);
 #pragma unroll
@@ -401,6 +433,7 @@ __global__ void __launch_bounds__(kSThreads, 1)
 
   // Teardown: no copy or product may be in flight when the CTA leaves.  In the normal path
   // every phase below has completed already; after a timeout the waits are bounded.
+  if (warp >= 2) tc::bulk_wait_group0();  // this thread's reduces into C have completed
   __syncthreads();
   if (warp == 0 && lane == 0) {
     const int issued = s_issued;
@@ -432,20 +465,20 @@ cudaError_t split_init_attributes() {
 }
 
 cudaError_t launch_split_rows(const double* A, int64_t lda, int rows, SplitOperand op,
-                              cudaStream_t s) {
+                              cudaStream_t s, int tri) {
   if (rows <= 0) return cudaSuccess;
   if ((reinterpret_cast<uintptr_t>(A) & 15) || (lda & 1)) return cudaErrorInvalidValue;
   split_rows_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, s>>>(A, lda, rows, op.plane_rows,
-                                                               op.digits, op.ex);
+                                                               op.digits, op.ex, tri);
   count_launches(1);
   return cudaGetLastError();
 }
 
 cudaError_t launch_split_cols(const double* X, int64_t ldx, int cols, SplitOperand op,
-                              cudaStream_t s) {
+                              cudaStream_t s, int tri) {
   if (cols <= 0) return cudaSuccess;
   split_cols_kernel<<<(unsigned)((cols + 31) / 32), 256, kSplitColsSmem, s>>>(
-      X, ldx, cols, op.plane_rows, op.digits, op.ex);
+      X, ldx, cols, op.plane_rows, op.digits, op.ex, tri);
   count_launches(1);
   return cudaGetLastError();
 }
