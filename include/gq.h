@@ -298,6 +298,44 @@ gq_status gq_ssqr_quantize_layer(const void* d_W, gq_dtype w_dtype, int64_t m, i
                                  float* d_values, int64_t nnz_capacity, double* d_loss,
                                  void* d_ws, size_t ws_bytes, gq_stream_t stream);
 
+/* Workspace bytes gq_hptq_quantize_layer needs for an m x n layer (0 if out of range). */
+size_t gq_hptq_workspace_size(int64_t m, int64_t n);
+
+/*
+ * HPTQ rate control ("The Geometry of LLM Quantization", section 3, HPTQ: normal and outlier
+ * weights share one unconstrained integer lattice, and Huffman coding of the integers gives a
+ * variable bit width that meets a compression budget).  The layer is quantized with the GPTQ
+ * column loop on the lattice s Z of each row (zero point 0, no clamp), s = alpha (hi - lo) /
+ * (2^b - 1) with [lo, hi] (lo <= 0 <= hi) the row's range and ONE factor alpha for the whole
+ * layer.  The budget counts the canonical Huffman code of all m n integers alone (as
+ * gq_huffman_encode writes it; scales and the code table are not counted), in bits per weight:
+ * alpha is the smallest factor (finest lattice) whose coded size is at most budget * m * n
+ * bits, found by doubling alpha from 1 until the layer fits (at most max_doublings times) and
+ * then `steps` bisection steps in log2 alpha between the last value that did not fit (2^-8
+ * when alpha = 1 already fits) and the one that does; the result always fits.  alpha = 2^t is
+ * computed on the host as pow(2, t).  Natural column order.  SYNCHRONIZES `stream` once per
+ * pass of the search (1 + doublings + steps + 1 passes).
+ *
+ *   d_W, w_dtype, m, n, d_U, d_dead, d_delta   as gq_quantize_layer (reverse = 0).
+ *   bits          2..8 (the min-max step the factor multiplies).   budget  > 0, bits/weight.
+ *   steps         0..60 (12 usual).   max_doublings  0..30.
+ *   d_codes       m x n int32, written: the integers, original column order.
+ *   d_scales      m fp32, written: the step s of each row (dequantized weight = s * code).
+ *   d_alpha       1 double, written: the chosen factor.
+ *   d_total_bits  1 int64, written: the coded size at that factor.
+ *   d_loss        3 doubles, written as by gq_quantize_layer ([2], the Theorem 5 sum, is the
+ *                 no-clipping bound of the chosen lattice).
+ *   d_ws          workspace of at least gq_hptq_workspace_size(m, n) bytes.
+ * Device-detected errors: GQ_ERR_NO_FIT (the layer does not fit even after max_doublings),
+ * GQ_ERR_UNSUPPORTED (a pass spans more than 4096 distinct integers).
+ */
+gq_status gq_hptq_quantize_layer(const void* d_W, gq_dtype w_dtype, int64_t m, int64_t n,
+                                 const float* d_U, const uint8_t* d_dead, const double* d_delta,
+                                 int bits, double budget, int steps, int max_doublings,
+                                 int32_t* d_codes, float* d_scales, double* d_alpha,
+                                 int64_t* d_total_bits, double* d_loss, void* d_ws,
+                                 size_t ws_bytes, gq_stream_t stream);
+
 /*
  * The ZSIC column factors kappa_j = U_jj / geomean(U_kk) ("WaterSIC", section 2) of a factor
  * from gq_prepare_hinv(_ordered), exactly as gq_quantize_layer uses them with spacing = 1; a

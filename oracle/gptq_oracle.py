@@ -49,6 +49,8 @@ __all__ = [
     "babai_sic_reverse",
     "ssqr_columns",
     "ssqr_search",
+    "hptq_rate",
+    "hptq_search",
     "zsic_spacing",
     "pack_codes",
     "huffman_lengths",
@@ -241,7 +243,7 @@ def gptq_columns(W, U, bits: int, group: int = 0, clip: bool = True, alpha=None,
     clip=False: codes are unconstrained integers (no clamp) on the ``clipfree_grid`` with the
     per-row factor ``alpha`` (group must be 0).  clip="unbounded" (HPTQ reading, [GEOM]
     section 3: one unconstrained integer grid for normal and outlier weights): the lattice
-    s Z with the min-max step of the row, zero point 0, no clamp.  ``grid`` = (s, z) fixes the per-row grid
+    s Z with the min-max step of the row (times ``alpha`` when given), zero point 0, no clamp.  ``grid`` = (s, z) fixes the per-row grid
     instead (a fixed lattice).  ``col_scale`` (per-row grids only) multiplies the step of
     column j by col_scale[j]: the grid of column j is s col_scale[j] (c - z).
 
@@ -291,6 +293,8 @@ def gptq_columns(W, U, bits: int, group: int = 0, clip: bool = True, alpha=None,
             s, z = (np.asarray(g, dtype=np.float64).copy() for g in grid)
         elif unbounded:
             s, _ = minmax_grid(w, bits)
+            if alpha is not None:
+                s = s * _f64(alpha)
             z = np.zeros(m)
         elif clip:
             s, z = minmax_grid(w, bits)
@@ -387,6 +391,62 @@ def ssqr_search(W, U, bits: int, density: float, steps: int = 20, max_doublings:
         lo = np.where(ok, lo, mid)
     alpha = 2.0 ** hi
     return ssqr_columns(w, U, bits, alpha), alpha, lo
+
+
+def hptq_rate(codes) -> float:
+    """Bits per weight of the canonical Huffman code of integer codes ([GEOM] section 3, HPTQ):
+    the symbols are the codes minus their minimum, counted over the whole array; the size is
+    sum over symbols of count x code length (``huffman_lengths``), divided by the number of
+    codes."""
+    c = np.asarray(codes, dtype=np.int64)
+    counts = np.bincount((c - c.min()).ravel())
+    ln = huffman_lengths(counts)
+    return float(np.sum(counts * ln[:counts.size])) / c.size
+
+
+def hptq_search(W, U, bits: int, budget: float, steps: int = 12, max_doublings: int = 12):
+    """HPTQ's rate control ([GEOM] section 3, HPTQ: one unconstrained integer lattice for normal
+    and outlier weights, Huffman-coded so that a variable bit width meets a compression budget).
+
+    reading: one factor alpha for the whole layer multiplies every row's min-max step (the
+    unbounded lattice of ``gptq_columns``); the budget counts the Huffman-coded integers alone
+    (``hptq_rate``), in bits per weight; alpha is the smallest factor (finest lattice) whose
+    coded size, sum of count x length, is at most budget x (number of weights) bits.  The search
+    is the one ``ssqr_search`` runs per row, here for the layer: alpha = 2^t from t = 0, t += 1
+    until the layer fits (at most ``max_doublings`` times), then ``steps`` bisection steps in t
+    between the last value that did not fit (t - 1, or -8 when t = 0 fits) and the one that
+    does.  alpha = 2.0 ** t.  Returns (gptq_columns result at the chosen alpha, alpha, coded
+    bits at alpha, the last t that did not fit).
+    """
+    w = _f64(W)
+    m, n = w.shape
+    limit = budget * float(m * n)
+
+    def coded_bits(t):
+        r = gptq_columns(w, U, bits, clip="unbounded", alpha=np.full(m, 2.0 ** t))
+        c = r["codes"]
+        counts = np.bincount((c - c.min()).ravel())
+        return r, int(np.sum(counts * huffman_lengths(counts)[:counts.size]))
+
+    hi = 0.0
+    r, b = coded_bits(hi)
+    lo = -8.0
+    doublings = 0
+    while b > limit:
+        if doublings == max_doublings:
+            raise ValueError("the layer exceeds the budget even at the widest lattice")
+        lo, hi = hi, hi + 1.0
+        r, b = coded_bits(hi)
+        doublings += 1
+    for _ in range(steps):
+        mid = 0.5 * (lo + hi)
+        _, bm = coded_bits(mid)
+        if bm <= limit:
+            hi = mid
+        else:
+            lo = mid
+    r, b = coded_bits(hi)
+    return r, 2.0 ** hi, b, lo
 
 
 def babai_sic_reverse(W, L, bits: int, clip: bool = False, alpha=None):

@@ -328,6 +328,43 @@ gq_status gq_ssqr_quantize_layer(const void* d_W, gq_dtype w_dtype, int64_t m, i
   return run_ssqr(a, o, (cudaStream_t)stream);  // synchronizes per doubling round
 }
 
+size_t gq_hptq_workspace_size(int64_t m, int64_t n) {
+  if (m < 1 || m > kMaxM || n < 1 || n > kMaxN || m * n > (int64_t(1) << 31) - 1) return 0;
+  return hptq_ws_bytes(m, n);
+}
+
+gq_status gq_hptq_quantize_layer(const void* d_W, gq_dtype w_dtype, int64_t m, int64_t n,
+                                 const float* d_U, const uint8_t* d_dead, const double* d_delta,
+                                 int bits, double budget, int steps, int max_doublings,
+                                 int32_t* d_codes, float* d_scales, double* d_alpha,
+                                 int64_t* d_total_bits, double* d_loss, void* d_ws,
+                                 size_t ws_bytes, gq_stream_t stream) {
+  if (m < 1 || m > kMaxM || n < 1 || n > kMaxN || m * n > (int64_t(1) << 31) - 1)
+    return GQ_ERR_INVALID_ARG;
+  if (w_dtype != GQ_BF16 && w_dtype != GQ_FP32) return GQ_ERR_INVALID_ARG;
+  if (bits < 2 || bits > 8 || !(budget > 0.0 && budget < 64.0)) return GQ_ERR_INVALID_ARG;
+  if (steps < 0 || steps > 60 || max_doublings < 0 || max_doublings > 30)
+    return GQ_ERR_INVALID_ARG;
+  if (!d_W || !d_U || !d_codes || !d_scales || !d_alpha || !d_total_bits || !d_loss || !d_ws)
+    return GQ_ERR_INVALID_ARG;
+  if (!aligned256(d_ws) || ws_bytes < hptq_ws_bytes(m, n)) return GQ_ERR_WORKSPACE;
+  if ((reinterpret_cast<uintptr_t>(d_U) & 15u) != 0 ||
+      (reinterpret_cast<uintptr_t>(d_alpha) & 7u) != 0 ||
+      (reinterpret_cast<uintptr_t>(d_total_bits) & 7u) != 0)
+    return GQ_ERR_INVALID_ARG;
+  gq_status st = ensure_device_setup();
+  if (st != GQ_OK) return st;
+  QuantArgs a{};
+  a.W = d_W; a.wt = w_dtype; a.m = m; a.n = n; a.U = d_U; a.dead = d_dead; a.delta = d_delta;
+  a.cfg = gq_quant_cfg{bits, 0, 0, 2, 1.25f, 0, 0};
+  a.codes = reinterpret_cast<uint32_t*>(d_codes); a.scales = d_scales; a.zeros = nullptr;
+  a.loss = d_loss; a.ws = d_ws; a.perm = nullptr;
+  HptqArgs o{};
+  o.budget = budget; o.steps = steps; o.max_doublings = max_doublings; o.alpha = d_alpha;
+  o.total_bits = reinterpret_cast<long long*>(d_total_bits);
+  return run_hptq(a, o, (cudaStream_t)stream);  // synchronizes once per pass
+}
+
 gq_status gq_zsic_spacing(const float* d_U, int64_t n, double* d_kappa, gq_stream_t stream) {
   if (n < 1 || n > kMaxN || !d_U || !d_kappa) return GQ_ERR_INVALID_ARG;
   gq_status st = ensure_device_setup();

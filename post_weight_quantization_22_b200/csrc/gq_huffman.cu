@@ -384,4 +384,23 @@ cudaError_t launch_huffman(const int* codes, int64_t count, unsigned long long* 
   return cudaGetLastError();
 }
 
+// The code's statistics alone (range, histogram, build): info[2] = the total bits of the
+// Huffman-coded stream, lengths / words the canonical code.  Nothing is encoded.
+cudaError_t launch_huffman_stats(const int* codes, int64_t count, uint8_t* lengths,
+                                 unsigned long long* words, long long* info, void* ws,
+                                 cudaStream_t s) {
+  HuffLayout L = huff_layout(ws, count);
+  cudaError_t e;
+  if ((e = cudaMemsetAsync(L.hdr, 0, sizeof(WsHeader), s))) return e;
+  huff_init_kernel<<<1, 1024, 0, s>>>(L.state, L.hist);
+  const unsigned grid = (unsigned)std::min<int64_t>((count + 255) / 256, 148 * 8);
+  huff_range_kernel<<<grid, 256, 0, s>>>(codes, count, L.state);
+  huff_hist_kernel<<<grid, 256, 0, s>>>(codes, count, L.state, L.hist);
+  // a stream capacity no total reaches (2^63 bits): only the code's own limits are reported
+  huff_build_kernel<<<1, 1024, kHuffBuildSmem, s>>>(L.state, L.hist, (int64_t)1 << 57, lengths,
+                                                    words, info, L.hdr);
+  count_launches(4);
+  return cudaGetLastError();
+}
+
 }  // namespace gq

@@ -76,6 +76,7 @@ struct QuantArgs {
   double* loss;
   void* ws;
   const int* perm;  // processing order (null: natural, or reversed when cfg.reverse)
+  double lattice_alpha = 1.0;  // unconstrained lattice (clip 2): step = min-max step x this
 };
 size_t quantize_ws_bytes(int64_t m, int64_t n, const gq_quant_cfg& cfg);
 // SSQR outlier search (cfg.clip = 3, one grid per row, natural order): its workspace, and the
@@ -98,6 +99,21 @@ cudaError_t huffman_init_attributes();
 cudaError_t launch_huffman(const int* codes, int64_t count, unsigned long long* stream_words,
                            int64_t nwords, uint8_t* lengths, unsigned long long* words,
                            long long* info, void* ws, cudaStream_t s);
+// range, histogram and canonical code only: info[2] = total bits of the coded stream
+cudaError_t launch_huffman_stats(const int* codes, int64_t count, uint8_t* lengths,
+                                 unsigned long long* words, long long* info, void* ws,
+                                 cudaStream_t s);
+// HPTQ rate control (cfg.clip = 2, one grid per row, natural order): the smallest lattice
+// factor alpha whose Huffman-coded codes fit a budget in bits per weight.
+size_t hptq_ws_bytes(int64_t m, int64_t n);
+struct HptqArgs {
+  double budget;          // bits per weight
+  int steps, max_doublings;
+  double* alpha;          // 1, out
+  long long* total_bits;  // 1, out: coded size of the codes at alpha
+};
+// Synchronizes the stream once per pass of the search.
+gq_status run_hptq(const QuantArgs& a, const HptqArgs& o, cudaStream_t s);
 // Returns GQ_OK or an error; the clip-free ladder synchronizes the stream per round.
 gq_status run_quantize(const QuantArgs& a, cudaStream_t s);
 // Synchronizes the stream once per doubling round of the search.

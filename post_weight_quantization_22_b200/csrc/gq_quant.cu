@@ -122,6 +122,35 @@ size_t quantize_ws_bytes(int64_t m, int64_t n, const gq_quant_cfg& cfg) {
 
 size_t ssqr_ws_bytes(int64_t m, int64_t n) { return q_layout(nullptr, m, n, false, true).bytes; }
 
+// HPTQ: the quantize workspace (unconstrained lattice), then the Huffman statistics' workspace,
+// the code table and the info words.
+struct HptqLayout {
+  QLayout q;
+  void* huff_ws;
+  uint8_t* lengths;
+  unsigned long long* words;
+  long long* info;
+  uint8_t* zeros;  // m: the per-row zero points the grid kernel writes (all 0 here)
+  size_t bytes;
+};
+static HptqLayout hptq_layout(void* ws, int64_t m, int64_t n) {
+  HptqLayout H;
+  H.q = q_layout(ws, m, n, true, false);
+  Carver c(ws);
+  c.off = H.q.bytes;
+  c.off = (c.off + 255) / 256 * 256;
+  H.huff_ws = ws ? static_cast<char*>(ws) + c.off : nullptr;
+  c.off += huffman_ws_bytes(m * n);
+  c.off = (c.off + 255) / 256 * 256;
+  H.words = c.take<unsigned long long>(4096);
+  H.info = c.take<long long>(4);
+  H.lengths = c.take<uint8_t>(4096);
+  H.zeros = c.take<uint8_t>((size_t)m);
+  H.bytes = c.off;
+  return H;
+}
+size_t hptq_ws_bytes(int64_t m, int64_t n) { return hptq_layout(nullptr, m, n).bytes; }
+
 // ------------------------------------------------------------------------------------------
 // setup kernels
 // ------------------------------------------------------------------------------------------
@@ -188,7 +217,8 @@ __global__ void perm_invert_kernel(const int* perm, int64_t n, int* iperm, WsHea
 // 2 unconstrained lattice; 3 outliers (centred, step widened by the fp64 factor alpha_d).
 __global__ void q_row_grid_kernel(const float* Wf, int64_t n, int64_t k_rows, const int* rowlist,
                                   int bits, int clip, const float* alpha, const double* alpha_d,
-                                  double* row_s, double* row_z, float* scales, uint8_t* zeros) {
+                                  double lattice_alpha, double* row_s, double* row_z,
+                                  float* scales, uint8_t* zeros) {
   int64_t rr = blockIdx.x * (int64_t)(blockDim.x / 32) + threadIdx.x / 32;
   int lane = threadIdx.x & 31;
   if (rr >= k_rows) return;
@@ -208,8 +238,8 @@ __global__ void q_row_grid_kernel(const float* Wf, int64_t n, int64_t k_rows, co
     if (clip == 1) {
       s = (dhi - dlo) / maxq;
       z = rint(-dlo / s);
-    } else if (clip == 2) {  // unconstrained lattice s Z: the min-max step, zero point 0
-      s = (dhi - dlo) / maxq;
+    } else if (clip == 2) {  // unconstrained lattice s Z: the min-max step x alpha, zero point 0
+      s = ((dhi - dlo) / maxq) * lattice_alpha;
       z = 0.0;
     } else {
       const double al = clip == 3 ? alpha_d[row] : (double)alpha[row];
@@ -819,8 +849,8 @@ static gq_status quant_pass(const QuantArgs& a, const QLayout& L, int64_t k_rows
   if (G == 0) {
     unsigned grid = (unsigned)((k_rows + 7) / 8);
     q_row_grid_kernel<<<grid, 256, 0, s>>>(L.Wf, n, k_rows, rowlist, cfg.bits, cfg.clip,
-                                           L.alpha, L.alpha_d, L.row_s, L.row_z, a.scales,
-                                           a.zeros);
+                                           L.alpha, L.alpha_d, a.lattice_alpha, L.row_s, L.row_z,
+                                           a.scales, a.zeros);
     count_launches(1);
     Q_TRY(cudaGetLastError());
   }
@@ -1175,6 +1205,85 @@ gq_status run_ssqr(const QuantArgs& a, const SsqrArgs& o, cudaStream_t s) {
                                              o.capacity, o.col_idx, o.values);
   count_launches(1);
   Q_TRY(cudaGetLastError());
+  return GQ_OK;
+}
+
+// ---------------------------------------------------------------------------------------------
+// HPTQ rate control ("The Geometry of LLM Quantization", section 3, HPTQ: normal and outlier
+// weights share one unconstrained integer lattice, and Huffman coding of the integers gives a
+// variable bit width that meets a compression budget).  Reading: one factor alpha for the whole
+// layer multiplies every row's min-max step; the budget counts the Huffman-coded integers
+// alone, in bits per weight; alpha is the smallest factor (finest lattice) whose coded size is
+// at most budget x m x n bits, found in log2 alpha as the outlier search does: doubling from 1
+// until the layer fits, then a fixed number of bisection steps between the last value that
+// did not fit (or -8 when 1 fits) and the one that does.  The host drives the search (alpha
+// = 2^t computed on the host, the coded size read back after each pass).
+// ---------------------------------------------------------------------------------------------
+gq_status run_hptq(const QuantArgs& a0, const HptqArgs& o, cudaStream_t s) {
+  const int64_t m = a0.m, n = a0.n, count = m * n;
+  HptqLayout H = hptq_layout(a0.ws, m, n);
+  const QLayout& L = H.q;
+  gq_status st = quant_setup(a0, L, s);
+  if (st != GQ_OK) return st;
+  QuantArgs a = a0;
+  a.zeros = H.zeros;
+  const double limit = o.budget * (double)count;
+  long long info[4] = {0, 0, 0, 0};
+  // one pass at alpha = 2^t: the codes, their coded size; false when it exceeds the budget
+  auto fits = [&](double t, bool* ok) -> gq_status {
+    a.lattice_alpha = pow(2.0, t);
+    gq_status e = quant_pass(a, L, m, nullptr, s);
+    if (e != GQ_OK) return e;
+    Q_TRY(launch_huffman_stats(L.codes32, count, H.lengths, H.words, H.info, H.huff_ws, s));
+    Q_TRY(cudaMemcpyAsync(info, H.info, sizeof(info), cudaMemcpyDeviceToHost, s));
+    int hstat = 0, qstat = 0;
+    Q_TRY(cudaMemcpyAsync(&hstat, H.huff_ws, sizeof(int), cudaMemcpyDeviceToHost, s));
+    Q_TRY(cudaMemcpyAsync(&qstat, &L.hdr->status, sizeof(int), cudaMemcpyDeviceToHost, s));
+    Q_TRY(cudaStreamSynchronize(s));
+    if (qstat != 0) return GQ_OK;  // reported through the workspace status; the search stops
+    if (hstat != 0) {              // more distinct integers than the code table holds
+      const int code = hstat;
+      Q_TRY(cudaMemcpyAsync(&L.hdr->status, &code, sizeof(int), cudaMemcpyHostToDevice, s));
+      Q_TRY(cudaStreamSynchronize(s));
+      return GQ_OK;
+    }
+    *ok = (double)info[2] <= limit;
+    return GQ_OK;
+  };
+  auto failed = [&](bool* bad) -> gq_status {
+    int cur = 0;
+    Q_TRY(cudaMemcpyAsync(&cur, &L.hdr->status, sizeof(int), cudaMemcpyDeviceToHost, s));
+    Q_TRY(cudaStreamSynchronize(s));
+    *bad = cur != 0;
+    return GQ_OK;
+  };
+  bool ok = false, bad = false;
+  double hi = 0.0, lo = -8.0;
+  if ((st = fits(hi, &ok)) != GQ_OK) return st;
+  if ((st = failed(&bad)) != GQ_OK || bad) return st;
+  for (int d = 0; d < o.max_doublings && !ok; ++d) {
+    lo = hi;
+    hi += 1.0;
+    if ((st = fits(hi, &ok)) != GQ_OK) return st;
+    if ((st = failed(&bad)) != GQ_OK || bad) return st;
+  }
+  if (!ok) return record_no_fit(L, s);
+  for (int k = 0; k < o.steps; ++k) {
+    const double mid = 0.5 * (lo + hi);
+    bool mok = false;
+    if ((st = fits(mid, &mok)) != GQ_OK) return st;
+    if ((st = failed(&bad)) != GQ_OK || bad) return st;
+    if (mok) hi = mid; else lo = mid;
+  }
+  // the result at the feasible alpha: codes, scales, losses, and its coded size
+  if ((st = fits(hi, &ok)) != GQ_OK) return st;
+  if ((st = failed(&bad)) != GQ_OK || bad) return st;
+  if ((st = quant_finish(a, L, s)) != GQ_OK) return st;
+  const double alpha = a.lattice_alpha;
+  const long long total = info[2];
+  Q_TRY(cudaMemcpyAsync(o.alpha, &alpha, sizeof(double), cudaMemcpyHostToDevice, s));
+  Q_TRY(cudaMemcpyAsync(o.total_bits, &total, sizeof(long long), cudaMemcpyHostToDevice, s));
+  Q_TRY(cudaStreamSynchronize(s));  // the host values above must outlive the copies
   return GQ_OK;
 }
 

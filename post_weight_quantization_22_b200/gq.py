@@ -73,6 +73,11 @@ def _load():
     lib.gq_ssqr_quantize_layer.restype = I
     lib.gq_ssqr_quantize_layer.argtypes = [P, I, I64, I64, P, P, P, I, ctypes.c_double, I, I, P,
                                            P, P, P, P, P, P, I64, P, P, SZ, P]
+    lib.gq_hptq_workspace_size.restype = SZ
+    lib.gq_hptq_workspace_size.argtypes = [I64, I64]
+    lib.gq_hptq_quantize_layer.restype = I
+    lib.gq_hptq_quantize_layer.argtypes = [P, I, I64, I64, P, P, P, I, ctypes.c_double, I, I, P,
+                                           P, P, P, P, P, SZ, P]
     lib.gq_zsic_spacing.restype = I
     lib.gq_zsic_spacing.argtypes = [P, I64, P, P]
     lib.gq_debug_wait_test.restype = I
@@ -89,7 +94,8 @@ EXPORTED = ("gq_version", "gq_status_string", "gq_hessian_accumulate", "gq_hessi
             "gq_workspace_status", "gq_prepare_hinv_static", "gq_prepare_hinv_ordered",
             "gq_quantize_layer_ordered", "gq_zsic_spacing", "gq_huffman_workspace_size",
             "gq_huffman_encode", "gq_debug_wait_test", "gq_kernel_launches",
-            "gq_ssqr_workspace_size", "gq_ssqr_quantize_layer")
+            "gq_ssqr_workspace_size", "gq_ssqr_quantize_layer", "gq_hptq_workspace_size",
+            "gq_hptq_quantize_layer")
 
 
 def _ptr(t):
@@ -332,6 +338,36 @@ def gq_ssqr_quantize_layer(W: torch.Tensor, U: torch.Tensor, dead, delta, bits: 
            "gq_ssqr_quantize_layer")
     return dict(codes=codes, scales=scales, zeros=zeros, alpha=alpha, row_ptr=row_ptr,
                 col_idx=col_idx, values=values, loss=loss, ws=ws)
+
+
+def gq_hptq_quantize_layer(W: torch.Tensor, U: torch.Tensor, dead, delta, bits: int,
+                           budget: float, steps: int = 12, max_doublings: int = 12, ws=None,
+                           stream=None):
+    """HPTQ rate control on the device: one lattice factor for the layer, the smallest whose
+    Huffman-coded integers fit ``budget`` bits per weight.  Returns dict(codes int32 [m, n],
+    scales [m], alpha [1] fp64, total_bits [1] int64, loss, ws)."""
+    m, n = W.shape
+    if not W.is_cuda or not W.is_contiguous():
+        raise ValueError("W must be a contiguous cuda tensor")
+    dev = W.device
+    _need(U, torch.float32, (n, n), "U")
+    if dead is not None:
+        _need(dead, torch.uint8, (n,), "dead")
+    if delta is not None:
+        _need(delta, torch.float64, (1,), "delta")
+    codes = torch.empty((m, n), dtype=torch.int32, device=dev)
+    scales = torch.empty(m, dtype=torch.float32, device=dev)
+    alpha = torch.empty(1, dtype=torch.float64, device=dev)
+    total = torch.empty(1, dtype=torch.int64, device=dev)
+    loss = torch.empty(3, dtype=torch.float64, device=dev)
+    ws = workspace(int(LIB.gq_hptq_workspace_size(m, n)), dev) if ws is None else ws
+    _check(LIB.gq_hptq_quantize_layer(_ptr(W), _dtype_code(W), m, n, _ptr(U), _ptr(dead),
+                                      _ptr(delta), int(bits), float(budget), int(steps),
+                                      int(max_doublings), _ptr(codes), _ptr(scales),
+                                      _ptr(alpha), _ptr(total), _ptr(loss), _ptr(ws),
+                                      ws.numel(), _stream(stream)),
+           "gq_hptq_quantize_layer")
+    return dict(codes=codes, scales=scales, alpha=alpha, total_bits=total, loss=loss, ws=ws)
 
 
 def gq_zsic_spacing(U: torch.Tensor, kappa=None, stream=None) -> torch.Tensor:

@@ -117,3 +117,16 @@ def test_ssqr_entry_rejects_bad_arguments_without_gpu():
         rc = G.LIB.gq_ssqr_quantize_layer(*args, bits, density, 20, 12, None, None, None, None,
                                           None, None, None, 0, None, None, 0, None)
         assert rc == 1, (bits, density, rc)
+
+
+def test_hptq_entry_rejects_bad_arguments_without_gpu():
+    from post_weight_quantization_22_b200 import gq as G
+    assert G.LIB.gq_hptq_workspace_size(0, 16) == 0
+    assert G.LIB.gq_hptq_workspace_size(16, 16) > G.LIB.gq_huffman_workspace_size(256)
+    # budget not positive, bits outside 2..8, steps outside 0..60: rejected before any device work
+    args = [None, 0, 16, 16, None, None, None]
+    for bits, budget, steps in ((3, 0.0, 12), (3, -1.0, 12), (1, 3.0, 12), (9, 3.0, 12),
+                                (3, 3.0, 61)):
+        rc = G.LIB.gq_hptq_quantize_layer(*args, bits, budget, steps, 12, None, None, None,
+                                          None, None, None, 0, None)
+        assert rc == 1, (bits, budget, steps, rc)

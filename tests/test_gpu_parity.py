@@ -705,3 +705,36 @@ def test_min_pivot_order_full_size_sampled_rows():
     o = O.quantize_layer(W, X, bits=4, group=128, rows=rows, H=H, order=perm, tie_tol=TIE_TOL,
                          follow=dict(codes=g["codes"][rows], zeros=g["zeros"][rows]))
     _compare(g, o, W, 4, 128, rows=rows, perm=perm)
+
+
+def test_hptq_rate_control_ragged_against_oracle():
+    """HPTQ rate control at a ragged size (200 x 700, 4-bit min-max base step, budget 3.0
+    bits/weight): the device's factor and coded size against the oracle's search on the
+    device's factor, then the codes at that factor (near-ties followed)."""
+    from post_weight_quantization_22_b200 import gq as G
+    from post_weight_quantization_22_b200.pipeline import LayerQuantizer
+    W, X, spec = synth.workload("q_proj_4096x4096", m=200, n=700, T=900)
+    m, n = W.shape
+    lq = LayerQuantizer(m, n, G.QuantCfg(bits=4), device="cuda")
+    lq.hessian(X.cuda())
+    lq.prepare()
+    budget, steps = 3.0, 8
+    res = G.gq_hptq_quantize_layer(W.cuda(), lq.U, lq.dead, lq.delta, 4, budget, steps=steps)
+    torch.cuda.synchronize()
+    assert G.gq_workspace_status(res["ws"])[0] == 0
+    alpha = float(res["alpha"].item())
+    bits = int(res["total_bits"].item())
+    codes = res["codes"].cpu().numpy().astype(np.int64)
+    U = lq.U.cpu().numpy().astype(np.float64)
+    w0 = O.fix_dead_features(O.hessian(X), W)[1]
+    o_r, o_alpha, o_bits, o_lo = O.hptq_search(w0, U, 4, budget, steps=steps)
+    print(f"alpha gpu {alpha} oracle {o_alpha}; bits gpu {bits} oracle {o_bits}")
+    assert alpha == o_alpha
+    assert bits <= budget * m * n
+    assert abs(bits - o_bits) <= 1e-3 * o_bits
+    f = O.gptq_columns(w0, U, 4, clip="unbounded", alpha=np.full(m, alpha),
+                       follow=dict(codes=codes), tie_tol=TIE_TOL)
+    assert f["disagree"] == 0 and f["followed"] <= FOLLOW_FRAC * codes.size + 2
+    assert np.array_equal(f["codes"], codes)
+    np.testing.assert_allclose(res["scales"].cpu().numpy(), f["scales"][:, 0], rtol=1e-6)
+    assert O.hptq_rate(codes) * codes.size == bits

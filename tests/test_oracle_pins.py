@@ -784,3 +784,61 @@ def test_follow_is_refused_where_it_has_no_meaning():
         O.quantize_layer(W, X, bits=3, reverse=True, follow=f)
     with pytest.raises(ValueError):
         O.quantize_layer(W, X, bits=3, clip=False, follow=f)
+
+
+# ---------------------------------------------------------------------------------------------
+# HPTQ rate control: the coded size of the integers and the search for a budget
+# ---------------------------------------------------------------------------------------------
+
+def test_hptq_rate_hand_values():
+    # two symbols, equal counts: one bit each
+    assert O.hptq_rate([[0, 0, 1, 1]]) == 1.0
+    # counts 5, 2, 1, 1: merges 1+1, 2+2, 4+5 give lengths 1, 2, 3, 3 -> 5 + 4 + 3 + 3 = 15 bits
+    codes = np.array([0] * 5 + [1] * 2 + [2, 3])
+    assert O.hptq_rate(codes) == 15 / 9
+    # only the differences between codes matter
+    assert O.hptq_rate(codes - 7) == 15 / 9
+    # one symbol still costs one bit per weight
+    assert O.hptq_rate(np.zeros(6, dtype=np.int64)) == 1.0
+
+
+def test_hptq_search_hand_trace():
+    """U = I (nothing fed forward), one row [0, 1, 2, 3], 2-bit min-max step s = 1, lattice
+    alpha s Z.  Coded sizes: alpha 1 -> [0,1,2,3], 8 bits; alpha 2 -> [0,0,1,2] (half to even),
+    6 bits; alpha 2^0.5 -> [0,1,1,2], 6 bits; alpha 2^0.25 -> [0,1,2,3], 8 bits.  Budget 1.5
+    bits/weight (6 bits): t = 0 does not fit, t = 1 does; bisection: t = 0.5 fits, t = 0.25
+    does not."""
+    U = np.eye(4)
+    w = np.array([[0.0, 1.0, 2.0, 3.0]])
+    r, alpha, bits, lo = O.hptq_search(w, U, 2, 1.5, steps=2, max_doublings=4)
+    assert alpha == 2.0 ** 0.5 and bits == 6 and lo == 0.25
+    assert r["codes"].tolist() == [[0, 1, 1, 2]]
+    np.testing.assert_allclose(r["scales"][:, 0], [2.0 ** 0.5])
+    # alpha = 1 already fits a 2-bit budget: the bracket starts at t = -8, and t = -4 fits too
+    r, alpha, bits, lo = O.hptq_search(w, U, 2, 2.0, steps=1)
+    assert alpha == 2.0 ** -4 and lo == -8.0
+    assert r["codes"].tolist() == [[0, 16, 32, 48]] and bits == 8
+    # below one bit per weight nothing fits
+    with pytest.raises(ValueError):
+        O.hptq_search(w, U, 2, 0.5, steps=2, max_doublings=3)
+
+
+@pytest.mark.parametrize("budget", [2.5, 3.5])
+def test_hptq_search_brackets_the_budget(budget):
+    """On a random layer the result fits, the last value that did not fit does not, and the
+    bracket has the width the bisection leaves."""
+    rng = np.random.default_rng(3)
+    W = rng.standard_normal((6, 48))
+    X = rng.standard_normal((300, 48))
+    H = O.hessian(X)
+    hd, _ = O.dampen(H, 0.01)
+    U = O.hinv_upper_factor(hd)
+    steps = 6
+    r, alpha, bits, lo = O.hptq_search(W, U, 4, budget, steps=steps)
+    t = np.log2(alpha)
+    assert bits <= budget * W.size
+    assert O.hptq_rate(r["codes"]) * W.size == bits
+    if lo > -8.0:
+        assert t - lo == 2.0 ** -steps
+        r_lo = O.gptq_columns(W, U, 4, clip="unbounded", alpha=np.full(6, 2.0 ** lo))
+        assert O.hptq_rate(r_lo["codes"]) > budget
