@@ -172,47 +172,57 @@ __global__ void __launch_bounds__(256) split_rows_kernel(const double* A, int64_
 }
 
 // Column j of X (kSplitK rows x cols, leading dimension ldx) as an operand row: exponent ex[j]
-// and digit planes D[s][j][k] = digit s of X[k][j] 2^-ex[j].  A CTA takes 32 columns; thread
-// (ty, tx) = (tid / 32, tid % 32) owns rows kPerTy ty .. + kPerTy - 1 of column j0 + tx (reads
-// coalesced along tx): a max pass, then per 8 consecutive rows the digits packed into one 8-byte
-// shared-memory store per plane; the CTA writes the 32 rows of each plane out with coalesced
-// 8-byte stores.  tri: X is a lower triangular block whose diagonal starts at (0, 0); entries
-// with row k < column j count as zero.
-constexpr int kPerTy = kSplitK / 8;
-constexpr int kColPitch = kSplitK + 8;  // bytes per staged row (8-byte stores at distinct banks)
-constexpr size_t kSplitColsSmem = (size_t)kSplitDigits * 32 * kColPitch + 8 * 32 * sizeof(double);
-__global__ void __launch_bounds__(256) split_cols_kernel(const double* X, int64_t ldx, int cols,
-                                                         int64_t plane_rows, int8_t* D, int* ex,
-                                                         int tri) {
+// and digit planes D[s][j][k] = digit s of X[k][j] 2^-ex[j].  A CTA takes 32 columns with 512
+// threads; thread (ty, tx) = (tid / 32, tid % 32) holds rows kPerTy ty .. + kPerTy - 1 of
+// column j0 + tx in registers (read once, coalesced along tx, every load in flight together),
+// the column's maximum comes from a shared-memory reduction over ty, and per 8 consecutive rows
+// the digits are packed into one 8-byte shared-memory store per plane; the CTA writes the 32
+// rows of each plane out with coalesced 8-byte stores.  tri: X is a lower triangular block
+// whose diagonal starts at (0, 0); entries with row k < column j count as zero.
+constexpr int kColTy = 16;                   // threads down one column
+constexpr int kPerTy = kSplitK / kColTy;     // rows per thread
+constexpr int kSplitColsThreads = 32 * kColTy;
+constexpr int kColPitch = kSplitK + 8;  // bytes per staged row (8-byte stores spread over banks)
+constexpr size_t kSplitColsSmem =
+    (size_t)kSplitDigits * 32 * kColPitch + (size_t)kColTy * 32 * sizeof(double);
+__global__ void __launch_bounds__(kSplitColsThreads) split_cols_kernel(const double* X,
+                                                                       int64_t ldx, int cols,
+                                                                       int64_t plane_rows,
+                                                                       int8_t* D, int* ex,
+                                                                       int tri) {
   extern __shared__ __align__(16) uint8_t sc_smem[];
   uint8_t* sD = sc_smem;  // [s][32 columns][kColPitch]
   double* red = reinterpret_cast<double*>(sc_smem + (size_t)kSplitDigits * 32 * kColPitch);
   const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
   const int j0 = blockIdx.x * 32, j = j0 + tx;
   const bool act = j < cols;
-  const double* xcol = X + (int64_t)(kPerTy * ty) * ldx + j;
-  const int kmin = tri ? j : 0;  // rows below kmin of this column count as zero
+  const double* xcol = X + (int64_t)(kPerTy * ty) * ldx + (act ? j : 0);
+  const int kmin = tri ? j : 0;  // rows above kmin of this column count as zero
+  double v[kPerTy];
+#pragma unroll
+  for (int i = 0; i < kPerTy; ++i) {
+    const int k = kPerTy * ty + i;
+    v[i] = (act && k >= kmin) ? xcol[(int64_t)i * ldx] : 0.0;
+  }
   double mx = 0.0;
-  if (act)
-    for (int i = 0; i < kPerTy; ++i)
-      if (kPerTy * ty + i >= kmin) mx = fmax(mx, fabs(xcol[(int64_t)i * ldx]));
+#pragma unroll
+  for (int i = 0; i < kPerTy; ++i) mx = fmax(mx, fabs(v[i]));
   red[ty * 32 + tx] = mx;
   __syncthreads();
   mx = 0.0;
 #pragma unroll
-  for (int y = 0; y < 8; ++y) mx = fmax(mx, red[y * 32 + tx]);
+  for (int y = 0; y < kColTy; ++y) mx = fmax(mx, red[y * 32 + tx]);
   const int e = split_exponent(mx);
   if (ty == 0 && act) ex[j] = e;
   const double sc = pow2(-e);
-#pragma unroll 1
+#pragma unroll
   for (int g8 = 0; g8 < kPerTy / 8; ++g8) {
     uint64_t packed[kSplitDigits];
 #pragma unroll
     for (int s = 0; s < kSplitDigits; ++s) packed[s] = 0;
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-      const int k = kPerTy * ty + 8 * g8 + i;
-      double x = (act && k >= kmin) ? xcol[(int64_t)(8 * g8 + i) * ldx] * sc : 0.0;
+      double x = v[8 * g8 + i] * sc;
 #pragma unroll
       for (int s = 0; s < kSplitDigits; ++s) {
         x *= 128.0;
@@ -230,7 +240,7 @@ __global__ void __launch_bounds__(256) split_cols_kernel(const double* X, int64_
   // plane s, rows j0 .. j0 + 31: kSplitK / 8 words each, written in order by consecutive threads
   constexpr int kWords = kSplitK / 8;
   for (int s = 0; s < kSplitDigits; ++s) {
-    for (int idx = threadIdx.x; idx < 32 * kWords; idx += 256) {
+    for (int idx = threadIdx.x; idx < 32 * kWords; idx += kSplitColsThreads) {
       const int rr = idx / kWords, w = idx % kWords;
       if (j0 + rr < cols)
         *reinterpret_cast<uint64_t*>(D + (int64_t)s * plane_rows * kSplitK +
@@ -477,7 +487,7 @@ cudaError_t launch_split_rows(const double* A, int64_t lda, int rows, SplitOpera
 cudaError_t launch_split_cols(const double* X, int64_t ldx, int cols, SplitOperand op,
                               cudaStream_t s, int tri) {
   if (cols <= 0) return cudaSuccess;
-  split_cols_kernel<<<(unsigned)((cols + 31) / 32), 256, kSplitColsSmem, s>>>(
+  split_cols_kernel<<<(unsigned)((cols + 31) / 32), kSplitColsThreads, kSplitColsSmem, s>>>(
       X, ldx, cols, op.plane_rows, op.digits, op.ex, tri);
   count_launches(1);
   return cudaGetLastError();
