@@ -88,17 +88,39 @@ __global__ void huff_range_kernel(const int* codes, int64_t count, int* state) {
   }
 }
 
-__global__ void huff_hist_kernel(const int* codes, int64_t count, const int* state,
-                                 unsigned long long* hist) {
+constexpr int kHistThreads = 128;
+constexpr int kPrivSym = 64;  // spans up to this many values count in lane-private counters
+static_assert((kHistThreads / 32) * kPrivSym * 32 * 4 <= kHuffMaxSym * 8, "counters fit the bins");
+__global__ void __launch_bounds__(kHistThreads) huff_hist_kernel(const int* codes, int64_t count,
+                                                                 const int* state,
+                                                                 unsigned long long* hist) {
   __shared__ unsigned long long bins[kHuffMaxSym];
   const int lo = state[0];
   const long long K = (long long)state[1] - lo + 1;
   if (K > kHuffMaxSym) return;  // the same for every CTA; the build kernel reports it
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  if (K <= kPrivSym) {
+    // few values (low-bit codes): every lane counts into its own column of its warp's
+    // counters, [warp][symbol][lane] (consecutive lanes in consecutive banks), no atomics
+    unsigned* priv = reinterpret_cast<unsigned*>(bins);
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    for (int i = threadIdx.x; i < (kHistThreads / 32) * kPrivSym * 32; i += blockDim.x) priv[i] = 0u;
+    __syncthreads();
+    unsigned* mine = priv + (size_t)warp * kPrivSym * 32 + lane;
+    for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < count; e += stride)
+      mine[(codes[e] - lo) * 32] += 1u;
+    __syncthreads();
+    if (threadIdx.x < K) {
+      unsigned long long c = 0ull;
+      for (int w = 0; w < kHistThreads / 32; ++w)
+        for (int l = 0; l < 32; ++l) c += priv[((size_t)w * kPrivSym + threadIdx.x) * 32 + l];
+      if (c) atomicAdd(&hist[threadIdx.x], c);
+    }
+    return;
+  }
   for (int i = threadIdx.x; i < K; i += blockDim.x) bins[i] = 0ull;
   __syncthreads();
-  // the lanes of a warp that hold the same symbol add their count with one atomic (low-bit
-  // codes have a handful of distinct values, so per-code atomics would serialise on them)
-  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  // the lanes of a warp that hold the same symbol add their count with one atomic
   const int64_t e_end = (count + stride - 1) / stride * stride;  // every lane runs each round
   for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < e_end; e += stride) {
     const int sym = e < count ? codes[e] - lo : -1;
@@ -140,17 +162,20 @@ __global__ void __launch_bounds__(1024) huff_build_kernel(int* state,
     return;
   }
   __syncthreads();
-  // used symbols as (count << 12 | symbol); unused sort last
-  for (int i = tid; i < kHuffMaxSym; i += blockDim.x) {
+  // used symbols as (count << 12 | symbol); unused sort last.  Only the spanned symbols are
+  // sorted: the next power of two at or above K.
+  int KP = 2;
+  while (KP < K) KP <<= 1;
+  for (int i = tid; i < KP; i += blockDim.x) {
     const unsigned long long c = i < K ? hist[i] : 0ull;
     keys[i] = c ? ((c << 12) | (unsigned long long)i) : ~0ull;
     if (c) atomicAdd(&s_nz, 1);
     lens[i] = 0;
   }
   __syncthreads();
-  for (int k = 2; k <= kHuffMaxSym; k <<= 1) {
+  for (int k = 2; k <= KP; k <<= 1) {
     for (int j = k >> 1; j > 0; j >>= 1) {
-      for (int i = tid; i < kHuffMaxSym; i += blockDim.x) {
+      for (int i = tid; i < KP; i += blockDim.x) {
         const int ixj = i ^ j;
         if (ixj > i) {
           const unsigned long long a = keys[i], b = keys[ixj];
@@ -196,8 +221,8 @@ __global__ void __launch_bounds__(1024) huff_build_kernel(int* state,
       code = (code + (unsigned long long)bl_count[ln - 1]) << 1;
       next_code[ln] = code;
     }
-    for (int sym = 0; sym < kHuffMaxSym; ++sym) {
-      const int ln = sym < K ? lens[sym] : 0;
+    for (int sym = 0; sym < K; ++sym) {
+      const int ln = lens[sym];
       keys[sym] = ln ? next_code[ln]++ : 0ull;
     }
     s_maxlen = maxlen;
@@ -214,8 +239,8 @@ __global__ void __launch_bounds__(1024) huff_build_kernel(int* state,
     state[2] = (s_bad || !fits) ? 1 : 0;
     info[0] = lo; info[1] = K; info[2] = (long long)total; info[3] = s_maxlen;
   }
-  for (int i = tid; i < kHuffMaxSym; i += blockDim.x) {
-    lengths_out[i] = i < K ? lens[i] : 0;
+  for (int i = tid; i < K; i += blockDim.x) {
+    lengths_out[i] = lens[i];
     words_out[i] = keys[i];
   }
 }
@@ -254,9 +279,10 @@ __global__ void __launch_bounds__(kHuffThreads) huff_tile_sum_kernel(const int* 
   __shared__ uint8_t sl[kHuffMaxSym];
   __shared__ unsigned long long red[kHuffThreads / 32];
   if (state[2]) return;
-  for (int i = threadIdx.x; i < kHuffMaxSym; i += blockDim.x) sl[i] = lengths[i];
-  __syncthreads();
   const int lo = state[0];
+  const int K = state[1] - lo + 1;  // <= kHuffMaxSym once the build has passed
+  for (int i = threadIdx.x; i < K; i += blockDim.x) sl[i] = lengths[i];
+  __syncthreads();
   const int64_t t0 = (int64_t)blockIdx.x * kHuffTile;
   unsigned long long acc = 0ull;
   for (int i = threadIdx.x; i < kHuffTile; i += blockDim.x) {
@@ -299,12 +325,13 @@ __global__ void __launch_bounds__(kHuffThreads) huff_encode_kernel(
   __shared__ unsigned long long sw[kHuffMaxSym];
   __shared__ unsigned long long wsum[kHuffThreads / 32];
   if (state[2]) return;
-  for (int i = threadIdx.x; i < kHuffMaxSym; i += blockDim.x) {
+  const int lo = state[0];
+  const int K = state[1] - lo + 1;  // <= kHuffMaxSym once the build has passed
+  for (int i = threadIdx.x; i < K; i += blockDim.x) {
     sl[i] = lengths[i];
     sw[i] = words[i];
   }
   __syncthreads();
-  const int lo = state[0];
   const int64_t e0 = (int64_t)blockIdx.x * kHuffTile + (int64_t)threadIdx.x * kHuffPer;
   int sym[kHuffPer];
   unsigned long long mine = 0ull;
@@ -369,8 +396,10 @@ cudaError_t launch_huffman(const int* codes, int64_t count, unsigned long long* 
   if ((e = cudaMemsetAsync(L.hdr, 0, sizeof(WsHeader), s))) return e;
   huff_init_kernel<<<1, 1024, 0, s>>>(L.state, L.hist);
   const unsigned grid = (unsigned)std::min<int64_t>((count + 255) / 256, 148 * 8);
+  const unsigned hgrid = (unsigned)std::min<int64_t>((count + kHistThreads - 1) / kHistThreads,
+                                                     148 * 16);
   huff_range_kernel<<<grid, 256, 0, s>>>(codes, count, L.state);
-  huff_hist_kernel<<<grid, 256, 0, s>>>(codes, count, L.state, L.hist);
+  huff_hist_kernel<<<hgrid, kHistThreads, 0, s>>>(codes, count, L.state, L.hist);
   huff_build_kernel<<<1, 1024, kHuffBuildSmem, s>>>(L.state, L.hist, nwords, lengths, words,
                                                     info, L.hdr);
   huff_tile_sum_kernel<<<(unsigned)ntiles, kHuffThreads, 0, s>>>(codes, count, L.state, lengths,
@@ -394,8 +423,10 @@ cudaError_t launch_huffman_stats(const int* codes, int64_t count, uint8_t* lengt
   if ((e = cudaMemsetAsync(L.hdr, 0, sizeof(WsHeader), s))) return e;
   huff_init_kernel<<<1, 1024, 0, s>>>(L.state, L.hist);
   const unsigned grid = (unsigned)std::min<int64_t>((count + 255) / 256, 148 * 8);
+  const unsigned hgrid = (unsigned)std::min<int64_t>((count + kHistThreads - 1) / kHistThreads,
+                                                     148 * 16);
   huff_range_kernel<<<grid, 256, 0, s>>>(codes, count, L.state);
-  huff_hist_kernel<<<grid, 256, 0, s>>>(codes, count, L.state, L.hist);
+  huff_hist_kernel<<<hgrid, kHistThreads, 0, s>>>(codes, count, L.state, L.hist);
   // a stream capacity no total reaches (2^63 bits): only the code's own limits are reported
   huff_build_kernel<<<1, 1024, kHuffBuildSmem, s>>>(L.state, L.hist, (int64_t)1 << 57, lengths,
                                                     words, info, L.hdr);

@@ -50,7 +50,8 @@ constexpr uint32_t kSEpiBytes = 8 * 32 * kSEpiPitch;  // eight epilogue warps x 
 constexpr size_t kSSmem = kSStages * kSStage + 1024 + 256 + kSEpiBytes;
 constexpr int kSEpiWarps = 8;        // two per TMEM lane quadrant, 32 columns each
 constexpr int kSThreads = 32 * (2 + kSEpiWarps);  // warp 0 producer, warp 1 MMA, then epilogue
-constexpr int kSTilesPerCta = 4;     // CTAs retire regularly, so other streams' kernels get SMs
+constexpr int kSTilesPerCta = 4;     // tiles per CTA aimed at (CTAs retire regularly, so other
+                                     // streams' kernels get SMs)
 constexpr uint32_t kSTmemCols = 512; // kSplitDigits x 64 columns, rounded up to a power of two
 static_assert(kSplitDigits * kSBN <= (int)kSTmemCols, "class accumulators must fit in TMEM");
 static_assert(kSplitDigits % 2 == 0, "the epilogue reads the classes two at a time");
@@ -71,6 +72,7 @@ struct SplitArgs {
   double alpha;
   int lower;         // only entries with column <= row
   int tiles, ntn;    // tiles enumerated, column tiles
+  int ctas;          // CTAs of the launch; CTA c runs tiles [c tiles / ctas, (c + 1) tiles / ctas)
   WsHeader* hdr;
 };
 
@@ -268,8 +270,8 @@ __global__ void __launch_bounds__(kSThreads, 1)
   __shared__ int s_issued;
   __shared__ __align__(16) double s_colscale[kSEpiWarps][32];  // per epilogue warp: 2^eb of its columns
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int t_begin = blockIdx.x * kSTilesPerCta;
-  const int t_end = min(t_begin + kSTilesPerCta, g.tiles);
+  const int t_begin = (int)((int64_t)blockIdx.x * g.tiles / g.ctas);
+  const int t_end = (int)((int64_t)(blockIdx.x + 1) * g.tiles / g.ctas);
   if (tid == 0) {
     for (int s = 0; s < kSStages; ++s) {
       tc::mbar_init(&full[s], 1);
@@ -520,8 +522,16 @@ cudaError_t launch_split_gemm(double* C, int64_t ldc, int M, int N, const SplitO
   } else {
     g.tiles = mt * g.ntn;
   }
-  const unsigned ctas = (unsigned)((g.tiles + kSTilesPerCta - 1) / kSTilesPerCta);
-  split_gemm_kernel<<<ctas, kSThreads, kSSmem, s>>>(ma, mb, g);
+  // whole waves over the SMs (the nearest count of waves of kSTilesPerCta tiles, at least one),
+  // the tiles split evenly: no short last wave, and a small product spreads over every SM
+  int dev = 0, sms = 148;
+  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+  if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+    return e;
+  const int per_wave = sms * kSTilesPerCta;
+  const int waves = std::max(1, (g.tiles + per_wave / 2) / per_wave);
+  g.ctas = std::min(g.tiles, sms * waves);
+  split_gemm_kernel<<<(unsigned)g.ctas, kSThreads, kSSmem, s>>>(ma, mb, g);
   count_launches(1);
   return cudaGetLastError();
 }
