@@ -25,7 +25,9 @@ namespace gq {
 constexpr int kNB = 64;      // Cholesky panel width (the leaf)
 constexpr int kSuper = 256;  // super-panel width (trailing-update depth) of the fp64 path
 constexpr int kPnPitch = 68;  // shared-memory pitch (doubles) of the panel kernel's tiles
-constexpr size_t kPnSmem = (size_t)(kNB + 32) * kPnPitch * sizeof(double);
+// the leaf's L11^-1 (64 rows), a chunk of the panel (32), the previous panel's rows of the
+// diagonal block (64) and of the chunk (32)
+constexpr size_t kPnSmem = (size_t)(2 * kNB + 64) * kPnPitch * sizeof(double);
 
 // ---------------------------------------------------------------------------------------
 // dead fix + damping statistics (one CTA)
@@ -300,11 +302,18 @@ __device__ __forceinline__ double recip_newton(double p) {
 // one FMA and a store.  A row block whose rows are all eliminated leaves with arrive_drop.
 // The pivot loop is unrolled 4 deep (register indices fixed, the body small enough to stay in
 // the instruction cache).  Waits are bounded: a timeout is recorded and the kernel finishes.
+// Look-ahead inside a super-panel (cp >= 0, the previous panel's first column): the previous
+// panel's update of this panel's columns is applied here, not by a separate product, so the
+// chain runs one kernel per panel.  Every CTA subtracts Lp Lp^T from its copy of the diagonal
+// block (Lp = L[c0 .. c0 + 63][cp .. cp + 63], fp64 MMAs into shared memory) and, for each of
+// its chunks, Lr Lp^T from the chunk before the solve (Lr = the chunk's rows of L in the
+// previous panel's columns).  The later columns of the super-panel take the previous panel's
+// update on another stream, overlapped with this kernel.
 // ---------------------------------------------------------------------------------------
 __global__ void __launch_bounds__(256, 1) potrf_panel_kernel(double* M, int64_t ldm, int64_t n,
-                                                             int64_t c0, int w, double* Dinv,
-                                                             WsHeader* hdr, uint32_t polls,
-                                                             int withhold) {
+                                                             int64_t c0, int w, int64_t cp,
+                                                             double* Dinv, WsHeader* hdr,
+                                                             uint32_t polls, int withhold) {
   extern __shared__ __align__(16) double pn_smem[];
   __shared__ __align__(16) double colbuf[2][kNB];
   __shared__ __align__(16) double rowbuf[2][kNB];
@@ -327,6 +336,46 @@ __global__ void __launch_bounds__(256, 1) potrf_panel_kernel(double* M, int64_t 
       sv[i][j] = v;
       av[i][j] = (q == r) ? 1.0 : 0.0;
     }
+  const int warp = tid >> 5, lane = tid & 31, g = lane >> 2, t = lane & 3;
+  double* sQ = pn_smem + (kNB + 32) * kPnPitch;   // 64 x kPnPitch: Lp
+  double* sR = pn_smem + (2 * kNB + 32) * kPnPitch;  // 32 x kPnPitch: a chunk's Lr
+  if (cp >= 0) {  // diagonal block -= Lp Lp^T
+    double* sG = pn_smem;  // 64 x kPnPitch, free until the leaf's result is written
+    for (int e = tid; e < kNB * 32; e += 256) {
+      const int rr = e >> 5, cc2 = (e & 31) * 2;
+      double2 v = make_double2(0.0, 0.0);
+      if (rr < w) v = *reinterpret_cast<const double2*>(M + (c0 + rr) * ldm + cp + cc2);
+      *reinterpret_cast<double2*>(sQ + rr * kPnPitch + cc2) = v;
+    }
+    __syncthreads();
+    const int gm = warp & 3, gn = warp >> 2;  // rows 16 gm .., columns 32 gn ..
+    double acc[4][4] = {};
+#pragma unroll
+    for (int kb = 0; kb < kNB; kb += 8) {
+      const double* pa = sQ + (gm * 16 + g) * kPnPitch + kb + t;
+      const double af[4] = {pa[0], pa[8 * kPnPitch], pa[4], pa[8 * kPnPitch + 4]};
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const double* pb = sQ + (gn * 32 + u * 8 + g) * kPnPitch + kb + t;
+        const double bf[2] = {pb[0], pb[4]};
+        tc::dmma_m16n8k8(acc[u], af, bf);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+#pragma unroll
+      for (int h = 0; h < 2; ++h)
+        *reinterpret_cast<double2*>(sG + (gm * 16 + g + 8 * h) * kPnPitch + gn * 32 + u * 8 +
+                                    2 * t) = make_double2(acc[u][2 * h], acc[u][2 * h + 1]);
+    __syncthreads();
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int r = 4 * a + i, q = 4 * b + j;
+        if (r < w && q <= r) sv[i][j] -= sG[r * kPnPitch + q];
+      }
+  }
   if (tid == 0) tc::mbar_init(&bar, 256);
   __syncthreads();
   // pivot 0's column and row, then phase 0
@@ -434,7 +483,6 @@ __global__ void __launch_bounds__(256, 1) potrf_panel_kernel(double* M, int64_t 
   // fp64 MMAs; the padded pitch makes the fragment loads conflict-free.
   const int64_t rem = n - c0 - w;
   if (rem <= 0) return;
-  const int warp = tid >> 5, lane = tid & 31, g = lane >> 2, t = lane & 3;
   const int mi = warp & 1, np = warp >> 1;
   const int64_t nch = (rem + 31) / 32;
   for (int64_t ch = blockIdx.x; ch < nch; ch += gridDim.x) {
@@ -442,11 +490,38 @@ __global__ void __launch_bounds__(256, 1) potrf_panel_kernel(double* M, int64_t 
     __syncthreads();  // sL written / the previous chunk consumed
     for (int e = tid; e < 32 * 32; e += 256) {
       const int rr = e >> 5, cc2 = (e & 31) * 2;
-      double2 v = make_double2(0.0, 0.0);
-      if (r0 + rr < n) v = *reinterpret_cast<const double2*>(M + (r0 + rr) * ldm + c0 + cc2);
+      double2 v = make_double2(0.0, 0.0), vr = make_double2(0.0, 0.0);
+      if (r0 + rr < n) {
+        v = *reinterpret_cast<const double2*>(M + (r0 + rr) * ldm + c0 + cc2);
+        if (cp >= 0) vr = *reinterpret_cast<const double2*>(M + (r0 + rr) * ldm + cp + cc2);
+      }
       *reinterpret_cast<double2*>(sP + rr * kPnPitch + cc2) = v;
+      if (cp >= 0) *reinterpret_cast<double2*>(sR + rr * kPnPitch + cc2) = vr;
     }
     __syncthreads();
+    if (cp >= 0) {  // chunk -= Lr Lp^T (each entry of the chunk owned by one thread)
+      double up[2][4] = {{0.0, 0.0, 0.0, 0.0}, {0.0, 0.0, 0.0, 0.0}};
+#pragma unroll
+      for (int kb = 0; kb < kNB; kb += 8) {
+        const double* pa = sR + (mi * 16 + g) * kPnPitch + kb + t;
+        const double af[4] = {pa[0], pa[8 * kPnPitch], pa[4], pa[8 * kPnPitch + 4]};
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          const double* pb = sQ + ((2 * np + u) * 8 + g) * kPnPitch + kb + t;
+          const double bf[2] = {pb[0], pb[4]};
+          tc::dmma_m16n8k8(up[u], af, bf);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < 2; ++u)
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          double* pp = sP + (mi * 16 + g + 8 * h) * kPnPitch + (2 * np + u) * 8 + 2 * t;
+          pp[0] -= up[u][2 * h];
+          pp[1] -= up[u][2 * h + 1];
+        }
+      __syncthreads();
+    }
     double acc[2][4] = {{0.0, 0.0, 0.0, 0.0}, {0.0, 0.0, 0.0, 0.0}};
 #pragma unroll
     for (int kb = 0; kb < kNB; kb += 8) {
@@ -672,8 +747,9 @@ static cudaError_t invert_diag_block(double* M, int64_t n, int64_t ldm, int64_t 
 // One set per host thread and device, created on first use and kept.
 struct PrepStreams {
   bool ready = false;
-  cudaStream_t a = nullptr, b = nullptr, c = nullptr;
-  cudaEvent_t fork = nullptr, panel[2] = {}, far[2] = {}, join[3] = {};
+  cudaStream_t a = nullptr, b = nullptr, c = nullptr, d = nullptr;
+  cudaEvent_t fork = nullptr, panel[2] = {}, far[2] = {}, join[4] = {}, pk = nullptr,
+              upd[2] = {};
 };
 thread_local PrepStreams t_prep_streams[128];
 
@@ -688,8 +764,10 @@ static cudaError_t prep_streams(PrepStreams** out) {
     GQ_TRY(cudaStreamCreateWithPriority(&p.a, cudaStreamNonBlocking, greatest));
     GQ_TRY(cudaStreamCreateWithPriority(&p.b, cudaStreamNonBlocking, (least + greatest) / 2));
     GQ_TRY(cudaStreamCreateWithPriority(&p.c, cudaStreamNonBlocking, least));
+    GQ_TRY(cudaStreamCreateWithPriority(&p.d, cudaStreamNonBlocking, greatest));
     cudaEvent_t* evs[] = {&p.fork, &p.panel[0], &p.panel[1], &p.far[0], &p.far[1],
-                          &p.join[0], &p.join[1], &p.join[2]};
+                          &p.join[0], &p.join[1], &p.join[2], &p.join[3], &p.pk,
+                          &p.upd[0], &p.upd[1]};
     for (cudaEvent_t* e : evs) GQ_TRY(cudaEventCreateWithFlags(e, cudaEventDisableTiming));
     p.ready = true;
   }
@@ -707,11 +785,12 @@ cudaError_t launch_prepare(const double* H, int64_t n, double damp, int order, i
   PrepStreams* ps = nullptr;
   GQ_TRY(prep_streams(&ps));
   const WaitTest wt = wait_test();
-  cudaStream_t s = ps->a, sb = ps->b, sc = ps->c;
+  cudaStream_t s = ps->a, sb = ps->b, sc = ps->c, sd = ps->d;
   GQ_TRY(cudaEventRecord(ps->fork, s0));
   GQ_TRY(cudaStreamWaitEvent(s, ps->fork, 0));
   GQ_TRY(cudaStreamWaitEvent(sb, ps->fork, 0));
   GQ_TRY(cudaStreamWaitEvent(sc, ps->fork, 0));
+  GQ_TRY(cudaStreamWaitEvent(sd, ps->fork, 0));
   GQ_TRY(cudaMemsetAsync(L.hdr, 0, sizeof(WsHeader), s));
   diag_stats_kernel<<<1, 1024, 0, s>>>(H, n, damp, dead, delta, L.hdr);
   count_launches(1);
@@ -866,23 +945,32 @@ cudaError_t launch_prepare(const double* H, int64_t n, double damp, int order, i
     const int64_t sp0 = (c0 / sup) * sup;                       // super-panel start
     const int64_t sp1 = std::min<int64_t>(sp0 + sup, n);        // super-panel end
     const int64_t rem = n - c0 - w;
+    // Look-ahead inside the super-panel: the panel kernel applies the previous panel's update
+    // to its own columns; the previous panel's update of the columns two panels on and later
+    // runs on stream D beside it, and this panel waits for the one two panels back.
+    const int64_t cp = c0 > sp0 ? c0 - kNB : -1;
+    if (c0 - sp0 >= 2 * kNB) GQ_TRY(cudaStreamWaitEvent(s, ps->upd[(k - 2) & 1], 0));
     {  // leaf (every CTA) + P <- P L11^-T for the rows below, one wave of CTAs
       const int64_t nch = rem > 0 ? (rem + 31) / 32 : 1;
       const int grid = (int)std::min<int64_t>(nch, sms);
-      potrf_panel_kernel<<<grid, 256, kPnSmem, s>>>(L.M, ldm, n, c0, w,
+      potrf_panel_kernel<<<grid, 256, kPnSmem, s>>>(L.M, ldm, n, c0, w, cp,
                                                     L.Dinv + (c0 / kNB) * kNB * kNB, L.hdr,
                                                     wt.polls, wt.withhold);
       count_launches(1);
       GQ_TRY(cudaGetLastError());
     }
-    const int64_t inw = sp1 - (c0 + w);  // columns of the super-panel after this panel
-    if (rem > 0 && inw > 0) {  // A[:, c0+w : sp1] -= L21 L21[c0+w : sp1]^T for every row below
+    const int64_t c2 = c0 + 2 * kNB;  // first column this panel updates on stream D
+    if (rem > 0 && c2 < sp1) {  // A[c2:, c2 : sp1] -= L21[c2:] L21[c2 : sp1]^T (stream D)
+      GQ_TRY(cudaEventRecord(ps->pk, s));
+      GQ_TRY(cudaStreamWaitEvent(sd, ps->pk, 0));
       DgemmCall g{};
-      g.M = (int)rem; g.N = (int)inw; g.K = w; g.batch = 1; g.alpha = -1.0; g.beta_one = 1;
-      g.A = Mop(c0 + w, c0);
-      g.B = Mop(c0 + w, c0); g.b_nmajor = 0;
-      g.C = L.M + (c0 + w) * ldm + (c0 + w); g.ldc = ldm; g.lower_tiles = 1; g.hdr = L.hdr;
-      GQ_TRY(launch_dgemm(g, s));
+      g.M = (int)(n - c2); g.N = (int)(sp1 - c2); g.K = w; g.batch = 1; g.alpha = -1.0;
+      g.beta_one = 1;
+      g.A = Mop(c2, c0);
+      g.B = Mop(c2, c0); g.b_nmajor = 0;
+      g.C = L.M + c2 * ldm + c2; g.ldc = ldm; g.lower_tiles = 1; g.hdr = L.hdr;
+      GQ_TRY(launch_dgemm(g, sd));
+      GQ_TRY(cudaEventRecord(ps->upd[k & 1], sd));
     }
     if (c0 + w != sp1) continue;
     // super-panel [sp0, sp1) factored; on the split path its columns of L below it become
@@ -933,8 +1021,10 @@ cudaError_t launch_prepare(const double* H, int64_t n, double damp, int order, i
   }
   GQ_TRY(cudaEventRecord(ps->join[1], sb));
   GQ_TRY(cudaEventRecord(ps->join[2], sc));
+  GQ_TRY(cudaEventRecord(ps->join[3], sd));
   GQ_TRY(cudaStreamWaitEvent(s, ps->join[1], 0));
   GQ_TRY(cudaStreamWaitEvent(s, ps->join[2], 0));
+  GQ_TRY(cudaStreamWaitEvent(s, ps->join[3], 0));
   {
     dim3 grid((unsigned)((n + 255) / 256), (unsigned)n);
     flip_to_u_kernel<<<grid, 256, 0, s>>>(L.M, n, ldm, U);

@@ -171,6 +171,13 @@ __global__ void __launch_bounds__(kLThreads, kDeep ? 1 : 2)
     } else {  // the accumulators added in fp64, one fp32 rounding into the work matrix
 #pragma unroll
       for (int cc = 0; cc < 2; ++cc) {
+        // this chunk of the work matrix is loaded first, so the loads overlap the reads of the
+        // accumulators and their fp64 sum
+        float4 wc[8];
+        if (full_row) {
+#pragma unroll
+          for (int i = 0; i < 8; ++i) wc[i] = *reinterpret_cast<const float4*>(wrow + cc * 32 + 4 * i);
+        }
         double u[32];
 #pragma unroll
         for (int i = 0; i < 32; ++i) u[i] = 0.0;
@@ -184,7 +191,7 @@ __global__ void __launch_bounds__(kLThreads, kDeep ? 1 : 2)
         if (full_row) {
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
-            const float4 w0 = *reinterpret_cast<const float4*>(wrow + cc * 32 + 4 * i);
+            const float4 w0 = wc[i];
             float4 w;
             w.x = (float)((double)w0.x - u[4 * i]);
             w.y = (float)((double)w0.y - u[4 * i + 1]);
