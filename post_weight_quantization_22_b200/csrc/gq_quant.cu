@@ -375,8 +375,8 @@ struct ColArgs {
 // lane t are taken as columns 2t and 2t + 1).  This is GPTQ's lazy batch applied again inside
 // the block; the group grid, taken at a group's first column, sees the same error-fed values
 // as the column-by-column recursion.  The register array is rotated by one tile after each
-// tile, and the tile loop is unrolled in full: the rotation then costs no moves (the copies
-// fold into register renaming), and every tile issues only the MMAs of the tiles after it.
+// tile so that the body, compiled once, refers to fixed registers (a fully unrolled tile loop
+// measured 73 us per block against 33: the code no longer fits the instruction cache).
 //
 // The recursion runs in fp64: the in-block feedback sums cancel strongly when the grid is
 // coarse, and an fp32 recursion flips ~1-3 % of the codes on ill-conditioned layers (measured
@@ -452,7 +452,7 @@ __global__ void __launch_bounds__(kColThreads, 1) colloop_kernel(ColArgs a) {
   const bool outl = a.clip == 3;
   int nout = 0;
 
-#pragma unroll
+#pragma unroll 1
   for (int T = 0; T < kTiles; ++T) {
     if (8 * T >= bw) break;
     if constexpr (G > 0) {
