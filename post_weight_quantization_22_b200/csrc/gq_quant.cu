@@ -383,9 +383,12 @@ struct ColArgs {
 // against the fp64 oracle), while fp64 here with fp32 storage of W, E and U between blocks
 // reproduces the oracle's codes.
 // Z: ZSIC spacing (per-row grid only): column j's step is the row step times kappa_j.
-template <int G, bool Z = false>
+// CM: the grid's clip mode (a compile-time copy of the call's clip: 0 clip-free with the
+// ladder's overflow flags, 1 clamped, 2 unconstrained lattice with int32 codes, 3 outliers).
+template <int G, bool Z, int CM>
 __global__ void __launch_bounds__(kColThreads, 1) colloop_kernel(ColArgs a) {
   static_assert(!Z || G == 0, "per-column spacing takes a per-row grid");
+  static_assert(G == 0 || CM == 1, "group grids are clamped");
   constexpr uint32_t kCopy = Z ? kUBlkBytesZ : kUBlkBytes;
   extern __shared__ __align__(16) double q_smem[];
   const float* Ut = reinterpret_cast<const float*>(q_smem);
@@ -444,12 +447,12 @@ __global__ void __launch_bounds__(kColThreads, 1) colloop_kernel(ColArgs a) {
   if (G == 0 && act) { s = a.row_s[row]; z = a.row_z[row]; inv_s = 1.0 / s; }
   double e2 = 0.0, bnd = 0.0;
   int ovf = 0;
-  const bool clip = a.clip == 1;      // clamp to [0, 2^b - 1]
-  const bool track = a.clip == 0;     // clip-free: flag codes outside the range for the ladder
+  constexpr bool clip = CM == 1;      // clamp to [0, 2^b - 1]
+  constexpr bool track = CM == 0;     // clip-free: flag codes outside the range for the ladder
   // outliers ("The Geometry of LLM Quantization", section 3, SSQR): an entry whose code leaves
   // [0, 2^b - 1] keeps its current (error-fed) value in full precision: error 0, nothing fed
   // forward, code 0 in the packed stream
-  const bool outl = a.clip == 3;
+  constexpr bool outl = CM == 3;
   int nout = 0;
 
 #pragma unroll 1
@@ -530,7 +533,7 @@ __global__ void __launch_bounds__(kColThreads, 1) colloop_kernel(ColArgs a) {
         lo2.x = f0 - hi2.x; lo2.y = f1 - hi2.y;
         *reinterpret_cast<float2*>(a.Ehi + rr * a.ldE + j0 + col) = hi2;
         *reinterpret_cast<float2*>(a.Elo + rr * a.ldE + j0 + col) = lo2;
-        if (a.codes32) {  // unconstrained lattice: z = 0, any integer
+        if constexpr (CM == 2) {  // unconstrained lattice: z = 0, any integer
           int* cp = a.codes32 + row * n + j0 + col;
           cp[0] = (int)ca[0];
           if (col + 1 < bw) cp[1] = (int)ca[1];
@@ -711,34 +714,56 @@ constexpr size_t kColSmemZ = (size_t)kUBlkBytesZ + 16;
 cudaError_t quant_init_attributes() {
   const int smem = (int)kColSmem;
   cudaError_t e;
-  if ((e = cudaFuncSetAttribute(colloop_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem))) return e;
-  if ((e = cudaFuncSetAttribute(colloop_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem))) return e;
-  if ((e = cudaFuncSetAttribute(colloop_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem))) return e;
-  if ((e = cudaFuncSetAttribute(colloop_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem))) return e;
-  if ((e = cudaFuncSetAttribute(colloop_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem))) return e;
-  if ((e = cudaFuncSetAttribute(colloop_kernel<0, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kColSmemZ))) return e;
+  if ((e = cudaFuncSetAttribute(colloop_kernel<0, false, 0>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem))) return e;
+  if ((e = cudaFuncSetAttribute(colloop_kernel<0, false, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem))) return e;
+  if ((e = cudaFuncSetAttribute(colloop_kernel<0, false, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem))) return e;
+  if ((e = cudaFuncSetAttribute(colloop_kernel<0, false, 3>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem))) return e;
+  if ((e = cudaFuncSetAttribute(colloop_kernel<16, false, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem))) return e;
+  if ((e = cudaFuncSetAttribute(colloop_kernel<32, false, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem))) return e;
+  if ((e = cudaFuncSetAttribute(colloop_kernel<64, false, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem))) return e;
+  if ((e = cudaFuncSetAttribute(colloop_kernel<128, false, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem))) return e;
+  if ((e = cudaFuncSetAttribute(colloop_kernel<0, true, 0>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kColSmemZ))) return e;
+  if ((e = cudaFuncSetAttribute(colloop_kernel<0, true, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kColSmemZ))) return e;
+  if ((e = cudaFuncSetAttribute(colloop_kernel<0, true, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kColSmemZ))) return e;
   const int row_smem = 32768 * (int)sizeof(float);  // a staged row of the widest layer
   if ((e = cudaFuncSetAttribute(q_load_perm_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, row_smem))) return e;
   return cudaFuncSetAttribute(q_load_perm_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, row_smem);
 }
 
-template <int G, bool Z = false>
+template <int G, bool Z, int CM>
 static cudaError_t launch_colloop(const ColArgs& ca, cudaStream_t s) {
   const size_t smem = Z ? kColSmemZ : kColSmem;
   unsigned grid = (unsigned)((ca.k_rows + kRowsPerCta - 1) / kRowsPerCta);
-  colloop_kernel<G, Z><<<grid, kColThreads, smem, s>>>(ca);
+  colloop_kernel<G, Z, CM><<<grid, kColThreads, smem, s>>>(ca);
   count_launches(1);
   return cudaGetLastError();
 }
 
 static cudaError_t colloop_dispatch(int group, int spacing, const ColArgs& ca, cudaStream_t s) {
-  if (spacing) return group == 0 ? launch_colloop<0, true>(ca, s) : cudaErrorInvalidValue;
+  if (spacing) {
+    if (group != 0) return cudaErrorInvalidValue;
+    switch (ca.clip) {
+      case 0: return launch_colloop<0, true, 0>(ca, s);
+      case 1: return launch_colloop<0, true, 1>(ca, s);
+      case 2: return launch_colloop<0, true, 2>(ca, s);
+      default: return cudaErrorInvalidValue;
+    }
+  }
+  if (group == 0) {
+    switch (ca.clip) {
+      case 0: return launch_colloop<0, false, 0>(ca, s);
+      case 1: return launch_colloop<0, false, 1>(ca, s);
+      case 2: return launch_colloop<0, false, 2>(ca, s);
+      case 3: return launch_colloop<0, false, 3>(ca, s);
+      default: return cudaErrorInvalidValue;
+    }
+  }
+  if (ca.clip != 1) return cudaErrorInvalidValue;
   switch (group) {
-    case 0: return launch_colloop<0>(ca, s);
-    case 16: return launch_colloop<16>(ca, s);
-    case 32: return launch_colloop<32>(ca, s);
-    case 64: return launch_colloop<64>(ca, s);
-    case 128: return launch_colloop<128>(ca, s);
+    case 16: return launch_colloop<16, false, 1>(ca, s);
+    case 32: return launch_colloop<32, false, 1>(ca, s);
+    case 64: return launch_colloop<64, false, 1>(ca, s);
+    case 128: return launch_colloop<128, false, 1>(ca, s);
     default: return cudaErrorInvalidValue;
   }
 }

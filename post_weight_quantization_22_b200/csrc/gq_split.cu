@@ -24,8 +24,9 @@
 // Kernels: split_rows_kernel (digits of row-major rows, K contiguous: the panel's rows of L),
 // split_cols_kernel (digits of the columns of a row-major block, transposed through shared
 // memory: a block row of the inverse), and split_gemm_kernel (tcgen05 kind::i8, 128 x 64 tiles,
-// TMA-fed 4-stage ring of 36 KB stages (one 32-deep k-step each, 32-byte rows with the 32-byte
-// swizzle: three stages' loads in flight while one is multiplied), warp-specialised: a producer warp, an MMA warp and
+// TMA-fed 2-stage ring of 72 KB stages (two 32-deep k-steps each, 64-byte swizzled rows; a
+// 4-stage ring of 36 KB one-k-step stages with the 32-byte swizzle measured 12 % slower),
+// warp-specialised: a producer warp, an MMA warp and
 // eight epilogue warps; a CTA runs a few tiles and hands the accumulator back to the MMA warp
 // as soon as the epilogue has read it, so the update of C overlaps the next tile's products).
 // For one A digit the products with consecutive B digits are one instruction of N up to 256
@@ -40,11 +41,11 @@ namespace gq {
 
 namespace {
 constexpr int kSBM = 128, kSBN = 64;  // output tile
-constexpr int kSBK = 32;              // K bytes per stage (one MMA k-step; 32-byte rows)
-constexpr int kSStages = 4;
-constexpr uint32_t kSATile = kSBM * kSBK;                  // 4 KB per digit plane
-constexpr uint32_t kSBTile = kSBN * kSBK;                  // 2 KB per digit plane
-constexpr uint32_t kSStage = kSplitDigits * (kSATile + kSBTile);  // 36 KB
+constexpr int kSBK = 64;              // K bytes per stage (two MMA k-steps of 32)
+constexpr int kSStages = 2;
+constexpr uint32_t kSATile = kSBM * kSBK;                  // 8 KB per digit plane
+constexpr uint32_t kSBTile = kSBN * kSBK;                  // 4 KB per digit plane
+constexpr uint32_t kSStage = kSplitDigits * (kSATile + kSBTile);  // 72 KB
 constexpr int kSEpiPitch = 32 * 8 + 16;  // bytes per staged row of 32 doubles (padded: the
                                          // 16-byte stores of a warp spread over the banks)
 constexpr uint32_t kSEpiBytes = 8 * 32 * kSEpiPitch;  // eight epilogue warps x 32 rows
@@ -342,9 +343,8 @@ __global__ void __launch_bounds__(kSThreads, 1)
           // the stage's descriptors once; an operand at a constant byte offset from the stage
           // is the same descriptor with offset / 16 added to its start-address field (the
           // field holds address / 16 in 14 bits, and no address here reaches 2^18)
-          // K-major, 32-byte rows with the 32-byte swizzle: 8-row groups 256 bytes apart
-          const uint64_t ad0 = tc::sdesc(a0, 16, 256, tc::kLayoutSW32);
-          const uint64_t bd0 = tc::sdesc(b0, 16, 256, tc::kLayoutSW32);
+          const uint64_t ad0 = tc::sdesc(a0, 16, 512, tc::kLayoutSW64);
+          const uint64_t bd0 = tc::sdesc(b0, 16, 512, tc::kLayoutSW64);
           // Digit pairs (p, q) with p + q < S (weight >= 2^-7(S+1)).  For one p the products
           // with q = 0 .. S-1-p go to classes p .. S-1, which sit side by side in TMEM, and the
           // B planes q = 0 .. sit back to back in shared memory (64 rows each, the same swizzle
@@ -501,7 +501,7 @@ static cudaError_t encode_digits_map(CUtensorMap* map, const int8_t* D, int64_t 
                                      uint32_t box_rows) {
   return encode_tmap_2d(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, D,
                         (int64_t)kSplitDigits * plane_rows, kSplitK, kSplitK, kSBK, box_rows,
-                        CU_TENSOR_MAP_SWIZZLE_32B);
+                        CU_TENSOR_MAP_SWIZZLE_64B);
 }
 
 cudaError_t launch_split_gemm(double* C, int64_t ldc, int M, int N, const SplitOperand& A,

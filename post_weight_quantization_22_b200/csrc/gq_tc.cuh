@@ -222,7 +222,7 @@ __device__ __forceinline__ void tmem_ld32x2(uint32_t taddr0, uint32_t taddr1, ui
 // Layout 4, 64-byte swizzle: K-major operands with 64-byte rows, 8-row groups SBO = 512 apart.
 // Layout 1, 128-byte swizzle with 32-byte chunks (4-row period): the only layout for 32-bit
 //   MN-major operands; 128-byte runs along M/N with LBO between runs, 4-row K groups SBO apart.
-constexpr uint32_t kLayoutSW128 = 2, kLayoutSW128Base32B = 1, kLayoutSW64 = 4, kLayoutSW32 = 6;
+constexpr uint32_t kLayoutSW128 = 2, kLayoutSW128Base32B = 1, kLayoutSW64 = 4;
 __device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo, uint32_t sbo,
                                           uint32_t layout) {
   uint64_t d = 0;
