@@ -252,6 +252,17 @@ FACTOR_SPLIT_MIN_N = 1536
 FACTOR_DIGIT_PRODUCTS = 21
 
 
+# DRAM bytes (read + written) of one call of a stage, from one ncu capture of every kernel of
+# that call (dram__bytes_read.sum + dram__bytes_write.sum, one pass each), keyed by stage and
+# width; valid only for the kernels as captured (profiles/factor_dram_traffic_*.md).
+STAGE_DRAM_BYTES = {
+    ("factor", 4096): {"bytes": 1.374e9,
+                       "source": "ncu dram__bytes_read.sum + dram__bytes_write.sum over the 238 "
+                                 "kernels of one gq_prepare_hinv call at n = 4096 (cold caches "
+                                 "between kernels), profiles/factor_dram_traffic_4096.md"},
+}
+
+
 def factor_work(n: int):
     """(multiply-adds done as int8 digit products, remaining fp64 flops) of one factor of
     width n; the two add up to the algorithmic 2 n^3 / 3 flops."""
@@ -597,6 +608,11 @@ def run_gq(args):
             "peak": round(d["work"] / (d["t_roof_ms"] * 1e-3) / 1e12, 3),
             "unit": "TFLOP/s", "frac": d["frac"], "traffic": None,
             "peak_source": d["peak"] + "; achieved = algorithmic flops / event-timed call"}
+    if not sweep and len(layers) == 1:
+        tb = STAGE_DRAM_BYTES.get((dname, layers[0][2]))
+        if tb is not None:
+            roof["traffic"] = tb["bytes"]
+            roof["traffic_source"] = tb["source"]
 
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
