@@ -270,12 +270,18 @@ def factor_work(n: int):
     if n < FACTOR_SPLIT_MIN_N:
         return 0.0, total
     macs = 0.0
-    for sp0 in range(0, n, FACTOR_SUPER):
-        sp1 = sp0 + FACTOR_SUPER
-        if sp1 >= n:
-            break
+    K = FACTOR_SUPER
+    for sp0 in range(0, n, K):
+        sp1 = sp0 + K
+        if sp1 > n:
+            break  # a narrower last block row: its inverse products stay fp64
         r = n - sp1
-        macs += (r * (r + 1) / 2.0 + r * sp0) * FACTOR_SUPER
+        # trailing update of the rest (lower triangle) and the inverse's T[k1:, <k0] += L X
+        macs += (r * (r + 1) / 2.0 + r * sp0) * K
+        # the inverse's full-width block row products with the triangular X_KK (half of its
+        # K x K entries are zero: the algorithmic count is half the issued one):
+        # T[k1:, K] = L X_KK and X[K, <k0] = -X_KK T
+        macs += (r * K * K + K * sp0 * K) / 2.0
     return macs, max(total - 2.0 * macs, 0.0)
 
 
