@@ -260,6 +260,11 @@ STAGE_DRAM_BYTES = {
                        "source": "ncu dram__bytes_read.sum + dram__bytes_write.sum over the 238 "
                                  "kernels of one gq_prepare_hinv call at n = 4096 (cold caches "
                                  "between kernels), profiles/factor_dram_traffic_4096.md"},
+    ("factor", 14336): {"bytes": 4.029e10,
+                        "source": "ncu dram__bytes_read.sum + dram__bytes_write.sum over the 858 "
+                                  "kernels of one gq_prepare_hinv call at n = 14336 (one pass "
+                                  "each, cold caches between kernels), "
+                                  "profiles/factor_dram_traffic_14336.md"},
 }
 
 
