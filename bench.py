@@ -254,17 +254,17 @@ FACTOR_DIGIT_PRODUCTS = 21
 
 # DRAM bytes (read + written) of one call of a stage, from one ncu capture of every kernel of
 # that call (dram__bytes_read.sum + dram__bytes_write.sum, one pass each), keyed by stage and
-# width; valid only for the kernels as captured (profiles/factor_dram_traffic_*.md).
+# width; valid only for the kernels as captured (commit 0b9f7bc).
 STAGE_DRAM_BYTES = {
     ("factor", 4096): {"bytes": 1.374e9,
                        "source": "ncu dram__bytes_read.sum + dram__bytes_write.sum over the 238 "
                                  "kernels of one gq_prepare_hinv call at n = 4096 (cold caches "
-                                 "between kernels), profiles/factor_dram_traffic_4096.md"},
+                                 "between kernels; kernels of commit 0b9f7bc)"},
     ("factor", 14336): {"bytes": 4.029e10,
                         "source": "ncu dram__bytes_read.sum + dram__bytes_write.sum over the 858 "
                                   "kernels of one gq_prepare_hinv call at n = 14336 (one pass "
-                                  "each, cold caches between kernels), "
-                                  "profiles/factor_dram_traffic_14336.md"},
+                                  "each, cold caches between kernels; kernels of commit "
+                                  "0b9f7bc)"},
 }
 
 
@@ -307,7 +307,7 @@ def stage_model(inputs, layers, bits: int, group: int, w_bytes: int, peaks: dict
                 stage_ms: dict) -> tuple[dict, dict]:
     """Per-stage algorithmic work, the floor time on the pipe each stage runs on, and the
     achieved fraction; plus the whole step against the sum of the floors (as built) and
-    against the floors as the survey states them (bf16 H, 3xTF32 factor and lazy updates,
+    against the floors of the nominal-precision plan (bf16 H, 3xTF32 factor and lazy updates,
     FP32 column recursion, HBM packing)."""
     hbm = peaks["hbm_gbs"] * 1e9
     fp64 = peaks["fp64_tflops"] * 1e12
