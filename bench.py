@@ -268,6 +268,14 @@ STAGE_DRAM_BYTES = {
 }
 
 
+def stage_traffic(stage: str, layers, sweep: bool):
+    """The measured DRAM traffic of one call of ``stage`` for a single-layer step whose width
+    was captured, else None (a sweep step runs several widths)."""
+    if sweep or len(layers) != 1:
+        return None
+    return STAGE_DRAM_BYTES.get((stage, layers[0][2]))
+
+
 def factor_work(n: int):
     """(multiply-adds done as int8 digit products, remaining fp64 flops) of one factor of
     width n; the two add up to the algorithmic 2 n^3 / 3 flops."""
@@ -619,11 +627,10 @@ def run_gq(args):
             "peak": round(d["work"] / (d["t_roof_ms"] * 1e-3) / 1e12, 3),
             "unit": "TFLOP/s", "frac": d["frac"], "traffic": None,
             "peak_source": d["peak"] + "; achieved = algorithmic flops / event-timed call"}
-    if not sweep and len(layers) == 1:
-        tb = STAGE_DRAM_BYTES.get((dname, layers[0][2]))
-        if tb is not None:
-            roof["traffic"] = tb["bytes"]
-            roof["traffic_source"] = tb["source"]
+    tb = stage_traffic(dname, layers, sweep)
+    if tb is not None:
+        roof["traffic"] = tb["bytes"]
+        roof["traffic_source"] = tb["source"]
 
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:

@@ -129,3 +129,16 @@ def test_factor_work_model_matches_the_library_split_policy():
         assert 2 * macs + fp64 == pytest.approx(2 * n ** 3 / 3, rel=1e-12)
     macs, fp64 = bench.factor_work(14336)
     assert 2 * macs / (2 * 14336 ** 3 / 3) > 0.9   # nearly all of the factor at that width
+
+
+def test_stage_traffic_only_for_captured_single_layer_widths():
+    sys.path.insert(0, ROOT)
+    import bench
+    one = [("w", 4096, 14336, "x")]
+    got = bench.stage_traffic("factor", one, sweep=False)
+    assert got is not None and got["bytes"] > 1e10          # the 14336-wide factor call
+    assert bench.stage_traffic("factor", [("w", 4096, 4096, "x")], False)["bytes"] < got["bytes"]
+    assert bench.stage_traffic("factor", [("w", 4096, 5000, "x")], False) is None
+    assert bench.stage_traffic("column_loop", one, False) is None
+    assert bench.stage_traffic("factor", one + one, False) is None
+    assert bench.stage_traffic("factor", one, True) is None
