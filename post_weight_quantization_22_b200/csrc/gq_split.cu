@@ -46,11 +46,12 @@ constexpr int kSStages = 2;
 constexpr uint32_t kSATile = kSBM * kSBK;                  // 8 KB per digit plane
 constexpr uint32_t kSBTile = kSBN * kSBK;                  // 4 KB per digit plane
 constexpr uint32_t kSStage = kSplitDigits * (kSATile + kSBTile);  // 72 KB
+constexpr int kSEpiWarps = 8;        // two per TMEM lane quadrant, 32 columns each
 constexpr int kSEpiPitch = 32 * 8 + 16;  // bytes per staged row of 32 doubles (padded: the
                                          // 16-byte stores of a warp spread over the banks)
-constexpr uint32_t kSEpiBytes = 8 * 32 * kSEpiPitch;  // eight epilogue warps x 32 rows
+constexpr uint32_t kSEpiBytes = kSEpiWarps * 32 * kSEpiPitch;  // each epilogue warp's 32 rows
 constexpr size_t kSSmem = kSStages * kSStage + 1024 + 256 + kSEpiBytes;
-constexpr int kSEpiWarps = 8;        // two per TMEM lane quadrant, 32 columns each
+static_assert(kSSmem <= 227 * 1024, "the stages and the epilogue staging fit one CTA's shared memory");
 constexpr int kSThreads = 32 * (2 + kSEpiWarps);  // warp 0 producer, warp 1 MMA, then epilogue
 constexpr int kSTilesPerCta = 4;     // tiles per CTA aimed at (CTAs retire regularly, so other
                                      // streams' kernels get SMs)
