@@ -842,3 +842,18 @@ def test_hptq_search_brackets_the_budget(budget):
         assert t - lo == 2.0 ** -steps
         r_lo = O.gptq_columns(W, U, 4, clip="unbounded", alpha=np.full(6, 2.0 ** lo))
         assert O.hptq_rate(r_lo["codes"]) > budget
+
+
+@pytest.mark.parametrize("seed", [0, 1, 2])
+def test_hptq_rate_lies_within_one_bit_of_the_entropy(seed):
+    """Shannon's bound for a Huffman code: H <= rate < H + 1 bits per symbol, H the empirical
+    entropy of the codes; equal to H when every probability is a power of two."""
+    rng = np.random.default_rng(seed)
+    codes = np.rint(rng.standard_normal(5000) * (1.0 + seed)).astype(np.int64)
+    _, counts = np.unique(codes, return_counts=True)
+    p = counts / counts.sum()
+    H = float(-(p * np.log2(p)).sum())
+    r = O.hptq_rate(codes)
+    assert H - 1e-12 <= r < H + 1.0
+    dyadic = np.repeat([0, 1, 2, 3], [8, 4, 2, 2])           # p = 1/2, 1/4, 1/8, 1/8
+    assert O.hptq_rate(dyadic) == pytest.approx(1.75)
