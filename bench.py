@@ -751,7 +751,8 @@ def run_reference(args):
 
 
 def run_case(args):
-    """One invocation for profilers: `layer` (the q_proj recipe at --case-n, or --workload
+    """One invocation for profilers: `searches` (the SSQR and HPTQ searches on the q_proj
+    layer, event-timed, one JSON line), `layer` (the q_proj recipe at --case-n, or --workload
     at its full size when --case-n is not given, two calls so a profiler can skip the first), `factor`
     (gq_prepare_hinv on a seeded SPD fp64 H of width --case-n), or `huffman` (the Huffman
     encoder on the unconstrained-lattice codes of that layer, event-timed, one JSON line with
@@ -762,7 +763,41 @@ def run_case(args):
 
     torch.cuda.set_device(0)
     n = args.case_n if args.case_n is not None else 2048
-    if args.case == "layer":
+    if args.case == "searches":
+        W, X, spec = synth.workload("q_proj_4096x4096")
+        m, n = W.shape
+        lq = LayerQuantizer(m, n, G.QuantCfg(bits=4), device="cuda", max_tokens=X.shape[0])
+        Wd, Xd = W.cuda(), X.cuda()
+        lq.hessian(Xd)
+        lq.prepare()
+        torch.cuda.synchronize()
+
+        def timed(fn, reps=3):
+            fn()
+            torch.cuda.synchronize()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            for _ in range(reps):
+                r = fn()
+            b.record()
+            torch.cuda.synchronize()
+            return a.elapsed_time(b) / reps, r
+
+        out = {"case": "searches", "workload": "q_proj_4096x4096"}
+        ms, r = timed(lambda: G.gq_ssqr_quantize_layer(Wd, lq.U, lq.dead, lq.delta, bits=3,
+                                                         density=0.01, steps=20))
+        out.update(ssqr_3bit_density_0p01_steps_20_ms=ms,
+                   ssqr_status=G.gq_workspace_status(r["ws"])[0])
+        ms, r = timed(lambda: G.gq_hptq_quantize_layer(Wd, lq.U, lq.dead, lq.delta, bits=4,
+                                                         budget=3.125, steps=12))
+        out.update(hptq_budget_3p125_steps_12_ms=ms, hptq_alpha=float(r["alpha"].item()),
+                   hptq_bits_per_weight=int(r["total_bits"].item()) / (m * n),
+                   hptq_status=G.gq_workspace_status(r["ws"])[0])
+        ms, _ = timed(lambda: G.gq_quantize_layer(Wd, lq.U, lq.dead, lq.delta,
+                                                  G.QuantCfg(bits=4, clip="unbounded")))
+        out["one_unbounded_lattice_pass_ms"] = ms
+        print(json.dumps(out))
+    elif args.case == "layer":
         if args.case_n is None:
             W, X, spec = synth.workload(args.workload)
         else:
@@ -828,7 +863,7 @@ def main(argv=None):
     ap.add_argument("--cpu-n", type=int, default=6144)
     ap.add_argument("--cpu-rows", type=int, default=64)
     ap.add_argument("--ref-rows", type=int, default=8)
-    ap.add_argument("--case", choices=["layer", "factor", "huffman"], default=None,
+    ap.add_argument("--case", choices=["layer", "factor", "huffman", "searches"], default=None,
                     help="run one untimed invocation (for profilers) and exit")
     ap.add_argument("--case-n", type=int, default=None,
                     help="size of the case (default: 2048; `layer`: --workload at full size)")
